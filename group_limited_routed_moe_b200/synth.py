@@ -1,0 +1,211 @@
+"""Seeded synthetic inputs for the routed MoE layer.
+
+This module holds no arithmetic of the method: only random draws and dtype
+packing.  It is the one piece of code that both the CUDA path (tests, bench,
+smoke) and the float64 oracle consume, so that both see identical bytes.  It
+never imports the CUDA binding or the oracle.
+
+Recipe (the distributions of the layer's workloads):
+
+* activations x ~ N(0, 1), stored as bf16 [T, 1536];
+* router logits ~ N(0, 1) fp32 [T, 128], per-expert bias ~ N(0, 0.1) fp32 [128];
+* the skewed prefill adds +2.0 to the logits of 16 "hot" experts drawn
+  without replacement (Zipf-like load imbalance);
+* expert weights ~ N(0, 0.02), bf16: W_gate, W_up [128, 1536, 512] and
+  W_down [128, 512, 1536] per layer, used as x @ W.
+
+Activations, logits and bias are drawn with NumPy's PCG64 (host).  Expert
+weights (up to 23 x 604 MB) come from a counter-based generator so that the
+same bytes can be produced on the device in bulk or on the host for any
+single expert: a 32-bit integer hash of (seed, layer, matrix, expert, element)
+picks one of 65,536 normal quantiles Phi^-1((k + 1/2) / 65536), scaled by
+0.02 and rounded once to bf16.  After bf16 rounding this is indistinguishable
+from N(0, 0.02) except that the tails are cut at 4.33 sigma.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+HIDDEN = 1536
+INTER = 512
+N_EXPERTS = 128
+TOPK = 8
+WEIGHT_STD = 0.02
+
+# matrix ids inside a layer
+W_GATE, W_UP, W_DOWN = 0, 1, 2
+_W_SHAPES = {W_GATE: (HIDDEN, INTER), W_UP: (HIDDEN, INTER), W_DOWN: (INTER, HIDDEN)}
+
+
+# ----------------------------------------------------------------------------
+# dtype packing
+# ----------------------------------------------------------------------------
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> raw bf16 bits (uint16), round to nearest even (finite input)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    r = u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return (r >> np.uint32(16)).astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# counter-based weight generator
+# ----------------------------------------------------------------------------
+
+_M1 = 0x7FEB352D
+_M2 = 0x846CA68B
+_TABLE_BITS: np.ndarray | None = None
+
+
+def _quantile_table_bits() -> np.ndarray:
+    """65,536 bf16 values: bf16(float32(Phi^-1((k + 0.5) / 65536)) * 0.02)."""
+    global _TABLE_BITS
+    if _TABLE_BITS is None:
+        from scipy.special import ndtri
+        q = ndtri((np.arange(65536, dtype=np.float64) + 0.5) / 65536.0).astype(np.float32)
+        _TABLE_BITS = f32_to_bf16_bits(q * np.float32(WEIGHT_STD))
+    return _TABLE_BITS
+
+
+def _mix32_np(x: np.ndarray) -> np.ndarray:
+    """32-bit avalanche hash (xorshift-multiply, 'lowbias32' constants), uint32."""
+    x = x.astype(np.uint32, copy=True)
+    x ^= x >> np.uint32(16)
+    x *= np.uint32(_M1)
+    x ^= x >> np.uint32(15)
+    x *= np.uint32(_M2)
+    x ^= x >> np.uint32(16)
+    return x
+
+
+def _stream_keys(seed: int, layer: int, which: int, experts: np.ndarray):
+    sid = ((np.uint64(seed) * np.uint64(64) + np.uint64(layer)) * np.uint64(4)
+           + np.uint64(which)) * np.uint64(128) + experts.astype(np.uint64)
+    sid = (sid & np.uint64(0xFFFFFFFF)).astype(np.uint32)
+    k1 = _mix32_np(sid ^ np.uint32(0xA511E9B3))
+    k2 = _mix32_np(sid ^ np.uint32(0x63D83595))
+    return k1, k2
+
+
+def weight_bits_np(seed: int, layer: int, which: int,
+                   experts=None) -> np.ndarray:
+    """Expert matrix ``which`` of ``layer`` as bf16 bits [len(experts), rows, cols]."""
+    experts = np.arange(N_EXPERTS) if experts is None else np.asarray(experts)
+    rows, cols = _W_SHAPES[which]
+    n = rows * cols
+    k1, k2 = _stream_keys(seed, layer, which, experts)
+    i = np.arange(n, dtype=np.uint32)
+    table = _quantile_table_bits()
+    out = np.empty((len(experts), n), dtype=np.uint16)
+    for j in range(len(experts)):
+        u = _mix32_np(_mix32_np(i ^ k1[j]) ^ k2[j])
+        out[j] = table[u >> np.uint32(16)]
+    return out.reshape(len(experts), rows, cols)
+
+
+def layer_weights_np(seed: int, layer: int, experts=None):
+    """(W_gate, W_up, W_down) bf16 bits of one layer on the host."""
+    return tuple(weight_bits_np(seed, layer, w, experts) for w in (W_GATE, W_UP, W_DOWN))
+
+
+def _mix32_torch(x):
+    """Same hash as ``_mix32_np`` on int64 tensors holding values < 2**32.
+
+    Multiplication modulo 2**32 is split into 16-bit halves so that no
+    intermediate leaves the int64 range on any device.
+    """
+    def mul32(v, c):
+        lo = (v & 0xFFFF) * c
+        hi = (((v >> 16) * c) & 0xFFFF) << 16
+        return (lo + hi) & 0xFFFFFFFF
+    x = x ^ (x >> 16)
+    x = mul32(x, _M1)
+    x = x ^ (x >> 15)
+    x = mul32(x, _M2)
+    x = x ^ (x >> 16)
+    return x
+
+
+def weight_bits_torch(seed: int, layer: int, which: int, device, out=None):
+    """Same bytes as ``weight_bits_np`` for all 128 experts, made on ``device``.
+
+    Returns (or fills) a torch.bfloat16 tensor [128, rows, cols].
+    """
+    import torch
+    rows, cols = _W_SHAPES[which]
+    n = rows * cols
+    k1, k2 = _stream_keys(seed, layer, which, np.arange(N_EXPERTS))
+    table = torch.from_numpy(_quantile_table_bits().view(np.int16)).to(device)
+    if out is None:
+        out = torch.empty((N_EXPERTS, rows, cols), dtype=torch.bfloat16, device=device)
+    flat = out.view(N_EXPERTS, n).view(torch.int16)
+    i = torch.arange(n, dtype=torch.int64, device=device)[None, :]
+    k1t = torch.from_numpy(k1.astype(np.int64)).to(device)[:, None]
+    k2t = torch.from_numpy(k2.astype(np.int64)).to(device)[:, None]
+    step = 16
+    for e0 in range(0, N_EXPERTS, step):
+        u = _mix32_torch(_mix32_torch(i ^ k1t[e0:e0 + step]) ^ k2t[e0:e0 + step])
+        flat[e0:e0 + step].copy_(table[u >> 16])
+    return out
+
+
+# ----------------------------------------------------------------------------
+# token-side inputs
+# ----------------------------------------------------------------------------
+
+@dataclass
+class TokenInputs:
+    x_bits: np.ndarray        # [T, 1536] uint16 (bf16 bits)
+    logits: np.ndarray        # [T, 128] float32
+    bias: np.ndarray          # [128] float32
+    hot_experts: np.ndarray = field(default_factory=lambda: np.zeros(0, np.int64))
+
+
+def make_tokens(T: int, seed: int, hot: int = 0, hot_boost: float = 2.0,
+                layer: int = 0) -> TokenInputs:
+    """x, router logits and bias for ``T`` tokens from PCG64(seed, layer)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, layer])))
+    x = rng.standard_normal((T, HIDDEN), dtype=np.float32)
+    logits = rng.standard_normal((T, N_EXPERTS), dtype=np.float32)
+    bias = (rng.standard_normal(N_EXPERTS, dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    hot_ids = np.zeros(0, np.int64)
+    if hot:
+        hot_ids = np.sort(rng.choice(N_EXPERTS, size=hot, replace=False)).astype(np.int64)
+        logits[:, hot_ids] += np.float32(hot_boost)
+    return TokenInputs(f32_to_bf16_bits(x), logits, bias, hot_ids)
+
+
+def layer_logits(T: int, seed: int, layer: int):
+    """Router logits [T,128] and bias [128] of one layer of the stack."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 1000 + layer])))
+    logits = rng.standard_normal((T, N_EXPERTS), dtype=np.float32)
+    bias = (rng.standard_normal(N_EXPERTS, dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    return logits, bias
+
+
+# ----------------------------------------------------------------------------
+# named workloads
+# ----------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int                 # tokens actually processed
+    T_buf: int             # rows allocated (>= T)
+    seed: int
+    hot: int = 0
+    layers: int = 1
+    weight_seed: int = 0
+
+
+WORKLOADS = {
+    "decode_T16": Workload("decode_T16", 16, 16, 0),
+    **{f"decode_T4_seed{s}": Workload(f"decode_T4_seed{s}", 4, 4, s) for s in range(1, 9)},
+    "prefill_T2048_skewed": Workload("prefill_T2048_skewed", 2048, 2048, 2, hot=16),
+    "prefill_T8189": Workload("prefill_T8189", 8189, 8192, 3),
+    "stack23_T1": Workload("stack23_T1", 1, 1, 4, layers=23, weight_seed=4),
+    "stack23_T8189": Workload("stack23_T8189", 8189, 8192, 4, layers=23, weight_seed=4),
+}

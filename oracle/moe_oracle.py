@@ -1,0 +1,276 @@
+"""Float64 CPU oracle for the group-limited routed MoE layer of Ling-3.0-tiny.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+link this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA library (no kernels, headers, helpers or tables) and
+imports nothing from the ``group_limited_routed_moe_b200`` package.
+
+What it computes is the plain definition of the layer, evaluated in float64
+from the exact bf16 / fp32 input values, with no blocking, fusion or
+reordering beyond what the definition states:
+
+* Grid.  128 routed experts per layer in 8 groups of 16; each token keeps 4
+  groups and then uses 8 experts; hidden size 1536.  Sources: "Ling-3.0-tiny
+  on a Qualcomm board" (TensorFold issue #1247), first comment, opening
+  paragraph (tiny's config: "128 experts in 8 groups of 16 keeping 4",
+  hidden 1536); "HelloSun/ling30tiny", table "模型與路由" (model and
+  routing): 128 experts per layer, 8 experts active per token.
+* Routing is group-limited (issue #1247, "What it does not cover", the bullet
+  that lists the CUDA C kernels).  The pages name the rule but not its
+  arithmetic; the reading used here (and in the CUDA path) is:
+  score s_e = sigmoid(logit_e + bias_e); group score = sum of the group's two
+  largest s; keep the 4 groups with the largest score (ties: lower group
+  index); pick the 8 largest s among the 64 experts of the kept groups (ties:
+  lower expert index), in that order; combine weight
+  w_i = sigmoid(logit_{e_i}) / sum_j sigmoid(logit_{e_j}) (bias excluded).
+* Expert FFN: each expert has gate, up and down matrices ("HelloSun/
+  ling30tiny", table "模型與路由", row "expert 權重": gate/up and down), i.e.
+  a SwiGLU FFN  y = (silu(x W_gate) * (x W_up)) W_down  with silu(a) =
+  a * sigmoid(a) and no clamp (issue #1247, opening paragraph: "null SwiGLU
+  limit lists").  Intermediate size 512.
+* Layer output: out_t = sum_i w_i * FFN_{e_i}(x_t) -- the "real MoE routing
+  + weighted layer" of "HelloSun/ling30tiny", section "數值檢查摘要"
+  (numeric check summary).
+* Expert row sets: each expert runs on exactly the rows that picked it
+  (issue #1247, "What it does not cover", bullet on bf16 experts).  The
+  permutation below is the stable (token-ascending) counting sort of those
+  rows, which the CUDA path must reproduce bit for bit.
+* Stack: 23 MoE layers (24 layers with dense layer 0 -- issue #1247, opening
+  paragraph), residual stream kept in bf16: h <- bf16(h + moe(h)).
+
+Every function is pinned by tests in ``tests/test_oracle_*.py`` against
+brute force, closed forms and invariants (see each test's docstring).
+"""
+
+from __future__ import annotations
+
+import itertools
+from dataclasses import dataclass
+
+import numpy as np
+
+HIDDEN = 1536
+INTER = 512
+N_EXPERTS = 128
+N_GROUPS = 8
+KEEP_GROUPS = 4
+TOPK = 8
+N_MOE_LAYERS = 23
+
+
+# ----------------------------------------------------------------------------
+# bf16 <-> float64 (the oracle's own conversions; exact / round-to-nearest-even)
+# ----------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of raw bfloat16 bits (uint16) as float64."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round float64 values to bfloat16 (round to nearest, ties to even).
+
+    Rounds directly from float64 to 8 significant bits (no intermediate
+    float32 rounding, which could round twice).  Finite normal-range values
+    only; zero is kept.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    mant, expo = np.frexp(v)                  # v = mant * 2**expo, 0.5 <= |mant| < 1
+    q = np.rint(mant * 256.0)                 # 8 significant bits, half to even
+    r = np.ldexp(q, expo - 8)                 # exactly representable in bf16
+    return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# Routing
+# ----------------------------------------------------------------------------
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    """Logistic function in float64."""
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+@dataclass
+class RouteResult:
+    topk_idx: np.ndarray      # [T, k] int64, slot order = descending score, ties -> lower index
+    topk_w: np.ndarray        # [T, k] float64 combine weights
+    kept_groups: np.ndarray   # [T, keep] int64, descending group score, ties -> lower index
+    group_margin: np.ndarray  # [T] float64: (keep-th best group score) - (next one)
+    expert_margin: np.ndarray  # [T] float64: (k-th best candidate score) - (next one)
+
+
+def route(logits: np.ndarray, bias: np.ndarray | None,
+          n_groups: int = N_GROUPS, keep: int = KEEP_GROUPS,
+          topk: int = TOPK) -> RouteResult:
+    """Group-limited top-k routing of every token (float64).
+
+    Steps, per token (the reading stated in the module docstring):
+      1. z_e = logit_e + bias_e and s_e = sigmoid(z_e);
+      2. group score g_j = s_(1) + s_(2), the two largest s inside group j;
+      3. kept groups = the ``keep`` largest g_j, ties to the lower group index;
+      4. the ``topk`` largest s among the experts of the kept groups, ties to
+         the lower expert index, in that order (the slot order);
+      5. w_i = sigmoid(logit_{e_i}) / sum_i' sigmoid(logit_{e_i'}).
+    The grid sizes are parameters so that tests can brute-force small grids.
+    """
+    lg = np.asarray(logits, dtype=np.float64)
+    T, n_exp = lg.shape
+    if n_exp % n_groups:
+        raise ValueError("experts must split evenly into groups")
+    gsize = n_exp // n_groups
+    z = lg + (np.asarray(bias, dtype=np.float64)[None, :] if bias is not None else 0.0)
+    s = sigmoid(z)
+
+    two_best = np.sort(s.reshape(T, n_groups, gsize), axis=2)[:, :, -2:]
+    gscore = two_best[:, :, 0] + two_best[:, :, 1]
+    g_order = np.argsort(-gscore, axis=1, kind="stable")      # ties keep lower index first
+    kept = g_order[:, :keep]
+    rows = np.arange(T)[:, None]
+    g_sorted = gscore[rows, g_order]
+    group_margin = (g_sorted[:, keep - 1] - g_sorted[:, keep]) if keep < n_groups \
+        else np.full(T, np.inf)
+
+    in_kept = np.zeros((T, n_groups), dtype=bool)
+    in_kept[rows, kept] = True
+    cand = np.where(np.repeat(in_kept, gsize, axis=1), s, -np.inf)
+    e_order = np.argsort(-cand, axis=1, kind="stable")
+    idx = e_order[:, :topk]
+    c_sorted = cand[rows, e_order]
+    n_cand = keep * gsize
+    expert_margin = (c_sorted[:, topk - 1] - c_sorted[:, topk]) if topk < n_cand \
+        else np.full(T, np.inf)
+
+    sw = sigmoid(lg[rows, idx])
+    w = sw / sw.sum(axis=1, keepdims=True)
+    return RouteResult(idx.astype(np.int64), w, kept.astype(np.int64),
+                       group_margin, expert_margin)
+
+
+def route_bruteforce(logits_row: np.ndarray, bias_row: np.ndarray | None,
+                     n_groups: int, keep: int, topk: int):
+    """Routing of ONE token by exhaustive enumeration (pure Python, tiny grids).
+
+    Enumerates every subset of ``keep`` groups and keeps the one with the
+    largest total group score (a group's score being the sum of its two
+    largest member scores, found here by scanning all member pairs); then
+    enumerates every ``topk``-subset of the kept groups' experts and keeps the
+    one with the largest total score.  Exact ties are broken by preferring the
+    lexicographically smaller index tuple.  Returns (kept groups sorted,
+    chosen experts sorted by descending score then index, weights).
+    """
+    n_exp = len(logits_row)
+    gsize = n_exp // n_groups
+    b = [0.0] * n_exp if bias_row is None else [float(v) for v in bias_row]
+    s = [1.0 / (1.0 + np.exp(-(float(logits_row[e]) + b[e]))) for e in range(n_exp)]
+
+    def gscore(j):
+        mem = range(j * gsize, (j + 1) * gsize)
+        return max(s[a] + s[c] for a in mem for c in mem if a < c)
+
+    gs = [gscore(j) for j in range(n_groups)]
+    best_g, best_val = None, None
+    for sub in itertools.combinations(range(n_groups), keep):
+        val = sum(sorted((gs[j] for j in sub), reverse=True))
+        if best_val is None or val > best_val:
+            best_g, best_val = sub, val
+    cands = [e for j in best_g for e in range(j * gsize, (j + 1) * gsize)]
+    best_e, best_v = None, None
+    for sub in itertools.combinations(sorted(cands), topk):
+        val = sum(sorted((s[e] for e in sub), reverse=True))
+        if best_v is None or val > best_v:
+            best_e, best_v = sub, val
+    chosen = sorted(best_e, key=lambda e: (-s[e], e))
+    sig = [1.0 / (1.0 + np.exp(-float(logits_row[e]))) for e in chosen]
+    tot = sum(sig)
+    return sorted(best_g), chosen, [v / tot for v in sig]
+
+
+# ----------------------------------------------------------------------------
+# Permutation (rows that picked each expert)
+# ----------------------------------------------------------------------------
+
+@dataclass
+class PermuteResult:
+    counts: np.ndarray    # [E] int64
+    offsets: np.ndarray   # [E+1] int64, exclusive prefix of counts
+    perm_src: np.ndarray  # [T*k] int64: permuted row r holds item t*k + slot
+    inv_perm: np.ndarray  # [T*k] int64: item t*k + slot sits at permuted row inv_perm[...]
+
+
+def permute(topk_idx: np.ndarray, n_experts: int = N_EXPERTS) -> PermuteResult:
+    """Stable counting sort of the (token, slot) items by expert id.
+
+    Items are numbered t*k + slot; rows are grouped expert-major and, inside
+    an expert, kept in item order (token ascending, since a token picks an
+    expert at most once).
+    """
+    flat = np.asarray(topk_idx, dtype=np.int64).reshape(-1)
+    counts = np.bincount(flat, minlength=n_experts).astype(np.int64)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    perm_src = np.argsort(flat, kind="stable").astype(np.int64)
+    inv_perm = np.empty_like(perm_src)
+    inv_perm[perm_src] = np.arange(flat.size, dtype=np.int64)
+    return PermuteResult(counts, offsets, perm_src, inv_perm)
+
+
+# ----------------------------------------------------------------------------
+# Expert FFN, layer, stack
+# ----------------------------------------------------------------------------
+
+def silu(a: np.ndarray) -> np.ndarray:
+    """silu(a) = a * sigmoid(a), float64, no clamp."""
+    return a * sigmoid(a)
+
+
+def expert_ffn(x: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray,
+               w_down: np.ndarray) -> np.ndarray:
+    """SwiGLU expert on rows x [M, H] (float64): (silu(x Wg) * (x Wu)) Wd."""
+    return (silu(x @ w_gate) * (x @ w_up)) @ w_down
+
+
+def moe_layer(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | None,
+              w_gate_bits: np.ndarray, w_up_bits: np.ndarray,
+              w_down_bits: np.ndarray, route_result: RouteResult | None = None
+              ) -> np.ndarray:
+    """Routed MoE layer output [T, H] in float64 (no intermediate rounding).
+
+    x_bits: [T, H] bf16 bits; logits [T, E] fp32; bias [E] fp32 or None;
+    w_gate_bits, w_up_bits: [E, H, I] bf16 bits; w_down_bits: [E, I, H].
+    Each token only depends on its own row, so calling this on a subset of
+    rows gives those rows of the full result.
+    """
+    rr = route_result if route_result is not None else route(logits, bias)
+    x = bf16_bits_to_f64(x_bits)
+    T = x.shape[0]
+    out = np.zeros((T, w_down_bits.shape[2]), dtype=np.float64)
+    for e in np.unique(rr.topk_idx):
+        tok, slot = np.nonzero(rr.topk_idx == e)
+        y = expert_ffn(x[tok], bf16_bits_to_f64(w_gate_bits[e]),
+                       bf16_bits_to_f64(w_up_bits[e]), bf16_bits_to_f64(w_down_bits[e]))
+        out[tok] += rr.topk_w[tok, slot][:, None] * y
+    return out
+
+
+def moe_stack(x_bits: np.ndarray, layers) -> np.ndarray:
+    """Stack of MoE layers with a bf16 residual stream.
+
+    ``layers`` yields (logits, bias, w_gate_bits, w_up_bits, w_down_bits) per
+    layer; the router logits of every layer are given (they do not depend on
+    the activations in this reading).  After each layer the residual stream is
+    rounded to bf16: h <- bf16(h + moe(h)).  Returns the final bf16 bits.
+    """
+    h = np.asarray(x_bits, dtype=np.uint16)
+    for (lg, b, wg, wu, wd) in layers:
+        upd = moe_layer(h, lg, b, wg, wu, wd)
+        h = f64_to_bf16_bits(bf16_bits_to_f64(h) + upd)
+    return h
+
+
+def rel_l2(a: np.ndarray, ref: np.ndarray) -> float:
+    """||a - ref||_2 / ||ref||_2 in float64."""
+    a = np.asarray(a, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(a - ref) / den) if den > 0 else float(np.linalg.norm(a))

@@ -1,0 +1,227 @@
+"""Pins for the oracle's permutation, expert FFN, layer and stack (no GPU).
+
+Checked against: a pure-Python brute-force permutation, a hand-worked SwiGLU
+example (tests/golden/ffn_worked_example.json), a scalar triple-loop FFN on
+tiny shapes, the dense special case (every token forced onto the same 8
+experts, computed with whole-matrix products), invariances (token
+permutation, row subsets, linearity in W_down, zero W_down), exhaustive
+bf16 rounding against a neighbour search, and the page-derived sizes
+(tests/golden/pages_facts.json).
+"""
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(rng, shape, std):
+    v = (rng.standard_normal(shape) * std).astype(np.float32)
+    return O.f64_to_bf16_bits(v.astype(np.float64))
+
+
+def _weights(rng, E, H, I):
+    return _bf16(rng, (E, H, I), 0.02), _bf16(rng, (E, H, I), 0.02), _bf16(rng, (E, I, H), 0.02)
+
+
+# ---------------------------------------------------------------- permutation
+
+def test_permute_matches_bruteforce():
+    rng = np.random.default_rng(0)
+    lg = rng.standard_normal((37, 128)).astype(np.float32)
+    rr = O.route(lg, None)
+    p = O.permute(rr.topk_idx)
+    T, k = rr.topk_idx.shape
+    ref = []
+    for e in range(128):
+        for t in range(T):
+            for s in range(k):
+                if rr.topk_idx[t, s] == e:
+                    ref.append(t * k + s)
+    assert p.perm_src.tolist() == ref
+    assert p.counts.sum() == T * k and p.offsets[0] == 0 and p.offsets[-1] == T * k
+    assert np.all(np.diff(p.offsets) == p.counts)
+    assert np.array_equal(p.inv_perm[p.perm_src], np.arange(T * k))
+    for e in range(128):
+        rows = p.perm_src[p.offsets[e]:p.offsets[e + 1]]
+        assert np.all(rr.topk_idx.reshape(-1)[rows] == e)
+        assert np.all(np.diff(rows // k) > 0)          # token ascending inside an expert
+
+
+def test_permute_empty():
+    p = O.permute(np.zeros((0, 8), np.int64))
+    assert p.counts.sum() == 0 and p.offsets.tolist() == [0] * 129
+    assert p.perm_src.size == 0
+
+
+# ---------------------------------------------------------------- bf16 helpers
+
+def test_bf16_decode_known_values():
+    bits = np.array([0x3F80, 0xC000, 0x3F81, 0x0000, 0x8000, 0x4049], np.uint16)
+    assert O.bf16_bits_to_f64(bits).tolist() == [1.0, -2.0, 1.0078125, 0.0, -0.0, 3.140625]
+
+
+def _bf16_nearest_even_bruteforce(v):
+    """Nearest bf16 by scanning the neighbouring bit patterns (ties to even)."""
+    f = np.float32(v)
+    b0 = int(np.array([f], np.float32).view(np.uint32)[0] >> 16)
+    best = None
+    for b in range(max(b0 - 2, 0), b0 + 3):
+        for sign in (0, 0x8000):
+            bb = (b & 0x7FFF) | sign
+            val = float(O.bf16_bits_to_f64(np.array([bb], np.uint16))[0])
+            key = (abs(val - v), bb & 1)
+            if best is None or key < best[0]:
+                best = (key, bb)
+    return best[1]
+
+
+def test_bf16_round_nearest_even_against_bruteforce():
+    rng = np.random.default_rng(1)
+    vals = list(rng.standard_normal(2000) * 10.0)
+    # exact ties and values just off a tie (which float32 would round twice)
+    for m in range(128, 256, 7):
+        base = m / 128.0
+        half = 1.0 / 256.0
+        vals += [base + half, -(base + half), base + half + 2.0 ** -40, base + half - 2.0 ** -40]
+    got = O.f64_to_bf16_bits(np.array(vals))
+    ref = [_bf16_nearest_even_bruteforce(v) for v in vals]
+    assert got.tolist() == ref
+
+
+# ---------------------------------------------------------------- expert FFN
+
+def test_ffn_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "ffn_worked_example.json")))
+    y = O.expert_ffn(np.array([g["x"]]), np.array(g["w_gate"]), np.array(g["w_up"]),
+                     np.array(g["w_down"]))
+    np.testing.assert_allclose(y[0], g["y"], rtol=0, atol=1e-14)
+
+
+def test_ffn_scalar_loops_tiny_shapes():
+    rng = np.random.default_rng(2)
+    M, H, I = 3, 5, 4
+    x = rng.standard_normal((M, H))
+    wg, wu, wd = rng.standard_normal((H, I)), rng.standard_normal((H, I)), rng.standard_normal((I, H))
+    y = O.expert_ffn(x, wg, wu, wd)
+    for m in range(M):
+        for n in range(H):
+            acc = 0.0
+            for c in range(I):
+                a = sum(x[m, kk] * wg[kk, c] for kk in range(H))
+                u = sum(x[m, kk] * wu[kk, c] for kk in range(H))
+                acc += (a / (1.0 + math.exp(-a))) * u * wd[c, n]
+            assert abs(y[m, n] - acc) < 1e-12
+
+
+def test_silu_identities():
+    a = np.linspace(-30, 30, 601)
+    np.testing.assert_allclose(O.silu(a) - O.silu(-a), a, atol=1e-13)
+    assert O.silu(np.array([0.0]))[0] == 0.0
+
+
+# ---------------------------------------------------------------- layer
+
+def test_layer_dense_special_case():
+    """All tokens forced onto experts {3,4,21,22,40,41,90,91} (bias +1e3 gives
+    score 1.0 to exactly these): the layer equals the dense weighted sum of
+    those 8 FFNs over the whole token matrix."""
+    rng = np.random.default_rng(3)
+    E, H, I, T = 128, 64, 32, 10
+    wg, wu, wd = _weights(rng, E, H, I)
+    x = _bf16(rng, (T, H), 1.0)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    bias = np.zeros(E, np.float32)
+    forced = [3, 4, 21, 22, 40, 41, 90, 91]
+    bias[forced] = 1000.0
+    out = O.moe_layer(x, lg, bias, wg, wu, wd)
+    X = O.bf16_bits_to_f64(x)
+    sig = 1.0 / (1.0 + np.exp(-lg[:, forced].astype(np.float64)))
+    w = sig / sig.sum(axis=1, keepdims=True)
+    ref = np.zeros((T, H))
+    for i, e in enumerate(forced):
+        G = X @ O.bf16_bits_to_f64(wg[e])
+        U = X @ O.bf16_bits_to_f64(wu[e])
+        ref += w[:, i:i + 1] * ((G / (1 + np.exp(-G))) * U @ O.bf16_bits_to_f64(wd[e]))
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_layer_invariances():
+    rng = np.random.default_rng(4)
+    E, H, I, T = 128, 48, 16, 24
+    wg, wu, wd = _weights(rng, E, H, I)
+    x = _bf16(rng, (T, H), 1.0)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(E)).astype(np.float32)
+    out = O.moe_layer(x, lg, b, wg, wu, wd)
+    # token permutation
+    perm = rng.permutation(T)
+    np.testing.assert_allclose(O.moe_layer(x[perm], lg[perm], b, wg, wu, wd), out[perm],
+                               rtol=1e-13, atol=1e-15)
+    # row subset
+    sub = np.array([0, 5, 6, 23])
+    np.testing.assert_allclose(O.moe_layer(x[sub], lg[sub], b, wg, wu, wd), out[sub],
+                               rtol=1e-13, atol=1e-15)
+    # doubling W_down doubles the output exactly (exponent +1 on every bf16)
+    wd2 = (wd.astype(np.uint32) + np.where((wd & 0x7FFF) != 0, 0x80, 0)).astype(np.uint16)
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(wd2), 2 * O.bf16_bits_to_f64(wd))
+    assert np.array_equal(O.moe_layer(x, lg, b, wg, wu, wd2), 2 * out)
+    # zero W_down gives zero output
+    assert np.all(O.moe_layer(x, lg, b, wg, wu, np.zeros_like(wd)) == 0)
+
+
+def test_stack_residual():
+    rng = np.random.default_rng(6)
+    E, H, I, T = 128, 32, 16, 5
+    layers = []
+    for _ in range(3):
+        wg, wu, wd = _weights(rng, E, H, I)
+        layers.append((rng.standard_normal((T, E)).astype(np.float32),
+                       (0.1 * rng.standard_normal(E)).astype(np.float32), wg, wu, wd))
+    x = _bf16(rng, (T, H), 1.0)
+    # one layer: bf16(x + layer(x))
+    h1 = O.moe_stack(x, layers[:1])
+    ref1 = O.f64_to_bf16_bits(O.bf16_bits_to_f64(x) + O.moe_layer(x, *layers[0]))
+    assert np.array_equal(h1, ref1)
+    # three layers equal three chained one-layer stacks
+    h = x
+    for L in layers:
+        h = O.moe_stack(h, [L])
+    assert np.array_equal(O.moe_stack(x, layers), h)
+    # zero down-projections leave the residual stream unchanged
+    zl = [(a, b, c, d, np.zeros_like(e)) for (a, b, c, d, e) in layers]
+    assert np.array_equal(O.moe_stack(x, zl), x)
+
+
+# ---------------------------------------------------------------- page facts
+
+def test_constants_match_pages():
+    f = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
+    assert O.N_EXPERTS == f["n_experts"]["value"]
+    assert O.N_GROUPS == f["n_groups"]["value"]
+    assert O.N_EXPERTS // O.N_GROUPS == f["group_size"]["value"]
+    assert O.KEEP_GROUPS == f["keep_groups"]["value"]
+    assert O.TOPK == f["topk"]["value"]
+    assert O.HIDDEN == f["hidden"]["value"]
+    assert O.N_MOE_LAYERS == f["layers_total"]["value"] - 1   # dense layer 0
+
+
+def test_intermediate_size_from_expert_weight_size():
+    """The pages do not print the expert intermediate size; the 4.2 GiB of
+    gate/up (Q4_K) + down (Q6_K) expert weights pins it: only I = 512 over the
+    23 MoE layers rounds to 4.2 GiB."""
+    f = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
+    q4, q6 = f["q4_k_bits_per_weight"]["value"], f["q6_k_bits_per_weight"]["value"]
+
+    def gib(layers, inter):
+        n = layers * O.N_EXPERTS * O.HIDDEN * inter
+        return n * (2 * q4 + q6) / 8 / 2 ** 30
+
+    assert round(gib(O.N_MOE_LAYERS, O.INTER), 1) == f["expert_weight_gib"]["value"]
+    for alt in (256, 384, 640, 768, 1024):
+        assert round(gib(O.N_MOE_LAYERS, alt), 1) != f["expert_weight_gib"]["value"]
+    assert round(gib(24, O.INTER), 1) != f["expert_weight_gib"]["value"]
