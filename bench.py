@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Throughput of the group-limited routed MoE layer (Ling-3.0-tiny shapes) on B200.
+
+One step = one whole layer (route -> permute -> gate/up GEMM -> down GEMM ->
+combine) through the C ABI on one batch of seeded synthetic tokens that are
+already resident in HBM.  The headline workload is the long-prompt prefill
+(8,189 real tokens in buffers of 8,192); the decode batch of 16 tokens is
+measured the same way and reported beside it.
+
+Timing: W warm-up steps, then exactly K timed steps between a barrier and a
+device synchronize.  Before every step a 256 MB buffer is overwritten to flush
+the 126 MB L2 (outside the step's events); each step is bracketed by CUDA
+events on the launching stream, with events between the five steps for the
+per-kernel breakdown.  Multi-GPU (torchrun): every rank runs its own
+independent batch (data-parallel replicas, weak scaling, no data-path
+collective); the reported time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from group_limited_routed_moe_b200 import synth  # noqa: E402
+
+GATE_UP_BYTES_PER_EXPERT = 2 * 1536 * 512 * 2
+DOWN_BYTES_PER_EXPERT = 1536 * 512 * 2
+FLOPS_PER_ROW = 2 * (1536 * 1024 + 512 * 1536)          # one (token, expert) pair
+GATE_UP_FLOPS_PER_ROW = 2 * 1536 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_T8189", choices=["prefill_T8189", "decode_T16"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the decode_T16 measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens in the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "group_limited_routed_moe_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    sha, traffic = None, None
+    for line in open(p):
+        if line.startswith("source_sha:"):
+            sha = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if sha == kernel_source_sha() else None
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML every few ms."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = str(e)
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": names}
+
+
+# --------------------------------------------------------------------- our arm
+
+class LayerRun:
+    """Device buffers and the five-call step of one workload."""
+
+    def __init__(self, wl: synth.Workload, dev, weights):
+        import torch
+        from group_limited_routed_moe_b200 import moe
+        self.moe, self.torch, self.wl, self.dev = moe, torch, wl, dev
+        self.T = wl.T
+        tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
+        self.tok = tok
+        T, Tb = wl.T, wl.T_buf
+        bf = torch.bfloat16
+        self.x = torch.zeros((Tb, 1536), dtype=bf, device=dev)
+        self.x[:T] = torch.from_numpy(tok.x_bits.view(np.int16)).to(dev).view(bf)
+        self.logits = torch.zeros((Tb, 128), dtype=torch.float32, device=dev)
+        self.logits[:T] = torch.from_numpy(tok.logits).to(dev)
+        self.bias = torch.from_numpy(tok.bias).to(dev)
+        self.packed = weights
+        n = T * 8
+        i32 = torch.int32
+        self.idx = torch.empty((T, 8), dtype=i32, device=dev)
+        self.w = torch.empty((T, 8), dtype=torch.float32, device=dev)
+        self.counts = torch.empty(128, dtype=i32, device=dev)
+        self.offsets = torch.empty(129, dtype=i32, device=dev)
+        self.perm_src = torch.empty(n, dtype=i32, device=dev)
+        self.inv_perm = torch.empty(n, dtype=i32, device=dev)
+        wsb = moe.permute_workspace_bytes(T)
+        self.pws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev) if wsb else None
+        self.h = torch.empty((n, 512), dtype=bf, device=dev)
+        self.y = torch.empty((n, 1536), dtype=bf, device=dev)
+        self.out = torch.empty((Tb, 1536), dtype=bf, device=dev)
+        self.launches_per_step = 5 if T <= 1024 else 7
+        self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream()
+
+    def flush(self):
+        self.flush_buf.fill_(1)
+
+    def step(self, ev=None):
+        m, T, s = self.moe, self.T, self.stream
+        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        rec(0)
+        m.moe_route(self.logits[:T], self.bias, self.idx, self.w, stream=s)
+        rec(1)
+        m.moe_permute(self.idx, self.counts, self.offsets, self.perm_src, self.inv_perm,
+                      self.pws, stream=s)
+        rec(2)
+        m.moe_expert_gate_up(self.x[:T], self.packed, self.offsets, self.perm_src, self.h, stream=s)
+        rec(3)
+        m.moe_expert_down(self.h, self.packed, self.offsets, self.y, stream=s)
+        rec(4)
+        m.moe_combine(self.y, self.w, self.inv_perm, out=self.out[:T], stream=s)
+        rec(5)
+
+    def timed(self, steps, warmup, barrier):
+        torch = self.torch
+        for _ in range(warmup):
+            self.flush()
+            self.step()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for k in range(steps):
+            self.flush()
+            self.step(evs[k])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        barrier()
+        per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)]
+                        for k in range(steps)])  # ms
+        return per, wall
+
+    def e2e(self, steps, warmup):
+        """Same layer from pinned host buffers: H2D x + logits, layer, D2H out."""
+        torch, moe = self.torch, self.moe
+        T = self.T
+        x_h = torch.from_numpy(self.tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        lg_h = torch.from_numpy(self.tok.logits).pin_memory()
+        out_h = torch.empty((T, 1536), dtype=torch.bfloat16).pin_memory()
+        ws = moe.alloc_layer_workspace(T, self.dev)
+        s = self.stream
+
+        def one():
+            moe.moe_layer_from_host(x_h, lg_h, self.bias, self.packed, self.x[:T],
+                                    self.logits[:T], self.out[:T], out_h, ws, stream=s)
+        for _ in range(warmup):
+            self.flush()
+            one()
+        times = []
+        for _ in range(steps):
+            self.flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            one()
+            b.record(s)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        return float(np.mean(times)), x_h.numel() * 2 + lg_h.numel() * 4, out_h.numel() * 2
+
+
+def distinct_experts(tok):
+    import oracle as O  # the oracle's routing fixes which experts a batch touches
+    return int(np.unique(O.route(tok.logits, tok.bias).topk_idx).size)
+
+
+def roofline_for(wl, tok, per_ms, peaks, peak_kind):
+    """Roofline of the dominant kernel (the gate/up GEMM) of one workload."""
+    gate_up_ms = float(per_ms[:, 2].mean())
+    T = wl.T
+    if T >= 2048:
+        flops = GATE_UP_FLOPS_PER_ROW * 8 * T
+        key = "bf16_tflops"
+        peak = float(peaks[key])
+        achieved = flops / (gate_up_ms * 1e-3) / 1e12
+        return {"kernel": "ffn_gemm_kernel<1> (gate/up + SwiGLU)", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} {key} (burst)",
+                "algorithmic_per_launch": flops,
+                "traffic": profiled_traffic("gate_up", wl.name)}
+    d = distinct_experts(tok)
+    nbytes = d * GATE_UP_BYTES_PER_EXPERT + T * 1536 * 2 + 8 * T * 512 * 2
+    peak = float(peaks["hbm_gbs"])
+    achieved = nbytes / (gate_up_ms * 1e-3) / 1e9
+    return {"kernel": "ffn_gemm_kernel<1> (gate/up + SwiGLU)", "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_per_launch": nbytes, "distinct_experts": d,
+            "traffic": profiled_traffic("gate_up", wl.name)}
+
+
+def layer_fractions(wl, tok, per_ms, peaks):
+    """Whole-layer fractions (context): tokens/s against the HBM bound of the
+    distinct experts' weights and against the tensor bound of the useful flops."""
+    layer_s = float(per_ms.sum(axis=1).mean()) * 1e-3
+    d = distinct_experts(tok)
+    nbytes = d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + wl.T * (1536 * 4 + 512)
+    flops = FLOPS_PER_ROW * 8 * wl.T
+    return {"layer_us": round(layer_s * 1e6, 2),
+            "hbm_frac": round(nbytes / layer_s / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "tensor_frac": round(flops / layer_s / 1e12 / float(peaks["bf16_tflops"]), 4),
+            "kernel_us": {k: round(float(per_ms[:, i].mean()) * 1e3, 2) for i, k in
+                          enumerate(["route", "permute", "gate_up", "down", "combine"])},
+            "distinct_experts": d}
+
+
+def cpu_baseline(wl, tok, host_w, sample):
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    n = min(sample, wl.T)
+    rows = np.arange(n)
+    t0 = time.perf_counter()
+    O.moe_layer(tok.x_bits[rows], tok.logits[rows], tok.bias, *host_w)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n} of {wl.T} tokens of {wl.name}, float64 NumPy oracle, {dt:.2f} s"}
+
+
+def run_ours(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    from group_limited_routed_moe_b200 import moe
+    peaks, peak_kind = load_peaks()
+
+    wg = synth.weight_bits_torch(0, 0, synth.W_GATE, dev)
+    wu = synth.weight_bits_torch(0, 0, synth.W_UP, dev)
+    wd = synth.weight_bits_torch(0, 0, synth.W_DOWN, dev)
+    packed = moe.moe_pack_weights(wg, wu, wd)
+    torch.cuda.synchronize()
+
+    def host_weights():
+        def h(t):
+            return t.view(torch.int16).cpu().numpy().view(np.uint16)
+        return h(wg), h(wu), h(wd)
+
+    wl = synth.WORKLOADS[args.workload]
+    run = LayerRun(wl, dev, packed)
+    clk = ClockSampler(local)
+    with clk:
+        per, wall = run.timed(args.steps, args.warmup, barrier)
+    step_ms = float(per.sum(axis=1).mean())
+    elapsed = torch.tensor([step_ms * args.steps], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(elapsed, op=dist.ReduceOp.MAX)
+    ms_per_step = float(elapsed.item()) / args.steps
+    value = wl.T * world / (ms_per_step * 1e-3)
+    e2e_ms, h2d, d2h = run.e2e(max(3, args.steps // 4), 2)
+
+    line = {
+        "metric": f"MoE-layer tokens/s ({wl.name}: T={wl.T}, hidden 1536, 128 experts top-8)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "T_buf": wl.T_buf, "hidden": 1536,
+                   "experts": 128, "groups": 8, "keep_groups": 4, "topk": 8, "inter": 512,
+                   "parallelism": f"dp{world} (independent batch per GPU)",
+                   "l2": "256 MB buffer overwritten before every step (outside the timed events)",
+                   "wall_s_timed_region": round(wall, 4)},
+        "roofline": roofline_for(wl, run.tok, per, peaks, peak_kind),
+        "layer": layer_fractions(wl, run.tok, per, peaks),
+        "e2e": {"value": round(wl.T * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": run.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_secondary and wl.name != "decode_T16":
+        wl2 = synth.WORKLOADS["decode_T16"]
+        run2 = LayerRun(wl2, dev, packed)
+        clk2 = ClockSampler(local)
+        with clk2:
+            per2, wall2 = run2.timed(max(args.steps, 50), args.warmup, barrier)
+        e2e2, h2d2, d2h2 = run2.e2e(20, 3)
+        ms2 = float(per2.sum(axis=1).mean())
+        line["decode_T16"] = {
+            "value": round(wl2.T / (ms2 * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms2, 5),
+            "roofline": roofline_for(wl2, run2.tok, per2, peaks, peak_kind),
+            "layer": layer_fractions(wl2, run2.tok, per2, peaks),
+            "e2e": {"value": round(wl2.T / (e2e2 * 1e-3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d2, "d2h_bytes_per_step": d2h2},
+            "gpu_launches": run2.launches_per_step * max(args.steps, 50),
+            "clocks": clk2.summary()}
+        line["gpu_launches"] += line["decode_T16"]["gpu_launches"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, run.tok, host_weights(), args.cpu_sample)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The float64 oracle as the reference arm: rank 0 only, host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    wl = synth.WORKLOADS[args.workload]
+    tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
+    per_step = min(wl.T, 64)
+    rr = O.route(tok.logits, tok.bias)
+    host_w = synth.layer_weights_np(0, 0)
+    for k in range(args.warmup):
+        rows = (np.arange(per_step) + k * per_step) % wl.T
+        O.moe_layer(tok.x_bits[rows], tok.logits[rows], tok.bias, *host_w)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        rows = (np.arange(per_step) + k * per_step) % wl.T
+        O.moe_layer(tok.x_bits[rows], tok.logits[rows], tok.bias, *host_w)
+    dt = time.perf_counter() - t0
+    del rr
+    value = per_step * args.steps / dt
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    line = {
+        "impl": "reference",
+        "metric": f"MoE-layer tokens/s ({wl.name}: T={wl.T}, hidden 1536, 128 experts top-8)",
+        "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "T_buf": wl.T_buf,
+                   "step": f"{per_step} tokens of the batch per step"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"{per_step} tokens per step x {args.steps} steps of {wl.name}"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,68 @@
+// combine.cuh -- step 4: weighted combine of the 8 expert outputs of every
+// token, back in token order.
+//
+// out[t] = bf16( residual[t] + sum_{slot} w[t,slot] * y_perm[inv_perm[8t+slot]] )
+// The "real MoE routing + weighted layer" of "HelloSun/ling30tiny" (section
+// 數值檢查摘要) is this sum.  It is done in gather form: each token reads its 8
+// rows, adds them in fp32 in slot order and rounds once, so the result is
+// deterministic (no atomics) and independent of how tokens are ordered.
+// One thread owns 8 consecutive columns (one 16-byte vector) of one token.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kCombineThreads = kH / 8;  // 192
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const float* __restrict__ topk_w,
+                   const int32_t* __restrict__ inv_perm, int64_t T,
+                   const __nv_bfloat16* residual, __nv_bfloat16* out) {
+  const int64_t t = blockIdx.x;
+  if (t >= T) return;
+  const int col = threadIdx.x * 8;
+  const int64_t nrows = T * kTopK;
+
+  uint4 v[kTopK];
+  float w[kTopK];
+#pragma unroll
+  for (int s = 0; s < kTopK; ++s) {
+    const int64_t r = __ldg(inv_perm + t * kTopK + s);
+    w[s] = __ldg(topk_w + t * kTopK + s);
+    if (r >= 0 && r < nrows) {
+      v[s] = __ldg(reinterpret_cast<const uint4*>(y_perm + r * kH + col));
+    } else {
+      v[s] = make_uint4(0u, 0u, 0u, 0u);
+      w[s] = 0.f;
+    }
+  }
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int s = 0; s < kTopK; ++s) {
+    const uint32_t q[4] = {v[s].x, v[s].y, v[s].z, v[s].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] = fmaf(w[s], bf16_lo(q[i]), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(w[s], bf16_hi(q[i]), acc[2 * i + 1]);
+    }
+  }
+  if (residual != nullptr) {
+    const uint4 rv = *reinterpret_cast<const uint4*>(residual + t * kH + col);
+    const uint32_t q[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += bf16_lo(q[i]);
+      acc[2 * i + 1] += bf16_hi(q[i]);
+    }
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(out + t * kH + col) = o;
+}
+
+}  // namespace moe

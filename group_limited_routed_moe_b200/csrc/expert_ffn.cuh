@@ -1,0 +1,363 @@
+// expert_ffn.cuh -- step 3: the grouped SwiGLU expert FFN as two persistent
+// tcgen05 GEMMs over the permuted rows.
+//
+// Every expert has gate, up and down matrices ("HelloSun/ling30tiny", table
+// 模型與路由, row on expert weights) and no SwiGLU clamp ("Ling-3.0-tiny on a
+// Qualcomm board", TensorFold issue #1247, first comment: "null SwiGLU limit
+// lists").  The same issue names the missing piece this replaces: the bf16
+// experts there have "no grouped kernel" and run a per-expert row loop.
+//
+//   phase 1 (gate/up):  h[r]      = silu(x[tok(r)] W_gate[e]) * (x[tok(r)] W_up[e])
+//                       M_e x N 1024 x K 1536 per expert, N tiled by 256 =
+//                       128 gate + 128 up columns, SwiGLU in the epilogue.
+//   phase 2 (down):     y_perm[r] = h[r] W_down[e]
+//                       M_e x N 1536 x K 512 per expert, N tiled by 256.
+//
+// Work is cut into tiles (expert e, n-tile j, m-tile m) of 128 rows x 256
+// columns; tile ids run expert-major, then j, then m, so consecutive CTAs
+// share an expert's weight tile through L2.  A persistent grid of one CTA per
+// SM walks the ids round-robin.  The tile table is built by each CTA from the
+// device-side expert offsets, so the host never reads them.
+//
+// Warp roles inside a CTA (one CTA per SM: ~194 KB of shared memory, all 512
+// TMEM columns):
+//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SwiGLU / bf16, stores
+//   warps 4-7  (phase 1) A producers: gather the tile's 128 token rows of x
+//              with cp.async into the 128B-swizzled operand layout
+//   next warp  TMA producer: weight tiles (and, in phase 2, h tiles)
+//   next warp  MMA issuer: tcgen05.mma 128x256x16, accumulator in TMEM,
+//              double-buffered (2 x 256 columns) so the epilogue of tile i
+//              overlaps the MMAs of tile i+1.
+// Shared-memory ring: 4 stages of (A 128x64 + B 256x64) bf16.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+namespace ffn {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int TILE_BYTES = STAGES * (A_BYTES + B_BYTES);
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int GATHER_LAG = 2;  // cp.async groups kept in flight per producer thread
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+template <int PHASE>
+struct Cfg;
+template <>
+struct Cfg<1> {
+  static constexpr int KDIM = kH;                 // 1536
+  static constexpr int NT = kI / 128;             // 4 n-tiles of 128 gate + 128 up
+  static constexpr int B_ROWS_PER_EXPERT = 2 * kI;  // 1024 packed rows
+  static constexpr int OUT_COLS = kI;             // h row length
+  static constexpr int THREADS = 320;
+  static constexpr int TMA_WARP = 8;
+  static constexpr int MMA_WARP = 9;
+  static constexpr int FULL_COUNT = 1 + 4;        // TMA arrive + 4 gather warps
+};
+template <>
+struct Cfg<2> {
+  static constexpr int KDIM = kI;                 // 512
+  static constexpr int NT = kH / BN;              // 6
+  static constexpr int B_ROWS_PER_EXPERT = kH;    // 1536 packed rows
+  static constexpr int OUT_COLS = kH;             // y_perm row length
+  static constexpr int THREADS = 192;
+  static constexpr int TMA_WARP = 4;
+  static constexpr int MMA_WARP = 5;
+  static constexpr int FULL_COUNT = 1;
+};
+
+struct SmemTail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int wsum[4];
+  int tile_start[kE + 1];
+  int cnt[kE];
+  int off[kE];
+};
+constexpr int SMEM_BYTES = TILE_BYTES + static_cast<int>(sizeof(SmemTail)) + 1024;
+
+__device__ __forceinline__ void decode_tile(const SmemTail* S, int tile, int NT, int& e, int& m,
+                                            int& j) {
+  int lo = 0, hi = kE - 1;  // largest e with tile_start[e] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (S->tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int rem = tile - S->tile_start[e];
+  const int mt = (S->cnt[e] + BM - 1) / BM;
+  j = rem / mt;
+  m = rem - j * mt;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+template <int PHASE>
+__global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
+    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_a,
+                    const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
+                    const int32_t* __restrict__ perm_src, int64_t T,
+                    __nv_bfloat16* __restrict__ out, uint64_t timeout_ns) {
+  using C = Cfg<PHASE>;
+  constexpr int KB = C::KDIM / BK;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;                       // STAGES x 16 KB
+  uint8_t* sB = smem + STAGES * A_BYTES;    // STAGES x 32 KB
+  SmemTail* S = reinterpret_cast<SmemTail*>(smem + TILE_BYTES);
+  volatile int* abort_flag = &S->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nrows = T * kTopK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&S->full[s], C::FULL_COUNT);
+      mbar_init(&S->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&S->tfull[a], 1);
+      mbar_init(&S->tempty[a], 4);
+    }
+    mbar_init(&S->drain, 1);
+    S->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == C::TMA_WARP && lane == 0) {
+    tma_prefetch_desc(&tmap_b);
+    if (PHASE == 2) tma_prefetch_desc(&tmap_a);
+  }
+
+  // tile table: tiles of expert e = ceil(count_e / 128) * NT, exclusive prefix
+  int my_tiles = 0;
+  if (threadIdx.x < kE) {
+    const int e = threadIdx.x;
+    const int o0 = offsets[e], o1 = offsets[e + 1];
+    int c = o1 - o0;
+    if (o0 < 0 || c < 0 || static_cast<int64_t>(o1) > nrows) {
+      record_status(kSiteBadIndex);
+      c = 0;
+    }
+    S->cnt[e] = c;
+    S->off[e] = o0;
+    my_tiles = ((c + BM - 1) / BM) * C::NT;
+  }
+  int incl = my_tiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
+
+  if (warp == C::MMA_WARP) tmem_alloc(&S->tmem_base, TMEM_COLS);
+  __syncthreads();
+  if (threadIdx.x < kE) {
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += S->wsum[w];
+    S->tile_start[threadIdx.x] = base + incl - my_tiles;
+    if (threadIdx.x == kE - 1) S->tile_start[kE] = base + incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = S->tmem_base;
+  const int total_tiles = S->tile_start[kE];
+
+  if (warp == C::TMA_WARP) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int e, m, j;
+        decode_tile(S, tile, C::NT, e, m, j);
+        const int brow = e * C::B_ROWS_PER_EXPERT + j * BN;
+        const int arow = S->off[e] + m * BM;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&S->empty[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
+            ok = false;
+            break;
+          }
+          if (PHASE == 2) {
+            mbar_arrive_expect_tx(&S->full[s], A_BYTES + B_BYTES);
+            tma_load_2d(smem_u32(sA + s * A_BYTES), &tmap_a, kb * BK, arow, &S->full[s]);
+          } else {
+            mbar_arrive_expect_tx(&S->full[s], B_BYTES);
+          }
+          tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b, kb * BK, brow, &S->full[s]);
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the block can exit
+        for (int i = max(0, it - STAGES); i < it; ++i)
+          mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, abort_flag, 10000000ull, kSiteFfnFull);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tc) {
+        const int a = tc & 1;
+        const uint32_t use = tc >> 1;
+        if (!mbar_wait(&S->tempty[a], (use & 1) ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + a * BN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&S->full[s], ph, abort_flag, timeout_ns, kSiteFfnFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_BYTES));
+          const uint64_t bdesc = smem_desc_k128(smem_u32(sB + s * B_BYTES));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(d, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&S->empty[s]);
+        }
+        if (ok) umma_commit(&S->tfull[a]);
+      }
+      // every MMA this thread issued must be complete before TMEM is freed
+      umma_commit(&S->drain);
+      mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
+    }
+  } else if (PHASE == 1 && warp >= 4 && warp < 8) {
+    // ------------------------------------------------ A gather producers
+    const int r = threadIdx.x - 128;  // row of the tile
+    const uint32_t swz = static_cast<uint32_t>(r & 7);
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, m, j;
+      decode_tile(S, tile, C::NT, e, m, j);
+      const int row_in_e = m * BM + r;
+      const char* src = reinterpret_cast<const char*>(x);
+      uint32_t nbytes = 0;
+      if (row_in_e < S->cnt[e]) {
+        const int p = perm_src[S->off[e] + row_in_e];
+        if (p >= 0 && static_cast<int64_t>(p) < nrows) {
+          src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
+          nbytes = 16;
+        }
+      }
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(&S->empty[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = smem_u32(sA + s * A_BYTES) + r * 128;
+        const char* g = src + kb * BK * 2;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          cp_async_16(dst + ((static_cast<uint32_t>(c) ^ swz) << 4), g + c * 16, nbytes);
+        cp_async_commit();
+        if (it >= GATHER_LAG) {
+          cp_async_wait_group<GATHER_LAG>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S->full[(it - GATHER_LAG) % STAGES]);
+        }
+      }
+    }
+    cp_async_wait_group<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (ok && lane == 0)
+      for (int i = max(0, it - GATHER_LAG); i < it; ++i) mbar_arrive(&S->full[i % STAGES]);
+  } else if (warp < 4) {
+    // ------------------------------------------------ epilogue
+    const int r = threadIdx.x;  // row of the tile == TMEM lane
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
+      int e, m, j;
+      decode_tile(S, tile, C::NT, e, m, j);
+      const int a = tc & 1;
+      const uint32_t use = tc >> 1;
+      if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
+      tc_fence_after();
+      const int row_in_e = m * BM + r;
+      const bool valid = row_in_e < S->cnt[e];
+      const int64_t prow = static_cast<int64_t>(S->off[e]) + row_in_e;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * BN;
+      if (PHASE == 1) {
+        __nv_bfloat16* dst = out + prow * C::OUT_COLS + j * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld_2x32(tbase + c * 32, tbase + 128 + c * 32, g, u);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                silu_mul(__uint_as_float(g[2 * i + 1]),
+                                         __uint_as_float(u[2 * i + 1])));
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              st_global_v4(dst + c * 32 + q * 8, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                           pk[4 * q + 3]);
+          }
+        }
+      } else {
+        __nv_bfloat16* dst = out + prow * C::OUT_COLS + j * BN;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_2x32(tbase + c * 64, tbase + c * 64 + 32, v0, v1);
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+            pk[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+          }
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              st_global_v4(dst + c * 64 + q * 8, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                           pk[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->tempty[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace ffn
+}  // namespace moe

@@ -1,0 +1,462 @@
+// moe.cu -- libmoe: the C ABI declared in include/moe.h.
+//
+// Host code here only validates arguments, encodes TMA descriptors and
+// launches kernels; it never allocates, synchronises or reads device memory
+// (moe_get_device_status() excepted, which copies one status word).
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "combine.cuh"
+#include "common.cuh"
+#include "expert_ffn.cuh"
+#include "pack.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr int64_t kMaxTokens = int64_t(1) << 22;
+constexpr int kMaxDevices = 64;
+
+thread_local char g_err[512] = "";
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MOE_CUDA(call, what)                    \
+  do {                                          \
+    cudaError_t e_ = (call);                    \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---- per-device setup (once): SM count, arch check, kernel attributes -------
+struct DeviceInfo {
+  int sms = 0;
+  int status = -1;  // -1 unset, otherwise moe_status
+  char msg[256] = "";
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_setup(int* dev_out, int* sms_out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.status < 0) {
+    cudaDeviceProp prop;
+    cudaError_t e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0) {
+      d.status = MOE_ERR_UNSUPPORTED;
+      snprintf(d.msg, sizeof(d.msg), "libmoe is built for sm_100a (B200); device %d is sm_%d%d",
+               dev, prop.major, prop.minor);
+    } else {
+      d.sms = prop.multiProcessorCount;
+      e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<1>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      if (g_encode == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+          return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      }
+      d.status = MOE_OK;
+    }
+  }
+  if (d.status != MOE_OK) return fail(d.status, "%s", d.msg);
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = d.sms;
+  return MOE_OK;
+}
+
+// 2-D bf16 tensor map: `rows` rows of `cols` elements, box of 64 x box_rows,
+// 128-byte swizzle (matches the UMMA K-major SW128 operand layout).
+int make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MOE_OK;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int check_T(int64_t T) {
+  if (T < 0 || T > kMaxTokens)
+    return fail(MOE_ERR_INVALID_ARG, "T=%lld outside [0, %lld]", static_cast<long long>(T),
+                static_cast<long long>(kMaxTokens));
+  return MOE_OK;
+}
+
+#define REQUIRE(cond, ...)                                         \
+  do {                                                             \
+    if (!(cond)) return fail(MOE_ERR_INVALID_ARG, __VA_ARGS__);    \
+  } while (0)
+
+int launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return MOE_OK;
+}
+
+// ---- step launchers (arguments already validated) ----------------------------
+int do_route(const float* logits, const float* bias, int64_t T, int32_t* idx, float* w,
+             cudaStream_t s) {
+  const int64_t blocks = (T + kRouteWarps - 1) / kRouteWarps;
+  route_kernel<<<static_cast<unsigned>(blocks), kRouteWarps * 32, 0, s>>>(logits, bias, T, idx, w);
+  return launch_check("route_kernel launch");
+}
+
+size_t permute_ws_bytes(int64_t T) {
+  if (T <= kPermSmallMaxT) return 0;
+  const int64_t nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  return align_up(static_cast<size_t>(nb) * kE * sizeof(int32_t), 256);
+}
+
+int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets, int32_t* perm_src,
+               int32_t* inv_perm, void* ws, cudaStream_t s) {
+  if (T <= kPermSmallMaxT) {
+    permute_small_kernel<<<1, 1024, 0, s>>>(idx, static_cast<int>(T), counts, offsets, perm_src,
+                                            inv_perm);
+    return launch_check("permute_small_kernel launch");
+  }
+  const int64_t nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  int32_t* hist = static_cast<int32_t*>(ws);
+  permute_count_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(idx, T, hist);
+  int rc = launch_check("permute_count_kernel launch");
+  if (rc) return rc;
+  permute_scan_kernel<<<1, 1024, 0, s>>>(hist, static_cast<int>(nb), counts, offsets);
+  rc = launch_check("permute_scan_kernel launch");
+  if (rc) return rc;
+  permute_scatter_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(idx, T, hist, offsets, perm_src,
+                                                                   inv_perm);
+  return launch_check("permute_scatter_kernel launch");
+}
+
+int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
+               const int32_t* perm_src, int64_t T, moe_bf16* h, int sms, cudaStream_t s) {
+  CUtensorMap tb1;
+  int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN);
+  if (rc) return rc;
+  ffn::ffn_gemm_kernel<1><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
+      tb1, tb1, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+      reinterpret_cast<__nv_bfloat16*>(h), g_timeout_ns.load());
+  return launch_check("ffn_gemm_kernel<1> launch");
+}
+
+int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, int64_t T,
+            moe_bf16* y, int sms, cudaStream_t s) {
+  CUtensorMap tb2, ta2;
+  const uint64_t rows = static_cast<uint64_t>(T) * kTopK;
+  int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN);
+  if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM);
+  if (rc) return rc;
+  ffn::ffn_gemm_kernel<2><<<sms, ffn::Cfg<2>::THREADS, ffn::SMEM_BYTES, s>>>(
+      tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<__nv_bfloat16*>(y),
+      g_timeout_ns.load());
+  return launch_check("ffn_gemm_kernel<2> launch");
+}
+
+int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
+                  const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, int sms,
+                  cudaStream_t s) {
+  int rc = do_gate_up(x, packed, offsets, perm_src, T, h, sms, s);
+  if (rc) return rc;
+  return do_down(h, packed, offsets, T, y, sms, s);
+}
+
+int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
+               const moe_bf16* residual, moe_bf16* out, cudaStream_t s) {
+  combine_kernel<<<static_cast<unsigned>(T), kCombineThreads, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(y), w, inv, T,
+      reinterpret_cast<const __nv_bfloat16*>(residual), reinterpret_cast<__nv_bfloat16*>(out));
+  return launch_check("combine_kernel launch");
+}
+
+// workspace carve-up of moe_layer
+struct LayerWs {
+  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, total;
+};
+LayerWs layer_ws(int64_t T) {
+  LayerWs L{};
+  const size_t n = static_cast<size_t>(T) * kTopK;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 1024);
+    return at;
+  };
+  L.idx = take(n * 4);
+  L.w = take(n * 4);
+  L.counts = take(kE * 4);
+  L.offsets = take((kE + 1) * 4);
+  L.perm_src = take(n * 4);
+  L.inv_perm = take(n * 4);
+  L.perm_ws = take(permute_ws_bytes(T));
+  L.h = take(n * kI * 2);
+  L.y = take(n * kH * 2);
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+// =============================================================================
+extern "C" {
+
+int moe_abi_version(void) { return kAbiVersion; }
+int64_t moe_max_tokens(void) { return kMaxTokens; }
+const char* moe_last_error_string(void) { return g_err; }
+
+int moe_get_device_status(int device) {
+  int prev = 0;
+  MOE_CUDA(cudaGetDevice(&prev), "cudaGetDevice");
+  MOE_CUDA(cudaSetDevice(device), "cudaSetDevice");
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  const unsigned zero = 0;
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (v == 0) return MOE_OK;
+  if ((v & 0x7FFFFFFFu) == kSiteBadIndex)
+    return fail(MOE_ERR_INVALID_ARG, "a kernel met an out-of-range index (status 0x%08x)", v);
+  return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out (status 0x%08x, site %u)", v,
+              v & 0x7FFFFFFFu);
+}
+
+int moe_set_wait_timeout_ns(uint64_t ns) {
+  if (ns < 1000ull) return fail(MOE_ERR_INVALID_ARG, "timeout below 1 us");
+  g_timeout_ns.store(ns);
+  return MOE_OK;
+}
+
+size_t moe_packed_weight_bytes(void) { return static_cast<size_t>(kPackElems) * 2; }
+
+int moe_pack_weights(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                     moe_bf16* packed, moe_stream_t stream) {
+  REQUIRE(w_gate && w_up && w_down && packed, "null pointer");
+  REQUIRE(aligned(packed, 128), "packed must be 128-byte aligned");
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 ggu(kI / 32, kH / 32, kE), gd(kH / 32, kI / 32, kE);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_gate, packed, kH, kI, 0);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_up, packed, kH, kI, 1);
+  pack_transpose_kernel<<<gd, 256, 0, s>>>(w_down, packed, kI, kH, 2);
+  return launch_check("pack_transpose_kernel launch");
+}
+
+int moe_route(const float* logits, const float* bias, int64_t T, int32_t* topk_idx, float* topk_w,
+              moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(logits && topk_idx && topk_w, "null pointer");
+  REQUIRE(aligned(logits, 16) && (!bias || aligned(bias, 16)) && aligned(topk_idx, 16) &&
+              aligned(topk_w, 16),
+          "pointers must be 16-byte aligned");
+  rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  return do_route(logits, bias, T, topk_idx, topk_w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_permute_workspace_bytes(int64_t T) {
+  if (T < 0 || T > kMaxTokens) return 0;
+  return permute_ws_bytes(T);
+}
+
+int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts, int32_t* offsets,
+                int32_t* perm_src, int32_t* inv_perm, void* workspace, size_t workspace_bytes,
+                moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  REQUIRE(counts && offsets, "null pointer");
+  if (T > 0) REQUIRE(topk_idx && perm_src && inv_perm, "null pointer");
+  const size_t need = permute_ws_bytes(T);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(MOE_ERR_WORKSPACE, "permute workspace needs %zu bytes, got %zu", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (need > 0) REQUIRE(aligned(workspace, 16), "workspace must be 16-byte aligned");
+  rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, kE * sizeof(int32_t), s), "cudaMemsetAsync");
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (kE + 1) * sizeof(int32_t), s), "cudaMemsetAsync");
+    return MOE_OK;
+  }
+  return do_permute(topk_idx, T, counts, offsets, perm_src, inv_perm, workspace, s);
+}
+
+int moe_expert_ffn(const moe_bf16* x, const moe_bf16* packed_w, const int32_t* offsets,
+                   const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y_perm,
+                   moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && packed_w && offsets && perm_src && h && y_perm, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_w, 128) && aligned(h, 128),
+          "x, packed_w and h must be 128-byte aligned");
+  REQUIRE(aligned(y_perm, 16) && aligned(offsets, 16) && aligned(perm_src, 16),
+          "pointers must be 16-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y_perm, sms,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_gate_up(const moe_bf16* x, const moe_bf16* packed_w, const int32_t* offsets,
+                       const int32_t* perm_src, int64_t T, moe_bf16* h, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && packed_w && offsets && perm_src && h, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_w, 128) && aligned(h, 128),
+          "x, packed_w and h must be 128-byte aligned");
+  REQUIRE(aligned(offsets, 16) && aligned(perm_src, 16), "pointers must be 16-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_gate_up(x, packed_w, offsets, perm_src, T, h, sms,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_down(const moe_bf16* h, const moe_bf16* packed_w, const int32_t* offsets,
+                    int64_t T, moe_bf16* y_perm, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(h && packed_w && offsets && y_perm, "null pointer");
+  REQUIRE(aligned(packed_w, 128) && aligned(h, 128), "packed_w and h must be 128-byte aligned");
+  REQUIRE(aligned(y_perm, 16) && aligned(offsets, 16), "pointers must be 16-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_down(h, packed_w, offsets, T, y_perm, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_combine(const moe_bf16* y_perm, const float* topk_w, const int32_t* inv_perm, int64_t T,
+                const moe_bf16* residual, moe_bf16* out, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(y_perm && topk_w && inv_perm && out, "null pointer");
+  REQUIRE(aligned(y_perm, 16) && aligned(topk_w, 16) && aligned(inv_perm, 16) &&
+              aligned(out, 16) && (!residual || aligned(residual, 16)),
+          "pointers must be 16-byte aligned");
+  rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  return do_combine(y_perm, topk_w, inv_perm, T, residual, out,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_layer_workspace_bytes(int64_t T) {
+  if (T < 0 || T > kMaxTokens) return 0;
+  return layer_ws(T).total;
+}
+
+int moe_layer(const moe_bf16* x, const float* logits, const float* bias, const moe_bf16* packed_w,
+              int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+              float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && logits && packed_w && out && workspace, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_w, 128), "x and packed_w must be 128-byte aligned");
+  REQUIRE(aligned(workspace, 1024), "workspace must be 1024-byte aligned");
+  REQUIRE(aligned(logits, 16) && (!bias || aligned(bias, 16)) && aligned(out, 16) &&
+              (!residual || aligned(residual, 16)) && (!topk_idx_out || aligned(topk_idx_out, 16)) &&
+              (!topk_w_out || aligned(topk_w_out, 16)),
+          "pointers must be 16-byte aligned");
+  const LayerWs L = layer_ws(T);
+  if (workspace_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE, "moe_layer workspace needs %zu bytes, got %zu", L.total,
+                workspace_bytes);
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
+  int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  moe_bf16* h = reinterpret_cast<moe_bf16*>(ws + L.h);
+  moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
+
+  rc = do_route(logits, bias, T, idx, w, s);
+  if (!rc) rc = do_permute(idx, T, counts, offsets, perm_src, inv_perm, ws + L.perm_ws, s);
+  if (!rc) rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
+  if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s);
+  return rc;
+}
+
+}  // extern "C"
+
+// ---- timeout self-test ------------------------------------------------------
+namespace {
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, int* done_flag) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // nothing ever arrives
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, &abort_flag, timeout_ns, kSiteSelftest);
+    (void)ok;
+  }
+  __syncthreads();
+}
+}  // namespace
+
+extern "C" int moe_selftest_wait_timeout(moe_stream_t stream) {
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(g_timeout_ns.load(),
+                                                                             nullptr);
+  return launch_check("selftest_wait_kernel launch");
+}

@@ -1,0 +1,192 @@
+// permute.cuh -- step 2: device-side stable counting sort of the T*8
+// (token, slot) items by expert.
+//
+// Each expert must run on exactly the rows that picked it; in the GB10 path of
+// "Ling-3.0-tiny on a Qualcomm board" (TensorFold issue #1247, "What it does
+// not cover", bullet on bf16 experts) finding those rows costs a host sync per
+// layer.  Here the row sets are built on the device and never leave it.
+//
+// Because a token picks an expert at most once, the rank of item (t, slot)
+// inside expert e is the number of earlier tokens that picked e.  A bitmap
+// [expert][token] answers that with popcounts, so the sort needs no atomics on
+// global memory and its output is deterministic:
+//   row(t, slot) = offsets[e] + (tokens before this block that picked e)
+//                             + popcount(bitmap[e][tokens of this block before t]).
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermSmallMaxT = 1024;   // single-block path up to this many tokens
+constexpr int kPermBlockTokens = 128;  // tokens per block on the multi-block path
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+// Exclusive scan of cnt[0..127] into off[0..128], run by warp 0 only.
+__device__ __forceinline__ void scan_experts_warp0(const int* cnt, int* off, int lane) {
+  const int c0 = cnt[4 * lane], c1 = cnt[4 * lane + 1], c2 = cnt[4 * lane + 2],
+            c3 = cnt[4 * lane + 3];
+  const int loc = c0 + c1 + c2 + c3;
+  const int incl = warp_incl_scan(loc, lane);
+  const int base = incl - loc;
+  off[4 * lane] = base;
+  off[4 * lane + 1] = base + c0;
+  off[4 * lane + 2] = base + c0 + c1;
+  off[4 * lane + 3] = base + c0 + c1 + c2;
+  if (lane == 31) off[kE] = incl;
+}
+
+// ---- single block, T <= 1024: bitmap of 128 experts x 1024 tokens ---------
+__global__ void __launch_bounds__(1024)
+    permute_small_kernel(const int32_t* __restrict__ idx, int T, int32_t* __restrict__ counts,
+                         int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
+                         int32_t* __restrict__ inv_perm) {
+  __shared__ uint32_t bm[kE][32];
+  __shared__ uint32_t pre[kE][32];
+  __shared__ int cnt[kE];
+  __shared__ int off[kE + 1];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int words = (T + 31) >> 5;
+
+  for (int i = tid; i < kE * 32; i += blockDim.x) (&bm[0][0])[i] = 0u;
+  __syncthreads();
+  const int n = T * kTopK;
+  for (int p = tid; p < n; p += blockDim.x) {
+    const int e = idx[p];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
+      record_status(kSiteBadIndex);
+      continue;
+    }
+    const int t = p >> 3;
+    atomicOr(&bm[e][t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  for (int e = warp; e < kE; e += 32) {
+    const int c = lane < words ? __popc(bm[e][lane]) : 0;
+    const int incl = warp_incl_scan(c, lane);
+    pre[e][lane] = incl - c;
+    if (lane == 31) cnt[e] = incl;
+  }
+  __syncthreads();
+  if (warp == 0) scan_experts_warp0(cnt, off, lane);
+  __syncthreads();
+  if (tid < kE) {
+    counts[tid] = cnt[tid];
+    offsets[tid] = off[tid];
+  }
+  if (tid == 0) offsets[kE] = off[kE];
+  for (int p = tid; p < n; p += blockDim.x) {
+    const int e = idx[p];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    const int t = p >> 3;
+    const int r = off[e] + pre[e][t >> 5] + __popc(bm[e][t >> 5] & ((1u << (t & 31)) - 1u));
+    perm_src[r] = p;
+    inv_perm[p] = r;
+  }
+}
+
+// ---- multi-block path -----------------------------------------------------
+// (a) per-block expert histogram hist[b][e]
+__global__ void __launch_bounds__(256)
+    permute_count_kernel(const int32_t* __restrict__ idx, int64_t T, int32_t* __restrict__ hist) {
+  __shared__ uint32_t bm[kE][kPermBlockTokens / 32];
+  const int tid = threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPermBlockTokens;
+  const int nt = static_cast<int>((T - t0) < kPermBlockTokens ? (T - t0) : kPermBlockTokens);
+  for (int i = tid; i < kE * (kPermBlockTokens / 32); i += blockDim.x) (&bm[0][0])[i] = 0u;
+  __syncthreads();
+  for (int q = tid; q < nt * kTopK; q += blockDim.x) {
+    const int e = idx[t0 * kTopK + q];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
+      record_status(kSiteBadIndex);
+      continue;
+    }
+    const int tl = q >> 3;
+    atomicOr(&bm[e][tl >> 5], 1u << (tl & 31));
+  }
+  __syncthreads();
+  if (tid < kE) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kPermBlockTokens / 32; ++w) c += __popc(bm[tid][w]);
+    hist[static_cast<int64_t>(blockIdx.x) * kE + tid] = c;
+  }
+}
+
+// (b) column scans: hist[b][e] <- rows of e in blocks before b; counts, offsets.
+//     One block of 1024 threads: thread (part, e) owns a contiguous range of blocks.
+__global__ void __launch_bounds__(1024)
+    permute_scan_kernel(int32_t* __restrict__ hist, int nb, int32_t* __restrict__ counts,
+                        int32_t* __restrict__ offsets) {
+  constexpr int kParts = 1024 / kE;  // 8
+  __shared__ int part_sum[kParts][kE];
+  __shared__ int cnt[kE];
+  __shared__ int off[kE + 1];
+  const int tid = threadIdx.x, e = tid % kE, part = tid / kE, lane = tid & 31;
+  const int per = (nb + kParts - 1) / kParts;
+  const int b0 = min(nb, part * per), b1 = min(nb, b0 + per);
+  int s = 0;
+  for (int b = b0; b < b1; ++b) s += hist[static_cast<int64_t>(b) * kE + e];
+  part_sum[part][e] = s;
+  __syncthreads();
+  int run = 0;
+  for (int p = 0; p < part; ++p) run += part_sum[p][e];
+  if (part == kParts - 1) cnt[e] = run + s;
+  for (int b = b0; b < b1; ++b) {
+    const int64_t i = static_cast<int64_t>(b) * kE + e;
+    const int h = hist[i];
+    hist[i] = run;
+    run += h;
+  }
+  __syncthreads();
+  if (tid < 32) scan_experts_warp0(cnt, off, lane);
+  __syncthreads();
+  if (tid < kE) {
+    counts[tid] = cnt[tid];
+    offsets[tid] = off[tid];
+  }
+  if (tid == 0) offsets[kE] = off[kE];
+}
+
+// (c) stable scatter of the block's items
+__global__ void __launch_bounds__(256)
+    permute_scatter_kernel(const int32_t* __restrict__ idx, int64_t T,
+                           const int32_t* __restrict__ before, const int32_t* __restrict__ offsets,
+                           int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm) {
+  constexpr int W = kPermBlockTokens / 32;
+  __shared__ uint32_t bm[kE][W];
+  __shared__ int base[kE];
+  const int tid = threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPermBlockTokens;
+  const int nt = static_cast<int>((T - t0) < kPermBlockTokens ? (T - t0) : kPermBlockTokens);
+  for (int i = tid; i < kE * W; i += blockDim.x) (&bm[0][0])[i] = 0u;
+  if (tid < kE) base[tid] = offsets[tid] + before[static_cast<int64_t>(blockIdx.x) * kE + tid];
+  __syncthreads();
+  for (int q = tid; q < nt * kTopK; q += blockDim.x) {
+    const int e = idx[t0 * kTopK + q];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    const int tl = q >> 3;
+    atomicOr(&bm[e][tl >> 5], 1u << (tl & 31));
+  }
+  __syncthreads();
+  for (int q = tid; q < nt * kTopK; q += blockDim.x) {
+    const int e = idx[t0 * kTopK + q];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    const int tl = q >> 3, w = tl >> 5;
+    int rank = __popc(bm[e][w] & ((1u << (tl & 31)) - 1u));
+    for (int v = 0; v < w; ++v) rank += __popc(bm[e][v]);
+    const int64_t p = t0 * kTopK + q;
+    const int r = base[e] + rank;
+    perm_src[r] = static_cast<int32_t>(p);
+    inv_perm[p] = r;
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,257 @@
+"""Thin ctypes binding of libmoe (the C ABI in include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory (tensors) and the current CUDA
+stream.  Loading fails loudly when ``libmoe.so`` has not been built -- there is
+no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+HIDDEN, INTER, N_EXPERTS, N_GROUPS, KEEP_GROUPS, TOPK = 1536, 512, 128, 8, 4, 8
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
+    MOE_ERR_UNSUPPORTED = range(6)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'`"
+            " (there is no CPU or Python fallback for the MoE layer)")
+    return ctypes.CDLL(LIB_PATH)
+
+
+lib = _load()
+
+_p, _i64, _sz, _i32, _u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint64
+_SIGS = {
+    "moe_abi_version": ([], _i32),
+    "moe_max_tokens": ([], _i64),
+    "moe_last_error_string": ([], ctypes.c_char_p),
+    "moe_get_device_status": ([_i32], _i32),
+    "moe_set_wait_timeout_ns": ([_u64], _i32),
+    "moe_selftest_wait_timeout": ([_p], _i32),
+    "moe_packed_weight_bytes": ([], _sz),
+    "moe_pack_weights": ([_p, _p, _p, _p, _p], _i32),
+    "moe_route": ([_p, _p, _i64, _p, _p, _p], _i32),
+    "moe_permute_workspace_bytes": ([_i64], _sz),
+    "moe_permute": ([_p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_expert_ffn": ([_p, _p, _p, _p, _i64, _p, _p, _p], _i32),
+    "moe_expert_gate_up": ([_p, _p, _p, _p, _i64, _p, _p], _i32),
+    "moe_expert_down": ([_p, _p, _p, _i64, _p, _p], _i32),
+    "moe_combine": ([_p, _p, _p, _i64, _p, _p, _p], _i32),
+    "moe_layer_workspace_bytes": ([_i64], _sz),
+    "moe_layer": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+}
+for _name, (_args, _ret) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _ret
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/moe.h declares."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(fn, rc, lib.moe_last_error_string().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def last_error() -> str:
+    return lib.moe_last_error_string().decode()
+
+
+# ----------------------------------------------------------------- weights
+
+def packed_weight_bytes() -> int:
+    return int(lib.moe_packed_weight_bytes())
+
+
+def moe_pack_weights(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                     packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Re-layout one layer's bf16 expert weights (see include/moe.h)."""
+    for t, shp in ((w_gate, (N_EXPERTS, HIDDEN, INTER)), (w_up, (N_EXPERTS, HIDDEN, INTER)),
+                   (w_down, (N_EXPERTS, INTER, HIDDEN))):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shp or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"expected contiguous CUDA bf16 {shp}, got {t.dtype} {tuple(t.shape)}")
+    if packed is None:
+        packed = torch.empty(packed_weight_bytes() // 2, dtype=torch.bfloat16, device=w_gate.device)
+    _check("moe_pack_weights", lib.moe_pack_weights(_ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                                    _ptr(packed), _stream(stream)))
+    return packed
+
+
+# ----------------------------------------------------------------- steps
+
+def moe_route(logits: torch.Tensor, bias: torch.Tensor | None, topk_idx=None, topk_w=None,
+              stream=None):
+    T = logits.shape[0]
+    dev = logits.device
+    if topk_idx is None:
+        topk_idx = torch.empty((T, TOPK), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, TOPK), dtype=torch.float32, device=dev)
+    _check("moe_route", lib.moe_route(_ptr(logits), _ptr(bias), T, _ptr(topk_idx), _ptr(topk_w),
+                                      _stream(stream)))
+    return topk_idx, topk_w
+
+
+def permute_workspace_bytes(T: int) -> int:
+    return int(lib.moe_permute_workspace_bytes(T))
+
+
+def moe_permute(topk_idx: torch.Tensor, counts=None, offsets=None, perm_src=None, inv_perm=None,
+                workspace=None, stream=None):
+    """Returns (counts[128], offsets[129], perm_src[8T], inv_perm[8T]) int32."""
+    T = topk_idx.shape[0]
+    dev = topk_idx.device
+    if counts is None:
+        counts = torch.empty(N_EXPERTS, dtype=torch.int32, device=dev)
+    if offsets is None:
+        offsets = torch.empty(N_EXPERTS + 1, dtype=torch.int32, device=dev)
+    if perm_src is None:
+        perm_src = torch.empty(max(T * TOPK, 1), dtype=torch.int32, device=dev)
+    if inv_perm is None:
+        inv_perm = torch.empty(max(T * TOPK, 1), dtype=torch.int32, device=dev)
+    wsb = permute_workspace_bytes(T)
+    if workspace is None and wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    _check("moe_permute", lib.moe_permute(_ptr(topk_idx), T, _ptr(counts), _ptr(offsets),
+                                          _ptr(perm_src), _ptr(inv_perm),
+                                          _ptr(workspace) if wsb else None,
+                                          workspace.numel() if wsb else 0, _stream(stream)))
+    return counts, offsets, perm_src[:T * TOPK], inv_perm[:T * TOPK]
+
+
+def moe_expert_ffn(x: torch.Tensor, packed_w: torch.Tensor, offsets: torch.Tensor,
+                   perm_src: torch.Tensor, h=None, y_perm=None, stream=None):
+    """Returns (h [8T,512], y_perm [8T,1536]) bf16."""
+    T = x.shape[0]
+    dev = x.device
+    if h is None:
+        h = torch.empty((T * TOPK, INTER), dtype=torch.bfloat16, device=dev)
+    if y_perm is None:
+        y_perm = torch.empty((T * TOPK, HIDDEN), dtype=torch.bfloat16, device=dev)
+    _check("moe_expert_ffn", lib.moe_expert_ffn(_ptr(x), _ptr(packed_w), _ptr(offsets),
+                                                _ptr(perm_src), T, _ptr(h), _ptr(y_perm),
+                                                _stream(stream)))
+    return h, y_perm
+
+
+def moe_expert_gate_up(x: torch.Tensor, packed_w: torch.Tensor, offsets: torch.Tensor,
+                       perm_src: torch.Tensor, h=None, stream=None):
+    T = x.shape[0]
+    if h is None:
+        h = torch.empty((T * TOPK, INTER), dtype=torch.bfloat16, device=x.device)
+    _check("moe_expert_gate_up", lib.moe_expert_gate_up(_ptr(x), _ptr(packed_w), _ptr(offsets),
+                                                        _ptr(perm_src), T, _ptr(h),
+                                                        _stream(stream)))
+    return h
+
+
+def moe_expert_down(h: torch.Tensor, packed_w: torch.Tensor, offsets: torch.Tensor,
+                    y_perm=None, stream=None):
+    T = h.shape[0] // TOPK
+    if y_perm is None:
+        y_perm = torch.empty((T * TOPK, HIDDEN), dtype=torch.bfloat16, device=h.device)
+    _check("moe_expert_down", lib.moe_expert_down(_ptr(h), _ptr(packed_w), _ptr(offsets), T,
+                                                  _ptr(y_perm), _stream(stream)))
+    return y_perm
+
+
+def moe_combine(y_perm: torch.Tensor, topk_w: torch.Tensor, inv_perm: torch.Tensor,
+                residual=None, out=None, stream=None):
+    T = topk_w.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=topk_w.device)
+    _check("moe_combine", lib.moe_combine(_ptr(y_perm), _ptr(topk_w), _ptr(inv_perm), T,
+                                          _ptr(residual), _ptr(out), _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------- fused layer
+
+def layer_workspace_bytes(T: int) -> int:
+    return int(lib.moe_layer_workspace_bytes(T))
+
+
+def alloc_layer_workspace(T: int, device) -> torch.Tensor:
+    """A uint8 view of at least layer_workspace_bytes(T) bytes, 1024-byte aligned."""
+    n = layer_workspace_bytes(T)
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 1024
+    return raw[off:off + n]
+
+
+def moe_layer(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
+              packed_w: torch.Tensor, residual=None, out=None, topk_idx_out=None,
+              topk_w_out=None, workspace: torch.Tensor | None = None, stream=None):
+    """out = bf16(residual + MoE(x)) for x [T,1536] bf16 (see include/moe.h)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = alloc_layer_workspace(T, x.device)
+    _check("moe_layer", lib.moe_layer(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_w), T,
+                                      _ptr(residual), _ptr(out), _ptr(topk_idx_out),
+                                      _ptr(topk_w_out), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)))
+    return out
+
+
+def moe_layer_from_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: torch.Tensor | None,
+                        packed_w: torch.Tensor, x_dev: torch.Tensor, logits_dev: torch.Tensor,
+                        out_dev: torch.Tensor, out_host: torch.Tensor,
+                        workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """End-to-end call from pinned host buffers: H2D copy of x and the router
+    logits, the layer, D2H copy of the output, all on one stream."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        x_dev.copy_(x_host, non_blocking=True)
+        logits_dev.copy_(logits_host, non_blocking=True)
+        moe_layer(x_dev, logits_dev, bias, packed_w, out=out_dev, workspace=workspace, stream=s)
+        out_host.copy_(out_dev, non_blocking=True)
+    return out_host
+
+
+# ----------------------------------------------------------------- status
+
+def get_device_status(device: int = 0) -> int:
+    return int(lib.moe_get_device_status(device))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _check("moe_set_wait_timeout_ns", lib.moe_set_wait_timeout_ns(ns))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    _check("moe_selftest_wait_timeout", lib.moe_selftest_wait_timeout(_stream(stream)))

@@ -1,0 +1,205 @@
+/*
+ * moe.h -- C ABI of libmoe, the B200 (sm_100a) routed-expert MoE layer of
+ * Ling-3.0-tiny: group-limited top-k routing, token-to-expert permutation,
+ * grouped SwiGLU expert FFN on tcgen05 tensor cores, weighted combine.
+ *
+ * Layer shape, as the pages state it:
+ *   - 128 routed experts per layer in 8 groups of 16, 4 groups kept per
+ *     token, hidden size 1536: "Ling-3.0-tiny on a Qualcomm board" (TensorFold
+ *     issue #1247), first comment, opening paragraph.
+ *   - 8 experts active per token: "HelloSun/ling30tiny", table 模型與路由
+ *     (model and routing), row on experts active per token.
+ *   - experts with gate, up and down matrices (a SwiGLU FFN), no SwiGLU
+ *     clamp ("null SwiGLU limit lists"): same table, row on expert weights;
+ *     issue #1247, opening paragraph.  Intermediate size 512.
+ *
+ * Conventions shared by every entry point
+ *   - Return value: a moe_status code.  No C++ exception crosses the ABI.
+ *     moe_last_error_string() describes the last failure of the calling
+ *     thread.
+ *   - Pointers are caller-owned DEVICE memory unless stated otherwise.  The
+ *     library never allocates, frees or reads device memory from the host,
+ *     and never synchronises a stream; every call is asynchronous on
+ *     `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *   - Arrays are dense row-major.  Every pointer must be 16-byte aligned;
+ *     bf16 matrices read by the tensor-memory-accelerator (x, packed weights,
+ *     the h workspace) must be 128-byte aligned.
+ *   - T (tokens) is int64_t; 0 <= T <= moe_max_tokens().  T == 0 is a valid
+ *     no-op.  Invalid arguments return MOE_ERR_INVALID_ARG before anything is
+ *     launched.  Internal address arithmetic is 64-bit ("Add TML Inkling
+ *     architecture", llama.cpp PR #25731, description: int64 indices because
+ *     large MoEs overflow 32-bit ones).
+ *   - bf16 values are passed as raw 16-bit patterns (moe_bf16).
+ *   - Device-side waits inside the kernels are bounded in time.  A wait that
+ *     runs out sets a per-device error word and makes the kernel return;
+ *     moe_get_device_status() reports it as MOE_ERR_TIMEOUT.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* cudaStream_t */
+typedef uint16_t moe_bf16;                /* raw bfloat16 bits */
+
+enum {
+  MOE_HIDDEN = 1536,     /* H: model width */
+  MOE_INTER = 512,       /* I: expert intermediate size */
+  MOE_EXPERTS = 128,     /* E: routed experts per layer */
+  MOE_GROUPS = 8,        /* expert groups */
+  MOE_GROUP_SIZE = 16,   /* experts per group */
+  MOE_KEEP_GROUPS = 4,   /* groups kept per token */
+  MOE_TOPK = 8           /* experts used per token */
+};
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer */
+  MOE_ERR_WORKSPACE = 2,   /* workspace smaller than the query says */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
+  MOE_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out */
+  MOE_ERR_UNSUPPORTED = 5  /* device is not sm_100 */
+} moe_status;
+
+/* ---- library information ------------------------------------------------ */
+
+/* ABI version of this header (bumped on any signature change). */
+int moe_abi_version(void);
+
+/* Largest T accepted by every entry point. */
+int64_t moe_max_tokens(void);
+
+/* Text of the calling thread's last error ("" when none).  The pointer stays
+ * valid until the next call on that thread. */
+const char* moe_last_error_string(void);
+
+/* Reads and clears the error word of `device` that bounded kernel waits set.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT, or MOE_ERR_CUDA if the query failed.
+ * This is the one call that synchronises: it copies 4 bytes to the host. */
+int moe_get_device_status(int device);
+
+/* Time limit of every bounded device-side wait, in nanoseconds (default 2e9).
+ * Applies to launches issued after the call. */
+int moe_set_wait_timeout_ns(uint64_t ns);
+
+/* Launches one block whose bounded wait on a barrier that nothing completes
+ * must run out after the current limit: a self-test of the timeout path.  The
+ * kernel returns normally and leaves the context usable; afterwards
+ * moe_get_device_status() returns MOE_ERR_TIMEOUT. */
+int moe_selftest_wait_timeout(moe_stream_t stream);
+
+/* ---- weights ------------------------------------------------------------ */
+
+/* Bytes of one layer's packed expert weights (604 MB). */
+size_t moe_packed_weight_bytes(void);
+
+/* One-time re-layout of one layer's expert weights into the tensor-core
+ * operand order used by moe_expert_ffn.
+ *   w_gate, w_up : [128][1536][512] bf16, the layer computes x @ W_gate[e]
+ *   w_down       : [128][512][1536] bf16, the layer computes h @ W_down[e]
+ *   packed       : moe_packed_weight_bytes() bytes, 128-byte aligned, output.
+ * Packed layout: per expert, W_gate/W_up transposed to K-major [512][1536] and
+ * interleaved in blocks of 128 output columns (gate block j, up block j, ...),
+ * followed later by W_down transposed to [1536][512].  Inputs must not alias
+ * `packed`. */
+int moe_pack_weights(const moe_bf16* w_gate, const moe_bf16* w_up,
+                     const moe_bf16* w_down, moe_bf16* packed,
+                     moe_stream_t stream);
+
+/* ---- the four steps ----------------------------------------------------- */
+
+/* Step 1: group-limited top-8 routing, one warp per token.
+ * Group-limited routing runs as its own kernel in the GB10 CUDA path of issue
+ * #1247 ("What it does not cover", bullet on the CUDA C kernels); the score
+ * rule used here:
+ *   s_e = sigmoid(logit[t,e] + bias[e])                 (float64)
+ *   group score = sum of the two largest s_e of the group
+ *   keep the 4 best groups (ties: lower group index)
+ *   topk_idx[t,0..7] = the 8 largest s_e inside kept groups, in descending
+ *                      order (ties: lower expert index)
+ *   topk_w[t,i] = sigmoid(logit[t,e_i]) / sum_j sigmoid(logit[t,e_j])
+ *   logits : [T][128] fp32          bias : [128] fp32, or NULL for zeros
+ *   topk_idx : [T][8] int32 (out)   topk_w : [T][8] fp32 (out)  */
+int moe_route(const float* logits, const float* bias, int64_t T,
+              int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* Scratch bytes moe_permute needs for T tokens (0 when T <= 1024). */
+size_t moe_permute_workspace_bytes(int64_t T);
+
+/* Step 2: device-side stable counting sort of the T*8 (token, slot) items by
+ * expert, so that each expert runs on exactly the rows that picked it with no
+ * host round trip (issue #1247, "What it does not cover", bullet on bf16
+ * experts: the per-expert row loop there needs a host sync per layer).
+ *   topk_idx : [T][8] int32 (from moe_route)
+ *   counts   : [128] int32 (out)  rows per expert
+ *   offsets  : [129] int32 (out)  exclusive prefix of counts; offsets[128] = 8T
+ *   perm_src : [8T] int32 (out)   permuted row r holds item t*8+slot; rows are
+ *                                 expert-major, token-ascending inside an expert
+ *   inv_perm : [8T] int32 (out)   item t*8+slot sits at row inv_perm[t*8+slot]
+ *   workspace: moe_permute_workspace_bytes(T) bytes (may be NULL when 0). */
+int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts,
+                int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
+                void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Step 3: grouped SwiGLU expert FFN over the permuted rows, persistent
+ * tcgen05 GEMMs (the grouped kernel that issue #1247 names as missing):
+ *   h[r]      = silu(x[t] W_gate[e]) * (x[t] W_up[e])   (fp32 accumulate, bf16 out)
+ *   y_perm[r] = h[r] W_down[e]                          (fp32 accumulate, bf16 out)
+ * for every permuted row r = offsets[e] + i, i < counts[e], t = perm_src[r]/8.
+ *   x        : [T][1536] bf16, 128-byte aligned
+ *   packed_w : from moe_pack_weights
+ *   offsets, perm_src : from moe_permute
+ *   h        : [8T][512] bf16 workspace (out), 128-byte aligned
+ *   y_perm   : [8T][1536] bf16 (out) */
+int moe_expert_ffn(const moe_bf16* x, const moe_bf16* packed_w,
+                   const int32_t* offsets, const int32_t* perm_src, int64_t T,
+                   moe_bf16* h, moe_bf16* y_perm, moe_stream_t stream);
+
+/* Step 4: weighted combine back into token order ("HelloSun/ling30tiny",
+ * section 數值檢查摘要: routing plus the weighted layer):
+ *   out[t] = bf16( residual[t] + sum_{slot 0..7} topk_w[t,slot] * y_perm[inv_perm[8t+slot]] )
+ * summed in fp32 in slot order and rounded once (deterministic, no atomics).
+ *   residual : [T][1536] bf16 or NULL (then 0).  `out` may alias `residual`. */
+int moe_combine(const moe_bf16* y_perm, const float* topk_w,
+                const int32_t* inv_perm, int64_t T, const moe_bf16* residual,
+                moe_bf16* out, moe_stream_t stream);
+
+/* Step 3, first half alone: h[r] = silu(x[t] W_gate[e]) * (x[t] W_up[e]),
+ * arguments as in moe_expert_ffn (one persistent tcgen05 GEMM launch). */
+int moe_expert_gate_up(const moe_bf16* x, const moe_bf16* packed_w,
+                       const int32_t* offsets, const int32_t* perm_src, int64_t T,
+                       moe_bf16* h, moe_stream_t stream);
+
+/* Step 3, second half alone: y_perm[r] = h[r] W_down[e] (one persistent
+ * tcgen05 GEMM launch).  h: [8T][512] bf16 from moe_expert_gate_up. */
+int moe_expert_down(const moe_bf16* h, const moe_bf16* packed_w,
+                    const int32_t* offsets, int64_t T, moe_bf16* y_perm,
+                    moe_stream_t stream);
+
+/* ---- the fused layer ---------------------------------------------------- */
+
+/* Workspace bytes moe_layer needs for T tokens. */
+size_t moe_layer_workspace_bytes(int64_t T);
+
+/* The whole layer: route -> permute -> expert FFN -> combine, back to back on
+ * `stream` with no host synchronisation.  Arguments as in the steps above;
+ *   residual   : NULL, or [T][1536] bf16 added before the final rounding
+ *                (a stack layer computes h <- bf16(h + moe(h)) with
+ *                residual = x = out allowed)
+ *   topk_idx_out, topk_w_out : optional [T][8] copies of the routing (NULL to skip)
+ *   workspace  : moe_layer_workspace_bytes(T) bytes of device memory, 1024-byte aligned. */
+int moe_layer(const moe_bf16* x, const float* logits, const float* bias,
+              const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
+              moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
+              void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

@@ -1,0 +1,68 @@
+"""The C-ABI library loads on a CPU-only machine, exports every function that
+include/moe.h declares, and rejects bad arguments on the host before any
+CUDA call (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from group_limited_routed_moe_b200 import moe
+
+
+def test_exports_every_declared_symbol():
+    names = moe.header_functions()
+    assert len(names) >= 15
+    missing = [n for n in names if not hasattr(moe.lib, n)]
+    assert missing == []
+    assert moe.lib.moe_abi_version() == 1
+
+
+def test_sizes():
+    assert moe.packed_weight_bytes() == 128 * 3 * 1536 * 512 * 2
+    assert moe.lib.moe_max_tokens() == 1 << 22
+    assert moe.lib.moe_permute_workspace_bytes(1024) == 0
+    assert moe.lib.moe_permute_workspace_bytes(1025) == 9 * 128 * 4 + (256 - (9 * 128 * 4) % 256) % 256
+    assert moe.lib.moe_permute_workspace_bytes(-1) == 0
+    prev = 0
+    for T in (1, 4, 16, 2048, 8192):
+        b = moe.layer_workspace_bytes(T)
+        # h and y_perm dominate: 8T rows of (512 + 1536) bf16
+        assert b >= T * 8 * (512 + 1536) * 2 and b % 1024 == 0 and b > prev
+        prev = b
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_host_validation_without_gpu():
+    L = moe.lib
+    # T out of range
+    assert L.moe_route(_p(256), None, -1, _p(256), _p(256), None) == moe.MOE_ERR_INVALID_ARG
+    assert "outside" in moe.last_error()
+    assert L.moe_route(_p(256), None, (1 << 22) + 1, _p(256), _p(256), None) == moe.MOE_ERR_INVALID_ARG
+    # T == 0 is a no-op that touches nothing
+    assert L.moe_route(None, None, 0, None, None, None) == moe.MOE_OK
+    assert L.moe_expert_ffn(None, None, None, None, 0, None, None, None) == moe.MOE_OK
+    assert L.moe_combine(None, None, None, 0, None, None, None) == moe.MOE_OK
+    assert L.moe_layer(None, None, None, None, 0, None, None, None, None, None, 0, None) == moe.MOE_OK
+    # null and misaligned pointers
+    assert L.moe_route(None, None, 4, _p(256), _p(256), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(_p(260), None, 4, _p(256), _p(256), None) == moe.MOE_ERR_INVALID_ARG
+    assert "aligned" in moe.last_error()
+    assert L.moe_expert_ffn(_p(64), _p(128), _p(16), _p(16), 4, _p(128), _p(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_weights(None, _p(128), _p(128), _p(128), None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small / missing
+    assert L.moe_permute(_p(256), 2048, _p(256), _p(256), _p(256), _p(256), None, 0, None) \
+        == moe.MOE_ERR_WORKSPACE
+    ws = moe.layer_workspace_bytes(16)
+    assert L.moe_layer(_p(1024), _p(1024), None, _p(1024), 16, None, _p(1024), None, None,
+                       _p(1024), ws - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_layer(_p(1024), _p(1024), None, _p(1024), 16, None, _p(1024), None, None,
+                       _p(1040), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_set_wait_timeout_ns(10) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_binding_raises_with_message():
+    with pytest.raises(moe.MoeError) as ei:
+        moe._check("moe_route", moe.MOE_ERR_INVALID_ARG)
+    assert "status 1" in str(ei.value)

@@ -1,0 +1,154 @@
+"""GPU parity of the fused layer (moe_layer) on every single-layer workload,
+plus the invariances the layer must satisfy bit for bit on the device.
+
+Tolerances: routing ids bit-exact, weights <= 1e-6, output rel-L2 <= 5e-3
+against the float64 oracle (bf16 inputs, fp32 accumulation, bf16 h / y / out).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from group_limited_routed_moe_b200 import synth
+from gpu_helpers import (DEV, REL_L2_TOL, W_TOL, layer0_weights, oracle_layer, to_dev_bf16,
+                         to_host_bits, tokens_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _moe():
+    from group_limited_routed_moe_b200 import moe
+    return moe
+
+
+def _run_layer(tok, T_buf=None, residual=None):
+    moe = _moe()
+    W = layer0_weights()
+    T = tok.x_bits.shape[0]
+    x, lg, bias = tokens_dev(tok, T_buf)
+    idx = torch.empty((T, 8), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, 8), dtype=torch.float32, device=DEV)
+    out = torch.full((x.shape[0], 1536), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_layer(x[:T], lg[:T], bias, W.packed, residual=residual, out=out[:T],
+                  topk_idx_out=idx, topk_w_out=w)
+    torch.cuda.synchronize()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    return out, idx, w
+
+
+@pytest.mark.parametrize("name", ["decode_T16"] + [f"decode_T4_seed{s}" for s in range(1, 9)] +
+                         ["prefill_T2048_skewed"])
+def test_layer_parity_full(name):
+    wl = synth.WORKLOADS[name]
+    tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
+    out, idx, w = _run_layer(tok)
+    ref, rr = oracle_layer(tok, layer0_weights())
+    assert np.array_equal(idx.cpu().numpy(), rr.topk_idx)
+    assert np.abs(w.cpu().numpy() - rr.topk_w).max() <= W_TOL
+    err = O.rel_l2(O.bf16_bits_to_f64(to_host_bits(out)), ref)
+    assert err <= REL_L2_TOL, f"{name}: rel-L2 {err:.3e}"
+    if wl.hot:
+        counts = np.bincount(rr.topk_idx.ravel(), minlength=128)
+        assert counts[tok.hot_experts].mean() > 4 * counts.mean()
+
+
+def test_layer_parity_prefill_T8189():
+    """Long-prompt prefill: 8,189 real tokens in buffers of 8,192.  The oracle
+    checks every token; rows 8189..8191 of the output buffer stay untouched."""
+    wl = synth.WORKLOADS["prefill_T8189"]
+    tok = synth.make_tokens(wl.T, wl.seed)
+    out, idx, w = _run_layer(tok, T_buf=wl.T_buf)
+    ref, rr = oracle_layer(tok, layer0_weights())
+    assert np.array_equal(idx.cpu().numpy(), rr.topk_idx)
+    assert np.abs(w.cpu().numpy() - rr.topk_w).max() <= W_TOL
+    got = O.bf16_bits_to_f64(to_host_bits(out[:wl.T]))
+    err = O.rel_l2(got, ref)
+    assert err <= REL_L2_TOL, f"rel-L2 {err:.3e}"
+    # token-wise: no single token far off
+    per_tok = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert per_tok.max() <= 4 * REL_L2_TOL
+    assert torch.isnan(out[wl.T:].float()).all()
+
+
+def test_layer_permutation_and_batch_invariance():
+    """out(P x) = P out(x) and rows of a T=16 call equal T=4 + T=12 calls, bit
+    for bit (the combine is deterministic, every token is independent)."""
+    tok = synth.make_tokens(16, 0)
+    out, _, _ = _run_layer(tok)
+    perm = np.random.default_rng(0).permutation(16)
+    tok_p = synth.TokenInputs(tok.x_bits[perm].copy(), tok.logits[perm].copy(), tok.bias)
+    out_p, _, _ = _run_layer(tok_p)
+    assert torch.equal(out_p.view(torch.int16), out[torch.as_tensor(perm, device=DEV)].view(torch.int16))
+    a = synth.TokenInputs(tok.x_bits[:4].copy(), tok.logits[:4].copy(), tok.bias)
+    b = synth.TokenInputs(tok.x_bits[4:].copy(), tok.logits[4:].copy(), tok.bias)
+    oa, _, _ = _run_layer(a)
+    ob, _, _ = _run_layer(b)
+    assert torch.equal(torch.cat([oa, ob]).view(torch.int16), out.view(torch.int16))
+
+
+def test_layer_deterministic():
+    tok = synth.make_tokens(2048, 2, hot=16)
+    o1, _, _ = _run_layer(tok)
+    o2, _, _ = _run_layer(tok)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def test_layer_residual():
+    """out = bf16(residual + moe(x)), in place on the residual buffer."""
+    tok = synth.make_tokens(16, 0)
+    x, lg, bias = tokens_dev(tok)
+    moe = _moe()
+    W = layer0_weights()
+    h = x.clone()
+    moe.moe_layer(x, lg, bias, W.packed, residual=h, out=h)
+    torch.cuda.synchronize()
+    ref, _ = oracle_layer(tok, W)
+    ref = ref + O.bf16_bits_to_f64(tok.x_bits)
+    got = O.bf16_bits_to_f64(to_host_bits(h))
+    assert O.rel_l2(got - O.bf16_bits_to_f64(tok.x_bits), ref - O.bf16_bits_to_f64(tok.x_bits)) \
+        <= REL_L2_TOL * 2
+    # the stored values are bf16 roundings of the fp32 sum: within one ulp of the exact sum
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-3)
+
+
+def test_layer_from_host_e2e():
+    moe = _moe()
+    W = layer0_weights()
+    tok = synth.make_tokens(16, 0)
+    x_h = torch.from_numpy(tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_h = torch.from_numpy(tok.logits).pin_memory()
+    x_d = torch.empty((16, 1536), dtype=torch.bfloat16, device=DEV)
+    lg_d = torch.empty((16, 128), dtype=torch.float32, device=DEV)
+    out_d = torch.empty_like(x_d)
+    out_h = torch.empty((16, 1536), dtype=torch.bfloat16).pin_memory()
+    ws = moe.alloc_layer_workspace(16, DEV)
+    bias = torch.from_numpy(tok.bias).to(DEV)
+    moe.moe_layer_from_host(x_h, lg_h, bias, W.packed, x_d, lg_d, out_d, out_h, ws)
+    torch.cuda.synchronize()
+    ref, _ = oracle_layer(tok, W)
+    got = O.bf16_bits_to_f64(out_h.view(torch.int16).numpy().view(np.uint16))
+    assert O.rel_l2(got, ref) <= REL_L2_TOL
+
+
+def test_layer_graph_capture():
+    """The layer is capturable in a CUDA graph and replays to the same bits."""
+    moe = _moe()
+    W = layer0_weights()
+    tok = synth.make_tokens(16, 0)
+    x, lg, bias = tokens_dev(tok)
+    ws = moe.alloc_layer_workspace(16, DEV)
+    out = torch.empty_like(x)
+    moe.moe_layer(x, lg, bias, W.packed, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    ref = out.clone()
+    out.zero_()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            moe.moe_layer(x, lg, bias, W.packed, out=out, workspace=ws, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    del g

@@ -1,0 +1,177 @@
+"""GPU parity of each step through the C ABI against the float64 oracle.
+
+Routing ids, per-expert counts and the permutation are compared bit for bit;
+routing weights within 1e-6; expert outputs within the layer tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from group_limited_routed_moe_b200 import synth
+from gpu_helpers import DEV, REL_L2_TOL, W_TOL, layer0_weights, to_dev_bf16, to_host_bits, tokens_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _moe():
+    from group_limited_routed_moe_b200 import moe
+    return moe
+
+
+def _route_check(lg_np, bias_np):
+    moe = _moe()
+    T = lg_np.shape[0]
+    lg = torch.from_numpy(lg_np).to(DEV)
+    b = None if bias_np is None else torch.from_numpy(bias_np).to(DEV)
+    idx, w = moe.moe_route(lg, b)
+    torch.cuda.synchronize()
+    rr = O.route(lg_np, bias_np)
+    gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+    # audit: a float64 near-tie would be reported, not counted as a mismatch
+    ambiguous = (rr.group_margin < 1e-12) | (rr.expert_margin < 1e-12)
+    assert not ambiguous.any(), f"{ambiguous.sum()} near-tied tokens in the inputs"
+    assert np.array_equal(gi, rr.topk_idx), "routing ids differ"
+    assert np.abs(gw - rr.topk_w).max() <= W_TOL
+    return gi, gw, rr
+
+
+@pytest.mark.parametrize("name", ["decode_T16", "decode_T4_seed1", "decode_T4_seed8",
+                                  "prefill_T2048_skewed", "prefill_T8189"])
+def test_route_parity_workloads(name):
+    wl = synth.WORKLOADS[name]
+    tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
+    _route_check(tok.logits, tok.bias)
+
+
+@pytest.mark.parametrize("T", [1, 7, 33, 257])
+def test_route_ragged_and_no_bias(T):
+    rng = np.random.default_rng(T)
+    _route_check(rng.standard_normal((T, 128)).astype(np.float32), None)
+
+
+def test_route_special_cases():
+    moe = _moe()
+    # all equal -> groups 0-3, experts 0..7, w = 1/8
+    lg = torch.full((5, 128), 0.7, dtype=torch.float32, device=DEV)
+    idx, w = moe.moe_route(lg, torch.zeros(128, device=DEV))
+    assert idx.cpu().tolist() == [list(range(8))] * 5
+    assert torch.all(w == 0.125)
+    # exact ties between groups and experts resolve to the lower index
+    a = np.full((1, 128), -3.0, np.float32)
+    a[0, [32, 33, 80, 81]] = 2.0
+    a[0, [34, 35, 82, 83]] = 1.0
+    gi, _, _ = _route_check(a, None)
+    assert gi[0].tolist() == [32, 33, 80, 81, 34, 35, 82, 83]
+    # dominant expert and an excluded group
+    rng = np.random.default_rng(3)
+    lg2 = rng.standard_normal((16, 128)).astype(np.float32)
+    b2 = (0.1 * rng.standard_normal(128)).astype(np.float32)
+    lg2[:, 77] = 12.0
+    b2[16:32] = -40.0
+    gi, _, _ = _route_check(lg2, b2)
+    assert np.all(gi[:, 0] == 77) and not np.any((gi >= 16) & (gi < 32))
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 1000, 1024, 1025, 2048, 8189])
+def test_permute_parity(T):
+    moe = _moe()
+    tok = synth.make_tokens(T, 100 + T)
+    lg = torch.from_numpy(tok.logits).to(DEV)
+    idx, _ = moe.moe_route(lg, torch.from_numpy(tok.bias).to(DEV))
+    counts, offsets, perm_src, inv_perm = moe.moe_permute(idx)
+    torch.cuda.synchronize()
+    ref = O.permute(idx.cpu().numpy().astype(np.int64))
+    assert np.array_equal(counts.cpu().numpy(), ref.counts)
+    assert np.array_equal(offsets.cpu().numpy(), ref.offsets)
+    assert np.array_equal(perm_src.cpu().numpy(), ref.perm_src)
+    assert np.array_equal(inv_perm.cpu().numpy(), ref.inv_perm)
+    # and the routing that fed it is the oracle's
+    assert np.array_equal(idx.cpu().numpy(), O.route(tok.logits, tok.bias).topk_idx)
+
+
+def test_permute_skewed_and_forced():
+    """All tokens on the same 8 experts (counts 8T on 8 experts, 0 elsewhere)."""
+    moe = _moe()
+    T = 3000
+    idx = torch.tensor([[5, 6, 7, 40, 41, 100, 101, 127]] * T, dtype=torch.int32, device=DEV)
+    counts, offsets, perm_src, inv_perm = moe.moe_permute(idx)
+    ref = O.permute(idx.cpu().numpy().astype(np.int64))
+    assert np.array_equal(counts.cpu().numpy(), ref.counts)
+    assert np.array_equal(perm_src.cpu().numpy(), ref.perm_src)
+    assert np.array_equal(inv_perm.cpu().numpy(), ref.inv_perm)
+
+
+def _ffn_check(T, seed, forced=None):
+    """Runs route -> permute -> expert_ffn and compares every computed y_perm
+    row with the oracle's expert FFN of that (token, expert)."""
+    moe = _moe()
+    W = layer0_weights()
+    tok = synth.make_tokens(T, seed)
+    if forced is not None:
+        tok.bias[:] = 0
+        tok.bias[forced] = 1000.0
+    x, lg, bias = tokens_dev(tok)
+    idx, w = moe.moe_route(lg, bias)
+    counts, offsets, perm_src, inv_perm = moe.moe_permute(idx)
+    h, y = moe.moe_expert_ffn(x, W.packed, offsets, perm_src)
+    torch.cuda.synchronize()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    rr = O.route(tok.logits, tok.bias)
+    assert np.array_equal(idx.cpu().numpy(), rr.topk_idx)
+    wg, wu, wd = W.host(rr.topk_idx)
+    ps = perm_src.cpu().numpy()
+    yh = O.bf16_bits_to_f64(to_host_bits(y))
+    xh = O.bf16_bits_to_f64(tok.x_bits)
+    ref = np.empty_like(yh)
+    for e in np.unique(rr.topk_idx):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        toks = ps[r0:r1] // 8
+        ref[r0:r1] = O.expert_ffn(xh[toks], O.bf16_bits_to_f64(wg[e]), O.bf16_bits_to_f64(wu[e]),
+                                  O.bf16_bits_to_f64(wd[e]))
+    err = O.rel_l2(yh, ref)
+    assert err <= REL_L2_TOL, f"y_perm rel-L2 {err:.3e}"
+    # per-expert check too, so that one bad tile cannot hide in the total
+    for e in np.unique(rr.topk_idx):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        assert O.rel_l2(yh[r0:r1], ref[r0:r1]) <= 2 * REL_L2_TOL, f"expert {e}"
+    return err
+
+
+@pytest.mark.parametrize("T,seed", [(1, 11), (4, 1), (16, 0), (300, 5)])
+def test_expert_ffn_parity(T, seed):
+    _ffn_check(T, seed)
+
+
+def test_expert_ffn_dense_special_case():
+    """Every token forced onto the same 8 experts: each expert runs a dense
+    [T, 1536] x [1536, 1024] GEMM over several 128-row tiles and a ragged tail."""
+    _ffn_check(333, 21, forced=[3, 4, 21, 22, 40, 41, 90, 91])
+
+
+def test_combine_parity():
+    moe = _moe()
+    rng = np.random.default_rng(9)
+    T = 37
+    y_bits = synth.f32_to_bf16_bits(rng.standard_normal((T * 8, 1536)).astype(np.float32))
+    w = rng.random((T, 8)).astype(np.float32)
+    inv = rng.permutation(T * 8).astype(np.int32)
+    res_bits = synth.f32_to_bf16_bits(rng.standard_normal((T, 1536)).astype(np.float32))
+    out = moe.moe_combine(to_dev_bf16(y_bits), torch.from_numpy(w).to(DEV),
+                          torch.from_numpy(inv).to(DEV), residual=to_dev_bf16(res_bits))
+    torch.cuda.synchronize()
+    yv = O.bf16_bits_to_f64(y_bits)
+    ref = O.bf16_bits_to_f64(res_bits) + np.einsum("ts,tsh->th", w.astype(np.float64),
+                                                   yv[inv.reshape(T, 8)])
+    got = O.bf16_bits_to_f64(to_host_bits(out))
+    # fp32 accumulation then one bf16 rounding: within one bf16 ulp (2**-8 relative)
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+
+
+def test_generator_device_bytes_equal_host_bytes():
+    """The oracle reads expert weights made on the device by the input
+    generator; they are the same bytes as the host generator's."""
+    W = layer0_weights()
+    for which, t in ((synth.W_GATE, W.wg), (synth.W_DOWN, W.wd)):
+        host = synth.weight_bits_np(0, 0, which, experts=[0, 77, 127])
+        assert np.array_equal(to_host_bits(t[[0, 77, 127]]), host)
