@@ -2,6 +2,7 @@
 // token, back in token order.
 //
 // out[t] = bf16( residual[t] + sum_{slot} w[t,slot] * y_perm[inv_perm[8t+slot]] )
+// with y_perm in fp16 (the down GEMM's output) and the residual in bf16.
 // The "real MoE routing + weighted layer" of "HelloSun/ling30tiny" (section
 // 數值檢查摘要) is this sum.  It is done in gather form: each token reads its 8
 // rows, adds them in fp32 in slot order and rounds once, so the result is
@@ -15,7 +16,7 @@ namespace moe {
 constexpr int kCombineThreads = kH / 8;  // 192
 
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const float* __restrict__ topk_w,
+    combine_kernel(const uint16_t* __restrict__ y_perm, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ inv_perm, int64_t T,
                    const __nv_bfloat16* residual, __nv_bfloat16* out) {
   const int64_t t = blockIdx.x;
@@ -44,8 +45,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     const uint32_t q[4] = {v[s].x, v[s].y, v[s].z, v[s].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      acc[2 * i] = fmaf(w[s], bf16_lo(q[i]), acc[2 * i]);
-      acc[2 * i + 1] = fmaf(w[s], bf16_hi(q[i]), acc[2 * i + 1]);
+      acc[2 * i] = fmaf(w[s], f16_lo(q[i]), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(w[s], f16_hi(q[i]), acc[2 * i + 1]);
     }
   }
   if (residual != nullptr) {

@@ -10,8 +10,14 @@
 //   phase 1 (gate/up):  h[r]      = silu(x[tok(r)] W_gate[e]) * (x[tok(r)] W_up[e])
 //                       M_e x N 1024 x K 1536 per expert, N tiled by 256 =
 //                       128 gate + 128 up columns, SwiGLU in the epilogue.
+//                       bf16 x bf16 -> fp32 accumulate -> fp16 h.
 //   phase 2 (down):     y_perm[r] = h[r] W_down[e]
 //                       M_e x N 1536 x K 512 per expert, N tiled by 256.
+//                       fp16 x fp16 (W_down packed as fp16, exact for bf16
+//                       weights in the fp16 normal range) -> fp32 -> fp16 y.
+// The two intermediates are fp16 rather than bf16: same bytes and the same
+// tensor-core rate, 8x smaller rounding error.  A value outside the fp16 range
+// sets the device status word (kSiteFp16Range) instead of passing silently.
 //
 // Work is cut into tiles (expert e, n-tile j, m-tile m) of 128 rows x 256
 // columns; tile ids run expert-major, then j, then m, so consecutive CTAs
@@ -21,14 +27,26 @@
 //
 // Warp roles inside a CTA (one CTA per SM: ~194 KB of shared memory, all 512
 // TMEM columns):
-//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SwiGLU / bf16, stores
-//   warps 4-7  (phase 1) A producers: gather the tile's 128 token rows of x
-//              with cp.async into the 128B-swizzled operand layout
+//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SwiGLU, fp16 stores
+//   warps 4-7  (phase 1) A producers: gather the tile's token rows of x with
+//              cp.async into the 128B-swizzled operand layout; each thread
+//              signals the stage's barrier through cp.async.mbarrier.arrive,
+//              so the gather keeps all stages in flight.  Rows past the
+//              expert's count are not loaded (a row of A only reaches the
+//              same, never stored, accumulator row).  With ZERO_PAD they are
+//              kept at zero by a zero-fill cp.async, issued only when the
+//              slot last held data (start-up, valid -> padding change): when
+//              most rows are padding (small batches) the gate/up GEMM ran up
+//              to 2x slower with stale bits there than with zeros, while with
+//              few padding rows (large batches) leaving them stale was ~15%
+//              faster.  The host picks ZERO_PAD for T <= 4096.
 //   next warp  TMA producer: weight tiles (and, in phase 2, h tiles)
 //   next warp  MMA issuer: tcgen05.mma 128x256x16, accumulator in TMEM,
 //              double-buffered (2 x 256 columns) so the epilogue of tile i
 //              overlaps the MMAs of tile i+1.
-// Shared-memory ring: 4 stages of (A 128x64 + B 256x64) bf16.
+// Shared-memory ring: 4 stages of (A 128x64 + B 256x64) 16-bit elements.
+// The epilogue transposes each warp's 32 x 32 fp16 block through a padded
+// shared tile so that global stores are whole 64-byte row segments.
 #pragma once
 #include "common.cuh"
 
@@ -37,14 +55,14 @@ namespace ffn {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int BK = 64;  // one 128-byte swizzle row of 16-bit elements
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int TILE_BYTES = STAGES * (A_BYTES + B_BYTES);
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int GATHER_LAG = 2;  // cp.async groups kept in flight per producer thread
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr int STAGE_ROW = 80;                      // padded 64-byte row of the epilogue tile
+constexpr int EPI_WARP_BYTES = 32 * STAGE_ROW;     // one warp's 32 x 32 fp16 block
 
 template <int PHASE>
 struct Cfg;
@@ -57,7 +75,8 @@ struct Cfg<1> {
   static constexpr int THREADS = 320;
   static constexpr int TMA_WARP = 8;
   static constexpr int MMA_WARP = 9;
-  static constexpr int FULL_COUNT = 1 + 4;        // TMA arrive + 4 gather warps
+  static constexpr int FULL_COUNT = 1 + 128;      // TMA arrive + 128 gather threads
+  static constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kFmtBF16);
 };
 template <>
 struct Cfg<2> {
@@ -69,6 +88,7 @@ struct Cfg<2> {
   static constexpr int TMA_WARP = 4;
   static constexpr int MMA_WARP = 5;
   static constexpr int FULL_COUNT = 1;
+  static constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kFmtF16);
 };
 
 struct SmemTail {
@@ -84,7 +104,8 @@ struct SmemTail {
   int cnt[kE];
   int off[kE];
 };
-constexpr int SMEM_BYTES = TILE_BYTES + static_cast<int>(sizeof(SmemTail)) + 1024;
+constexpr int TAIL_BYTES = (static_cast<int>(sizeof(SmemTail)) + 127) / 128 * 128;
+constexpr int SMEM_BYTES = TILE_BYTES + TAIL_BYTES + 4 * EPI_WARP_BYTES + 1024;
 
 __device__ __forceinline__ void decode_tile(const SmemTail* S, int tile, int NT, int& e, int& m,
                                             int& j) {
@@ -102,13 +123,32 @@ __device__ __forceinline__ void decode_tile(const SmemTail* S, int tile, int NT,
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-template <int PHASE>
+// Stores one warp's 32 rows x 32 fp16 columns (lane = row, 16 packed pairs in
+// registers) as row segments of 64 bytes: written to the warp's padded shared
+// tile, read back 4 lanes per row, stored 16 bytes per lane.  Rows >= nvalid
+// are skipped.  g0 points at (row 0, first column); ld is the row stride.
+__device__ __forceinline__ void store_block_32x32(const uint32_t (&pk)[16], uint32_t stage,
+                                                  uint16_t* g0, int64_t ld, int nvalid, int lane) {
+  const uint32_t mine = stage + lane * STAGE_ROW;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) st_shared_v4(mine + q * 16, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = i * 8 + (lane >> 2), ch = lane & 3;
+    const uint4 v = ld_shared_v4(stage + row * STAGE_ROW + ch * 16);
+    if (row < nvalid) st_global_v4(g0 + row * ld + ch * 8, v.x, v.y, v.z, v.w);
+  }
+  __syncwarp();
+}
+
+template <int PHASE, bool ZERO_PAD>
 __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_a,
                     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                     const int32_t* __restrict__ perm_src, int64_t T,
-                    __nv_bfloat16* __restrict__ out, uint64_t timeout_ns) {
+                    uint16_t* __restrict__ out, uint64_t timeout_ns) {
   using C = Cfg<PHASE>;
   constexpr int KB = C::KDIM / BK;
 
@@ -118,6 +158,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   uint8_t* sA = smem;                       // STAGES x 16 KB
   uint8_t* sB = smem + STAGES * A_BYTES;    // STAGES x 32 KB
   SmemTail* S = reinterpret_cast<SmemTail*>(smem + TILE_BYTES);
+  uint8_t* sEpi = smem + TILE_BYTES + TAIL_BYTES;  // 4 x 2.5 KB
   volatile int* abort_flag = &S->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,7 +278,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           const uint64_t bdesc = smem_desc_k128(smem_u32(sB + s * B_BYTES));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(d, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&S->empty[s]);
         }
         if (ok) umma_commit(&S->tfull[a]);
@@ -250,20 +291,18 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     // ------------------------------------------------ A gather producers
     const int r = threadIdx.x - 128;  // row of the tile
     const uint32_t swz = static_cast<uint32_t>(r & 7);
+    uint32_t dirty = (1u << STAGES) - 1;  // stage slots whose row r may be non-zero
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       int e, m, j;
       decode_tile(S, tile, C::NT, e, m, j);
       const int row_in_e = m * BM + r;
-      const char* src = reinterpret_cast<const char*>(x);
-      uint32_t nbytes = 0;
+      const char* src = nullptr;
       if (row_in_e < S->cnt[e]) {
         const int p = perm_src[S->off[e] + row_in_e];
-        if (p >= 0 && static_cast<int64_t>(p) < nrows) {
+        if (p >= 0 && static_cast<int64_t>(p) < nrows)
           src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
-          nbytes = 16;
-        }
       }
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int s = it % STAGES;
@@ -273,27 +312,27 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           break;
         }
         const uint32_t dst = smem_u32(sA + s * A_BYTES) + r * 128;
-        const char* g = src + kb * BK * 2;
+        if (src != nullptr) {
+          const char* g = src + kb * BK * 2;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          cp_async_16(dst + ((static_cast<uint32_t>(c) ^ swz) << 4), g + c * 16, nbytes);
-        cp_async_commit();
-        if (it >= GATHER_LAG) {
-          cp_async_wait_group<GATHER_LAG>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S->full[(it - GATHER_LAG) % STAGES]);
+          for (int c = 0; c < 8; ++c)
+            cp_async_16(dst + ((static_cast<uint32_t>(c) ^ swz) << 4), g + c * 16, 16);
+          cp_async_arrive_noinc(&S->full[s]);
+          dirty |= 1u << s;
+        } else {
+          if (ZERO_PAD && (dirty & (1u << s))) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cp_async_16(dst + c * 16, x, 0);
+            dirty &= ~(1u << s);
+          }
+          cp_async_arrive_noinc(&S->full[s]);
         }
       }
     }
-    cp_async_wait_group<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (ok && lane == 0)
-      for (int i = max(0, it - GATHER_LAG); i < it; ++i) mbar_arrive(&S->full[i % STAGES]);
+    cp_async_wait_all();
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue
-    const int r = threadIdx.x;  // row of the tile == TMEM lane
+    bool range_bad = false;  // thread (warp w, lane l) owns row 32w + l == TMEM lane
     int tc = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
       int e, m, j;
@@ -302,12 +341,13 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       const uint32_t use = tc >> 1;
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
       tc_fence_after();
-      const int row_in_e = m * BM + r;
-      const bool valid = row_in_e < S->cnt[e];
-      const int64_t prow = static_cast<int64_t>(S->off[e]) + row_in_e;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * BN;
+      const int nvalid = min(32, max(0, S->cnt[e] - (m * BM + warp * 32)));
+      const uint32_t stage = smem_u32(sEpi + warp * EPI_WARP_BYTES);
+      bool bad = false;  // range check of this thread's row; rows >= nvalid hold garbage
+      uint16_t* g0 = out + (static_cast<int64_t>(S->off[e]) + m * BM + warp * 32) * C::OUT_COLS;
       if (PHASE == 1) {
-        __nv_bfloat16* dst = out + prow * C::OUT_COLS + j * 128;
+        g0 += j * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t g[32], u[32];
@@ -315,40 +355,36 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                silu_mul(__uint_as_float(g[2 * i + 1]),
-                                         __uint_as_float(u[2 * i + 1])));
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              st_global_v4(dst + c * 32 + q * 8, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                           pk[4 * q + 3]);
-          }
+            pk[i] = pack_f16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                               silu_mul(__uint_as_float(g[2 * i + 1]),
+                                        __uint_as_float(u[2 * i + 1])),
+                               bad);
+          if (nvalid > 0) store_block_32x32(pk, stage, g0 + c * 32, C::OUT_COLS, nvalid, lane);
         }
       } else {
-        __nv_bfloat16* dst = out + prow * C::OUT_COLS + j * BN;
+        g0 += j * BN;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v0[32], v1[32];
           tmem_ld_2x32(tbase + c * 64, tbase + c * 64 + 32, v0, v1);
-          uint32_t pk[32];
+          uint32_t p0[16], p1[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            pk[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
-            pk[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+            p0[i] = pack_f16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]), bad);
+            p1[i] = pack_f16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]), bad);
           }
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              st_global_v4(dst + c * 64 + q * 8, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                           pk[4 * q + 3]);
+          if (nvalid > 0) {
+            store_block_32x32(p0, stage, g0 + c * 64, C::OUT_COLS, nvalid, lane);
+            store_block_32x32(p1, stage, g0 + c * 64 + 32, C::OUT_COLS, nvalid, lane);
           }
         }
       }
+      range_bad |= bad && lane < nvalid;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->tempty[a]);
     }
+    if (range_bad) record_status(kSiteFp16Range);
   }
 
   tc_fence_before();

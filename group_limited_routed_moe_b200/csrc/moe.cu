@@ -26,6 +26,7 @@ namespace {
 constexpr int kAbiVersion = 1;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
+constexpr int64_t kZeroPadMaxT = 4096;  // gate/up keeps padding rows of A zeroed up to this T
 
 thread_local char g_err[512] = "";
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
@@ -78,10 +79,13 @@ int device_setup(int* dev_out, int* sms_out) {
                dev, prop.major, prop.minor);
     } else {
       d.sms = prop.multiProcessorCount;
-      e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<1>,
+      e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<1, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<2>,
+        e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<1, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<2, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       if (g_encode == nullptr) {
@@ -101,14 +105,15 @@ int device_setup(int* dev_out, int* sms_out) {
   return MOE_OK;
 }
 
-// 2-D bf16 tensor map: `rows` rows of `cols` elements, box of 64 x box_rows,
-// 128-byte swizzle (matches the UMMA K-major SW128 operand layout).
-int make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// 2-D tensor map of 16-bit elements: `rows` rows of `cols` elements, box of
+// 64 x box_rows, 128-byte swizzle (the UMMA K-major SW128 operand layout).
+int make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+              CUtensorMapDataType dtype) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  CUresult r = g_encode(m, dtype, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -173,11 +178,17 @@ int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets,
 int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                const int32_t* perm_src, int64_t T, moe_bf16* h, int sms, cudaStream_t s) {
   CUtensorMap tb1;
-  int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN);
+  int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   if (rc) return rc;
-  ffn::ffn_gemm_kernel<1><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
-      tb1, tb1, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-      reinterpret_cast<__nv_bfloat16*>(h), g_timeout_ns.load());
+  const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  auto* hb = reinterpret_cast<uint16_t*>(h);
+  if (T <= kZeroPadMaxT)
+    ffn::ffn_gemm_kernel<1, true><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
+        tb1, tb1, xb, offsets, perm_src, T, hb, g_timeout_ns.load());
+  else
+    ffn::ffn_gemm_kernel<1, false><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
+        tb1, tb1, xb, offsets, perm_src, T, hb, g_timeout_ns.load());
   return launch_check("ffn_gemm_kernel<1> launch");
 }
 
@@ -185,12 +196,12 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
             moe_bf16* y, int sms, cudaStream_t s) {
   CUtensorMap tb2, ta2;
   const uint64_t rows = static_cast<uint64_t>(T) * kTopK;
-  int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN);
-  if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM);
+  int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
-  ffn::ffn_gemm_kernel<2><<<sms, ffn::Cfg<2>::THREADS, ffn::SMEM_BYTES, s>>>(
-      tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<__nv_bfloat16*>(y),
-      g_timeout_ns.load());
+  ffn::ffn_gemm_kernel<2, false><<<sms, ffn::Cfg<2>::THREADS, ffn::SMEM_BYTES, s>>>(
+      tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
   return launch_check("ffn_gemm_kernel<2> launch");
 }
 
@@ -205,7 +216,7 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
                const moe_bf16* residual, moe_bf16* out, cudaStream_t s) {
   combine_kernel<<<static_cast<unsigned>(T), kCombineThreads, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(y), w, inv, T,
+      reinterpret_cast<const uint16_t*>(y), w, inv, T,
       reinterpret_cast<const __nv_bfloat16*>(residual), reinterpret_cast<__nv_bfloat16*>(out));
   return launch_check("combine_kernel launch");
 }
@@ -258,6 +269,8 @@ int moe_get_device_status(int device) {
   if (v == 0) return MOE_OK;
   if ((v & 0x7FFFFFFFu) == kSiteBadIndex)
     return fail(MOE_ERR_INVALID_ARG, "a kernel met an out-of-range index (status 0x%08x)", v);
+  if ((v & 0x7FFFFFFFu) == kSiteFp16Range)
+    return fail(MOE_ERR_RANGE, "a value of h, y_perm or W_down exceeded the fp16 range");
   return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out (status 0x%08x, site %u)", v,
               v & 0x7FFFFFFFu);
 }

@@ -8,10 +8,13 @@
 // that one 256-wide accumulator tile holds matching gate and up columns and
 // the SwiGLU can be applied in the epilogue.
 //
-// Packed layout of one layer (bf16 elements):
-//   region GU: [128 experts][1024 rows][1536]   row 256j + r:  r < 128 -> gate col 128j + r
-//                                                             r >= 128 -> up col 128j + r - 128
-//   region D : [128 experts][1536 rows][512]    row n = output column n of W_down[e]
+// Packed layout of one layer (16-bit elements):
+//   region GU: [128 experts][1024 rows][1536] bf16  row 256j + r: r < 128 -> gate col 128j + r
+//                                                                r >= 128 -> up col 128j + r - 128
+//   region D : [128 experts][1536 rows][512]  fp16  row n = output column n of W_down[e]
+// W_down is stored as fp16 so that the down GEMM multiplies the fp16 h by an
+// operand of the same type; every bf16 value in the fp16 normal range
+// converts exactly, and a weight beyond the fp16 range sets the status word.
 #pragma once
 #include "common.cuh"
 
@@ -32,6 +35,7 @@ __global__ void __launch_bounds__(256)
   const int e = blockIdx.z;
   const int n0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  bool bad = false;
   const uint16_t* s = src + static_cast<int64_t>(e) * K * N;
 #pragma unroll
   for (int i = 0; i < 32; i += 8) tile[ty + i][tx] = s[static_cast<int64_t>(k0 + ty + i) * N + n0 + tx];
@@ -50,8 +54,15 @@ __global__ void __launch_bounds__(256)
     const int n = n0 + ty + i;
     int64_t row = n;
     if (mode != 2) row = 256 * (n >> 7) + (n & 127) + (mode == 1 ? 128 : 0);
-    d[row * row_len + k0 + tx] = tile[tx][ty + i];
+    uint16_t v = tile[tx][ty + i];
+    if (mode == 2) {
+      const float f = __uint_as_float(static_cast<uint32_t>(v) << 16);
+      bad |= !(fabsf(f) <= 65504.f);
+      v = __half_as_ushort(__float2half_rn(f));
+    }
+    d[row * row_len + k0 + tx] = v;
   }
+  if (bad) record_status(kSiteFp16Range);
 }
 
 }  // namespace moe

@@ -74,37 +74,42 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   }
   const bool kept = rank < kKeep;
 
-  // candidates: scores of kept experts, -1 (below any sigmoid) otherwise
-  double c[4];
+  // Candidates: kept experts' scores.  A score s lies in [0, 1], and the bit
+  // pattern of a non-negative double orders exactly like its value, so the
+  // key (hi word + 2^30, lo word) compares candidates exactly; 0 marks an
+  // excluded or already-taken expert.  Each round takes the warp maximum of
+  // the high words, then of the low words among lanes holding that high
+  // word, then the lowest expert index among exact ties.
+  uint32_t khi[4], klo[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) c[i] = kept ? s[i] : -1.0;
+  for (int i = 0; i < 4; ++i) {
+    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(s[i]));
+    khi[i] = kept ? static_cast<uint32_t>(b >> 32) + 0x40000000u : 0u;
+    klo[i] = kept ? static_cast<uint32_t>(b) : 0u;
+  }
 
   int sel = -1;  // lane k (k < 8) ends up holding the k-th selected expert
 #pragma unroll 1
   for (int k = 0; k < kTopK; ++k) {
-    double bv = c[0];
+    // lane-local best (ties: lower index, i.e. first)
+    uint32_t bh = khi[0], bl = klo[0];
     int bi = 0;
 #pragma unroll
     for (int i = 1; i < 4; ++i) {
-      if (c[i] > bv) {
-        bv = c[i];
+      if (khi[i] > bh || (khi[i] == bh && klo[i] > bl)) {
+        bh = khi[i];
+        bl = klo[i];
         bi = i;
       }
     }
-    int be = 4 * lane + bi;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const double ov = __shfl_xor_sync(FULL, bv, off);
-      const int oe = __shfl_xor_sync(FULL, be, off);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if (lane == k) sel = be;
+    const uint32_t mh = __reduce_max_sync(FULL, bh);
+    const uint32_t ml = __reduce_max_sync(FULL, bh == mh ? bl : 0u);
+    const bool mine = (bh == mh) && (bl == ml);
+    const uint32_t be = __reduce_min_sync(FULL, mine ? static_cast<uint32_t>(4 * lane + bi) : 0xFFFFFFFFu);
+    if (lane == k) sel = static_cast<int>(be);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (be == 4 * lane + i) c[i] = -2.0;
+      if (static_cast<uint32_t>(4 * lane + i) == be) khi[i] = klo[i] = 0u;
   }
 
   // combine weights: sigmoid of the raw logit, renormalised over the 8

@@ -20,7 +20,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 HIDDEN, INTER, N_EXPERTS, N_GROUPS, KEEP_GROUPS, TOPK = 1536, 512, 128, 8, 4, 8
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
-    MOE_ERR_UNSUPPORTED = range(6)
+    MOE_ERR_UNSUPPORTED, MOE_ERR_RANGE = range(7)
 
 
 class MoeError(RuntimeError):
@@ -154,13 +154,13 @@ def moe_permute(topk_idx: torch.Tensor, counts=None, offsets=None, perm_src=None
 
 def moe_expert_ffn(x: torch.Tensor, packed_w: torch.Tensor, offsets: torch.Tensor,
                    perm_src: torch.Tensor, h=None, y_perm=None, stream=None):
-    """Returns (h [8T,512], y_perm [8T,1536]) bf16."""
+    """Returns (h [8T,512], y_perm [8T,1536]) fp16."""
     T = x.shape[0]
     dev = x.device
     if h is None:
-        h = torch.empty((T * TOPK, INTER), dtype=torch.bfloat16, device=dev)
+        h = torch.empty((T * TOPK, INTER), dtype=torch.float16, device=dev)
     if y_perm is None:
-        y_perm = torch.empty((T * TOPK, HIDDEN), dtype=torch.bfloat16, device=dev)
+        y_perm = torch.empty((T * TOPK, HIDDEN), dtype=torch.float16, device=dev)
     _check("moe_expert_ffn", lib.moe_expert_ffn(_ptr(x), _ptr(packed_w), _ptr(offsets),
                                                 _ptr(perm_src), T, _ptr(h), _ptr(y_perm),
                                                 _stream(stream)))
@@ -171,7 +171,7 @@ def moe_expert_gate_up(x: torch.Tensor, packed_w: torch.Tensor, offsets: torch.T
                        perm_src: torch.Tensor, h=None, stream=None):
     T = x.shape[0]
     if h is None:
-        h = torch.empty((T * TOPK, INTER), dtype=torch.bfloat16, device=x.device)
+        h = torch.empty((T * TOPK, INTER), dtype=torch.float16, device=x.device)
     _check("moe_expert_gate_up", lib.moe_expert_gate_up(_ptr(x), _ptr(packed_w), _ptr(offsets),
                                                         _ptr(perm_src), T, _ptr(h),
                                                         _stream(stream)))
@@ -182,7 +182,7 @@ def moe_expert_down(h: torch.Tensor, packed_w: torch.Tensor, offsets: torch.Tens
                     y_perm=None, stream=None):
     T = h.shape[0] // TOPK
     if y_perm is None:
-        y_perm = torch.empty((T * TOPK, HIDDEN), dtype=torch.bfloat16, device=h.device)
+        y_perm = torch.empty((T * TOPK, HIDDEN), dtype=torch.float16, device=h.device)
     _check("moe_expert_down", lib.moe_expert_down(_ptr(h), _ptr(packed_w), _ptr(offsets), T,
                                                   _ptr(y_perm), _stream(stream)))
     return y_perm

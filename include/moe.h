@@ -46,6 +46,7 @@ extern "C" {
 
 typedef struct CUstream_st* moe_stream_t; /* cudaStream_t */
 typedef uint16_t moe_bf16;                /* raw bfloat16 bits */
+typedef uint16_t moe_f16;                 /* raw IEEE binary16 bits */
 
 enum {
   MOE_HIDDEN = 1536,     /* H: model width */
@@ -63,7 +64,10 @@ typedef enum moe_status {
   MOE_ERR_WORKSPACE = 2,   /* workspace smaller than the query says */
   MOE_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
   MOE_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out */
-  MOE_ERR_UNSUPPORTED = 5  /* device is not sm_100 */
+  MOE_ERR_UNSUPPORTED = 5, /* device is not sm_100 */
+  MOE_ERR_RANGE = 6        /* an fp16 intermediate (h, y_perm, packed W_down)
+                              left the fp16 range; reported by
+                              moe_get_device_status() */
 } moe_status;
 
 /* ---- library information ------------------------------------------------ */
@@ -78,8 +82,10 @@ int64_t moe_max_tokens(void);
  * valid until the next call on that thread. */
 const char* moe_last_error_string(void);
 
-/* Reads and clears the error word of `device` that bounded kernel waits set.
- * Returns MOE_OK, MOE_ERR_TIMEOUT, or MOE_ERR_CUDA if the query failed.
+/* Reads and clears the error word of `device` that the kernels set: a bounded
+ * wait that ran out (MOE_ERR_TIMEOUT), an fp16 intermediate out of range
+ * (MOE_ERR_RANGE) or an out-of-range index in caller data
+ * (MOE_ERR_INVALID_ARG).  MOE_OK when clean; MOE_ERR_CUDA if the query failed.
  * This is the one call that synchronises: it copies 4 bytes to the host. */
 int moe_get_device_status(int device);
 
@@ -99,14 +105,16 @@ int moe_selftest_wait_timeout(moe_stream_t stream);
 size_t moe_packed_weight_bytes(void);
 
 /* One-time re-layout of one layer's expert weights into the tensor-core
- * operand order used by moe_expert_ffn.
+ * operand order used by moe_expert_ffn (W_down converted to fp16, exact for
+ * bf16 values in the fp16 normal range).
  *   w_gate, w_up : [128][1536][512] bf16, the layer computes x @ W_gate[e]
  *   w_down       : [128][512][1536] bf16, the layer computes h @ W_down[e]
  *   packed       : moe_packed_weight_bytes() bytes, 128-byte aligned, output.
  * Packed layout: per expert, W_gate/W_up transposed to K-major [512][1536] and
  * interleaved in blocks of 128 output columns (gate block j, up block j, ...),
- * followed later by W_down transposed to [1536][512].  Inputs must not alias
- * `packed`. */
+ * followed (after all experts' gate/up blocks, 128 x 1024 x 1536 elements)
+ * by every expert's W_down transposed to [1536][512] in fp16.  Inputs must not
+ * alias `packed`. */
 int moe_pack_weights(const moe_bf16* w_gate, const moe_bf16* w_up,
                      const moe_bf16* w_down, moe_bf16* packed,
                      moe_stream_t stream);
@@ -148,24 +156,25 @@ int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts,
 
 /* Step 3: grouped SwiGLU expert FFN over the permuted rows, persistent
  * tcgen05 GEMMs (the grouped kernel that issue #1247 names as missing):
- *   h[r]      = silu(x[t] W_gate[e]) * (x[t] W_up[e])   (fp32 accumulate, bf16 out)
- *   y_perm[r] = h[r] W_down[e]                          (fp32 accumulate, bf16 out)
+ *   h[r]      = silu(x[t] W_gate[e]) * (x[t] W_up[e])   (bf16 in, fp32 accumulate, fp16 out)
+ *   y_perm[r] = h[r] W_down[e]                          (fp16 in, fp32 accumulate, fp16 out)
  * for every permuted row r = offsets[e] + i, i < counts[e], t = perm_src[r]/8.
  *   x        : [T][1536] bf16, 128-byte aligned
  *   packed_w : from moe_pack_weights
  *   offsets, perm_src : from moe_permute
- *   h        : [8T][512] bf16 workspace (out), 128-byte aligned
- *   y_perm   : [8T][1536] bf16 (out) */
+ *   h        : [8T][512] fp16 workspace (out), 128-byte aligned
+ *   y_perm   : [8T][1536] fp16 (out) */
 int moe_expert_ffn(const moe_bf16* x, const moe_bf16* packed_w,
                    const int32_t* offsets, const int32_t* perm_src, int64_t T,
-                   moe_bf16* h, moe_bf16* y_perm, moe_stream_t stream);
+                   moe_f16* h, moe_f16* y_perm, moe_stream_t stream);
 
 /* Step 4: weighted combine back into token order ("HelloSun/ling30tiny",
  * section 數值檢查摘要: routing plus the weighted layer):
  *   out[t] = bf16( residual[t] + sum_{slot 0..7} topk_w[t,slot] * y_perm[inv_perm[8t+slot]] )
  * summed in fp32 in slot order and rounded once (deterministic, no atomics).
+ *   y_perm   : [8T][1536] fp16 (from moe_expert_ffn / moe_expert_down)
  *   residual : [T][1536] bf16 or NULL (then 0).  `out` may alias `residual`. */
-int moe_combine(const moe_bf16* y_perm, const float* topk_w,
+int moe_combine(const moe_f16* y_perm, const float* topk_w,
                 const int32_t* inv_perm, int64_t T, const moe_bf16* residual,
                 moe_bf16* out, moe_stream_t stream);
 
@@ -173,12 +182,12 @@ int moe_combine(const moe_bf16* y_perm, const float* topk_w,
  * arguments as in moe_expert_ffn (one persistent tcgen05 GEMM launch). */
 int moe_expert_gate_up(const moe_bf16* x, const moe_bf16* packed_w,
                        const int32_t* offsets, const int32_t* perm_src, int64_t T,
-                       moe_bf16* h, moe_stream_t stream);
+                       moe_f16* h, moe_stream_t stream);
 
 /* Step 3, second half alone: y_perm[r] = h[r] W_down[e] (one persistent
- * tcgen05 GEMM launch).  h: [8T][512] bf16 from moe_expert_gate_up. */
-int moe_expert_down(const moe_bf16* h, const moe_bf16* packed_w,
-                    const int32_t* offsets, int64_t T, moe_bf16* y_perm,
+ * tcgen05 GEMM launch).  h: [8T][512] fp16 from moe_expert_gate_up. */
+int moe_expert_down(const moe_f16* h, const moe_bf16* packed_w,
+                    const int32_t* offsets, int64_t T, moe_f16* y_perm,
                     moe_stream_t stream);
 
 /* ---- the fused layer ---------------------------------------------------- */

@@ -94,7 +94,12 @@ def test_layer_deterministic():
 
 
 def test_layer_residual():
-    """out = bf16(residual + moe(x)), in place on the residual buffer."""
+    """out = bf16(residual + moe(x)), in place on the residual buffer.
+
+    The oracle's value is bf16(x + moe_exact).  The GPU rounds x + moe_fp32,
+    and moe_fp32 differs from moe_exact by the layer's own error, so the two
+    roundings agree except where a bf16 boundary lies between them: every
+    element is within one bf16 ulp of the oracle and almost all are equal."""
     tok = synth.make_tokens(16, 0)
     x, lg, bias = tokens_dev(tok)
     moe = _moe()
@@ -102,13 +107,16 @@ def test_layer_residual():
     h = x.clone()
     moe.moe_layer(x, lg, bias, W.packed, residual=h, out=h)
     torch.cuda.synchronize()
-    ref, _ = oracle_layer(tok, W)
-    ref = ref + O.bf16_bits_to_f64(tok.x_bits)
-    got = O.bf16_bits_to_f64(to_host_bits(h))
-    assert O.rel_l2(got - O.bf16_bits_to_f64(tok.x_bits), ref - O.bf16_bits_to_f64(tok.x_bits)) \
-        <= REL_L2_TOL * 2
-    # the stored values are bf16 roundings of the fp32 sum: within one ulp of the exact sum
-    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-3)
+    upd, _ = oracle_layer(tok, W)
+    exact = O.bf16_bits_to_f64(tok.x_bits) + upd
+    ref_bits = O.f64_to_bf16_bits(exact)
+    got_bits = to_host_bits(h)
+    got, ref = O.bf16_bits_to_f64(got_bits), O.bf16_bits_to_f64(ref_bits)
+    assert O.rel_l2(got, exact) <= REL_L2_TOL
+    assert np.mean(got_bits == ref_bits) >= 0.9
+    # one bf16 ulp of the sum plus the layer's own error (a few 1e-3 of the update)
+    ulp = np.ldexp(1.0, np.frexp(np.abs(exact))[1] - 8)
+    assert np.all(np.abs(got - exact) <= ulp + 0.02 * np.sqrt(np.mean(upd ** 2)))
 
 
 def test_layer_from_host_e2e():

@@ -19,7 +19,7 @@ def _moe():
     return moe
 
 
-def _route_check(lg_np, bias_np):
+def _route_check(lg_np, bias_np, exact_ties=False):
     moe = _moe()
     T = lg_np.shape[0]
     lg = torch.from_numpy(lg_np).to(DEV)
@@ -29,8 +29,10 @@ def _route_check(lg_np, bias_np):
     rr = O.route(lg_np, bias_np)
     gi, gw = idx.cpu().numpy(), w.cpu().numpy()
     # audit: a float64 near-tie would be reported, not counted as a mismatch
+    # (inputs built with exact ties are exempt: equal values are equal on both sides)
     ambiguous = (rr.group_margin < 1e-12) | (rr.expert_margin < 1e-12)
-    assert not ambiguous.any(), f"{ambiguous.sum()} near-tied tokens in the inputs"
+    if not exact_ties:
+        assert not ambiguous.any(), f"{ambiguous.sum()} near-tied tokens in the inputs"
     assert np.array_equal(gi, rr.topk_idx), "routing ids differ"
     assert np.abs(gw - rr.topk_w).max() <= W_TOL
     return gi, gw, rr
@@ -61,7 +63,7 @@ def test_route_special_cases():
     a = np.full((1, 128), -3.0, np.float32)
     a[0, [32, 33, 80, 81]] = 2.0
     a[0, [34, 35, 82, 83]] = 1.0
-    gi, _, _ = _route_check(a, None)
+    gi, _, _ = _route_check(a, None, exact_ties=True)
     assert gi[0].tolist() == [32, 33, 80, 81, 34, 35, 82, 83]
     # dominant expert and an excluded group
     rng = np.random.default_rng(3)
@@ -121,7 +123,7 @@ def _ffn_check(T, seed, forced=None):
     assert np.array_equal(idx.cpu().numpy(), rr.topk_idx)
     wg, wu, wd = W.host(rr.topk_idx)
     ps = perm_src.cpu().numpy()
-    yh = O.bf16_bits_to_f64(to_host_bits(y))
+    yh = y.double().cpu().numpy()                 # fp16 -> float64 is exact
     xh = O.bf16_bits_to_f64(tok.x_bits)
     ref = np.empty_like(yh)
     for e in np.unique(rr.topk_idx):
@@ -153,14 +155,14 @@ def test_combine_parity():
     moe = _moe()
     rng = np.random.default_rng(9)
     T = 37
-    y_bits = synth.f32_to_bf16_bits(rng.standard_normal((T * 8, 1536)).astype(np.float32))
+    y16 = rng.standard_normal((T * 8, 1536)).astype(np.float16)
     w = rng.random((T, 8)).astype(np.float32)
     inv = rng.permutation(T * 8).astype(np.int32)
     res_bits = synth.f32_to_bf16_bits(rng.standard_normal((T, 1536)).astype(np.float32))
-    out = moe.moe_combine(to_dev_bf16(y_bits), torch.from_numpy(w).to(DEV),
+    out = moe.moe_combine(torch.from_numpy(y16).to(DEV), torch.from_numpy(w).to(DEV),
                           torch.from_numpy(inv).to(DEV), residual=to_dev_bf16(res_bits))
     torch.cuda.synchronize()
-    yv = O.bf16_bits_to_f64(y_bits)
+    yv = y16.astype(np.float64)
     ref = O.bf16_bits_to_f64(res_bits) + np.einsum("ts,tsh->th", w.astype(np.float64),
                                                    yv[inv.reshape(T, 8)])
     got = O.bf16_bits_to_f64(to_host_bits(out))
