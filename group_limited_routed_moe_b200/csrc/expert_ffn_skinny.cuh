@@ -1,0 +1,356 @@
+// expert_ffn_skinny.cuh -- step 3 for small batches: the same two grouped
+// GEMMs as expert_ffn.cuh with the operands swapped, so that the weights are
+// the 128-row MMA operand and the few tokens of an expert are the narrow one.
+//
+// At decode an expert sees one or two of a batch's tokens.  A 128-row token
+// tile would spend 127 rows of tensor work on padding; here a tile is 128
+// weight rows x 32 tokens (tcgen05.mma M=128, N=32), each pipeline stage holds
+// 16 KB of weights and 4 KB of token rows, and eight stages keep 128 KB of
+// weights in flight per SM, so the kernel streams the selected experts'
+// weights at HBM speed (the layer's bound at small batches).
+//
+//   phase 1: D[f][t] = sum_k W_gu[f][k] x[tok(t)][k] over 128 weight rows f =
+//            64 gate rows + the 64 matching up rows (two TMA boxes), so that
+//            h[t][f] = silu(D_gate) * D_up pairs TMEM lanes f and f+64; the up
+//            half is handed to the gate half through a padded shared tile.
+//   phase 2: D[n][t] = sum_k W_down[n][k] h[t][k] over 128 output columns n.
+// Tiles are (expert, 128-row weight block, 32-token chunk), chunk fastest, so
+// the CTAs that share a weight block run together and read it from L2 once.
+//
+// Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31), 4 token gather (phase 1:
+// cp.async of x rows by perm_src, barrier-tracked; padding rows kept at zero),
+// 5 TMA producer, 6 MMA issuer.  Accumulators: 2 x 32 TMEM columns.  Every
+// wait, including the up -> gate hand-off, is a bounded mbarrier wait.
+#pragma once
+#include "common.cuh"
+#include "expert_ffn.cuh"
+
+namespace moe {
+namespace skinny {
+
+constexpr int BMW = 128;  // weight rows per tile (MMA M)
+constexpr int BNT = 32;   // tokens per tile (MMA N)
+constexpr int BK = 64;
+constexpr int STAGES = 8;
+constexpr int A_BYTES = BMW * BK * 2;  // 16 KB
+constexpr int B_BYTES = BNT * BK * 2;  // 4 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
+constexpr int TMEM_COLS = 2 * BNT;
+constexpr int XSTRIDE = BNT + 1;  // floats per row of the up-value exchange tile
+constexpr int XCHG_BYTES = 64 * XSTRIDE * 4;
+constexpr int THREADS = 224;
+constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;
+
+template <int PHASE>
+struct SCfg;
+template <>
+struct SCfg<1> {
+  static constexpr int KDIM = kH;
+  static constexpr int FBLK = 8;  // 4 pairs x 2 halves of 64 gate + 64 up rows
+  static constexpr int OUT_COLS = kI;
+  static constexpr int FULL_COUNT = 1 + 32;  // TMA arrive + 32 gather lanes
+  static constexpr uint32_t TX = A_BYTES;
+  static constexpr uint32_t IDESC = idesc_f32acc(BMW, BNT, kFmtBF16);
+};
+template <>
+struct SCfg<2> {
+  static constexpr int KDIM = kI;
+  static constexpr int FBLK = kH / BMW;  // 12
+  static constexpr int OUT_COLS = kH;
+  static constexpr int FULL_COUNT = 1;
+  static constexpr uint32_t TX = A_BYTES + B_BYTES;
+  static constexpr uint32_t IDESC = idesc_f32acc(BMW, BNT, kFmtF16);
+};
+
+struct Tail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t xfull;   // up half written to the exchange tile (64 lane arrivals)
+  uint64_t xempty;  // gate half done reading it (64 lane arrivals)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int wsum[4];
+  int tile_start[kE + 1];
+  int cnt[kE];
+  int off[kE];
+};
+constexpr int TAIL_BYTES = (static_cast<int>(sizeof(Tail)) + 127) / 128 * 128;
+constexpr int SMEM_BYTES = TILE_BYTES + TAIL_BYTES + XCHG_BYTES + 1024;
+
+__device__ __forceinline__ void decode_tile(const Tail* S, int tile, int FBLK, int& e, int& f,
+                                            int& c) {
+  int lo = 0, hi = kE - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (S->tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int rem = tile - S->tile_start[e];
+  const int nch = (S->cnt[e] + BNT - 1) / BNT;
+  f = rem / nch;
+  c = rem - f * nch;
+}
+
+template <int PHASE>
+__global__ void __launch_bounds__(THREADS, 1)
+    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_h,
+                       const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
+                       const int32_t* __restrict__ perm_src, int64_t T,
+                       uint16_t* __restrict__ out, uint64_t timeout_ns) {
+  using C = SCfg<PHASE>;
+  constexpr int KB = C::KDIM / BK;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Tail* S = reinterpret_cast<Tail*>(smem + TILE_BYTES);
+  float* xchg = reinterpret_cast<float*>(smem + TILE_BYTES + TAIL_BYTES);
+  volatile int* abort_flag = &S->abort_flag;
+  uint64_t* fullb = S->full;
+  uint64_t* emptyb = S->empty;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nrows = T * kTopK;
+  auto sA = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto sB = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&fullb[s], C::FULL_COUNT);
+      mbar_init(&emptyb[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&S->tfull[a], 1);
+      mbar_init(&S->tempty[a], 4);
+    }
+    mbar_init(&S->xfull, 64);
+    mbar_init(&S->xempty, 64);
+    mbar_init(&S->drain, 1);
+    S->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == TMA_WARP && lane == 0) {
+    tma_prefetch_desc(&tmap_w);
+    if (PHASE == 2) tma_prefetch_desc(&tmap_h);
+  }
+
+  int my_tiles = 0;
+  if (threadIdx.x < kE) {
+    const int e = threadIdx.x;
+    const int o0 = offsets[e], o1 = offsets[e + 1];
+    int c = o1 - o0;
+    if (o0 < 0 || c < 0 || static_cast<int64_t>(o1) > nrows) {
+      record_status(kSiteBadIndex);
+      c = 0;
+    }
+    S->cnt[e] = c;
+    S->off[e] = o0;
+    my_tiles = ((c + BNT - 1) / BNT) * C::FBLK;
+  }
+  int incl = my_tiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
+  if (warp == MMA_WARP) tmem_alloc(&S->tmem_base, TMEM_COLS);
+  __syncthreads();
+  if (threadIdx.x < kE) {
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += S->wsum[w];
+    S->tile_start[threadIdx.x] = base + incl - my_tiles;
+    if (threadIdx.x == kE - 1) S->tile_start[kE] = base + incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = S->tmem_base;
+  const int total_tiles = S->tile_start[kE];
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int e, f, c;
+        decode_tile(S, tile, C::FBLK, e, f, c);
+        int wrow0, wrow1 = 0;
+        if (PHASE == 1) {  // pair j = f/2, half = f%2: gate rows then the matching up rows
+          const int j = f >> 1, half = f & 1;
+          wrow0 = e * 2 * kI + 256 * j + 64 * half;
+          wrow1 = wrow0 + 128;
+        } else {
+          wrow0 = e * kH + f * BMW;
+        }
+        const int hrow = S->off[e] + c * BNT;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&fullb[s], C::TX);
+          if (PHASE == 1) {
+            tma_load_2d(smem_u32(sA(s)), &tmap_w, kb * BK, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)) + A_BYTES / 2, &tmap_w, kb * BK, wrow1, &fullb[s]);
+          } else {
+            tma_load_2d(smem_u32(sA(s)), &tmap_w, kb * BK, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * BK, hrow, &fullb[s]);
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = max(0, it - STAGES); i < it; ++i)
+          mbar_wait(&fullb[i % STAGES], (i / STAGES) & 1, abort_flag, 10000000ull, kSiteFfnFull);
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tc) {
+        const int a = tc & 1;
+        const uint32_t use = tc >> 1;
+        if (!mbar_wait(&S->tempty[a], (use & 1) ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + a * BNT;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&fullb[s], ph, abort_flag, timeout_ns, kSiteFfnFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_k128(smem_u32(sA(s)));
+          const uint64_t bdesc = smem_desc_k128(smem_u32(sB(s)));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&emptyb[s]);
+        }
+        if (ok) umma_commit(&S->tfull[a]);
+      }
+      umma_commit(&S->drain);
+      mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
+    }
+  } else if (PHASE == 1 && warp == GATHER_WARP) {
+    const uint32_t swz = static_cast<uint32_t>(lane & 7);
+    uint32_t dirty = 0xFFu;  // stage slots whose row `lane` may hold non-zero data
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, f, c;
+      decode_tile(S, tile, C::FBLK, e, f, c);
+      const int row_in_e = c * BNT + lane;
+      const char* src = nullptr;
+      if (row_in_e < S->cnt[e]) {
+        const int p = perm_src[S->off[e] + row_in_e];
+        if (p >= 0 && static_cast<int64_t>(p) < nrows)
+          src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
+      }
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = smem_u32(sB(s)) + lane * 128;
+        if (src != nullptr) {
+          const char* g = src + kb * BK * 2;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            cp_async_16(dst + ((static_cast<uint32_t>(q) ^ swz) << 4), g + q * 16, 16);
+          dirty |= 1u << s;
+        } else if (dirty & (1u << s)) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) cp_async_16(dst + q * 16, x, 0);
+          dirty &= ~(1u << s);
+        }
+        cp_async_arrive_noinc(&fullb[s]);
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp < 4) {
+    // ------------------------------------------------ epilogue
+    bool range_bad = false;
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
+      int e, f, c;
+      decode_tile(S, tile, C::FBLK, e, f, c);
+      const int a = tc & 1;
+      const uint32_t use = tc >> 1;
+      if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * BNT, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->tempty[a]);  // accumulator copied out: MMA may reuse it
+      const int ntok = min(BNT, S->cnt[e] - c * BNT);
+      const int64_t row0 = static_cast<int64_t>(S->off[e]) + c * BNT;
+      if (PHASE == 1) {
+        const uint32_t xph = static_cast<uint32_t>(tc) & 1;
+        if (warp >= 2) {  // up half: hand the values to the gate half
+          if (!mbar_wait(&S->xempty, xph ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) break;
+          float* xr = xchg + ((warp - 2) * 32 + lane) * XSTRIDE;
+#pragma unroll
+          for (int t = 0; t < BNT; ++t) xr[t] = __uint_as_float(v[t]);
+          mbar_arrive(&S->xfull);
+        } else {
+          if (!mbar_wait(&S->xfull, xph, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
+          const int j = f >> 1, half = f & 1;
+          const int col = 128 * j + 64 * half + warp * 32 + lane;  // h column (intermediate feature)
+          const float* xr = xchg + (warp * 32 + lane) * XSTRIDE;
+          float up[BNT];
+#pragma unroll
+          for (int t = 0; t < BNT; ++t) up[t] = xr[t];
+          mbar_arrive(&S->xempty);  // exchange tile free for the next tile
+#pragma unroll
+          for (int t = 0; t < BNT; ++t) {
+            if (t < ntok) {
+              const float hv = ffn::silu_mul(__uint_as_float(v[t]), up[t]);
+              range_bad |= !(fabsf(hv) <= 65504.f);
+              st_global_b16(out + (row0 + t) * C::OUT_COLS + col,
+                            __half_as_ushort(__float2half_rn(hv)));
+            }
+          }
+        }
+      } else {
+        const int col = f * BMW + warp * 32 + lane;  // y column (model feature)
+#pragma unroll
+        for (int t = 0; t < BNT; ++t) {
+          if (t < ntok) {
+            const float yv = __uint_as_float(v[t]);
+            range_bad |= !(fabsf(yv) <= 65504.f);
+            st_global_b16(out + (row0 + t) * C::OUT_COLS + col, __half_as_ushort(__float2half_rn(yv)));
+          }
+        }
+      }
+    }
+    if (range_bad) record_status(kSiteFp16Range);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace skinny
+}  // namespace moe

@@ -15,6 +15,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "expert_ffn.cuh"
+#include "expert_ffn_skinny.cuh"
 #include "pack.cuh"
 #include "permute.cuh"
 #include "route.cuh"
@@ -27,6 +28,7 @@ constexpr int kAbiVersion = 1;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 4096;  // gate/up keeps padding rows of A zeroed up to this T
+constexpr int64_t kSkinnyMaxT = 256;    // weights-as-M (skinny) GEMMs up to this T
 
 thread_local char g_err[512] = "";
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
@@ -87,6 +89,12 @@ int device_setup(int* dev_out, int* sms_out) {
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<2, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       if (g_encode == nullptr) {
         cudaDriverEntryPointQueryResult q;
@@ -177,6 +185,15 @@ int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets,
 
 int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                const int32_t* perm_src, int64_t T, moe_bf16* h, int sms, cudaStream_t s) {
+  if (T <= kSkinnyMaxT) {
+    CUtensorMap tw;
+    int rc = make_tmap(&tw, packed, kH, uint64_t(kE) * 2 * kI, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    if (rc) return rc;
+    skinny::skinny_gemm_kernel<1><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
+        tw, tw, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+        reinterpret_cast<uint16_t*>(h), g_timeout_ns.load());
+    return launch_check("skinny_gemm_kernel<1> launch");
+  }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
@@ -196,6 +213,15 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
             moe_bf16* y, int sms, cudaStream_t s) {
   CUtensorMap tb2, ta2;
   const uint64_t rows = static_cast<uint64_t>(T) * kTopK;
+  if (T <= kSkinnyMaxT) {
+    int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, skinny::BMW,
+                       CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (!rc) rc = make_tmap(&ta2, h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+    skinny::skinny_gemm_kernel<2><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
+        tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
+    return launch_check("skinny_gemm_kernel<2> launch");
+  }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);

@@ -151,6 +151,12 @@ def test_expert_ffn_dense_special_case():
     _ffn_check(333, 21, forced=[3, 4, 21, 22, 40, 41, 90, 91])
 
 
+def test_expert_ffn_forced_small_batch():
+    """Small batch (weights-as-M kernels) with every token forced onto the same 8
+    experts: 200 rows per expert = seven 32-token chunks, the last one ragged."""
+    _ffn_check(200, 22, forced=[0, 1, 16, 17, 32, 33, 48, 49])
+
+
 def test_combine_parity():
     moe = _moe()
     rng = np.random.default_rng(9)
