@@ -29,7 +29,10 @@
 // TMEM columns):
 //   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SwiGLU, fp16 stores
 //   warps 4-7  (phase 1) A producers: gather the tile's token rows of x with
-//              cp.async into the 128B-swizzled operand layout; each thread
+//              cp.async into the 128B-swizzled operand layout, eight threads
+//              per row so that each warp instruction moves whole 128-byte
+//              lines (16-byte-per-row access touched every L2 sector twice
+//              and cost ~40% of the gate/up time at T=8189); each thread
 //              signals the stage's barrier through cp.async.mbarrier.arrive,
 //              so the gather keeps all stages in flight.  Rows past the
 //              expert's count are not loaded (a row of A only reaches the
@@ -289,20 +292,29 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     }
   } else if (PHASE == 1 && warp >= 4 && warp < 8) {
     // ------------------------------------------------ A gather producers
-    const int r = threadIdx.x - 128;  // row of the tile
-    const uint32_t swz = static_cast<uint32_t>(r & 7);
-    uint32_t dirty = (1u << STAGES) - 1;  // stage slots whose row r may be non-zero
+    // Thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 16 i, i < 8, so a
+    // warp instruction moves four whole 128-byte rows (full L2 lines).  The
+    // swizzled chunk slot (chunk ^ (row & 7)) is the same for all of a
+    // thread's rows because the row stride is 16.
+    const int t = threadIdx.x - 128;
+    const int chunk = t & 7, rsub = t >> 3;
+    const uint32_t slot = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
+    uint32_t dirty = 0xFFFFFFFFu;  // bit 8*s + i: row rsub+16i of stage s may be non-zero
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       int e, m, j;
       decode_tile(S, tile, C::NT, e, m, j);
-      const int row_in_e = m * BM + r;
-      const char* src = nullptr;
-      if (row_in_e < S->cnt[e]) {
-        const int p = perm_src[S->off[e] + row_in_e];
-        if (p >= 0 && static_cast<int64_t>(p) < nrows)
-          src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
+      const char* src[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        src[i] = nullptr;
+        const int row_in_e = m * BM + rsub + 16 * i;
+        if (row_in_e < S->cnt[e]) {
+          const int p = perm_src[S->off[e] + row_in_e];
+          if (p >= 0 && static_cast<int64_t>(p) < nrows)
+            src[i] = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH) + chunk * 16;
+        }
       }
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int s = it % STAGES;
@@ -311,22 +323,19 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           ok = false;
           break;
         }
-        const uint32_t dst = smem_u32(sA + s * A_BYTES) + r * 128;
-        if (src != nullptr) {
-          const char* g = src + kb * BK * 2;
+        const uint32_t base = smem_u32(sA + s * A_BYTES) + rsub * 128 + slot;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            cp_async_16(dst + ((static_cast<uint32_t>(c) ^ swz) << 4), g + c * 16, 16);
-          cp_async_arrive_noinc(&S->full[s]);
-          dirty |= 1u << s;
-        } else {
-          if (ZERO_PAD && (dirty & (1u << s))) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) cp_async_16(dst + c * 16, x, 0);
-            dirty &= ~(1u << s);
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t bit = 1u << (8 * s + i);
+          if (src[i] != nullptr) {
+            cp_async_16(base + i * 16 * 128, src[i] + kb * BK * 2, 16);
+            dirty |= bit;
+          } else if (ZERO_PAD && (dirty & bit)) {
+            cp_async_16(base + i * 16 * 128, x, 0);
+            dirty &= ~bit;
           }
-          cp_async_arrive_noinc(&S->full[s]);
         }
+        cp_async_arrive_noinc(&S->full[s]);
       }
     }
     cp_async_wait_all();

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "expert_ffn.cuh"
 #include "expert_ffn_skinny.cuh"
+#include "expert_ffn_pair.cuh"
 #include "pack.cuh"
 #include "permute.cuh"
 #include "route.cuh"
@@ -29,6 +30,7 @@ constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 4096;  // gate/up keeps padding rows of A zeroed up to this T
 constexpr int64_t kSkinnyMaxT = 256;    // weights-as-M (skinny) GEMMs up to this T
+constexpr int64_t kPairMinT = 1025;     // CTA-pair (M = 256) GEMMs from this T
 
 thread_local char g_err[512] = "";
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
@@ -95,6 +97,12 @@ int device_setup(int* dev_out, int* sms_out) {
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<2>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(pair::pair_gemm_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(pair::pair_gemm_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       if (g_encode == nullptr) {
         cudaDriverEntryPointQueryResult q;
@@ -194,6 +202,16 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
         reinterpret_cast<uint16_t*>(h), g_timeout_ns.load());
     return launch_check("skinny_gemm_kernel<1> launch");
   }
+  if (T >= kPairMinT) {
+    CUtensorMap tw;
+    int rc = make_tmap(&tw, packed, kH, uint64_t(kE) * 2 * kI, pair::BN / 2,
+                       CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    if (rc) return rc;
+    pair::pair_gemm_kernel<1><<<sms / 2 * 2, pair::PCfg<1>::THREADS, pair::SMEM_BYTES, s>>>(
+        tw, tw, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+        reinterpret_cast<uint16_t*>(h), g_timeout_ns.load());
+    return launch_check("pair_gemm_kernel<1> launch");
+  }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
@@ -221,6 +239,15 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
     skinny::skinny_gemm_kernel<2><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
         tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
     return launch_check("skinny_gemm_kernel<2> launch");
+  }
+  if (T >= kPairMinT) {
+    int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, pair::BN / 2,
+                       CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (!rc) rc = make_tmap(&ta2, h, kI, rows, pair::BMC, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+    pair::pair_gemm_kernel<2><<<sms / 2 * 2, pair::PCfg<2>::THREADS, pair::SMEM_BYTES, s>>>(
+        tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
+    return launch_check("pair_gemm_kernel<2> launch");
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);

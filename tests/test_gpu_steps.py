@@ -157,6 +157,12 @@ def test_expert_ffn_forced_small_batch():
     _ffn_check(200, 22, forced=[0, 1, 16, 17, 32, 33, 48, 49])
 
 
+def test_expert_ffn_forced_large_batch():
+    """Large batch (CTA-pair kernels, 256-row tiles) with every token forced onto
+    the same 8 experts: 1500 rows per expert = six pair tiles, the last ragged."""
+    _ffn_check(1500, 24, forced=[2, 3, 50, 51, 64, 65, 126, 127])
+
+
 def test_combine_parity():
     moe = _moe()
     rng = np.random.default_rng(9)
