@@ -167,7 +167,7 @@ class LayerRun:
         self.idx = torch.empty((T, 8), dtype=i32, device=dev)
         self.w = torch.empty((T, 8), dtype=torch.float32, device=dev)
         self.counts = torch.empty(128, dtype=i32, device=dev)
-        self.offsets = torch.empty(129, dtype=i32, device=dev)
+        self.offsets = torch.empty(moe.OFFSETS_LEN, dtype=i32, device=dev)
         self.perm_src = torch.empty(n, dtype=i32, device=dev)
         self.inv_perm = torch.empty(n, dtype=i32, device=dev)
         wsb = moe.permute_workspace_bytes(T)

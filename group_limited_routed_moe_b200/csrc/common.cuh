@@ -34,6 +34,7 @@ enum StatusSite : unsigned {
   kSiteFfnTmemFull = 18,
   kSiteFfnTmemEmpty = 19,
   kSiteFfnDrain = 20,
+  kSiteTileQueue = 21,
   kSiteSelftest = 30,
 };
 
@@ -268,106 +269,66 @@ __device__ __forceinline__ void st_global_b16(void* p, uint16_t v) {
   asm volatile("st.global.b16 [%0], %1;" ::"l"(p), "h"(v) : "memory");
 }
 
-// ---------------------------------------------------------------- CTA pairs (cluster of 2)
+// ---------------------------------------------------------------- dynamic tile queue
+// Persistent GEMM CTAs take their first tile statically (blockIdx.x) and then
+// grab tiles from a global counter, so that a CTA that met slow tiles (weights
+// from HBM rather than L2, stalls) takes fewer of them.  Inside a CTA one
+// thread grabs tile ids and publishes them through a small shared-memory queue
+// that every warp role reads in the same order.  The counter words live after
+// the expert offsets (see kSchedWord): moe_permute zeroes them, and the last
+// CTA of every GEMM launch sets them back to zero.
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
+constexpr int kTileQ = 4;          // queue slots
+constexpr int kSchedWord = 132;    // offsets[132..135]: scheduler words (2 per GEMM phase)
+constexpr int kOffsetsLen = 136;   // length of the offsets array
 
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
+struct TileQueue {
+  int tile[kTileQ];
+  uint64_t full[kTileQ];
+  uint64_t empty[kTileQ];
+};
 
-// Arrive on an mbarrier of another CTA of the cluster (cluster-scope release).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire (for barriers that the peer CTA
-// arrives on).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint64_t timeout_ns,
-                                                  unsigned site) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((n & 31u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > timeout_ns) {
-        record_status(site);
-        *abort_flag = 1;
-        return false;
-      }
-    }
+__device__ __forceinline__ void tileq_init(TileQueue* q, uint32_t consumers) {
+  for (int i = 0; i < kTileQ; ++i) {
+    mbar_init(&q->full[i], 1);
+    mbar_init(&q->empty[i], consumers);
   }
 }
 
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
+// Producer side (one thread): publish tile id `tile` (or -1 = no more work) as
+// the n-th entry.  Returns false if the wait for a free slot ran out.
+__device__ __forceinline__ bool tileq_push(TileQueue* q, int n, int tile, volatile int* abort_flag,
+                                           uint64_t timeout_ns) {
+  const int slot = n % kTileQ;
+  const uint32_t ph = (n / kTileQ) & 1;
+  if (!mbar_wait(&q->empty[slot], ph ^ 1, abort_flag, timeout_ns, kSiteTileQueue)) return false;
+  reinterpret_cast<volatile int*>(q->tile)[slot] = tile;
+  mbar_arrive(&q->full[slot]);
+  return true;
 }
 
-// TMA tile load of a CTA pair: the bytes land in this CTA's shared memory and
-// are counted on `bar_cluster`, an mbarrier that may live in the peer CTA.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0,
-                                                 int32_t c1, uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
-      : "memory");
+// Consumer side: the n-th tile id (-1: no more work, -2: wait ran out).  Every
+// lane of a consuming warp calls this; lane 0 (or the single consuming
+// thread) releases the slot after the whole warp has read it.
+__device__ __forceinline__ int tileq_pop(TileQueue* q, int n, bool release,
+                                         volatile int* abort_flag, uint64_t timeout_ns) {
+  const int slot = n % kTileQ;
+  const uint32_t ph = (n / kTileQ) & 1;
+  if (!mbar_wait(&q->full[slot], ph, abort_flag, timeout_ns, kSiteTileQueue)) return -2;
+  const int tile = reinterpret_cast<volatile int*>(q->tile)[slot];
+  __syncwarp(__activemask());
+  if (release) mbar_arrive(&q->empty[slot]);
+  return tile;
 }
 
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(slot_smem)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, M = 256.
-__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive on `bar` (same offset) in every CTA of `mask` once the pair MMAs
-// issued so far by this thread are done.
-__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"(mask)
-      : "memory");
+// End of a launch: the last CTA to finish zeroes the two counter words.
+__device__ __forceinline__ void tileq_retire(int* sched) {
+  __threadfence();
+  const int done = atomicAdd(sched + 1, 1);
+  if (done == static_cast<int>(gridDim.x) - 1) {
+    atomicExch(sched, 0);
+    atomicExch(sched + 1, 0);
+  }
 }
 
 // ---------------------------------------------------------------- misc

@@ -20,10 +20,13 @@
 // sets the device status word (kSiteFp16Range) instead of passing silently.
 //
 // Work is cut into tiles (expert e, n-tile j, m-tile m) of 128 rows x 256
-// columns; tile ids run expert-major, then j, then m, so consecutive CTAs
-// share an expert's weight tile through L2.  A persistent grid of one CTA per
-// SM walks the ids round-robin.  The tile table is built by each CTA from the
-// device-side expert offsets, so the host never reads them.
+// columns; tile ids run expert-major, then j, then m, so CTAs that run at the
+// same time share an expert's weight tile through L2.  A persistent grid of
+// one CTA per SM takes tile ids from a global counter (first tile: blockIdx.x),
+// so that CTAs held up by slow tiles take fewer of them; static round-robin
+// left some CTAs up to 1.5x longer than the median.  The tile table is built
+// by each CTA from the device-side expert offsets, so the host never reads
+// them.
 //
 // Warp roles inside a CTA (one CTA per SM: ~194 KB of shared memory, all 512
 // TMEM columns):
@@ -100,6 +103,7 @@ struct SmemTail {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  TileQueue tq;
   uint32_t tmem_base;
   int abort_flag;
   int wsum[4];
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_a,
                     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                     const int32_t* __restrict__ perm_src, int64_t T,
-                    uint16_t* __restrict__ out, uint64_t timeout_ns) {
+                    uint16_t* __restrict__ out, int* __restrict__ sched, uint64_t timeout_ns) {
   using C = Cfg<PHASE>;
   constexpr int KB = C::KDIM / BK;
 
@@ -177,6 +181,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       mbar_init(&S->tempty[a], 4);
     }
     mbar_init(&S->drain, 1);
+    tileq_init(&S->tq, (PHASE == 1 ? 4 : 0) + 1 + 4);  // gather warps, MMA thread, epilogue warps
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -208,6 +213,14 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   }
   if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
 
+  if (PHASE == 1) {
+    // Start the A ring at zero: rows past an expert's count are never loaded,
+    // and with whatever the previous kernel left in shared memory there the
+    // tensor cores ran measurably slower than with zeros or stale x rows.
+    for (int i = threadIdx.x; i < STAGES * A_BYTES / 16; i += blockDim.x)
+      st_shared_v4(smem_u32(sA) + i * 16, 0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   if (warp == C::MMA_WARP) tmem_alloc(&S->tmem_base, TMEM_COLS);
   __syncthreads();
   if (threadIdx.x < kE) {
@@ -226,9 +239,17 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   if (warp == C::TMA_WARP) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      int it = 0;
+      int it = 0, n = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int tile = blockIdx.x;
+      while (ok) {
+        const int pub = tile < total_tiles ? tile : -1;
+        if (!tileq_push(&S->tq, n++, pub, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        if (pub < 0) break;
+        const int next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);  // used after the loads
         int e, m, j;
         decode_tile(S, tile, C::NT, e, m, j);
         const int brow = e * C::B_ROWS_PER_EXPERT + j * BN;
@@ -248,6 +269,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           }
           tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b, kb * BK, brow, &S->full[s]);
         }
+        tile = next;
       }
       if (!ok) {
         // let the copies already issued land before the block can exit
@@ -260,7 +282,12 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     if (lane == 0) {
       int it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tc) {
+      for (;; ++tc) {
+        const int tile = tileq_pop(&S->tq, tc, true, abort_flag, timeout_ns);
+        if (tile < 0) {
+          ok = tile == -1;
+          break;
+        }
         const int a = tc & 1;
         const uint32_t use = tc >> 1;
         if (!mbar_wait(&S->tempty[a], (use & 1) ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) {
@@ -299,10 +326,12 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     const int t = threadIdx.x - 128;
     const int chunk = t & 7, rsub = t >> 3;
     const uint32_t slot = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
-    uint32_t dirty = 0xFFFFFFFFu;  // bit 8*s + i: row rsub+16i of stage s may be non-zero
-    int it = 0;
+    uint32_t dirty = 0u;  // bit 8*s + i: row rsub+16i of stage s may be non-zero (ring starts zeroed)
+    int it = 0, n = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+    while (ok) {
+      const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
+      if (tile < 0) break;
       int e, m, j;
       decode_tile(S, tile, C::NT, e, m, j);
       const char* src[8];
@@ -342,8 +371,9 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue
     bool range_bad = false;  // thread (warp w, lane l) owns row 32w + l == TMEM lane
-    int tc = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
+    for (int tc = 0;; ++tc) {
+      const int tile = tileq_pop(&S->tq, tc, lane == 0, abort_flag, timeout_ns);
+      if (tile < 0) break;
       int e, m, j;
       decode_tile(S, tile, C::NT, e, m, j);
       const int a = tc & 1;
@@ -398,6 +428,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) tileq_retire(sched);
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

@@ -71,6 +71,7 @@ struct Tail {
   uint64_t xfull;   // up half written to the exchange tile (64 lane arrivals)
   uint64_t xempty;  // gate half done reading it (64 lane arrivals)
   uint64_t drain;
+  TileQueue tq;
   uint32_t tmem_base;
   int abort_flag;
   int wsum[4];
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                        const __grid_constant__ CUtensorMap tmap_h,
                        const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                        const int32_t* __restrict__ perm_src, int64_t T,
-                       uint16_t* __restrict__ out, uint64_t timeout_ns) {
+                       uint16_t* __restrict__ out, int* __restrict__ sched, uint64_t timeout_ns) {
   using C = SCfg<PHASE>;
   constexpr int KB = C::KDIM / BK;
 
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&S->xfull, 64);
     mbar_init(&S->xempty, 64);
     mbar_init(&S->drain, 1);
+    tileq_init(&S->tq, (PHASE == 1 ? 1 : 0) + 1 + 4);  // gather warp, MMA thread, epilogue warps
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -177,9 +179,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == TMA_WARP) {
     if (lane == 0) {
-      int it = 0;
+      int it = 0, n = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int tile = blockIdx.x;
+      while (ok) {
+        const int pub = tile < total_tiles ? tile : -1;
+        if (!tileq_push(&S->tq, n++, pub, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        if (pub < 0) break;
+        const int next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);
         int e, f, c;
         decode_tile(S, tile, C::FBLK, e, f, c);
         int wrow0, wrow1 = 0;
@@ -207,6 +217,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * BK, hrow, &fullb[s]);
           }
         }
+        tile = next;
       }
       if (!ok) {
         for (int i = max(0, it - STAGES); i < it; ++i)
@@ -217,7 +228,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tc) {
+      for (;; ++tc) {
+        const int tile = tileq_pop(&S->tq, tc, true, abort_flag, timeout_ns);
+        if (tile < 0) {
+          ok = tile == -1;
+          break;
+        }
         const int a = tc & 1;
         const uint32_t use = tc >> 1;
         if (!mbar_wait(&S->tempty[a], (use & 1) ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) {
@@ -249,9 +265,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (PHASE == 1 && warp == GATHER_WARP) {
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
     uint32_t dirty = 0xFFu;  // stage slots whose row `lane` may hold non-zero data
-    int it = 0;
+    int it = 0, n = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+    while (ok) {
+      const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
+      if (tile < 0) break;
       int e, f, c;
       decode_tile(S, tile, C::FBLK, e, f, c);
       const int row_in_e = c * BNT + lane;
@@ -287,8 +305,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue
     bool range_bad = false;
-    int tc = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
+    for (int tc = 0;; ++tc) {
+      const int tile = tileq_pop(&S->tq, tc, lane == 0, abort_flag, timeout_ns);
+      if (tile < 0) break;
       int e, f, c;
       decode_tile(S, tile, C::FBLK, e, f, c);
       const int a = tc & 1;
@@ -346,6 +365,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) tileq_retire(sched);
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

@@ -16,7 +16,6 @@
 #include "common.cuh"
 #include "expert_ffn.cuh"
 #include "expert_ffn_skinny.cuh"
-#include "expert_ffn_pair.cuh"
 #include "pack.cuh"
 #include "permute.cuh"
 #include "route.cuh"
@@ -28,9 +27,8 @@ namespace {
 constexpr int kAbiVersion = 1;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
-constexpr int64_t kZeroPadMaxT = 4096;  // gate/up keeps padding rows of A zeroed up to this T
+constexpr int64_t kZeroPadMaxT = 1024;  // gate/up keeps padding rows of A zeroed up to this T
 constexpr int64_t kSkinnyMaxT = 256;    // weights-as-M (skinny) GEMMs up to this T
-constexpr int64_t kPairMinT = 1025;     // CTA-pair (M = 256) GEMMs from this T
 
 thread_local char g_err[512] = "";
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
@@ -97,12 +95,6 @@ int device_setup(int* dev_out, int* sms_out) {
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<2>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(pair::pair_gemm_kernel<1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(pair::pair_gemm_kernel<2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       if (g_encode == nullptr) {
         cudaDriverEntryPointQueryResult q;
@@ -160,7 +152,7 @@ int launch_check(const char* what) {
 // ---- step launchers (arguments already validated) ----------------------------
 int do_route(const float* logits, const float* bias, int64_t T, int32_t* idx, float* w,
              cudaStream_t s) {
-  const int64_t blocks = (T + kRouteWarps - 1) / kRouteWarps;
+  const int64_t blocks = (T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock;
   route_kernel<<<static_cast<unsigned>(blocks), kRouteWarps * 32, 0, s>>>(logits, bias, T, idx, w);
   return launch_check("route_kernel launch");
 }
@@ -183,12 +175,23 @@ int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets,
   permute_count_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(idx, T, hist);
   int rc = launch_check("permute_count_kernel launch");
   if (rc) return rc;
+  if (nb <= kPermFusedMaxBlocks) {
+    permute_scan_scatter_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(
+        idx, T, hist, static_cast<int>(nb), counts, offsets, perm_src, inv_perm);
+    return launch_check("permute_scan_scatter_kernel launch");
+  }
   permute_scan_kernel<<<1, 1024, 0, s>>>(hist, static_cast<int>(nb), counts, offsets);
   rc = launch_check("permute_scan_kernel launch");
   if (rc) return rc;
   permute_scatter_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(idx, T, hist, offsets, perm_src,
                                                                    inv_perm);
   return launch_check("permute_scatter_kernel launch");
+}
+
+// The GEMMs' tile counters live after the expert offsets (zeroed by the permute
+// kernels, left zero by the GEMMs): words kSchedWord.. (gate/up), +2 (down).
+int* sched_words(const int32_t* offsets, int phase) {
+  return const_cast<int*>(offsets) + kSchedWord + 2 * (phase - 1);
 }
 
 int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
@@ -199,18 +202,8 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
     if (rc) return rc;
     skinny::skinny_gemm_kernel<1><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
         tw, tw, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-        reinterpret_cast<uint16_t*>(h), g_timeout_ns.load());
+        reinterpret_cast<uint16_t*>(h), sched_words(offsets, 1), g_timeout_ns.load());
     return launch_check("skinny_gemm_kernel<1> launch");
-  }
-  if (T >= kPairMinT) {
-    CUtensorMap tw;
-    int rc = make_tmap(&tw, packed, kH, uint64_t(kE) * 2 * kI, pair::BN / 2,
-                       CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-    if (rc) return rc;
-    pair::pair_gemm_kernel<1><<<sms / 2 * 2, pair::PCfg<1>::THREADS, pair::SMEM_BYTES, s>>>(
-        tw, tw, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-        reinterpret_cast<uint16_t*>(h), g_timeout_ns.load());
-    return launch_check("pair_gemm_kernel<1> launch");
   }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -220,10 +213,10 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
   auto* hb = reinterpret_cast<uint16_t*>(h);
   if (T <= kZeroPadMaxT)
     ffn::ffn_gemm_kernel<1, true><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
-        tb1, tb1, xb, offsets, perm_src, T, hb, g_timeout_ns.load());
+        tb1, tb1, xb, offsets, perm_src, T, hb, sched_words(offsets, 1), g_timeout_ns.load());
   else
     ffn::ffn_gemm_kernel<1, false><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
-        tb1, tb1, xb, offsets, perm_src, T, hb, g_timeout_ns.load());
+        tb1, tb1, xb, offsets, perm_src, T, hb, sched_words(offsets, 1), g_timeout_ns.load());
   return launch_check("ffn_gemm_kernel<1> launch");
 }
 
@@ -237,24 +230,17 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
     if (!rc) rc = make_tmap(&ta2, h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
     skinny::skinny_gemm_kernel<2><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
-        tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
+        tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y),
+        sched_words(offsets, 2), g_timeout_ns.load());
     return launch_check("skinny_gemm_kernel<2> launch");
-  }
-  if (T >= kPairMinT) {
-    int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, pair::BN / 2,
-                       CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-    if (!rc) rc = make_tmap(&ta2, h, kI, rows, pair::BMC, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-    if (rc) return rc;
-    pair::pair_gemm_kernel<2><<<sms / 2 * 2, pair::PCfg<2>::THREADS, pair::SMEM_BYTES, s>>>(
-        tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
-    return launch_check("pair_gemm_kernel<2> launch");
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
   ffn::ffn_gemm_kernel<2, false><<<sms, ffn::Cfg<2>::THREADS, ffn::SMEM_BYTES, s>>>(
-      tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y), g_timeout_ns.load());
+      tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y),
+        sched_words(offsets, 2), g_timeout_ns.load());
   return launch_check("ffn_gemm_kernel<2> launch");
 }
 
@@ -290,7 +276,7 @@ LayerWs layer_ws(int64_t T) {
   L.idx = take(n * 4);
   L.w = take(n * 4);
   L.counts = take(kE * 4);
-  L.offsets = take((kE + 1) * 4);
+  L.offsets = take(kOffsetsLen * 4);
   L.perm_src = take(n * 4);
   L.inv_perm = take(n * 4);
   L.perm_ws = take(permute_ws_bytes(T));
@@ -386,7 +372,7 @@ int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts, int32_t* of
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (T == 0) {
     MOE_CUDA(cudaMemsetAsync(counts, 0, kE * sizeof(int32_t), s), "cudaMemsetAsync");
-    MOE_CUDA(cudaMemsetAsync(offsets, 0, (kE + 1) * sizeof(int32_t), s), "cudaMemsetAsync");
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, kOffsetsLen * sizeof(int32_t), s), "cudaMemsetAsync");
     return MOE_OK;
   }
   return do_permute(topk_idx, T, counts, offsets, perm_src, inv_perm, workspace, s);

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(1024)
     offsets[tid] = off[tid];
   }
   if (tid == 0) offsets[kE] = off[kE];
+  if (tid < kOffsetsLen - kSchedWord) offsets[kSchedWord + tid] = 0;  // GEMM tile counters
   for (int p = tid; p < n; p += blockDim.x) {
     const int e = idx[p];
     if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
@@ -153,6 +154,74 @@ __global__ void __launch_bounds__(1024)
     offsets[tid] = off[tid];
   }
   if (tid == 0) offsets[kE] = off[kE];
+  if (tid < kOffsetsLen - kSchedWord) offsets[kSchedWord + tid] = 0;  // GEMM tile counters
+}
+
+// (b') fused scan + scatter for up to kPermFusedMaxBlocks blocks: every block
+//      re-derives the expert offsets and its own bases from the histogram
+//      (nb x 128 reads per block), so no separate scan launch is needed.
+constexpr int kPermFusedMaxBlocks = 256;
+
+__global__ void __launch_bounds__(256)
+    permute_scan_scatter_kernel(const int32_t* __restrict__ idx, int64_t T,
+                                const int32_t* __restrict__ hist, int nb,
+                                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm) {
+  constexpr int W = kPermBlockTokens / 32;
+  __shared__ uint32_t bm[kE][W];
+  __shared__ int part[2][kE];
+  __shared__ int before_s[2][kE];
+  __shared__ int cnt[kE];
+  __shared__ int off[kE + 1];
+  __shared__ int base[kE];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int b = blockIdx.x;
+  const int64_t t0 = static_cast<int64_t>(b) * kPermBlockTokens;
+  const int nt = static_cast<int>((T - t0) < kPermBlockTokens ? (T - t0) : kPermBlockTokens);
+  for (int i = tid; i < kE * W; i += blockDim.x) (&bm[0][0])[i] = 0u;
+  {  // column sums: thread (h, e) sums blocks h, h+2, h+4, ...
+    const int e = tid & (kE - 1), h = tid >> 7;
+    int tot = 0, bef = 0;
+    for (int bb = h; bb < nb; bb += 2) {
+      const int v = hist[static_cast<int64_t>(bb) * kE + e];
+      tot += v;
+      if (bb < b) bef += v;
+    }
+    part[h][e] = tot;
+    before_s[h][e] = bef;
+  }
+  __syncthreads();
+  if (tid < kE) cnt[tid] = part[0][tid] + part[1][tid];
+  __syncthreads();
+  if (tid < 32) scan_experts_warp0(cnt, off, lane);
+  __syncthreads();
+  if (tid < kE) base[tid] = off[tid] + before_s[0][tid] + before_s[1][tid];
+  if (b == 0) {
+    if (tid < kE) {
+      counts[tid] = cnt[tid];
+      offsets[tid] = off[tid];
+    }
+    if (tid == 0) offsets[kE] = off[kE];
+    if (tid < kOffsetsLen - kSchedWord) offsets[kSchedWord + tid] = 0;  // GEMM tile counters
+  }
+  for (int q = tid; q < nt * kTopK; q += blockDim.x) {
+    const int e = idx[t0 * kTopK + q];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    const int tl = q >> 3;
+    atomicOr(&bm[e][tl >> 5], 1u << (tl & 31));
+  }
+  __syncthreads();
+  for (int q = tid; q < nt * kTopK; q += blockDim.x) {
+    const int e = idx[t0 * kTopK + q];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    const int tl = q >> 3, w = tl >> 5;
+    int rank = __popc(bm[e][w] & ((1u << (tl & 31)) - 1u));
+    for (int v = 0; v < w; ++v) rank += __popc(bm[e][v]);
+    const int64_t p = t0 * kTopK + q;
+    const int r = base[e] + rank;
+    perm_src[r] = static_cast<int32_t>(p);
+    inv_perm[p] = r;
+  }
 }
 
 // (c) stable scatter of the block's items

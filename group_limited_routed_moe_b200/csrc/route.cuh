@@ -1,4 +1,4 @@
-// route.cuh -- step 1: group-limited top-8 routing, one warp per token.
+// route.cuh -- step 1: group-limited top-8 routing.
 //
 // Layer facts: 128 experts in 8 groups of 16, 4 groups kept ("Ling-3.0-tiny
 // on a Qualcomm board", TensorFold issue #1247, first comment, opening
@@ -8,16 +8,23 @@
 // best s inside them (ties to the lower expert index) in descending order;
 // weights sigmoid(logit) renormalised over the 8.
 //
+// Eight lanes route one token (four tokens per warp): lane g of the segment
+// owns group g, so the group's top-2 is lane-local, the group ranking is eight
+// segment shuffles, and each of the 8 selection rounds is a lane-local scan
+// plus three shuffle levels.
+//
 // The selection keys are float64, so that the decisions match a float64
-// evaluation of the same rule (a near-tie would have to be closer than about
-// 1e-16 to flip).  Lane l owns experts 4l..4l+3, so group j is lanes 4j..4j+3
-// and the group top-2 merge needs two shuffles.
+// evaluation of the same rule.  For s in [0, 1] the bit pattern of the double
+// orders exactly like the value, so a candidate's key is bits(s) + 1 as an
+// unsigned 64-bit integer (0 marks an excluded or already-taken expert).
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kRouteWarps = 8;  // tokens per block
+constexpr int kRouteTokensPerWarp = 4;
+constexpr int kRouteWarps = 8;
+constexpr int kRouteTokensPerBlock = kRouteTokensPerWarp * kRouteWarps;  // 32
 
 __device__ __forceinline__ double sigmoid_f64(double z) { return 1.0 / (1.0 + exp(-z)); }
 
@@ -26,101 +33,96 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const unsigned FULL = 0xFFFFFFFFu;
   const int lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps + (threadIdx.x >> 5);
-  if (t >= T) return;  // uniform per warp
+  const int g = lane & 7;  // group owned by this lane; also its slot in the segment
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock +
+                    (threadIdx.x >> 5) * kRouteTokensPerWarp + (lane >> 3);
+  const bool active = t < T;  // the whole segment agrees; inactive lanes still shuffle
 
-  const float4 lg = __ldg(reinterpret_cast<const float4*>(logits + t * kE) + lane);
-  float4 bs = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (bias != nullptr) bs = __ldg(reinterpret_cast<const float4*>(bias) + lane);
-
-  double s[4];
-  s[0] = sigmoid_f64(static_cast<double>(lg.x) + static_cast<double>(bs.x));
-  s[1] = sigmoid_f64(static_cast<double>(lg.y) + static_cast<double>(bs.y));
-  s[2] = sigmoid_f64(static_cast<double>(lg.z) + static_cast<double>(bs.z));
-  s[3] = sigmoid_f64(static_cast<double>(lg.w) + static_cast<double>(bs.w));
-
-  // top-2 values of the lane's four scores
-  double a1 = fmax(s[0], s[1]), a2 = fmin(s[0], s[1]);
+  // this lane's 16 logits and biases (the segment reads the token's 512 bytes)
+  float lg[16], bs[16];
+  {
+    const float4* src = reinterpret_cast<const float4*>(logits + (active ? t : 0) * kE + g * kGS);
+    const float4* bsrc = reinterpret_cast<const float4*>(bias + g * kGS);
 #pragma unroll
-  for (int i = 2; i < 4; ++i) {
-    if (s[i] > a1) {
-      a2 = a1;
-      a1 = s[i];
-    } else if (s[i] > a2) {
-      a2 = s[i];
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = __ldg(src + q);
+      lg[4 * q] = v.x;
+      lg[4 * q + 1] = v.y;
+      lg[4 * q + 2] = v.z;
+      lg[4 * q + 3] = v.w;
+      const float4 b = bias != nullptr ? __ldg(bsrc + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      bs[4 * q] = b.x;
+      bs[4 * q + 1] = b.y;
+      bs[4 * q + 2] = b.z;
+      bs[4 * q + 3] = b.w;
     }
   }
-  // merge with the other three lanes of the group
+
+  // scores, their keys, and the group's two best scores
+  unsigned long long key[16];
+  double a1 = -1.0, a2 = -1.0;
 #pragma unroll
-  for (int off = 1; off <= 2; off <<= 1) {
-    const double b1 = __shfl_xor_sync(FULL, a1, off);
-    const double b2 = __shfl_xor_sync(FULL, a2, off);
-    if (a1 >= b1) {
-      a2 = fmax(a2, b1);
-    } else {
-      a2 = fmax(b2, a1);
-      a1 = b1;
+  for (int i = 0; i < 16; ++i) {
+    const double sv = sigmoid_f64(static_cast<double>(lg[i]) + static_cast<double>(bs[i]));
+    key[i] = static_cast<unsigned long long>(__double_as_longlong(sv)) + 1ull;
+    if (sv > a1) {
+      a2 = a1;
+      a1 = sv;
+    } else if (sv > a2) {
+      a2 = sv;
     }
   }
   const double gscore = a1 + a2;
-  const int my_group = lane >> 2;
 
-  // rank of this lane's group among the 8 (ties: lower index ranks first)
+  // rank of this group among the token's 8 (ties: lower index ranks first)
   int rank = 0;
 #pragma unroll
   for (int j = 0; j < kG; ++j) {
-    const double gj = __shfl_sync(FULL, gscore, 4 * j);
-    rank += (gj > gscore) || (gj == gscore && j < my_group);
+    const double gj = __shfl_sync(FULL, gscore, j, 8);
+    rank += (gj > gscore) || (gj == gscore && j < g);
   }
-  const bool kept = rank < kKeep;
-
-  // Candidates: kept experts' scores.  A score s lies in [0, 1], and the bit
-  // pattern of a non-negative double orders exactly like its value, so the
-  // key (hi word + 2^30, lo word) compares candidates exactly; 0 marks an
-  // excluded or already-taken expert.  Each round takes the warp maximum of
-  // the high words, then of the low words among lanes holding that high
-  // word, then the lowest expert index among exact ties.
-  uint32_t khi[4], klo[4];
+  if (rank >= kKeep) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(s[i]));
-    khi[i] = kept ? static_cast<uint32_t>(b >> 32) + 0x40000000u : 0u;
-    klo[i] = kept ? static_cast<uint32_t>(b) : 0u;
+    for (int i = 0; i < 16; ++i) key[i] = 0ull;
   }
 
-  int sel = -1;  // lane k (k < 8) ends up holding the k-th selected expert
+  int sel = -1;  // segment lane k ends up holding the k-th selected expert
 #pragma unroll 1
   for (int k = 0; k < kTopK; ++k) {
-    // lane-local best (ties: lower index, i.e. first)
-    uint32_t bh = khi[0], bl = klo[0];
+    unsigned long long bk = key[0];
     int bi = 0;
 #pragma unroll
-    for (int i = 1; i < 4; ++i) {
-      if (khi[i] > bh || (khi[i] == bh && klo[i] > bl)) {
-        bh = khi[i];
-        bl = klo[i];
+    for (int i = 1; i < 16; ++i) {
+      if (key[i] > bk) {  // strict: keeps the lower index on exact ties
+        bk = key[i];
         bi = i;
       }
     }
-    const uint32_t mh = __reduce_max_sync(FULL, bh);
-    const uint32_t ml = __reduce_max_sync(FULL, bh == mh ? bl : 0u);
-    const bool mine = (bh == mh) && (bl == ml);
-    const uint32_t be = __reduce_min_sync(FULL, mine ? static_cast<uint32_t>(4 * lane + bi) : 0xFFFFFFFFu);
-    if (lane == k) sel = static_cast<int>(be);
+    int be = g * kGS + bi;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (static_cast<uint32_t>(4 * lane + i) == be) khi[i] = klo[i] = 0u;
+    for (int off = 4; off >= 1; off >>= 1) {
+      const unsigned long long ok = __shfl_xor_sync(FULL, bk, off, 8);
+      const int oe = __shfl_xor_sync(FULL, be, off, 8);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    if (g == k) sel = be;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (g * kGS + i == be) key[i] = 0ull;
   }
 
   // combine weights: sigmoid of the raw logit, renormalised over the 8
-  double sig = 0.0;
-  if (lane < kTopK) sig = sigmoid_f64(static_cast<double>(__ldg(logits + t * kE + sel)));
+  const double sig =
+      active ? sigmoid_f64(static_cast<double>(__ldg(logits + t * kE + sel))) : 0.0;
   double tot = sig;
 #pragma unroll
-  for (int off = 1; off < 8; off <<= 1) tot += __shfl_xor_sync(FULL, tot, off);
-  if (lane < kTopK) {
-    topk_idx[t * kTopK + lane] = sel;
-    topk_w[t * kTopK + lane] = static_cast<float>(sig / tot);
+  for (int off = 1; off < 8; off <<= 1) tot += __shfl_xor_sync(FULL, tot, off, 8);
+  if (active) {
+    topk_idx[t * kTopK + g] = sel;
+    topk_w[t * kTopK + g] = static_cast<float>(sig / tot);
   }
 }
 

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 HIDDEN, INTER, N_EXPERTS, N_GROUPS, KEEP_GROUPS, TOPK = 1536, 512, 128, 8, 4, 8
+OFFSETS_LEN = 136  # 129 expert offsets + scratch words used by the expert-FFN kernels
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
     MOE_ERR_UNSUPPORTED, MOE_ERR_RANGE = range(7)
 
@@ -131,13 +132,18 @@ def permute_workspace_bytes(T: int) -> int:
 
 def moe_permute(topk_idx: torch.Tensor, counts=None, offsets=None, perm_src=None, inv_perm=None,
                 workspace=None, stream=None):
-    """Returns (counts[128], offsets[129], perm_src[8T], inv_perm[8T]) int32."""
+    """Returns (counts[128], offsets[129], perm_src[8T], inv_perm[8T]) int32.
+
+    ``offsets`` is a view of the first 129 words of an OFFSETS_LEN-word buffer;
+    pass it on unchanged to the expert-FFN calls (they use the trailing words)."""
     T = topk_idx.shape[0]
     dev = topk_idx.device
     if counts is None:
         counts = torch.empty(N_EXPERTS, dtype=torch.int32, device=dev)
     if offsets is None:
-        offsets = torch.empty(N_EXPERTS + 1, dtype=torch.int32, device=dev)
+        offsets = torch.empty(OFFSETS_LEN, dtype=torch.int32, device=dev)
+    if offsets.numel() < OFFSETS_LEN:
+        raise ValueError(f"offsets needs {OFFSETS_LEN} int32 words")
     if perm_src is None:
         perm_src = torch.empty(max(T * TOPK, 1), dtype=torch.int32, device=dev)
     if inv_perm is None:
@@ -149,7 +155,7 @@ def moe_permute(topk_idx: torch.Tensor, counts=None, offsets=None, perm_src=None
                                           _ptr(perm_src), _ptr(inv_perm),
                                           _ptr(workspace) if wsb else None,
                                           workspace.numel() if wsb else 0, _stream(stream)))
-    return counts, offsets, perm_src[:T * TOPK], inv_perm[:T * TOPK]
+    return counts, offsets[:N_EXPERTS + 1], perm_src[:T * TOPK], inv_perm[:T * TOPK]
 
 
 def moe_expert_ffn(x: torch.Tensor, packed_w: torch.Tensor, offsets: torch.Tensor,

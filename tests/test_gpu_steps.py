@@ -158,8 +158,8 @@ def test_expert_ffn_forced_small_batch():
 
 
 def test_expert_ffn_forced_large_batch():
-    """Large batch (CTA-pair kernels, 256-row tiles) with every token forced onto
-    the same 8 experts: 1500 rows per expert = six pair tiles, the last ragged."""
+    """Large batch (128-row token tiles, no padding zeroing) with every token
+    forced onto the same 8 experts: 1500 rows per expert = 12 tiles, the last ragged."""
     _ffn_check(1500, 24, forced=[2, 3, 50, 51, 64, 65, 126, 127])
 
 
