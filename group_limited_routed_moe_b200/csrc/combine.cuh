@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint16_t* __restrict__ y_perm, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ inv_perm, int64_t T,
                    const __nv_bfloat16* residual, __nv_bfloat16* out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int64_t t = blockIdx.x;
   if (t >= T) return;
   const int col = threadIdx.x * 8;

@@ -269,6 +269,18 @@ __device__ __forceinline__ void st_global_b16(void* p, uint16_t v) {
   asm volatile("st.global.b16 [%0], %1;" ::"l"(p), "h"(v) : "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// The layer's kernels are launched with programmatic stream serialisation: a
+// kernel may be scheduled while its predecessor finishes, runs its prologue,
+// and waits (griddep_wait) for the predecessor's completion and memory before
+// touching anything the predecessor produces or reads.  Every kernel lets its
+// successor launch as soon as all of its own CTAs are resident.  Launched
+// without the attribute, both instructions do nothing.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- dynamic tile queue
 // Persistent GEMM CTAs take their first tile statically (blockIdx.x) and then
 // grab tiles from a global counter, so that a CTA that met slow tiles (weights

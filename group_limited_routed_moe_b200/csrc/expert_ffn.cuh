@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nrows = T * kTopK;
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -192,6 +193,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   }
 
   // tile table: tiles of expert e = ceil(count_e / 128) * NT, exclusive prefix
+  griddep_wait();  // offsets, perm_src and (phase 2) h come from the preceding kernels
   int my_tiles = 0;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;

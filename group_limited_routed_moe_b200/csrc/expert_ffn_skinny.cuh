@@ -5,7 +5,7 @@
 // At decode an expert sees one or two of a batch's tokens.  A 128-row token
 // tile would spend 127 rows of tensor work on padding; here a tile is 128
 // weight rows x 32 tokens (tcgen05.mma M=128, N=32), each pipeline stage holds
-// 16 KB of weights and 4 KB of token rows, and eight stages keep 128 KB of
+// 16 KB of weights and 4 KB of token rows, and ten stages keep 160 KB of
 // weights in flight per SM, so the kernel streams the selected experts'
 // weights at HBM speed (the layer's bound at small batches).
 //
@@ -31,7 +31,7 @@ namespace skinny {
 constexpr int BMW = 128;  // weight rows per tile (MMA M)
 constexpr int BNT = 32;   // tokens per tile (MMA N)
 constexpr int BK = 64;
-constexpr int STAGES = 8;
+constexpr int STAGES = 10;
 constexpr int A_BYTES = BMW * BK * 2;  // 16 KB
 constexpr int B_BYTES = BNT * BK * 2;  // 4 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nrows = T * kTopK;
+  griddep_launch_dependents();
   auto sA = [&](int s) { return smem + s * STAGE_BYTES; };
   auto sB = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
 
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (PHASE == 2) tma_prefetch_desc(&tmap_h);
   }
 
+  griddep_wait();  // offsets, perm_src and (phase 2) h come from the preceding kernels
   int my_tiles = 0;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (PHASE == 1 && warp == GATHER_WARP) {
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
-    uint32_t dirty = 0xFFu;  // stage slots whose row `lane` may hold non-zero data
+    uint32_t dirty = (1u << STAGES) - 1;  // stage slots whose row `lane` may hold non-zero data
     int it = 0, n = 0;
     bool ok = true;
     while (ok) {

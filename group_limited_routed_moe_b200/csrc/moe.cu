@@ -143,6 +143,25 @@ int check_T(int64_t T) {
     if (!(cond)) return fail(MOE_ERR_INVALID_ARG, __VA_ARGS__);    \
   } while (0)
 
+// Launch with programmatic stream serialisation (see griddep_wait).
+template <typename... KArgs, typename... Args>
+int launch_pdl(const char* what, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+               cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return MOE_OK;
+}
+
 int launch_check(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -153,8 +172,8 @@ int launch_check(const char* what) {
 int do_route(const float* logits, const float* bias, int64_t T, int32_t* idx, float* w,
              cudaStream_t s) {
   const int64_t blocks = (T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock;
-  route_kernel<<<static_cast<unsigned>(blocks), kRouteWarps * 32, 0, s>>>(logits, bias, T, idx, w);
-  return launch_check("route_kernel launch");
+  return launch_pdl("route_kernel launch", route_kernel, dim3(static_cast<unsigned>(blocks)),
+                    dim3(kRouteWarps * 32), 0, s, logits, bias, T, idx, w);
 }
 
 size_t permute_ws_bytes(int64_t T) {
@@ -166,26 +185,27 @@ size_t permute_ws_bytes(int64_t T) {
 int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets, int32_t* perm_src,
                int32_t* inv_perm, void* ws, cudaStream_t s) {
   if (T <= kPermSmallMaxT) {
-    permute_small_kernel<<<1, 1024, 0, s>>>(idx, static_cast<int>(T), counts, offsets, perm_src,
-                                            inv_perm);
-    return launch_check("permute_small_kernel launch");
+    return launch_pdl("permute_small_kernel launch", permute_small_kernel, dim3(1), dim3(1024), 0,
+                      s, idx, static_cast<int>(T), counts, offsets, perm_src, inv_perm);
   }
   const int64_t nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
   int32_t* hist = static_cast<int32_t*>(ws);
-  permute_count_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(idx, T, hist);
-  int rc = launch_check("permute_count_kernel launch");
+  int rc = launch_pdl("permute_count_kernel launch", permute_count_kernel,
+                      dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T, hist);
   if (rc) return rc;
   if (nb <= kPermFusedMaxBlocks) {
-    permute_scan_scatter_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(
-        idx, T, hist, static_cast<int>(nb), counts, offsets, perm_src, inv_perm);
-    return launch_check("permute_scan_scatter_kernel launch");
+    return launch_pdl("permute_scan_scatter_kernel launch", permute_scan_scatter_kernel,
+                      dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T,
+                      static_cast<const int32_t*>(hist), static_cast<int>(nb), counts, offsets,
+                      perm_src, inv_perm);
   }
-  permute_scan_kernel<<<1, 1024, 0, s>>>(hist, static_cast<int>(nb), counts, offsets);
-  rc = launch_check("permute_scan_kernel launch");
+  rc = launch_pdl("permute_scan_kernel launch", permute_scan_kernel, dim3(1), dim3(1024), 0, s,
+                  hist, static_cast<int>(nb), counts, offsets);
   if (rc) return rc;
-  permute_scatter_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(idx, T, hist, offsets, perm_src,
-                                                                   inv_perm);
-  return launch_check("permute_scatter_kernel launch");
+  return launch_pdl("permute_scatter_kernel launch", permute_scatter_kernel,
+                    dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T,
+                    static_cast<const int32_t*>(hist), static_cast<const int32_t*>(offsets),
+                    perm_src, inv_perm);
 }
 
 // The GEMMs' tile counters live after the expert offsets (zeroed by the permute
@@ -200,10 +220,10 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
     CUtensorMap tw;
     int rc = make_tmap(&tw, packed, kH, uint64_t(kE) * 2 * kI, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc) return rc;
-    skinny::skinny_gemm_kernel<1><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
-        tw, tw, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-        reinterpret_cast<uint16_t*>(h), sched_words(offsets, 1), g_timeout_ns.load());
-    return launch_check("skinny_gemm_kernel<1> launch");
+    return launch_pdl("skinny_gemm_kernel<1> launch", skinny::skinny_gemm_kernel<1>, dim3(sms),
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw, tw,
+                      reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+                      reinterpret_cast<uint16_t*>(h), sched_words(offsets, 1), g_timeout_ns.load());
   }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -211,13 +231,10 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
   if (rc) return rc;
   const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   auto* hb = reinterpret_cast<uint16_t*>(h);
-  if (T <= kZeroPadMaxT)
-    ffn::ffn_gemm_kernel<1, true><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
-        tb1, tb1, xb, offsets, perm_src, T, hb, sched_words(offsets, 1), g_timeout_ns.load());
-  else
-    ffn::ffn_gemm_kernel<1, false><<<sms, ffn::Cfg<1>::THREADS, ffn::SMEM_BYTES, s>>>(
-        tb1, tb1, xb, offsets, perm_src, T, hb, sched_words(offsets, 1), g_timeout_ns.load());
-  return launch_check("ffn_gemm_kernel<1> launch");
+  return launch_pdl("ffn_gemm_kernel<1> launch",
+                    T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<1, true> : ffn::ffn_gemm_kernel<1, false>,
+                    dim3(sms), dim3(ffn::Cfg<1>::THREADS), ffn::SMEM_BYTES, s, tb1, tb1, xb, offsets,
+                    perm_src, T, hb, sched_words(offsets, 1), g_timeout_ns.load());
 }
 
 int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, int64_t T,
@@ -229,19 +246,21 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                        CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (!rc) rc = make_tmap(&ta2, h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
-    skinny::skinny_gemm_kernel<2><<<sms, skinny::THREADS, skinny::SMEM_BYTES, s>>>(
-        tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y),
-        sched_words(offsets, 2), g_timeout_ns.load());
-    return launch_check("skinny_gemm_kernel<2> launch");
+    return launch_pdl("skinny_gemm_kernel<2> launch", skinny::skinny_gemm_kernel<2>, dim3(sms),
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tb2, ta2,
+                      static_cast<const __nv_bfloat16*>(nullptr), offsets,
+                      static_cast<const int32_t*>(nullptr), T, reinterpret_cast<uint16_t*>(y),
+                      sched_words(offsets, 2), g_timeout_ns.load());
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
-  ffn::ffn_gemm_kernel<2, false><<<sms, ffn::Cfg<2>::THREADS, ffn::SMEM_BYTES, s>>>(
-      tb2, ta2, nullptr, offsets, nullptr, T, reinterpret_cast<uint16_t*>(y),
-        sched_words(offsets, 2), g_timeout_ns.load());
-  return launch_check("ffn_gemm_kernel<2> launch");
+  return launch_pdl("ffn_gemm_kernel<2> launch", ffn::ffn_gemm_kernel<2, false>, dim3(sms),
+                    dim3(ffn::Cfg<2>::THREADS), ffn::SMEM_BYTES, s, tb2, ta2,
+                    static_cast<const __nv_bfloat16*>(nullptr), offsets,
+                    static_cast<const int32_t*>(nullptr), T, reinterpret_cast<uint16_t*>(y),
+                    sched_words(offsets, 2), g_timeout_ns.load());
 }
 
 int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
@@ -254,10 +273,10 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
 
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
                const moe_bf16* residual, moe_bf16* out, cudaStream_t s) {
-  combine_kernel<<<static_cast<unsigned>(T), kCombineThreads, 0, s>>>(
-      reinterpret_cast<const uint16_t*>(y), w, inv, T,
-      reinterpret_cast<const __nv_bfloat16*>(residual), reinterpret_cast<__nv_bfloat16*>(out));
-  return launch_check("combine_kernel launch");
+  return launch_pdl("combine_kernel launch", combine_kernel, dim3(static_cast<unsigned>(T)),
+                    dim3(kCombineThreads), 0, s, reinterpret_cast<const uint16_t*>(y), w, inv, T,
+                    reinterpret_cast<const __nv_bfloat16*>(residual),
+                    reinterpret_cast<__nv_bfloat16*>(out));
 }
 
 // workspace carve-up of moe_layer

@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(1024)
     permute_small_kernel(const int32_t* __restrict__ idx, int T, int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
                          int32_t* __restrict__ inv_perm) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ uint32_t bm[kE][32];
   __shared__ uint32_t pre[kE][32];
   __shared__ int cnt[kE];
@@ -97,6 +99,8 @@ __global__ void __launch_bounds__(1024)
 // (a) per-block expert histogram hist[b][e]
 __global__ void __launch_bounds__(256)
     permute_count_kernel(const int32_t* __restrict__ idx, int64_t T, int32_t* __restrict__ hist) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ uint32_t bm[kE][kPermBlockTokens / 32];
   const int tid = threadIdx.x;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPermBlockTokens;
@@ -126,6 +130,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(1024)
     permute_scan_kernel(int32_t* __restrict__ hist, int nb, int32_t* __restrict__ counts,
                         int32_t* __restrict__ offsets) {
+  griddep_launch_dependents();
+  griddep_wait();
   constexpr int kParts = 1024 / kE;  // 8
   __shared__ int part_sum[kParts][kE];
   __shared__ int cnt[kE];
@@ -167,6 +173,8 @@ __global__ void __launch_bounds__(256)
                                 const int32_t* __restrict__ hist, int nb,
                                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                 int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm) {
+  griddep_launch_dependents();
+  griddep_wait();
   constexpr int W = kPermBlockTokens / 32;
   __shared__ uint32_t bm[kE][W];
   __shared__ int part[2][kE];
@@ -229,6 +237,8 @@ __global__ void __launch_bounds__(256)
     permute_scatter_kernel(const int32_t* __restrict__ idx, int64_t T,
                            const int32_t* __restrict__ before, const int32_t* __restrict__ offsets,
                            int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm) {
+  griddep_launch_dependents();
+  griddep_wait();
   constexpr int W = kPermBlockTokens / 32;
   __shared__ uint32_t bm[kE][W];
   __shared__ int base[kE];

@@ -13,10 +13,18 @@
 // segment shuffles, and each of the 8 selection rounds is a lane-local scan
 // plus three shuffle levels.
 //
-// The selection keys are float64, so that the decisions match a float64
-// evaluation of the same rule.  For s in [0, 1] the bit pattern of the double
-// orders exactly like the value, so a candidate's key is bits(s) + 1 as an
-// unsigned 64-bit integer (0 marks an excluded or already-taken expert).
+// Decisions match a float64 evaluation of the rule bit for bit.  The sigmoid
+// is strictly increasing, so "the two largest s of a group" and "the 8 largest
+// s among kept experts" can be decided on z = logit + bias (exact in float64)
+// instead of on s, with one guard: equal float64 sigmoids must tie exactly as
+// the float64 rule sees them.  For -700 <= z <= 10, z is a sum of two fp32
+// values, so two distinct z differ by far more than sigmoid(z) needs to move
+// by one ulp of s: distinct z give distinct s in the same order.  Outside that
+// range s saturates to 1 or underflows, so there the key is the float64
+// sigmoid itself, in a tier that sorts above (z > 10) or below (z < -700) the
+// middle one.  Only the 2 best scores of each group (the group score) and the
+// 8 chosen experts' weights need a float64 sigmoid: 24 per token, not 136.
+// Keys are unsigned 64-bit integers; 0 marks an excluded or taken expert.
 #pragma once
 #include "common.cuh"
 
@@ -28,10 +36,25 @@ constexpr int kRouteTokensPerBlock = kRouteTokensPerWarp * kRouteWarps;  // 32
 
 __device__ __forceinline__ double sigmoid_f64(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+// Order-preserving 64-bit key of a score given its z (see above); always >= 1.
+__device__ __forceinline__ unsigned long long route_key(double z) {
+  if (z > 10.0) {  // s in (0.99995, 1]: float64 sigmoid bits, above every middle key
+    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(sigmoid_f64(z)));
+    return 0xD000000000000000ull + (b - 0x3FE0000000000000ull);
+  }
+  if (z < -700.0)  // s below 1e-304: float64 sigmoid bits (may be 0), below every middle key
+    return static_cast<unsigned long long>(__double_as_longlong(sigmoid_f64(z))) + 1ull;
+  // middle: z itself, mapped to unsigned order (negative doubles bit-flipped)
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(z));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int64_t T,
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const unsigned FULL = 0xFFFFFFFFu;
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int g = lane & 7;  // group owned by this lane; also its slot in the segment
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock +
@@ -58,21 +81,25 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     }
   }
 
-  // scores, their keys, and the group's two best scores
+  // keys, and the group's two best scores (found on the keys, evaluated in float64)
   unsigned long long key[16];
-  double a1 = -1.0, a2 = -1.0;
+  unsigned long long k1 = 0ull, k2 = 0ull;
+  double z1 = 0.0, z2 = 0.0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const double sv = sigmoid_f64(static_cast<double>(lg[i]) + static_cast<double>(bs[i]));
-    key[i] = static_cast<unsigned long long>(__double_as_longlong(sv)) + 1ull;
-    if (sv > a1) {
-      a2 = a1;
-      a1 = sv;
-    } else if (sv > a2) {
-      a2 = sv;
+    const double z = static_cast<double>(lg[i]) + static_cast<double>(bs[i]);
+    key[i] = route_key(z);
+    if (key[i] > k1) {
+      k2 = k1;
+      z2 = z1;
+      k1 = key[i];
+      z1 = z;
+    } else if (key[i] > k2) {
+      k2 = key[i];
+      z2 = z;
     }
   }
-  const double gscore = a1 + a2;
+  const double gscore = sigmoid_f64(z1) + sigmoid_f64(z2);
 
   // rank of this group among the token's 8 (ties: lower index ranks first)
   int rank = 0;
@@ -114,15 +141,22 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
       if (g * kGS + i == be) key[i] = 0ull;
   }
 
-  // combine weights: sigmoid of the raw logit, renormalised over the 8
-  const double sig =
-      active ? sigmoid_f64(static_cast<double>(__ldg(logits + t * kE + sel))) : 0.0;
-  double tot = sig;
+  // combine weights: sigmoid of the raw logit, renormalised over the 8, as
+  // r / sum r with r = sigmoid(l) / sigmoid(m), m the largest chosen logit;
+  // for m < 0, r = exp(l - m) (1 + exp(m)) / (1 + exp(l)) keeps the ratio
+  // finite when every sigmoid underflows.
+  const double l = active ? static_cast<double>(__ldg(logits + t * kE + sel)) : 0.0;
+  double m = l;
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) m = fmax(m, __shfl_xor_sync(FULL, m, off, 8));
+  const double r = m >= 0.0 ? sigmoid_f64(l) / sigmoid_f64(m)
+                            : exp(l - m) * (1.0 + exp(m)) / (1.0 + exp(l));
+  double tot = r;
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) tot += __shfl_xor_sync(FULL, tot, off, 8);
   if (active) {
     topk_idx[t * kTopK + g] = sel;
-    topk_w[t * kTopK + g] = static_cast<float>(sig / tot);
+    topk_w[t * kTopK + g] = static_cast<float>(r / tot);
   }
 }
 

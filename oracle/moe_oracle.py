@@ -142,10 +142,26 @@ def route(logits: np.ndarray, bias: np.ndarray | None,
     expert_margin = (c_sorted[:, topk - 1] - c_sorted[:, topk]) if topk < n_cand \
         else np.full(T, np.inf)
 
-    sw = sigmoid(lg[rows, idx])
-    w = sw / sw.sum(axis=1, keepdims=True)
+    w = combine_weights(lg[rows, idx])
     return RouteResult(idx.astype(np.int64), w, kept.astype(np.int64),
                        group_margin, expert_margin)
+
+
+def combine_weights(l: np.ndarray) -> np.ndarray:
+    """w_i = sigmoid(l_i) / sum_j sigmoid(l_j) over each row of chosen raw logits.
+
+    Evaluated as r_i / sum_j r_j with r_i = sigmoid(l_i) / sigmoid(m), m the
+    row's largest logit -- the same quantity, but for m < 0 written as
+    exp(l_i - m) (1 + exp(m)) / (1 + exp(l_i)), whose terms stay finite and
+    non-zero when every sigmoid(l_i) underflows (logits below about -745).
+    """
+    l = np.asarray(l, dtype=np.float64)
+    m = l.max(axis=1, keepdims=True)
+    with np.errstate(over="ignore"):
+        direct = sigmoid(l) / sigmoid(m)
+        shifted = np.exp(l - m) * (1.0 + np.exp(m)) / (1.0 + np.exp(l))
+    r = np.where(m >= 0.0, direct, shifted)
+    return r / r.sum(axis=1, keepdims=True)
 
 
 def route_bruteforce(logits_row: np.ndarray, bias_row: np.ndarray | None,

@@ -150,3 +150,19 @@ def test_sigmoid_closed_forms():
     z = np.linspace(-20, 20, 401)
     np.testing.assert_allclose(O.sigmoid(z) + O.sigmoid(-z), 1.0, atol=1e-15)
     assert abs(O.sigmoid(np.array([1.0]))[0] - 1 / (1 + math.e ** -1)) < 1e-16
+
+
+def test_combine_weights_against_plain_formula_and_limit():
+    """The weights equal sigmoid(l)/sum sigmoid(l) wherever that is finite, and
+    when every sigmoid underflows they tend to the softmax of the logits."""
+    rng = np.random.default_rng(21)
+    for scale, shift in ((1.0, 0.0), (5.0, -20.0), (3.0, 15.0), (0.5, -3.0)):
+        l = rng.standard_normal((200, 8)) * scale + shift
+        plain = O.sigmoid(l) / O.sigmoid(l).sum(axis=1, keepdims=True)
+        np.testing.assert_allclose(O.combine_weights(l), plain, rtol=1e-13, atol=1e-16)
+    l = -800.0 - rng.random((20, 8)) * 30.0
+    soft = np.exp(l - l.max(axis=1, keepdims=True))
+    soft /= soft.sum(axis=1, keepdims=True)
+    w = O.combine_weights(l)
+    assert np.all(np.isfinite(w))
+    np.testing.assert_allclose(w, soft, rtol=1e-12, atol=1e-300)
