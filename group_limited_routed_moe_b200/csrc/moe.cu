@@ -531,3 +531,78 @@ extern "C" int moe_selftest_wait_timeout(moe_stream_t stream) {
                                                                              nullptr);
   return launch_check("selftest_wait_kernel launch");
 }
+
+// ---- permutation with library-owned scratch ----------------------------------
+// moe_permute takes its per-block histogram from a caller workspace, which the
+// caller has to allocate.  Some callers cannot allocate when they permute:
+//   - a serving runtime that reserves all of its device memory once at
+//     start-up and hands every byte to a fixed plan, so a later request has
+//     nowhere to come from;
+//   - code that runs inside a memory allocator's own bookkeeping, where a
+//     nested allocation would re-enter the allocator;
+//   - latency-bound loops that must not pay for an allocator miss, or for the
+//     device-wide synchronisation that freeing device memory implies.
+// For those, the histogram lives in a file-scope device array of fixed size
+// that belongs to the library, so the call allocates nothing.
+namespace {
+constexpr int64_t kFixedPermMaxT = 65536;
+constexpr int64_t kFixedPermBlocks = (kFixedPermMaxT + kPermBlockTokens - 1) / kPermBlockTokens;
+// hist[b][e] for up to 512 blocks of 128 tokens: 256 KiB per device.  The count
+// kernel writes every entry that the scan and scatter kernels later read, so no
+// word of it has to start at zero; the only words that must start at zero, the
+// expert-FFN work counters offsets[132..135], are written by the permute
+// kernels themselves.
+static __device__ __align__(256) int32_t g_fixed_perm_hist[kFixedPermBlocks * kE];
+
+int32_t* g_fixed_perm_ptr[kMaxDevices] = {};
+std::mutex g_fixed_perm_mu;
+
+// Device address of the array on the current device, looked up the first time
+// a device asks for it (with that device current) and kept afterwards.
+int fixed_perm_scratch(int32_t** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_fixed_perm_mu);
+  if (g_fixed_perm_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fixed_perm_hist);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fixed permute scratch)");
+    if (p == nullptr || !aligned(p, 256))
+      return fail(MOE_ERR_CUDA, "fixed permute scratch has a bad device address");
+    g_fixed_perm_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_fixed_perm_ptr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" int64_t moe_permute_fixed_scratch_max_tokens(void) { return kFixedPermMaxT; }
+
+extern "C" int moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t T, int32_t* counts,
+                                         int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
+                                         moe_stream_t stream) {
+  if (T < 0 || T > kFixedPermMaxT)
+    return fail(MOE_ERR_INVALID_ARG,
+                "T=%lld outside [0, %lld]: the fixed permute scratch holds %lld blocks of %d "
+                "tokens; use moe_permute with a workspace for more",
+                static_cast<long long>(T), static_cast<long long>(kFixedPermMaxT),
+                static_cast<long long>(kFixedPermBlocks), kPermBlockTokens);
+  REQUIRE(counts && offsets, "null pointer");
+  if (T > 0) REQUIRE(topk_idx && perm_src && inv_perm, "null pointer");
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  int32_t* hist = nullptr;
+  rc = fixed_perm_scratch(&hist);
+  if (rc) return rc;
+  if (permute_ws_bytes(T) > sizeof(g_fixed_perm_hist))
+    return fail(MOE_ERR_WORKSPACE, "fixed permute scratch too small for T=%lld",
+                static_cast<long long>(T));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, kE * sizeof(int32_t), s), "cudaMemsetAsync");
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, kOffsetsLen * sizeof(int32_t), s), "cudaMemsetAsync");
+    return MOE_OK;
+  }
+  return do_permute(topk_idx, T, counts, offsets, perm_src, inv_perm, hist, s);
+}

@@ -59,6 +59,8 @@ _SIGS = {
     "moe_combine": ([_p, _p, _p, _i64, _p, _p, _p], _i32),
     "moe_layer_workspace_bytes": ([_i64], _sz),
     "moe_layer": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_permute_fixed_scratch_max_tokens": ([], _i64),
+    "moe_permute_fixed_scratch": ([_p, _i64, _p, _p, _p, _p, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -155,6 +157,21 @@ def moe_permute(topk_idx: torch.Tensor, counts=None, offsets=None, perm_src=None
                                           _ptr(perm_src), _ptr(inv_perm),
                                           _ptr(workspace) if wsb else None,
                                           workspace.numel() if wsb else 0, _stream(stream)))
+    return counts, offsets[:N_EXPERTS + 1], perm_src[:T * TOPK], inv_perm[:T * TOPK]
+
+
+def moe_permute_fixed_scratch(topk_idx: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
+                              perm_src: torch.Tensor, inv_perm: torch.Tensor, stream=None):
+    """moe_permute with the library's fixed scratch (T <= 65536): every output is
+    caller-provided, and the call allocates no device memory."""
+    T = topk_idx.shape[0]
+    if offsets.numel() < OFFSETS_LEN or counts.numel() < N_EXPERTS:
+        raise ValueError(f"counts needs {N_EXPERTS} and offsets {OFFSETS_LEN} int32 words")
+    if perm_src.numel() < T * TOPK or inv_perm.numel() < T * TOPK:
+        raise ValueError(f"perm_src and inv_perm need {T * TOPK} int32 words")
+    _check("moe_permute_fixed_scratch",
+           lib.moe_permute_fixed_scratch(_ptr(topk_idx), T, _ptr(counts), _ptr(offsets),
+                                         _ptr(perm_src), _ptr(inv_perm), _stream(stream)))
     return counts, offsets[:N_EXPERTS + 1], perm_src[:T * TOPK], inv_perm[:T * TOPK]
 
 

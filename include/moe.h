@@ -212,6 +212,29 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias,
               moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
               void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
+/* ---- permutation without a caller workspace ------------------------------ */
+
+/* The pages describe no such call: it is moe_permute for callers that cannot
+ * allocate device memory at the moment they permute (a runtime whose device
+ * memory is all reserved up front, code running inside an allocator, loops
+ * that must not wait on an allocator).  The per-block histogram that
+ * moe_permute takes from `workspace` lives instead in a fixed array of 256 KiB
+ * per device owned by the library, so the call allocates nothing.
+ *   Limit  : 0 <= T <= moe_permute_fixed_scratch_max_tokens() (65536);
+ *            larger T returns MOE_ERR_INVALID_ARG with nothing launched.
+ *   Outputs: identical, bit for bit, to moe_permute's for the same topk_idx.
+ *   Set-up : the first call on a device (with that device current) looks up
+ *            the array's device address; make that first call before any
+ *            stream capture.
+ *   Races  : one array per device serves every call, so two calls whose
+ *            kernels may overlap (different streams with no ordering between
+ *            them, or several host threads) corrupt each other's result.
+ *            Order them on one stream or with events. */
+int64_t moe_permute_fixed_scratch_max_tokens(void);
+int moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t T, int32_t* counts,
+                              int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
+                              moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,83 @@
+"""moe_permute_fixed_scratch (library-owned scratch, no device allocation)
+against moe_permute, called through the C ABI.
+
+Collected last so that it also runs after every other GPU test in one process;
+it passes on its own in a fresh process as well.  Each case makes two calls in
+a row on different routings: the second must not see anything the first left
+in the shared scratch.  Integer outputs, so the comparison is bit-exact."""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from group_limited_routed_moe_b200 import moe as M
+
+N_EXPERTS, TOPK, OFFSETS_LEN = M.N_EXPERTS, M.TOPK, M.OFFSETS_LEN
+
+
+def _routing(T, seed, hot=0):
+    """[T][8] distinct expert ids per token; `hot` > 0 sends most tokens to the
+    first `hot` experts (a skewed load)."""
+    g = torch.Generator().manual_seed(seed)
+    score = torch.rand((T, N_EXPERTS), generator=g)
+    if hot:
+        score[:, :hot] += 0.9
+    return score.argsort(dim=1, descending=True)[:, :TOPK].to(torch.int32).contiguous()
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _fixed(idx_dev, stream):
+    T = idx_dev.shape[0]
+    dev = idx_dev.device
+    counts = torch.full((N_EXPERTS,), -7, dtype=torch.int32, device=dev)
+    offsets = torch.full((OFFSETS_LEN,), -7, dtype=torch.int32, device=dev)
+    perm = torch.full((max(T * TOPK, 1),), -7, dtype=torch.int32, device=dev)
+    inv = torch.full((max(T * TOPK, 1),), -7, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    rc = M.lib.moe_permute_fixed_scratch(_p(idx_dev), T, _p(counts), _p(offsets), _p(perm),
+                                         _p(inv), ctypes.c_void_p(stream.cuda_stream))
+    assert rc == M.MOE_OK, M.last_error()
+    return counts, offsets, perm[:T * TOPK], inv[:T * TOPK]
+
+
+def _same(got, ref):
+    counts, offsets, perm, inv = got
+    r_counts, r_offsets, r_perm, r_inv = ref
+    assert torch.equal(counts.cpu(), r_counts.cpu())
+    assert torch.equal(offsets[:N_EXPERTS + 1].cpu(), r_offsets.cpu())
+    assert torch.equal(offsets[132:136].cpu(), torch.zeros(4, dtype=torch.int32))
+    assert torch.equal(perm.cpu(), r_perm.cpu())
+    assert torch.equal(inv.cpu(), r_inv.cpu())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,hot", [(0, 0), (700, 0), (8189, 16), (40000, 0), (65536, 4)])
+def test_fixed_scratch_permute_matches_moe_permute(T, hot):
+    assert M.lib.moe_permute_fixed_scratch_max_tokens() == 65536
+    stream = torch.cuda.current_stream()
+    for call, seed in enumerate((11 + T, 12 + T)):  # two calls in a row
+        idx = _routing(T, seed, hot if call == 0 else 0).cuda()
+        ref = M.moe_permute(idx)
+        got = _fixed(idx, stream)
+        torch.cuda.synchronize()
+        _same(got, ref)
+        if T:
+            rows = np.sort(got[2].cpu().numpy())
+            assert np.array_equal(rows, np.arange(T * TOPK))
+    torch.cuda.synchronize()
+    assert M.lib.moe_get_device_status(torch.cuda.current_device()) == M.MOE_OK
+
+
+@pytest.mark.gpu
+def test_fixed_scratch_permute_rejects_too_many_tokens():
+    T = M.lib.moe_permute_fixed_scratch_max_tokens() + 1
+    dummy = torch.zeros(OFFSETS_LEN, dtype=torch.int32, device="cuda")
+    rc = M.lib.moe_permute_fixed_scratch(_p(dummy), T, _p(dummy), _p(dummy), _p(dummy),
+                                         _p(dummy), None)
+    assert rc == M.MOE_ERR_INVALID_ARG
+    assert "65536" in M.last_error()
