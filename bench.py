@@ -11,8 +11,11 @@ Timing: W warm-up steps, then exactly K timed steps between a barrier and a
 device synchronize.  Before every step a 256 MB buffer is overwritten to flush
 the 126 MB L2, and a short device-side sleep lets the host enqueue the whole
 step before the GPU reaches it (both outside the step's events); each step is
-bracketed by CUDA events on the launching stream, with events between the five
-steps for the per-kernel breakdown.  The decode batch is also timed as a
+bracketed by one pair of CUDA events on the launching stream, with nothing
+between its launches (so programmatic dependent launch overlaps each kernel's
+prologue with its predecessor's tail, as in any real run).  The per-kernel
+breakdown, and the dominant kernel's roofline, come from a second pass of K
+steps over the same batch with events between the five steps.  The decode batch is also timed as a
 replayed CUDA graph of the fused moe_layer call.  Multi-GPU (torchrun): every rank runs its own
 independent batch (data-parallel replicas, weak scaling, no data-path
 collective); the reported time is the max over ranks.
@@ -66,10 +69,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+GEMM_SOURCES = ("common.cuh", "expert_ffn.cuh", "expert_ffn_skinny.cuh")
+
+
 def kernel_source_sha():
+    """sha256 (first 16 hex digits) of the sources that define the grouped GEMM
+    kernels, the ones whose ncu traffic the bench line reports."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "group_limited_routed_moe_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in GEMM_SOURCES:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -175,12 +183,22 @@ class LayerRun:
         self.h = torch.empty((n, 512), dtype=torch.float16, device=dev)
         self.y = torch.empty((n, 1536), dtype=torch.float16, device=dev)
         self.out = torch.empty((Tb, 1536), dtype=bf, device=dev)
-        self.launches_per_step = 5 if T <= 1024 else 7
+        # route, permute (1 kernel up to 1024 tokens; count + fused scan/scatter up to
+        # 256 blocks of 128 tokens; count + scan + scatter beyond), gate/up, down, combine
+        nb = (T + 127) // 128
+        self.launches_per_step = 5 if T <= 1024 else (6 if nb <= 256 else 7)
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+        self.write_only_flush = False
         self.stream = torch.cuda.current_stream()
 
     def flush(self, prime=True):
+        # Overwrite 256 MB (evicts every line of the step's inputs from the 126 MB
+        # L2), then read another 256 MB so that the dirty lines of that write are
+        # written back here rather than inside the first kernel of the step.
         self.flush_buf.fill_(1)
+        if not self.write_only_flush:
+            self.read_buf.max()
         if prime:  # ~0.5 ms spin so that the five launches are queued before the GPU gets there
             self.torch.cuda._sleep(1_000_000)
 
@@ -201,23 +219,48 @@ class LayerRun:
         rec(5)
 
     def timed(self, steps, warmup, barrier):
+        """K whole steps, each between one pair of events; returns ms per step."""
         torch = self.torch
         for _ in range(warmup):
             self.flush()
             self.step()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        s = self.stream
         barrier()
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         for k in range(steps):
             self.flush()
-            self.step(evs[k])
+            evs[k][0].record(s)
+            self.step()
+            evs[k][1].record(s)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
         barrier()
-        per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)]
-                        for k in range(steps)])  # ms
-        return per, wall
+        return np.array([e[0].elapsed_time(e[1]) for e in evs]), wall
+
+    def dirty_l2_steps(self, steps, barrier):
+        """Context only: the same K steps after a write-only flush, which leaves
+        about 126 MB of dirty lines in L2 for the step's first kernels to write
+        back.  Mean ms per step."""
+        self.write_only_flush = True
+        try:
+            st, _ = self.timed(steps, 2, barrier)
+        finally:
+            self.write_only_flush = False
+        return float(st.mean())
+
+    def breakdown(self, steps):
+        """K more steps with events between the five launches: ms [K][5]."""
+        torch = self.torch
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        for k in range(steps):
+            self.flush()
+            self.step(evs[k])
+        torch.cuda.synchronize()
+        return np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)]
+                         for k in range(steps)])
 
     def graph_layer_us(self, steps, warmup):
         """The fused moe_layer call captured once in a CUDA graph and replayed."""
@@ -278,12 +321,12 @@ class LayerRun:
         return float(np.mean(times)), x_h.numel() * 2 + lg_h.numel() * 4, out_h.numel() * 2
 
 
-def distinct_experts(tok):
-    import oracle as O  # the oracle's routing fixes which experts a batch touches
-    return int(np.unique(O.route(tok.logits, tok.bias).topk_idx).size)
+def distinct_experts(run):
+    """Experts with at least one row in the timed steps (the permute's counts)."""
+    return int((run.counts > 0).sum().item())
 
 
-def roofline_for(wl, tok, per_ms, peaks, peak_kind):
+def roofline_for(wl, run, per_ms, peaks, peak_kind):
     """Roofline of the dominant kernel (the gate/up GEMM) of one workload."""
     gate_up_ms = float(per_ms[:, 2].mean())
     T = wl.T
@@ -297,22 +340,24 @@ def roofline_for(wl, tok, per_ms, peaks, peak_kind):
                 "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} {key} (burst)",
                 "algorithmic_per_launch": flops,
                 "traffic": profiled_traffic("gate_up", wl.name)}
-    d = distinct_experts(tok)
+    d = distinct_experts(run)
     nbytes = d * GATE_UP_BYTES_PER_EXPERT + T * 1536 * 2 + 8 * T * 512 * 2
     peak = float(peaks["hbm_gbs"])
     achieved = nbytes / (gate_up_ms * 1e-3) / 1e9
-    return {"kernel": "ffn_gemm_kernel<1> (gate/up + SwiGLU)", "bound": "hbm",
+    kernel = ("skinny_gemm_kernel<1> (weights-as-M gate/up + SwiGLU)" if T <= 256
+              else "ffn_gemm_kernel<1> (gate/up + SwiGLU)")
+    return {"kernel": kernel, "bound": "hbm",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
             "algorithmic_per_launch": nbytes, "distinct_experts": d,
             "traffic": profiled_traffic("gate_up", wl.name)}
 
 
-def layer_fractions(wl, tok, per_ms, peaks):
+def layer_fractions(wl, run, step_ms, per_ms, peaks):
     """Whole-layer fractions (context): tokens/s against the HBM bound of the
     distinct experts' weights and against the tensor bound of the useful flops."""
-    layer_s = float(per_ms.sum(axis=1).mean()) * 1e-3
-    d = distinct_experts(tok)
+    layer_s = float(step_ms.mean()) * 1e-3
+    d = distinct_experts(run)
     nbytes = d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + wl.T * (1536 * 4 + 512)
     flops = FLOPS_PER_ROW * 8 * wl.T
     return {"layer_us": round(layer_s * 1e6, 2),
@@ -320,6 +365,7 @@ def layer_fractions(wl, tok, per_ms, peaks):
             "tensor_frac": round(flops / layer_s / 1e12 / float(peaks["bf16_tflops"]), 4),
             "kernel_us": {k: round(float(per_ms[:, i].mean()) * 1e3, 2) for i, k in
                           enumerate(["route", "permute", "gate_up", "down", "combine"])},
+            "kernel_us_sum": round(float(per_ms.sum(axis=1).mean()) * 1e3, 2),
             "distinct_experts": d}
 
 
@@ -371,8 +417,10 @@ def run_ours(args):
     run = LayerRun(wl, dev, packed)
     clk = ClockSampler(local)
     with clk:
-        per, wall = run.timed(args.steps, args.warmup, barrier)
-    step_ms = float(per.sum(axis=1).mean())
+        steps_ms, wall = run.timed(args.steps, args.warmup, barrier)
+    per = run.breakdown(args.steps)
+    dirty_ms = run.dirty_l2_steps(args.steps, barrier)
+    step_ms = float(steps_ms.mean())
     elapsed = torch.tensor([step_ms * args.steps], device=dev, dtype=torch.float64)
     if dist is not None:
         dist.all_reduce(elapsed, op=dist.ReduceOp.MAX)
@@ -388,10 +436,13 @@ def run_ours(args):
         "config": {"workload": wl.name, "T": wl.T, "T_buf": wl.T_buf, "hidden": 1536,
                    "experts": 128, "groups": 8, "keep_groups": 4, "topk": 8, "inter": 512,
                    "parallelism": f"dp{world} (independent batch per GPU)",
-                   "l2": "256 MB buffer overwritten before every step (outside the timed events)",
+                   "l2": ("256 MB buffer overwritten, then another 256 MB buffer read, before "
+                          "every step (outside the timed events): no line of the inputs and no "
+                          "dirty line is left in L2"),
                    "wall_s_timed_region": round(wall, 4)},
-        "roofline": roofline_for(wl, run.tok, per, peaks, peak_kind),
-        "layer": layer_fractions(wl, run.tok, per, peaks),
+        "roofline": roofline_for(wl, run, per, peaks, peak_kind),
+        "layer": dict(layer_fractions(wl, run, steps_ms, per, peaks),
+                      layer_us_after_write_only_flush=round(dirty_ms * 1e3, 2)),
         "e2e": {"value": round(wl.T * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -403,14 +454,17 @@ def run_ours(args):
         run2 = LayerRun(wl2, dev, packed)
         clk2 = ClockSampler(local)
         with clk2:
-            per2, wall2 = run2.timed(max(args.steps, 50), args.warmup, barrier)
+            steps2, wall2 = run2.timed(max(args.steps, 50), args.warmup, barrier)
+        per2 = run2.breakdown(max(args.steps, 50))
+        dirty2 = run2.dirty_l2_steps(max(args.steps, 50), barrier)
         e2e2, h2d2, d2h2 = run2.e2e(20, 3)
         graph_us = run2.graph_layer_us(50, 3)
-        ms2 = float(per2.sum(axis=1).mean())
+        ms2 = float(steps2.mean())
         line["decode_T16"] = {
             "value": round(wl2.T / (ms2 * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms2, 5),
-            "roofline": roofline_for(wl2, run2.tok, per2, peaks, peak_kind),
-            "layer": layer_fractions(wl2, run2.tok, per2, peaks),
+            "roofline": roofline_for(wl2, run2, per2, peaks, peak_kind),
+            "layer": dict(layer_fractions(wl2, run2, steps2, per2, peaks),
+                          layer_us_after_write_only_flush=round(dirty2 * 1e3, 2)),
             "graph_replay": {"layer_us": round(graph_us, 2),
                              "value": round(wl2.T / (graph_us * 1e-6), 1), "unit": "tokens/s"},
             "e2e": {"value": round(wl2.T / (e2e2 * 1e-3), 1), "unit": "tokens/s",

@@ -13,17 +13,17 @@
 // segment shuffles, and each of the 8 selection rounds is a lane-local scan
 // plus three shuffle levels.
 //
-// Decisions match a float64 evaluation of the rule bit for bit.  The sigmoid
-// is strictly increasing, so "the two largest s of a group" and "the 8 largest
-// s among kept experts" can be decided on z = logit + bias (exact in float64)
-// instead of on s, with one guard: equal float64 sigmoids must tie exactly as
-// the float64 rule sees them.  For -700 <= z <= 10, z is a sum of two fp32
-// values, so two distinct z differ by far more than sigmoid(z) needs to move
-// by one ulp of s: distinct z give distinct s in the same order.  Outside that
-// range s saturates to 1 or underflows, so there the key is the float64
-// sigmoid itself, in a tier that sorts above (z > 10) or below (z < -700) the
-// middle one.  Only the 2 best scores of each group (the group score) and the
-// 8 chosen experts' weights need a float64 sigmoid: 24 per token, not 136.
+// The sigmoid is strictly increasing, so "the two largest s of a group" and
+// "the 8 largest s among kept experts" are decided on z = logit + bias (float64)
+// instead of on s: this is the exact order of the scores.  A float64 sigmoid
+// can only add ties, between two z closer than about one ulp of s divided by
+// s'(z); such a pair has a float64 score margin of at most an ulp, the same
+// size as the difference between two float64 exp implementations.  Where s
+// saturates to 1 (z > 10) or underflows (z < -700), many z share one float64
+// s, so there the key is the float64 sigmoid itself, in a tier that sorts
+// above or below the middle one, and those ties are exactly the float64 ones.
+// Only the 2 best scores of each group (the group score) and the 8 chosen
+// experts' weights need a float64 sigmoid: 24 per token, not 136.
 // Keys are unsigned 64-bit integers; 0 marks an excluded or taken expert.
 #pragma once
 #include "common.cuh"
