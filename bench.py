@@ -8,17 +8,20 @@ already resident in HBM.  The headline workload is the long-prompt prefill
 measured the same way and reported beside it.
 
 Timing: W warm-up steps, then exactly K timed steps between a barrier and a
-device synchronize.  Before every step a 256 MB buffer is overwritten to flush
-the 126 MB L2, and a short device-side sleep lets the host enqueue the whole
-step before the GPU reaches it (both outside the step's events); each step is
-bracketed by one pair of CUDA events on the launching stream, with nothing
-between its launches (so programmatic dependent launch overlaps each kernel's
-prologue with its predecessor's tail, as in any real run).  The per-kernel
-breakdown, and the dominant kernel's roofline, come from a second pass of K
-steps over the same batch with events between the five steps.  The decode batch is also timed as a
-replayed CUDA graph of the fused moe_layer call.  Multi-GPU (torchrun): every rank runs its own
-independent batch (data-parallel replicas, weak scaling, no data-path
-collective); the reported time is the max over ranks.
+device synchronize.  A step is one moe_layer call (the public layer API; a
+workspace allocated once).  Before every step a 256 MB buffer is overwritten
+and another 256 MB read, so that L2 holds neither the inputs nor dirty lines,
+and a short device-side sleep lets the host enqueue the whole step before the
+GPU reaches it (all outside the step's events).  Each step is bracketed by one
+pair of CUDA events on the launching stream, with nothing between its
+launches, so programmatic dependent launch overlaps each kernel's prologue
+with its predecessor's tail as in any real run.  The per-kernel breakdown and
+the dominant kernel's roofline come from a second pass of K steps over the
+same batch through the five step calls, with events between them.  The
+decode batch is also timed as a replayed CUDA graph of the moe_layer call.
+Multi-GPU (torchrun): every rank runs its own independent batch (data-parallel
+replicas, weak scaling, no data-path collective); the reported time is the
+max over ranks.
 
 ``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
 """
@@ -183,10 +186,13 @@ class LayerRun:
         self.h = torch.empty((n, 512), dtype=torch.float16, device=dev)
         self.y = torch.empty((n, 1536), dtype=torch.float16, device=dev)
         self.out = torch.empty((Tb, 1536), dtype=bf, device=dev)
-        # route, permute (1 kernel up to 1024 tokens; count + fused scan/scatter up to
-        # 256 blocks of 128 tokens; count + scan + scatter beyond), gate/up, down, combine
+        # moe_layer launches: route + permute (one fused kernel up to 64 tokens;
+        # route and one permute kernel up to 1024; route, count and fused scan/scatter
+        # up to 256 blocks of 128 tokens; route, count, scan, scatter beyond), then
+        # gate/up, down, combine
         nb = (T + 127) // 128
-        self.launches_per_step = 5 if T <= 1024 else (6 if nb <= 256 else 7)
+        self.launches_per_step = 4 if T <= 64 else 5 if T <= 1024 else (6 if nb <= 256 else 7)
+        self.lws = moe.alloc_layer_workspace(T, dev)
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
         self.write_only_flush = False
@@ -202,9 +208,15 @@ class LayerRun:
         if prime:  # ~0.5 ms spin so that the five launches are queued before the GPU gets there
             self.torch.cuda._sleep(1_000_000)
 
-    def step(self, ev=None):
+    def step(self):
+        """One layer through the public layer call (what a user runs)."""
+        self.moe.moe_layer(self.x[:self.T], self.logits[:self.T], self.bias, self.packed,
+                           out=self.out[:self.T], workspace=self.lws, stream=self.stream)
+
+    def step_parts(self, ev):
+        """The same layer through the five step calls, with an event between each."""
         m, T, s = self.moe, self.T, self.stream
-        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        rec = lambda i: ev[i].record(s)  # noqa: E731
         rec(0)
         m.moe_route(self.logits[:T], self.bias, self.idx, self.w, stream=s)
         rec(1)
@@ -257,7 +269,7 @@ class LayerRun:
         torch.cuda.synchronize()
         for k in range(steps):
             self.flush()
-            self.step(evs[k])
+            self.step_parts(evs[k])
         torch.cuda.synchronize()
         return np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)]
                          for k in range(steps)])

@@ -19,6 +19,7 @@
 #include "pack.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "route_permute_small.cuh"
 
 using namespace moe;
 
@@ -206,6 +207,20 @@ int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets,
                     dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T,
                     static_cast<const int32_t*>(hist), static_cast<const int32_t*>(offsets),
                     perm_src, inv_perm);
+}
+
+// Steps 1 and 2 as moe_layer runs them: one fused block for a few tokens.
+int do_route_permute(const float* logits, const float* bias, int64_t T, int32_t* idx, float* w,
+                     int32_t* counts, int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
+                     void* perm_ws, cudaStream_t s) {
+  if (T <= kFusedRoutePermMaxT) {
+    return launch_pdl("route_permute_small_kernel launch", route_permute_small_kernel, dim3(1),
+                      dim3(kFusedRoutePermThreads), 0, s, logits, bias, static_cast<int>(T), idx,
+                      w, counts, offsets, perm_src, inv_perm);
+  }
+  int rc = do_route(logits, bias, T, idx, w, s);
+  if (rc) return rc;
+  return do_permute(idx, T, counts, offsets, perm_src, inv_perm, perm_ws, s);
 }
 
 // The GEMMs' tile counters live after the expert offsets (zeroed by the permute
@@ -496,8 +511,8 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias, const m
   moe_bf16* h = reinterpret_cast<moe_bf16*>(ws + L.h);
   moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
 
-  rc = do_route(logits, bias, T, idx, w, s);
-  if (!rc) rc = do_permute(idx, T, counts, offsets, perm_src, inv_perm, ws + L.perm_ws, s);
+  rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
+                        ws + L.perm_ws, s);
   if (!rc) rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
   if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s);
   return rc;

@@ -66,6 +66,29 @@ def layer0_weights() -> LayerWeights:
     return LayerWeights(0, 0)
 
 
+def extreme_logits():
+    """Router logits at the ends of the sigmoid, with a bias: 8 tokens.
+
+    z in (10, 36): distinct scores close to 1; z > 37: float64 sigmoid == 1.0
+    exactly, so ties are broken by index; z < -745: the sigmoid underflows to 0
+    (ties, and weights that only the shifted ratio keeps finite); mixed with
+    ordinary values."""
+    rng = np.random.default_rng(17)
+    lg = rng.standard_normal((8, 128)).astype(np.float32)
+    lg[0, [5, 9, 70, 71]] = [40.0, 45.0, 50.0, 38.0]              # saturated ties in slot order
+    lg[1, [3, 4, 20, 21, 22]] = [12.0, 12.5, 30.0, 29.0, 35.5]     # large but distinct
+    lg[2, :] = -800.0                                              # everything underflows
+    lg[2, [100, 101]] = [-1.0, 0.5]
+    lg[3, :64] = -760.0
+    lg[3, 64:] = -900.0
+    lg[4, [0, 16, 32, 48, 64, 80, 96, 112]] = 60.0                 # one saturated expert per group
+    lg[5, 16:32] = 11.0                                            # a whole group tied above 10
+    lg[6, ::2] = 37.5
+    lg[7, :] = 0.0
+    b = (0.1 * rng.standard_normal(128)).astype(np.float32)
+    return lg, b
+
+
 def tokens_dev(tok: synth.TokenInputs, T_buf: int | None = None):
     T = tok.x_bits.shape[0]
     T_buf = T_buf or T

@@ -9,7 +9,8 @@ import torch
 
 import oracle as O
 from group_limited_routed_moe_b200 import synth
-from gpu_helpers import DEV, REL_L2_TOL, W_TOL, layer0_weights, to_dev_bf16, to_host_bits, tokens_dev
+from gpu_helpers import (DEV, REL_L2_TOL, W_TOL, extreme_logits, layer0_weights, to_dev_bf16,
+                         to_host_bits, tokens_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -79,20 +80,8 @@ def test_route_extreme_logits():
     """Scores at the ends of the sigmoid: z in (10, 36) (distinct, close to 1),
     z > 37 (float64 sigmoid == 1.0 exactly: ties broken by index), z < -745
     (sigmoid underflows to 0: ties), mixed with ordinary values."""
-    rng = np.random.default_rng(17)
-    lg = rng.standard_normal((8, 128)).astype(np.float32)
-    lg[0, [5, 9, 70, 71]] = [40.0, 45.0, 50.0, 38.0]              # saturated ties in slot order
-    lg[1, [3, 4, 20, 21, 22]] = [12.0, 12.5, 30.0, 29.0, 35.5]     # large but distinct
-    lg[2, :] = -800.0                                              # everything underflows
-    lg[2, [100, 101]] = [-1.0, 0.5]
-    lg[3, :64] = -760.0
-    lg[3, 64:] = -900.0
-    lg[4, [0, 16, 32, 48, 64, 80, 96, 112]] = 60.0                 # one saturated expert per group
-    lg[5, 16:32] = 11.0                                            # a whole group tied above 10
-    lg[6, ::2] = 37.5
-    lg[7, :] = 0.0
+    lg, b = extreme_logits()
     _route_check(lg, None, exact_ties=True)
-    b = (0.1 * rng.standard_normal(128)).astype(np.float32)
     _route_check(lg, b, exact_ties=True)
 
 
