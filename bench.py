@@ -188,10 +188,15 @@ class LayerRun:
         self.out = torch.empty((Tb, 1536), dtype=bf, device=dev)
         # moe_layer launches: route + permute (one fused kernel up to 64 tokens;
         # route and one permute kernel up to 1024; route, count and fused scan/scatter
-        # up to 256 blocks of 128 tokens; route, count, scan, scatter beyond), then
-        # gate/up, down, combine
+        # up to 256 blocks of 128 tokens; route, count, scan, scatter beyond), the
+        # expert FFN (one launch up to 256 tokens, gate/up and down above), combine
         nb = (T + 127) // 128
-        self.launches_per_step = 4 if T <= 64 else 5 if T <= 1024 else (6 if nb <= 256 else 7)
+        n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
+        self.fused_ffn = T <= 256
+        self.launches_per_step = n_rp + (1 if self.fused_ffn else 2) + 1
+        # the breakdown pass times the same kernels the layer call runs
+        self.part_names = (["route", "permute", "expert_ffn", "combine"] if self.fused_ffn
+                           else ["route", "permute", "gate_up", "down", "combine"])
         self.lws = moe.alloc_layer_workspace(T, dev)
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
@@ -214,21 +219,28 @@ class LayerRun:
                            out=self.out[:self.T], workspace=self.lws, stream=self.stream)
 
     def step_parts(self, ev):
-        """The same layer through the five step calls, with an event between each."""
+        """The same layer through the step calls, with an event between each."""
         m, T, s = self.moe, self.T, self.stream
-        rec = lambda i: ev[i].record(s)  # noqa: E731
-        rec(0)
+        k = iter(range(len(ev)))
+        rec = lambda: ev[next(k)].record(s)  # noqa: E731
+        rec()
         m.moe_route(self.logits[:T], self.bias, self.idx, self.w, stream=s)
-        rec(1)
+        rec()
         m.moe_permute(self.idx, self.counts, self.offsets, self.perm_src, self.inv_perm,
                       self.pws, stream=s)
-        rec(2)
-        m.moe_expert_gate_up(self.x[:T], self.packed, self.offsets, self.perm_src, self.h, stream=s)
-        rec(3)
-        m.moe_expert_down(self.h, self.packed, self.offsets, self.y, stream=s)
-        rec(4)
+        rec()
+        if self.fused_ffn:
+            m.moe_expert_ffn(self.x[:T], self.packed, self.offsets, self.perm_src, self.h, self.y,
+                             stream=s)
+            rec()
+        else:
+            m.moe_expert_gate_up(self.x[:T], self.packed, self.offsets, self.perm_src, self.h,
+                                 stream=s)
+            rec()
+            m.moe_expert_down(self.h, self.packed, self.offsets, self.y, stream=s)
+            rec()
         m.moe_combine(self.y, self.w, self.inv_perm, out=self.out[:T], stream=s)
-        rec(5)
+        rec()
 
     def timed(self, steps, warmup, barrier):
         """K whole steps, each between one pair of events; returns ms per step."""
@@ -263,15 +275,16 @@ class LayerRun:
         return float(st.mean())
 
     def breakdown(self, steps):
-        """K more steps with events between the five launches: ms [K][5]."""
+        """K more steps with events between the step calls: ms [K][parts]."""
         torch = self.torch
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        n = len(self.part_names)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
         torch.cuda.synchronize()
         for k in range(steps):
             self.flush()
             self.step_parts(evs[k])
         torch.cuda.synchronize()
-        return np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)]
+        return np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n)]
                          for k in range(steps)])
 
     def graph_layer_us(self, steps, warmup):
@@ -339,9 +352,22 @@ def distinct_experts(run):
 
 
 def roofline_for(wl, run, per_ms, peaks, peak_kind):
-    """Roofline of the dominant kernel (the gate/up GEMM) of one workload."""
-    gate_up_ms = float(per_ms[:, 2].mean())
+    """Roofline of the dominant kernel of one workload: the gate/up GEMM, or for
+    T <= 256 the single launch that runs both expert GEMMs."""
     T = wl.T
+    if run.fused_ffn:
+        ffn_ms = float(per_ms[:, run.part_names.index("expert_ffn")].mean())
+        d = distinct_experts(run)
+        nbytes = (d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * 1536 * 2
+                  + 8 * T * 1536 * 2)
+        peak = float(peaks["hbm_gbs"])
+        achieved = nbytes / (ffn_ms * 1e-3) / 1e9
+        return {"kernel": "skinny_gemm_kernel<3> (gate/up + SwiGLU + down in one launch)",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_per_launch": nbytes, "distinct_experts": d,
+                "traffic": profiled_traffic("expert_ffn", wl.name)}
+    gate_up_ms = float(per_ms[:, run.part_names.index("gate_up")].mean())
     if T >= 2048:
         flops = GATE_UP_FLOPS_PER_ROW * 8 * T
         key = "bf16_tflops"
@@ -356,8 +382,7 @@ def roofline_for(wl, run, per_ms, peaks, peak_kind):
     nbytes = d * GATE_UP_BYTES_PER_EXPERT + T * 1536 * 2 + 8 * T * 512 * 2
     peak = float(peaks["hbm_gbs"])
     achieved = nbytes / (gate_up_ms * 1e-3) / 1e9
-    kernel = ("skinny_gemm_kernel<1> (weights-as-M gate/up + SwiGLU)" if T <= 256
-              else "ffn_gemm_kernel<1> (gate/up + SwiGLU)")
+    kernel = "ffn_gemm_kernel<1> (gate/up + SwiGLU)"
     return {"kernel": kernel, "bound": "hbm",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
@@ -376,7 +401,7 @@ def layer_fractions(wl, run, step_ms, per_ms, peaks):
             "hbm_frac": round(nbytes / layer_s / 1e9 / float(peaks["hbm_gbs"]), 4),
             "tensor_frac": round(flops / layer_s / 1e12 / float(peaks["bf16_tflops"]), 4),
             "kernel_us": {k: round(float(per_ms[:, i].mean()) * 1e3, 2) for i, k in
-                          enumerate(["route", "permute", "gate_up", "down", "combine"])},
+                          enumerate(run.part_names)},
             "kernel_us_sum": round(float(per_ms.sum(axis=1).mean()) * 1e3, 2),
             "distinct_experts": d}
 

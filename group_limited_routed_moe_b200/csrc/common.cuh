@@ -35,6 +35,7 @@ enum StatusSite : unsigned {
   kSiteFfnTmemEmpty = 19,
   kSiteFfnDrain = 20,
   kSiteTileQueue = 21,
+  kSiteFfnDone = 22,  // a down tile waiting for its expert's gate/up tiles
   kSiteSelftest = 30,
 };
 
@@ -287,12 +288,13 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 // from HBM rather than L2, stalls) takes fewer of them.  Inside a CTA one
 // thread grabs tile ids and publishes them through a small shared-memory queue
 // that every warp role reads in the same order.  The counter words live after
-// the expert offsets (see kSchedWord): moe_permute zeroes them, and the last
-// CTA of every GEMM launch sets them back to zero.
+// the expert offsets (see kSchedWord), followed by 128 per-expert completion
+// counters of the single-launch expert FFN: moe_permute zeroes them all, and
+// the last CTA of every GEMM launch sets the ones it used back to zero.
 
 constexpr int kTileQ = 4;          // queue slots
 constexpr int kSchedWord = 132;    // offsets[132..135]: scheduler words (2 per GEMM phase)
-constexpr int kOffsetsLen = 136;   // length of the offsets array
+constexpr int kOffsetsLen = 264;   // length of the offsets array ([136..263]: expert counters)
 
 struct TileQueue {
   int tile[kTileQ];
@@ -333,13 +335,15 @@ __device__ __forceinline__ int tileq_pop(TileQueue* q, int n, bool release,
   return tile;
 }
 
-// End of a launch: the last CTA to finish zeroes the two counter words.
-__device__ __forceinline__ void tileq_retire(int* sched) {
+// End of a launch: the last CTA to finish zeroes the two counter words (and
+// the n_extra words at `extra`, if any).
+__device__ __forceinline__ void tileq_retire(int* sched, int* extra = nullptr, int n_extra = 0) {
   __threadfence();
-  const int done = atomicAdd(sched + 1, 1);
-  if (done == static_cast<int>(gridDim.x) - 1) {
+  const int fin = atomicAdd(sched + 1, 1);
+  if (fin == static_cast<int>(gridDim.x) - 1) {
     atomicExch(sched, 0);
     atomicExch(sched + 1, 0);
+    for (int i = 0; i < n_extra; ++i) atomicExch(extra + i, 0);
   }
 }
 

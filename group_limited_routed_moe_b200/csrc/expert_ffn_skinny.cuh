@@ -17,6 +17,18 @@
 // Tiles are (expert, 128-row weight block, 32-token chunk), chunk fastest, so
 // the CTAs that share a weight block run together and read it from L2 once.
 //
+// One launch can run both phases (MODE 3, used by moe_layer and
+// moe_expert_ffn): all gate/up tiles come first in the tile order, then the
+// down tiles.  A down tile of expert e needs all of e's h rows, so the TMA
+// producer waits (bounded) until a per-expert counter says every gate/up tile
+// of e has stored its h values; the gate/up epilogue makes its stores visible
+// to the TMA (async proxy) and then increments the counter with release
+// semantics.  Each CTA receives tile ids in increasing order, so the gate/up
+// tiles a waiting producer depends on were all handed out before, to CTAs that
+// run them without waiting: the wait always ends.  SMs that finish their last
+// gate/up tile go straight on to down tiles of experts that are ready instead
+// of idling until the slowest gate/up tile ends and a second launch ramps up.
+//
 // Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31), 4 token gather (phase 1:
 // cp.async of x rows by perm_src, barrier-tracked; padding rows kept at zero),
 // 5 TMA producer, 6 MMA issuer.  Accumulators: 2 x 32 TMEM columns.  Every
@@ -42,26 +54,16 @@ constexpr int XCHG_BYTES = 64 * XSTRIDE * 4;
 constexpr int THREADS = 224;
 constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;
 
-template <int PHASE>
-struct SCfg;
-template <>
-struct SCfg<1> {
-  static constexpr int KDIM = kH;
-  static constexpr int FBLK = 8;  // 4 pairs x 2 halves of 64 gate + 64 up rows
-  static constexpr int OUT_COLS = kI;
-  static constexpr int FULL_COUNT = 1 + 32;  // TMA arrive + 32 gather lanes
-  static constexpr uint32_t TX = A_BYTES;
-  static constexpr uint32_t IDESC = idesc_f32acc(BMW, BNT, kFmtBF16);
-};
-template <>
-struct SCfg<2> {
-  static constexpr int KDIM = kI;
-  static constexpr int FBLK = kH / BMW;  // 12
-  static constexpr int OUT_COLS = kH;
-  static constexpr int FULL_COUNT = 1;
-  static constexpr uint32_t TX = A_BYTES + B_BYTES;
-  static constexpr uint32_t IDESC = idesc_f32acc(BMW, BNT, kFmtF16);
-};
+// Per-phase constants.  Phase 1: 8 weight blocks per 32-token chunk (4 pairs
+// x 2 halves of 64 gate + 64 up rows), K = 1536; phase 2: 12 blocks, K = 512.
+__host__ __device__ constexpr int fblk(int phase) { return phase == 1 ? 8 : kH / BMW; }
+__host__ __device__ constexpr int kblocks(int phase) { return (phase == 1 ? kH : kI) / BK; }
+constexpr uint32_t kIdesc1 = idesc_f32acc(BMW, BNT, kFmtBF16);
+constexpr uint32_t kIdesc2 = idesc_f32acc(BMW, BNT, kFmtF16);
+// Counter increments a gate/up tile makes when its h values are stored (one per
+// storing warp): a down tile of expert e waits for kDoneStep * 8 * chunks(e).
+constexpr int kDoneStep = 2;
+constexpr int kDoneWord = kSchedWord + 4;  // offsets[136 .. 263]: per-expert done counters
 
 struct Tail {
   uint64_t full[STAGES];
@@ -75,36 +77,73 @@ struct Tail {
   uint32_t tmem_base;
   int abort_flag;
   int wsum[4];
-  int tile_start[kE + 1];
+  int cstart[kE + 1];  // exclusive prefix of the experts' 32-token chunk counts
   int cnt[kE];
   int off[kE];
 };
 constexpr int TAIL_BYTES = (static_cast<int>(sizeof(Tail)) + 127) / 128 * 128;
 constexpr int SMEM_BYTES = TILE_BYTES + TAIL_BYTES + XCHG_BYTES + 1024;
 
-__device__ __forceinline__ void decode_tile(const Tail* S, int tile, int FBLK, int& e, int& f,
+// Tile u of a phase whose experts have FBLK weight blocks per chunk.
+__device__ __forceinline__ void decode_tile(const Tail* S, int u, int FBLK, int& e, int& f,
                                             int& c) {
-  int lo = 0, hi = kE - 1;
+  int lo = 0, hi = kE - 1;  // largest e with cstart[e] * FBLK <= u
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (S->tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    if (S->cstart[mid] * FBLK <= u) lo = mid; else hi = mid - 1;
   }
   e = lo;
-  const int rem = tile - S->tile_start[e];
+  const int rem = u - S->cstart[e] * FBLK;
   const int nch = (S->cnt[e] + BNT - 1) / BNT;
   f = rem / nch;
   c = rem - f * nch;
 }
 
-template <int PHASE>
+// Phase and coordinates of tile id `tile` of a launch in mode MODE (1: gate/up,
+// 2: down, 3: both, gate/up tile ids first).
+struct TileInfo {
+  int phase, e, f, c;
+};
+template <int MODE>
+__device__ __forceinline__ TileInfo tile_info(const Tail* S, int tile, int total1) {
+  TileInfo t;
+  t.phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
+  const int u = (MODE == 3 && t.phase == 2) ? tile - total1 : tile;
+  decode_tile(S, u, fblk(t.phase), t.e, t.f, t.c);
+  return t;
+}
+
+// Waits until *counter >= need (acquire), bounded in time; then orders the
+// async proxy (TMA) after it.
+__device__ __forceinline__ bool wait_count(const int* counter, int need, volatile int* abort_flag,
+                                           uint64_t timeout_ns, unsigned site) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 0;; ++n) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= need) break;
+    if (*abort_flag) return false;
+    if ((n & 15u) == 15u && global_timer_ns() - t0 > timeout_ns) {
+      record_status(site);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
-    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                       const __grid_constant__ CUtensorMap tmap_h,
+    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w1,  // gate/up weights (phase 1)
+                       const __grid_constant__ CUtensorMap tmap_w2,  // down weights (phase 2)
+                       const __grid_constant__ CUtensorMap tmap_h,   // h rows (phase 2)
                        const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                        const int32_t* __restrict__ perm_src, int64_t T,
-                       uint16_t* __restrict__ out, int* __restrict__ sched, uint64_t timeout_ns) {
-  using C = SCfg<PHASE>;
-  constexpr int KB = C::KDIM / BK;
+                       uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
+                       int* __restrict__ sched, int* __restrict__ done, uint64_t timeout_ns) {
+  constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -123,7 +162,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&fullb[s], C::FULL_COUNT);
+      mbar_init(&fullb[s], HAS1 ? 1 + 32 : 1);  // TMA arrive (+ 32 gather lanes)
       mbar_init(&emptyb[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -133,18 +172,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&S->xfull, 64);
     mbar_init(&S->xempty, 64);
     mbar_init(&S->drain, 1);
-    tileq_init(&S->tq, (PHASE == 1 ? 1 : 0) + 1 + 4);  // gather warp, MMA thread, epilogue warps
+    tileq_init(&S->tq, (HAS1 ? 1 : 0) + 1 + 4);  // gather warp, MMA thread, epilogue warps
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
   if (warp == TMA_WARP && lane == 0) {
-    tma_prefetch_desc(&tmap_w);
-    if (PHASE == 2) tma_prefetch_desc(&tmap_h);
+    if (HAS1) tma_prefetch_desc(&tmap_w1);
+    if (HAS2) {
+      tma_prefetch_desc(&tmap_w2);
+      tma_prefetch_desc(&tmap_h);
+    }
   }
 
-  griddep_wait();  // offsets, perm_src and (phase 2) h come from the preceding kernels
-  int my_tiles = 0;
+  griddep_wait();  // offsets, perm_src and (down alone) h come from the preceding kernels
+  int my_chunks = 0;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;
     const int o0 = offsets[e], o1 = offsets[e + 1];
@@ -155,9 +197,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     S->cnt[e] = c;
     S->off[e] = o0;
-    my_tiles = ((c + BNT - 1) / BNT) * C::FBLK;
+    my_chunks = (c + BNT - 1) / BNT;
   }
-  int incl = my_tiles;
+  int incl = my_chunks;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -169,17 +211,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x < kE) {
     int base = 0;
     for (int w = 0; w < warp; ++w) base += S->wsum[w];
-    S->tile_start[threadIdx.x] = base + incl - my_tiles;
-    if (threadIdx.x == kE - 1) S->tile_start[kE] = base + incl;
+    S->cstart[threadIdx.x] = base + incl - my_chunks;
+    if (threadIdx.x == kE - 1) S->cstart[kE] = base + incl;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem_base = S->tmem_base;
-  const int total_tiles = S->tile_start[kE];
+  const int nchunks = S->cstart[kE];
+  const int total1 = HAS1 ? nchunks * fblk(1) : 0;
+  const int total_tiles = total1 + (HAS2 ? nchunks * fblk(2) : 0);
 
   if (warp == TMA_WARP) {
+    // ------------------------------------------------ TMA producer
     if (lane == 0) {
       int it = 0, n = 0;
       bool ok = true;
@@ -192,10 +237,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (pub < 0) break;
         const int next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);
-        int e, f, c;
-        decode_tile(S, tile, C::FBLK, e, f, c);
+        const TileInfo ti = tile_info<MODE>(S, tile, total1);
+        const int e = ti.e, f = ti.f, c = ti.c;
+        if (MODE == 3 && ti.phase == 2) {
+          // every gate/up tile of expert e has stored its h values
+          const int need = kDoneStep * fblk(1) * ((S->cnt[e] + BNT - 1) / BNT);
+          if (!wait_count(done + e, need, abort_flag, timeout_ns, kSiteFfnDone)) {
+            ok = false;
+            break;
+          }
+        }
         int wrow0, wrow1 = 0;
-        if (PHASE == 1) {  // pair j = f/2, half = f%2: gate rows then the matching up rows
+        if (ti.phase == 1) {  // pair j = f/2, half = f%2: gate rows then the matching up rows
           const int j = f >> 1, half = f & 1;
           wrow0 = e * 2 * kI + 256 * j + 64 * half;
           wrow1 = wrow0 + 128;
@@ -203,6 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           wrow0 = e * kH + f * BMW;
         }
         const int hrow = S->off[e] + c * BNT;
+        const int KB = kblocks(ti.phase);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -210,12 +264,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&fullb[s], C::TX);
-          if (PHASE == 1) {
-            tma_load_2d(smem_u32(sA(s)), &tmap_w, kb * BK, wrow0, &fullb[s]);
-            tma_load_2d(smem_u32(sA(s)) + A_BYTES / 2, &tmap_w, kb * BK, wrow1, &fullb[s]);
+          if (ti.phase == 1) {
+            mbar_arrive_expect_tx(&fullb[s], A_BYTES);
+            tma_load_2d(smem_u32(sA(s)), &tmap_w1, kb * BK, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)) + A_BYTES / 2, &tmap_w1, kb * BK, wrow1, &fullb[s]);
           } else {
-            tma_load_2d(smem_u32(sA(s)), &tmap_w, kb * BK, wrow0, &fullb[s]);
+            mbar_arrive_expect_tx(&fullb[s], A_BYTES + B_BYTES);
+            tma_load_2d(smem_u32(sA(s)), &tmap_w2, kb * BK, wrow0, &fullb[s]);
             tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * BK, hrow, &fullb[s]);
           }
         }
@@ -227,6 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == MMA_WARP) {
+    // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, tc = 0;
       bool ok = true;
@@ -236,6 +292,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = tile == -1;
           break;
         }
+        const int phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
+        const int KB = kblocks(phase);
+        const uint32_t idesc = phase == 1 ? kIdesc1 : kIdesc2;
         const int a = tc & 1;
         const uint32_t use = tc >> 1;
         if (!mbar_wait(&S->tempty[a], (use & 1) ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) {
@@ -256,7 +315,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t bdesc = smem_desc_k128(smem_u32(sB(s)));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&emptyb[s]);
         }
         if (ok) umma_commit(&S->tfull[a]);
@@ -264,7 +323,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma_commit(&S->drain);
       mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
     }
-  } else if (PHASE == 1 && warp == GATHER_WARP) {
+  } else if (HAS1 && warp == GATHER_WARP) {
+    // ------------------------------------------------ token gather (phase 1)
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
     uint32_t dirty = (1u << STAGES) - 1;  // stage slots whose row `lane` may hold non-zero data
     int it = 0, n = 0;
@@ -272,16 +332,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     while (ok) {
       const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      int e, f, c;
-      decode_tile(S, tile, C::FBLK, e, f, c);
-      const int row_in_e = c * BNT + lane;
+      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      if (ti.phase == 2) {
+        // down tile: the TMA brings the h rows; only keep the stage barriers' count
+        for (int kb = 0; kb < kblocks(2); ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive(&fullb[s]);
+        }
+        continue;
+      }
+      const int row_in_e = ti.c * BNT + lane;
       const char* src = nullptr;
-      if (row_in_e < S->cnt[e]) {
-        const int p = perm_src[S->off[e] + row_in_e];
+      if (row_in_e < S->cnt[ti.e]) {
+        const int p = perm_src[S->off[ti.e] + row_in_e];
         if (p >= 0 && static_cast<int64_t>(p) < nrows)
           src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
       }
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = 0; kb < kblocks(1); ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
@@ -307,11 +379,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue
     bool range_bad = false;
+    int n1 = 0;  // gate/up tiles seen so far (exchange-tile phase)
     for (int tc = 0;; ++tc) {
       const int tile = tileq_pop(&S->tq, tc, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      int e, f, c;
-      decode_tile(S, tile, C::FBLK, e, f, c);
+      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      const int e = ti.e, f = ti.f, c = ti.c;
       const int a = tc & 1;
       const uint32_t use = tc >> 1;
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
@@ -323,8 +396,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&S->tempty[a]);  // accumulator copied out: MMA may reuse it
       const int ntok = min(BNT, S->cnt[e] - c * BNT);
       const int64_t row0 = static_cast<int64_t>(S->off[e]) + c * BNT;
-      if (PHASE == 1) {
-        const uint32_t xph = static_cast<uint32_t>(tc) & 1;
+      if (ti.phase == 1) {
+        const uint32_t xph = static_cast<uint32_t>(n1++) & 1;
         if (warp >= 2) {  // up half: hand the values to the gate half
           if (!mbar_wait(&S->xempty, xph ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) break;
           float* xr = xchg + ((warp - 2) * 32 + lane) * XSTRIDE;
@@ -345,9 +418,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (t < ntok) {
               const float hv = ffn::silu_mul(__uint_as_float(v[t]), up[t]);
               range_bad |= !(fabsf(hv) <= 65504.f);
-              st_global_b16(out + (row0 + t) * C::OUT_COLS + col,
-                            __half_as_ushort(__float2half_rn(hv)));
+              st_global_b16(h_out + (row0 + t) * kI + col, __half_as_ushort(__float2half_rn(hv)));
             }
+          }
+          if (MODE == 3) {
+            // publish: this warp's h values of the tile are stored (TMA reads them later)
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(done + e, 1);
           }
         }
       } else {
@@ -357,7 +436,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (t < ntok) {
             const float yv = __uint_as_float(v[t]);
             range_bad |= !(fabsf(yv) <= 65504.f);
-            st_global_b16(out + (row0 + t) * C::OUT_COLS + col, __half_as_ushort(__float2half_rn(yv)));
+            st_global_b16(y_out + (row0 + t) * kH + col, __half_as_ushort(__float2half_rn(yv)));
           }
         }
       }
@@ -367,7 +446,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) tileq_retire(sched);
+  if (threadIdx.x == 0) tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

@@ -25,7 +25,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 1024;  // gate/up keeps padding rows of A zeroed up to this T
@@ -95,6 +95,9 @@ int device_setup(int* dev_out, int* sms_out) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       if (g_encode == nullptr) {
@@ -236,9 +239,10 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
     int rc = make_tmap(&tw, packed, kH, uint64_t(kE) * 2 * kI, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc) return rc;
     return launch_pdl("skinny_gemm_kernel<1> launch", skinny::skinny_gemm_kernel<1>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw, tw,
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw, tw, tw,
                       reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-                      reinterpret_cast<uint16_t*>(h), sched_words(offsets, 1), g_timeout_ns.load());
+                      reinterpret_cast<uint16_t*>(h), static_cast<uint16_t*>(nullptr),
+                      sched_words(offsets, 1), static_cast<int*>(nullptr), g_timeout_ns.load());
   }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -262,10 +266,11 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
     if (!rc) rc = make_tmap(&ta2, h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
     return launch_pdl("skinny_gemm_kernel<2> launch", skinny::skinny_gemm_kernel<2>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tb2, ta2,
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tb2, tb2, ta2,
                       static_cast<const __nv_bfloat16*>(nullptr), offsets,
-                      static_cast<const int32_t*>(nullptr), T, reinterpret_cast<uint16_t*>(y),
-                      sched_words(offsets, 2), g_timeout_ns.load());
+                      static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
+                      reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
+                      static_cast<int*>(nullptr), g_timeout_ns.load());
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -281,6 +286,22 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
 int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                   const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, int sms,
                   cudaStream_t s) {
+  if (T <= kSkinnyMaxT) {  // both GEMMs in one launch (see expert_ffn_skinny.cuh)
+    CUtensorMap tw1, tw2, th;
+    int rc = make_tmap(&tw1, packed, kH, uint64_t(kE) * 2 * kI, 64,
+                       CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    if (!rc) rc = make_tmap(&tw2, packed + kPackGuElems, kI, uint64_t(kE) * kH, skinny::BMW,
+                            CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
+                            CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+    return launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw1, tw2, th,
+                      reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+                      reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
+                      sched_words(offsets, 1), const_cast<int*>(offsets) + skinny::kDoneWord,
+                      g_timeout_ns.load());
+  }
   int rc = do_gate_up(x, packed, offsets, perm_src, T, h, sms, s);
   if (rc) return rc;
   return do_down(h, packed, offsets, T, y, sms, s);
@@ -565,7 +586,7 @@ constexpr int64_t kFixedPermBlocks = (kFixedPermMaxT + kPermBlockTokens - 1) / k
 // hist[b][e] for up to 512 blocks of 128 tokens: 256 KiB per device.  The count
 // kernel writes every entry that the scan and scatter kernels later read, so no
 // word of it has to start at zero; the only words that must start at zero, the
-// expert-FFN work counters offsets[132..135], are written by the permute
+// expert-FFN work counters offsets[132..263], are written by the permute
 // kernels themselves.
 static __device__ __align__(256) int32_t g_fixed_perm_hist[kFixedPermBlocks * kE];
 

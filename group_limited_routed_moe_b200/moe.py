@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 HIDDEN, INTER, N_EXPERTS, N_GROUPS, KEEP_GROUPS, TOPK = 1536, 512, 128, 8, 4, 8
-OFFSETS_LEN = 136  # 129 expert offsets + scratch words used by the expert-FFN kernels
+OFFSETS_LEN = 264  # 129 expert offsets + scratch words used by the expert-FFN kernels
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
     MOE_ERR_UNSUPPORTED, MOE_ERR_RANGE = range(7)
 

@@ -56,7 +56,7 @@ enum {
   MOE_GROUP_SIZE = 16,   /* experts per group */
   MOE_KEEP_GROUPS = 4,   /* groups kept per token */
   MOE_TOPK = 8,          /* experts used per token */
-  MOE_OFFSETS_LEN = 136  /* int32 words of the offsets array (129 offsets + scratch) */
+  MOE_OFFSETS_LEN = 264  /* int32 words of the offsets array (129 offsets + scratch) */
 };
 
 typedef enum moe_status {
@@ -147,7 +147,7 @@ size_t moe_permute_workspace_bytes(int64_t T);
  *   topk_idx : [T][8] int32 (from moe_route)
  *   counts   : [128] int32 (out)  rows per expert
  *   offsets  : [MOE_OFFSETS_LEN] int32 (out): [0..128] exclusive prefix of counts,
- *              offsets[128] = 8T; [132..135] zeroed work counters that the
+ *              offsets[128] = 8T; [132..263] zeroed work counters that the
  *              expert-FFN kernels use and leave at zero (words 129..131 unused)
  *   perm_src : [8T] int32 (out)   permuted row r holds item t*8+slot; rows are
  *                                 expert-major, token-ascending inside an expert
@@ -164,11 +164,13 @@ int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts,
  * for every permuted row r = offsets[e] + i, i < counts[e], t = perm_src[r]/8.
  *   x        : [T][1536] bf16, 128-byte aligned
  *   packed_w : from moe_pack_weights
- *   offsets, perm_src : from moe_permute (the work counters in offsets[132..135]
+ *   offsets, perm_src : from moe_permute (the work counters in offsets[132..263]
  *                       are updated during the call and are zero again after it;
  *                       two calls sharing one offsets array must not overlap)
  *   h        : [8T][512] fp16 workspace (out), 128-byte aligned
- *   y_perm   : [8T][1536] fp16 (out) */
+ *   y_perm   : [8T][1536] fp16 (out)
+ * For T <= 256 both GEMMs run in one persistent launch (a down tile starts as
+ * soon as its expert's gate/up tiles have stored h); above, two launches. */
 int moe_expert_ffn(const moe_bf16* x, const moe_bf16* packed_w,
                    const int32_t* offsets, const int32_t* perm_src, int64_t T,
                    moe_f16* h, moe_f16* y_perm, moe_stream_t stream);

@@ -13,7 +13,7 @@ def test_exports_every_declared_symbol():
     assert len(names) >= 15
     missing = [n for n in names if not hasattr(moe.lib, n)]
     assert missing == []
-    assert moe.lib.moe_abi_version() == 1
+    assert moe.lib.moe_abi_version() == 2
 
 
 def test_sizes():

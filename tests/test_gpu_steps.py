@@ -199,3 +199,33 @@ def test_generator_device_bytes_equal_host_bytes():
     for which, t in ((synth.W_GATE, W.wg), (synth.W_DOWN, W.wd)):
         host = synth.weight_bits_np(0, 0, which, experts=[0, 77, 127])
         assert np.array_equal(to_host_bits(t[[0, 77, 127]]), host)
+
+
+@pytest.mark.parametrize("T,seed,forced", [(1, 31, None), (16, 32, None), (77, 33, None),
+                                           (200, 34, [0, 1, 16, 17, 32, 33, 48, 49]),
+                                           (256, 35, None)])
+def test_expert_ffn_single_launch_equals_two_launches(T, seed, forced):
+    """For T <= 256 moe_expert_ffn runs gate/up and down in one launch, a down
+    tile starting when its expert's gate/up tiles have stored h.  Its h and
+    y_perm must equal, bit for bit, those of the two separate launches
+    (moe_expert_gate_up then moe_expert_down), on repeated calls: a down tile
+    that read h too early would differ."""
+    moe = _moe()
+    W = layer0_weights()
+    tok = synth.make_tokens(T, seed)
+    if forced is not None:
+        tok.bias[:] = 0
+        tok.bias[forced] = 1000.0
+    x, lg, bias = tokens_dev(tok)
+    idx, w = moe.moe_route(lg, bias)
+    counts, offsets, perm_src, inv_perm = moe.moe_permute(idx)
+    h2 = moe.moe_expert_gate_up(x, W.packed, offsets, perm_src)
+    y2 = moe.moe_expert_down(h2, W.packed, offsets)
+    for _ in range(3):
+        h1 = torch.full_like(h2, float("nan"))
+        y1 = torch.full_like(y2, float("nan"))
+        moe.moe_expert_ffn(x, W.packed, offsets, perm_src, h1, y1)
+        torch.cuda.synchronize()
+        assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+        assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
