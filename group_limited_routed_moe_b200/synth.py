@@ -36,8 +36,9 @@ TOPK = 8
 WEIGHT_STD = 0.02
 
 # matrix ids inside a layer
-W_GATE, W_UP, W_DOWN = 0, 1, 2
-_W_SHAPES = {W_GATE: (HIDDEN, INTER), W_UP: (HIDDEN, INTER), W_DOWN: (INTER, HIDDEN)}
+W_GATE, W_UP, W_DOWN, W_ROUTER = 0, 1, 2, 3
+_W_SHAPES = {W_GATE: (HIDDEN, INTER), W_UP: (HIDDEN, INTER), W_DOWN: (INTER, HIDDEN),
+             W_ROUTER: (HIDDEN, N_EXPERTS)}
 
 
 # ----------------------------------------------------------------------------
@@ -104,6 +105,12 @@ def weight_bits_np(seed: int, layer: int, which: int,
         u = _mix32_np(_mix32_np(i ^ k1[j]) ^ k2[j])
         out[j] = table[u >> np.uint32(16)]
     return out.reshape(len(experts), rows, cols)
+
+
+def router_weight_bits_np(seed: int, layer: int) -> np.ndarray:
+    """Router matrix W_router [1536, 128] of ``layer`` as bf16 bits (one matrix,
+    from the same counter generator as the expert weights: N(0, 0.02))."""
+    return weight_bits_np(seed, layer, W_ROUTER, experts=[0])[0]
 
 
 def layer_weights_np(seed: int, layer: int, experts=None):

@@ -87,6 +87,19 @@ def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
 # Routing
 # ----------------------------------------------------------------------------
 
+def router_logits(x_bits: np.ndarray, w_router_bits: np.ndarray) -> np.ndarray:
+    """Router projection: logits[t, e] = sum_k x[t, k] * W_router[k, e], float64.
+
+    x_bits [T, 1536] and w_router_bits [1536, 128] are bf16 bits; the result is
+    the exact product of their values up to float64 rounding.  The pages name
+    the routing kernel this feeds ("Ling-3.0-tiny on a Qualcomm board", issue
+    #1247, "What it does not cover", first bullet) but not the projection
+    itself; the reading here is the usual bias-free linear gate of the hidden
+    state onto the 128 experts (the bias of the routing rule is added after it).
+    """
+    return bf16_bits_to_f64(x_bits) @ bf16_bits_to_f64(w_router_bits)
+
+
 def sigmoid(z: np.ndarray) -> np.ndarray:
     """Logistic function in float64."""
     return 1.0 / (1.0 + np.exp(-z))
