@@ -263,6 +263,35 @@ class LayerRun:
         barrier()
         return np.array([e[0].elapsed_time(e[1]) for e in evs]), wall
 
+    def router(self, steps, peaks):
+        """The router projection (moe_router) alone on this batch: K launches after
+        the same L2 flush, against the HBM roofline (x, W_router and the logits
+        cross HBM once; 2 flop per byte of x per expert is far below the ridge)."""
+        torch, moe = self.torch, self.moe
+        T = self.T
+        w_bits = synth.router_weight_bits_np(0, 0)
+        w = torch.from_numpy(w_bits.view(np.int16)).to(self.dev).view(torch.bfloat16)
+        packed = moe.moe_pack_router(w)
+        logits = torch.empty((T, 128), dtype=torch.float32, device=self.dev)
+        moe.moe_router(self.x[:T], packed, logits)
+        times = []
+        for _ in range(steps):
+            self.flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            moe.moe_router(self.x[:T], packed, logits, stream=self.stream)
+            b.record(self.stream)
+            times.append((a, b))
+        torch.cuda.synchronize()
+        us = float(np.mean([a.elapsed_time(b) for a, b in times])) * 1e3
+        nbytes = T * 1536 * 2 + 1536 * 128 * 2 + T * 128 * 4
+        achieved = nbytes / (us * 1e-6) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        return {"kernel": "router_kernel (logits = x W_router, tcgen05)", "us": round(us, 2),
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "algorithmic_per_launch": nbytes,
+                "flops_per_launch": 2 * T * 1536 * 128}
+
     def dirty_l2_steps(self, steps, barrier):
         """Context only: the same K steps after a write-only flush, which leaves
         about 126 MB of dirty lines in L2 for the step's first kernels to write
@@ -457,6 +486,7 @@ def run_ours(args):
         steps_ms, wall = run.timed(args.steps, args.warmup, barrier)
     per = run.breakdown(args.steps)
     dirty_ms = run.dirty_l2_steps(args.steps, barrier)
+    router = run.router(max(10, args.steps // 5), peaks)
     step_ms = float(steps_ms.mean())
     elapsed = torch.tensor([step_ms * args.steps], device=dev, dtype=torch.float64)
     if dist is not None:
@@ -478,6 +508,7 @@ def run_ours(args):
                           "dirty line is left in L2"),
                    "wall_s_timed_region": round(wall, 4)},
         "roofline": roofline_for(wl, run, per, peaks, peak_kind),
+        "router": router,
         "layer": dict(layer_fractions(wl, run, steps_ms, per, peaks),
                       layer_us_after_write_only_flush=round(dirty_ms * 1e3, 2)),
         "e2e": {"value": round(wl.T * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
@@ -494,12 +525,14 @@ def run_ours(args):
             steps2, wall2 = run2.timed(max(args.steps, 50), args.warmup, barrier)
         per2 = run2.breakdown(max(args.steps, 50))
         dirty2 = run2.dirty_l2_steps(max(args.steps, 50), barrier)
+        router2 = run2.router(20, peaks)
         e2e2, h2d2, d2h2 = run2.e2e(20, 3)
         graph_us = run2.graph_layer_us(50, 3)
         ms2 = float(steps2.mean())
         line["decode_T16"] = {
             "value": round(wl2.T / (ms2 * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms2, 5),
             "roofline": roofline_for(wl2, run2, per2, peaks, peak_kind),
+            "router": router2,
             "layer": dict(layer_fractions(wl2, run2, steps2, per2, peaks),
                           layer_us_after_write_only_flush=round(dirty2 * 1e3, 2)),
             "graph_replay": {"layer_us": round(graph_us, 2),

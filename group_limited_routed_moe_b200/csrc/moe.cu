@@ -20,6 +20,7 @@
 #include "permute.cuh"
 #include "route.cuh"
 #include "route_permute_small.cuh"
+#include "router.cuh"
 
 using namespace moe;
 
@@ -99,6 +100,9 @@ int device_setup(int* dev_out, int* sms_out) {
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(router::router_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, router::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       if (g_encode == nullptr) {
         cudaDriverEntryPointQueryResult q;
@@ -212,6 +216,21 @@ int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets,
                     perm_src, inv_perm);
 }
 
+// Router projection: logits [T][128] fp32 from x and the packed router.
+int do_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, float* logits, int sms,
+              cudaStream_t s) {
+  CUtensorMap tw, tx;
+  int rc = make_tmap(&tw, packed_router, kH, kE, router::BM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  if (!rc)
+    rc = make_tmap(&tx, x, kH, static_cast<uint64_t>(T), router::BN, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  if (rc) return rc;
+  const int64_t ntiles = (T + router::BN - 1) / router::BN;
+  const unsigned grid = static_cast<unsigned>(ntiles < sms ? ntiles : sms);
+  return launch_pdl("router_kernel launch", router::router_kernel, dim3(grid),
+                    dim3(router::THREADS), router::SMEM_BYTES, s, tw, tx, T, logits,
+                    g_timeout_ns.load());
+}
+
 // Steps 1 and 2 as moe_layer runs them: one fused block for a few tokens.
 int do_route_permute(const float* logits, const float* bias, int64_t T, int32_t* idx, float* w,
                      int32_t* counts, int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
@@ -317,7 +336,7 @@ int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
 
 // workspace carve-up of moe_layer
 struct LayerWs {
-  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, total;
+  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, total;
 };
 LayerWs layer_ws(int64_t T) {
   LayerWs L{};
@@ -337,6 +356,7 @@ LayerWs layer_ws(int64_t T) {
   L.perm_ws = take(permute_ws_bytes(T));
   L.h = take(n * kI * 2);
   L.y = take(n * kH * 2);
+  L.logits = take(static_cast<size_t>(T) * kE * 4);  // used by moe_layer_routed
   L.total = o;
   return L;
 }
@@ -501,22 +521,29 @@ size_t moe_layer_workspace_bytes(int64_t T) {
   return layer_ws(T).total;
 }
 
-int moe_layer(const moe_bf16* x, const float* logits, const float* bias, const moe_bf16* packed_w,
-              int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
-              float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// The layer from given router logits, or (packed_router != NULL) from the
+// router projection of x computed into the workspace first.
+int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
+               const moe_bf16* packed_router, const float* bias, const moe_bf16* packed_w,
+               int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+               float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
   int rc = check_T(T);
   if (rc) return rc;
   if (T == 0) return MOE_OK;
-  REQUIRE(x && logits && packed_w && out && workspace, "null pointer");
-  REQUIRE(aligned(x, 128) && aligned(packed_w, 128), "x and packed_w must be 128-byte aligned");
+  REQUIRE(x && (logits || packed_router) && packed_w && out && workspace, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_w, 128) && (!packed_router || aligned(packed_router, 128)),
+          "x, packed_w and packed_router must be 128-byte aligned");
   REQUIRE(aligned(workspace, 1024), "workspace must be 1024-byte aligned");
-  REQUIRE(aligned(logits, 16) && (!bias || aligned(bias, 16)) && aligned(out, 16) &&
+  REQUIRE((!logits || aligned(logits, 16)) && (!bias || aligned(bias, 16)) && aligned(out, 16) &&
               (!residual || aligned(residual, 16)) && (!topk_idx_out || aligned(topk_idx_out, 16)) &&
               (!topk_w_out || aligned(topk_w_out, 16)),
           "pointers must be 16-byte aligned");
   const LayerWs L = layer_ws(T);
   if (workspace_bytes < L.total)
-    return fail(MOE_ERR_WORKSPACE, "moe_layer workspace needs %zu bytes, got %zu", L.total,
+    return fail(MOE_ERR_WORKSPACE, "%s workspace needs %zu bytes, got %zu", fn, L.total,
                 workspace_bytes);
   int sms = 0;
   rc = device_setup(nullptr, &sms);
@@ -532,11 +559,64 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias, const m
   moe_bf16* h = reinterpret_cast<moe_bf16*>(ws + L.h);
   moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
 
-  rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
-                        ws + L.perm_ws, s);
+  if (packed_router != nullptr) {
+    float* lg = reinterpret_cast<float*>(ws + L.logits);
+    rc = do_router(x, packed_router, T, lg, sms, s);
+    logits = lg;
+  }
+  if (!rc)
+    rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
+                          ws + L.perm_ws, s);
   if (!rc) rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
   if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s);
   return rc;
+}
+}  // namespace
+
+extern "C" {
+
+int moe_layer(const moe_bf16* x, const float* logits, const float* bias, const moe_bf16* packed_w,
+              int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+              float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  if (T > 0 && logits == nullptr) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+  return layer_impl("moe_layer", x, logits, nullptr, bias, packed_w, T, residual, out,
+                    topk_idx_out, topk_w_out, workspace, workspace_bytes, stream);
+}
+
+int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
+                     const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
+                     moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                     size_t workspace_bytes, moe_stream_t stream) {
+  if (T > 0 && packed_router == nullptr) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+  return layer_impl("moe_layer_routed", x, nullptr, packed_router, bias, packed_w, T, residual,
+                    out, topk_idx_out, topk_w_out, workspace, workspace_bytes, stream);
+}
+
+size_t moe_router_packed_bytes(void) { return static_cast<size_t>(kE) * kH * 2; }
+
+int moe_pack_router(const moe_bf16* w_router, moe_bf16* packed_router, moe_stream_t stream) {
+  REQUIRE(w_router && packed_router, "null pointer");
+  REQUIRE(aligned(packed_router, 128), "packed_router must be 128-byte aligned");
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  router::router_pack_kernel<<<dim3(kE / 32, kH / 32), 256, 0,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint16_t*>(w_router), reinterpret_cast<uint16_t*>(packed_router));
+  return launch_check("router_pack_kernel launch");
+}
+
+int moe_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, float* logits,
+               moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && packed_router && logits, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_router, 128), "x and packed_router must be 128-byte aligned");
+  REQUIRE(aligned(logits, 16), "logits must be 16-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_router(x, packed_router, T, logits, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -59,6 +59,10 @@ _SIGS = {
     "moe_combine": ([_p, _p, _p, _i64, _p, _p, _p], _i32),
     "moe_layer_workspace_bytes": ([_i64], _sz),
     "moe_layer": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_router_packed_bytes": ([], _sz),
+    "moe_pack_router": ([_p, _p, _p], _i32),
+    "moe_router": ([_p, _p, _i64, _p, _p], _i32),
+    "moe_layer_routed": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_permute_fixed_scratch_max_tokens": ([], _i64),
     "moe_permute_fixed_scratch": ([_p, _i64, _p, _p, _p, _p, _p], _i32),
 }
@@ -248,6 +252,42 @@ def moe_layer(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
                                       _ptr(residual), _ptr(out), _ptr(topk_idx_out),
                                       _ptr(topk_w_out), _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
+    return out
+
+
+def moe_pack_router(w_router: torch.Tensor, packed=None, stream=None) -> torch.Tensor:
+    """W_router [1536,128] bf16 -> packed K-major [128,1536] (see include/moe.h)."""
+    if w_router.dtype != torch.bfloat16 or tuple(w_router.shape) != (HIDDEN, N_EXPERTS) \
+            or not w_router.is_contiguous() or not w_router.is_cuda:
+        raise ValueError(f"expected contiguous CUDA bf16 ({HIDDEN}, {N_EXPERTS})")
+    if packed is None:
+        packed = torch.empty((N_EXPERTS, HIDDEN), dtype=torch.bfloat16, device=w_router.device)
+    _check("moe_pack_router", lib.moe_pack_router(_ptr(w_router), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_router(x: torch.Tensor, packed_router: torch.Tensor, logits=None, stream=None):
+    """logits [T,128] fp32 = x [T,1536] bf16 @ W_router."""
+    T = x.shape[0]
+    if logits is None:
+        logits = torch.empty((T, N_EXPERTS), dtype=torch.float32, device=x.device)
+    _check("moe_router", lib.moe_router(_ptr(x), _ptr(packed_router), T, _ptr(logits),
+                                        _stream(stream)))
+    return logits
+
+
+def moe_layer_routed(x: torch.Tensor, packed_router: torch.Tensor, bias: torch.Tensor | None,
+                     packed_w: torch.Tensor, residual=None, out=None, topk_idx_out=None,
+                     topk_w_out=None, workspace: torch.Tensor | None = None, stream=None):
+    """moe_layer with the router projection of x in front (see include/moe.h)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = alloc_layer_workspace(T, x.device)
+    _check("moe_layer_routed", lib.moe_layer_routed(
+        _ptr(x), _ptr(packed_router), _ptr(bias), _ptr(packed_w), T, _ptr(residual), _ptr(out),
+        _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 
 

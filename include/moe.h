@@ -197,6 +197,28 @@ int moe_expert_down(const moe_f16* h, const moe_bf16* packed_w,
                     const int32_t* offsets, int64_t T, moe_f16* y_perm,
                     moe_stream_t stream);
 
+/* ---- router projection (the step before routing) ----------------------- */
+
+/* The pages name the group-limited routing kernel of the CUDA path ("Ling-3.0-
+ * tiny on a Qualcomm board", TensorFold issue #1247, "What it does not cover",
+ * first bullet); its input is the projection of the hidden state onto the 128
+ * experts, computed here as
+ *   logits[t][e] = sum_k x[t][k] W_router[k][e]   (bf16 in, fp32 accumulate, fp32 out)
+ * on the tensor cores.  The routing rule's bias is added afterwards by moe_route. */
+
+/* Bytes of the packed router matrix (128 x 1536 bf16). */
+size_t moe_router_packed_bytes(void);
+
+/* One-time re-layout of W_router [1536][128] bf16 into the K-major [128][1536]
+ * operand order of moe_router.  packed_router: moe_router_packed_bytes()
+ * bytes, 128-byte aligned, caller-owned. */
+int moe_pack_router(const moe_bf16* w_router, moe_bf16* packed_router, moe_stream_t stream);
+
+/* logits [T][128] fp32 (out) = x [T][1536] bf16 (128-byte aligned) times the
+ * packed router.  One persistent tcgen05 GEMM launch (64 tokens per tile). */
+int moe_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, float* logits,
+               moe_stream_t stream);
+
 /* ---- the fused layer ---------------------------------------------------- */
 
 /* Workspace bytes moe_layer needs for T tokens. */
@@ -213,6 +235,14 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias,
               const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
               moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
               void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* moe_layer with the router projection in front: the logits come from
+ * moe_router(x, packed_router) into the workspace (same workspace size as
+ * moe_layer), then route -> permute -> expert FFN -> combine as above. */
+int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
+                     const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
+                     moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
+                     void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* ---- permutation without a caller workspace ------------------------------ */
 
