@@ -1,11 +1,12 @@
-"""moe_layer's fused route + permute for small batches (T <= 64: one block, a
-warp per token, counting sort from shared memory) against the separate step
-kernels (moe_route, moe_permute, ...) and the float64 oracle.
+"""moe_layer's fused launches for small batches against the separate step
+kernels (moe_route, moe_permute, moe_expert_gate_up, moe_expert_down,
+moe_combine) and the float64 oracle: route + permute in one block for T <= 64
+(a warp per token, counting sort from shared memory), and gate/up and down in
+one persistent launch for T <= 256.
 
 The fused kernel must reproduce the step kernels exactly: same expert ids, the
 same fp32 weights bit for bit, the same permutation, hence a bit-identical
-layer output.  T = 65 is the first batch that takes the unfused path inside
-moe_layer and checks the same identity there."""
+layer output.  T = 65 and T = 257 are the first batches past each fused path."""
 import numpy as np
 import pytest
 import torch
@@ -47,7 +48,7 @@ def _same_bits(a, b):
                        b.contiguous().view(torch.int16 if b.element_size() == 2 else torch.int32))
 
 
-@pytest.mark.parametrize("T", [1, 2, 16, 31, 32, 33, 64, 65])
+@pytest.mark.parametrize("T", [1, 2, 16, 31, 32, 33, 64, 65, 128, 256, 257])
 def test_fused_small_layer_equals_steps_and_oracle(T):
     moe = _moe()
     W = layer0_weights()
