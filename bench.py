@@ -375,6 +375,21 @@ class LayerRun:
         return float(np.mean(times)), x_h.numel() * 2 + lg_h.numel() * 4, out_h.numel() * 2
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's `value` (each rank's own when dist is None)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's batch over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
 def distinct_experts(run):
     """Experts with at least one row in the timed steps (the permute's counts)."""
     return int((run.counts > 0).sum().item())
@@ -488,11 +503,8 @@ def run_ours(args):
     dirty_ms = run.dirty_l2_steps(args.steps, barrier)
     router = run.router(max(10, args.steps // 5), peaks)
     step_ms = float(steps_ms.mean())
-    elapsed = torch.tensor([step_ms * args.steps], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(elapsed, op=dist.ReduceOp.MAX)
-    ms_per_step = float(elapsed.item()) / args.steps
-    value = wl.T * world / (ms_per_step * 1e-3)
+    ms_per_step = max_over_ranks(step_ms * args.steps, dist, dev) / args.steps
+    value = job_tokens_per_s(wl.T, world, ms_per_step)
     e2e_ms, h2d, d2h = run.e2e(max(3, args.steps // 4), 2)
 
     line = {
