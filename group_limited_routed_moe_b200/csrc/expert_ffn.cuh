@@ -387,7 +387,10 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       const uint32_t stage = smem_u32(sEpi + warp * EPI_WARP_BYTES);
       bool bad = false;  // range check of this thread's row; rows >= nvalid hold garbage
       uint16_t* g0 = out + (static_cast<int64_t>(S->off[e]) + m * BM + warp * 32) * C::OUT_COLS;
-      if (PHASE == 1) {
+      // A warp whose 32 rows are all padding has nothing to read or store (at
+      // T=2048 with skewed routing that was a fifth of the gate/up time).
+      if (nvalid == 0) {
+      } else if (PHASE == 1) {
         g0 += j * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
                                silu_mul(__uint_as_float(g[2 * i + 1]),
                                         __uint_as_float(u[2 * i + 1])),
                                bad);
-          if (nvalid > 0) store_block_32x32(pk, stage, g0 + c * 32, C::OUT_COLS, nvalid, lane);
+          store_block_32x32(pk, stage, g0 + c * 32, C::OUT_COLS, nvalid, lane);
         }
       } else {
         g0 += j * BN;
@@ -414,10 +417,8 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
             p0[i] = pack_f16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]), bad);
             p1[i] = pack_f16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]), bad);
           }
-          if (nvalid > 0) {
-            store_block_32x32(p0, stage, g0 + c * 64, C::OUT_COLS, nvalid, lane);
-            store_block_32x32(p1, stage, g0 + c * 64 + 32, C::OUT_COLS, nvalid, lane);
-          }
+          store_block_32x32(p0, stage, g0 + c * 64, C::OUT_COLS, nvalid, lane);
+          store_block_32x32(p1, stage, g0 + c * 64 + 32, C::OUT_COLS, nvalid, lane);
         }
       }
       range_bad |= bad && lane < nvalid;
