@@ -128,7 +128,12 @@ __device__ __forceinline__ void decode_tile(const SmemTail* S, int tile, int NT,
   m = rem - j * mt;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// silu(g) * u = g / (1 + exp(-g)) * u.  The fast division (2 ulp of fp32) is
+// far below the fp16 rounding of h that follows; for very negative g the
+// denominator overflows and the result is 0, the limit of silu.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
 
 // Stores one warp's 32 rows x 32 fp16 columns (lane = row, 16 packed pairs in
 // registers) as row segments of 64 bytes: written to the warp's padded shared
