@@ -28,16 +28,18 @@
 // by each CTA from the device-side expert offsets, so the host never reads
 // them.
 //
-// Warp roles inside a CTA (one CTA per SM: ~194 KB of shared memory, all 512
+// Warp roles inside a CTA (one CTA per SM: ~205 KB of shared memory, all 512
 // TMEM columns):
 //   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SwiGLU, fp16 stores
-//   warps 4-7  (phase 1) A producers: gather the tile's token rows of x with
+//   warps 4-11 (phase 1) A producers: gather the tile's token rows of x with
 //              cp.async into the 128B-swizzled operand layout, eight threads
 //              per row so that each warp instruction moves whole 128-byte
 //              lines (16-byte-per-row access touched every L2 sector twice
 //              and cost ~40% of the gate/up time at T=8189); each thread
 //              signals the stage's barrier through cp.async.mbarrier.arrive,
-//              so the gather keeps all stages in flight.  Rows past the
+//              so the gather keeps all stages in flight.  Eight warps of 4
+//              rows a thread issue the 1024 copies of a k-block faster than
+//              four warps of 8 (gate/up 199 -> 191 us at T=8189).  Rows past the
 //              expert's count are not loaded (a row of A only reaches the
 //              same, never stored, accumulator row).  With ZERO_PAD they are
 //              kept at zero by a zero-fill cp.async, issued only when the
@@ -78,10 +80,10 @@ struct Cfg<1> {
   static constexpr int NT = kI / 128;             // 4 n-tiles of 128 gate + 128 up
   static constexpr int B_ROWS_PER_EXPERT = 2 * kI;  // 1024 packed rows
   static constexpr int OUT_COLS = kI;             // h row length
-  static constexpr int THREADS = 320;
-  static constexpr int TMA_WARP = 8;
-  static constexpr int MMA_WARP = 9;
-  static constexpr int FULL_COUNT = 1 + 128;      // TMA arrive + 128 gather threads
+  static constexpr int THREADS = 448;
+  static constexpr int TMA_WARP = 12;
+  static constexpr int MMA_WARP = 13;
+  static constexpr int FULL_COUNT = 1 + 256;      // TMA arrive + 256 gather threads
   static constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kFmtBF16);
 };
 template <>
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       mbar_init(&S->tempty[a], 4);
     }
     mbar_init(&S->drain, 1);
-    tileq_init(&S->tq, (PHASE == 1 ? 4 : 0) + 1 + 4);  // gather warps, MMA thread, epilogue warps
+    tileq_init(&S->tq, (PHASE == 1 ? 8 : 0) + 1 + 4);  // gather warps, MMA thread, epilogue warps
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -324,16 +326,16 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       umma_commit(&S->drain);
       mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
     }
-  } else if (PHASE == 1 && warp >= 4 && warp < 8) {
+  } else if (PHASE == 1 && warp >= 4 && warp < 12) {
     // ------------------------------------------------ A gather producers
-    // Thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 16 i, i < 8, so a
+    // Thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 32 i, i < 4, so a
     // warp instruction moves four whole 128-byte rows (full L2 lines).  The
     // swizzled chunk slot (chunk ^ (row & 7)) is the same for all of a
-    // thread's rows because the row stride is 16.
+    // thread's rows because the row stride is 32.
     const int t = threadIdx.x - 128;
-    const int chunk = t & 7, rsub = t >> 3;
+    const int chunk = t & 7, rsub = t >> 3;  // rsub < 32: rows rsub + 32 i, i < 4
     const uint32_t slot = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
-    uint32_t dirty = 0u;  // bit 8*s + i: row rsub+16i of stage s may be non-zero (ring starts zeroed)
+    uint32_t dirty = 0u;  // bit 4*s + i: row rsub+32i of stage s may be non-zero (ring starts zeroed)
     int it = 0, n = 0;
     bool ok = true;
     while (ok) {
@@ -341,11 +343,11 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       if (tile < 0) break;
       int e, m, j;
       decode_tile(S, tile, C::NT, e, m, j);
-      const char* src[8];
+      const char* src[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         src[i] = nullptr;
-        const int row_in_e = m * BM + rsub + 16 * i;
+        const int row_in_e = m * BM + rsub + 32 * i;
         if (row_in_e < S->cnt[e]) {
           const int p = perm_src[S->off[e] + row_in_e];
           if (p >= 0 && static_cast<int64_t>(p) < nrows)
@@ -361,13 +363,13 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
         }
         const uint32_t base = smem_u32(sA + s * A_BYTES) + rsub * 128 + slot;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t bit = 1u << (8 * s + i);
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t bit = 1u << (4 * s + i);
           if (src[i] != nullptr) {
-            cp_async_16(base + i * 16 * 128, src[i] + kb * BK * 2, 16);
+            cp_async_16(base + i * 32 * 128, src[i] + kb * BK * 2, 16);
             dirty |= bit;
           } else if (ZERO_PAD && (dirty & bit)) {
-            cp_async_16(base + i * 16 * 128, x, 0);
+            cp_async_16(base + i * 32 * 128, x, 0);
             dirty &= ~bit;
           }
         }
