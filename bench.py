@@ -47,7 +47,6 @@ from group_limited_routed_moe_b200 import synth  # noqa: E402
 GATE_UP_BYTES_PER_EXPERT = 2 * 1536 * 512 * 2
 DOWN_BYTES_PER_EXPERT = 1536 * 512 * 2
 FLOPS_PER_ROW = 2 * (1536 * 1024 + 512 * 1536)          # one (token, expert) pair
-GATE_UP_FLOPS_PER_ROW = 2 * 1536 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -189,14 +188,12 @@ class LayerRun:
         # moe_layer launches: route + permute (one fused kernel up to 64 tokens;
         # route and one permute kernel up to 1024; route, count and fused scan/scatter
         # up to 256 blocks of 128 tokens; route, count, scan, scatter beyond), the
-        # expert FFN (one launch up to 256 tokens, gate/up and down above), combine
+        # expert FFN (gate/up and down in one launch), combine
         nb = (T + 127) // 128
         n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
-        self.fused_ffn = T <= 256
-        self.launches_per_step = n_rp + (1 if self.fused_ffn else 2) + 1
+        self.launches_per_step = n_rp + 2  # + the expert FFN (one launch) + combine
         # the breakdown pass times the same kernels the layer call runs
-        self.part_names = (["route", "permute", "expert_ffn", "combine"] if self.fused_ffn
-                           else ["route", "permute", "gate_up", "down", "combine"])
+        self.part_names = ["route", "permute", "expert_ffn", "combine"]
         self.lws = moe.alloc_layer_workspace(T, dev)
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
@@ -229,16 +226,9 @@ class LayerRun:
         m.moe_permute(self.idx, self.counts, self.offsets, self.perm_src, self.inv_perm,
                       self.pws, stream=s)
         rec()
-        if self.fused_ffn:
-            m.moe_expert_ffn(self.x[:T], self.packed, self.offsets, self.perm_src, self.h, self.y,
-                             stream=s)
-            rec()
-        else:
-            m.moe_expert_gate_up(self.x[:T], self.packed, self.offsets, self.perm_src, self.h,
-                                 stream=s)
-            rec()
-            m.moe_expert_down(self.h, self.packed, self.offsets, self.y, stream=s)
-            rec()
+        m.moe_expert_ffn(self.x[:T], self.packed, self.offsets, self.perm_src, self.h, self.y,
+                         stream=s)
+        rec()
         m.moe_combine(self.y, self.w, self.inv_perm, out=self.out[:T], stream=s)
         rec()
 
@@ -396,42 +386,33 @@ def distinct_experts(run):
 
 
 def roofline_for(wl, run, per_ms, peaks, peak_kind):
-    """Roofline of the dominant kernel of one workload: the gate/up GEMM, or for
-    T <= 256 the single launch that runs both expert GEMMs."""
+    """Roofline of the dominant kernel of one workload: the expert FFN launch
+    (gate/up + SwiGLU + down).  Prefill-sized batches are bound by the tensor
+    cores (both GEMMs' flops), decode-sized ones by HBM (the touched experts'
+    weights, x read, y_perm written)."""
     T = wl.T
-    if run.fused_ffn:
-        ffn_ms = float(per_ms[:, run.part_names.index("expert_ffn")].mean())
-        d = distinct_experts(run)
-        nbytes = (d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * 1536 * 2
-                  + 8 * T * 1536 * 2)
-        peak = float(peaks["hbm_gbs"])
-        achieved = nbytes / (ffn_ms * 1e-3) / 1e9
-        return {"kernel": "skinny_gemm_kernel<3> (gate/up + SwiGLU + down in one launch)",
-                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                "algorithmic_per_launch": nbytes, "distinct_experts": d,
-                "traffic": profiled_traffic("expert_ffn", wl.name)}
-    gate_up_ms = float(per_ms[:, run.part_names.index("gate_up")].mean())
+    ffn_ms = float(per_ms[:, run.part_names.index("expert_ffn")].mean())
     if T >= 2048:
-        flops = GATE_UP_FLOPS_PER_ROW * 8 * T
+        flops = FLOPS_PER_ROW * 8 * T
         key = "bf16_tflops"
         peak = float(peaks[key])
-        achieved = flops / (gate_up_ms * 1e-3) / 1e12
-        return {"kernel": "ffn_gemm_kernel<1> (gate/up + SwiGLU)", "bound": "tensor",
-                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} {key} (burst)",
-                "algorithmic_per_launch": flops,
-                "traffic": profiled_traffic("gate_up", wl.name)}
+        achieved = flops / (ffn_ms * 1e-3) / 1e12
+        return {"kernel": "ffn_gemm_kernel<3> (gate/up + SwiGLU + down in one launch)",
+                "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_kind} {key} (burst)", "algorithmic_per_launch": flops,
+                "traffic": profiled_traffic("expert_ffn", wl.name)}
     d = distinct_experts(run)
-    nbytes = d * GATE_UP_BYTES_PER_EXPERT + T * 1536 * 2 + 8 * T * 512 * 2
+    nbytes = (d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * 1536 * 2
+              + 8 * T * 1536 * 2)
     peak = float(peaks["hbm_gbs"])
-    achieved = nbytes / (gate_up_ms * 1e-3) / 1e9
-    kernel = "ffn_gemm_kernel<1> (gate/up + SwiGLU)"
-    return {"kernel": kernel, "bound": "hbm",
-            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-            "algorithmic_per_launch": nbytes, "distinct_experts": d,
-            "traffic": profiled_traffic("gate_up", wl.name)}
+    achieved = nbytes / (ffn_ms * 1e-3) / 1e9
+    kernel = ("skinny_gemm_kernel<3>" if T <= 256 else "ffn_gemm_kernel<3>") + \
+        " (gate/up + SwiGLU + down in one launch)"
+    return {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_per_launch": nbytes,
+            "distinct_experts": d, "traffic": profiled_traffic("expert_ffn", wl.name)}
 
 
 def layer_fractions(wl, run, step_ms, per_ms, peaks):

@@ -347,6 +347,29 @@ __device__ __forceinline__ void tileq_retire(int* sched, int* extra = nullptr, i
   }
 }
 
+constexpr int kDoneWord = kSchedWord + 4;  // offsets[136 .. 263]: per-expert done counters
+
+// Waits until *counter >= need (acquire), bounded in time; then orders the
+// async proxy (TMA) after it.
+__device__ __forceinline__ bool wait_count(const int* counter, int need, volatile int* abort_flag,
+                                           uint64_t timeout_ns, unsigned site) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 0;; ++n) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= need) break;
+    if (*abort_flag) return false;
+    if ((n & 15u) == 15u && global_timer_ns() - t0 > timeout_ns) {
+      record_status(site);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

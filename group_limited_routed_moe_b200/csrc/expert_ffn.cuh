@@ -72,31 +72,26 @@ constexpr int TMEM_COLS = 2 * BN;
 constexpr int STAGE_ROW = 80;                      // padded 64-byte row of the epilogue tile
 constexpr int EPI_WARP_BYTES = 32 * STAGE_ROW;     // one warp's 32 x 32 fp16 block
 
-template <int PHASE>
-struct Cfg;
-template <>
-struct Cfg<1> {
-  static constexpr int KDIM = kH;                 // 1536
-  static constexpr int NT = kI / 128;             // 4 n-tiles of 128 gate + 128 up
-  static constexpr int B_ROWS_PER_EXPERT = 2 * kI;  // 1024 packed rows
-  static constexpr int OUT_COLS = kI;             // h row length
-  static constexpr int THREADS = 448;
-  static constexpr int TMA_WARP = 12;
-  static constexpr int MMA_WARP = 13;
-  static constexpr int FULL_COUNT = 1 + 256;      // TMA arrive + 256 gather threads
-  static constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kFmtBF16);
-};
-template <>
-struct Cfg<2> {
-  static constexpr int KDIM = kI;                 // 512
-  static constexpr int NT = kH / BN;              // 6
-  static constexpr int B_ROWS_PER_EXPERT = kH;    // 1536 packed rows
-  static constexpr int OUT_COLS = kH;             // y_perm row length
-  static constexpr int THREADS = 192;
-  static constexpr int TMA_WARP = 4;
-  static constexpr int MMA_WARP = 5;
-  static constexpr int FULL_COUNT = 1;
-  static constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kFmtF16);
+// Per-phase constants (phase 1: gate/up, phase 2: down).
+__host__ __device__ constexpr int nt_of(int phase) { return phase == 1 ? kI / 128 : kH / BN; }  // n-tiles
+__host__ __device__ constexpr int kb_of(int phase) { return (phase == 1 ? kH : kI) / BK; }  // k-blocks
+__host__ __device__ constexpr int brows_of(int phase) { return phase == 1 ? 2 * kI : kH; }  // packed rows
+constexpr uint32_t kIdesc1 = idesc_f32acc(BM, BN, kFmtBF16);  // bf16 x bf16
+constexpr uint32_t kIdesc2 = idesc_f32acc(BM, BN, kFmtF16);   // fp16 x fp16
+// Increments a gate/up tile makes when its h rows are stored (its 4 epilogue
+// warps): a down tile of expert e waits for kDoneStep * 4 n-tiles * mtiles(e).
+constexpr int kDoneStep = 4;
+
+// MODE 1: gate/up only, 2: down only, 3: both in one launch (gate/up tile ids
+// first, then down).
+template <int MODE>
+struct Cfg {
+  static constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
+  static constexpr int GATHER_WARP0 = 4;                // warps 4-11 when HAS1
+  static constexpr int TMA_WARP = HAS1 ? 12 : 4;
+  static constexpr int MMA_WARP = TMA_WARP + 1;
+  static constexpr int THREADS = 32 * (MMA_WARP + 1);   // 448 or 192
+  static constexpr int FULL_COUNT = HAS1 ? 1 + 256 : 1; // TMA arrive (+ 256 gather threads)
 };
 
 struct SmemTail {
@@ -109,25 +104,39 @@ struct SmemTail {
   uint32_t tmem_base;
   int abort_flag;
   int wsum[4];
-  int tile_start[kE + 1];
+  int mstart[kE + 1];  // exclusive prefix of the experts' 128-row m-tile counts
   int cnt[kE];
   int off[kE];
 };
 constexpr int TAIL_BYTES = (static_cast<int>(sizeof(SmemTail)) + 127) / 128 * 128;
 constexpr int SMEM_BYTES = TILE_BYTES + TAIL_BYTES + 4 * EPI_WARP_BYTES + 1024;
 
-__device__ __forceinline__ void decode_tile(const SmemTail* S, int tile, int NT, int& e, int& m,
+// Tile u of a phase with NT n-tiles per expert: expert e, m-tile m, n-tile j
+// (expert-major, then j, then m).
+__device__ __forceinline__ void decode_tile(const SmemTail* S, int u, int NT, int& e, int& m,
                                             int& j) {
-  int lo = 0, hi = kE - 1;  // largest e with tile_start[e] <= tile
+  int lo = 0, hi = kE - 1;  // largest e with mstart[e] * NT <= u
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (S->tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    if (S->mstart[mid] * NT <= u) lo = mid; else hi = mid - 1;
   }
   e = lo;
-  const int rem = tile - S->tile_start[e];
+  const int rem = u - S->mstart[e] * NT;
   const int mt = (S->cnt[e] + BM - 1) / BM;
   j = rem / mt;
   m = rem - j * mt;
+}
+
+struct TileInfo {
+  int phase, e, m, j;
+};
+template <int MODE>
+__device__ __forceinline__ TileInfo tile_info(const SmemTail* S, int tile, int total1) {
+  TileInfo t;
+  t.phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
+  const int u = (MODE == 3 && t.phase == 2) ? tile - total1 : tile;
+  decode_tile(S, u, nt_of(t.phase), t.e, t.m, t.j);
+  return t;
 }
 
 // silu(g) * u = g / (1 + exp(-g)) * u.  The fast division (2 ulp of fp32) is
@@ -156,15 +165,16 @@ __device__ __forceinline__ void store_block_32x32(const uint32_t (&pk)[16], uint
   __syncwarp();
 }
 
-template <int PHASE, bool ZERO_PAD>
-__global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
-    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b,
-                    const __grid_constant__ CUtensorMap tmap_a,
+template <int MODE, bool ZERO_PAD>
+__global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
+    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b1,  // packed W_gate/W_up (phase 1)
+                    const __grid_constant__ CUtensorMap tmap_b2,  // packed W_down (phase 2)
+                    const __grid_constant__ CUtensorMap tmap_a2,  // h rows (phase 2)
                     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                     const int32_t* __restrict__ perm_src, int64_t T,
-                    uint16_t* __restrict__ out, int* __restrict__ sched, uint64_t timeout_ns) {
-  using C = Cfg<PHASE>;
-  constexpr int KB = C::KDIM / BK;
+                    uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
+                    int* __restrict__ sched, int* __restrict__ done, uint64_t timeout_ns) {
+  using C = Cfg<MODE>;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -189,19 +199,22 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       mbar_init(&S->tempty[a], 4);
     }
     mbar_init(&S->drain, 1);
-    tileq_init(&S->tq, (PHASE == 1 ? 8 : 0) + 1 + 4);  // gather warps, MMA thread, epilogue warps
+    tileq_init(&S->tq, (C::HAS1 ? 8 : 0) + 1 + 4);  // gather warps, MMA thread, epilogue warps
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
   if (warp == C::TMA_WARP && lane == 0) {
-    tma_prefetch_desc(&tmap_b);
-    if (PHASE == 2) tma_prefetch_desc(&tmap_a);
+    if (C::HAS1) tma_prefetch_desc(&tmap_b1);
+    if (C::HAS2) {
+      tma_prefetch_desc(&tmap_b2);
+      tma_prefetch_desc(&tmap_a2);
+    }
   }
 
-  // tile table: tiles of expert e = ceil(count_e / 128) * NT, exclusive prefix
-  griddep_wait();  // offsets, perm_src and (phase 2) h come from the preceding kernels
-  int my_tiles = 0;
+  // tile table: m-tiles of expert e = ceil(count_e / 128), exclusive prefix
+  griddep_wait();  // offsets, perm_src and (down alone) h come from the preceding kernels
+  int my_mt = 0;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;
     const int o0 = offsets[e], o1 = offsets[e + 1];
@@ -212,9 +225,9 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     }
     S->cnt[e] = c;
     S->off[e] = o0;
-    my_tiles = ((c + BM - 1) / BM) * C::NT;
+    my_mt = (c + BM - 1) / BM;
   }
-  int incl = my_tiles;
+  int incl = my_mt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -222,7 +235,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   }
   if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
 
-  if (PHASE == 1) {
+  if (C::HAS1) {
     // Start the A ring at zero: rows past an expert's count are never loaded,
     // and with whatever the previous kernel left in shared memory there the
     // tensor cores ran measurably slower than with zeros or stale x rows.
@@ -235,15 +248,17 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
   if (threadIdx.x < kE) {
     int base = 0;
     for (int w = 0; w < warp; ++w) base += S->wsum[w];
-    S->tile_start[threadIdx.x] = base + incl - my_tiles;
-    if (threadIdx.x == kE - 1) S->tile_start[kE] = base + incl;
+    S->mstart[threadIdx.x] = base + incl - my_mt;
+    if (threadIdx.x == kE - 1) S->mstart[kE] = base + incl;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem_base = S->tmem_base;
-  const int total_tiles = S->tile_start[kE];
+  const int mtiles = S->mstart[kE];
+  const int total1 = C::HAS1 ? mtiles * nt_of(1) : 0;
+  const int total_tiles = total1 + (C::HAS2 ? mtiles * nt_of(2) : 0);
 
   if (warp == C::TMA_WARP) {
     // ------------------------------------------------ TMA producer
@@ -259,24 +274,32 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
         }
         if (pub < 0) break;
         const int next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);  // used after the loads
-        int e, m, j;
-        decode_tile(S, tile, C::NT, e, m, j);
-        const int brow = e * C::B_ROWS_PER_EXPERT + j * BN;
-        const int arow = S->off[e] + m * BM;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        const TileInfo ti = tile_info<MODE>(S, tile, total1);
+        if (MODE == 3 && ti.phase == 2) {
+          // every gate/up tile of expert e has stored its h rows
+          const int need = kDoneStep * nt_of(1) * ((S->cnt[ti.e] + BM - 1) / BM);
+          if (!wait_count(done + ti.e, need, abort_flag, timeout_ns, kSiteFfnDone)) {
+            ok = false;
+            break;
+          }
+        }
+        const int brow = ti.e * brows_of(ti.phase) + ti.j * BN;
+        const int arow = S->off[ti.e] + ti.m * BM;
+        for (int kb = 0; kb < kb_of(ti.phase); ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&S->empty[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
             ok = false;
             break;
           }
-          if (PHASE == 2) {
+          if (ti.phase == 2) {
             mbar_arrive_expect_tx(&S->full[s], A_BYTES + B_BYTES);
-            tma_load_2d(smem_u32(sA + s * A_BYTES), &tmap_a, kb * BK, arow, &S->full[s]);
+            tma_load_2d(smem_u32(sA + s * A_BYTES), &tmap_a2, kb * BK, arow, &S->full[s]);
+            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b2, kb * BK, brow, &S->full[s]);
           } else {
             mbar_arrive_expect_tx(&S->full[s], B_BYTES);
+            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b1, kb * BK, brow, &S->full[s]);
           }
-          tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b, kb * BK, brow, &S->full[s]);
         }
         tile = next;
       }
@@ -297,6 +320,8 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           ok = tile == -1;
           break;
         }
+        const int phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
+        const uint32_t idesc = phase == 1 ? kIdesc1 : kIdesc2;
         const int a = tc & 1;
         const uint32_t use = tc >> 1;
         if (!mbar_wait(&S->tempty[a], (use & 1) ^ 1, abort_flag, timeout_ns, kSiteFfnTmemEmpty)) {
@@ -305,7 +330,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + a * BN;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = 0; kb < kb_of(phase); ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&S->full[s], ph, abort_flag, timeout_ns, kSiteFfnFull)) {
@@ -317,7 +342,7 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
           const uint64_t bdesc = smem_desc_k128(smem_u32(sB + s * B_BYTES));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&S->empty[s]);
         }
         if (ok) umma_commit(&S->tfull[a]);
@@ -326,13 +351,15 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       umma_commit(&S->drain);
       mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
     }
-  } else if (PHASE == 1 && warp >= 4 && warp < 12) {
-    // ------------------------------------------------ A gather producers
+  } else if (C::HAS1 && warp >= C::GATHER_WARP0 && warp < C::GATHER_WARP0 + 8) {
+    // ------------------------------------------------ A gather producers (gate/up tiles)
     // Thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 32 i, i < 4, so a
     // warp instruction moves four whole 128-byte rows (full L2 lines).  The
     // swizzled chunk slot (chunk ^ (row & 7)) is the same for all of a
-    // thread's rows because the row stride is 32.
-    const int t = threadIdx.x - 128;
+    // thread's rows because the row stride is 32.  For a down tile (single
+    // launch) the TMA brings A; the gather threads only keep the stage
+    // barriers' arrival count.
+    const int t = threadIdx.x - 32 * C::GATHER_WARP0;
     const int chunk = t & 7, rsub = t >> 3;  // rsub < 32: rows rsub + 32 i, i < 4
     const uint32_t slot = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
     uint32_t dirty = 0u;  // bit 4*s + i: row rsub+32i of stage s may be non-zero (ring starts zeroed)
@@ -341,20 +368,31 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     while (ok) {
       const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      int e, m, j;
-      decode_tile(S, tile, C::NT, e, m, j);
+      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      if (ti.phase == 2) {
+        for (int kb = 0; kb < kb_of(2); ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&S->empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, timeout_ns,
+                         kSiteFfnEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive(&S->full[s]);
+        }
+        continue;
+      }
       const char* src[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         src[i] = nullptr;
-        const int row_in_e = m * BM + rsub + 32 * i;
-        if (row_in_e < S->cnt[e]) {
-          const int p = perm_src[S->off[e] + row_in_e];
+        const int row_in_e = ti.m * BM + rsub + 32 * i;
+        if (row_in_e < S->cnt[ti.e]) {
+          const int p = perm_src[S->off[ti.e] + row_in_e];
           if (p >= 0 && static_cast<int64_t>(p) < nrows)
             src[i] = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH) + chunk * 16;
         }
       }
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = 0; kb < kb_of(1); ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(&S->empty[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
@@ -383,8 +421,8 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
     for (int tc = 0;; ++tc) {
       const int tile = tileq_pop(&S->tq, tc, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      int e, m, j;
-      decode_tile(S, tile, C::NT, e, m, j);
+      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      const int e = ti.e, m = ti.m, j = ti.j;
       const int a = tc & 1;
       const uint32_t use = tc >> 1;
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
@@ -393,12 +431,12 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
       const int nvalid = min(32, max(0, S->cnt[e] - (m * BM + warp * 32)));
       const uint32_t stage = smem_u32(sEpi + warp * EPI_WARP_BYTES);
       bool bad = false;  // range check of this thread's row; rows >= nvalid hold garbage
-      uint16_t* g0 = out + (static_cast<int64_t>(S->off[e]) + m * BM + warp * 32) * C::OUT_COLS;
+      const int64_t row0 = static_cast<int64_t>(S->off[e]) + m * BM + warp * 32;
       // A warp whose 32 rows are all padding has nothing to read or store (at
       // T=2048 with skewed routing that was a fifth of the gate/up time).
       if (nvalid == 0) {
-      } else if (PHASE == 1) {
-        g0 += j * 128;
+      } else if (ti.phase == 1) {
+        uint16_t* g0 = h_out + row0 * kI + j * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t g[32], u[32];
@@ -410,10 +448,10 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
                                silu_mul(__uint_as_float(g[2 * i + 1]),
                                         __uint_as_float(u[2 * i + 1])),
                                bad);
-          store_block_32x32(pk, stage, g0 + c * 32, C::OUT_COLS, nvalid, lane);
+          store_block_32x32(pk, stage, g0 + c * 32, kI, nvalid, lane);
         }
       } else {
-        g0 += j * BN;
+        uint16_t* g0 = y_out + row0 * kH + j * BN;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v0[32], v1[32];
@@ -424,21 +462,28 @@ __global__ void __launch_bounds__(Cfg<PHASE>::THREADS, 1)
             p0[i] = pack_f16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]), bad);
             p1[i] = pack_f16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]), bad);
           }
-          store_block_32x32(p0, stage, g0 + c * 64, C::OUT_COLS, nvalid, lane);
-          store_block_32x32(p1, stage, g0 + c * 64 + 32, C::OUT_COLS, nvalid, lane);
+          store_block_32x32(p0, stage, g0 + c * 64, kH, nvalid, lane);
+          store_block_32x32(p1, stage, g0 + c * 64 + 32, kH, nvalid, lane);
         }
       }
       range_bad |= bad && lane < nvalid;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->tempty[a]);
+      if (MODE == 3 && ti.phase == 1) {
+        // publish: this warp's h rows of the tile are stored (a down tile's TMA reads them)
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(done + e, 1);
+      }
     }
     if (range_bad) record_status(kSiteFp16Range);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) tileq_retire(sched);
+  if (threadIdx.x == 0) tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

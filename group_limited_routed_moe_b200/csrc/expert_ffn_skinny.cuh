@@ -63,7 +63,6 @@ constexpr uint32_t kIdesc2 = idesc_f32acc(BMW, BNT, kFmtF16);
 // Counter increments a gate/up tile makes when its h values are stored (one per
 // storing warp): a down tile of expert e waits for kDoneStep * 8 * chunks(e).
 constexpr int kDoneStep = 2;
-constexpr int kDoneWord = kSchedWord + 4;  // offsets[136 .. 263]: per-expert done counters
 
 struct Tail {
   uint64_t full[STAGES];
@@ -111,27 +110,6 @@ __device__ __forceinline__ TileInfo tile_info(const Tail* S, int tile, int total
   const int u = (MODE == 3 && t.phase == 2) ? tile - total1 : tile;
   decode_tile(S, u, fblk(t.phase), t.e, t.f, t.c);
   return t;
-}
-
-// Waits until *counter >= need (acquire), bounded in time; then orders the
-// async proxy (TMA) after it.
-__device__ __forceinline__ bool wait_count(const int* counter, int need, volatile int* abort_flag,
-                                           uint64_t timeout_ns, unsigned site) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t n = 0;; ++n) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
-    if (v >= need) break;
-    if (*abort_flag) return false;
-    if ((n & 15u) == 15u && global_timer_ns() - t0 > timeout_ns) {
-      record_status(site);
-      *abort_flag = 1;
-      return false;
-    }
-    __nanosleep(64);
-  }
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  return true;
 }
 
 template <int MODE>

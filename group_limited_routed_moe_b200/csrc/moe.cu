@@ -92,6 +92,12 @@ int device_setup(int* dev_out, int* sms_out) {
         e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<2, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
       if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<3, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ffn::ffn_gemm_kernel<3, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ffn::SMEM_BYTES);
+      if (e == cudaSuccess)
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<1>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e == cudaSuccess)
@@ -271,8 +277,9 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
   auto* hb = reinterpret_cast<uint16_t*>(h);
   return launch_pdl("ffn_gemm_kernel<1> launch",
                     T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<1, true> : ffn::ffn_gemm_kernel<1, false>,
-                    dim3(sms), dim3(ffn::Cfg<1>::THREADS), ffn::SMEM_BYTES, s, tb1, tb1, xb, offsets,
-                    perm_src, T, hb, sched_words(offsets, 1), g_timeout_ns.load());
+                    dim3(sms), dim3(ffn::Cfg<1>::THREADS), ffn::SMEM_BYTES, s, tb1, tb1, tb1, xb,
+                    offsets, perm_src, T, hb, static_cast<uint16_t*>(nullptr),
+                    sched_words(offsets, 1), static_cast<int*>(nullptr), g_timeout_ns.load());
 }
 
 int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, int64_t T,
@@ -296,10 +303,11 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
   if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
   return launch_pdl("ffn_gemm_kernel<2> launch", ffn::ffn_gemm_kernel<2, false>, dim3(sms),
-                    dim3(ffn::Cfg<2>::THREADS), ffn::SMEM_BYTES, s, tb2, ta2,
+                    dim3(ffn::Cfg<2>::THREADS), ffn::SMEM_BYTES, s, tb2, tb2, ta2,
                     static_cast<const __nv_bfloat16*>(nullptr), offsets,
-                    static_cast<const int32_t*>(nullptr), T, reinterpret_cast<uint16_t*>(y),
-                    sched_words(offsets, 2), g_timeout_ns.load());
+                    static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
+                    reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
+                    static_cast<int*>(nullptr), g_timeout_ns.load());
 }
 
 int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
@@ -318,12 +326,25 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                       dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw1, tw2, th,
                       reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                       reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
-                      sched_words(offsets, 1), const_cast<int*>(offsets) + skinny::kDoneWord,
+                      sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
                       g_timeout_ns.load());
   }
-  int rc = do_gate_up(x, packed, offsets, perm_src, T, h, sms, s);
+  // both GEMMs in one launch (see expert_ffn.cuh)
+  CUtensorMap tb1, tb2, ta2;
+  int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  if (!rc) rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (!rc) rc = make_tmap(&ta2, h, kI, static_cast<uint64_t>(T) * kTopK, ffn::BM,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
-  return do_down(h, packed, offsets, T, y, sms, s);
+  return launch_pdl("ffn_gemm_kernel<3> launch",
+                    T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<3, true> : ffn::ffn_gemm_kernel<3, false>,
+                    dim3(sms), dim3(ffn::Cfg<3>::THREADS), ffn::SMEM_BYTES, s, tb1, tb2, ta2,
+                    reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+                    reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
+                    sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
+                    g_timeout_ns.load());
 }
 
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,

@@ -203,13 +203,16 @@ def test_generator_device_bytes_equal_host_bytes():
 
 @pytest.mark.parametrize("T,seed,forced", [(1, 31, None), (16, 32, None), (77, 33, None),
                                            (200, 34, [0, 1, 16, 17, 32, 33, 48, 49]),
-                                           (256, 35, None)])
+                                           (256, 35, None), (333, 36, None),
+                                           (1500, 37, [2, 3, 50, 51, 64, 65, 126, 127]),
+                                           (2048, 38, None), (8189, 39, None)])
 def test_expert_ffn_single_launch_equals_two_launches(T, seed, forced):
-    """For T <= 256 moe_expert_ffn runs gate/up and down in one launch, a down
-    tile starting when its expert's gate/up tiles have stored h.  Its h and
-    y_perm must equal, bit for bit, those of the two separate launches
-    (moe_expert_gate_up then moe_expert_down), on repeated calls: a down tile
-    that read h too early would differ."""
+    """moe_expert_ffn runs gate/up and down in one launch (weights-as-M tiles
+    for T <= 256, 128-row token tiles above), a down tile starting when its
+    expert's gate/up tiles have stored h.  Its h and y_perm must equal, bit for
+    bit, those of the two separate launches (moe_expert_gate_up then
+    moe_expert_down), on repeated calls: a down tile that read h too early
+    would differ."""
     moe = _moe()
     W = layer0_weights()
     tok = synth.make_tokens(T, seed)
