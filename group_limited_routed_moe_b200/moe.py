@@ -306,6 +306,56 @@ def moe_layer_from_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: t
     return out_host
 
 
+class HostPipeline:
+    """Layer calls from pinned host buffers with `depth` calls in flight.
+
+    Each slot owns device buffers (x, logits, out, workspace) and a stream; call
+    k uses slot k % depth.  Its host-to-device copies may overlap the previous
+    call's layer, and its device-to-host copy the next call's layer, but the
+    layers themselves run one after another (each waits for the previous
+    call's layer), so two calls never share the weights they stream through
+    L2.  Stream order keeps a slot's buffers from being reused before its
+    previous call has finished.  The output of call k lands in the `out_host`
+    passed to submit(); it is complete once `drain()` returns.
+    """
+
+    def __init__(self, T: int, device, depth: int = 2):
+        self.T, self.depth, self.k = T, depth, 0
+        self.last_layer = None
+        self.slots = []
+        for _ in range(depth):
+            self.slots.append({
+                "stream": torch.cuda.Stream(device),
+                "x": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
+                "logits": torch.empty((T, N_EXPERTS), dtype=torch.float32, device=device),
+                "out": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
+                "ws": alloc_layer_workspace(T, device),
+            })
+
+    def submit(self, x_host, logits_host, out_host, bias, packed_w):
+        slot = self.slots[self.k % self.depth]
+        self.k += 1
+        st = slot["stream"]
+        with torch.cuda.stream(st):
+            slot["x"].copy_(x_host, non_blocking=True)
+            slot["logits"].copy_(logits_host, non_blocking=True)
+            if self.last_layer is not None:
+                st.wait_event(self.last_layer)
+            moe_layer(slot["x"], slot["logits"], bias, packed_w, out=slot["out"],
+                      workspace=slot["ws"], stream=st)
+            self.last_layer = torch.cuda.Event()
+            self.last_layer.record(st)
+            out_host.copy_(slot["out"], non_blocking=True)
+        return out_host
+
+    def streams(self):
+        return [slot["stream"] for slot in self.slots]
+
+    def drain(self):
+        for st in self.streams():
+            st.synchronize()
+
+
 # ----------------------------------------------------------------- status
 
 def get_device_status(device: int = 0) -> int:

@@ -160,3 +160,31 @@ def test_layer_graph_capture():
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
     del g
+
+
+@pytest.mark.parametrize("T,depth", [(16, 3), (1000, 2)])
+def test_host_pipeline_outputs_equal_direct_calls(T, depth):
+    """moe.HostPipeline keeps `depth` host-buffer calls in flight (copies of one
+    overlapping the layer of another).  Six different batches go through it; each
+    output must equal, bit for bit, moe_layer on that batch: no call may read or
+    overwrite another call's buffers."""
+    moe = _moe()
+    W = layer0_weights()
+    pipe = moe.HostPipeline(T, DEV, depth)
+    toks = [synth.make_tokens(T, 300 + k) for k in range(6)]
+    bias = torch.from_numpy(toks[0].bias).to(DEV)
+    hosts = []
+    for tok in toks:
+        x_h = torch.from_numpy(tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        lg_h = torch.from_numpy(tok.logits).pin_memory()
+        out_h = torch.full((T, 1536), float("nan"), dtype=torch.bfloat16).pin_memory()
+        hosts.append((x_h, lg_h, out_h))
+    for x_h, lg_h, out_h in hosts:
+        pipe.submit(x_h, lg_h, out_h, bias, W.packed)
+    pipe.drain()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    for tok, (x_h, lg_h, out_h) in zip(toks, hosts):
+        x, lg, _ = tokens_dev(tok)
+        ref = moe.moe_layer(x, lg, bias, W.packed)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h.view(torch.int16), ref.cpu().view(torch.int16))
