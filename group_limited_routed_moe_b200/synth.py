@@ -21,6 +21,15 @@ single expert: a 32-bit integer hash of (seed, layer, matrix, expert, element)
 picks one of 65,536 normal quantiles Phi^-1((k + 1/2) / 65536), scaled by
 0.02 and rounded once to bf16.  After bf16 rounding this is indistinguishable
 from N(0, 0.02) except that the tails are cut at 4.33 sigma.
+
+Block-FP8 expert weights (the synthetic counterpart of a block-FP8
+checkpoint) are those bf16 weights written the way such a file is written:
+per 128 x 128 block a scale s, and every weight stored as the FP8 E4M3 code
+nearest to w / s (round to nearest even, by PyTorch's float8_e4m3fn cast).
+Scale modes: "pow2" takes the smallest power of two with max|w| <= 448 s (the
+power-of-two block scales of UE8M0-style checkpoints); "amax" takes
+s = fp32(max|w| / 448).  This is input synthesis: the layer only reads codes
+and scales.
 """
 
 from __future__ import annotations
@@ -157,6 +166,66 @@ def weight_bits_torch(seed: int, layer: int, which: int, device, out=None):
         u = _mix32_torch(_mix32_torch(i ^ k1t[e0:e0 + step]) ^ k2t[e0:e0 + step])
         flat[e0:e0 + step].copy_(table[u >> 16])
     return out
+
+
+# ----------------------------------------------------------------------------
+# block-FP8 expert weights
+# ----------------------------------------------------------------------------
+
+FP8_BLOCK = 128
+FP8_MAX = 448.0
+
+
+def _quantize_block_fp8(w, mode: str):
+    """torch float32 [n, R, C] -> (uint8 codes [n, R, C], fp32 scales [n, R/128, C/128])."""
+    import torch
+    n, R, C = w.shape
+    blk = w.reshape(n, R // FP8_BLOCK, FP8_BLOCK, C // FP8_BLOCK, FP8_BLOCK)
+    amax = blk.abs().amax(dim=(2, 4))
+    if mode == "pow2":
+        # smallest e with amax <= 448 * 2**e; amax = m * 2**k, 0.5 <= m < 1, 448 = 0.875 * 2**9
+        m, k = torch.frexp(amax)
+        e = k - 9 + (m > 0.875).to(k.dtype)
+        scale = torch.ldexp(torch.ones_like(amax), e)
+    elif mode == "amax":
+        scale = amax / FP8_MAX
+    else:
+        raise ValueError(f"unknown scale mode {mode!r}")
+    scale = torch.where(amax > 0, scale, torch.ones_like(scale)).to(torch.float32)
+    q = (blk / scale[:, :, None, :, None]).to(torch.float8_e4m3fn)
+    return q.reshape(n, R, C).view(torch.uint8), scale
+
+
+def fp8_weights_np(seed: int, layer: int, which: int, experts=None, mode: str = "pow2"):
+    """Block-FP8 form of expert matrix ``which`` of ``layer`` on the host:
+    (codes uint8 [len(experts), R, C], scales float32 [len(experts), R/128, C/128])."""
+    import torch
+    bits = weight_bits_np(seed, layer, which, experts)
+    w = (torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)).to(torch.float32)
+    q, s = _quantize_block_fp8(w, mode)
+    return q.numpy(), s.numpy()
+
+
+def fp8_weights_torch(seed: int, layer: int, which: int, device, mode: str = "pow2"):
+    """Same bytes as ``fp8_weights_np`` for all 128 experts, made on ``device``."""
+    import torch
+    w = weight_bits_torch(seed, layer, which, device)
+    codes = torch.empty(w.shape, dtype=torch.uint8, device=device)
+    scales = []
+    for e0 in range(0, N_EXPERTS, 16):  # bounded float32 temporaries
+        q, s = _quantize_block_fp8(w[e0:e0 + 16].to(torch.float32), mode)
+        codes[e0:e0 + 16].copy_(q)
+        scales.append(s)
+    return codes, torch.cat(scales)
+
+
+def fp8_scale_jitter(shape, seed: int) -> np.ndarray:
+    """Per-block factors 2**j, j uniform in {-2, ..., 2}, from PCG64(seed):
+    multiplied into power-of-two scales they give blocks of different scales
+    (the generator's own scales are nearly uniform, since every block of
+    N(0, 0.02) weights has about the same max |w|)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 77])))
+    return np.exp2(rng.integers(-2, 3, size=shape)).astype(np.float32)
 
 
 # ----------------------------------------------------------------------------

@@ -38,6 +38,10 @@ reordering beyond what the definition states:
   rows, which the CUDA path must reproduce bit for bit.
 * Stack: 23 MoE layers (24 layers with dense layer 0 -- issue #1247, opening
   paragraph), residual stream kept in bf16: h <- bf16(h + moe(h)).
+* Block-FP8 experts (issue #1247, "What it does not cover", third bullet: the
+  CUDA path reads bf16, block FP8 and NVFP4 experts): E4M3 codes with one fp32
+  scale per 128 x 128 block, weight = value(code) * scale; the layer is the
+  definition above with those weights (``moe_layer_fp8``).
 
 Every function is pinned by tests in ``tests/test_oracle_*.py`` against
 brute force, closed forms and invariants (see each test's docstring).
@@ -295,6 +299,89 @@ def moe_stack(x_bits: np.ndarray, layers) -> np.ndarray:
         upd = moe_layer(h, lg, b, wg, wu, wd)
         h = f64_to_bf16_bits(bf16_bits_to_f64(h) + upd)
     return h
+
+
+# ----------------------------------------------------------------------------
+# Block-FP8 expert weights
+# ----------------------------------------------------------------------------
+# The CUDA path of "Ling-3.0-tiny on a Qualcomm board" (TensorFold issue
+# #1247, first comment, "What it does not cover", third bullet) reads expert
+# weights in bf16, in block FP8 and in NVFP4, and the issue mentions an
+# official FP8 release of tiny.  The pages do not spell the block-FP8 format
+# out; the reading here is the usual one for block-FP8 checkpoints: every
+# weight is an FP8 E4M3 code (OCP 8-bit floating point, the "FN" variant
+# without infinities), and every 128 x 128 block of a matrix carries one fp32
+# scale, the weight being  value(code) * scale  exactly.  The layer is then the
+# bf16 layer's definition with those weights.
+
+FP8_BLOCK = 128
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Exact value of FP8 E4M3 codes (uint8) as float64.
+
+    Bit 7 is the sign, bits 6..3 the exponent field E (bias 7), bits 2..0 the
+    mantissa m.  E = 0 encodes the subnormals m/8 * 2**-6; otherwise the value
+    is (1 + m/8) * 2**(E - 7).  The two codes with every exponent and mantissa
+    bit set (0x7F, 0xFF) are NaN; there are no infinities, so the largest
+    finite magnitude is 1.75 * 2**8 = 448.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c & 0x80) != 0, -1.0, 1.0)
+    E = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(E == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(E - 7.0))
+    v = sign * mag
+    return np.where((c & 0x7F) == 0x7F, np.nan, v)
+
+
+def dequant_block_fp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Weights of a block-FP8 matrix (or stack of matrices) in float64.
+
+    codes [..., R, C] uint8 E4M3 codes; scales [..., R/128, C/128] fp32, one per
+    128 x 128 block.  W[..., r, c] = value(codes[..., r, c]) * scales[..., r // 128,
+    c // 128], exact in float64 (a 4-bit significand times a 24-bit one).
+    """
+    v = e4m3_to_f64(codes)
+    s = np.asarray(scales, dtype=np.float64)
+    R, C = v.shape[-2:]
+    if s.shape[-2:] != (R // FP8_BLOCK, C // FP8_BLOCK) or R % FP8_BLOCK or C % FP8_BLOCK:
+        raise ValueError(f"scales {s.shape} do not tile codes {v.shape} in {FP8_BLOCK}-blocks")
+    full = np.repeat(np.repeat(s, FP8_BLOCK, axis=-2), FP8_BLOCK, axis=-1)
+    return v * full
+
+
+def moe_layer_f64(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | None,
+                  expert_weights, route_result: RouteResult | None = None) -> np.ndarray:
+    """The routed layer of ``moe_layer`` with float64 expert weights.
+
+    ``expert_weights(e)`` returns (W_gate [H, I], W_up [H, I], W_down [I, H]) of
+    expert e in float64; it is called once for every expert some token uses.
+    """
+    rr = route_result if route_result is not None else route(logits, bias)
+    x = bf16_bits_to_f64(x_bits)
+    out = np.zeros((x.shape[0], HIDDEN), dtype=np.float64)
+    for e in np.unique(rr.topk_idx):
+        tok, slot = np.nonzero(rr.topk_idx == e)
+        wg, wu, wd = expert_weights(int(e))
+        out[tok] += rr.topk_w[tok, slot][:, None] * expert_ffn(x[tok], wg, wu, wd)
+    return out
+
+
+def moe_layer_fp8(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | None,
+                  q_gate: np.ndarray, s_gate: np.ndarray, q_up: np.ndarray, s_up: np.ndarray,
+                  q_down: np.ndarray, s_down: np.ndarray,
+                  route_result: RouteResult | None = None) -> np.ndarray:
+    """Routed layer with block-FP8 experts, float64, no intermediate rounding.
+
+    q_gate, q_up: [E, 1536, 512] uint8 codes, s_gate, s_up: [E, 12, 4] fp32;
+    q_down: [E, 512, 1536] codes, s_down: [E, 4, 12].  Only the experts that
+    some token uses are read.
+    """
+    def weights(e):
+        return (dequant_block_fp8(q_gate[e], s_gate[e]), dequant_block_fp8(q_up[e], s_up[e]),
+                dequant_block_fp8(q_down[e], s_down[e]))
+    return moe_layer_f64(x_bits, logits, bias, weights, route_result)
 
 
 def rel_l2(a: np.ndarray, ref: np.ndarray) -> float:

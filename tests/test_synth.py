@@ -45,3 +45,31 @@ def test_bf16_packing_round_nearest_even():
     r = np.random.default_rng(0).standard_normal(10000).astype(np.float32)
     ref = torch.from_numpy(r).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(S.f32_to_bf16_bits(r), ref)
+
+
+def test_fp8_weights_are_block_quantised_bf16_weights():
+    """The synthetic FP8 checkpoint: power-of-two scales with max|w| in
+    (224 s, 448 s], no NaN code, and every code the E4M3 value nearest to w/s
+    (the dequantised weight is within half an E4M3 spacing of w); the "amax"
+    mode puts a code of magnitude 448 into every block."""
+    w = S.weight_bits_np(0, 2, S.W_DOWN, experts=[5])
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)[0]
+    q, s = S.fp8_weights_np(0, 2, S.W_DOWN, experts=[5])
+    assert q.shape == (1, 512, 1536) and q.dtype == np.uint8 and s.shape == (1, 4, 12)
+    assert np.all((q & 0x7F) != 0x7F)
+    m, _ = np.frexp(s)
+    assert np.all(m == 0.5)                                   # powers of two
+    amax = np.abs(wf).reshape(4, 128, 12, 128).max(axis=(1, 3))
+    assert np.all(amax <= 448 * s[0]) and np.all(amax > 224 * s[0])
+    v = torch.from_numpy(q[0]).view(torch.float8_e4m3fn).double().numpy()
+    full_s = np.repeat(np.repeat(s[0].astype(np.float64), 128, 0), 128, 1)
+    a = np.abs(wf / full_s)
+    # spacing of E4M3 around |a|: 2**-9 below 2**-6, else 2**(floor(log2 a) - 3)
+    spacing = np.where(a < 2.0 ** -6, 2.0 ** -9, np.exp2(np.floor(np.log2(np.maximum(a, 2.0 ** -6))) - 3))
+    assert np.all(np.abs(v - wf / full_s) <= spacing / 2)
+    q2, s2 = S.fp8_weights_np(0, 2, S.W_DOWN, experts=[5], mode="amax")
+    assert np.allclose(s2[0], (amax / 448).astype(np.float32), rtol=0, atol=0)
+    blocks = (q2[0] & 0x7F).reshape(4, 128, 12, 128).max(axis=(1, 3))
+    assert np.all(blocks == 0x7E)
+    j = S.fp8_scale_jitter((3, 12, 4), 1)
+    assert set(np.log2(j).ravel().tolist()) <= {-2.0, -1.0, 0.0, 1.0, 2.0}
