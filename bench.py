@@ -50,6 +50,8 @@ from group_limited_routed_moe_b200 import synth  # noqa: E402
 
 GATE_UP_BYTES_PER_EXPERT = 2 * 1536 * 512 * 2
 DOWN_BYTES_PER_EXPERT = 1536 * 512 * 2
+# block-FP8 expert: one byte per weight, one fp32 scale per 128 x 128 block
+FP8_BYTES_PER_EXPERT = 3 * 1536 * 512 + (2 * 12 * 4 + 4 * 12) * 4
 FLOPS_PER_ROW = 2 * (1536 * 1024 + 512 * 1536)          # one (token, expert) pair
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -61,7 +63,11 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_T8189", choices=["prefill_T8189", "decode_T16"])
-    ap.add_argument("--no-secondary", action="store_true", help="skip the decode_T16 measurement")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weights of the main line: bf16, or block FP8 (E4M3 codes, "
+                         "power-of-two 128x128 block scales)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the decode_T16 (bf16 and FP8) measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens in the oracle sample")
     return ap.parse_args()
@@ -75,7 +81,7 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-GEMM_SOURCES = ("common.cuh", "expert_ffn.cuh", "expert_ffn_skinny.cuh")
+GEMM_SOURCES = ("common.cuh", "expert_ffn.cuh", "expert_ffn_skinny.cuh", "fp8.cuh")
 
 
 def kernel_source_sha():
@@ -161,10 +167,11 @@ class ClockSampler:
 class LayerRun:
     """Device buffers and the five-call step of one workload."""
 
-    def __init__(self, wl: synth.Workload, dev, weights):
+    def __init__(self, wl: synth.Workload, dev, weights, fp8: bool = False):
         import torch
         from group_limited_routed_moe_b200 import moe
         self.moe, self.torch, self.wl, self.dev = moe, torch, wl, dev
+        self.fp8 = fp8  # weights: a packed block-FP8 layer (moe_layer_fp8)
         self.T = wl.T
         tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
         self.tok = tok
@@ -196,9 +203,13 @@ class LayerRun:
         nb = (T + 127) // 128
         n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
         self.launches_per_step = n_rp + 2  # + the expert FFN (one launch) + combine
+        fws = moe.lib.moe_expert_ffn_fp8_workspace_bytes(T) if fp8 else 0
+        self.ffn_ws = torch.empty(fws, dtype=torch.uint8, device=dev) if fws else None
+        if fws:
+            self.launches_per_step += 1  # FP8 above 256 tokens: the expansion pass
         # the breakdown pass times the same kernels the layer call runs
         self.part_names = ["route", "permute", "expert_ffn", "combine"]
-        self.lws = moe.alloc_layer_workspace(T, dev)
+        self.lws = moe.alloc_layer_workspace(T, dev, fp8=fp8)
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
         self.write_only_flush = False
@@ -216,8 +227,9 @@ class LayerRun:
 
     def step(self):
         """One layer through the public layer call (what a user runs)."""
-        self.moe.moe_layer(self.x[:self.T], self.logits[:self.T], self.bias, self.packed,
-                           out=self.out[:self.T], workspace=self.lws, stream=self.stream)
+        layer = self.moe.moe_layer_fp8 if self.fp8 else self.moe.moe_layer
+        layer(self.x[:self.T], self.logits[:self.T], self.bias, self.packed,
+              out=self.out[:self.T], workspace=self.lws, stream=self.stream)
 
     def step_parts(self, ev):
         """The same layer through the step calls, with an event between each."""
@@ -230,8 +242,12 @@ class LayerRun:
         m.moe_permute(self.idx, self.counts, self.offsets, self.perm_src, self.inv_perm,
                       self.pws, stream=s)
         rec()
-        m.moe_expert_ffn(self.x[:T], self.packed, self.offsets, self.perm_src, self.h, self.y,
-                         stream=s)
+        if self.fp8:
+            m.moe_expert_ffn_fp8(self.x[:T], self.packed, self.offsets, self.perm_src, self.h,
+                                 self.y, workspace=self.ffn_ws, stream=s)
+        else:
+            m.moe_expert_ffn(self.x[:T], self.packed, self.offsets, self.perm_src, self.h,
+                             self.y, stream=s)
         rec()
         m.moe_combine(self.y, self.w, self.inv_perm, out=self.out[:T], stream=s)
         rec()
@@ -314,16 +330,17 @@ class LayerRun:
         """The fused moe_layer call captured once in a CUDA graph and replayed."""
         torch, moe = self.torch, self.moe
         T = self.T
-        ws = moe.alloc_layer_workspace(T, self.dev)
+        ws = moe.alloc_layer_workspace(T, self.dev, fp8=self.fp8)
+        layer = moe.moe_layer_fp8 if self.fp8 else moe.moe_layer
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            moe.moe_layer(self.x[:T], self.logits[:T], self.bias, self.packed, out=self.out[:T],
-                          workspace=ws, stream=s)
+            layer(self.x[:T], self.logits[:T], self.bias, self.packed, out=self.out[:T],
+                  workspace=ws, stream=s)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                moe.moe_layer(self.x[:T], self.logits[:T], self.bias, self.packed,
-                              out=self.out[:T], workspace=ws, stream=s)
+                layer(self.x[:T], self.logits[:T], self.bias, self.packed, out=self.out[:T],
+                      workspace=ws, stream=s)
         torch.cuda.synchronize()
         cur = torch.cuda.current_stream()
         for _ in range(warmup):
@@ -354,7 +371,7 @@ class LayerRun:
         x_h = torch.from_numpy(self.tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
         lg_h = torch.from_numpy(self.tok.logits).pin_memory()
         outs_h = [torch.empty((T, 1536), dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
-        pipe = moe.HostPipeline(T, self.dev, depth)
+        pipe = moe.HostPipeline(T, self.dev, depth, fp8=self.fp8)
 
         def run(n):
             for k in range(n):
@@ -406,16 +423,31 @@ def roofline_for(wl, run, per_ms, peaks, peak_kind):
     weights, x read, y_perm written)."""
     T = wl.T
     ffn_ms = float(per_ms[:, run.part_names.index("expert_ffn")].mean())
+    if run.fp8 and T <= 256:
+        # block-FP8 codes and scales of the touched experts, x read, y_perm written
+        d = distinct_experts(run)
+        nbytes = d * FP8_BYTES_PER_EXPERT + T * 1536 * 2 + 8 * T * 1536 * 2
+        peak = float(peaks["hbm_gbs"])
+        achieved = nbytes / (ffn_ms * 1e-3) / 1e9
+        return {"kernel": "skinny_gemm_kernel<3, fp8> (E4M3 codes dequantised in shared memory; "
+                          "gate/up + SwiGLU + down in one launch)",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_per_launch": nbytes, "distinct_experts": d,
+                "traffic": profiled_traffic("expert_ffn_fp8", wl.name)}
     if T >= 2048:
         flops = FLOPS_PER_ROW * 8 * T
         key = "bf16_tflops"
         peak = float(peaks[key])
         achieved = flops / (ffn_ms * 1e-3) / 1e12
-        return {"kernel": "ffn_gemm_kernel<3> (gate/up + SwiGLU + down in one launch)",
+        kernel = "ffn_gemm_kernel<3> (gate/up + SwiGLU + down in one launch)"
+        if run.fp8:
+            kernel = "dequant_fp8_kernel + " + kernel + ", timed together"
+        return {"kernel": kernel,
                 "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_kind} {key} (burst)", "algorithmic_per_launch": flops,
-                "traffic": profiled_traffic("expert_ffn", wl.name)}
+                "traffic": None if run.fp8 else profiled_traffic("expert_ffn", wl.name)}
     d = distinct_experts(run)
     nbytes = (d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * 1536 * 2
               + 8 * T * 1536 * 2)
@@ -434,7 +466,8 @@ def layer_fractions(wl, run, step_ms, per_ms, peaks):
     distinct experts' weights and against the tensor bound of the useful flops."""
     layer_s = float(step_ms.mean()) * 1e-3
     d = distinct_experts(run)
-    nbytes = d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + wl.T * (1536 * 4 + 512)
+    per_expert = FP8_BYTES_PER_EXPERT if run.fp8 else GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT
+    nbytes = d * per_expert + wl.T * (1536 * 4 + 512)
     flops = FLOPS_PER_ROW * 8 * wl.T
     return {"layer_us": round(layer_s * 1e6, 2),
             "hbm_frac": round(nbytes / layer_s / 1e9 / float(peaks["hbm_gbs"]), 4),
@@ -445,17 +478,65 @@ def layer_fractions(wl, run, step_ms, per_ms, peaks):
             "distinct_experts": d}
 
 
-def cpu_baseline(wl, tok, host_w, sample):
+def cpu_baseline(wl, tok, host_w, sample, fp8=False):
+    """The float64 oracle on the first `sample` tokens.  host_w: bf16 bits
+    (W_gate, W_up, W_down), or with fp8 the codes and scales (q_gate, s_gate,
+    q_up, s_up, q_down, s_down)."""
     import oracle as O
     from threadpoolctl import threadpool_info
     n = min(sample, wl.T)
     rows = np.arange(n)
     t0 = time.perf_counter()
-    O.moe_layer(tok.x_bits[rows], tok.logits[rows], tok.bias, *host_w)
+    (O.moe_layer_fp8 if fp8 else O.moe_layer)(tok.x_bits[rows], tok.logits[rows], tok.bias,
+                                              *host_w)
     dt = time.perf_counter() - t0
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {n} of {wl.T} tokens of {wl.name}, float64 NumPy oracle, {dt:.2f} s"}
+            "sample": (f"first {n} of {wl.T} tokens of {wl.name}"
+                       f"{' (block-FP8 experts)' if fp8 else ''}, float64 NumPy oracle, {dt:.2f} s")}
+
+
+def decode_line(wl2, dev, packed, fp8, steps, warmup, peaks, peak_kind, barrier):
+    """The decode batch measured beside the main line: whole-layer steps,
+    breakdown and roofline, router, CUDA-graph replay, end to end."""
+    run2 = LayerRun(wl2, dev, packed, fp8=fp8)
+    clk2 = ClockSampler(int(dev.index or 0))
+    n = max(steps, 50)
+    with clk2:
+        steps2, _ = run2.timed(n, warmup, barrier)
+    per2 = run2.breakdown(n)
+    dirty2 = run2.dirty_l2_steps(n, barrier)
+    e2e2, h2d2, d2h2 = run2.e2e(40, 3)
+    graph_us = run2.graph_layer_us(50, 3)
+    ms2 = float(steps2.mean())
+    out = {
+        "value": round(wl2.T / (ms2 * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms2, 5),
+        "roofline": roofline_for(wl2, run2, per2, peaks, peak_kind)}
+    if not fp8:
+        out["router"] = run2.router(20, peaks)
+    out.update({
+        "layer": dict(layer_fractions(wl2, run2, steps2, per2, peaks),
+                      layer_us_after_write_only_flush=round(dirty2 * 1e3, 2)),
+        "graph_replay": {"layer_us": round(graph_us, 2),
+                         "value": round(wl2.T / (graph_us * 1e-6), 1), "unit": "tokens/s"},
+        "e2e": {"value": round(wl2.T / (e2e2 * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(e2e2, 4), "h2d_bytes_per_step": h2d2,
+                "d2h_bytes_per_step": d2h2, "in_flight": 3},
+        "gpu_launches": run2.launches_per_step * n,
+        "clocks": clk2.summary()})
+    return out
+
+
+def fp8_layer(dev):
+    """The synthetic block-FP8 checkpoint of layer 0 (power-of-two block scales),
+    packed, and its host codes and scales."""
+    from group_limited_routed_moe_b200 import moe
+    qs = []
+    for which in (synth.W_GATE, synth.W_UP, synth.W_DOWN):
+        q, sc = synth.fp8_weights_torch(0, 0, which, dev, "pow2")
+        qs += [q, sc]
+    packed = moe.moe_pack_weights_fp8(*qs)
+    return packed, qs
 
 
 def run_ours(args):
@@ -489,8 +570,12 @@ def run_ours(args):
             return t.view(torch.int16).cpu().numpy().view(np.uint16)
         return h(wg), h(wu), h(wd)
 
+    fp8_packed, fp8_dev = fp8_layer(dev) if (args.weights == "fp8" or not args.no_secondary) \
+        else (None, None)
+    torch.cuda.synchronize()
+    fp8 = args.weights == "fp8"
     wl = synth.WORKLOADS[args.workload]
-    run = LayerRun(wl, dev, packed)
+    run = LayerRun(wl, dev, fp8_packed if fp8 else packed, fp8=fp8)
     clk = ClockSampler(local)
     with clk:
         steps_ms, wall = run.timed(args.steps, args.warmup, barrier)
@@ -509,6 +594,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "T_buf": wl.T_buf, "hidden": 1536,
+                   "weights": ("block-FP8 experts (E4M3 codes, power-of-two 128x128 block scales)"
+                               if fp8 else "bf16 experts"),
                    "experts": 128, "groups": 8, "keep_groups": 4, "topk": 8, "inter": 512,
                    "parallelism": f"dp{world} (independent batch per GPU)",
                    "l2": ("256 MB buffer overwritten, then another 256 MB buffer read, before "
@@ -529,34 +616,20 @@ def run_ours(args):
         "gpu_launches": run.launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-    if not args.no_secondary and wl.name != "decode_T16":
+    if not args.no_secondary:
         wl2 = synth.WORKLOADS["decode_T16"]
-        run2 = LayerRun(wl2, dev, packed)
-        clk2 = ClockSampler(local)
-        with clk2:
-            steps2, wall2 = run2.timed(max(args.steps, 50), args.warmup, barrier)
-        per2 = run2.breakdown(max(args.steps, 50))
-        dirty2 = run2.dirty_l2_steps(max(args.steps, 50), barrier)
-        router2 = run2.router(20, peaks)
-        e2e2, h2d2, d2h2 = run2.e2e(40, 3)
-        graph_us = run2.graph_layer_us(50, 3)
-        ms2 = float(steps2.mean())
-        line["decode_T16"] = {
-            "value": round(wl2.T / (ms2 * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms2, 5),
-            "roofline": roofline_for(wl2, run2, per2, peaks, peak_kind),
-            "router": router2,
-            "layer": dict(layer_fractions(wl2, run2, steps2, per2, peaks),
-                          layer_us_after_write_only_flush=round(dirty2 * 1e3, 2)),
-            "graph_replay": {"layer_us": round(graph_us, 2),
-                             "value": round(wl2.T / (graph_us * 1e-6), 1), "unit": "tokens/s"},
-            "e2e": {"value": round(wl2.T / (e2e2 * 1e-3), 1), "unit": "tokens/s",
-                    "ms_per_step": round(e2e2, 4), "h2d_bytes_per_step": h2d2,
-                    "d2h_bytes_per_step": d2h2, "in_flight": 3},
-            "gpu_launches": run2.launches_per_step * max(args.steps, 50),
-            "clocks": clk2.summary()}
-        line["gpu_launches"] += line["decode_T16"]["gpu_launches"]
+        for key, p2, f2 in (("decode_T16", packed, False), ("decode_T16_fp8", fp8_packed, True)):
+            if wl2.name == wl.name and f2 == fp8:
+                continue  # that is the main line
+            line[key] = decode_line(wl2, dev, p2, f2, args.steps, args.warmup, peaks, peak_kind,
+                                    barrier)
+            line["gpu_launches"] += line[key]["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, run.tok, host_weights(), args.cpu_sample)
+        if fp8:
+            hw = [t.cpu().numpy() for t in fp8_dev]
+        else:
+            hw = host_weights()
+        line["cpu_baseline"] = cpu_baseline(wl, run.tok, hw, args.cpu_sample, fp8=fp8)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

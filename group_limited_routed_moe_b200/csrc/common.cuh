@@ -36,6 +36,7 @@ enum StatusSite : unsigned {
   kSiteFfnDrain = 20,
   kSiteTileQueue = 21,
   kSiteFfnDone = 22,  // a down tile waiting for its expert's gate/up tiles
+  kSiteFp8Nan = 23,   // a NaN E4M3 code in packed block-FP8 weights
   kSiteSelftest = 30,
 };
 
@@ -157,6 +158,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), completing on `bar` like a TMA load.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -190,6 +202,49 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand read from tensor memory
+// (row i of A in lane i, consecutive K elements packed two per 32-bit column),
+// B from a shared-memory descriptor; 16-bit inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Eight MMAs over K = 128 with A in tensor memory (columns a_tmem + 8k) and B
+// as two 64-wide SW128 tiles (descriptors b0 for k < 4, b1 for k >= 4, each
+// advanced by 32 bytes per k); the first accumulates into D only if
+// `accumulate`, the other seven always.
+__device__ __forceinline__ void umma_f16_ta_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                                 uint64_t b1, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "setp.eq.b32 q, %5, %5;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
+      "add.u32 a, %1, 8;\n\tadd.u64 b, %2, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
+      "add.u32 a, %1, 16;\n\tadd.u64 b, %2, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
+      "add.u32 a, %1, 24;\n\tadd.u64 b, %2, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
+      "add.u32 a, %1, 32;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %3, %4, q;\n\t"
+      "add.u32 a, %1, 40;\n\tadd.u64 b, %3, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
+      "add.u32 a, %1, 48;\n\tadd.u64 b, %3, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
+      "add.u32 a, %1, 56;\n\tadd.u64 b, %3, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -259,6 +314,24 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&a)[32]) {
         "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
       : "r"(taddr)
       : "memory");
+}
+
+// Stores 32 consecutive 32-bit columns of the calling warp's 32 TMEM lanes
+// (one lane per thread), asynchronously: tmem_wait_st() waits for them.
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* a) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+      "r"(a[8]), "r"(a[9]), "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]),
+      "r"(a[15]), "r"(a[16]), "r"(a[17]), "r"(a[18]), "r"(a[19]), "r"(a[20]), "r"(a[21]),
+      "r"(a[22]), "r"(a[23]), "r"(a[24]), "r"(a[25]), "r"(a[26]), "r"(a[27]), "r"(a[28]),
+      "r"(a[29]), "r"(a[30]), "r"(a[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Barrier among `nthreads` threads (multiple of 32) of the block, id 1..15.

@@ -33,9 +33,24 @@
 // cp.async of x rows by perm_src, barrier-tracked; padding rows kept at zero),
 // 5 TMA producer, 6 MMA issuer.  Accumulators: 2 x 32 TMEM columns.  Every
 // wait, including the up -> gate hand-off, is a bounded mbarrier wait.
+//
+// Block-FP8 weights (WQ = true, MODE 3 only): the weight stream is 8-bit E4M3
+// codes, half the bytes.  A stage covers K = 128 (one scale block): the TMA
+// brings 128 rows x 128 codes (16 KB, 128-byte swizzle) into an 8-stage ring
+// that also takes the stage's token rows (two 64-wide SW128 tiles, gathered x
+// or TMA'd h, as above).  Converter warps, one thread per weight row,
+// dequantise a row's 128 codes with the block's scale and store the 64
+// columns of bf16 (gate/up) or fp16 (down) pairs straight into tensor memory,
+// in one of 4 operand slots; the MMA then reads A from tensor memory and B
+// (the token rows) from the ring, 8 instructions per stage.  The weights never
+// make a second trip through shared memory, no proxy fence sits between the
+// converters and the tensor core, and the single issuing thread handles half
+// as many stages per weight byte as with 64-wide stages (its per-stage
+// barrier round trips, not the MMAs, bound a skinny GEMM).
 #pragma once
 #include "common.cuh"
 #include "expert_ffn.cuh"
+#include "fp8.cuh"
 
 namespace moe {
 namespace skinny {
@@ -53,11 +68,45 @@ constexpr int XSTRIDE = BNT + 1;  // floats per row of the up-value exchange til
 constexpr int XCHG_BYTES = 64 * XSTRIDE * 4;
 constexpr int THREADS = 224;
 constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;
+constexpr int CONV_WARP0 = 7;  // block-FP8: converter warps 7 .. 7 + NCONV - 1
+constexpr int kConvGroups = 2;  // block-FP8: converter warps per tensor-memory lane quarter
+
+// Ring geometry.  bf16 weights: STAGES x (16 KB weights + 4 KB tokens) of
+// K = 64, two 32-column accumulators in tensor memory.  Block-FP8 weights:
+// RSTAGES x (16 KB codes + 8 KB tokens + the tile's block scales, 1 KB
+// reserved) of K = 128 in the same 200 KB, and tensor memory also holds NA
+// dequantised 128 x 128 weight tiles (64 columns each) after the accumulators.
+constexpr int kMaxStages = 10;
+template <bool WQ>
+struct Ring {
+  static constexpr int KS = WQ ? 128 : BK;                // K per stage
+  static constexpr int RA_BYTES = WQ ? BMW * KS : A_BYTES;  // codes or operands
+  static constexpr int RB_BYTES = BNT * KS * 2;             // token rows
+  static constexpr int RSC_BYTES = WQ ? 1024 : 0;           // block scales of the tile
+  static constexpr int RSTAGE_BYTES = RA_BYTES + RB_BYTES + RSC_BYTES;
+  static constexpr int RSTAGES = WQ ? 8 : STAGES;
+  static constexpr int BYTES = RSTAGES * RSTAGE_BYTES;
+  static constexpr int NA = WQ ? 4 : 0;
+  static constexpr int A_COLS = KS / 2;  // 32-bit columns of one operand slot
+  static constexpr int A_COL0 = 2 * BNT;
+  static constexpr int TMEM_COLS = WQ ? 512 : 2 * BNT;
+  static constexpr int NCONV = WQ ? 4 * kConvGroups : 0;
+  static constexpr int THREADS = skinny::THREADS + 32 * NCONV;
+};
+static_assert(Ring<true>::BYTES <= TILE_BYTES, "the FP8 ring must fit the bf16 ring's space");
+static_assert(Ring<true>::RSTAGES <= kMaxStages && Ring<false>::RSTAGES <= kMaxStages, "stages");
+static_assert(Ring<true>::RSTAGE_BYTES % 1024 == 0 && Ring<true>::RA_BYTES % 1024 == 0,
+              "SW128 tiles must stay 1024-byte aligned in the ring");
+static_assert(Ring<true>::A_COL0 + Ring<true>::A_COLS * Ring<true>::NA <= Ring<true>::TMEM_COLS,
+              "operand slots must fit the tensor-memory allocation");
+static_assert(Ring<true>::RSTAGES % Ring<true>::NA == 0, "slot reuse follows the ring");
 
 // Per-phase constants.  Phase 1: 8 weight blocks per 32-token chunk (4 pairs
 // x 2 halves of 64 gate + 64 up rows), K = 1536; phase 2: 12 blocks, K = 512.
 __host__ __device__ constexpr int fblk(int phase) { return phase == 1 ? 8 : kH / BMW; }
-__host__ __device__ constexpr int kblocks(int phase) { return (phase == 1 ? kH : kI) / BK; }
+__host__ __device__ constexpr int kblocks(int phase, int ks = BK) {
+  return (phase == 1 ? kH : kI) / ks;
+}
 constexpr uint32_t kIdesc1 = idesc_f32acc(BMW, BNT, kFmtBF16);
 constexpr uint32_t kIdesc2 = idesc_f32acc(BMW, BNT, kFmtF16);
 // Counter increments a gate/up tile makes when its h values are stored (one per
@@ -65,10 +114,11 @@ constexpr uint32_t kIdesc2 = idesc_f32acc(BMW, BNT, kFmtF16);
 constexpr int kDoneStep = 2;
 
 struct Tail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t afull[4];  // block-FP8: operand slot written (one arrival per lane quarter)
   uint64_t xfull;   // up half written to the exchange tile (64 lane arrivals)
   uint64_t xempty;  // gate half done reading it (64 lane arrivals)
   uint64_t drain;
@@ -112,16 +162,23 @@ __device__ __forceinline__ TileInfo tile_info(const Tail* S, int tile, int total
   return t;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int MODE, bool WQ = false>
+__global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w1,  // gate/up weights (phase 1)
                        const __grid_constant__ CUtensorMap tmap_w2,  // down weights (phase 2)
                        const __grid_constant__ CUtensorMap tmap_h,   // h rows (phase 2)
                        const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                        const int32_t* __restrict__ perm_src, int64_t T,
                        uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
-                       int* __restrict__ sched, int* __restrict__ done, uint64_t timeout_ns) {
+                       int* __restrict__ sched, int* __restrict__ done,
+                       const float* __restrict__ wscale,  // block-FP8 scales (SGU, then SD)
+                       uint64_t timeout_ns) {
   constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
+  static_assert(!WQ || MODE == 3, "block-FP8 weights only in the single-launch form");
+  using R = Ring<WQ>;
+  constexpr int RST = R::RSTAGES;
+  constexpr int NA = R::NA > 0 ? R::NA : 1;
+  constexpr int KS = R::KS;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -135,14 +192,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nrows = T * kTopK;
   griddep_launch_dependents();
-  auto sA = [&](int s) { return smem + s * STAGE_BYTES; };
-  auto sB = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+  auto sA = [&](int s) { return smem + s * R::RSTAGE_BYTES; };
+  auto sB = [&](int s) { return smem + s * R::RSTAGE_BYTES + R::RA_BYTES; };
+  auto sC = [&](int s) { return sB(s) + R::RB_BYTES; };  // block-FP8: the tile's scales
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < RST; ++s) {
       mbar_init(&fullb[s], HAS1 ? 1 + 32 : 1);  // TMA arrive (+ 32 gather lanes)
-      mbar_init(&emptyb[s], 1);
+      mbar_init(&emptyb[s], 1);                  // MMA commit
     }
+    for (int a = 0; a < R::NA; ++a) mbar_init(&S->afull[a], 4);  // one warp per lane quarter
     for (int a = 0; a < 2; ++a) {
       mbar_init(&S->tfull[a], 1);
       mbar_init(&S->tempty[a], 4);
@@ -150,7 +209,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&S->xfull, 64);
     mbar_init(&S->xempty, 64);
     mbar_init(&S->drain, 1);
-    tileq_init(&S->tq, (HAS1 ? 1 : 0) + 1 + 4);  // gather warp, MMA thread, epilogue warps
+    // gather warp, MMA thread, epilogue warps, converter warps
+    tileq_init(&S->tq, (HAS1 ? 1 : 0) + 1 + 4 + R::NCONV);
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -184,7 +244,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane >= o) incl += v;
   }
   if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
-  if (warp == MMA_WARP) tmem_alloc(&S->tmem_base, TMEM_COLS);
+  if (warp == MMA_WARP) tmem_alloc(&S->tmem_base, R::TMEM_COLS);
   __syncthreads();
   if (threadIdx.x < kE) {
     int base = 0;
@@ -234,15 +294,32 @@ __global__ void __launch_bounds__(THREADS, 1)
           wrow0 = e * kH + f * BMW;
         }
         const int hrow = S->off[e] + c * BNT;
-        const int KB = kblocks(ti.phase);
+        const int KB = kblocks(ti.phase, KS);
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
+          const int s = it % RST;
+          const uint32_t ph = (it / RST) & 1;
           if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
             ok = false;
             break;
           }
-          if (ti.phase == 1) {
+          if (WQ) {  // codes: two 64-row boxes of 128 bytes; in phase 2 two 64-wide h tiles
+            const int r1 = ti.phase == 1 ? wrow1 : wrow0 + 64;
+            const CUtensorMap* tw = ti.phase == 1 ? &tmap_w1 : &tmap_w2;
+            // the tile's block scales: 12 gate + 12 up (phase 1) or 4 (phase 2), contiguous
+            const float* scl = ti.phase == 1
+                                   ? wscale + fp8::sgu_index(e, 256 * (f >> 1), 0)
+                                   : wscale + kE * fp8::kSguPerExpert + fp8::sd_index(e, f * BMW, 0);
+            const uint32_t scl_bytes = ti.phase == 1 ? 96 : 16;
+            mbar_arrive_expect_tx(&fullb[s], R::RA_BYTES + (ti.phase == 2 ? R::RB_BYTES : 0) +
+                                                 scl_bytes);
+            bulk_load(smem_u32(sC(s)), scl, scl_bytes, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)), tw, kb * KS, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)) + R::RA_BYTES / 2, tw, kb * KS, r1, &fullb[s]);
+            if (ti.phase == 2) {
+              tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * KS, hrow, &fullb[s]);
+              tma_load_2d(smem_u32(sB(s)) + B_BYTES, &tmap_h, kb * KS + BK, hrow, &fullb[s]);
+            }
+          } else if (ti.phase == 1) {
             mbar_arrive_expect_tx(&fullb[s], A_BYTES);
             tma_load_2d(smem_u32(sA(s)), &tmap_w1, kb * BK, wrow0, &fullb[s]);
             tma_load_2d(smem_u32(sA(s)) + A_BYTES / 2, &tmap_w1, kb * BK, wrow1, &fullb[s]);
@@ -255,8 +332,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tile = next;
       }
       if (!ok) {
-        for (int i = max(0, it - STAGES); i < it; ++i)
-          mbar_wait(&fullb[i % STAGES], (i / STAGES) & 1, abort_flag, 10000000ull, kSiteFfnFull);
+        for (int i = max(0, it - RST); i < it; ++i)
+          mbar_wait(&fullb[i % RST], (i / RST) & 1, abort_flag, 10000000ull, kSiteFfnFull);
       }
     }
   } else if (warp == MMA_WARP) {
@@ -271,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const int phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
-        const int KB = kblocks(phase);
+        const int KB = kblocks(phase, KS);
         const uint32_t idesc = phase == 1 ? kIdesc1 : kIdesc2;
         const int a = tc & 1;
         const uint32_t use = tc >> 1;
@@ -282,19 +359,36 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + a * BNT;
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&fullb[s], ph, abort_flag, timeout_ns, kSiteFfnFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t adesc = smem_desc_k128(smem_u32(sA(s)));
+          const int s = it % RST;
+          const uint32_t ph = (it / RST) & 1;
           const uint64_t bdesc = smem_desc_k128(smem_u32(sB(s)));
+          if constexpr (WQ) {
+            // A: the dequantised tile in operand slot it % NA of tensor memory;
+            // B: two 64-wide SW128 token tiles.  The converters waited for the
+            // stage's loads before they arrived on afull, so that wait orders
+            // the token rows too.
+            const int a = it % NA;
+            if (!mbar_wait(&S->afull[a], (it / NA) & 1, abort_flag, timeout_ns, kSiteFfnFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            umma_f16_ta_k128(d, tmem_base + R::A_COL0 + R::A_COLS * a, bdesc,
+                             bdesc + (B_BYTES >> 4), idesc, kb != 0 ? 1u : 0u);
+            // frees the ring stage and, for the converters, operand slot a
+            umma_commit(&emptyb[s]);
+          } else {
+            if (!mbar_wait(&fullb[s], ph, abort_flag, timeout_ns, kSiteFfnFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t adesc = smem_desc_k128(smem_u32(sA(s)));
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          umma_commit(&emptyb[s]);
+            for (int k = 0; k < BK / 16; ++k)
+              umma_f16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_commit(&emptyb[s]);
+          }
         }
         if (ok) umma_commit(&S->tfull[a]);
       }
@@ -304,7 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (HAS1 && warp == GATHER_WARP) {
     // ------------------------------------------------ token gather (phase 1)
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
-    uint32_t dirty = (1u << STAGES) - 1;  // stage slots whose row `lane` may hold non-zero data
+    uint32_t dirty = (1u << RST) - 1;  // stage slots whose row `lane` may hold non-zero data
     int it = 0, n = 0;
     bool ok = true;
     while (ok) {
@@ -313,9 +407,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       const TileInfo ti = tile_info<MODE>(S, tile, total1);
       if (ti.phase == 2) {
         // down tile: the TMA brings the h rows; only keep the stage barriers' count
-        for (int kb = 0; kb < kblocks(2); ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
+        for (int kb = 0; kb < kblocks(2, KS); ++kb, ++it) {
+          const int s = it % RST;
+          const uint32_t ph = (it / RST) & 1;
           if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
             ok = false;
             break;
@@ -331,29 +425,111 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (p >= 0 && static_cast<int64_t>(p) < nrows)
           src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
       }
-      for (int kb = 0; kb < kblocks(1); ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
+      for (int kb = 0; kb < kblocks(1, KS); ++kb, ++it) {
+        const int s = it % RST;
+        const uint32_t ph = (it / RST) & 1;
         if (!mbar_wait(&emptyb[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
           ok = false;
           break;
         }
-        const uint32_t dst = smem_u32(sB(s)) + lane * 128;
-        if (src != nullptr) {
-          const char* g = src + kb * BK * 2;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            cp_async_16(dst + ((static_cast<uint32_t>(q) ^ swz) << 4), g + q * 16, 16);
-          dirty |= 1u << s;
-        } else if (dirty & (1u << s)) {
+        for (int t2 = 0; t2 < KS / BK; ++t2) {  // 64-wide SW128 token tiles of the stage
+          const uint32_t dst = smem_u32(sB(s)) + t2 * B_BYTES + lane * 128;
+          if (src != nullptr) {
+            const char* g = src + (kb * KS + t2 * BK) * 2;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) cp_async_16(dst + q * 16, x, 0);
-          dirty &= ~(1u << s);
+            for (int q = 0; q < 8; ++q)
+              cp_async_16(dst + ((static_cast<uint32_t>(q) ^ swz) << 4), g + q * 16, 16);
+          } else if (dirty & (1u << s)) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) cp_async_16(dst + q * 16, x, 0);
+          }
         }
+        if (src != nullptr)
+          dirty |= 1u << s;
+        else
+          dirty &= ~(1u << s);
         cp_async_arrive_noinc(&fullb[s]);
       }
     }
     cp_async_wait_all();
+  } else if (WQ && warp >= CONV_WARP0) {
+    // ------------------------------------------------ block-FP8 converters
+    // One thread per weight row: warp w may only access tensor-memory lanes
+    // 32 (w % 4) .. 32 (w % 4) + 31, so it takes those rows.  The converter
+    // warps form kConvGroups groups of four (one per lane quarter) that take
+    // the stages in turn, so that one group's loads, stores and hand-off
+    // overlap the next group's arithmetic.  The TMA wrote each 128-byte row of
+    // codes with the 128-byte swizzle (16-byte chunk j of row r at chunk
+    // j ^ (r % 8)), which spreads a warp's reads of one chunk over all banks.
+    // Operand slot it % NA is free again once the MMA of stage it - NA is done,
+    // which the ring's own empty barrier of that stage says.
+    const int quarter = warp & 3;
+    const int cgroup = (warp - CONV_WARP0) >> 2;
+    const int row = 32 * quarter + lane;
+    const uint32_t rsw = static_cast<uint32_t>(row & 7);
+    const bool up_rows = quarter >= 2;  // rows 64..127 of a gate/up tile are up rows
+    const uint32_t a_lane = static_cast<uint32_t>(32 * quarter) << 16;
+    int it = 0, n = 0;
+    bool ok = true;
+    while (ok) {
+      const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
+      if (tile < 0) break;
+      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      for (int kb = 0; kb < kblocks(ti.phase, KS); ++kb, ++it) {
+        if (it % kConvGroups != cgroup) continue;
+        const int s = it % RST;
+        const uint32_t ph = (it / RST) & 1;
+        const int a = it % NA;
+        bool got = mbar_wait(&fullb[s], ph, abort_flag, timeout_ns, kSiteFfnFull);
+        if (got && it >= NA) {
+          const int prev = it - NA;  // the stage that last used slot a
+          got = mbar_wait(&emptyb[prev % RST], (prev / RST) & 1, abort_flag, timeout_ns,
+                          kSiteFfnEmpty);
+        }
+        if (!got) {
+          ok = false;
+          break;
+        }
+        // this stage's block scale, from the tile's scales the TMA brought with
+        // the stage: 12 gate then 12 up (phase 1), or 4 (phase 2), one per k block
+        const float sc = reinterpret_cast<const float*>(
+            sC(s))[(ti.phase == 1 && up_rows ? 12 : 0) + kb];
+        const uint32_t src = smem_u32(sA(s)) + row * 128;
+        const uint32_t dst = tmem_base + a_lane + R::A_COL0 + R::A_COLS * a;
+        uint32_t v[32];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {  // two halves of 64 codes -> 32 columns each
+          if (ti.phase == 1) {
+            const uint32_t mult = fp8::pow2_multiplier<false>(sc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t o[8];
+              const uint32_t jj = static_cast<uint32_t>(4 * h2 + j);
+              fp8::dequant16<false>(ld_shared_v4(src + ((jj ^ rsw) << 4)), sc, mult, o);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[8 * j + i] = o[i];
+            }
+          } else {
+            const uint32_t mult = fp8::pow2_multiplier<true>(sc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t o[8];
+              const uint32_t jj = static_cast<uint32_t>(4 * h2 + j);
+              fp8::dequant16<true>(ld_shared_v4(src + ((jj ^ rsw) << 4)), sc, mult, o);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[8 * j + i] = o[i];
+            }
+          }
+          tmem_st_x32(dst + 32 * h2, v);
+          if (h2 == 0) tmem_wait_st();  // v is rewritten next
+        }
+        tmem_wait_st();
+        tc_fence_before();  // operand stores -> the MMA thread's tcgen05.mma
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S->afull[a]);
+      }
+    }
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue
     bool range_bad = false;
@@ -427,7 +603,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
   if (warp == MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, R::TMEM_COLS);
   }
 }
 

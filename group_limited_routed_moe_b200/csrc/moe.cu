@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "expert_ffn.cuh"
 #include "expert_ffn_skinny.cuh"
+#include "fp8.cuh"
 #include "pack.cuh"
 #include "permute.cuh"
 #include "route.cuh"
@@ -26,7 +27,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 1024;  // gate/up keeps padding rows of A zeroed up to this T
@@ -107,6 +108,9 @@ int device_setup(int* dev_out, int* sms_out) {
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
+      if (e == cudaSuccess)
         e = cudaFuncSetAttribute(router::router_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, router::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -140,6 +144,22 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MOE_OK;
+}
+
+// 2-D tensor map of 8-bit codes: `rows` rows of `cols` bytes, box of 128 x 64,
+// 128-byte swizzle (the converter warps read each row's eight 16-byte chunks;
+// the swizzle keeps a warp's reads free of bank conflicts).
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {128, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", int(r));
   return MOE_OK;
 }
 
@@ -267,7 +287,8 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
                       dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw, tw, tw,
                       reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                       reinterpret_cast<uint16_t*>(h), static_cast<uint16_t*>(nullptr),
-                      sched_words(offsets, 1), static_cast<int*>(nullptr), g_timeout_ns.load());
+                      sched_words(offsets, 1), static_cast<int*>(nullptr),
+                      static_cast<const float*>(nullptr), g_timeout_ns.load());
   }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -296,7 +317,8 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                       static_cast<const __nv_bfloat16*>(nullptr), offsets,
                       static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
                       reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
-                      static_cast<int*>(nullptr), g_timeout_ns.load());
+                      static_cast<int*>(nullptr), static_cast<const float*>(nullptr),
+                      g_timeout_ns.load());
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -327,7 +349,7 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                       reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                       reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
                       sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                      g_timeout_ns.load());
+                      static_cast<const float*>(nullptr), g_timeout_ns.load());
   }
   // both GEMMs in one launch (see expert_ffn.cuh)
   CUtensorMap tb1, tb2, ta2;
@@ -347,6 +369,41 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                     g_timeout_ns.load());
 }
 
+// Packed block-FP8 layer -> packed bf16/fp16 layer.
+int do_dequant_fp8(const void* packed8, moe_bf16* packed, int sms, cudaStream_t s) {
+  return launch_pdl("dequant_fp8_kernel launch", fp8::dequant_fp8_kernel, dim3(sms * 8),
+                    dim3(256), 0, s, static_cast<const uint8_t*>(packed8),
+                    reinterpret_cast<uint16_t*>(packed));
+}
+
+// Expert FFN with block-FP8 weights.  Up to kSkinnyMaxT tokens the skinny
+// single-launch kernel dequantises each weight tile in shared memory (half
+// the weight bytes from HBM); above it, where the GEMMs are bound by the
+// tensor cores rather than by the weight stream, the layer is expanded into
+// `dq` (moe_packed_weight_bytes) and run by the bf16 kernel.
+int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* offsets,
+                      const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, moe_bf16* dq,
+                      int sms, cudaStream_t s) {
+  if (T > kSkinnyMaxT) {
+    int rc = do_dequant_fp8(packed8, dq, sms, s);
+    if (rc) return rc;
+    return do_expert_ffn(x, dq, offsets, perm_src, T, h, y, sms, s);
+  }
+  const uint8_t* p8 = static_cast<const uint8_t*>(packed8);
+  CUtensorMap tw1, tw2, th;
+  int rc = make_tmap_u8(&tw1, p8, kH, uint64_t(kE) * 2 * kI);
+  if (!rc) rc = make_tmap_u8(&tw2, p8 + fp8::kGuBytes, kI, uint64_t(kE) * kH);
+  if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (rc) return rc;
+  return launch_pdl("skinny_gemm_kernel<3, fp8> launch", skinny::skinny_gemm_kernel<3, true>,
+                    dim3(sms), dim3(skinny::Ring<true>::THREADS), skinny::SMEM_BYTES, s, tw1, tw2,
+                    th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+                    reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
+                    sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
+                    reinterpret_cast<const float*>(p8 + fp8::kSguOff), g_timeout_ns.load());
+}
+
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
                const moe_bf16* residual, moe_bf16* out, cudaStream_t s) {
   return launch_pdl("combine_kernel launch", combine_kernel, dim3(static_cast<unsigned>(T)),
@@ -357,9 +414,11 @@ int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
 
 // workspace carve-up of moe_layer
 struct LayerWs {
-  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, total;
+  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, dq, total;
 };
-LayerWs layer_ws(int64_t T) {
+// fp8: the block-FP8 layer, which above kSkinnyMaxT tokens also needs room for
+// the expanded bf16/fp16 layer.
+LayerWs layer_ws(int64_t T, bool fp8 = false) {
   LayerWs L{};
   const size_t n = static_cast<size_t>(T) * kTopK;
   size_t o = 0;
@@ -378,6 +437,7 @@ LayerWs layer_ws(int64_t T) {
   L.h = take(n * kI * 2);
   L.y = take(n * kH * 2);
   L.logits = take(static_cast<size_t>(T) * kE * 4);  // used by moe_layer_routed
+  L.dq = take(fp8 && T > kSkinnyMaxT ? static_cast<size_t>(kPackElems) * 2 : 0);
   L.total = o;
   return L;
 }
@@ -406,6 +466,8 @@ int moe_get_device_status(int device) {
     return fail(MOE_ERR_INVALID_ARG, "a kernel met an out-of-range index (status 0x%08x)", v);
   if ((v & 0x7FFFFFFFu) == kSiteFp16Range)
     return fail(MOE_ERR_RANGE, "a value of h, y_perm or W_down exceeded the fp16 range");
+  if ((v & 0x7FFFFFFFu) == kSiteFp8Nan)
+    return fail(MOE_ERR_RANGE, "a block-FP8 expert weight is a NaN code");
   return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out (status 0x%08x, site %u)", v,
               v & 0x7FFFFFFFu);
 }
@@ -547,22 +609,27 @@ size_t moe_layer_workspace_bytes(int64_t T) {
 namespace {
 // The layer from given router logits, or (packed_router != NULL) from the
 // router projection of x computed into the workspace first.
+// With packed_fp8 != NULL the experts are the block-FP8 layer it points to
+// (packed_w is then ignored).
 int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
                const moe_bf16* packed_router, const float* bias, const moe_bf16* packed_w,
                int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
-               float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+               float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream,
+               const void* packed_fp8 = nullptr) {
   int rc = check_T(T);
   if (rc) return rc;
   if (T == 0) return MOE_OK;
+  const bool fp8 = packed_fp8 != nullptr;
+  if (fp8) packed_w = static_cast<const moe_bf16*>(packed_fp8);
   REQUIRE(x && (logits || packed_router) && packed_w && out && workspace, "null pointer");
   REQUIRE(aligned(x, 128) && aligned(packed_w, 128) && (!packed_router || aligned(packed_router, 128)),
-          "x, packed_w and packed_router must be 128-byte aligned");
+          "x, the packed weights and packed_router must be 128-byte aligned");
   REQUIRE(aligned(workspace, 1024), "workspace must be 1024-byte aligned");
   REQUIRE((!logits || aligned(logits, 16)) && (!bias || aligned(bias, 16)) && aligned(out, 16) &&
               (!residual || aligned(residual, 16)) && (!topk_idx_out || aligned(topk_idx_out, 16)) &&
               (!topk_w_out || aligned(topk_w_out, 16)),
           "pointers must be 16-byte aligned");
-  const LayerWs L = layer_ws(T);
+  const LayerWs L = layer_ws(T, fp8);
   if (workspace_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE, "%s workspace needs %zu bytes, got %zu", fn, L.total,
                 workspace_bytes);
@@ -588,7 +655,13 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
   if (!rc)
     rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
                           ws + L.perm_ws, s);
-  if (!rc) rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
+  if (!rc) {
+    if (fp8)
+      rc = do_expert_ffn_fp8(x, packed_fp8, offsets, perm_src, T, h, y,
+                             reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
+    else
+      rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
+  }
   if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s);
   return rc;
 }
@@ -638,6 +711,85 @@ int moe_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, floa
   rc = device_setup(nullptr, &sms);
   if (rc) return rc;
   return do_router(x, packed_router, T, logits, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---- block-FP8 experts ---------------------------------------------------------
+size_t moe_packed_fp8_bytes(void) { return static_cast<size_t>(fp8::kPackedBytes); }
+
+int moe_pack_weights_fp8(const uint8_t* q_gate, const float* s_gate, const uint8_t* q_up,
+                         const float* s_up, const uint8_t* q_down, const float* s_down,
+                         void* packed_fp8, moe_stream_t stream) {
+  REQUIRE(q_gate && s_gate && q_up && s_up && q_down && s_down && packed_fp8, "null pointer");
+  REQUIRE(aligned(packed_fp8, 128), "packed_fp8 must be 128-byte aligned");
+  REQUIRE(aligned(s_gate, 4) && aligned(s_up, 4) && aligned(s_down, 4),
+          "scales must be 4-byte aligned");
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* p8 = static_cast<uint8_t*>(packed_fp8);
+  const dim3 ggu(kI / 32, kH / 32, kE), gd(kH / 32, kI / 32, kE);
+  fp8::pack_fp8_transpose_kernel<<<ggu, 256, 0, s>>>(q_gate, p8, kH, kI, 0, s_down);
+  fp8::pack_fp8_transpose_kernel<<<ggu, 256, 0, s>>>(q_up, p8, kH, kI, 1, s_down);
+  fp8::pack_fp8_transpose_kernel<<<gd, 256, 0, s>>>(q_down, p8, kI, kH, 2, s_down);
+  constexpr int n_sc = kE * (fp8::kSguPerExpert + fp8::kSdPerExpert);
+  fp8::pack_fp8_scales_kernel<<<(n_sc + 255) / 256, 256, 0, s>>>(
+      s_gate, s_up, s_down, reinterpret_cast<float*>(p8 + fp8::kSguOff),
+      reinterpret_cast<float*>(p8 + fp8::kSdOff));
+  return launch_check("pack_fp8 kernels launch");
+}
+
+int moe_dequant_fp8(const void* packed_fp8, moe_bf16* packed, moe_stream_t stream) {
+  REQUIRE(packed_fp8 && packed, "null pointer");
+  REQUIRE(aligned(packed_fp8, 128) && aligned(packed, 128),
+          "packed_fp8 and packed must be 128-byte aligned");
+  int sms = 0;
+  int rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_dequant_fp8(packed_fp8, packed, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_expert_ffn_fp8_workspace_bytes(int64_t T) {
+  if (T < 0 || T > kMaxTokens) return 0;
+  return T > kSkinnyMaxT ? static_cast<size_t>(kPackElems) * 2 : 0;
+}
+
+int moe_expert_ffn_fp8(const moe_bf16* x, const void* packed_fp8, const int32_t* offsets,
+                       const int32_t* perm_src, int64_t T, moe_f16* h, moe_f16* y_perm,
+                       void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && packed_fp8 && offsets && perm_src && h && y_perm, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_fp8, 128) && aligned(h, 128),
+          "x, packed_fp8 and h must be 128-byte aligned");
+  REQUIRE(aligned(y_perm, 16) && aligned(offsets, 16) && aligned(perm_src, 16),
+          "pointers must be 16-byte aligned");
+  const size_t need = moe_expert_ffn_fp8_workspace_bytes(T);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(MOE_ERR_WORKSPACE, "moe_expert_ffn_fp8 workspace needs %zu bytes, got %zu", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (need > 0) REQUIRE(aligned(workspace, 128), "workspace must be 128-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_expert_ffn_fp8(x, packed_fp8, offsets, perm_src, T, h, y_perm,
+                           static_cast<moe_bf16*>(workspace), sms,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_layer_fp8_workspace_bytes(int64_t T) {
+  if (T < 0 || T > kMaxTokens) return 0;
+  return layer_ws(T, true).total;
+}
+
+int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
+                  const void* packed_fp8, int64_t T, const moe_bf16* residual, moe_bf16* out,
+                  int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                  size_t workspace_bytes, moe_stream_t stream) {
+  if (T > 0 && (logits == nullptr || packed_fp8 == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "null pointer");
+  return layer_impl("moe_layer_fp8", x, logits, nullptr, bias, nullptr, T, residual, out,
+                    topk_idx_out, topk_w_out, workspace, workspace_bytes, stream, packed_fp8);
 }
 
 }  // extern "C"

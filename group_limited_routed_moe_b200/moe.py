@@ -65,6 +65,13 @@ _SIGS = {
     "moe_layer_routed": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_permute_fixed_scratch_max_tokens": ([], _i64),
     "moe_permute_fixed_scratch": ([_p, _i64, _p, _p, _p, _p, _p], _i32),
+    "moe_packed_fp8_bytes": ([], _sz),
+    "moe_pack_weights_fp8": ([_p, _p, _p, _p, _p, _p, _p, _p], _i32),
+    "moe_dequant_fp8": ([_p, _p, _p], _i32),
+    "moe_layer_fp8_workspace_bytes": ([_i64], _sz),
+    "moe_expert_ffn_fp8_workspace_bytes": ([_i64], _sz),
+    "moe_expert_ffn_fp8": ([_p, _p, _p, _p, _i64, _p, _p, _p, _sz, _p], _i32),
+    "moe_layer_fp8": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -231,9 +238,10 @@ def layer_workspace_bytes(T: int) -> int:
     return int(lib.moe_layer_workspace_bytes(T))
 
 
-def alloc_layer_workspace(T: int, device) -> torch.Tensor:
-    """A uint8 view of at least layer_workspace_bytes(T) bytes, 1024-byte aligned."""
-    n = layer_workspace_bytes(T)
+def alloc_layer_workspace(T: int, device, fp8: bool = False) -> torch.Tensor:
+    """A uint8 view of at least layer_workspace_bytes(T) bytes (or
+    layer_fp8_workspace_bytes(T) if fp8), 1024-byte aligned."""
+    n = layer_fp8_workspace_bytes(T) if fp8 else layer_workspace_bytes(T)
     raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
     off = (-raw.data_ptr()) % 1024
     return raw[off:off + n]
@@ -291,6 +299,84 @@ def moe_layer_routed(x: torch.Tensor, packed_router: torch.Tensor, bias: torch.T
     return out
 
 
+# ----------------------------------------------------------------- block-FP8 experts
+
+def packed_fp8_bytes() -> int:
+    return int(lib.moe_packed_fp8_bytes())
+
+
+def layer_fp8_workspace_bytes(T: int) -> int:
+    return int(lib.moe_layer_fp8_workspace_bytes(T))
+
+
+def moe_pack_weights_fp8(q_gate: torch.Tensor, s_gate: torch.Tensor, q_up: torch.Tensor,
+                         s_up: torch.Tensor, q_down: torch.Tensor, s_down: torch.Tensor,
+                         packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Re-layout one layer's block-FP8 experts: uint8 E4M3 codes and fp32
+    128 x 128 block scales (see include/moe.h)."""
+    nb_h, nb_i = HIDDEN // 128, INTER // 128
+    for t, shp, dt in ((q_gate, (N_EXPERTS, HIDDEN, INTER), torch.uint8),
+                       (q_up, (N_EXPERTS, HIDDEN, INTER), torch.uint8),
+                       (q_down, (N_EXPERTS, INTER, HIDDEN), torch.uint8),
+                       (s_gate, (N_EXPERTS, nb_h, nb_i), torch.float32),
+                       (s_up, (N_EXPERTS, nb_h, nb_i), torch.float32),
+                       (s_down, (N_EXPERTS, nb_i, nb_h), torch.float32)):
+        if t.dtype != dt or tuple(t.shape) != shp or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"expected contiguous CUDA {dt} {shp}, got {t.dtype} {tuple(t.shape)}")
+    if packed is None:
+        packed = torch.empty(packed_fp8_bytes(), dtype=torch.uint8, device=q_gate.device)
+    _check("moe_pack_weights_fp8",
+           lib.moe_pack_weights_fp8(_ptr(q_gate), _ptr(s_gate), _ptr(q_up), _ptr(s_up),
+                                    _ptr(q_down), _ptr(s_down), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_dequant_fp8(packed_fp8: torch.Tensor, packed: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """The packed bf16/fp16 layer (moe_pack_weights layout) of a packed FP8 layer."""
+    if packed is None:
+        packed = torch.empty(packed_weight_bytes() // 2, dtype=torch.bfloat16,
+                             device=packed_fp8.device)
+    _check("moe_dequant_fp8", lib.moe_dequant_fp8(_ptr(packed_fp8), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_expert_ffn_fp8(x: torch.Tensor, packed_fp8: torch.Tensor, offsets: torch.Tensor,
+                       perm_src: torch.Tensor, h=None, y_perm=None, workspace=None, stream=None):
+    """Step 3 with block-FP8 experts (see include/moe.h); returns (h, y_perm)."""
+    T = x.shape[0]
+    n = T * TOPK
+    if h is None:
+        h = torch.empty((n, INTER), dtype=torch.float16, device=x.device)
+    if y_perm is None:
+        y_perm = torch.empty((n, HIDDEN), dtype=torch.float16, device=x.device)
+    need = int(lib.moe_expert_ffn_fp8_workspace_bytes(T))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check("moe_expert_ffn_fp8",
+           lib.moe_expert_ffn_fp8(_ptr(x), _ptr(packed_fp8), _ptr(offsets), _ptr(perm_src), T,
+                                  _ptr(h), _ptr(y_perm), _ptr(workspace),
+                                  workspace.numel() if workspace is not None else 0,
+                                  _stream(stream)))
+    return h, y_perm
+
+
+def moe_layer_fp8(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
+                  packed_fp8: torch.Tensor, residual=None, out=None, topk_idx_out=None,
+                  topk_w_out=None, workspace: torch.Tensor | None = None, stream=None):
+    """moe_layer with block-FP8 experts (see include/moe.h)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = alloc_layer_workspace(T, x.device, fp8=True)
+    _check("moe_layer_fp8", lib.moe_layer_fp8(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_fp8),
+                                              T, _ptr(residual), _ptr(out), _ptr(topk_idx_out),
+                                              _ptr(topk_w_out), _ptr(workspace), workspace.numel(),
+                                              _stream(stream)))
+    return out
+
+
 def moe_layer_from_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: torch.Tensor | None,
                         packed_w: torch.Tensor, x_dev: torch.Tensor, logits_dev: torch.Tensor,
                         out_dev: torch.Tensor, out_host: torch.Tensor,
@@ -316,11 +402,13 @@ class HostPipeline:
     call's layer), so two calls never share the weights they stream through
     L2.  Stream order keeps a slot's buffers from being reused before its
     previous call has finished.  The output of call k lands in the `out_host`
-    passed to submit(); it is complete once `drain()` returns.
+    passed to submit(); it is complete once `drain()` returns.  With fp8=True
+    the weights passed to submit() are a packed block-FP8 layer and every call
+    runs moe_layer_fp8.
     """
 
-    def __init__(self, T: int, device, depth: int = 2):
-        self.T, self.depth, self.k = T, depth, 0
+    def __init__(self, T: int, device, depth: int = 2, fp8: bool = False):
+        self.T, self.depth, self.k, self.fp8 = T, depth, 0, fp8
         self.last_layer = None
         self.slots = []
         for _ in range(depth):
@@ -329,7 +417,7 @@ class HostPipeline:
                 "x": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
                 "logits": torch.empty((T, N_EXPERTS), dtype=torch.float32, device=device),
                 "out": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
-                "ws": alloc_layer_workspace(T, device),
+                "ws": alloc_layer_workspace(T, device, fp8=fp8),
             })
 
     def submit(self, x_host, logits_host, out_host, bias, packed_w):
@@ -341,8 +429,9 @@ class HostPipeline:
             slot["logits"].copy_(logits_host, non_blocking=True)
             if self.last_layer is not None:
                 st.wait_event(self.last_layer)
-            moe_layer(slot["x"], slot["logits"], bias, packed_w, out=slot["out"],
-                      workspace=slot["ws"], stream=st)
+            (moe_layer_fp8 if self.fp8 else moe_layer)(
+                slot["x"], slot["logits"], bias, packed_w, out=slot["out"], workspace=slot["ws"],
+                stream=st)
             self.last_layer = torch.cuda.Event()
             self.last_layer.record(st)
             out_host.copy_(slot["out"], non_blocking=True)

@@ -67,8 +67,8 @@ typedef enum moe_status {
   MOE_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out */
   MOE_ERR_UNSUPPORTED = 5, /* device is not sm_100 */
   MOE_ERR_RANGE = 6        /* an fp16 intermediate (h, y_perm, packed W_down)
-                              left the fp16 range; reported by
-                              moe_get_device_status() */
+                              left the fp16 range, or a block-FP8 weight is
+                              a NaN code; reported by moe_get_device_status() */
 } moe_status;
 
 /* ---- library information ------------------------------------------------ */
@@ -243,6 +243,77 @@ int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const flo
                      const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
                      moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
                      void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---- block-FP8 experts ---------------------------------------------------- */
+
+/* The CUDA path of issue #1247 reads experts in bf16, block FP8 and NVFP4
+ * ("What it does not cover", third bullet); the pages do not spell the block-
+ * FP8 format out.  Read here as the usual block-FP8 checkpoint form: every
+ * weight an FP8 E4M3 code (OCP 8-bit float, no infinities, 0x7F/0xFF NaN,
+ * largest finite 448) and every 128 x 128 block of a matrix one fp32 scale,
+ *   weight = value(code) * scale.
+ * The kernels dequantise each weight to the tensor-core operand type as
+ * fp32(value * scale) rounded once to bf16 (gate/up) or fp16 (down).  With
+ * power-of-two scales that is exact, and moe_layer_fp8 returns bit for bit
+ * what moe_layer returns on the dequantised weights; other scales add one
+ * rounding per weight (relative 2^-9 for bf16, 2^-12 for fp16). */
+
+/* Bytes of one layer's packed block-FP8 experts (302 MB: codes, then scales). */
+size_t moe_packed_fp8_bytes(void);
+
+/* One-time re-layout of one layer's block-FP8 experts.
+ *   q_gate, q_up : [128][1536][512] uint8 E4M3 codes (the layer computes x @ W)
+ *   s_gate, s_up : [128][12][4] fp32: scale of rows 128i..128i+127 (of 1536) and
+ *                  columns 128j..128j+127 (of 512) at [e][i][j]
+ *   q_down       : [128][512][1536] codes;  s_down : [128][4][12] fp32
+ *   packed_fp8   : moe_packed_fp8_bytes() bytes, 128-byte aligned, output:
+ *                  codes in the operand order of moe_pack_weights (K-major,
+ *                  gate/up interleaved in 128-column blocks), then the scales
+ *                  reordered to match.
+ * Within every aligned group of 4 codes along k the packed bytes hold the
+ * elements in the order k+2, k, k+3, k+1 (the dequantisation reads them so).
+ * A down weight whose dequantised value lies outside the fp16 range, or a
+ * NaN code (0x7F, 0xFF) in any matrix, sets the device error word
+ * (moe_get_device_status(): MOE_ERR_RANGE); the packed bytes are written
+ * regardless, and the layer's results on such weights are unspecified. */
+int moe_pack_weights_fp8(const uint8_t* q_gate, const float* s_gate, const uint8_t* q_up,
+                         const float* s_up, const uint8_t* q_down, const float* s_down,
+                         void* packed_fp8, moe_stream_t stream);
+
+/* Expands a packed block-FP8 layer into the packed bf16/fp16 layer that
+ * moe_pack_weights writes (packed: moe_packed_weight_bytes() bytes, 128-byte
+ * aligned, output).  With power-of-two scales it equals moe_pack_weights of
+ * the dequantised weights, byte for byte. */
+int moe_dequant_fp8(const void* packed_fp8, moe_bf16* packed, moe_stream_t stream);
+
+/* Scratch bytes moe_expert_ffn_fp8 needs: 0 for T <= 256, else
+ * moe_packed_weight_bytes() (the expanded layer). */
+size_t moe_expert_ffn_fp8_workspace_bytes(int64_t T);
+
+/* Step 3 with block-FP8 experts: moe_expert_ffn's arguments, with packed_fp8
+ * (from moe_pack_weights_fp8) in place of packed_w, plus a scratch workspace
+ * of moe_expert_ffn_fp8_workspace_bytes(T) bytes (128-byte aligned; may be
+ * NULL when that is 0).  Up to 256 tokens one persistent launch streams the
+ * codes and dequantises each weight tile in shared memory; above, the layer
+ * is expanded into the workspace and the bf16 expert FFN runs on it. */
+int moe_expert_ffn_fp8(const moe_bf16* x, const void* packed_fp8, const int32_t* offsets,
+                       const int32_t* perm_src, int64_t T, moe_f16* h, moe_f16* y_perm,
+                       void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Workspace bytes moe_layer_fp8 needs for T tokens: moe_layer's, plus room
+ * for the expanded layer (moe_packed_weight_bytes()) when T > 256. */
+size_t moe_layer_fp8_workspace_bytes(int64_t T);
+
+/* moe_layer with block-FP8 experts (packed_fp8 from moe_pack_weights_fp8),
+ * other arguments as in moe_layer.  For T <= 256 the single-launch expert FFN
+ * streams the 8-bit codes and dequantises every weight tile in shared memory
+ * on its way to the tensor cores (half the weight bytes of the bf16 layer);
+ * above, the layer is first expanded into the workspace (moe_dequant_fp8) and
+ * the bf16 expert FFN runs on it. */
+int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
+                  const void* packed_fp8, int64_t T, const moe_bf16* residual,
+                  moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
+                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* ---- permutation without a caller workspace ------------------------------ */
 

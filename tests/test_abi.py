@@ -13,7 +13,7 @@ def test_exports_every_declared_symbol():
     assert len(names) >= 15
     missing = [n for n in names if not hasattr(moe.lib, n)]
     assert missing == []
-    assert moe.lib.moe_abi_version() == 2
+    assert moe.lib.moe_abi_version() == 3
 
 
 def test_sizes():
@@ -66,3 +66,24 @@ def test_binding_raises_with_message():
     with pytest.raises(moe.MoeError) as ei:
         moe._check("moe_route", moe.MOE_ERR_INVALID_ARG)
     assert "status 1" in str(ei.value)
+
+
+def test_fp8_sizes_and_host_validation():
+    L = moe.lib
+    gu, d = 128 * 1024 * 1536, 128 * 1536 * 512
+    assert moe.packed_fp8_bytes() == gu + d + 128 * (96 + 48) * 4
+    # up to 256 tokens the FP8 layer streams codes; above, it expands the layer
+    # into the workspace first
+    for T in (1, 16, 256):
+        assert moe.layer_fp8_workspace_bytes(T) == moe.layer_workspace_bytes(T)
+    for T in (257, 2048):
+        assert moe.layer_fp8_workspace_bytes(T) == moe.layer_workspace_bytes(T) + moe.packed_weight_bytes()
+    assert L.moe_layer_fp8(None, None, None, None, 0, None, None, None, None, None, 0, None) == moe.MOE_OK
+    assert L.moe_layer_fp8(_p(1024), _p(1024), None, None, 16, None, _p(1024), None, None,
+                           _p(1024), 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    ws = moe.layer_fp8_workspace_bytes(300)
+    assert L.moe_layer_fp8(_p(1024), _p(1024), None, _p(1024), 300, None, _p(1024), None, None,
+                           _p(1024), ws - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_pack_weights_fp8(_p(128), _p(128), None, _p(128), _p(128), _p(128), _p(128),
+                                  None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dequant_fp8(_p(136), _p(128), None) == moe.MOE_ERR_INVALID_ARG
