@@ -100,6 +100,8 @@ static_assert(Ring<true>::RSTAGE_BYTES % 1024 == 0 && Ring<true>::RA_BYTES % 102
 static_assert(Ring<true>::A_COL0 + Ring<true>::A_COLS * Ring<true>::NA <= Ring<true>::TMEM_COLS,
               "operand slots must fit the tensor-memory allocation");
 static_assert(Ring<true>::RSTAGES % Ring<true>::NA == 0, "slot reuse follows the ring");
+static_assert(kConvGroups == 2 && kH / Ring<true>::KS % 2 == 0 && kI / Ring<true>::KS % 2 == 0,
+              "block-FP8 stages go in pairs, one per converter group, never across a tile");
 
 // Per-phase constants.  Phase 1: 8 weight blocks per 32-token chunk (4 pairs
 // x 2 halves of 64 gate + 64 up rows), K = 1536; phase 2: 12 blocks, K = 512.
@@ -118,7 +120,7 @@ struct Tail {
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t afull[4];  // block-FP8: operand slot written (one arrival per lane quarter)
+  uint64_t apair[2];  // block-FP8: the operand slots of a pair of stages written (8 arrivals)
   uint64_t xfull;   // up half written to the exchange tile (64 lane arrivals)
   uint64_t xempty;  // gate half done reading it (64 lane arrivals)
   uint64_t drain;
@@ -201,7 +203,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       mbar_init(&fullb[s], HAS1 ? 1 + 32 : 1);  // TMA arrive (+ 32 gather lanes)
       mbar_init(&emptyb[s], 1);                  // MMA commit
     }
-    for (int a = 0; a < R::NA; ++a) mbar_init(&S->afull[a], 4);  // one warp per lane quarter
+    // four lane-quarter warps per stage, two stages per pair
+    for (int p = 0; p < 2; ++p) mbar_init(&S->apair[p], 8);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&S->tfull[a], 1);
       mbar_init(&S->tempty[a], 4);
@@ -364,15 +367,20 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
           const uint64_t bdesc = smem_desc_k128(smem_u32(sB(s)));
           if constexpr (WQ) {
             // A: the dequantised tile in operand slot it % NA of tensor memory;
-            // B: two 64-wide SW128 token tiles.  The converters waited for the
-            // stage's loads before they arrived on afull, so that wait orders
-            // the token rows too.
-            const int a = it % NA;
-            if (!mbar_wait(&S->afull[a], (it / NA) & 1, abort_flag, timeout_ns, kSiteFfnFull)) {
-              ok = false;
-              break;
+            // B: two 64-wide SW128 token tiles.  Stages go in pairs (it even):
+            // one wait covers both, since any shared-memory access of this
+            // thread after tcgen05 work costs a few hundred cycles.  The
+            // converters waited for the stages' loads before they arrived, so
+            // that wait orders the token rows too.
+            if ((it & 1) == 0) {
+              if (!mbar_wait(&S->apair[(it >> 1) & 1], (it >> 2) & 1, abort_flag, timeout_ns,
+                             kSiteFfnFull)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            tc_fence_after();
+            const int a = it % NA;
             umma_f16_ta_k128(d, tmem_base + R::A_COL0 + R::A_COLS * a, bdesc,
                              bdesc + (B_BYTES >> 4), idesc, kb != 0 ? 1u : 0u);
             // frees the ring stage and, for the converters, operand slot a
@@ -527,7 +535,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
         tmem_wait_st();
         tc_fence_before();  // operand stores -> the MMA thread's tcgen05.mma
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S->afull[a]);
+        if (lane == 0) mbar_arrive(&S->apair[(it >> 1) & 1]);
       }
     }
   } else if (warp < 4) {

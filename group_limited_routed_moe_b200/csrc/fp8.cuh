@@ -96,6 +96,27 @@ __device__ __forceinline__ uint32_t pow2_multiplier(float scale) {
   return h | (h << 16);
 }
 
+// The conversion route of dequant16 (scales that are not powers of two).
+template <bool F16>
+__device__ __forceinline__ void dequant16_cvt(const uint4 q, const float scale, uint32_t (&o)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      // pair (k, k+1) sits in bytes (1, 3), pair (k+2, k+3) in bytes (0, 2)
+      const float2 f = e4m3x2_to_float2(__byte_perm(w[i], 0, h == 0 ? 0x0031 : 0x0020));
+      const float x0 = f.x * scale, x1 = f.y * scale;
+      if constexpr (F16) {
+        __half2 v = __floats2half2_rn(x0, x1);
+        o[2 * i + h] = *reinterpret_cast<uint32_t*>(&v);
+      } else {
+        o[2 * i + h] = pack_bf16x2(x0, x1);
+      }
+    }
+  }
+}
+
 // 16 codes (one packed 16-byte chunk) times `scale`, each product rounded once
 // from fp32 to the operand type: fp16 if F16, else bf16.  Eight 32-bit words
 // out, two values each, in element order.  mult: pow2_multiplier<F16>(scale);
@@ -121,21 +142,7 @@ __device__ __forceinline__ void dequant16(const uint4 q, const float scale, cons
     }
     return;
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      // pair (k, k+1) sits in bytes (1, 3), pair (k+2, k+3) in bytes (0, 2)
-      const float2 f = e4m3x2_to_float2(__byte_perm(w[i], 0, h == 0 ? 0x0031 : 0x0020));
-      const float x0 = f.x * scale, x1 = f.y * scale;
-      if constexpr (F16) {
-        __half2 v = __floats2half2_rn(x0, x1);
-        o[2 * i + h] = *reinterpret_cast<uint32_t*>(&v);
-      } else {
-        o[2 * i + h] = pack_bf16x2(x0, x1);
-      }
-    }
-  }
+  dequant16_cvt<F16>(q, scale, o);
 }
 
 // dst[e][map(n)][k] = src[e][k][n] for one [K][N] code matrix, 32 x 32 byte
