@@ -120,7 +120,7 @@ struct Tail {
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t apair[2];  // block-FP8: the operand slots of a pair of stages written (8 arrivals)
+  uint64_t apair[2];  // block-FP8: the operand slots of a pair of stages written
   uint64_t xfull;   // up half written to the exchange tile (64 lane arrivals)
   uint64_t xempty;  // gate half done reading it (64 lane arrivals)
   uint64_t drain;
@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       mbar_init(&fullb[s], HAS1 ? 1 + 32 : 1);  // TMA arrive (+ 32 gather lanes)
       mbar_init(&emptyb[s], 1);                  // MMA commit
     }
-    // four lane-quarter warps per stage, two stages per pair
-    for (int p = 0; p < 2; ++p) mbar_init(&S->apair[p], 8);
+    // every converter warp arrives once per stage, two stages per pair
+    for (int p = 0; p < 2; ++p) mbar_init(&S->apair[p], 2 * R::NCONV);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&S->tfull[a], 1);
       mbar_init(&S->tempty[a], 4);
@@ -465,9 +465,11 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     // ------------------------------------------------ block-FP8 converters
     // One thread per weight row: warp w may only access tensor-memory lanes
     // 32 (w % 4) .. 32 (w % 4) + 31, so it takes those rows.  The converter
-    // warps form kConvGroups groups of four (one per lane quarter) that take
-    // the stages in turn, so that one group's loads, stores and hand-off
-    // overlap the next group's arithmetic.  The TMA wrote each 128-byte row of
+    // warps form kConvGroups groups of four (one per lane quarter); in every
+    // stage group g converts the g-th 64 of a row's 128 codes, which halves
+    // the time from a stage's arrival to its hand-off to the MMA (the ring's
+    // cycle, not the converters' throughput, bounds the weight stream).  The
+    // TMA wrote each 128-byte row of
     // codes with the 128-byte swizzle (16-byte chunk j of row r at chunk
     // j ^ (r % 8)), which spreads a warp's reads of one chunk over all banks.
     // Operand slot it % NA is free again once the MMA of stage it - NA is done,
@@ -485,7 +487,6 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       if (tile < 0) break;
       const TileInfo ti = tile_info<MODE>(S, tile, total1);
       for (int kb = 0; kb < kblocks(ti.phase, KS); ++kb, ++it) {
-        if (it % kConvGroups != cgroup) continue;
         const int s = it % RST;
         const uint32_t ph = (it / RST) & 1;
         const int a = it % NA;
@@ -506,8 +507,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
         const uint32_t src = smem_u32(sA(s)) + row * 128;
         const uint32_t dst = tmem_base + a_lane + R::A_COL0 + R::A_COLS * a;
         uint32_t v[32];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {  // two halves of 64 codes -> 32 columns each
+        {
+          const int h2 = cgroup;  // this group's 64 codes -> 32 columns
           if (ti.phase == 1) {
             const uint32_t mult = fp8::pow2_multiplier<false>(sc);
 #pragma unroll
@@ -530,7 +531,6 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             }
           }
           tmem_st_x32(dst + 32 * h2, v);
-          if (h2 == 0) tmem_wait_st();  // v is rewritten next
         }
         tmem_wait_st();
         tc_fence_before();  // operand stores -> the MMA thread's tcgen05.mma
