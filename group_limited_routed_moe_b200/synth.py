@@ -14,6 +14,9 @@ Recipe (the distributions of the layer's workloads):
 * expert weights ~ N(0, 0.02), bf16: W_gate, W_up [128, 1536, 512] and
   W_down [128, 512, 1536] per layer, used as x @ W.
 
+Shared experts (when a layer has them) come from the same generator under
+seed + 1000, expert indices 0, 1, ...
+
 Activations, logits and bias are drawn with NumPy's PCG64 (host).  Expert
 weights (up to 23 x 604 MB) come from a counter-based generator so that the
 same bytes can be produced on the device in bulk or on the host for any
@@ -125,6 +128,18 @@ def router_weight_bits_np(seed: int, layer: int) -> np.ndarray:
 def layer_weights_np(seed: int, layer: int, experts=None):
     """(W_gate, W_up, W_down) bf16 bits of one layer on the host."""
     return tuple(weight_bits_np(seed, layer, w, experts) for w in (W_GATE, W_UP, W_DOWN))
+
+
+SHARED_SEED_OFFSET = 1000
+
+
+def shared_weights_np(seed: int, layer: int, n_shared: int):
+    """(W_gate, W_up, W_down) bf16 bits of ``n_shared`` shared experts of
+    ``layer``: the generator's expert matrices 0 .. n_shared-1 of seed
+    seed + 1000 (a stream no routed expert uses)."""
+    ex = np.arange(n_shared)
+    return tuple(weight_bits_np(seed + SHARED_SEED_OFFSET, layer, w, ex)
+                 for w in (W_GATE, W_UP, W_DOWN))
 
 
 def _mix32_torch(x):

@@ -38,6 +38,9 @@ reordering beyond what the definition states:
   rows, which the CUDA path must reproduce bit for bit.
 * Stack: 23 MoE layers (24 layers with dense layer 0 -- issue #1247, opening
   paragraph), residual stream kept in bf16: h <- bf16(h + moe(h)).
+* Shared experts ("khronnuz/Ling-3.0-flash-exl3", table of quants; "Add TML
+  Inkling architecture", model description): SwiGLU FFNs of the routed
+  shape applied to every token with weight 1 (``moe_layer_shared``).
 * Block-FP8 experts (issue #1247, "What it does not cover", third bullet: the
   CUDA path reads bf16, block FP8 and NVFP4 experts): E4M3 codes with one fp32
   scale per 128 x 128 block, weight = value(code) * scale; the layer is the
@@ -382,6 +385,37 @@ def moe_layer_fp8(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | Non
         return (dequant_block_fp8(q_gate[e], s_gate[e]), dequant_block_fp8(q_up[e], s_up[e]),
                 dequant_block_fp8(q_down[e], s_down[e]))
     return moe_layer_f64(x_bits, logits, bias, weights, route_result)
+
+
+# ----------------------------------------------------------------------------
+# Shared experts
+# ----------------------------------------------------------------------------
+# The Ling family's flash model has shared experts (its EXL3 card lists them
+# beside attention among the parts kept at higher precision: "khronnuz/
+# Ling-3.0-flash-exl3", table of quants), and the Inkling model has "256
+# experts top-6 plus 2 shared" ("Add TML Inkling architecture", llama.cpp PR
+# #25731, model description).  The pages give neither their size nor how they
+# enter the sum; the reading here is the usual one: each shared expert is a
+# SwiGLU FFN of the routed experts' shape that every token passes through
+# with weight 1, added to the routed sum.
+
+def moe_layer_shared(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | None,
+                     w_gate_bits: np.ndarray, w_up_bits: np.ndarray, w_down_bits: np.ndarray,
+                     s_gate_bits: np.ndarray, s_up_bits: np.ndarray, s_down_bits: np.ndarray,
+                     route_result: RouteResult | None = None) -> np.ndarray:
+    """Routed layer plus shared experts, float64, no intermediate rounding:
+    out_t = sum_i w_i FFN_{e_i}(x_t) + sum_s FFN_s(x_t).
+
+    s_gate_bits, s_up_bits: [S, 1536, 512] bf16 bits; s_down_bits: [S, 512, 1536]
+    (S shared experts, S = 0 allowed); the routed arguments as in moe_layer.
+    """
+    out = moe_layer(x_bits, logits, bias, w_gate_bits, w_up_bits, w_down_bits,
+                    route_result=route_result)
+    x = bf16_bits_to_f64(x_bits)
+    for s in range(np.asarray(s_gate_bits).shape[0]):
+        out += expert_ffn(x, bf16_bits_to_f64(s_gate_bits[s]), bf16_bits_to_f64(s_up_bits[s]),
+                          bf16_bits_to_f64(s_down_bits[s]))
+    return out
 
 
 def rel_l2(a: np.ndarray, ref: np.ndarray) -> float:
