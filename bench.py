@@ -66,8 +66,10 @@ def parse():
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weights of the main line: bf16, or block FP8 (E4M3 codes, "
                          "power-of-two 128x128 block scales)")
+    ap.add_argument("--shared", type=int, default=0,
+                    help="shared experts (0-8) added to the main line's layer")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the decode_T16 (bf16 and FP8) measurements")
+                    help="skip the decode_T16 (bf16, FP8, shared-expert) measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens in the oracle sample")
     return ap.parse_args()
@@ -167,11 +169,12 @@ class ClockSampler:
 class LayerRun:
     """Device buffers and the five-call step of one workload."""
 
-    def __init__(self, wl: synth.Workload, dev, weights, fp8: bool = False):
+    def __init__(self, wl: synth.Workload, dev, weights, fp8: bool = False, shared=None):
         import torch
         from group_limited_routed_moe_b200 import moe
         self.moe, self.torch, self.wl, self.dev = moe, torch, wl, dev
         self.fp8 = fp8  # weights: a packed block-FP8 layer (moe_layer_fp8)
+        self.shared = shared  # None, or (packed shared experts, n_shared): moe_layer_shared
         self.T = wl.T
         tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
         self.tok = tok
@@ -210,6 +213,12 @@ class LayerRun:
         # the breakdown pass times the same kernels the layer call runs
         self.part_names = ["route", "permute", "expert_ffn", "combine"]
         self.lws = moe.alloc_layer_workspace(T, dev, fp8=fp8)
+        if shared is not None:
+            n = moe.layer_shared_workspace_bytes(T, shared[1], fp8)
+            raw = torch.empty(n + 1024, dtype=torch.uint8, device=dev)
+            off = (-raw.data_ptr()) % 1024
+            self.lws = raw[off:off + n]
+            self.launches_per_step += 2  # the shared row set and the shared experts' FFN
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
         self.write_only_flush = False
@@ -227,6 +236,12 @@ class LayerRun:
 
     def step(self):
         """One layer through the public layer call (what a user runs)."""
+        if self.shared is not None:
+            kw = {"packed_fp8": self.packed} if self.fp8 else {"packed_w": self.packed}
+            self.moe.moe_layer_shared(self.x[:self.T], self.logits[:self.T], self.bias,
+                                      self.shared[0], self.shared[1], out=self.out[:self.T],
+                                      workspace=self.lws, stream=self.stream, **kw)
+            return
         layer = self.moe.moe_layer_fp8 if self.fp8 else self.moe.moe_layer
         layer(self.x[:self.T], self.logits[:self.T], self.bias, self.packed,
               out=self.out[:self.T], workspace=self.lws, stream=self.stream)
@@ -371,7 +386,7 @@ class LayerRun:
         x_h = torch.from_numpy(self.tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
         lg_h = torch.from_numpy(self.tok.logits).pin_memory()
         outs_h = [torch.empty((T, 1536), dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
-        pipe = moe.HostPipeline(T, self.dev, depth, fp8=self.fp8)
+        pipe = moe.HostPipeline(T, self.dev, depth, fp8=self.fp8, shared=self.shared)
 
         def run(n):
             for k in range(n):
@@ -527,6 +542,39 @@ def decode_line(wl2, dev, packed, fp8, steps, warmup, peaks, peak_kind, barrier)
     return out
 
 
+def shared_layer(dev, n_shared):
+    """n_shared synthetic shared experts of layer 0, packed."""
+    import torch
+    from group_limited_routed_moe_b200 import moe
+    bits = synth.shared_weights_np(0, 0, n_shared)
+    dev_t = [torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16) for b in bits]
+    return moe.moe_pack_shared(*dev_t), n_shared
+
+
+def shared_line(wl2, dev, packed, shared, routed_ms, steps, warmup, peaks, barrier):
+    """The decode batch with shared experts: whole-layer steps, and the shared
+    experts' extra time against the routed-only layer, over their HBM bytes."""
+    run = LayerRun(wl2, dev, packed, shared=shared)
+    clk = ClockSampler(int(dev.index or 0))
+    n = max(steps, 50)
+    with clk:
+        st, _ = run.timed(n, warmup, barrier)
+    ms = float(st.mean())
+    extra_us = (ms - routed_ms) * 1e3
+    nbytes = shared[1] * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + \
+        wl2.T * 1536 * 2 + shared[1] * wl2.T * 1536 * 2
+    peak = float(peaks["hbm_gbs"])
+    return {"value": round(wl2.T / (ms * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 5), "n_shared": shared[1],
+            "shared_extra_us": round(extra_us, 2),
+            "shared_roofline": {"bound": "hbm", "bytes": nbytes,
+                                "achieved": round(nbytes / max(extra_us, 1e-3) / 1e3, 1),
+                                "peak": peak, "unit": "GB/s",
+                                "note": "the shared experts' weights, x and their y rows over the "
+                                        "layer's extra time against the routed-only layer"},
+            "gpu_launches": run.launches_per_step * n, "clocks": clk.summary()}
+
+
 def fp8_layer(dev):
     """The synthetic block-FP8 checkpoint of layer 0 (power-of-two block scales),
     packed, and its host codes and scales."""
@@ -575,7 +623,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     fp8 = args.weights == "fp8"
     wl = synth.WORKLOADS[args.workload]
-    run = LayerRun(wl, dev, fp8_packed if fp8 else packed, fp8=fp8)
+    shared = shared_layer(dev, args.shared) if args.shared > 0 else None
+    run = LayerRun(wl, dev, fp8_packed if fp8 else packed, fp8=fp8, shared=shared)
     clk = ClockSampler(local)
     with clk:
         steps_ms, wall = run.timed(args.steps, args.warmup, barrier)
@@ -596,6 +645,7 @@ def run_ours(args):
         "config": {"workload": wl.name, "T": wl.T, "T_buf": wl.T_buf, "hidden": 1536,
                    "weights": ("block-FP8 experts (E4M3 codes, power-of-two 128x128 block scales)"
                                if fp8 else "bf16 experts"),
+                   "shared_experts": args.shared,
                    "experts": 128, "groups": 8, "keep_groups": 4, "topk": 8, "inter": 512,
                    "parallelism": f"dp{world} (independent batch per GPU)",
                    "l2": ("256 MB buffer overwritten, then another 256 MB buffer read, before "
@@ -623,6 +673,12 @@ def run_ours(args):
                 continue  # that is the main line
             line[key] = decode_line(wl2, dev, p2, f2, args.steps, args.warmup, peaks, peak_kind,
                                     barrier)
+            line["gpu_launches"] += line[key]["gpu_launches"]
+        if "decode_T16" in line:
+            key = "decode_T16_shared1"
+            line[key] = shared_line(wl2, dev, packed, shared_layer(dev, 1),
+                                    line["decode_T16"]["ms_per_step"], args.steps, args.warmup,
+                                    peaks, barrier)
             line["gpu_launches"] += line[key]["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         if fp8:

@@ -1,8 +1,10 @@
 // combine.cuh -- step 4: weighted combine of the 8 expert outputs of every
 // token, back in token order.
 //
-// out[t] = bf16( residual[t] + sum_{slot} w[t,slot] * y_perm[inv_perm[8t+slot]] )
-// with y_perm in fp16 (the down GEMM's output) and the residual in bf16.
+// out[t] = bf16( residual[t] + sum_{slot} w[t,slot] * y_perm[inv_perm[8t+slot]]
+//                 + sum_{s < n_shared} y_shared[s*T + t] )
+// with y_perm and y_shared in fp16 (the down GEMMs' outputs) and the residual
+// in bf16; the shared experts' rows (weight 1) follow the routed slots.
 // The "real MoE routing + weighted layer" of "HelloSun/ling30tiny" (section
 // 數值檢查摘要) is this sum.  It is done in gather form: each token reads its 8
 // rows, adds them in fp32 in slot order and rounds once, so the result is
@@ -18,7 +20,8 @@ constexpr int kCombineThreads = kH / 8;  // 192
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint16_t* __restrict__ y_perm, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ inv_perm, int64_t T,
-                   const __nv_bfloat16* residual, __nv_bfloat16* out) {
+                   const __nv_bfloat16* residual, __nv_bfloat16* out,
+                   const uint16_t* __restrict__ y_shared, int n_shared) {
   griddep_launch_dependents();
   griddep_wait();
   const int64_t t = blockIdx.x;
@@ -51,6 +54,15 @@ __global__ void __launch_bounds__(kCombineThreads)
       acc[2 * i + 1] = fmaf(w[s], f16_hi(q[i]), acc[2 * i + 1]);
     }
   }
+  for (int s = 0; s < n_shared; ++s) {
+    const uint4 sv = __ldg(reinterpret_cast<const uint4*>(y_shared + (s * T + t) * kH + col));
+    const uint32_t q[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += f16_lo(q[i]);
+      acc[2 * i + 1] += f16_hi(q[i]);
+    }
+  }
   if (residual != nullptr) {
     const uint4 rv = *reinterpret_cast<const uint4*>(residual + t * kH + col);
     const uint32_t q[4] = {rv.x, rv.y, rv.z, rv.w};
@@ -66,6 +78,25 @@ __global__ void __launch_bounds__(kCombineThreads)
   o.z = pack_bf16x2(acc[4], acc[5]);
   o.w = pack_bf16x2(acc[6], acc[7]);
   *reinterpret_cast<uint4*>(out + t * kH + col) = o;
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// The shared experts' row set: every token is one row of every shared expert,
+// expert s (< n_shared) owning rows s*T .. s*T + T-1 in token order, in the
+// offsets / perm_src form of the routed permutation (perm_src = 8t: token t,
+// slot 0).  Also zeroes the work counters offsets[129 ..] of the expert FFN.
+__global__ void __launch_bounds__(256)
+    shared_rows_kernel(int64_t T, int n_shared, int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ perm_src) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i < kOffsetsLen)
+    offsets[i] = i <= kE ? static_cast<int32_t>(T * (i < n_shared ? i : n_shared)) : 0;
+  if (i < n_shared * T) perm_src[i] = static_cast<int32_t>((i % T) * kTopK);
 }
 
 }  // namespace moe

@@ -5,6 +5,7 @@
 // (moe_get_device_status() excepted, which copies one status word).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -27,7 +28,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 1024;  // gate/up keeps padding rows of A zeroed up to this T
@@ -332,14 +333,16 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                     static_cast<int*>(nullptr), g_timeout_ns.load());
 }
 
+// n_exp: experts in the pack (128, or the shared experts' count), d_off: start
+// of its down region in elements; only experts with rows in `offsets` are read.
 int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                   const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, int sms,
-                  cudaStream_t s) {
+                  cudaStream_t s, int n_exp = kE, int64_t d_off = kPackGuElems) {
   if (T <= kSkinnyMaxT) {  // both GEMMs in one launch (see expert_ffn_skinny.cuh)
     CUtensorMap tw1, tw2, th;
-    int rc = make_tmap(&tw1, packed, kH, uint64_t(kE) * 2 * kI, 64,
+    int rc = make_tmap(&tw1, packed, kH, uint64_t(n_exp) * 2 * kI, 64,
                        CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-    if (!rc) rc = make_tmap(&tw2, packed + kPackGuElems, kI, uint64_t(kE) * kH, skinny::BMW,
+    if (!rc) rc = make_tmap(&tw2, packed + d_off, kI, uint64_t(n_exp) * kH, skinny::BMW,
                             CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
                             CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -353,9 +356,9 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
   }
   // both GEMMs in one launch (see expert_ffn.cuh)
   CUtensorMap tb1, tb2, ta2;
-  int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
+  int rc = make_tmap(&tb1, packed, kH, uint64_t(n_exp) * 2 * kI, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-  if (!rc) rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
+  if (!rc) rc = make_tmap(&tb2, packed + d_off, kI, uint64_t(n_exp) * kH, ffn::BN,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (!rc) rc = make_tmap(&ta2, h, kI, static_cast<uint64_t>(T) * kTopK, ffn::BM,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -405,20 +408,38 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
 }
 
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
-               const moe_bf16* residual, moe_bf16* out, cudaStream_t s) {
+               const moe_bf16* residual, moe_bf16* out, cudaStream_t s,
+               const moe_bf16* y_shared = nullptr, int n_shared = 0) {
   return launch_pdl("combine_kernel launch", combine_kernel, dim3(static_cast<unsigned>(T)),
                     dim3(kCombineThreads), 0, s, reinterpret_cast<const uint16_t*>(y), w, inv, T,
                     reinterpret_cast<const __nv_bfloat16*>(residual),
-                    reinterpret_cast<__nv_bfloat16*>(out));
+                    reinterpret_cast<__nv_bfloat16*>(out),
+                    reinterpret_cast<const uint16_t*>(y_shared), n_shared);
+}
+
+// The shared experts' FFN: their row set (every token, once per shared
+// expert), then the grouped FFN on the shared pack.
+constexpr int kMaxShared = kTopK;  // n_shared * T rows fit the routed buffers' bounds
+int do_shared_ffn(const moe_bf16* x, const moe_bf16* packed_shared, int n_shared, int64_t T,
+                  int32_t* offsets, int32_t* perm_src, moe_bf16* h, moe_bf16* y, int sms,
+                  cudaStream_t s) {
+  const int64_t n = std::max<int64_t>(kOffsetsLen, n_shared * T);
+  int rc = launch_pdl("shared_rows_kernel launch", shared_rows_kernel,
+                      dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, T, n_shared,
+                      offsets, perm_src);
+  if (rc) return rc;
+  return do_expert_ffn(x, packed_shared, offsets, perm_src, T, h, y, sms, s, n_shared,
+                       int64_t(n_shared) * kPackGuPerExpert);
 }
 
 // workspace carve-up of moe_layer
 struct LayerWs {
-  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, dq, total;
+  size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, dq;
+  size_t sh_offsets, sh_perm, sh_h, sh_y, total;
 };
 // fp8: the block-FP8 layer, which above kSkinnyMaxT tokens also needs room for
-// the expanded bf16/fp16 layer.
-LayerWs layer_ws(int64_t T, bool fp8 = false) {
+// the expanded bf16/fp16 layer; n_shared: shared experts' rows and results.
+LayerWs layer_ws(int64_t T, bool fp8 = false, int n_shared = 0) {
   LayerWs L{};
   const size_t n = static_cast<size_t>(T) * kTopK;
   size_t o = 0;
@@ -438,6 +459,11 @@ LayerWs layer_ws(int64_t T, bool fp8 = false) {
   L.y = take(n * kH * 2);
   L.logits = take(static_cast<size_t>(T) * kE * 4);  // used by moe_layer_routed
   L.dq = take(fp8 && T > kSkinnyMaxT ? static_cast<size_t>(kPackElems) * 2 : 0);
+  const size_t ns = static_cast<size_t>(n_shared) * static_cast<size_t>(T);
+  L.sh_offsets = take(n_shared ? kOffsetsLen * 4 : 0);
+  L.sh_perm = take(ns * 4);
+  L.sh_h = take(ns * kI * 2);
+  L.sh_y = take(ns * kH * 2);
   L.total = o;
   return L;
 }
@@ -488,9 +514,9 @@ int moe_pack_weights(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf1
   if (rc) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 ggu(kI / 32, kH / 32, kE), gd(kH / 32, kI / 32, kE);
-  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_gate, packed, kH, kI, 0);
-  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_up, packed, kH, kI, 1);
-  pack_transpose_kernel<<<gd, 256, 0, s>>>(w_down, packed, kI, kH, 2);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_gate, packed, kH, kI, 0, kPackGuElems);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_up, packed, kH, kI, 1, kPackGuElems);
+  pack_transpose_kernel<<<gd, 256, 0, s>>>(w_down, packed, kI, kH, 2, kPackGuElems);
   return launch_check("pack_transpose_kernel launch");
 }
 
@@ -615,7 +641,8 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
                const moe_bf16* packed_router, const float* bias, const moe_bf16* packed_w,
                int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
                float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream,
-               const void* packed_fp8 = nullptr) {
+               const void* packed_fp8 = nullptr, const moe_bf16* packed_shared = nullptr,
+               int n_shared = 0) {
   int rc = check_T(T);
   if (rc) return rc;
   if (T == 0) return MOE_OK;
@@ -629,7 +656,11 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
               (!residual || aligned(residual, 16)) && (!topk_idx_out || aligned(topk_idx_out, 16)) &&
               (!topk_w_out || aligned(topk_w_out, 16)),
           "pointers must be 16-byte aligned");
-  const LayerWs L = layer_ws(T, fp8);
+  REQUIRE(n_shared >= 0 && n_shared <= kMaxShared, "n_shared=%d outside [0, %d]", n_shared,
+          kMaxShared);
+  REQUIRE(n_shared == 0 || (packed_shared && aligned(packed_shared, 128)),
+          "packed_shared must be a 128-byte aligned pointer when n_shared > 0");
+  const LayerWs L = layer_ws(T, fp8, n_shared);
   if (workspace_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE, "%s workspace needs %zu bytes, got %zu", fn, L.total,
                 workspace_bytes);
@@ -662,7 +693,12 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
     else
       rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
   }
-  if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s);
+  moe_bf16* y_sh = reinterpret_cast<moe_bf16*>(ws + L.sh_y);
+  if (!rc && n_shared > 0)
+    rc = do_shared_ffn(x, packed_shared, n_shared, T, reinterpret_cast<int32_t*>(ws + L.sh_offsets),
+                       reinterpret_cast<int32_t*>(ws + L.sh_perm),
+                       reinterpret_cast<moe_bf16*>(ws + L.sh_h), y_sh, sms, s);
+  if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s, y_sh, n_shared);
   return rc;
 }
 }  // namespace
@@ -790,6 +826,48 @@ int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
     return fail(MOE_ERR_INVALID_ARG, "null pointer");
   return layer_impl("moe_layer_fp8", x, logits, nullptr, bias, nullptr, T, residual, out,
                     topk_idx_out, topk_w_out, workspace, workspace_bytes, stream, packed_fp8);
+}
+
+// ---- shared experts --------------------------------------------------------------
+size_t moe_packed_shared_bytes(int n_shared) {
+  if (n_shared < 0 || n_shared > kMaxShared) return 0;
+  return static_cast<size_t>(n_shared) * (kPackGuPerExpert + kPackDPerExpert) * 2;
+}
+
+int moe_pack_shared(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                    int n_shared, moe_bf16* packed_shared, moe_stream_t stream) {
+  REQUIRE(n_shared >= 1 && n_shared <= kMaxShared, "n_shared=%d outside [1, %d]", n_shared,
+          kMaxShared);
+  REQUIRE(w_gate && w_up && w_down && packed_shared, "null pointer");
+  REQUIRE(aligned(packed_shared, 128), "packed_shared must be 128-byte aligned");
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t d_off = int64_t(n_shared) * kPackGuPerExpert;
+  const dim3 ggu(kI / 32, kH / 32, n_shared), gd(kH / 32, kI / 32, n_shared);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_gate, packed_shared, kH, kI, 0, d_off);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_up, packed_shared, kH, kI, 1, d_off);
+  pack_transpose_kernel<<<gd, 256, 0, s>>>(w_down, packed_shared, kI, kH, 2, d_off);
+  return launch_check("pack_transpose_kernel launch (shared)");
+}
+
+size_t moe_layer_shared_workspace_bytes(int64_t T, int n_shared, int fp8_routed) {
+  if (T < 0 || T > kMaxTokens || n_shared < 0 || n_shared > kMaxShared) return 0;
+  return layer_ws(T, fp8_routed != 0, n_shared).total;
+}
+
+int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
+                     const moe_bf16* packed_w, const void* packed_fp8,
+                     const moe_bf16* packed_shared, int n_shared, int64_t T,
+                     const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+                     float* topk_w_out, void* workspace, size_t workspace_bytes,
+                     moe_stream_t stream) {
+  if (T > 0 && (logits == nullptr || (packed_w == nullptr) == (packed_fp8 == nullptr)))
+    return fail(MOE_ERR_INVALID_ARG,
+                "moe_layer_shared needs logits and exactly one of packed_w, packed_fp8");
+  return layer_impl("moe_layer_shared", x, logits, nullptr, bias, packed_w, T, residual, out,
+                    topk_idx_out, topk_w_out, workspace, workspace_bytes, stream, packed_fp8,
+                    packed_shared, n_shared);
 }
 
 }  // extern "C"

@@ -27,10 +27,11 @@ constexpr int64_t kPackElems = kPackGuElems + kE * kPackDPerExpert;
 
 // dst[e][map(n)][k] = src[e][k][n] for a [K][N] source, 32x32 tiles through
 // shared memory.  mode 0: gate (rows 256*(n/128) + n%128, row length 1536),
-// mode 1: up (+128), mode 2: down (row n, row length 512).
+// mode 1: up (+128), mode 2: down (row n, row length 512) in the region that
+// starts d_off elements into dst (after all experts' gate/up rows).
 __global__ void __launch_bounds__(256)
     pack_transpose_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int K,
-                          int N, int mode) {
+                          int N, int mode, int64_t d_off) {
   __shared__ uint16_t tile[32][33];
   const int e = blockIdx.z;
   const int n0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
@@ -43,7 +44,7 @@ __global__ void __launch_bounds__(256)
   uint16_t* d;
   int64_t row_len;
   if (mode == 2) {
-    d = dst + kPackGuElems + static_cast<int64_t>(e) * kPackDPerExpert;
+    d = dst + d_off + static_cast<int64_t>(e) * kPackDPerExpert;
     row_len = kI;
   } else {
     d = dst + static_cast<int64_t>(e) * kPackGuPerExpert;

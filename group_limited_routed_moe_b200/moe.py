@@ -71,6 +71,10 @@ _SIGS = {
     "moe_layer_fp8_workspace_bytes": ([_i64], _sz),
     "moe_expert_ffn_fp8_workspace_bytes": ([_i64], _sz),
     "moe_expert_ffn_fp8": ([_p, _p, _p, _p, _i64, _p, _p, _p, _sz, _p], _i32),
+    "moe_packed_shared_bytes": ([_i32], _sz),
+    "moe_pack_shared": ([_p, _p, _p, _i32, _p, _p], _i32),
+    "moe_layer_shared_workspace_bytes": ([_i64, _i32, _i32], _sz),
+    "moe_layer_shared": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_layer_fp8": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -377,6 +381,55 @@ def moe_layer_fp8(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | No
     return out
 
 
+# ----------------------------------------------------------------- shared experts
+
+def packed_shared_bytes(n_shared: int) -> int:
+    return int(lib.moe_packed_shared_bytes(n_shared))
+
+
+def layer_shared_workspace_bytes(T: int, n_shared: int, fp8_routed: bool) -> int:
+    return int(lib.moe_layer_shared_workspace_bytes(T, n_shared, int(bool(fp8_routed))))
+
+
+def moe_pack_shared(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                    packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Re-layout n_shared shared experts ([n, 1536, 512], [n, 1536, 512],
+    [n, 512, 1536] bf16; see include/moe.h)."""
+    n = w_gate.shape[0]
+    for t, shp in ((w_gate, (n, HIDDEN, INTER)), (w_up, (n, HIDDEN, INTER)),
+                   (w_down, (n, INTER, HIDDEN))):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shp or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"expected contiguous CUDA bf16 {shp}, got {t.dtype} {tuple(t.shape)}")
+    if packed is None:
+        packed = torch.empty(packed_shared_bytes(n) // 2, dtype=torch.bfloat16,
+                             device=w_gate.device)
+    _check("moe_pack_shared", lib.moe_pack_shared(_ptr(w_gate), _ptr(w_up), _ptr(w_down), n,
+                                                  _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_layer_shared(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
+                     packed_shared: torch.Tensor, n_shared: int, packed_w=None, packed_fp8=None,
+                     residual=None, out=None, topk_idx_out=None, topk_w_out=None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """moe_layer (packed_w) or moe_layer_fp8 (packed_fp8) plus n_shared shared
+    experts (see include/moe.h)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        n = layer_shared_workspace_bytes(T, n_shared, packed_fp8 is not None)
+        raw = torch.empty(n + 1024, dtype=torch.uint8, device=x.device)
+        off = (-raw.data_ptr()) % 1024
+        workspace = raw[off:off + n]
+    _check("moe_layer_shared",
+           lib.moe_layer_shared(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_w),
+                                _ptr(packed_fp8), _ptr(packed_shared), n_shared, T,
+                                _ptr(residual), _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out),
+                                _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 def moe_layer_from_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: torch.Tensor | None,
                         packed_w: torch.Tensor, x_dev: torch.Tensor, logits_dev: torch.Tensor,
                         out_dev: torch.Tensor, out_host: torch.Tensor,
@@ -404,11 +457,12 @@ class HostPipeline:
     previous call has finished.  The output of call k lands in the `out_host`
     passed to submit(); it is complete once `drain()` returns.  With fp8=True
     the weights passed to submit() are a packed block-FP8 layer and every call
-    runs moe_layer_fp8.
+    runs moe_layer_fp8.  With shared = (packed_shared, n_shared) every call
+    also runs the shared experts (moe_layer_shared).
     """
 
-    def __init__(self, T: int, device, depth: int = 2, fp8: bool = False):
-        self.T, self.depth, self.k, self.fp8 = T, depth, 0, fp8
+    def __init__(self, T: int, device, depth: int = 2, fp8: bool = False, shared=None):
+        self.T, self.depth, self.k, self.fp8, self.shared = T, depth, 0, fp8, shared
         self.last_layer = None
         self.slots = []
         for _ in range(depth):
@@ -417,8 +471,16 @@ class HostPipeline:
                 "x": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
                 "logits": torch.empty((T, N_EXPERTS), dtype=torch.float32, device=device),
                 "out": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
-                "ws": alloc_layer_workspace(T, device, fp8=fp8),
+                "ws": self._workspace(T, device),
             })
+
+    def _workspace(self, T, device):
+        if self.shared is None:
+            return alloc_layer_workspace(T, device, fp8=self.fp8)
+        n = layer_shared_workspace_bytes(T, self.shared[1], self.fp8)
+        raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+        off = (-raw.data_ptr()) % 1024
+        return raw[off:off + n]
 
     def submit(self, x_host, logits_host, out_host, bias, packed_w):
         slot = self.slots[self.k % self.depth]
@@ -429,9 +491,14 @@ class HostPipeline:
             slot["logits"].copy_(logits_host, non_blocking=True)
             if self.last_layer is not None:
                 st.wait_event(self.last_layer)
-            (moe_layer_fp8 if self.fp8 else moe_layer)(
-                slot["x"], slot["logits"], bias, packed_w, out=slot["out"], workspace=slot["ws"],
-                stream=st)
+            if self.shared is not None:
+                kw = {"packed_fp8": packed_w} if self.fp8 else {"packed_w": packed_w}
+                moe_layer_shared(slot["x"], slot["logits"], bias, self.shared[0], self.shared[1],
+                                 out=slot["out"], workspace=slot["ws"], stream=st, **kw)
+            else:
+                (moe_layer_fp8 if self.fp8 else moe_layer)(
+                    slot["x"], slot["logits"], bias, packed_w, out=slot["out"],
+                    workspace=slot["ws"], stream=st)
             self.last_layer = torch.cuda.Event()
             self.last_layer.record(st)
             out_host.copy_(slot["out"], non_blocking=True)

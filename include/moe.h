@@ -315,6 +315,47 @@ int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
                   moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
                   void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
+/* ---- shared experts --------------------------------------------------------- */
+
+/* The Ling family's flash model has shared experts ("khronnuz/Ling-3.0-flash-
+ * exl3", table of quants: kept at higher precision beside attention) and the
+ * Inkling model "256 experts top-6 plus 2 shared" ("Add TML Inkling
+ * architecture", llama.cpp PR #25731); the pages give neither their size nor
+ * how they enter the sum.  Read as the usual form: each shared expert is a
+ * SwiGLU FFN of the routed experts' shape (1536 -> 512 -> 1536) that every
+ * token passes through with weight 1:
+ *   out[t] = bf16( residual[t] + sum_slot w[t,slot] FFN_{e_slot}(x[t]) + sum_s FFN_s(x[t]) )
+ * summed in fp32 in that order (routed slots, then shared experts by index)
+ * and rounded once.  Shared experts stay bf16 with bf16 or FP8 routed experts. */
+
+/* Bytes of n_shared packed shared experts (0 <= n_shared <= 8). */
+size_t moe_packed_shared_bytes(int n_shared);
+
+/* One-time re-layout of n_shared (1..8) shared experts:
+ *   w_gate, w_up : [n_shared][1536][512] bf16;  w_down : [n_shared][512][1536] bf16
+ *   packed_shared: moe_packed_shared_bytes(n_shared) bytes, 128-byte aligned, output;
+ *                  the layout of moe_pack_weights for n_shared experts (gate/up
+ *                  K-major and interleaved, then W_down in fp16). */
+int moe_pack_shared(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                    int n_shared, moe_bf16* packed_shared, moe_stream_t stream);
+
+/* Workspace bytes moe_layer_shared needs (fp8_routed != 0: routed experts in
+ * block FP8). */
+size_t moe_layer_shared_workspace_bytes(int64_t T, int n_shared, int fp8_routed);
+
+/* moe_layer (packed_w, bf16 routed experts) or moe_layer_fp8 (packed_fp8):
+ * exactly one of the two is non-NULL; plus n_shared (0..8) shared experts
+ * from packed_shared.  The shared experts' rows (every token once per shared
+ * expert) go through the same grouped expert-FFN kernels as the routed ones,
+ * in a second launch; the combine adds their outputs.  With n_shared = 0 the
+ * result is bit for bit that of moe_layer / moe_layer_fp8. */
+int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
+                     const moe_bf16* packed_w, const void* packed_fp8,
+                     const moe_bf16* packed_shared, int n_shared, int64_t T,
+                     const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+                     float* topk_w_out, void* workspace, size_t workspace_bytes,
+                     moe_stream_t stream);
+
 /* ---- permutation without a caller workspace ------------------------------ */
 
 /* The pages describe no such call: it is moe_permute for callers that cannot

@@ -13,7 +13,7 @@ def test_exports_every_declared_symbol():
     assert len(names) >= 15
     missing = [n for n in names if not hasattr(moe.lib, n)]
     assert missing == []
-    assert moe.lib.moe_abi_version() == 3
+    assert moe.lib.moe_abi_version() == 4
 
 
 def test_sizes():
@@ -87,3 +87,29 @@ def test_fp8_sizes_and_host_validation():
     assert L.moe_pack_weights_fp8(_p(128), _p(128), None, _p(128), _p(128), _p(128), _p(128),
                                   None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_dequant_fp8(_p(136), _p(128), None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_shared_sizes_and_host_validation():
+    L = moe.lib
+    per = (1024 * 1536 + 1536 * 512) * 2
+    assert [moe.packed_shared_bytes(n) for n in (0, 1, 2, 8)] == [0, per, 2 * per, 8 * per]
+    assert moe.packed_shared_bytes(9) == 0
+    base = moe.layer_workspace_bytes(300)
+    assert moe.layer_shared_workspace_bytes(300, 0, False) == base
+    assert moe.layer_shared_workspace_bytes(300, 2, False) >= base + 2 * 300 * (4 + (512 + 1536) * 2)
+    assert moe.layer_shared_workspace_bytes(300, 2, True) >= moe.layer_fp8_workspace_bytes(300)
+    assert L.moe_pack_shared(_p(128), _p(128), _p(128), 0, _p(128), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_shared(_p(128), _p(128), _p(128), 9, _p(128), None) == moe.MOE_ERR_INVALID_ARG
+    ws = moe.layer_shared_workspace_bytes(16, 1, False)
+    # exactly one of the bf16 and FP8 routed packs
+    assert L.moe_layer_shared(_p(1024), _p(1024), None, _p(1024), _p(1024), _p(1024), 1, 16, None,
+                              _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_shared(_p(1024), _p(1024), None, None, None, _p(1024), 1, 16, None,
+                              _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
+    # shared pack required when n_shared > 0; n_shared bounded
+    assert L.moe_layer_shared(_p(1024), _p(1024), None, _p(1024), None, None, 1, 16, None,
+                              _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_shared(_p(1024), _p(1024), None, _p(1024), None, _p(1024), 9, 16, None,
+                              _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_shared(_p(1024), _p(1024), None, _p(1024), None, _p(1024), 1, 16, None,
+                              _p(1024), None, None, _p(1024), ws - 1, None) == moe.MOE_ERR_WORKSPACE
