@@ -38,6 +38,9 @@ reordering beyond what the definition states:
   rows, which the CUDA path must reproduce bit for bit.
 * Stack: 23 MoE layers (24 layers with dense layer 0 -- issue #1247, opening
   paragraph), residual stream kept in bf16: h <- bf16(h + moe(h)).
+* A second shape, 256 experts top-6 with 2 shared experts ("Add TML Inkling
+  architecture", model description), with tiny's group rule scaled to 8
+  groups of 32 keeping 4 (``route_e256``).
 * Shared experts ("khronnuz/Ling-3.0-flash-exl3", table of quants; "Add TML
   Inkling architecture", model description): SwiGLU FFNs of the routed
   shape applied to every token with weight 1 (``moe_layer_shared``).
@@ -385,6 +388,24 @@ def moe_layer_fp8(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | Non
         return (dequant_block_fp8(q_gate[e], s_gate[e]), dequant_block_fp8(q_up[e], s_up[e]),
                 dequant_block_fp8(q_down[e], s_down[e]))
     return moe_layer_f64(x_bits, logits, bias, weights, route_result)
+
+
+# ----------------------------------------------------------------------------
+# Second MoE shape: 256 experts, top-6
+# ----------------------------------------------------------------------------
+# The Inkling model has "256 experts top-6 plus 2 shared" ("Add TML Inkling
+# architecture", llama.cpp PR #25731, model description); the pages give no
+# group structure, hidden or intermediate size for it.  Read with tiny's group
+# rule scaled to 256 experts (8 groups of 32, 4 kept) and tiny's expert shape
+# (1536 -> 512 -> 1536), so that the same layer definition applies with 256
+# experts and 6 slots; the two shared experts are those of moe_layer_shared.
+
+E256_EXPERTS, E256_GROUPS, E256_KEEP, E256_TOPK = 256, 8, 4, 6
+
+
+def route_e256(logits: np.ndarray, bias: np.ndarray | None) -> RouteResult:
+    """route() on the second shape: logits [T, 256], 8 groups of 32, keep 4, top-6."""
+    return route(logits, bias, n_groups=E256_GROUPS, keep=E256_KEEP, topk=E256_TOPK)
 
 
 # ----------------------------------------------------------------------------
