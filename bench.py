@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weights of the main line: bf16, or block FP8 (E4M3 codes, "
                          "power-of-two 128x128 block scales)")
+    ap.add_argument("--e256-prefill", action="store_true",
+                    help="also time the 256-expert shape at T=8189 (secondary line)")
     ap.add_argument("--shared", type=int, default=0,
                     help="shared experts (0-8) added to the main line's layer")
     ap.add_argument("--no-secondary", action="store_true",
@@ -575,6 +577,70 @@ def shared_line(wl2, dev, packed, shared, routed_ms, steps, warmup, peaks, barri
             "gpu_launches": run.launches_per_step * n, "clocks": clk.summary()}
 
 
+def e256_line(T, dev, steps, warmup, peaks, barrier, seed=5):
+    """The second MoE shape (256 experts in 8 groups of 32, keep 4, top-6, plus
+    2 shared experts) on T synthetic tokens: whole-layer steps through
+    moe_layer_e256 after the same L2 flush, and the layer's fractions of the
+    HBM and tensor roofs (the touched experts' weights and the layer's flops)."""
+    import torch
+    from group_limited_routed_moe_b200 import moe
+    halves = []
+    for half in (0, 1):
+        w = [synth.e256_weight_bits_torch(0, 0, m, half, dev)
+             for m in (synth.W_GATE, synth.W_UP, synth.W_DOWN)]
+        halves.append(moe.moe_pack_weights(*w))
+        del w
+    sh_packed, n_sh = shared_layer(dev, 2)
+    tok = synth.make_tokens_e256(T, seed)
+    x = torch.from_numpy(tok.x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    lg = torch.from_numpy(tok.logits).to(dev)
+    bias = torch.from_numpy(tok.bias).to(dev)
+    out = torch.empty((T, 1536), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((T, 6), dtype=torch.int32, device=dev)
+    n = moe.layer_e256_workspace_bytes(T, n_sh)
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=dev)
+    ws = raw[(-raw.data_ptr()) % 1024:][:n]
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_layer_e256(x, lg, bias, halves[0], halves[1], sh_packed, n_sh, out=out,
+                           topk_idx_out=idx, workspace=ws, stream=stream)
+
+    def flush():
+        flush_w.fill_(1)
+        flush_r.max()
+        torch.cuda._sleep(1_000_000)
+    for _ in range(warmup):
+        flush()
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    clk = ClockSampler(int(dev.index or 0))
+    barrier()
+    torch.cuda.synchronize()
+    with clk:
+        for k in range(steps):
+            flush()
+            evs[k][0].record(stream)
+            step()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    d = int(np.unique(idx.cpu().numpy()).size)
+    nbytes = (d + n_sh) * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * (1536 * 4 + 512)
+    flops = FLOPS_PER_ROW * (6 + n_sh) * T
+    nb = (T + 127) // 128
+    launches = 4 + 2 + (2 if n_sh else 0) + 1  # route, count, scan, scatter; 2 FFN; shared; combine
+    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 5),
+            "shape": "256 experts in 8 groups of 32, keep 4, top-6, 2 shared experts",
+            "T": T, "distinct_experts": d, "count_sort_blocks": nb,
+            "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),
+            "gpu_launches": launches * steps, "clocks": clk.summary()}
+
+
 def fp8_layer(dev):
     """The synthetic block-FP8 checkpoint of layer 0 (power-of-two block scales),
     packed, and its host codes and scales."""
@@ -674,12 +740,19 @@ def run_ours(args):
             line[key] = decode_line(wl2, dev, p2, f2, args.steps, args.warmup, peaks, peak_kind,
                                     barrier)
             line["gpu_launches"] += line[key]["gpu_launches"]
+        line["decode_T16_e256"] = e256_line(16, dev, max(args.steps, 50), args.warmup, peaks,
+                                            barrier)
+        line["gpu_launches"] += line["decode_T16_e256"]["gpu_launches"]
         if "decode_T16" in line:
             key = "decode_T16_shared1"
             line[key] = shared_line(wl2, dev, packed, shared_layer(dev, 1),
                                     line["decode_T16"]["ms_per_step"], args.steps, args.warmup,
                                     peaks, barrier)
             line["gpu_launches"] += line[key]["gpu_launches"]
+    if args.e256_prefill:
+        line["prefill_T8189_e256"] = e256_line(8189, dev, max(5, args.steps // 5), args.warmup,
+                                               peaks, barrier)
+        line["gpu_launches"] += line["prefill_T8189_e256"]["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         if fp8:
             hw = [t.cpu().numpy() for t in fp8_dev]

@@ -17,6 +17,9 @@ namespace moe {
 
 constexpr int kCombineThreads = kH / 8;  // 192
 
+// NS: slots a token uses (8, or 6 in the 256-expert shape); topk_w has NS
+// entries per token, inv_perm always kTopK (slots NS .. 7 unused).
+template <int NS>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint16_t* __restrict__ y_perm, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ inv_perm, int64_t T,
@@ -29,12 +32,12 @@ __global__ void __launch_bounds__(kCombineThreads)
   const int col = threadIdx.x * 8;
   const int64_t nrows = T * kTopK;
 
-  uint4 v[kTopK];
-  float w[kTopK];
+  uint4 v[NS];
+  float w[NS];
 #pragma unroll
-  for (int s = 0; s < kTopK; ++s) {
+  for (int s = 0; s < NS; ++s) {
     const int64_t r = __ldg(inv_perm + t * kTopK + s);
-    w[s] = __ldg(topk_w + t * kTopK + s);
+    w[s] = __ldg(topk_w + t * NS + s);
     if (r >= 0 && r < nrows) {
       v[s] = __ldg(reinterpret_cast<const uint4*>(y_perm + r * kH + col));
     } else {
@@ -46,7 +49,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-  for (int s = 0; s < kTopK; ++s) {
+  for (int s = 0; s < NS; ++s) {
     const uint32_t q[4] = {v[s].x, v[s].y, v[s].z, v[s].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

@@ -1,0 +1,236 @@
+// e256.cuh -- routing and row permutation for the second MoE shape: 256
+// experts top-6 ("Add TML Inkling architecture", llama.cpp PR #25731, model
+// description: "256 experts top-6 plus 2 shared").  The pages give no group
+// structure for it; tiny's rule is scaled to 8 groups of 32 experts, 4 kept.
+// Scores, ties and combine weights follow route.cuh (same keys, same shifted
+// weight ratio).
+//
+// The expert FFN of this shape reuses the 128-expert grouped kernels
+// unchanged, on two packs (experts 0..127 and 128..255): the permutation below
+// is one stable counting sort over all 256 experts, and each half gets its own
+// 264-word offsets array whose 129 offsets are absolute rows of the shared
+// perm_src / h / y_perm buffers.  Items keep the 8-slot numbering t*8 + slot
+// of the 128-expert path (slots 6 and 7 unused), so the kernels' token index
+// perm_src >> 3 and the combine's inv_perm stride stay as they are.
+#pragma once
+#include "common.cuh"
+#include "route.cuh"
+
+namespace moe {
+namespace e256 {
+
+constexpr int kE2 = 256, kG2 = 8, kGS2 = 32, kKeep2 = 4, kTopK2 = 6;
+constexpr int kPerLane = kE2 / 32;        // 8 experts per lane, 4 lanes per group
+constexpr int kBlockTokens = 128;         // tokens per block of the counting sort
+constexpr int kRouteWarps2 = 8;           // tokens (warps) per route block
+
+// One warp per token.  Lane l owns experts 8l .. 8l+7 (group l / 4).
+__global__ void __launch_bounds__(kRouteWarps2 * 32)
+    route_e256_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                      int64_t T, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const unsigned FULL = 0xFFFFFFFFu;
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps2 + (threadIdx.x >> 5);
+  if (t >= T) return;  // whole warp
+  const int grp = lane >> 2;
+
+  float lg[kPerLane], bs[kPerLane];
+  {
+    const float4* src = reinterpret_cast<const float4*>(logits + t * kE2 + kPerLane * lane);
+    const float4* bsrc = reinterpret_cast<const float4*>(bias + kPerLane * lane);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float4 v = __ldg(src + q);
+      lg[4 * q] = v.x; lg[4 * q + 1] = v.y; lg[4 * q + 2] = v.z; lg[4 * q + 3] = v.w;
+      const float4 b = bias != nullptr ? __ldg(bsrc + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      bs[4 * q] = b.x; bs[4 * q + 1] = b.y; bs[4 * q + 2] = b.z; bs[4 * q + 3] = b.w;
+    }
+  }
+  // keys, and this lane's two best (key, z)
+  unsigned long long key[kPerLane];
+  unsigned long long k1 = 0ull, k2 = 0ull;
+  double z1 = 0.0, z2 = 0.0;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const double z = static_cast<double>(lg[i]) + static_cast<double>(bs[i]);
+    key[i] = route_key(z);
+    if (key[i] > k1) {
+      k2 = k1; z2 = z1; k1 = key[i]; z1 = z;
+    } else if (key[i] > k2) {
+      k2 = key[i]; z2 = z;
+    }
+  }
+  // the group's two best over its 4 lanes
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    const unsigned long long o1 = __shfl_xor_sync(FULL, k1, off);
+    const unsigned long long o2 = __shfl_xor_sync(FULL, k2, off);
+    const double y1 = __shfl_xor_sync(FULL, z1, off);
+    const double y2 = __shfl_xor_sync(FULL, z2, off);
+    // merge the sorted pairs (k1 >= k2) and (o1 >= o2)
+    if (o1 > k1) {
+      if (k1 > o2) { k2 = k1; z2 = z1; } else { k2 = o2; z2 = y2; }
+      k1 = o1; z1 = y1;
+    } else if (o1 > k2) {
+      k2 = o1; z2 = y1;
+    }
+  }
+  const double gscore = sigmoid_f64(z1) + sigmoid_f64(z2);
+  // rank of this lane's group among the 8 (ties: lower index first)
+  int rank = 0;
+#pragma unroll
+  for (int j = 0; j < kG2; ++j) {
+    const double gj = __shfl_sync(FULL, gscore, 4 * j);
+    rank += (gj > gscore) || (gj == gscore && j < grp);
+  }
+  if (rank >= kKeep2) {
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) key[i] = 0ull;
+  }
+  int sel = -1;  // lane k ends up holding the k-th chosen expert
+#pragma unroll 1
+  for (int k = 0; k < kTopK2; ++k) {
+    unsigned long long bk = key[0];
+    int bi = 0;
+#pragma unroll
+    for (int i = 1; i < kPerLane; ++i)
+      if (key[i] > bk) { bk = key[i]; bi = i; }  // strict: lower index on ties
+    int be = kPerLane * lane + bi;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const unsigned long long ok = __shfl_xor_sync(FULL, bk, off);
+      const int oe = __shfl_xor_sync(FULL, be, off);
+      if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
+    }
+    if (lane == k) sel = be;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)
+      if (kPerLane * lane + i == be) key[i] = 0ull;
+  }
+  // combine weights over the 6 chosen, as route.cuh
+  const bool mine = lane < kTopK2;
+  const double l = mine ? static_cast<double>(__ldg(logits + t * kE2 + sel)) : -INFINITY;
+  double m = l;
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) m = fmax(m, __shfl_xor_sync(FULL, m, off));
+  double r = 0.0;
+  if (mine)
+    r = m >= 0.0 ? sigmoid_f64(l) / sigmoid_f64(m) : exp(l - m) * (1.0 + exp(m)) / (1.0 + exp(l));
+  double tot = r;
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) tot += __shfl_xor_sync(FULL, tot, off);
+  if (mine) {
+    topk_idx[t * kTopK2 + lane] = sel;
+    topk_w[t * kTopK2 + lane] = static_cast<float>(r / tot);
+  }
+}
+
+// Counting sort, pass 1: per block of 128 tokens, the rows each expert gets.
+__global__ void __launch_bounds__(256)
+    count_e256_kernel(const int32_t* __restrict__ idx, int64_t T, int32_t* __restrict__ hist) {
+  __shared__ int cnt[kE2];
+  griddep_launch_dependents();
+  griddep_wait();
+  cnt[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kBlockTokens;
+  for (int i = threadIdx.x; i < kBlockTokens * kTopK2; i += blockDim.x) {
+    const int64_t t = t0 + i / kTopK2;
+    if (t < T) {
+      const int e = idx[t * kTopK2 + i % kTopK2];
+      if (e >= 0 && e < kE2) atomicAdd(&cnt[e], 1);
+      else record_status(kSiteBadIndex);
+    }
+  }
+  __syncthreads();
+  hist[static_cast<int64_t>(blockIdx.x) * kE2 + threadIdx.x] = cnt[threadIdx.x];
+}
+
+// Pass 2 (one block, a thread per expert): expert offsets, each block's first
+// row for each expert (in place of its count), and the two halves' 264-word
+// offsets arrays (work counters zeroed).
+__global__ void __launch_bounds__(256)
+    scan_e256_kernel(int32_t* __restrict__ hist, int nb, int32_t* __restrict__ counts,
+                     int32_t* __restrict__ offsets, int32_t* __restrict__ off_lo,
+                     int32_t* __restrict__ off_hi) {
+  __shared__ int wsum[8];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+  int c = 0;
+  for (int b = 0; b < nb; ++b) c += hist[static_cast<int64_t>(b) * kE2 + e];
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int j = 0; j < w; ++j) base += wsum[j];
+  const int start = base + incl - c;  // exclusive prefix
+  counts[e] = c;
+  offsets[e] = start;
+  if (e == kE2 - 1) offsets[kE2] = start + c;
+  int run = start;
+  for (int b = 0; b < nb; ++b) {
+    const int64_t i = static_cast<int64_t>(b) * kE2 + e;
+    const int v = hist[i];
+    hist[i] = run;
+    run += v;
+  }
+  // halves: absolute rows, then zeroed work counters
+  __syncthreads();
+  const int half = e >> 7, j = e & 127;
+  int32_t* dst = half ? off_hi : off_lo;
+  dst[j] = start;
+  if (j == 127) dst[128] = start + c;
+  for (int i = 129 + j; i < kOffsetsLen; i += 128) dst[i] = 0;
+}
+
+// Pass 3: rows.  Items of one block go to their expert's rows in token order:
+// the rank of token t among the block's tokens that chose e is the number of
+// bits below t in e's 128-bit token bitmap.
+__global__ void __launch_bounds__(256)
+    scatter_e256_kernel(const int32_t* __restrict__ idx, int64_t T,
+                        const int32_t* __restrict__ hist, int32_t* __restrict__ perm_src,
+                        int32_t* __restrict__ inv_perm) {
+  __shared__ uint32_t bits[kE2][kBlockTokens / 32];
+  griddep_launch_dependents();
+  griddep_wait();
+  for (int i = threadIdx.x; i < kE2 * (kBlockTokens / 32); i += blockDim.x)
+    (&bits[0][0])[i] = 0u;
+  __syncthreads();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kBlockTokens;
+  for (int i = threadIdx.x; i < kBlockTokens * kTopK2; i += blockDim.x) {
+    const int tl = i / kTopK2;
+    const int64_t t = t0 + tl;
+    if (t < T) {
+      const int e = idx[t * kTopK2 + i % kTopK2];
+      if (e >= 0 && e < kE2) atomicOr(&bits[e][tl >> 5], 1u << (tl & 31));
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBlockTokens * kTopK; i += blockDim.x) {
+    const int tl = i / kTopK, slot = i % kTopK;
+    const int64_t t = t0 + tl;
+    if (t >= T) continue;
+    if (slot >= kTopK2) {  // slots 6 and 7 of the 8-slot numbering are unused
+      inv_perm[t * kTopK + slot] = -1;
+      continue;
+    }
+    const int e = idx[t * kTopK2 + slot];
+    if (e < 0 || e >= kE2) continue;
+    int rank = __popc(bits[e][tl >> 5] & ((1u << (tl & 31)) - 1u));
+    for (int q = 0; q < (tl >> 5); ++q) rank += __popc(bits[e][q]);
+    const int row = hist[static_cast<int64_t>(blockIdx.x) * kE2 + e] + rank;
+    perm_src[row] = static_cast<int32_t>(t * kTopK + slot);
+    inv_perm[t * kTopK + slot] = row;
+  }
+}
+
+}  // namespace e256
+}  // namespace moe

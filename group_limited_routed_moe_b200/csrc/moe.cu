@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "expert_ffn.cuh"
 #include "expert_ffn_skinny.cuh"
+#include "e256.cuh"
 #include "fp8.cuh"
 #include "pack.cuh"
 #include "permute.cuh"
@@ -28,7 +29,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kAbiVersion = 4;
+constexpr int kAbiVersion = 5;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 1024;  // gate/up keeps padding rows of A zeroed up to this T
@@ -410,7 +411,7 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
                const moe_bf16* residual, moe_bf16* out, cudaStream_t s,
                const moe_bf16* y_shared = nullptr, int n_shared = 0) {
-  return launch_pdl("combine_kernel launch", combine_kernel, dim3(static_cast<unsigned>(T)),
+  return launch_pdl("combine_kernel launch", combine_kernel<kTopK>, dim3(static_cast<unsigned>(T)),
                     dim3(kCombineThreads), 0, s, reinterpret_cast<const uint16_t*>(y), w, inv, T,
                     reinterpret_cast<const __nv_bfloat16*>(residual),
                     reinterpret_cast<__nv_bfloat16*>(out),
@@ -868,6 +869,146 @@ int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
   return layer_impl("moe_layer_shared", x, logits, nullptr, bias, packed_w, T, residual, out,
                     topk_idx_out, topk_w_out, workspace, workspace_bytes, stream, packed_fp8,
                     packed_shared, n_shared);
+}
+
+}  // extern "C"
+
+// ---- second MoE shape: 256 experts top-6 ------------------------------------------
+namespace {
+struct E256Ws {
+  size_t idx, w, counts, offsets, off_lo, off_hi, perm_src, inv_perm, hist, h, y;
+  size_t sh_offsets, sh_perm, sh_h, sh_y, total;
+};
+E256Ws e256_ws(int64_t T, int n_shared) {
+  E256Ws L{};
+  const size_t n = static_cast<size_t>(T) * kTopK;  // 8-slot numbering, 6 used
+  const size_t nb = static_cast<size_t>((T + e256::kBlockTokens - 1) / e256::kBlockTokens);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 1024);
+    return at;
+  };
+  L.idx = take(static_cast<size_t>(T) * e256::kTopK2 * 4);
+  L.w = take(static_cast<size_t>(T) * e256::kTopK2 * 4);
+  L.counts = take(e256::kE2 * 4);
+  L.offsets = take((e256::kE2 + 1) * 4);
+  L.off_lo = take(kOffsetsLen * 4);
+  L.off_hi = take(kOffsetsLen * 4);
+  L.perm_src = take(n * 4);
+  L.inv_perm = take(n * 4);
+  L.hist = take(nb * e256::kE2 * 4);
+  L.h = take(n * kI * 2);
+  L.y = take(n * kH * 2);
+  const size_t ns = static_cast<size_t>(n_shared) * static_cast<size_t>(T);
+  L.sh_offsets = take(n_shared ? kOffsetsLen * 4 : 0);
+  L.sh_perm = take(ns * 4);
+  L.sh_h = take(ns * kI * 2);
+  L.sh_y = take(ns * kH * 2);
+  L.total = o;
+  return L;
+}
+
+int do_route_e256(const float* logits, const float* bias, int64_t T, int32_t* idx, float* w,
+                  cudaStream_t s) {
+  const int64_t blocks = (T + e256::kRouteWarps2 - 1) / e256::kRouteWarps2;
+  return launch_pdl("route_e256_kernel launch", e256::route_e256_kernel,
+                    dim3(static_cast<unsigned>(blocks)), dim3(e256::kRouteWarps2 * 32), 0, s,
+                    logits, bias, T, idx, w);
+}
+}  // namespace
+
+extern "C" {
+
+int moe_route_e256(const float* logits, const float* bias, int64_t T, int32_t* topk_idx,
+                   float* topk_w, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(logits && topk_idx && topk_w, "null pointer");
+  REQUIRE(aligned(logits, 16) && (!bias || aligned(bias, 16)) && aligned(topk_idx, 16) &&
+              aligned(topk_w, 16),
+          "pointers must be 16-byte aligned");
+  rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  return do_route_e256(logits, bias, T, topk_idx, topk_w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_layer_e256_workspace_bytes(int64_t T, int n_shared) {
+  if (T < 0 || T > kMaxTokens || n_shared < 0 || n_shared > kMaxShared) return 0;
+  return e256_ws(T, n_shared).total;
+}
+
+int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
+                   const moe_bf16* packed_lo, const moe_bf16* packed_hi,
+                   const moe_bf16* packed_shared, int n_shared, int64_t T,
+                   const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+                   float* topk_w_out, void* workspace, size_t workspace_bytes,
+                   moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && logits && packed_lo && packed_hi && out && workspace, "null pointer");
+  REQUIRE(n_shared >= 0 && n_shared <= kMaxShared, "n_shared=%d outside [0, %d]", n_shared,
+          kMaxShared);
+  REQUIRE(n_shared == 0 || (packed_shared && aligned(packed_shared, 128)),
+          "packed_shared must be a 128-byte aligned pointer when n_shared > 0");
+  REQUIRE(aligned(x, 128) && aligned(packed_lo, 128) && aligned(packed_hi, 128),
+          "x and the packed weights must be 128-byte aligned");
+  REQUIRE(aligned(workspace, 1024), "workspace must be 1024-byte aligned");
+  REQUIRE(aligned(logits, 16) && (!bias || aligned(bias, 16)) && aligned(out, 16) &&
+              (!residual || aligned(residual, 16)) && (!topk_idx_out || aligned(topk_idx_out, 16)) &&
+              (!topk_w_out || aligned(topk_w_out, 16)),
+          "pointers must be 16-byte aligned");
+  const E256Ws L = e256_ws(T, n_shared);
+  if (workspace_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE, "moe_layer_e256 workspace needs %zu bytes, got %zu", L.total,
+                workspace_bytes);
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* off_lo = reinterpret_cast<int32_t*>(ws + L.off_lo);
+  int32_t* off_hi = reinterpret_cast<int32_t*>(ws + L.off_hi);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
+  int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  moe_bf16* h = reinterpret_cast<moe_bf16*>(ws + L.h);
+  moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
+  const int nb = static_cast<int>((T + e256::kBlockTokens - 1) / e256::kBlockTokens);
+
+  rc = do_route_e256(logits, bias, T, idx, w, s);
+  if (!rc)
+    rc = launch_pdl("count_e256_kernel launch", e256::count_e256_kernel, dim3(nb), dim3(256), 0,
+                    s, static_cast<const int32_t*>(idx), T, hist);
+  if (!rc)
+    rc = launch_pdl("scan_e256_kernel launch", e256::scan_e256_kernel, dim3(1), dim3(256), 0, s,
+                    hist, nb, reinterpret_cast<int32_t*>(ws + L.counts),
+                    reinterpret_cast<int32_t*>(ws + L.offsets), off_lo, off_hi);
+  if (!rc)
+    rc = launch_pdl("scatter_e256_kernel launch", e256::scatter_e256_kernel, dim3(nb), dim3(256),
+                    0, s, static_cast<const int32_t*>(idx), T, static_cast<const int32_t*>(hist),
+                    perm_src, inv_perm);
+  // experts 0..127 and 128..255: the 128-expert kernels on each half's pack
+  if (!rc) rc = do_expert_ffn(x, packed_lo, off_lo, perm_src, T, h, y, sms, s);
+  if (!rc) rc = do_expert_ffn(x, packed_hi, off_hi, perm_src, T, h, y, sms, s);
+  moe_bf16* y_sh = reinterpret_cast<moe_bf16*>(ws + L.sh_y);
+  if (!rc && n_shared > 0)
+    rc = do_shared_ffn(x, packed_shared, n_shared, T, reinterpret_cast<int32_t*>(ws + L.sh_offsets),
+                       reinterpret_cast<int32_t*>(ws + L.sh_perm),
+                       reinterpret_cast<moe_bf16*>(ws + L.sh_h), y_sh, sms, s);
+  if (!rc)
+    rc = launch_pdl("combine_kernel launch", combine_kernel<e256::kTopK2>,
+                    dim3(static_cast<unsigned>(T)), dim3(kCombineThreads), 0, s,
+                    reinterpret_cast<const uint16_t*>(y), static_cast<const float*>(w),
+                    static_cast<const int32_t*>(inv_perm), T,
+                    reinterpret_cast<const __nv_bfloat16*>(residual),
+                    reinterpret_cast<__nv_bfloat16*>(out), reinterpret_cast<const uint16_t*>(y_sh),
+                    n_shared);
+  return rc;
 }
 
 }  // extern "C"

@@ -75,6 +75,9 @@ _SIGS = {
     "moe_pack_shared": ([_p, _p, _p, _i32, _p, _p], _i32),
     "moe_layer_shared_workspace_bytes": ([_i64, _i32, _i32], _sz),
     "moe_layer_shared": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_route_e256": ([_p, _p, _i64, _p, _p, _p], _i32),
+    "moe_layer_e256_workspace_bytes": ([_i64, _i32], _sz),
+    "moe_layer_e256": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_layer_fp8": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -427,6 +430,49 @@ def moe_layer_shared(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor |
                                 _ptr(packed_fp8), _ptr(packed_shared), n_shared, T,
                                 _ptr(residual), _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out),
                                 _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------- second shape (256 experts)
+
+E256_EXPERTS, E256_TOPK = 256, 6
+
+
+def layer_e256_workspace_bytes(T: int, n_shared: int) -> int:
+    return int(lib.moe_layer_e256_workspace_bytes(T, n_shared))
+
+
+def moe_route_e256(logits: torch.Tensor, bias: torch.Tensor | None, topk_idx=None, topk_w=None,
+                   stream=None):
+    """Routing on the second shape: logits [T, 256] -> ([T, 6] int32, [T, 6] fp32)."""
+    T = logits.shape[0]
+    if topk_idx is None:
+        topk_idx = torch.empty((T, E256_TOPK), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, E256_TOPK), dtype=torch.float32, device=logits.device)
+    _check("moe_route_e256", lib.moe_route_e256(_ptr(logits), _ptr(bias), T, _ptr(topk_idx),
+                                                _ptr(topk_w), _stream(stream)))
+    return topk_idx, topk_w
+
+
+def moe_layer_e256(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
+                   packed_lo: torch.Tensor, packed_hi: torch.Tensor, packed_shared=None,
+                   n_shared: int = 0, residual=None, out=None, topk_idx_out=None,
+                   topk_w_out=None, workspace: torch.Tensor | None = None, stream=None):
+    """The layer on the second shape (256 experts top-6, see include/moe.h)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        n = layer_e256_workspace_bytes(T, n_shared)
+        raw = torch.empty(n + 1024, dtype=torch.uint8, device=x.device)
+        off = (-raw.data_ptr()) % 1024
+        workspace = raw[off:off + n]
+    _check("moe_layer_e256",
+           lib.moe_layer_e256(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_lo), _ptr(packed_hi),
+                              _ptr(packed_shared), n_shared, T, _ptr(residual), _ptr(out),
+                              _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+                              workspace.numel(), _stream(stream)))
     return out
 
 

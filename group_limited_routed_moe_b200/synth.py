@@ -278,6 +278,43 @@ def layer_logits(T: int, seed: int, layer: int):
 
 
 # ----------------------------------------------------------------------------
+# second MoE shape: 256 experts
+# ----------------------------------------------------------------------------
+
+E256_SEED_OFFSET = (2000, 3000)  # generator seeds of experts 0..127 and 128..255
+
+
+def e256_weight_bits_np(seed: int, layer: int, which: int, experts) -> np.ndarray:
+    """Expert matrix ``which`` of the 256-expert shape for the given expert ids
+    (0..255): experts 0..127 are the generator's under seed + 2000, experts
+    128..255 its experts 0..127 under seed + 3000.  [len(experts), rows, cols]."""
+    experts = np.asarray(experts)
+    rows, cols = _W_SHAPES[which]
+    out = np.zeros((len(experts), rows, cols), np.uint16)
+    for half in (0, 1):
+        sel = np.nonzero((experts >= 128 * half) & (experts < 128 * (half + 1)))[0]
+        if len(sel):
+            out[sel] = weight_bits_np(seed + E256_SEED_OFFSET[half], layer, which,
+                                      experts[sel] - 128 * half)
+    return out
+
+
+def e256_weight_bits_torch(seed: int, layer: int, which: int, half: int, device):
+    """The 128 experts of one half (0: experts 0..127, 1: 128..255) on ``device``."""
+    return weight_bits_torch(seed + E256_SEED_OFFSET[half], layer, which, device)
+
+
+def make_tokens_e256(T: int, seed: int) -> TokenInputs:
+    """x [T, 1536] bf16 bits, router logits [T, 256] ~ N(0, 1) and bias [256]
+    ~ N(0, 0.1), from PCG64(seed, 256)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 256])))
+    x = rng.standard_normal((T, HIDDEN), dtype=np.float32)
+    logits = rng.standard_normal((T, 256), dtype=np.float32)
+    bias = (rng.standard_normal(256, dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    return TokenInputs(f32_to_bf16_bits(x), logits, bias)
+
+
+# ----------------------------------------------------------------------------
 # named workloads
 # ----------------------------------------------------------------------------
 

@@ -356,6 +356,39 @@ int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
                      float* topk_w_out, void* workspace, size_t workspace_bytes,
                      moe_stream_t stream);
 
+/* ---- second MoE shape: 256 experts, top-6 ------------------------------------- */
+
+/* The Inkling model has "256 experts top-6 plus 2 shared" ("Add TML Inkling
+ * architecture", llama.cpp PR #25731, model description); its group structure,
+ * hidden and intermediate sizes are not given.  Read with tiny's rule scaled
+ * to 256 experts: 8 groups of 32, 4 kept, 6 chosen, the same score, tie and
+ * weight rules as moe_route; expert FFNs of tiny's shape (1536 -> 512 -> 1536). */
+enum { MOE_E256_EXPERTS = 256, MOE_E256_TOPK = 6 };
+
+/* Routing on the second shape: logits [T][256] fp32, bias [256] fp32 or NULL;
+ * topk_idx [T][6] int32 and topk_w [T][6] fp32 (out), slot order = descending
+ * score.  One warp per token. */
+int moe_route_e256(const float* logits, const float* bias, int64_t T, int32_t* topk_idx,
+                   float* topk_w, moe_stream_t stream);
+
+/* Workspace bytes moe_layer_e256 needs. */
+size_t moe_layer_e256_workspace_bytes(int64_t T, int n_shared);
+
+/* The whole layer on the second shape: routing, a stable counting sort over
+ * the 256 experts, the grouped expert FFN of experts 0..127 (packed_lo) and
+ * 128..255 (packed_hi) -- each packed by moe_pack_weights from that half's
+ * [128][...] weights -- in two launches of the 128-expert kernels, the
+ * n_shared (0..8) shared experts of packed_shared (moe_pack_shared), and the
+ * combine:
+ *   out[t] = bf16( residual[t] + sum_{slot < 6} w[t,slot] FFN_{e_slot}(x[t]) + sum_s FFN_s(x[t]) ).
+ * topk_idx_out / topk_w_out: optional [T][6]. */
+int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
+                   const moe_bf16* packed_lo, const moe_bf16* packed_hi,
+                   const moe_bf16* packed_shared, int n_shared, int64_t T,
+                   const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
+                   float* topk_w_out, void* workspace, size_t workspace_bytes,
+                   moe_stream_t stream);
+
 /* ---- permutation without a caller workspace ------------------------------ */
 
 /* The pages describe no such call: it is moe_permute for callers that cannot

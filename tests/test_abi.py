@@ -13,7 +13,7 @@ def test_exports_every_declared_symbol():
     assert len(names) >= 15
     missing = [n for n in names if not hasattr(moe.lib, n)]
     assert missing == []
-    assert moe.lib.moe_abi_version() == 4
+    assert moe.lib.moe_abi_version() == 5
 
 
 def test_sizes():
@@ -113,3 +113,18 @@ def test_shared_sizes_and_host_validation():
                               _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_layer_shared(_p(1024), _p(1024), None, _p(1024), None, _p(1024), 1, 16, None,
                               _p(1024), None, None, _p(1024), ws - 1, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_e256_sizes_and_host_validation():
+    L = moe.lib
+    assert moe.layer_e256_workspace_bytes(16, 2) > moe.layer_e256_workspace_bytes(16, 0) > 0
+    assert moe.layer_e256_workspace_bytes(16, 9) == 0
+    ws = moe.layer_e256_workspace_bytes(16, 2)
+    assert L.moe_route_e256(None, None, 0, None, None, None) == moe.MOE_OK
+    assert L.moe_route_e256(_p(260), None, 4, _p(256), _p(256), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_e256(_p(1024), _p(1024), None, _p(1024), None, _p(1024), 2, 16, None,
+                            _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_e256(_p(1024), _p(1024), None, _p(1024), _p(1024), None, 2, 16, None,
+                            _p(1024), None, None, _p(1024), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_e256(_p(1024), _p(1024), None, _p(1024), _p(1024), _p(1024), 2, 16, None,
+                            _p(1024), None, None, _p(1024), ws - 1, None) == moe.MOE_ERR_WORKSPACE
