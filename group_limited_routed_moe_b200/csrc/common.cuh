@@ -408,6 +408,23 @@ __device__ __forceinline__ int tileq_pop(TileQueue* q, int n, bool release,
   return tile;
 }
 
+// Non-blocking look at the n-th tile id: returns it if the producer has
+// published it already, else -3.  The slot is not released (tileq_pop does
+// that when its turn comes).
+__device__ __forceinline__ int tileq_peek(TileQueue* q, int n) {
+  const int slot = n % kTileQ;
+  const uint32_t ph = (n / kTileQ) & 1;
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(&q->full[slot])), "r"(ph)
+      : "memory");
+  return ok ? reinterpret_cast<volatile int*>(q->tile)[slot] : -3;
+}
+
 // End of a launch: the last CTA to finish zeroes the two counter words (and
 // the n_extra words at `extra`, if any).
 __device__ __forceinline__ void tileq_retire(int* sched, int* extra = nullptr, int n_extra = 0) {

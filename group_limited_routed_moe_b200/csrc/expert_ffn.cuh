@@ -363,6 +363,18 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
     const int chunk = t & 7, rsub = t >> 3;  // rsub < 32: rows rsub + 32 i, i < 4
     const uint32_t slot = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
     uint32_t dirty = 0u;  // bit 4*s + i: row rsub+32i of stage s may be non-zero (ring starts zeroed)
+    // The row sources of the next gate/up tile, read a few stages before it
+    // starts (once the producer has published it), so that a new tile's first
+    // copies do not wait for perm_src to come from memory.
+    int pf_tile = -1;
+    int pf_p[4];
+    auto load_rows = [&](const TileInfo& tj, int (&pv)[4]) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row_in_e = tj.m * BM + rsub + 32 * i;
+        pv[i] = row_in_e < S->cnt[tj.e] ? perm_src[S->off[tj.e] + row_in_e] : -1;
+      }
+    };
     int it = 0, n = 0;
     bool ok = true;
     while (ok) {
@@ -381,20 +393,34 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
         }
         continue;
       }
+      int pv[4];
+      if (pf_tile == tile) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pv[i] = pf_p[i];
+      } else {
+        load_rows(ti, pv);
+      }
+      pf_tile = -1;
       const char* src[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         src[i] = nullptr;
-        const int row_in_e = ti.m * BM + rsub + 32 * i;
-        if (row_in_e < S->cnt[ti.e]) {
-          const int p = perm_src[S->off[ti.e] + row_in_e];
-          if (p >= 0 && static_cast<int64_t>(p) < nrows)
-            src[i] = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH) + chunk * 16;
-        }
+        if (pv[i] >= 0 && static_cast<int64_t>(pv[i]) < nrows)
+          src[i] = reinterpret_cast<const char*>(x + static_cast<int64_t>(pv[i] >> 3) * kH) + chunk * 16;
       }
       for (int kb = 0; kb < kb_of(1); ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
+        if (kb >= kb_of(1) - STAGES && pf_tile < 0) {  // the next tile, once it is published
+          const int nx = tileq_peek(&S->tq, n);
+          if (nx >= 0) {
+            const TileInfo tn = tile_info<MODE>(S, nx, total1);
+            if (tn.phase == 1) {
+              load_rows(tn, pf_p);
+              pf_tile = nx;
+            }
+          }
+        }
         if (!mbar_wait(&S->empty[s], ph ^ 1, abort_flag, timeout_ns, kSiteFfnEmpty)) {
           ok = false;
           break;
