@@ -138,23 +138,28 @@ class ClockSampler:
         self.samples, self.reasons = [], 0
         self._stop = threading.Event()
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(0.002)
 
     def __enter__(self):
         if self.ok:
+            self._sample()  # the thread may get few turns while the host enqueues
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
 
     def __exit__(self, *a):
         if self.ok:
+            self._sample()
             self._stop.set()
             self.t.join()
 
