@@ -243,6 +243,86 @@ def fp8_scale_jitter(shape, seed: int) -> np.ndarray:
     return np.exp2(rng.integers(-2, 3, size=shape)).astype(np.float32)
 
 
+# NVFP4 form of the synthetic experts, as ModelOpt quantises a linear weight
+# [out, in]: tensor scale g from the matrix's max |w| (so that the largest
+# block scale is at most 448), block scale = E4M3(max |w| of 16 / 6 / g)
+# rounded to nearest even, code = E2M1(w / (block scale * g)) rounded to
+# nearest even and saturated at 6.  mode "pow2" rounds g up to a power of two
+# (the dequantised weights are then bf16 values), "amax" keeps it as is.
+FP4_BLOCK = 16
+E2M1_MAX = 6.0
+_E2M1_MIDS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)  # between the 8 magnitudes
+
+
+def _encode_e2m1(q):
+    """torch float32 (|q| <= 6) -> uint8 E2M1 codes, nearest, ties to even."""
+    import torch
+    mids = torch.tensor(_E2M1_MIDS, dtype=torch.float32, device=q.device)
+    a = q.abs()
+    idx = torch.bucketize(a, mids)  # mids[idx-1] < a <= mids[idx]: ties go down
+    tie = (idx < len(_E2M1_MIDS)) & (a == mids[idx.clamp(max=len(_E2M1_MIDS) - 1)])
+    idx = idx + (tie & (idx % 2 == 1)).to(idx.dtype)  # ...unless that magnitude is odd
+    sign = ((q < 0) & (idx > 0)).to(idx.dtype) << 3
+    return (idx | sign).to(torch.uint8)
+
+
+def _quantize_nvfp4(w, mode: str):
+    """torch float32 [n, out, in] -> (packed uint8 [n, out, in/2], block-scale
+    E4M3 codes uint8 [n, out, in/16], tensor scales float32 [n])."""
+    import torch
+    n, R, C = w.shape
+    amax = w.abs().amax(dim=(1, 2))
+    g = amax / torch.tensor(E2M1_MAX * FP8_MAX, dtype=torch.float32, device=w.device)
+    if mode == "pow2":
+        m, k = torch.frexp(g)  # g = m * 2**k, 0.5 <= m < 1: the next power of two is 2**k
+        g = torch.ldexp(torch.ones_like(g), k - (m == 0.5).to(k.dtype))
+    elif mode != "amax":
+        raise ValueError(f"unknown scale mode {mode!r}")
+    g = torch.where(amax > 0, g, torch.ones_like(g)).to(torch.float32)
+    blk = w.reshape(n, R, C // FP4_BLOCK, FP4_BLOCK)
+    bmax = blk.abs().amax(dim=-1)
+    sc = (bmax / E2M1_MAX / g[:, None, None]).to(torch.float8_e4m3fn)
+    sc = torch.where(sc.to(torch.float32) > 0, sc,
+                     torch.full_like(sc, 0x01, dtype=torch.uint8).view(torch.float8_e4m3fn))
+    den = sc.to(torch.float32) * g[:, None, None]
+    q = (blk / den[..., None]).clamp(-E2M1_MAX, E2M1_MAX)
+    codes = _encode_e2m1(q).reshape(n, R, C)
+    packed = codes[..., 0::2] | (codes[..., 1::2] << 4)
+    return packed, sc.view(torch.uint8), g
+
+
+def _linear_form(w):
+    """[n, K, N] (x W form) -> [n, N, K] (a linear layer's [out, in] form)."""
+    return w.transpose(1, 2).contiguous()
+
+
+def nvfp4_weights_np(seed: int, layer: int, which: int, experts=None, mode: str = "pow2"):
+    """NVFP4 form of expert matrix ``which`` of ``layer`` on the host, [out, in]:
+    (packed codes uint8 [n, out, in/2], block scales uint8 [n, out, in/16],
+    tensor scales float32 [n])."""
+    import torch
+    bits = weight_bits_np(seed, layer, which, experts)
+    w = (torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)).to(torch.float32)
+    q, s, g = _quantize_nvfp4(_linear_form(w), mode)
+    return q.numpy(), s.numpy(), g.numpy()
+
+
+def nvfp4_weights_torch(seed: int, layer: int, which: int, device, mode: str = "pow2"):
+    """Same bytes as ``nvfp4_weights_np`` for all 128 experts, made on ``device``."""
+    import torch
+    w = weight_bits_torch(seed, layer, which, device)
+    K, N = w.shape[1], w.shape[2]
+    packed = torch.empty((N_EXPERTS, N, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((N_EXPERTS, N, K // FP4_BLOCK), dtype=torch.uint8, device=device)
+    gs = torch.empty(N_EXPERTS, dtype=torch.float32, device=device)
+    for e0 in range(0, N_EXPERTS, 16):  # bounded float32 temporaries
+        q, s, g = _quantize_nvfp4(_linear_form(w[e0:e0 + 16].to(torch.float32)), mode)
+        packed[e0:e0 + 16].copy_(q)
+        scales[e0:e0 + 16].copy_(s)
+        gs[e0:e0 + 16].copy_(g)
+    return packed, scales, gs
+
+
 # ----------------------------------------------------------------------------
 # token-side inputs
 # ----------------------------------------------------------------------------

@@ -48,6 +48,9 @@ reordering beyond what the definition states:
   CUDA path reads bf16, block FP8 and NVFP4 experts): E4M3 codes with one fp32
   scale per 128 x 128 block, weight = value(code) * scale; the layer is the
   definition above with those weights (``moe_layer_fp8``).
+* NVFP4 experts (same bullet): E2M1 codes, one E4M3 scale per 16 weights
+  along the input dimension and one fp32 scale per matrix, weight =
+  value(code) * value(block scale) * tensor scale (``moe_layer_nvfp4``).
 
 Every function is pinned by tests in ``tests/test_oracle_*.py`` against
 brute force, closed forms and invariants (see each test's docstring).
@@ -387,6 +390,89 @@ def moe_layer_fp8(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | Non
     def weights(e):
         return (dequant_block_fp8(q_gate[e], s_gate[e]), dequant_block_fp8(q_up[e], s_up[e]),
                 dequant_block_fp8(q_down[e], s_down[e]))
+    return moe_layer_f64(x_bits, logits, bias, weights, route_result)
+
+
+# ----------------------------------------------------------------------------
+# NVFP4 expert weights
+# ----------------------------------------------------------------------------
+# The same bullet of issue #1247 names ModelOpt NVFP4 as the third expert
+# format the CUDA path reads.  The format, as ModelOpt writes it for a linear
+# layer's weight [out, in]: every weight is a 4-bit E2M1 code (OCP
+# microscaling FP4: sign, 2-bit exponent with bias 1, 1-bit mantissa; no
+# infinities or NaN), two codes per byte along the input dimension with the
+# even element in the low nibble; every 16 consecutive weights along the input
+# dimension share one FP8 E4M3 block scale; the whole matrix shares one fp32
+# tensor scale.  weight = value(code) * value(block scale) * tensor scale,
+# exactly.  The matrices are held here in that [out, in] orientation (W_gate
+# and W_up of an expert as [512, 1536], W_down as [1536, 512]); the layer uses
+# their transposes in the x W form above.
+
+NVFP4_BLOCK = 16
+
+
+def e2m1_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Exact value of FP4 E2M1 codes (uint8 holding 0..15) as float64.
+
+    Bit 3 is the sign, bits 2..1 the exponent field E (bias 1), bit 0 the
+    mantissa m.  E = 0 encodes the subnormals 0 and 0.5 (m/2); otherwise the
+    value is (1 + m/2) * 2**(E - 1).  Magnitudes: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    if np.any(c > 15):
+        raise ValueError("E2M1 codes are 4-bit values")
+    sign = np.where((c & 0x8) != 0, -1.0, 1.0)
+    E = (c >> 1) & 0x3
+    m = (c & 0x1).astype(np.float64)
+    mag = np.where(E == 0, m / 2.0, (1.0 + m / 2.0) * np.exp2(E - 1.0))
+    return sign * mag
+
+
+def unpack_fp4(packed: np.ndarray) -> np.ndarray:
+    """[..., C/2] bytes -> [..., C] codes: element 2i is the low nibble of byte i,
+    element 2i + 1 the high nibble."""
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def dequant_nvfp4(packed: np.ndarray, scales: np.ndarray, tensor_scale) -> np.ndarray:
+    """Weights of an NVFP4 matrix (or stack of matrices) in float64, [out, in] form.
+
+    packed [..., R, C/2] uint8 (two E2M1 codes per byte, see unpack_fp4);
+    scales [..., R, C/16] uint8 E4M3 codes, one per 16 consecutive weights of a
+    row; tensor_scale: fp32, one per matrix (shape [...]).
+    W[..., r, c] = value(code[..., r, c]) * value(scales[..., r, c // 16]) * tensor_scale[...],
+    exact in float64 (2 + 4 + 24 significant bits).
+    """
+    v = e2m1_to_f64(unpack_fp4(packed))
+    s = e4m3_to_f64(scales)
+    R, C = v.shape[-2:]
+    if s.shape[-2:] != (R, C // NVFP4_BLOCK) or C % NVFP4_BLOCK:
+        raise ValueError(f"scales {s.shape} do not tile codes {v.shape} in 1 x {NVFP4_BLOCK} blocks")
+    g = np.asarray(tensor_scale, dtype=np.float64)
+    if g.shape != v.shape[:-2]:
+        raise ValueError(f"tensor scales {g.shape} do not match the matrices {v.shape[:-2]}")
+    return v * np.repeat(s, NVFP4_BLOCK, axis=-1) * g[..., None, None]
+
+
+def moe_layer_nvfp4(x_bits: np.ndarray, logits: np.ndarray, bias: np.ndarray | None,
+                    q_gate: np.ndarray, s_gate: np.ndarray, g_gate: np.ndarray,
+                    q_up: np.ndarray, s_up: np.ndarray, g_up: np.ndarray,
+                    q_down: np.ndarray, s_down: np.ndarray, g_down: np.ndarray,
+                    route_result: RouteResult | None = None) -> np.ndarray:
+    """Routed layer with NVFP4 experts, float64, no intermediate rounding.
+
+    q_gate, q_up: [E, 512, 768] packed codes ([out, in] form), s_gate, s_up:
+    [E, 512, 96] E4M3 codes, g_gate, g_up: [E] fp32; q_down: [E, 1536, 256],
+    s_down: [E, 1536, 32], g_down: [E].  Only the experts some token uses are read.
+    """
+    def weights(e):
+        return (dequant_nvfp4(q_gate[e], s_gate[e], g_gate[e]).T,
+                dequant_nvfp4(q_up[e], s_up[e], g_up[e]).T,
+                dequant_nvfp4(q_down[e], s_down[e], g_down[e]).T)
     return moe_layer_f64(x_bits, logits, bias, weights, route_result)
 
 

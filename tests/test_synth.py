@@ -73,3 +73,34 @@ def test_fp8_weights_are_block_quantised_bf16_weights():
     assert np.all(blocks == 0x7E)
     j = S.fp8_scale_jitter((3, 12, 4), 1)
     assert set(np.log2(j).ravel().tolist()) <= {-2.0, -1.0, 0.0, 1.0, 2.0}
+
+
+def test_nvfp4_weights_are_block_quantised_bf16_weights():
+    """The synthetic NVFP4 checkpoint ([out, in] form): a power-of-two tensor
+    scale g with max|w| <= 6 * 448 * g < 2 * max|w|, E4M3 block scales (no NaN)
+    of 16 weights along the input dimension, every code the E2M1 value nearest
+    to w / (s g) (within half an E2M1 spacing, saturated at 6), codes packed low
+    nibble first; the encoder agrees with ml_dtypes' float4_e2m1fn rounding."""
+    import ml_dtypes
+    w = S.weight_bits_np(0, 1, S.W_UP, experts=[9])
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)[0].T  # [512, 1536]
+    q, s, g = S.nvfp4_weights_np(0, 1, S.W_UP, experts=[9])
+    assert q.shape == (1, 512, 768) and s.shape == (1, 512, 96) and g.shape == (1,)
+    assert np.all((s & 0x7F) != 0x7F)
+    m, _ = np.frexp(g)
+    assert np.all(m == 0.5)
+    amax = np.abs(wf).max()
+    assert amax <= 6 * 448 * float(g[0]) < 2 * amax
+    codes = np.empty((512, 1536), np.uint8)
+    codes[:, 0::2], codes[:, 1::2] = q[0] & 0xF, q[0] >> 4
+    v = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    sv = torch.from_numpy(s[0]).view(torch.float8_e4m3fn).double().numpy()
+    a = wf / (np.repeat(sv, 16, axis=1) * float(g[0]))
+    spacing = np.where(np.abs(a) < 2, 0.5, np.where(np.abs(a) < 4, 1.0, 2.0))
+    assert np.all(np.abs(v - np.clip(a, -6, 6)) <= spacing / 2 + 1e-12)
+    enc = S._encode_e2m1(torch.from_numpy(np.clip(a, -6, 6).astype(np.float32))).numpy()
+    lib = np.clip(a, -6, 6).astype(np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    same = (enc == lib) | ((enc & 7) == 0) & ((lib & 7) == 0)  # +-0 either way
+    assert np.all(same)
+    _, _, g2 = S.nvfp4_weights_np(0, 1, S.W_UP, experts=[9], mode="amax")
+    assert g2[0] == np.float32(np.float32(amax) / np.float32(6 * 448))
