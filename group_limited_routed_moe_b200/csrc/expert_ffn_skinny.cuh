@@ -47,9 +47,18 @@
 // converters and the tensor core, and the single issuing thread handles half
 // as many stages per weight byte as with 64-wide stages (its per-stage
 // barrier round trips, not the MMAs, bound a skinny GEMM).
+//
+// NVFP4 weights (WQ = 2, MODE 3 only): the same ring and operand slots with
+// 4-bit E2M1 codes.  A K = 128 stage holds 128 rows x 64 bytes of codes (two
+// 64-row TMA boxes, 64-byte swizzle: 16-byte chunk j of row r at chunk
+// j ^ ((r / 2) % 4)), the token rows, and the 2 KB of the stage's 16-bit block
+// multipliers (one per 16 codes of a row, see fp4.cuh), loaded by one bulk
+// copy; a converter thread turns 64 codes of its row into 32 columns of
+// bf16 (gate/up) or fp16 (down) pairs with the integer route of fp4.cuh.
 #pragma once
 #include "common.cuh"
 #include "expert_ffn.cuh"
+#include "fp4.cuh"
 #include "fp8.cuh"
 
 namespace moe {
@@ -71,18 +80,20 @@ constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;
 constexpr int CONV_WARP0 = 7;  // block-FP8: converter warps 7 .. 7 + NCONV - 1
 constexpr int kConvGroups = 2;  // block-FP8: converter warps per tensor-memory lane quarter
 
-// Ring geometry.  bf16 weights: STAGES x (16 KB weights + 4 KB tokens) of
-// K = 64, two 32-column accumulators in tensor memory.  Block-FP8 weights:
-// RSTAGES x (16 KB codes + 8 KB tokens + the tile's block scales, 1 KB
-// reserved) of K = 128 in the same 200 KB, and tensor memory also holds NA
-// dequantised 128 x 128 weight tiles (64 columns each) after the accumulators.
+// Ring geometry (WQ: 0 bf16, 1 block-FP8, 2 NVFP4 weights).  bf16 weights:
+// STAGES x (16 KB weights + 4 KB tokens) of K = 64, two 32-column
+// accumulators in tensor memory.  Quantised weights: RSTAGES x (codes, 16 KB
+// FP8 or 8 KB FP4, + 8 KB tokens + the block scales, 1 KB reserved for the
+// FP8 tile's, 2 KB for the FP4 stage's multipliers) of K = 128 in the same
+// 200 KB, and tensor memory also holds NA dequantised 128 x 128 weight tiles
+// (64 columns each) after the accumulators.
 constexpr int kMaxStages = 10;
-template <bool WQ>
+template <int WQ>
 struct Ring {
-  static constexpr int KS = WQ ? 128 : BK;                // K per stage
-  static constexpr int RA_BYTES = WQ ? BMW * KS : A_BYTES;  // codes or operands
+  static constexpr int KS = WQ ? 128 : BK;                  // K per stage
+  static constexpr int RA_BYTES = WQ == 2 ? BMW * KS / 2 : WQ ? BMW * KS : A_BYTES;  // codes or operands
   static constexpr int RB_BYTES = BNT * KS * 2;             // token rows
-  static constexpr int RSC_BYTES = WQ ? 1024 : 0;           // block scales of the tile
+  static constexpr int RSC_BYTES = WQ == 2 ? fp4::kStageMultBytes : WQ ? 1024 : 0;  // block scales
   static constexpr int RSTAGE_BYTES = RA_BYTES + RB_BYTES + RSC_BYTES;
   static constexpr int RSTAGES = WQ ? 8 : STAGES;
   static constexpr int BYTES = RSTAGES * RSTAGE_BYTES;
@@ -93,15 +104,20 @@ struct Ring {
   static constexpr int NCONV = WQ ? 4 * kConvGroups : 0;
   static constexpr int THREADS = skinny::THREADS + 32 * NCONV;
 };
-static_assert(Ring<true>::BYTES <= TILE_BYTES, "the FP8 ring must fit the bf16 ring's space");
-static_assert(Ring<true>::RSTAGES <= kMaxStages && Ring<false>::RSTAGES <= kMaxStages, "stages");
-static_assert(Ring<true>::RSTAGE_BYTES % 1024 == 0 && Ring<true>::RA_BYTES % 1024 == 0,
-              "SW128 tiles must stay 1024-byte aligned in the ring");
-static_assert(Ring<true>::A_COL0 + Ring<true>::A_COLS * Ring<true>::NA <= Ring<true>::TMEM_COLS,
+static_assert(Ring<1>::BYTES <= TILE_BYTES && Ring<2>::BYTES <= TILE_BYTES,
+              "the quantised rings must fit the bf16 ring's space");
+static_assert(Ring<0>::RSTAGES <= kMaxStages && Ring<1>::RSTAGES <= kMaxStages &&
+                  Ring<2>::RSTAGES <= kMaxStages, "stages");
+static_assert(Ring<1>::RSTAGE_BYTES % 1024 == 0 && Ring<1>::RA_BYTES % 1024 == 0 &&
+                  Ring<2>::RSTAGE_BYTES % 1024 == 0 && Ring<2>::RA_BYTES % 1024 == 0,
+              "swizzled tiles must stay 1024-byte aligned in the ring");
+static_assert(Ring<1>::A_COL0 + Ring<1>::A_COLS * Ring<1>::NA <= Ring<1>::TMEM_COLS,
               "operand slots must fit the tensor-memory allocation");
-static_assert(Ring<true>::RSTAGES % Ring<true>::NA == 0, "slot reuse follows the ring");
-static_assert(kConvGroups == 2 && kH / Ring<true>::KS % 2 == 0 && kI / Ring<true>::KS % 2 == 0,
-              "block-FP8 stages go in pairs, one per converter group, never across a tile");
+static_assert(Ring<1>::RSTAGES % Ring<1>::NA == 0 && Ring<2>::RSTAGES % Ring<2>::NA == 0,
+              "slot reuse follows the ring");
+static_assert(kConvGroups == 2 && kH / Ring<1>::KS % 2 == 0 && kI / Ring<1>::KS % 2 == 0,
+              "quantised stages go in pairs, one per converter group, never across a tile");
+static_assert(Ring<2>::KS == fp4::kStageK, "an NVFP4 stage is one run of multipliers");
 
 // Per-phase constants.  Phase 1: 8 weight blocks per 32-token chunk (4 pairs
 // x 2 halves of 64 gate + 64 up rows), K = 1536; phase 2: 12 blocks, K = 512.
@@ -164,7 +180,7 @@ __device__ __forceinline__ TileInfo tile_info(const Tail* S, int tile, int total
   return t;
 }
 
-template <int MODE, bool WQ = false>
+template <int MODE, int WQ = 0>
 __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w1,  // gate/up weights (phase 1)
                        const __grid_constant__ CUtensorMap tmap_w2,  // down weights (phase 2)
@@ -173,10 +189,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
                        const int32_t* __restrict__ perm_src, int64_t T,
                        uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
                        int* __restrict__ sched, int* __restrict__ done,
-                       const float* __restrict__ wscale,  // block-FP8 scales (SGU, then SD)
+                       const void* __restrict__ wscale,  // FP8 scales (SGU, SD) or FP4 MGU, MD
                        uint64_t timeout_ns) {
   constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
-  static_assert(!WQ || MODE == 3, "block-FP8 weights only in the single-launch form");
+  static_assert(!WQ || MODE == 3, "quantised weights only in the single-launch form");
   using R = Ring<WQ>;
   constexpr int RST = R::RSTAGES;
   constexpr int NA = R::NA > 0 ? R::NA : 1;
@@ -196,7 +212,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
   griddep_launch_dependents();
   auto sA = [&](int s) { return smem + s * R::RSTAGE_BYTES; };
   auto sB = [&](int s) { return smem + s * R::RSTAGE_BYTES + R::RA_BYTES; };
-  auto sC = [&](int s) { return sB(s) + R::RB_BYTES; };  // block-FP8: the tile's scales
+  auto sC = [&](int s) { return sB(s) + R::RB_BYTES; };  // quantised: block scales
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < RST; ++s) {
@@ -305,19 +321,28 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             ok = false;
             break;
           }
-          if (WQ) {  // codes: two 64-row boxes of 128 bytes; in phase 2 two 64-wide h tiles
+          if (WQ) {  // codes: two 64-row boxes (128 or 64 bytes); in phase 2 two 64-wide h tiles
             const int r1 = ti.phase == 1 ? wrow1 : wrow0 + 64;
             const CUtensorMap* tw = ti.phase == 1 ? &tmap_w1 : &tmap_w2;
-            // the tile's block scales: 12 gate + 12 up (phase 1) or 4 (phase 2), contiguous
-            const float* scl = ti.phase == 1
-                                   ? wscale + fp8::sgu_index(e, 256 * (f >> 1), 0)
-                                   : wscale + kE * fp8::kSguPerExpert + fp8::sd_index(e, f * BMW, 0);
-            const uint32_t scl_bytes = ti.phase == 1 ? 96 : 16;
+            const void* scl;
+            uint32_t scl_bytes;
+            int kx;  // x coordinate of the code boxes, in bytes
+            if constexpr (WQ == 2) {  // this stage's multipliers, one contiguous run
+              scl = static_cast<const uint8_t*>(wscale) + fp4::stage_mult_offset(ti.phase, e, f, kb);
+              scl_bytes = fp4::kStageMultBytes;
+              kx = kb * KS / 2;
+            } else {  // the tile's block scales: 12 gate + 12 up (phase 1) or 4 (phase 2)
+              const float* sf = static_cast<const float*>(wscale);
+              scl = ti.phase == 1 ? sf + fp8::sgu_index(e, 256 * (f >> 1), 0)
+                                  : sf + kE * fp8::kSguPerExpert + fp8::sd_index(e, f * BMW, 0);
+              scl_bytes = ti.phase == 1 ? 96 : 16;
+              kx = kb * KS;
+            }
             mbar_arrive_expect_tx(&fullb[s], R::RA_BYTES + (ti.phase == 2 ? R::RB_BYTES : 0) +
                                                  scl_bytes);
             bulk_load(smem_u32(sC(s)), scl, scl_bytes, &fullb[s]);
-            tma_load_2d(smem_u32(sA(s)), tw, kb * KS, wrow0, &fullb[s]);
-            tma_load_2d(smem_u32(sA(s)) + R::RA_BYTES / 2, tw, kb * KS, r1, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)), tw, kx, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)) + R::RA_BYTES / 2, tw, kx, r1, &fullb[s]);
             if (ti.phase == 2) {
               tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * KS, hrow, &fullb[s]);
               tma_load_2d(smem_u32(sB(s)) + B_BYTES, &tmap_h, kb * KS + BK, hrow, &fullb[s]);
@@ -462,7 +487,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     }
     cp_async_wait_all();
   } else if (WQ && warp >= CONV_WARP0) {
-    // ------------------------------------------------ block-FP8 converters
+    // ------------------------------------------------ converters (block-FP8, NVFP4)
     // One thread per weight row: warp w may only access tensor-memory lanes
     // 32 (w % 4) .. 32 (w % 4) + 31, so it takes those rows.  The converter
     // warps form kConvGroups groups of four (one per lane quarter); in every
@@ -500,37 +525,62 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
           ok = false;
           break;
         }
-        // this stage's block scale, from the tile's scales the TMA brought with
-        // the stage: 12 gate then 12 up (phase 1), or 4 (phase 2), one per k block
-        const float sc = reinterpret_cast<const float*>(
-            sC(s))[(ti.phase == 1 && up_rows ? 12 : 0) + kb];
-        const uint32_t src = smem_u32(sA(s)) + row * 128;
         const uint32_t dst = tmem_base + a_lane + R::A_COL0 + R::A_COLS * a;
-        uint32_t v[32];
-        {
-          const int h2 = cgroup;  // this group's 64 codes -> 32 columns
-          if (ti.phase == 1) {
-            const uint32_t mult = fp8::pow2_multiplier<false>(sc);
+        if constexpr (WQ == 2) {
+          // NVFP4: this group's 64 codes are chunks 2g, 2g + 1 of the row's
+          // four (64-byte swizzle), its 4 block multipliers bytes 8g.. of the
+          // row's 16 in the stage's multiplier run
+          const uint32_t src = smem_u32(sA(s)) + row * 64;
+          const uint32_t msw = static_cast<uint32_t>((row >> 1) & 3);
+          const uint2 mm = fp4::ld_shared_v2(smem_u32(sC(s)) + row * 16 + 8 * cgroup);
+          const uint32_t mv[4] = {__byte_perm(mm.x, 0, 0x1010), __byte_perm(mm.x, 0, 0x3232),
+                                  __byte_perm(mm.y, 0, 0x1010), __byte_perm(mm.y, 0, 0x3232)};
+          uint32_t v[32];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint32_t o[8];
-              const uint32_t jj = static_cast<uint32_t>(4 * h2 + j);
-              fp8::dequant16<false>(ld_shared_v4(src + ((jj ^ rsw) << 4)), sc, mult, o);
+          for (int q = 0; q < 2; ++q) {
+            const uint4 c4 = ld_shared_v4(src + (((2 * static_cast<uint32_t>(cgroup) + q) ^ msw) << 4));
+            const uint32_t w[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[8 * j + i] = o[i];
-            }
-          } else {
-            const uint32_t mult = fp8::pow2_multiplier<true>(sc);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint32_t o[8];
-              const uint32_t jj = static_cast<uint32_t>(4 * h2 + j);
-              fp8::dequant16<true>(ld_shared_v4(src + ((jj ^ rsw) << 4)), sc, mult, o);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) v[8 * j + i] = o[i];
+            for (int i = 0; i < 4; ++i) {
+              if (ti.phase == 1)
+                fp4::dequant8<false>(w[i], mv[2 * q + (i >> 1)], v + 16 * q + 4 * i);
+              else
+                fp4::dequant8<true>(w[i], mv[2 * q + (i >> 1)], v + 16 * q + 4 * i);
             }
           }
-          tmem_st_x32(dst + 32 * h2, v);
+          tmem_st_x32(dst + 32 * cgroup, v);
+        } else {
+          // this stage's block scale, from the tile's scales the TMA brought with
+          // the stage: 12 gate then 12 up (phase 1), or 4 (phase 2), one per k block
+          const float sc = reinterpret_cast<const float*>(
+              sC(s))[(ti.phase == 1 && up_rows ? 12 : 0) + kb];
+          const uint32_t src = smem_u32(sA(s)) + row * 128;
+          uint32_t v[32];
+          {
+            const int h2 = cgroup;  // this group's 64 codes -> 32 columns
+            if (ti.phase == 1) {
+              const uint32_t mult = fp8::pow2_multiplier<false>(sc);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint32_t o[8];
+                const uint32_t jj = static_cast<uint32_t>(4 * h2 + j);
+                fp8::dequant16<false>(ld_shared_v4(src + ((jj ^ rsw) << 4)), sc, mult, o);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[8 * j + i] = o[i];
+              }
+            } else {
+              const uint32_t mult = fp8::pow2_multiplier<true>(sc);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint32_t o[8];
+                const uint32_t jj = static_cast<uint32_t>(4 * h2 + j);
+                fp8::dequant16<true>(ld_shared_v4(src + ((jj ^ rsw) << 4)), sc, mult, o);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[8 * j + i] = o[i];
+              }
+            }
+            tmem_st_x32(dst + 32 * h2, v);
+          }
         }
         tmem_wait_st();
         tc_fence_before();  // operand stores -> the MMA thread's tcgen05.mma

@@ -18,6 +18,7 @@
 #include "expert_ffn.cuh"
 #include "expert_ffn_skinny.cuh"
 #include "e256.cuh"
+#include "fp4.cuh"
 #include "fp8.cuh"
 #include "pack.cuh"
 #include "permute.cuh"
@@ -29,7 +30,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kAbiVersion = 5;
+constexpr int kAbiVersion = 6;
 constexpr int64_t kMaxTokens = int64_t(1) << 22;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kZeroPadMaxT = 1024;  // gate/up keeps padding rows of A zeroed up to this T
@@ -110,7 +111,10 @@ int device_setup(int* dev_out, int* sms_out) {
         e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3, true>,
+        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3, 1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(skinny::skinny_gemm_kernel<3, 2>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, skinny::SMEM_BYTES);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(router::router_kernel,
@@ -152,14 +156,18 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
 // 2-D tensor map of 8-bit codes: `rows` rows of `cols` bytes, box of 128 x 64,
 // 128-byte swizzle (the converter warps read each row's eight 16-byte chunks;
 // the swizzle keeps a warp's reads free of bank conflicts).
-int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
+// Byte rows of codes in boxes of 64 rows x box_bytes (128: 128-byte swizzle,
+// 64: 64-byte swizzle).
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                 uint32_t box_bytes = 128) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols};
-  const cuuint32_t box[2] = {128, 64};
+  const cuuint32_t box[2] = {box_bytes, 64};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", int(r));
   return MOE_OK;
@@ -400,12 +408,44 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
   if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
-  return launch_pdl("skinny_gemm_kernel<3, fp8> launch", skinny::skinny_gemm_kernel<3, true>,
-                    dim3(sms), dim3(skinny::Ring<true>::THREADS), skinny::SMEM_BYTES, s, tw1, tw2,
+  return launch_pdl("skinny_gemm_kernel<3, fp8> launch", skinny::skinny_gemm_kernel<3, 1>,
+                    dim3(sms), dim3(skinny::Ring<1>::THREADS), skinny::SMEM_BYTES, s, tw1, tw2,
                     th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                     reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
                     sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                    reinterpret_cast<const float*>(p8 + fp8::kSguOff), g_timeout_ns.load());
+                    static_cast<const void*>(p8 + fp8::kSguOff), g_timeout_ns.load());
+}
+
+// Packed NVFP4 layer -> packed bf16/fp16 layer.
+int do_dequant_fp4(const void* packed4, moe_bf16* packed, int sms, cudaStream_t s) {
+  return launch_pdl("dequant_fp4_kernel launch", fp4::dequant_fp4_kernel, dim3(sms * 8),
+                    dim3(256), 0, s, static_cast<const uint8_t*>(packed4),
+                    reinterpret_cast<uint16_t*>(packed));
+}
+
+// Expert FFN with NVFP4 weights: as do_expert_ffn_fp8, with 4-bit codes and
+// per-16 block multipliers in the skinny kernel up to kSkinnyMaxT tokens.
+int do_expert_ffn_fp4(const moe_bf16* x, const void* packed4, const int32_t* offsets,
+                      const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, moe_bf16* dq,
+                      int sms, cudaStream_t s) {
+  if (T > kSkinnyMaxT) {
+    int rc = do_dequant_fp4(packed4, dq, sms, s);
+    if (rc) return rc;
+    return do_expert_ffn(x, dq, offsets, perm_src, T, h, y, sms, s);
+  }
+  const uint8_t* p4 = static_cast<const uint8_t*>(packed4);
+  CUtensorMap tw1, tw2, th;
+  int rc = make_tmap_u8(&tw1, p4, fp4::kGuRowBytes, uint64_t(kE) * 2 * kI, 64);
+  if (!rc) rc = make_tmap_u8(&tw2, p4 + fp4::kGuBytes, fp4::kDRowBytes, uint64_t(kE) * kH, 64);
+  if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (rc) return rc;
+  return launch_pdl("skinny_gemm_kernel<3, nvfp4> launch", skinny::skinny_gemm_kernel<3, 2>,
+                    dim3(sms), dim3(skinny::Ring<2>::THREADS), skinny::SMEM_BYTES, s, tw1, tw2,
+                    th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
+                    reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
+                    sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
+                    static_cast<const void*>(p4 + fp4::kMguOff), g_timeout_ns.load());
 }
 
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
@@ -438,8 +478,9 @@ struct LayerWs {
   size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, dq;
   size_t sh_offsets, sh_perm, sh_h, sh_y, total;
 };
-// fp8: the block-FP8 layer, which above kSkinnyMaxT tokens also needs room for
-// the expanded bf16/fp16 layer; n_shared: shared experts' rows and results.
+// fp8: a quantised (block-FP8 or NVFP4) layer, which above kSkinnyMaxT tokens
+// also needs room for the expanded bf16/fp16 layer; n_shared: shared experts'
+// rows and results.
 LayerWs layer_ws(int64_t T, bool fp8 = false, int n_shared = 0) {
   LayerWs L{};
   const size_t n = static_cast<size_t>(T) * kTopK;
@@ -495,6 +536,10 @@ int moe_get_device_status(int device) {
     return fail(MOE_ERR_RANGE, "a value of h, y_perm or W_down exceeded the fp16 range");
   if ((v & 0x7FFFFFFFu) == kSiteFp8Nan)
     return fail(MOE_ERR_RANGE, "a block-FP8 expert weight is a NaN code");
+  if ((v & 0x7FFFFFFFu) == fp4::kSiteFp4Scale)
+    return fail(MOE_ERR_RANGE,
+                "an NVFP4 block scale is a NaN code, a tensor scale is not finite, or a block "
+                "multiplier leaves the normal range of its operand type");
   return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out (status 0x%08x, site %u)", v,
               v & 0x7FFFFFFFu);
 }
@@ -636,19 +681,19 @@ size_t moe_layer_workspace_bytes(int64_t T) {
 namespace {
 // The layer from given router logits, or (packed_router != NULL) from the
 // router projection of x computed into the workspace first.
-// With packed_fp8 != NULL the experts are the block-FP8 layer it points to
-// (packed_w is then ignored).
+// With packed_q != NULL the experts are the quantised layer it points to,
+// block-FP8 (qfmt 1) or NVFP4 (qfmt 2); packed_w is then ignored.
 int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
                const moe_bf16* packed_router, const float* bias, const moe_bf16* packed_w,
                int64_t T, const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
                float* topk_w_out, void* workspace, size_t workspace_bytes, moe_stream_t stream,
-               const void* packed_fp8 = nullptr, const moe_bf16* packed_shared = nullptr,
-               int n_shared = 0) {
+               const void* packed_q = nullptr, const moe_bf16* packed_shared = nullptr,
+               int n_shared = 0, int qfmt = 1) {
   int rc = check_T(T);
   if (rc) return rc;
   if (T == 0) return MOE_OK;
-  const bool fp8 = packed_fp8 != nullptr;
-  if (fp8) packed_w = static_cast<const moe_bf16*>(packed_fp8);
+  const bool quant = packed_q != nullptr;
+  if (quant) packed_w = static_cast<const moe_bf16*>(packed_q);
   REQUIRE(x && (logits || packed_router) && packed_w && out && workspace, "null pointer");
   REQUIRE(aligned(x, 128) && aligned(packed_w, 128) && (!packed_router || aligned(packed_router, 128)),
           "x, the packed weights and packed_router must be 128-byte aligned");
@@ -661,7 +706,7 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
           kMaxShared);
   REQUIRE(n_shared == 0 || (packed_shared && aligned(packed_shared, 128)),
           "packed_shared must be a 128-byte aligned pointer when n_shared > 0");
-  const LayerWs L = layer_ws(T, fp8, n_shared);
+  const LayerWs L = layer_ws(T, quant, n_shared);
   if (workspace_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE, "%s workspace needs %zu bytes, got %zu", fn, L.total,
                 workspace_bytes);
@@ -688,8 +733,11 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
     rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
                           ws + L.perm_ws, s);
   if (!rc) {
-    if (fp8)
-      rc = do_expert_ffn_fp8(x, packed_fp8, offsets, perm_src, T, h, y,
+    if (quant && qfmt == 2)
+      rc = do_expert_ffn_fp4(x, packed_q, offsets, perm_src, T, h, y,
+                             reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
+    else if (quant)
+      rc = do_expert_ffn_fp8(x, packed_q, offsets, perm_src, T, h, y,
                              reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
     else
       rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
@@ -827,6 +875,85 @@ int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
     return fail(MOE_ERR_INVALID_ARG, "null pointer");
   return layer_impl("moe_layer_fp8", x, logits, nullptr, bias, nullptr, T, residual, out,
                     topk_idx_out, topk_w_out, workspace, workspace_bytes, stream, packed_fp8);
+}
+
+// ---- NVFP4 experts ---------------------------------------------------------------
+size_t moe_packed_nvfp4_bytes(void) { return static_cast<size_t>(fp4::kPackedBytes); }
+
+int moe_pack_weights_nvfp4(const uint8_t* q_gate, const uint8_t* s_gate, const float* g_gate,
+                           const uint8_t* q_up, const uint8_t* s_up, const float* g_up,
+                           const uint8_t* q_down, const uint8_t* s_down, const float* g_down,
+                           void* packed_nvfp4, moe_stream_t stream) {
+  REQUIRE(q_gate && s_gate && g_gate && q_up && s_up && g_up && q_down && s_down && g_down &&
+              packed_nvfp4,
+          "null pointer");
+  REQUIRE(aligned(packed_nvfp4, 128), "packed_nvfp4 must be 128-byte aligned");
+  REQUIRE(aligned(q_gate, 4) && aligned(q_up, 4) && aligned(q_down, 4) && aligned(g_gate, 4) &&
+              aligned(g_up, 4) && aligned(g_down, 4),
+          "codes and tensor scales must be 4-byte aligned");
+  int sms = 0;
+  int rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* p4 = static_cast<uint8_t*>(packed_nvfp4);
+  const dim3 grid(sms * 8), block(256);
+  fp4::pack_fp4_codes_kernel<<<grid, block, 0, s>>>(reinterpret_cast<const uint32_t*>(q_gate), p4, 0);
+  fp4::pack_fp4_codes_kernel<<<grid, block, 0, s>>>(reinterpret_cast<const uint32_t*>(q_up), p4, 1);
+  fp4::pack_fp4_codes_kernel<<<grid, block, 0, s>>>(reinterpret_cast<const uint32_t*>(q_down), p4, 2);
+  fp4::pack_fp4_mult_kernel<<<grid, block, 0, s>>>(s_gate, s_up, s_down, g_gate, g_up, g_down,
+                                                   reinterpret_cast<uint16_t*>(p4 + fp4::kMguOff));
+  return launch_check("pack_fp4 kernels launch");
+}
+
+int moe_dequant_nvfp4(const void* packed_nvfp4, moe_bf16* packed, moe_stream_t stream) {
+  REQUIRE(packed_nvfp4 && packed, "null pointer");
+  REQUIRE(aligned(packed_nvfp4, 128) && aligned(packed, 128),
+          "packed_nvfp4 and packed must be 128-byte aligned");
+  int sms = 0;
+  int rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_dequant_fp4(packed_nvfp4, packed, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_expert_ffn_nvfp4_workspace_bytes(int64_t T) {
+  return moe_expert_ffn_fp8_workspace_bytes(T);
+}
+
+int moe_expert_ffn_nvfp4(const moe_bf16* x, const void* packed_nvfp4, const int32_t* offsets,
+                         const int32_t* perm_src, int64_t T, moe_f16* h, moe_f16* y_perm,
+                         void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && packed_nvfp4 && offsets && perm_src && h && y_perm, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_nvfp4, 128) && aligned(h, 128),
+          "x, packed_nvfp4 and h must be 128-byte aligned");
+  REQUIRE(aligned(y_perm, 16) && aligned(offsets, 16) && aligned(perm_src, 16),
+          "pointers must be 16-byte aligned");
+  const size_t need = moe_expert_ffn_nvfp4_workspace_bytes(T);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(MOE_ERR_WORKSPACE, "moe_expert_ffn_nvfp4 workspace needs %zu bytes, got %zu",
+                need, workspace ? workspace_bytes : size_t(0));
+  if (need > 0) REQUIRE(aligned(workspace, 128), "workspace must be 128-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_expert_ffn_fp4(x, packed_nvfp4, offsets, perm_src, T, h, y_perm,
+                           static_cast<moe_bf16*>(workspace), sms,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_layer_nvfp4_workspace_bytes(int64_t T) { return moe_layer_fp8_workspace_bytes(T); }
+
+int moe_layer_nvfp4(const moe_bf16* x, const float* logits, const float* bias,
+                    const void* packed_nvfp4, int64_t T, const moe_bf16* residual, moe_bf16* out,
+                    int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                    size_t workspace_bytes, moe_stream_t stream) {
+  if (T > 0 && (logits == nullptr || packed_nvfp4 == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "null pointer");
+  return layer_impl("moe_layer_nvfp4", x, logits, nullptr, bias, nullptr, T, residual, out,
+                    topk_idx_out, topk_w_out, workspace, workspace_bytes, stream, packed_nvfp4,
+                    nullptr, 0, 2);
 }
 
 // ---- shared experts --------------------------------------------------------------

@@ -79,6 +79,13 @@ _SIGS = {
     "moe_layer_e256_workspace_bytes": ([_i64, _i32], _sz),
     "moe_layer_e256": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_layer_fp8": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_packed_nvfp4_bytes": ([], _sz),
+    "moe_pack_weights_nvfp4": ([_p] * 10 + [_p], _i32),
+    "moe_dequant_nvfp4": ([_p, _p, _p], _i32),
+    "moe_layer_nvfp4_workspace_bytes": ([_i64], _sz),
+    "moe_expert_ffn_nvfp4_workspace_bytes": ([_i64], _sz),
+    "moe_expert_ffn_nvfp4": ([_p, _p, _p, _p, _i64, _p, _p, _p, _sz, _p], _i32),
+    "moe_layer_nvfp4": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -384,6 +391,88 @@ def moe_layer_fp8(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | No
     return out
 
 
+# ----------------------------------------------------------------- NVFP4 experts
+
+def packed_nvfp4_bytes() -> int:
+    return int(lib.moe_packed_nvfp4_bytes())
+
+
+def layer_nvfp4_workspace_bytes(T: int) -> int:
+    return int(lib.moe_layer_nvfp4_workspace_bytes(T))
+
+
+def moe_pack_weights_nvfp4(q_gate, s_gate, g_gate, q_up, s_up, g_up, q_down, s_down, g_down,
+                           packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Re-layout one layer's NVFP4 experts ([out, in] form: uint8 codes two per
+    byte, uint8 E4M3 block scales per 16 inputs, fp32 tensor scales; see
+    include/moe.h)."""
+    for t, shp, dt in ((q_gate, (N_EXPERTS, INTER, HIDDEN // 2), torch.uint8),
+                       (q_up, (N_EXPERTS, INTER, HIDDEN // 2), torch.uint8),
+                       (q_down, (N_EXPERTS, HIDDEN, INTER // 2), torch.uint8),
+                       (s_gate, (N_EXPERTS, INTER, HIDDEN // 16), torch.uint8),
+                       (s_up, (N_EXPERTS, INTER, HIDDEN // 16), torch.uint8),
+                       (s_down, (N_EXPERTS, HIDDEN, INTER // 16), torch.uint8),
+                       (g_gate, (N_EXPERTS,), torch.float32), (g_up, (N_EXPERTS,), torch.float32),
+                       (g_down, (N_EXPERTS,), torch.float32)):
+        if t.dtype != dt or tuple(t.shape) != shp or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"expected contiguous CUDA {dt} {shp}, got {t.dtype} {tuple(t.shape)}")
+    if packed is None:
+        packed = torch.empty(packed_nvfp4_bytes(), dtype=torch.uint8, device=q_gate.device)
+    _check("moe_pack_weights_nvfp4",
+           lib.moe_pack_weights_nvfp4(_ptr(q_gate), _ptr(s_gate), _ptr(g_gate), _ptr(q_up),
+                                      _ptr(s_up), _ptr(g_up), _ptr(q_down), _ptr(s_down),
+                                      _ptr(g_down), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_dequant_nvfp4(packed_nvfp4: torch.Tensor, packed: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """The packed bf16/fp16 layer (moe_pack_weights layout) of a packed NVFP4 layer."""
+    if packed is None:
+        packed = torch.empty(packed_weight_bytes() // 2, dtype=torch.bfloat16,
+                             device=packed_nvfp4.device)
+    _check("moe_dequant_nvfp4",
+           lib.moe_dequant_nvfp4(_ptr(packed_nvfp4), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_expert_ffn_nvfp4(x: torch.Tensor, packed_nvfp4: torch.Tensor, offsets: torch.Tensor,
+                         perm_src: torch.Tensor, h=None, y_perm=None, workspace=None,
+                         stream=None):
+    """Step 3 with NVFP4 experts (see include/moe.h); returns (h, y_perm)."""
+    T = x.shape[0]
+    n = T * TOPK
+    if h is None:
+        h = torch.empty((n, INTER), dtype=torch.float16, device=x.device)
+    if y_perm is None:
+        y_perm = torch.empty((n, HIDDEN), dtype=torch.float16, device=x.device)
+    need = int(lib.moe_expert_ffn_nvfp4_workspace_bytes(T))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check("moe_expert_ffn_nvfp4",
+           lib.moe_expert_ffn_nvfp4(_ptr(x), _ptr(packed_nvfp4), _ptr(offsets), _ptr(perm_src),
+                                    T, _ptr(h), _ptr(y_perm), _ptr(workspace),
+                                    workspace.numel() if workspace is not None else 0,
+                                    _stream(stream)))
+    return h, y_perm
+
+
+def moe_layer_nvfp4(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
+                    packed_nvfp4: torch.Tensor, residual=None, out=None, topk_idx_out=None,
+                    topk_w_out=None, workspace: torch.Tensor | None = None, stream=None):
+    """moe_layer with NVFP4 experts (see include/moe.h)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = alloc_layer_workspace(T, x.device, fp8=True)
+    _check("moe_layer_nvfp4",
+           lib.moe_layer_nvfp4(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_nvfp4), T,
+                               _ptr(residual), _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out),
+                               _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 # ----------------------------------------------------------------- shared experts
 
 def packed_shared_bytes(n_shared: int) -> int:
@@ -503,12 +592,16 @@ class HostPipeline:
     previous call has finished.  The output of call k lands in the `out_host`
     passed to submit(); it is complete once `drain()` returns.  With fp8=True
     the weights passed to submit() are a packed block-FP8 layer and every call
-    runs moe_layer_fp8.  With shared = (packed_shared, n_shared) every call
+    runs moe_layer_fp8; with nvfp4=True a packed NVFP4 layer (moe_layer_nvfp4).  With shared = (packed_shared, n_shared) every call
     also runs the shared experts (moe_layer_shared).
     """
 
-    def __init__(self, T: int, device, depth: int = 2, fp8: bool = False, shared=None):
-        self.T, self.depth, self.k, self.fp8, self.shared = T, depth, 0, fp8, shared
+    def __init__(self, T: int, device, depth: int = 2, fp8: bool = False, shared=None,
+                 nvfp4: bool = False):
+        if nvfp4 and (fp8 or shared is not None):
+            raise ValueError("nvfp4 runs alone: no fp8, no shared experts")
+        self.T, self.depth, self.k, self.shared = T, depth, 0, shared
+        self.fp8, self.nvfp4 = fp8 or nvfp4, nvfp4
         self.last_layer = None
         self.slots = []
         for _ in range(depth):
@@ -542,7 +635,7 @@ class HostPipeline:
                 moe_layer_shared(slot["x"], slot["logits"], bias, self.shared[0], self.shared[1],
                                  out=slot["out"], workspace=slot["ws"], stream=st, **kw)
             else:
-                (moe_layer_fp8 if self.fp8 else moe_layer)(
+                (moe_layer_nvfp4 if self.nvfp4 else moe_layer_fp8 if self.fp8 else moe_layer)(
                     slot["x"], slot["logits"], bias, packed_w, out=slot["out"],
                     workspace=slot["ws"], stream=st)
             self.last_layer = torch.cuda.Event()

@@ -67,8 +67,9 @@ typedef enum moe_status {
   MOE_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out */
   MOE_ERR_UNSUPPORTED = 5, /* device is not sm_100 */
   MOE_ERR_RANGE = 6        /* an fp16 intermediate (h, y_perm, packed W_down)
-                              left the fp16 range, or a block-FP8 weight is
-                              a NaN code; reported by moe_get_device_status() */
+                              left the fp16 range, a block-FP8 weight is a
+                              NaN code, or an NVFP4 block multiplier is out
+                              of range; reported by moe_get_device_status() */
 } moe_status;
 
 /* ---- library information ------------------------------------------------ */
@@ -314,6 +315,79 @@ int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
                   const void* packed_fp8, int64_t T, const moe_bf16* residual,
                   moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
                   void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---- NVFP4 experts ---------------------------------------------------------- */
+
+/* The third expert format of the same bullet: ModelOpt NVFP4.  For a weight
+ * matrix in a linear layer's [out, in] orientation:
+ *   - every weight a 4-bit E2M1 code (sign, 2-bit exponent with bias 1, 1-bit
+ *     mantissa; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), two codes per byte
+ *     along the input dimension, the even element in the low nibble;
+ *   - every 16 consecutive weights along the input dimension one FP8 E4M3
+ *     block scale (0x7F/0xFF are NaN);
+ *   - the matrix one fp32 tensor scale;
+ *   weight = value(code) * value(block scale) * tensor scale.
+ * The kernels dequantise each weight as value * M rounded once to bf16
+ * (gate/up) or fp16 (down), where M, block scale * tensor scale, is rounded to
+ * that type at pack time.  With a power-of-two tensor scale M is exact, and
+ * moe_layer_nvfp4 returns bit for bit what moe_layer returns on the
+ * dequantised weights; other tensor scales add one rounding of M (relative
+ * 2^-9 for bf16, 2^-11 for fp16). */
+
+/* Bytes of one layer's packed NVFP4 experts (189 MB: codes, then the block
+ * multipliers). */
+size_t moe_packed_nvfp4_bytes(void);
+
+/* One-time re-layout of one layer's NVFP4 experts ([out, in] orientation, the
+ * transposes of moe_pack_weights' matrices).
+ *   q_gate, q_up : [128][512][768] uint8, two codes per byte (4-byte aligned)
+ *   s_gate, s_up : [128][512][96] uint8 E4M3 block scales: [e][n][b] scales
+ *                  inputs 16b .. 16b+15 of output n
+ *   g_gate, g_up : [128] fp32 tensor scales
+ *   q_down       : [128][1536][256];  s_down : [128][1536][32];  g_down : [128]
+ *   packed_nvfp4 : moe_packed_nvfp4_bytes() bytes, 128-byte aligned, output:
+ *                  codes in the row order of moe_pack_weights (gate/up
+ *                  interleaved in 128-column blocks), then every block's
+ *                  16-bit multiplier in the order the kernels read them.
+ * A NaN block scale, a non-finite tensor scale, or a multiplier of a non-zero
+ * scale that is not a normal bf16 (gate/up: block scale * tensor scale must
+ * lie in [2^-252, 4)) or fp16 (down: [2^-28, 4)) number sets the device
+ * error word (moe_get_device_status(): MOE_ERR_RANGE); the packed bytes are
+ * written regardless, and the layer's results on such weights are
+ * unspecified. */
+int moe_pack_weights_nvfp4(const uint8_t* q_gate, const uint8_t* s_gate, const float* g_gate,
+                           const uint8_t* q_up, const uint8_t* s_up, const float* g_up,
+                           const uint8_t* q_down, const uint8_t* s_down, const float* g_down,
+                           void* packed_nvfp4, moe_stream_t stream);
+
+/* Expands a packed NVFP4 layer into the packed bf16/fp16 layer that
+ * moe_pack_weights writes (packed: moe_packed_weight_bytes() bytes, 128-byte
+ * aligned, output).  With power-of-two tensor scales it equals
+ * moe_pack_weights of the dequantised weights, byte for byte. */
+int moe_dequant_nvfp4(const void* packed_nvfp4, moe_bf16* packed, moe_stream_t stream);
+
+/* Scratch bytes moe_expert_ffn_nvfp4 needs: 0 for T <= 256, else
+ * moe_packed_weight_bytes() (the expanded layer). */
+size_t moe_expert_ffn_nvfp4_workspace_bytes(int64_t T);
+
+/* Step 3 with NVFP4 experts: moe_expert_ffn_fp8's arguments with packed_nvfp4
+ * (from moe_pack_weights_nvfp4).  Up to 256 tokens one persistent launch
+ * streams the 4-bit codes and dequantises each weight tile into tensor memory
+ * on its way to the tensor cores; above, the layer is expanded into the
+ * workspace and the bf16 expert FFN runs on it. */
+int moe_expert_ffn_nvfp4(const moe_bf16* x, const void* packed_nvfp4, const int32_t* offsets,
+                         const int32_t* perm_src, int64_t T, moe_f16* h, moe_f16* y_perm,
+                         void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Workspace bytes moe_layer_nvfp4 needs for T tokens (as moe_layer_fp8). */
+size_t moe_layer_nvfp4_workspace_bytes(int64_t T);
+
+/* moe_layer with NVFP4 experts (packed_nvfp4 from moe_pack_weights_nvfp4),
+ * other arguments as in moe_layer; the expert FFN as moe_expert_ffn_nvfp4. */
+int moe_layer_nvfp4(const moe_bf16* x, const float* logits, const float* bias,
+                    const void* packed_nvfp4, int64_t T, const moe_bf16* residual,
+                    moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
+                    void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* ---- shared experts --------------------------------------------------------- */
 

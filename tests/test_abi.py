@@ -13,7 +13,7 @@ def test_exports_every_declared_symbol():
     assert len(names) >= 15
     missing = [n for n in names if not hasattr(moe.lib, n)]
     assert missing == []
-    assert moe.lib.moe_abi_version() == 5
+    assert moe.lib.moe_abi_version() == 6
 
 
 def test_sizes():
@@ -87,6 +87,32 @@ def test_fp8_sizes_and_host_validation():
     assert L.moe_pack_weights_fp8(_p(128), _p(128), None, _p(128), _p(128), _p(128), _p(128),
                                   None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_dequant_fp8(_p(136), _p(128), None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_nvfp4_sizes_and_host_validation():
+    L = moe.lib
+    codes = 128 * 1024 * 768 + 128 * 1536 * 256        # two codes per byte
+    mult = (128 * 1024 * 96 + 128 * 1536 * 32) * 2      # one 16-bit multiplier per 16 weights
+    assert moe.packed_nvfp4_bytes() == codes + mult
+    for T in (1, 256, 257, 2048):
+        assert moe.layer_nvfp4_workspace_bytes(T) == moe.layer_fp8_workspace_bytes(T)
+        assert L.moe_expert_ffn_nvfp4_workspace_bytes(T) == L.moe_expert_ffn_fp8_workspace_bytes(T)
+    assert L.moe_layer_nvfp4(None, None, None, None, 0, None, None, None, None, None, 0,
+                             None) == moe.MOE_OK
+    assert L.moe_layer_nvfp4(_p(1024), _p(1024), None, None, 16, None, _p(1024), None, None,
+                             _p(1024), 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    ws = moe.layer_nvfp4_workspace_bytes(300)
+    assert L.moe_layer_nvfp4(_p(1024), _p(1024), None, _p(1024), 300, None, _p(1024), None,
+                             None, _p(1024), ws - 1, None) == moe.MOE_ERR_WORKSPACE
+    args = [_p(128)] * 9
+    for i in range(9):  # every input pointer is required
+        a = list(args)
+        a[i] = None
+        assert L.moe_pack_weights_nvfp4(*a, _p(128), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_weights_nvfp4(*args, _p(136), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dequant_nvfp4(_p(136), _p(128), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn_nvfp4(_p(128), _p(128), _p(128), _p(128), 300, _p(128), _p(128),
+                                  None, 0, None) == moe.MOE_ERR_WORKSPACE
 
 
 def test_shared_sizes_and_host_validation():
