@@ -52,6 +52,11 @@ GATE_UP_BYTES_PER_EXPERT = 2 * 1536 * 512 * 2
 DOWN_BYTES_PER_EXPERT = 1536 * 512 * 2
 # block-FP8 expert: one byte per weight, one fp32 scale per 128 x 128 block
 FP8_BYTES_PER_EXPERT = 3 * 1536 * 512 + (2 * 12 * 4 + 4 * 12) * 4
+# NVFP4 expert in its checkpoint form: half a byte per weight, one E4M3 byte per
+# 16 weights (the three fp32 tensor scales are negligible)
+NVFP4_BYTES_PER_EXPERT = 3 * 1536 * 512 // 2 + 3 * 1536 * 512 // 16
+# what the NVFP4 kernel streams: codes, and a 16-bit multiplier per 16 weights
+NVFP4_PACKED_BYTES_PER_EXPERT = 3 * 1536 * 512 // 2 + 3 * 1536 * 512 // 16 * 2
 FLOPS_PER_ROW = 2 * (1536 * 1024 + 512 * 1536)          # one (token, expert) pair
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -63,15 +68,16 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_T8189", choices=["prefill_T8189", "decode_T16"])
-    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
-                    help="expert weights of the main line: bf16, or block FP8 (E4M3 codes, "
-                         "power-of-two 128x128 block scales)")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8", "nvfp4"],
+                    help="expert weights of the main line: bf16, block FP8 (E4M3 codes, "
+                         "power-of-two 128x128 block scales) or NVFP4 (E2M1 codes, E4M3 "
+                         "scales per 16, power-of-two tensor scales)")
     ap.add_argument("--e256-prefill", action="store_true",
                     help="also time the 256-expert shape at T=8189 (secondary line)")
     ap.add_argument("--shared", type=int, default=0,
                     help="shared experts (0-8) added to the main line's layer")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the decode_T16 (bf16, FP8, shared-expert) measurements")
+                    help="skip the decode_T16 (bf16, FP8, NVFP4, shared-expert) measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens in the oracle sample")
     return ap.parse_args()
@@ -85,22 +91,31 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-GEMM_SOURCES = ("common.cuh", "expert_ffn.cuh", "expert_ffn_skinny.cuh", "fp8.cuh")
+# The sources each profiled expert-FFN kernel is built from: the wide
+# (tokens-as-M) kernel of batches above 256 tokens, and the skinny
+# (weights-as-M) kernel of smaller ones with its bf16, FP8 and NVFP4 forms.
+WIDE_SOURCES = ("common.cuh", "expert_ffn.cuh")
+SKINNY_SOURCES = ("common.cuh", "expert_ffn.cuh", "expert_ffn_skinny.cuh", "fp8.cuh", "fp4.cuh",
+                  "pack.cuh")
 
 
-def kernel_source_sha():
-    """sha256 (first 16 hex digits) of the sources that define the grouped GEMM
-    kernels, the ones whose ncu traffic the bench line reports."""
+def kernel_sources(workload: str):
+    return WIDE_SOURCES if synth.WORKLOADS[workload].T > 256 else SKINNY_SOURCES
+
+
+def kernel_source_sha(files):
+    """sha256 (first 16 hex digits) of the given kernel sources, concatenated
+    in order: what a profile's counters are valid for."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "group_limited_routed_moe_b200", "csrc")
-    for f in GEMM_SOURCES:
+    for f in files:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str, workload: str):
     """dram read+write bytes per launch from the committed ncu summary, if it
-    was taken on the current kernel sources; else None."""
+    was taken on the current sources of that workload's kernel; else None."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
@@ -110,7 +125,7 @@ def profiled_traffic(kernel: str, workload: str):
             sha = line.split(":", 1)[1].strip()
         if line.startswith("traffic_bytes_per_launch:"):
             traffic = float(line.split(":", 1)[1].strip())
-    return traffic if sha == kernel_source_sha() else None
+    return traffic if sha == kernel_source_sha(kernel_sources(workload)) else None
 
 
 # --------------------------------------------------------------------- clocks
@@ -176,11 +191,14 @@ class ClockSampler:
 class LayerRun:
     """Device buffers and the five-call step of one workload."""
 
-    def __init__(self, wl: synth.Workload, dev, weights, fp8: bool = False, shared=None):
+    def __init__(self, wl: synth.Workload, dev, weights, fp8: bool = False, shared=None,
+                 nvfp4: bool = False):
         import torch
         from group_limited_routed_moe_b200 import moe
         self.moe, self.torch, self.wl, self.dev = moe, torch, wl, dev
         self.fp8 = fp8  # weights: a packed block-FP8 layer (moe_layer_fp8)
+        self.nvfp4 = nvfp4  # weights: a packed NVFP4 layer (moe_layer_nvfp4)
+        quant = fp8 or nvfp4
         self.shared = shared  # None, or (packed shared experts, n_shared): moe_layer_shared
         self.T = wl.T
         tok = synth.make_tokens(wl.T, wl.seed, hot=wl.hot)
@@ -213,13 +231,13 @@ class LayerRun:
         nb = (T + 127) // 128
         n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
         self.launches_per_step = n_rp + 2  # + the expert FFN (one launch) + combine
-        fws = moe.lib.moe_expert_ffn_fp8_workspace_bytes(T) if fp8 else 0
+        fws = moe.lib.moe_expert_ffn_fp8_workspace_bytes(T) if quant else 0
         self.ffn_ws = torch.empty(fws, dtype=torch.uint8, device=dev) if fws else None
         if fws:
-            self.launches_per_step += 1  # FP8 above 256 tokens: the expansion pass
+            self.launches_per_step += 1  # FP8 / NVFP4 above 256 tokens: the expansion pass
         # the breakdown pass times the same kernels the layer call runs
         self.part_names = ["route", "permute", "expert_ffn", "combine"]
-        self.lws = moe.alloc_layer_workspace(T, dev, fp8=fp8)
+        self.lws = moe.alloc_layer_workspace(T, dev, fp8=quant)
         if shared is not None:
             n = moe.layer_shared_workspace_bytes(T, shared[1], fp8)
             raw = torch.empty(n + 1024, dtype=torch.uint8, device=dev)
@@ -249,9 +267,13 @@ class LayerRun:
                                       self.shared[0], self.shared[1], out=self.out[:self.T],
                                       workspace=self.lws, stream=self.stream, **kw)
             return
-        layer = self.moe.moe_layer_fp8 if self.fp8 else self.moe.moe_layer
-        layer(self.x[:self.T], self.logits[:self.T], self.bias, self.packed,
-              out=self.out[:self.T], workspace=self.lws, stream=self.stream)
+        self.layer_fn(self.x[:self.T], self.logits[:self.T], self.bias, self.packed,
+                      out=self.out[:self.T], workspace=self.lws, stream=self.stream)
+
+    @property
+    def layer_fn(self):
+        m = self.moe
+        return m.moe_layer_nvfp4 if self.nvfp4 else m.moe_layer_fp8 if self.fp8 else m.moe_layer
 
     def step_parts(self, ev):
         """The same layer through the step calls, with an event between each."""
@@ -264,9 +286,10 @@ class LayerRun:
         m.moe_permute(self.idx, self.counts, self.offsets, self.perm_src, self.inv_perm,
                       self.pws, stream=s)
         rec()
-        if self.fp8:
-            m.moe_expert_ffn_fp8(self.x[:T], self.packed, self.offsets, self.perm_src, self.h,
-                                 self.y, workspace=self.ffn_ws, stream=s)
+        if self.fp8 or self.nvfp4:
+            (m.moe_expert_ffn_nvfp4 if self.nvfp4 else m.moe_expert_ffn_fp8)(
+                self.x[:T], self.packed, self.offsets, self.perm_src, self.h, self.y,
+                workspace=self.ffn_ws, stream=s)
         else:
             m.moe_expert_ffn(self.x[:T], self.packed, self.offsets, self.perm_src, self.h,
                              self.y, stream=s)
@@ -352,8 +375,8 @@ class LayerRun:
         """The fused moe_layer call captured once in a CUDA graph and replayed."""
         torch, moe = self.torch, self.moe
         T = self.T
-        ws = moe.alloc_layer_workspace(T, self.dev, fp8=self.fp8)
-        layer = moe.moe_layer_fp8 if self.fp8 else moe.moe_layer
+        ws = moe.alloc_layer_workspace(T, self.dev, fp8=self.fp8 or self.nvfp4)
+        layer = self.layer_fn
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
@@ -393,7 +416,8 @@ class LayerRun:
         x_h = torch.from_numpy(self.tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
         lg_h = torch.from_numpy(self.tok.logits).pin_memory()
         outs_h = [torch.empty((T, 1536), dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
-        pipe = moe.HostPipeline(T, self.dev, depth, fp8=self.fp8, shared=self.shared)
+        pipe = moe.HostPipeline(T, self.dev, depth, fp8=self.fp8, shared=self.shared,
+                                nvfp4=self.nvfp4)
 
         def run(n):
             for k in range(n):
@@ -445,6 +469,23 @@ def roofline_for(wl, run, per_ms, peaks, peak_kind):
     weights, x read, y_perm written)."""
     T = wl.T
     ffn_ms = float(per_ms[:, run.part_names.index("expert_ffn")].mean())
+    if run.nvfp4 and T <= 256:
+        # NVFP4 codes and block scales of the touched experts in the checkpoint's form
+        # (the kernel reads 16-bit multipliers in place of the 8-bit scales: see
+        # "streamed_per_launch"), x read, y_perm written
+        d = distinct_experts(run)
+        act = T * 1536 * 2 + 8 * T * 1536 * 2
+        nbytes = d * NVFP4_BYTES_PER_EXPERT + act
+        peak = float(peaks["hbm_gbs"])
+        achieved = nbytes / (ffn_ms * 1e-3) / 1e9
+        return {"kernel": "skinny_gemm_kernel<3, 2> (E2M1 codes dequantised into tensor memory; "
+                          "gate/up + SwiGLU + down in one launch)",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_per_launch": nbytes,
+                "streamed_per_launch": d * NVFP4_PACKED_BYTES_PER_EXPERT + act,
+                "distinct_experts": d,
+                "traffic": profiled_traffic("expert_ffn_nvfp4", wl.name)}
     if run.fp8 and T <= 256:
         # block-FP8 codes and scales of the touched experts, x read, y_perm written
         d = distinct_experts(run)
@@ -463,13 +504,14 @@ def roofline_for(wl, run, per_ms, peaks, peak_kind):
         peak = float(peaks[key])
         achieved = flops / (ffn_ms * 1e-3) / 1e12
         kernel = "ffn_gemm_kernel<3> (gate/up + SwiGLU + down in one launch)"
-        if run.fp8:
-            kernel = "dequant_fp8_kernel + " + kernel + ", timed together"
+        if run.fp8 or run.nvfp4:
+            kernel = ("dequant_fp4_kernel + " if run.nvfp4 else "dequant_fp8_kernel + ") + \
+                kernel + ", timed together"
         return {"kernel": kernel,
                 "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_kind} {key} (burst)", "algorithmic_per_launch": flops,
-                "traffic": None if run.fp8 else profiled_traffic("expert_ffn", wl.name)}
+                "traffic": None if run.fp8 or run.nvfp4 else profiled_traffic("expert_ffn", wl.name)}
     d = distinct_experts(run)
     nbytes = (d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * 1536 * 2
               + 8 * T * 1536 * 2)
@@ -488,7 +530,8 @@ def layer_fractions(wl, run, step_ms, per_ms, peaks):
     distinct experts' weights and against the tensor bound of the useful flops."""
     layer_s = float(step_ms.mean()) * 1e-3
     d = distinct_experts(run)
-    per_expert = FP8_BYTES_PER_EXPERT if run.fp8 else GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT
+    per_expert = (NVFP4_BYTES_PER_EXPERT if run.nvfp4 else FP8_BYTES_PER_EXPERT if run.fp8
+                  else GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT)
     nbytes = d * per_expert + wl.T * (1536 * 4 + 512)
     flops = FLOPS_PER_ROW * 8 * wl.T
     return {"layer_us": round(layer_s * 1e6, 2),
@@ -500,28 +543,30 @@ def layer_fractions(wl, run, step_ms, per_ms, peaks):
             "distinct_experts": d}
 
 
-def cpu_baseline(wl, tok, host_w, sample, fp8=False):
+def cpu_baseline(wl, tok, host_w, sample, fp8=False, nvfp4=False):
     """The float64 oracle on the first `sample` tokens.  host_w: bf16 bits
     (W_gate, W_up, W_down), or with fp8 the codes and scales (q_gate, s_gate,
-    q_up, s_up, q_down, s_down)."""
+    q_up, s_up, q_down, s_down), or with nvfp4 the codes, block and tensor
+    scales of each matrix."""
     import oracle as O
     from threadpoolctl import threadpool_info
     n = min(sample, wl.T)
     rows = np.arange(n)
     t0 = time.perf_counter()
-    (O.moe_layer_fp8 if fp8 else O.moe_layer)(tok.x_bits[rows], tok.logits[rows], tok.bias,
-                                              *host_w)
+    fn = O.moe_layer_nvfp4 if nvfp4 else O.moe_layer_fp8 if fp8 else O.moe_layer
+    fn(tok.x_bits[rows], tok.logits[rows], tok.bias, *host_w)
     dt = time.perf_counter() - t0
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": (f"first {n} of {wl.T} tokens of {wl.name}"
-                       f"{' (block-FP8 experts)' if fp8 else ''}, float64 NumPy oracle, {dt:.2f} s")}
+                       f"{' (NVFP4 experts)' if nvfp4 else ' (block-FP8 experts)' if fp8 else ''}"
+                       f", float64 NumPy oracle, {dt:.2f} s")}
 
 
-def decode_line(wl2, dev, packed, fp8, steps, warmup, peaks, peak_kind, barrier):
+def decode_line(wl2, dev, packed, fp8, steps, warmup, peaks, peak_kind, barrier, nvfp4=False):
     """The decode batch measured beside the main line: whole-layer steps,
     breakdown and roofline, router, CUDA-graph replay, end to end."""
-    run2 = LayerRun(wl2, dev, packed, fp8=fp8)
+    run2 = LayerRun(wl2, dev, packed, fp8=fp8, nvfp4=nvfp4)
     clk2 = ClockSampler(int(dev.index or 0))
     n = max(steps, 50)
     with clk2:
@@ -534,7 +579,7 @@ def decode_line(wl2, dev, packed, fp8, steps, warmup, peaks, peak_kind, barrier)
     out = {
         "value": round(wl2.T / (ms2 * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms2, 5),
         "roofline": roofline_for(wl2, run2, per2, peaks, peak_kind)}
-    if not fp8:
+    if not (fp8 or nvfp4):
         out["router"] = run2.router(20, peaks)
     out.update({
         "layer": dict(layer_fractions(wl2, run2, steps2, per2, peaks),
@@ -658,6 +703,17 @@ def fp8_layer(dev):
     return packed, qs
 
 
+def nvfp4_layer(dev):
+    """The synthetic NVFP4 checkpoint of layer 0 (power-of-two tensor scales),
+    packed, and its codes and scales on the device."""
+    from group_limited_routed_moe_b200 import moe
+    qs = []
+    for which in (synth.W_GATE, synth.W_UP, synth.W_DOWN):
+        qs += list(synth.nvfp4_weights_torch(0, 0, which, dev, "pow2"))
+    packed = moe.moe_pack_weights_nvfp4(*qs)
+    return packed, qs
+
+
 def run_ours(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -691,11 +747,17 @@ def run_ours(args):
 
     fp8_packed, fp8_dev = fp8_layer(dev) if (args.weights == "fp8" or not args.no_secondary) \
         else (None, None)
+    fp4_packed, fp4_dev = nvfp4_layer(dev) if (args.weights == "nvfp4" or not args.no_secondary) \
+        else (None, None)
     torch.cuda.synchronize()
     fp8 = args.weights == "fp8"
+    nvfp4 = args.weights == "nvfp4"
+    if nvfp4 and args.shared:
+        raise SystemExit("--shared runs with bf16 or fp8 routed experts")
     wl = synth.WORKLOADS[args.workload]
     shared = shared_layer(dev, args.shared) if args.shared > 0 else None
-    run = LayerRun(wl, dev, fp8_packed if fp8 else packed, fp8=fp8, shared=shared)
+    main_w = fp4_packed if nvfp4 else fp8_packed if fp8 else packed
+    run = LayerRun(wl, dev, main_w, fp8=fp8, shared=shared, nvfp4=nvfp4)
     clk = ClockSampler(local)
     with clk:
         steps_ms, wall = run.timed(args.steps, args.warmup, barrier)
@@ -715,7 +777,9 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "T_buf": wl.T_buf, "hidden": 1536,
                    "weights": ("block-FP8 experts (E4M3 codes, power-of-two 128x128 block scales)"
-                               if fp8 else "bf16 experts"),
+                               if fp8 else
+                               "NVFP4 experts (E2M1 codes, E4M3 scales per 16, power-of-two "
+                               "tensor scales)" if nvfp4 else "bf16 experts"),
                    "shared_experts": args.shared,
                    "experts": 128, "groups": 8, "keep_groups": 4, "topk": 8, "inter": 512,
                    "parallelism": f"dp{world} (independent batch per GPU)",
@@ -739,11 +803,12 @@ def run_ours(args):
     }
     if not args.no_secondary:
         wl2 = synth.WORKLOADS["decode_T16"]
-        for key, p2, f2 in (("decode_T16", packed, False), ("decode_T16_fp8", fp8_packed, True)):
-            if wl2.name == wl.name and f2 == fp8:
+        for key, p2, fmt in (("decode_T16", packed, "bf16"), ("decode_T16_fp8", fp8_packed, "fp8"),
+                             ("decode_T16_nvfp4", fp4_packed, "nvfp4")):
+            if wl2.name == wl.name and fmt == args.weights:
                 continue  # that is the main line
-            line[key] = decode_line(wl2, dev, p2, f2, args.steps, args.warmup, peaks, peak_kind,
-                                    barrier)
+            line[key] = decode_line(wl2, dev, p2, fmt == "fp8", args.steps, args.warmup, peaks,
+                                    peak_kind, barrier, nvfp4=fmt == "nvfp4")
             line["gpu_launches"] += line[key]["gpu_launches"]
         line["decode_T16_e256"] = e256_line(16, dev, max(args.steps, 50), args.warmup, peaks,
                                             barrier)
@@ -759,11 +824,12 @@ def run_ours(args):
                                                peaks, barrier)
         line["gpu_launches"] += line["prefill_T8189_e256"]["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if fp8:
-            hw = [t.cpu().numpy() for t in fp8_dev]
+        if fp8 or nvfp4:
+            hw = [t.cpu().numpy() for t in (fp4_dev if nvfp4 else fp8_dev)]
         else:
             hw = host_weights()
-        line["cpu_baseline"] = cpu_baseline(wl, run.tok, hw, args.cpu_sample, fp8=fp8)
+        line["cpu_baseline"] = cpu_baseline(wl, run.tok, hw, args.cpu_sample, fp8=fp8,
+                                            nvfp4=nvfp4)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
