@@ -998,6 +998,18 @@ int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
                     packed_shared, n_shared);
 }
 
+int moe_layer_shared_nvfp4(const moe_bf16* x, const float* logits, const float* bias,
+                           const void* packed_nvfp4, const moe_bf16* packed_shared, int n_shared,
+                           int64_t T, const moe_bf16* residual, moe_bf16* out,
+                           int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                           size_t workspace_bytes, moe_stream_t stream) {
+  if (T > 0 && (logits == nullptr || packed_nvfp4 == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "null pointer");
+  return layer_impl("moe_layer_shared_nvfp4", x, logits, nullptr, bias, nullptr, T, residual,
+                    out, topk_idx_out, topk_w_out, workspace, workspace_bytes, stream,
+                    packed_nvfp4, packed_shared, n_shared, 2);
+}
+
 }  // extern "C"
 
 // ---- second MoE shape: 256 experts top-6 ------------------------------------------

@@ -75,6 +75,7 @@ _SIGS = {
     "moe_pack_shared": ([_p, _p, _p, _i32, _p, _p], _i32),
     "moe_layer_shared_workspace_bytes": ([_i64, _i32, _i32], _sz),
     "moe_layer_shared": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_layer_shared_nvfp4": ([_p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_route_e256": ([_p, _p, _i64, _p, _p, _p], _i32),
     "moe_layer_e256_workspace_bytes": ([_i64, _i32], _sz),
     "moe_layer_e256": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
@@ -503,17 +504,27 @@ def moe_pack_shared(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tens
 def moe_layer_shared(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | None,
                      packed_shared: torch.Tensor, n_shared: int, packed_w=None, packed_fp8=None,
                      residual=None, out=None, topk_idx_out=None, topk_w_out=None,
-                     workspace: torch.Tensor | None = None, stream=None):
-    """moe_layer (packed_w) or moe_layer_fp8 (packed_fp8) plus n_shared shared
-    experts (see include/moe.h)."""
+                     workspace: torch.Tensor | None = None, stream=None, packed_nvfp4=None):
+    """moe_layer (packed_w), moe_layer_fp8 (packed_fp8) or moe_layer_nvfp4
+    (packed_nvfp4) plus n_shared shared experts (see include/moe.h)."""
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        n = layer_shared_workspace_bytes(T, n_shared, packed_fp8 is not None)
+        quant = packed_fp8 is not None or packed_nvfp4 is not None
+        n = layer_shared_workspace_bytes(T, n_shared, quant)
         raw = torch.empty(n + 1024, dtype=torch.uint8, device=x.device)
         off = (-raw.data_ptr()) % 1024
         workspace = raw[off:off + n]
+    if packed_nvfp4 is not None:
+        if packed_w is not None or packed_fp8 is not None:
+            raise ValueError("exactly one of packed_w, packed_fp8, packed_nvfp4")
+        _check("moe_layer_shared_nvfp4",
+               lib.moe_layer_shared_nvfp4(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_nvfp4),
+                                          _ptr(packed_shared), n_shared, T, _ptr(residual),
+                                          _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)))
+        return out
     _check("moe_layer_shared",
            lib.moe_layer_shared(_ptr(x), _ptr(logits), _ptr(bias), _ptr(packed_w),
                                 _ptr(packed_fp8), _ptr(packed_shared), n_shared, T,
@@ -598,8 +609,8 @@ class HostPipeline:
 
     def __init__(self, T: int, device, depth: int = 2, fp8: bool = False, shared=None,
                  nvfp4: bool = False):
-        if nvfp4 and (fp8 or shared is not None):
-            raise ValueError("nvfp4 runs alone: no fp8, no shared experts")
+        if nvfp4 and fp8:
+            raise ValueError("one routed-expert format: fp8 or nvfp4")
         self.T, self.depth, self.k, self.shared = T, depth, 0, shared
         self.fp8, self.nvfp4 = fp8 or nvfp4, nvfp4
         self.last_layer = None
@@ -631,7 +642,8 @@ class HostPipeline:
             if self.last_layer is not None:
                 st.wait_event(self.last_layer)
             if self.shared is not None:
-                kw = {"packed_fp8": packed_w} if self.fp8 else {"packed_w": packed_w}
+                kw = ({"packed_nvfp4": packed_w} if self.nvfp4 else
+                      {"packed_fp8": packed_w} if self.fp8 else {"packed_w": packed_w})
                 moe_layer_shared(slot["x"], slot["logits"], bias, self.shared[0], self.shared[1],
                                  out=slot["out"], workspace=slot["ws"], stream=st, **kw)
             else:

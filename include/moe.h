@@ -414,7 +414,7 @@ int moe_pack_shared(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16
                     int n_shared, moe_bf16* packed_shared, moe_stream_t stream);
 
 /* Workspace bytes moe_layer_shared needs (fp8_routed != 0: routed experts in
- * block FP8). */
+ * block FP8 or NVFP4, for moe_layer_shared_nvfp4 too). */
 size_t moe_layer_shared_workspace_bytes(int64_t T, int n_shared, int fp8_routed);
 
 /* moe_layer (packed_w, bf16 routed experts) or moe_layer_fp8 (packed_fp8):
@@ -429,6 +429,16 @@ int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
                      const moe_bf16* residual, moe_bf16* out, int32_t* topk_idx_out,
                      float* topk_w_out, void* workspace, size_t workspace_bytes,
                      moe_stream_t stream);
+
+/* moe_layer_shared with NVFP4 routed experts (packed_nvfp4 from
+ * moe_pack_weights_nvfp4) and n_shared (0..8) bf16 shared experts; workspace
+ * as moe_layer_shared_workspace_bytes(T, n_shared, 1).  With n_shared = 0 the
+ * result is bit for bit that of moe_layer_nvfp4. */
+int moe_layer_shared_nvfp4(const moe_bf16* x, const float* logits, const float* bias,
+                           const void* packed_nvfp4, const moe_bf16* packed_shared, int n_shared,
+                           int64_t T, const moe_bf16* residual, moe_bf16* out,
+                           int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                           size_t workspace_bytes, moe_stream_t stream);
 
 /* ---- second MoE shape: 256 experts, top-6 ------------------------------------- */
 

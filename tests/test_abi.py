@@ -113,6 +113,15 @@ def test_nvfp4_sizes_and_host_validation():
     assert L.moe_dequant_nvfp4(_p(136), _p(128), None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_expert_ffn_nvfp4(_p(128), _p(128), _p(128), _p(128), 300, _p(128), _p(128),
                                   None, 0, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_layer_shared_nvfp4(None, None, None, None, None, 0, 0, None, None, None, None,
+                                    None, 0, None) == moe.MOE_OK
+    assert L.moe_layer_shared_nvfp4(_p(1024), _p(1024), None, None, _p(1024), 1, 16, None,
+                                    _p(1024), None, None, _p(1024), 1 << 30,
+                                    None) == moe.MOE_ERR_INVALID_ARG
+    ws = moe.layer_shared_workspace_bytes(300, 2, True)
+    assert L.moe_layer_shared_nvfp4(_p(1024), _p(1024), None, _p(1024), _p(1024), 2, 300, None,
+                                    _p(1024), None, None, _p(1024), ws - 1,
+                                    None) == moe.MOE_ERR_WORKSPACE
 
 
 def test_shared_sizes_and_host_validation():

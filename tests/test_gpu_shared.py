@@ -125,3 +125,26 @@ def test_shared_with_fp8_routed_experts(T):
     torch.cuda.synchronize()
     _status_ok()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("T", [16, 300])
+def test_shared_with_nvfp4_routed_experts(T):
+    """NVFP4 routed experts (power-of-two tensor scales) with bf16 shared
+    experts: bit for bit the layer with the bf16 pack of the dequantised routed
+    weights; with no shared expert, bit for bit moe_layer_nvfp4."""
+    from test_gpu_nvfp4 import pow2_bf16_packed as nv_bf16_packed
+    from test_gpu_nvfp4 import pow2_layer as nv_layer
+    moe = _moe()
+    L4 = nv_layer()
+    ref_packed = nv_bf16_packed()
+    bits, packed = shared_pack(2)
+    tok = synth.make_tokens(T, 1150 + T)
+    x, lg, bias = tokens_dev(tok)
+    a = moe.moe_layer_shared(x, lg, bias, packed, 2, packed_nvfp4=L4.packed, residual=x)
+    b = moe.moe_layer_shared(x, lg, bias, packed, 2, packed_w=ref_packed, residual=x)
+    c = moe.moe_layer_shared(x, lg, bias, packed, 0, packed_nvfp4=L4.packed)
+    d = moe.moe_layer_nvfp4(x, lg, bias, L4.packed)
+    torch.cuda.synchronize()
+    _status_ok()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(c.view(torch.int16), d.view(torch.int16))
