@@ -244,3 +244,29 @@ def test_pack_nvfp4_flags_bad_scales():
         assert "NVFP4" in moe.last_error()
         _status_ok()
         del tmp
+
+
+def test_host_pipeline_nvfp4_outputs_equal_direct_calls():
+    """moe.HostPipeline(nvfp4=True): four different batches from pinned host
+    buffers, two in flight; each output equals moe_layer_nvfp4 on that batch."""
+    moe = _moe()
+    L = pow2_layer()
+    T = 16
+    pipe = moe.HostPipeline(T, DEV, 2, nvfp4=True)
+    toks = [synth.make_tokens(T, 1300 + k) for k in range(4)]
+    bias = torch.from_numpy(toks[0].bias).to(DEV)
+    hosts = []
+    for tok in toks:
+        x_h = torch.from_numpy(tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        lg_h = torch.from_numpy(tok.logits).pin_memory()
+        out_h = torch.full((T, 1536), float("nan"), dtype=torch.bfloat16).pin_memory()
+        hosts.append((x_h, lg_h, out_h))
+    for x_h, lg_h, out_h in hosts:
+        pipe.submit(x_h, lg_h, out_h, bias, L.packed)
+    pipe.drain()
+    _status_ok()
+    for tok, (x_h, lg_h, out_h) in zip(toks, hosts):
+        x, lg, _ = tokens_dev(tok)
+        ref = moe.moe_layer_nvfp4(x, lg, bias, L.packed)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h.view(torch.int16), ref.cpu().view(torch.int16))
