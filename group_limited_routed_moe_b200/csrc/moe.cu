@@ -478,10 +478,10 @@ struct LayerWs {
   size_t idx, w, counts, offsets, perm_src, inv_perm, perm_ws, h, y, logits, dq;
   size_t sh_offsets, sh_perm, sh_h, sh_y, total;
 };
-// fp8: a quantised (block-FP8 or NVFP4) layer, which above kSkinnyMaxT tokens
+// quant: a quantised (block-FP8 or NVFP4) layer, which above kSkinnyMaxT tokens
 // also needs room for the expanded bf16/fp16 layer; n_shared: shared experts'
 // rows and results.
-LayerWs layer_ws(int64_t T, bool fp8 = false, int n_shared = 0) {
+LayerWs layer_ws(int64_t T, bool quant = false, int n_shared = 0) {
   LayerWs L{};
   const size_t n = static_cast<size_t>(T) * kTopK;
   size_t o = 0;
@@ -500,7 +500,7 @@ LayerWs layer_ws(int64_t T, bool fp8 = false, int n_shared = 0) {
   L.h = take(n * kI * 2);
   L.y = take(n * kH * 2);
   L.logits = take(static_cast<size_t>(T) * kE * 4);  // used by moe_layer_routed
-  L.dq = take(fp8 && T > kSkinnyMaxT ? static_cast<size_t>(kPackElems) * 2 : 0);
+  L.dq = take(quant && T > kSkinnyMaxT ? static_cast<size_t>(kPackElems) * 2 : 0);
   const size_t ns = static_cast<size_t>(n_shared) * static_cast<size_t>(T);
   L.sh_offsets = take(n_shared ? kOffsetsLen * 4 : 0);
   L.sh_perm = take(ns * 4);

@@ -254,8 +254,10 @@ def layer_workspace_bytes(T: int) -> int:
 
 
 def alloc_layer_workspace(T: int, device, fp8: bool = False) -> torch.Tensor:
-    """A uint8 view of at least layer_workspace_bytes(T) bytes (or
-    layer_fp8_workspace_bytes(T) if fp8), 1024-byte aligned."""
+    """A uint8 view of at least layer_workspace_bytes(T) bytes, 1024-byte
+    aligned.  fp8=True sizes it for a quantised layer (moe_layer_fp8 or
+    moe_layer_nvfp4: layer_fp8_workspace_bytes(T), which
+    layer_nvfp4_workspace_bytes(T) equals)."""
     n = layer_fp8_workspace_bytes(T) if fp8 else layer_workspace_bytes(T)
     raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
     off = (-raw.data_ptr()) % 1024
