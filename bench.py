@@ -78,6 +78,8 @@ def parse():
                     help="shared experts (0-8) added to the main line's layer")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the decode_T16 (bf16, FP8, NVFP4, shared-expert) measurements")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="skip the 23-layer stack lines (T=1 and T=8189, one CUDA graph each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens in the oracle sample")
     return ap.parse_args()
@@ -691,6 +693,89 @@ def e256_line(T, dev, steps, warmup, peaks, barrier, seed=5):
             "gpu_launches": launches * steps, "clocks": clk.summary()}
 
 
+STACK_LAYERS, STACK_SEED = 23, 4
+
+
+def stack_packs(dev):
+    """The stack's 23 layers of independent bf16 experts (seed 4, layers 0..22),
+    packed: 13.9 GB."""
+    import torch
+    from group_limited_routed_moe_b200 import moe
+    packs = []
+    for l in range(STACK_LAYERS):
+        w = [synth.weight_bits_torch(STACK_SEED, l, m, dev)
+             for m in (synth.W_GATE, synth.W_UP, synth.W_DOWN)]
+        packs.append(moe.moe_pack_weights(*w))
+        del w
+    torch.cuda.synchronize()
+    return packs
+
+
+def stack_line(T, dev, packs, steps, warmup, peaks, barrier):
+    """The 23-layer stack on T tokens: seeded router logits per layer, a bf16
+    residual add between layers, the 23 moe_layer calls captured once as a CUDA
+    graph and replayed (no host sync between layers).  Each replay streams every
+    layer's touched experts, far more than L2 holds, so there is no flush; the
+    input is restored before each replay, outside the timed events."""
+    import torch
+    from group_limited_routed_moe_b200 import moe
+    tok = synth.make_tokens(T, STACK_SEED)
+    x0 = torch.from_numpy(tok.x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    h = x0.clone()
+    lgs, bs = [], []
+    for l in range(STACK_LAYERS):
+        lg, b = synth.layer_logits(T, STACK_SEED, l)
+        lgs.append(torch.from_numpy(lg).to(dev))
+        bs.append(torch.from_numpy(b).to(dev))
+    idx = [torch.empty((T, 8), dtype=torch.int32, device=dev) for _ in range(STACK_LAYERS)]
+    ws = moe.alloc_layer_workspace(T, dev)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for l in range(STACK_LAYERS):
+                moe.moe_layer(h, lgs[l], bs[l], packs[l], residual=h, out=h, topk_idx_out=idx[l],
+                              workspace=ws, stream=s)
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    for _ in range(warmup):
+        h.copy_(x0)
+        g.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    clk = ClockSampler(int(dev.index or 0))
+    barrier()
+    torch.cuda.synchronize()
+    with clk:
+        for a, b in evs:
+            h.copy_(x0)
+            a.record(cur)
+            g.replay()
+            b.record(cur)
+        torch.cuda.synchronize()
+    barrier()
+    status = moe.get_device_status(int(dev.index or 0))
+    del g
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    distinct = sum(int(torch.unique(i).numel()) for i in idx)
+    nbytes = distinct * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + \
+        STACK_LAYERS * T * (1536 * 4 + 512)
+    flops = STACK_LAYERS * FLOPS_PER_ROW * 8 * T
+    nb = (T + 127) // 128
+    n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
+    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "layers": STACK_LAYERS, "T": T, "us_per_layer": round(ms * 1e3 / STACK_LAYERS, 2),
+            "distinct_experts_all_layers": distinct,
+            "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),
+            "note": ("one CUDA graph of 23 moe_layer calls per step (bf16 residual add fused into "
+                     "the combine), no host sync between layers; no L2 flush (each step streams "
+                     f"{nbytes / 1e9:.2f} GB of expert weights)"),
+            "status_ok": status == moe.MOE_OK,
+            "gpu_launches": (n_rp + 2) * STACK_LAYERS * steps, "clocks": clk.summary()}
+
+
 def fp8_layer(dev):
     """The synthetic block-FP8 checkpoint of layer 0 (power-of-two block scales),
     packed, and its host codes and scales."""
@@ -819,6 +904,13 @@ def run_ours(args):
                                     line["decode_T16"]["ms_per_step"], args.steps, args.warmup,
                                     peaks, barrier)
             line["gpu_launches"] += line[key]["gpu_launches"]
+    if not args.no_stack:
+        packs = stack_packs(dev)
+        for T_s, key in ((1, "stack23_T1"), (8189, "stack23_T8189")):
+            n = max(10, args.steps // 2) if T_s == 1 else max(5, args.steps // 10)
+            line[key] = stack_line(T_s, dev, packs, n, args.warmup, peaks, barrier)
+            line["gpu_launches"] += line[key]["gpu_launches"]
+        del packs
     if args.e256_prefill:
         line["prefill_T8189_e256"] = e256_line(8189, dev, max(5, args.steps // 5), args.warmup,
                                                peaks, barrier)
