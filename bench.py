@@ -241,7 +241,7 @@ class LayerRun:
         self.part_names = ["route", "permute", "expert_ffn", "combine"]
         self.lws = moe.alloc_layer_workspace(T, dev, fp8=quant)
         if shared is not None:
-            n = moe.layer_shared_workspace_bytes(T, shared[1], fp8)
+            n = moe.layer_shared_workspace_bytes(T, shared[1], quant)
             raw = torch.empty(n + 1024, dtype=torch.uint8, device=dev)
             off = (-raw.data_ptr()) % 1024
             self.lws = raw[off:off + n]
@@ -264,7 +264,8 @@ class LayerRun:
     def step(self):
         """One layer through the public layer call (what a user runs)."""
         if self.shared is not None:
-            kw = {"packed_fp8": self.packed} if self.fp8 else {"packed_w": self.packed}
+            kw = ({"packed_nvfp4": self.packed} if self.nvfp4 else
+                  {"packed_fp8": self.packed} if self.fp8 else {"packed_w": self.packed})
             self.moe.moe_layer_shared(self.x[:self.T], self.logits[:self.T], self.bias,
                                       self.shared[0], self.shared[1], out=self.out[:self.T],
                                       workspace=self.lws, stream=self.stream, **kw)
@@ -837,8 +838,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     fp8 = args.weights == "fp8"
     nvfp4 = args.weights == "nvfp4"
-    if nvfp4 and args.shared:
-        raise SystemExit("--shared runs with bf16 or fp8 routed experts")
     wl = synth.WORKLOADS[args.workload]
     shared = shared_layer(dev, args.shared) if args.shared > 0 else None
     main_w = fp4_packed if nvfp4 else fp8_packed if fp8 else packed
