@@ -307,10 +307,12 @@ size_t moe_layer_fp8_workspace_bytes(int64_t T);
 
 /* moe_layer with block-FP8 experts (packed_fp8 from moe_pack_weights_fp8),
  * other arguments as in moe_layer.  For T <= 256 the single-launch expert FFN
- * streams the 8-bit codes and dequantises every weight tile in shared memory
- * on its way to the tensor cores (half the weight bytes of the bf16 layer);
- * above, the layer is first expanded into the workspace (moe_dequant_fp8) and
- * the bf16 expert FFN runs on it. */
+ * streams the 8-bit codes and dequantises every weight tile on its way to the
+ * tensor cores (half the weight bytes of the bf16 layer); above, the layer is
+ * first expanded into the workspace (moe_dequant_fp8) and the bf16 expert FFN
+ * runs on it.  A caller with the HBM to spare can expand once with
+ * moe_dequant_fp8 and call moe_layer on the result, which gives the same
+ * output. */
 int moe_layer_fp8(const moe_bf16* x, const float* logits, const float* bias,
                   const void* packed_fp8, int64_t T, const moe_bf16* residual,
                   moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
@@ -383,7 +385,11 @@ int moe_expert_ffn_nvfp4(const moe_bf16* x, const void* packed_nvfp4, const int3
 size_t moe_layer_nvfp4_workspace_bytes(int64_t T);
 
 /* moe_layer with NVFP4 experts (packed_nvfp4 from moe_pack_weights_nvfp4),
- * other arguments as in moe_layer; the expert FFN as moe_expert_ffn_nvfp4. */
+ * other arguments as in moe_layer; the expert FFN as moe_expert_ffn_nvfp4.
+ * Above 256 tokens every call expands the layer first (about half the time of
+ * the layer at 8K tokens); a caller with the HBM to spare (604 MB per layer)
+ * can expand once with moe_dequant_nvfp4 and call moe_layer on the result,
+ * which gives the same output. */
 int moe_layer_nvfp4(const moe_bf16* x, const float* logits, const float* bias,
                     const void* packed_nvfp4, int64_t T, const moe_bf16* residual,
                     moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
