@@ -356,9 +356,15 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }
 
 // ---------------------------------------------------------------- dynamic tile queue
-// Persistent GEMM CTAs take their first tile statically (blockIdx.x) and then
-// grab tiles from a global counter, so that a CTA that met slow tiles (weights
-// from HBM rather than L2, stalls) takes fewer of them.  Inside a CTA one
+// Persistent GEMM CTAs take every tile id, the first one included, from a
+// global counter, so that a CTA that met slow tiles (weights from HBM rather
+// than L2, stalls) takes fewer of them, and so that only a CTA that is
+// running can own a tile: in the single-launch expert FFN a down tile waits
+// for its expert's gate/up tiles, and those were handed out earlier (the
+// counter only grows) to CTAs that were running then and finish them without
+// waiting on anything outside the CTA.  So the wait ends however many of the
+// grid's CTAs are resident at once (SMs shared with another stream's
+// kernels, MPS, a green context with fewer SMs).  Inside a CTA one
 // thread grabs tile ids and publishes them through a small shared-memory queue
 // that every warp role reads in the same order.  The counter words live after
 // the expert offsets (see kSchedWord), followed by 128 per-expert completion

@@ -22,7 +22,7 @@
 // Work is cut into tiles (expert e, n-tile j, m-tile m) of 128 rows x 256
 // columns; tile ids run expert-major, then j, then m, so CTAs that run at the
 // same time share an expert's weight tile through L2.  A persistent grid of
-// one CTA per SM takes tile ids from a global counter (first tile: blockIdx.x),
+// one CTA per SM takes tile ids from a global counter (the first one too),
 // so that CTAs held up by slow tiles take fewer of them; static round-robin
 // left some CTAs up to 1.5x longer than the median.  The tile table is built
 // by each CTA from the device-side expert offsets, so the host never reads
@@ -214,6 +214,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
 
   // tile table: m-tiles of expert e = ceil(count_e / 128), exclusive prefix
   griddep_wait();  // offsets, perm_src and (down alone) h come from the preceding kernels
+  // The producer takes its first tile id from the counter too (issued here so
+  // that the atomic's round trip overlaps the tile-table set-up below).
+  int first_tile = 0;
+  if (threadIdx.x == C::TMA_WARP * 32) first_tile = atomicAdd(sched, 1);
   int my_mt = 0;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
     if (lane == 0) {
       int it = 0, n = 0;
       bool ok = true;
-      int tile = blockIdx.x;
+      int tile = first_tile;
       while (ok) {
         const int pub = tile < total_tiles ? tile : -1;
         if (!tileq_push(&S->tq, n++, pub, abort_flag, timeout_ns)) {
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
           break;
         }
         if (pub < 0) break;
-        const int next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);  // used after the loads
+        const int next = atomicAdd(sched, 1);  // used after the loads
         const TileInfo ti = tile_info<MODE>(S, tile, total1);
         if (MODE == 3 && ti.phase == 2) {
           // every gate/up tile of expert e has stored its h rows

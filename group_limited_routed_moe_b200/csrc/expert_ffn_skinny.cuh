@@ -23,9 +23,10 @@
 // producer waits (bounded) until a per-expert counter says every gate/up tile
 // of e has stored its h values; the gate/up epilogue makes its stores visible
 // to the TMA (async proxy) and then increments the counter with release
-// semantics.  Each CTA receives tile ids in increasing order, so the gate/up
-// tiles a waiting producer depends on were all handed out before, to CTAs that
-// run them without waiting: the wait always ends.  SMs that finish their last
+// semantics.  Every tile id, a CTA's first included, comes from one global
+// counter, so the gate/up tiles a waiting producer depends on were all handed
+// out before, to CTAs that were running and run them without waiting: the
+// wait ends however many CTAs of the grid are resident.  SMs that finish their last
 // gate/up tile go straight on to down tiles of experts that are ready instead
 // of idling until the slowest gate/up tile ends and a second launch ramps up.
 //
@@ -243,6 +244,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
   }
 
   griddep_wait();  // offsets, perm_src and (down alone) h come from the preceding kernels
+  // The producer takes its first tile id from the counter too (issued here so
+  // that the atomic's round trip overlaps the tile-table set-up below).
+  int first_tile = 0;
+  if (threadIdx.x == TMA_WARP * 32) first_tile = atomicAdd(sched, 1);
   int my_chunks = 0;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;
@@ -285,7 +290,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     if (lane == 0) {
       int it = 0, n = 0;
       bool ok = true;
-      int tile = blockIdx.x;
+      int tile = first_tile;
       while (ok) {
         const int pub = tile < total_tiles ? tile : -1;
         if (!tileq_push(&S->tq, n++, pub, abort_flag, timeout_ns)) {
@@ -293,7 +298,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
           break;
         }
         if (pub < 0) break;
-        const int next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);
+        const int next = atomicAdd(sched, 1);
         const TileInfo ti = tile_info<MODE>(S, tile, total1);
         const int e = ti.e, f = ti.f, c = ti.c;
         if (MODE == 3 && ti.phase == 2) {

@@ -1253,3 +1253,11 @@ extern "C" int moe_permute_fixed_scratch(const int32_t* topk_idx, int64_t T, int
   }
   return do_permute(topk_idx, T, counts, offsets, perm_src, inv_perm, hist, s);
 }
+
+// ---- explicit per-device set-up ----------------------------------------------
+extern "C" int moe_init_device(void) {
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  int32_t* hist = nullptr;
+  return fixed_perm_scratch(&hist);
+}

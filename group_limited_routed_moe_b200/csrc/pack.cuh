@@ -13,8 +13,11 @@
 //                                                                r >= 128 -> up col 128j + r - 128
 //   region D : [128 experts][1536 rows][512]  fp16  row n = output column n of W_down[e]
 // W_down is stored as fp16 so that the down GEMM multiplies the fp16 h by an
-// operand of the same type; every bf16 value in the fp16 normal range
-// converts exactly, and a weight beyond the fp16 range sets the status word.
+// operand of the same type.  Every bf16 value in the fp16 normal range
+// (magnitudes 2^-14 .. 65504) converts exactly; a smaller magnitude is rounded
+// to the nearest fp16 subnormal, an absolute error of at most 2^-25 (about
+// 0.2% of N(0, 0.02) weights fall there); a weight beyond the fp16 range sets
+// the status word.
 #pragma once
 #include "common.cuh"
 

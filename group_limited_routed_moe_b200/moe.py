@@ -46,6 +46,7 @@ _SIGS = {
     "moe_max_tokens": ([], _i64),
     "moe_last_error_string": ([], ctypes.c_char_p),
     "moe_get_device_status": ([_i32], _i32),
+    "moe_init_device": ([], _i32),
     "moe_set_wait_timeout_ns": ([_u64], _i32),
     "moe_selftest_wait_timeout": ([_p], _i32),
     "moe_packed_weight_bytes": ([], _sz),
@@ -669,6 +670,12 @@ class HostPipeline:
 
 def get_device_status(device: int = 0) -> int:
     return int(lib.moe_get_device_status(device))
+
+
+def init_device() -> None:
+    """Per-device set-up of the library on the current device (do it before
+    capturing library calls into a CUDA graph)."""
+    _check("moe_init_device", lib.moe_init_device())
 
 
 def set_wait_timeout_ns(ns: int) -> None:

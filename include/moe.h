@@ -33,6 +33,18 @@
  *   - Device-side waits inside the kernels are bounded in time.  A wait that
  *     runs out sets a per-device error word and makes the kernel return;
  *     moe_get_device_status() reports it as MOE_ERR_TIMEOUT.
+ *   - The first call of the library on a device sets that device up: it
+ *     queries its properties, raises the kernels' shared-memory limits
+ *     (cudaFuncSetAttribute) and resolves the tensor-map encoder.  Those
+ *     calls are not stream operations, so make the first call on each device
+ *     outside stream capture (moe_init_device() does the set-up alone); later
+ *     calls only launch kernels and can be captured into a CUDA graph.
+ *   - Calls on different streams may run at the same time on one device (they
+ *     share nothing but the device status word), provided they do not share
+ *     a workspace or an offsets array.  The persistent expert-FFN kernels
+ *     hand out every tile, the first included, from a global counter, so a
+ *     kernel that gets fewer SMs than its grid (another stream's kernels, MPS
+ *     or a green context) still finishes: only running CTAs own work.
  */
 #ifndef MOE_B200_MOE_H
 #define MOE_B200_MOE_H
@@ -91,6 +103,14 @@ const char* moe_last_error_string(void);
  * This is the one call that synchronises: it copies 4 bytes to the host. */
 int moe_get_device_status(int device);
 
+/* Sets the current device up for the library (the set-up that the first call
+ * on a device does otherwise): checks that it is an sm_100 device, raises the
+ * kernels' shared-memory limits, resolves the tensor-map encoder and looks up
+ * the device address of moe_permute_fixed_scratch's scratch array.  Call it
+ * once per device, with that device current, before capturing any library
+ * call into a CUDA graph.  Idempotent; MOE_ERR_UNSUPPORTED on other devices. */
+int moe_init_device(void);
+
 /* Time limit of every bounded device-side wait, in nanoseconds (default 2e9).
  * Applies to launches issued after the call. */
 int moe_set_wait_timeout_ns(uint64_t ns);
@@ -107,8 +127,11 @@ int moe_selftest_wait_timeout(moe_stream_t stream);
 size_t moe_packed_weight_bytes(void);
 
 /* One-time re-layout of one layer's expert weights into the tensor-core
- * operand order used by moe_expert_ffn (W_down converted to fp16, exact for
- * bf16 values in the fp16 normal range).
+ * operand order used by moe_expert_ffn.  W_down is converted to fp16: exact
+ * for bf16 values in the fp16 normal range [2^-14, 65504]; a magnitude below
+ * 2^-14 is rounded to the nearest fp16 subnormal (an absolute error of at
+ * most 2^-25 per weight); a magnitude above 65504 is flagged (MOE_ERR_RANGE
+ * from moe_get_device_status()).
  *   w_gate, w_up : [128][1536][512] bf16, the layer computes x @ W_gate[e]
  *   w_down       : [128][512][1536] bf16, the layer computes h @ W_down[e]
  *   packed       : moe_packed_weight_bytes() bytes, 128-byte aligned, output.
@@ -123,8 +146,10 @@ int moe_pack_weights(const moe_bf16* w_gate, const moe_bf16* w_up,
 
 /* ---- the four steps ----------------------------------------------------- */
 
-/* Step 1: group-limited top-8 routing, one warp per token.
- * Group-limited routing runs as its own kernel in the GB10 CUDA path of issue
+/* Step 1: group-limited top-8 routing.  Up to 64 tokens one warp works on
+ * each token (moe_layer fuses this with step 2 in one block); above that, 8
+ * lanes share a token, one per group, which needs half the instructions per
+ * token at large T.  Group-limited routing runs as its own kernel in the GB10 CUDA path of issue
  * #1247 ("What it does not cover", bullet on the CUDA C kernels); the score
  * rule used here:
  *   s_e = sigmoid(logit[t,e] + bias[e])                 (float64)
@@ -170,8 +195,10 @@ int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts,
  *                       two calls sharing one offsets array must not overlap)
  *   h        : [8T][512] fp16 workspace (out), 128-byte aligned
  *   y_perm   : [8T][1536] fp16 (out)
- * For T <= 256 both GEMMs run in one persistent launch (a down tile starts as
- * soon as its expert's gate/up tiles have stored h); above, two launches. */
+ * Both GEMMs run in one persistent launch at every T: a down tile starts as
+ * soon as every gate/up tile of its expert has stored h.  Up to 256 tokens
+ * the weights are the 128-row MMA operand (128 weight rows x 32 tokens per
+ * tile); above, the tokens are (128 rows x 256 output columns per tile). */
 int moe_expert_ffn(const moe_bf16* x, const moe_bf16* packed_w,
                    const int32_t* offsets, const int32_t* perm_src, int64_t T,
                    moe_f16* h, moe_f16* y_perm, moe_stream_t stream);
@@ -491,8 +518,9 @@ int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
  *            larger T returns MOE_ERR_INVALID_ARG with nothing launched.
  *   Outputs: identical, bit for bit, to moe_permute's for the same topk_idx.
  *   Set-up : the first call on a device (with that device current) looks up
- *            the array's device address; make that first call before any
- *            stream capture.
+ *            the array's device address, unless moe_init_device() has done so;
+ *            make that first call, or moe_init_device(), before any stream
+ *            capture.
  *   Races  : one array per device serves every call, so two calls whose
  *            kernels may overlap (different streams with no ordering between
  *            them, or several host threads) corrupt each other's result.

@@ -2,17 +2,19 @@
 between layers, replayed from one CUDA graph with no host sync between
 layers.  Routing logits of every layer are independent seeded inputs.
 
-T=1 is checked on the whole output; T=8189 (buffers of 8192) on sampled
-tokens, each token's path through the 23 layers being independent of the
-others.
+T=1 is checked on the whole output; T=8189 (buffers of 8192) on 256 sampled
+tokens (seeded, first and last included), each token's path through the 23
+layers being independent of the others.
 
 Tolerances.  The stack output h_23 is compared with rel-L2 <= 5e-3, the
 layer tolerance.  Both sides round the residual stream to bf16 after every
-layer; they round slightly different values (the GPU's MoE output carries
-its ~2e-3 relative error), so a few percent of the elements land one bf16
-ulp apart per layer.  Over 23 layers those flips add up to roughly 1% of the
-accumulated update h_23 - x, so the update itself gets a looser, derived
-bound of 3e-2 -- a wrong expert, weight or sign would be off by O(1).
+layer; they round slightly different values (the GPU's MoE output carries a
+small relative error), and once one element lands one bf16 ulp apart the
+difference spreads through later layers' rounding.  The accumulated update
+h_23 - x is bounded by UPDATE_FACTOR x the floor that the oracle itself
+shows when each layer's update is perturbed by a relative 2e-3
+(tests/stack_noise.py, pinned by a CPU test); a wrong expert, weight or sign
+would be off by O(1).  The measured update error is printed beside the bound.
 """
 import numpy as np
 import pytest
@@ -20,6 +22,7 @@ import torch
 
 import oracle as O
 from group_limited_routed_moe_b200 import synth
+import stack_noise
 from gpu_helpers import DEV, REL_L2_TOL, LayerWeights, to_dev_bf16, to_host_bits
 
 pytestmark = pytest.mark.gpu
@@ -68,24 +71,30 @@ def _run_stack(layers, tok_x_bits, logits, T_buf):
 
 
 def _oracle(layers, x_bits, logits, rows):
-    per_layer = []
+    # one layer at a time (a one-layer stack applied 23 times is the 23-layer
+    # stack), so that only one layer's host weights are held at once
+    h = x_bits[rows]
     for l, W in enumerate(layers):
         lg, b = logits[l]
         lg = lg[rows]
         rr = O.route(lg, b)
-        per_layer.append((lg, b) + W.host(rr.topk_idx))
-    return O.moe_stack(x_bits[rows], per_layer)
+        h = O.moe_stack(h, [(lg, b) + W.host(rr.topk_idx)])
+    return h
 
 
-UPDATE_TOL = 3e-2
+UPDATE_TOL = stack_noise.UPDATE_FACTOR * stack_noise.UPDATE_FLOOR
+N_SAMPLED = 256
 
 
-def _compare(got_bits, ref_bits, x_bits):
+def _compare(got_bits, ref_bits, x_bits, what):
     got, ref = O.bf16_bits_to_f64(got_bits), O.bf16_bits_to_f64(ref_bits)
     x = O.bf16_bits_to_f64(x_bits)
     err = O.rel_l2(got, ref)
-    assert err <= REL_L2_TOL, f"rel-L2 of the stack output {err:.3e}"
     uerr = O.rel_l2(got - x, ref - x)
+    print(f"{what}: stack output rel-L2 {err:.3e} (bound {REL_L2_TOL:.1e}); update rel-L2 "
+          f"{uerr:.3e} (bound {UPDATE_TOL:.3e} = {stack_noise.UPDATE_FACTOR} x oracle floor "
+          f"{stack_noise.UPDATE_FLOOR:.2e})")
+    assert err <= REL_L2_TOL, f"rel-L2 of the stack output {err:.3e}"
     assert uerr <= UPDATE_TOL, f"rel-L2 of the stack update {uerr:.3e}"
 
 
@@ -94,7 +103,7 @@ def test_stack_T1(stack):
     logits = _logits(1)
     h = _run_stack(stack, x_bits, logits, 1)
     ref = _oracle(stack, x_bits, logits, np.arange(1))
-    _compare(to_host_bits(h), ref, x_bits)
+    _compare(to_host_bits(h), ref, x_bits, "T=1")
 
 
 def test_stack_T8189_sampled(stack):
@@ -102,7 +111,11 @@ def test_stack_T8189_sampled(stack):
     x_bits = synth.make_tokens(T, SEED).x_bits
     logits = _logits(T)
     h = _run_stack(stack, x_bits, logits, T_buf)
-    rows = np.array([0, 1, 2047, 4095, 6000, 8188])
+    rng = np.random.default_rng(8189)
+    rows = np.unique(np.concatenate([[0, T - 1], rng.choice(T, N_SAMPLED - 2, replace=False)]))
+    rows = rows[:N_SAMPLED]
+    assert len(rows) >= N_SAMPLED - 2
     ref = _oracle(stack, x_bits, logits, rows)
-    _compare(to_host_bits(h[torch.as_tensor(rows, device=DEV)]), ref, x_bits[rows])
+    _compare(to_host_bits(h[torch.as_tensor(rows, device=DEV)]), ref, x_bits[rows],
+             f"T=8189, {len(rows)} sampled tokens")
     assert torch.all(h[T:] == 0)

@@ -1,10 +1,13 @@
 """moe_permute_fixed_scratch (library-owned scratch, no device allocation)
-against moe_permute, called through the C ABI.
+against moe_permute and against the float64 oracle's permutation, called
+through the C ABI.
 
 Collected last so that it also runs after every other GPU test in one process;
 it passes on its own in a fresh process as well.  Each case makes two calls in
 a row on different routings: the second must not see anything the first left
-in the shared scratch.  Integer outputs, so the comparison is bit-exact."""
+in the shared scratch; one case goes from the largest T (512 histogram rows)
+to a smaller multi-block T, whose call must never read the stale rows past
+its own blocks.  Integer outputs, so the comparison is bit-exact."""
 
 import ctypes
 
@@ -12,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from group_limited_routed_moe_b200 import moe as M
 
 N_EXPERTS, TOPK, OFFSETS_LEN = M.N_EXPERTS, M.TOPK, M.OFFSETS_LEN
@@ -45,7 +49,7 @@ def _fixed(idx_dev, stream):
     return counts, offsets, perm[:T * TOPK], inv[:T * TOPK]
 
 
-def _same(got, ref):
+def _same(got, ref, idx):
     counts, offsets, perm, inv = got
     r_counts, r_offsets, r_perm, r_inv = ref
     assert torch.equal(counts.cpu(), r_counts.cpu())
@@ -53,6 +57,12 @@ def _same(got, ref):
     assert torch.equal(offsets[132:OFFSETS_LEN].cpu(), torch.zeros(OFFSETS_LEN - 132, dtype=torch.int32))
     assert torch.equal(perm.cpu(), r_perm.cpu())
     assert torch.equal(inv.cpu(), r_inv.cpu())
+    # and against the oracle's stable counting sort of the same routing
+    o = O.permute(idx.cpu().numpy())
+    np.testing.assert_array_equal(counts.cpu().numpy(), o.counts)
+    np.testing.assert_array_equal(offsets[:N_EXPERTS + 1].cpu().numpy(), o.offsets)
+    np.testing.assert_array_equal(perm.cpu().numpy(), o.perm_src)
+    np.testing.assert_array_equal(inv.cpu().numpy(), o.inv_perm)
 
 
 @pytest.mark.gpu
@@ -65,11 +75,25 @@ def test_fixed_scratch_permute_matches_moe_permute(T, hot):
         ref = M.moe_permute(idx)
         got = _fixed(idx, stream)
         torch.cuda.synchronize()
-        _same(got, ref)
+        _same(got, ref, idx)
         if T:
             rows = np.sort(got[2].cpu().numpy())
             assert np.array_equal(rows, np.arange(T * TOPK))
     torch.cuda.synchronize()
+    assert M.lib.moe_get_device_status(torch.cuda.current_device()) == M.MOE_OK
+
+
+@pytest.mark.gpu
+def test_fixed_scratch_permute_large_then_small():
+    """T = 65536 (512 blocks) fills every histogram row; T = 2000 (16 blocks,
+    the multi-block path) then runs on the same stream with rows 16..511 stale."""
+    stream = torch.cuda.current_stream()
+    for T, seed, hot in ((65536, 5, 0), (2000, 6, 16), (65536, 7, 8), (1100, 8, 0)):
+        idx = _routing(T, seed, hot).cuda()
+        ref = M.moe_permute(idx)
+        got = _fixed(idx, stream)
+        torch.cuda.synchronize()
+        _same(got, ref, idx)
     assert M.lib.moe_get_device_status(torch.cuda.current_device()) == M.MOE_OK
 
 
