@@ -78,6 +78,8 @@ def parse():
                     help="shared experts (0-8) added to the main line's layer")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the decode_T16 (bf16, FP8, NVFP4, shared-expert) measurements")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the decode_T4 (seeds 1-8) and prefill_T2048_skewed lines")
     ap.add_argument("--no-stack", action="store_true",
                     help="skip the 23-layer stack lines (T=1 and T=8189, one CUDA graph each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -597,6 +599,149 @@ def decode_line(wl2, dev, packed, fp8, steps, warmup, peaks, peak_kind, barrier,
     return out
 
 
+def ffn_trace_run(run):
+    """One more pass of the breakdown's step calls with the expert FFN's per-CTA
+    record switched on (moe_set_ffn_trace): how the launch's tiles spread over
+    the SMs.  Returns the tail summary of that launch."""
+    torch, moe = run.torch, run.moe
+    buf = torch.zeros((1024, 3), dtype=torch.int64, device=run.dev)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(run.part_names) + 1)]
+    run.flush()
+    moe.set_ffn_trace(buf)
+    try:
+        run.step_parts(evs)
+        torch.cuda.synchronize()
+    finally:
+        moe.set_ffn_trace(None)
+    tr = buf.cpu().numpy()
+    tr = tr[tr[:, 1] > 0]
+    return ffn_tail(tr)
+
+
+def ffn_tail(tr):
+    """Tail of one persistent FFN launch from its per-CTA record (rows: start ns,
+    end ns, tiles).  idle_sm_frac: the share of CTA-time between the first
+    CTA's start and the last CTA's end that CTAs spent not yet started or
+    already finished; tail_us: from the first CTA to run out of tiles to the
+    last one."""
+    start, end, tiles = tr[:, 0].astype(np.float64), tr[:, 1].astype(np.float64), tr[:, 2]
+    k0, k1 = start.min(), end.max()
+    span = k1 - k0
+    busy = end - start
+    return {"ctas": int(len(tr)), "span_us": round(span / 1e3, 2),
+            "idle_sm_frac": round(float(1.0 - busy.sum() / (len(tr) * span)), 4),
+            "tail_us": round((k1 - end.min()) / 1e3, 2),
+            "start_spread_us": round((start.max() - k0) / 1e3, 2),
+            "end_p50_us": round((float(np.median(end)) - k0) / 1e3, 2),
+            "tiles_per_cta": {"min": int(tiles.min()), "median": float(np.median(tiles)),
+                              "max": int(tiles.max())}}
+
+
+def skewed_line(dev, packed, steps, warmup, peaks, barrier):
+    """The chunked prefill with 16 hot experts (+2.0 on their logits): whole-layer
+    steps, the per-expert row counts, and the expert FFN against both roofs
+    (at a mean of 128 rows per expert it sits below the ridge, so HBM and the
+    tensor cores are both reported) with the tail of its grouped GEMM."""
+    wl = synth.WORKLOADS["prefill_T2048_skewed"]
+    run = LayerRun(wl, dev, packed)
+    clk = ClockSampler(int(dev.index or 0))
+    n = max(steps, 30)
+    with clk:
+        st, _ = run.timed(n, warmup, barrier)
+    per = run.breakdown(n)
+    tail = ffn_trace_run(run)
+    counts = run.counts.cpu().numpy()
+    T = wl.T
+    ffn_ms = float(per[:, run.part_names.index("expert_ffn")].mean())
+    d = int((counts > 0).sum())
+    nbytes = d * (GATE_UP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT) + T * 1536 * 2 + \
+        8 * T * 1536 * 2
+    flops = FLOPS_PER_ROW * 8 * T
+    ms = float(st.mean())
+    hot = set(int(e) for e in run.tok.hot_experts)
+    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 5),
+            "T": T, "hot_experts": sorted(hot),
+            "counts": [int(c) for c in counts],
+            "M": {"max": int(counts.max()), "mean": round(float(counts.mean()), 2),
+                  "max_over_mean": round(float(counts.max() / counts.mean()), 3),
+                  "mean_hot": round(float(np.mean([counts[e] for e in hot])), 1),
+                  "mean_other": round(float(np.mean([c for e, c in enumerate(counts)
+                                                     if e not in hot])), 1)},
+            "expert_ffn": {"us": round(ffn_ms * 1e3, 2), "distinct_experts": d,
+                           "hbm_frac": round(nbytes / (ffn_ms * 1e-3) / 1e9 /
+                                             float(peaks["hbm_gbs"]), 4),
+                           "tensor_frac": round(flops / (ffn_ms * 1e-3) / 1e12 /
+                                                float(peaks["bf16_tflops"]), 4),
+                           "tail": tail},
+            "layer": layer_fractions(wl, run, st, per, peaks),
+            "gpu_launches": run.launches_per_step * n + len(run.part_names),
+            "clocks": clk.summary()}
+
+
+def decode_T4_line(dev, packed, steps, warmup, peaks, peak_kind, barrier):
+    """Four concurrent decode streams, seeds 1..8, each seed its own batch:
+    per-seed whole-layer time and the expert FFN's HBM fraction, and their
+    medians."""
+    per_seed = []
+    launches = 0
+    clk = ClockSampler(int(dev.index or 0))
+    with clk:
+        for s in range(1, 9):
+            wl = synth.WORKLOADS[f"decode_T4_seed{s}"]
+            run = LayerRun(wl, dev, packed)
+            n = max(steps, 30)
+            st, _ = run.timed(n, warmup, barrier)
+            per = run.breakdown(n)
+            rf = roofline_for(wl, run, per, peaks, peak_kind)
+            lf = layer_fractions(wl, run, st, per, peaks)
+            per_seed.append({"seed": s, "layer_us": lf["layer_us"],
+                             "ffn_us": lf["kernel_us"]["expert_ffn"],
+                             "distinct_experts": rf["distinct_experts"],
+                             "ffn_hbm_frac": rf["frac"], "layer_hbm_frac": lf["hbm_frac"]})
+            launches += run.launches_per_step * n
+            del run
+    med = {k: round(float(np.median([p[k] for p in per_seed])), 4)
+           for k in ("layer_us", "ffn_us", "distinct_experts", "ffn_hbm_frac", "layer_hbm_frac")}
+    return {"value": round(4 / (med["layer_us"] * 1e-6), 1), "unit": "tokens/s",
+            "T": 4, "median": med, "per_seed": per_seed, "gpu_launches": launches,
+            "clocks": clk.summary()}
+
+
+def summary_of(line, main_name):
+    """A short digest of every configuration's headline numbers, placed last on
+    the JSON line so that the end of the output shows it."""
+    bound = line["roofline"]["bound"]
+    key = "tensor" if bound == "tensor" else "hbm"
+    out = {main_name: {"us": line["layer"]["layer_us"],
+                       f"ffn_{key}_frac": line["roofline"]["frac"],
+                       f"layer_{key}_frac": line["layer"][f"{key}_frac"]}}
+    if "decode_T16" in line:
+        d = line["decode_T16"]
+        out["decode_T16"] = {"us": d["layer"]["layer_us"], "ffn_hbm_frac": d["roofline"]["frac"],
+                             "layer_hbm_frac": d["layer"]["hbm_frac"]}
+    for k in ("decode_T16_fp8", "decode_T16_nvfp4"):
+        if k in line:
+            out[k] = {"us": line[k]["layer"]["layer_us"],
+                      "ffn_hbm_frac": line[k]["roofline"]["frac"]}
+    if "decode_T4" in line:
+        m = line["decode_T4"]["median"]
+        out["decode_T4_median"] = {"us": m["layer_us"], "ffn_hbm_frac": m["ffn_hbm_frac"]}
+    if "prefill_T2048_skewed" in line:
+        k = line["prefill_T2048_skewed"]
+        out["prefill_T2048_skewed"] = {
+            "us": round(k["ms_per_step"] * 1e3, 2), "max_over_mean_M": k["M"]["max_over_mean"],
+            "ffn_hbm_frac": k["expert_ffn"]["hbm_frac"],
+            "ffn_tensor_frac": k["expert_ffn"]["tensor_frac"],
+            "ffn_idle_sm_frac": k["expert_ffn"]["tail"]["idle_sm_frac"]}
+    for k in ("stack23_T1", "stack23_T8189"):
+        if k in line:
+            out[k] = {"us_per_layer": line[k]["us_per_layer"], "tok_s": line[k]["value"]}
+    for k in ("decode_T16_e256", "decode_T16_shared1"):
+        if k in line:
+            out[k] = {"us": round(line[k]["ms_per_step"] * 1e3, 2)}
+    return out
+
+
 def shared_layer(dev, n_shared):
     """n_shared synthetic shared experts of layer 0, packed."""
     import torch
@@ -903,6 +1048,13 @@ def run_ours(args):
                                     line["decode_T16"]["ms_per_step"], args.steps, args.warmup,
                                     peaks, barrier)
             line["gpu_launches"] += line[key]["gpu_launches"]
+    if not args.no_configs:
+        line["decode_T4"] = decode_T4_line(dev, packed, args.steps, args.warmup, peaks, peak_kind,
+                                           barrier)
+        line["gpu_launches"] += line["decode_T4"]["gpu_launches"]
+        line["prefill_T2048_skewed"] = skewed_line(dev, packed, args.steps, args.warmup, peaks,
+                                                   barrier)
+        line["gpu_launches"] += line["prefill_T2048_skewed"]["gpu_launches"]
     if not args.no_stack:
         packs = stack_packs(dev)
         for T_s, key in ((1, "stack23_T1"), (8189, "stack23_T8189")):
@@ -921,6 +1073,7 @@ def run_ours(args):
             hw = host_weights()
         line["cpu_baseline"] = cpu_baseline(wl, run.tok, hw, args.cpu_sample, fp8=fp8,
                                             nvfp4=nvfp4)
+    line["summary"] = summary_of(line, wl.name)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
                     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
                     const int32_t* __restrict__ perm_src, int64_t T,
                     uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
-                    int* __restrict__ sched, int* __restrict__ done, uint64_t timeout_ns) {
+                    int* __restrict__ sched, int* __restrict__ done, uint64_t timeout_ns,
+                    uint64_t* __restrict__ trace) {
   using C = Cfg<MODE>;
 
   extern __shared__ uint8_t smem_raw[];
@@ -216,6 +217,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
   griddep_wait();  // offsets, perm_src and (down alone) h come from the preceding kernels
   // The producer takes its first tile id from the counter too (issued here so
   // that the atomic's round trip overlaps the tile-table set-up below).
+  if (trace != nullptr && threadIdx.x == 0) trace[3 * blockIdx.x] = global_timer_ns();
   int first_tile = 0;
   if (threadIdx.x == C::TMA_WARP * 32) first_tile = atomicAdd(sched, 1);
   int my_mt = 0;
@@ -307,6 +309,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
         }
         tile = next;
       }
+      if (trace != nullptr) trace[3 * blockIdx.x + 2] = static_cast<uint64_t>(n - 1);  // tiles
       if (!ok) {
         // let the copies already issued land before the block can exit
         for (int i = max(0, it - STAGES); i < it; ++i)
@@ -513,7 +516,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
+  if (threadIdx.x == 0) {
+    if (trace != nullptr) trace[3 * blockIdx.x + 1] = global_timer_ns();
+    tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
+  }
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

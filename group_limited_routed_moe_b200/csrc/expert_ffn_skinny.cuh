@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
                        uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
                        int* __restrict__ sched, int* __restrict__ done,
                        const void* __restrict__ wscale,  // FP8 scales (SGU, SD) or FP4 MGU, MD
-                       uint64_t timeout_ns) {
+                       uint64_t timeout_ns,
+                       uint64_t* __restrict__ trace) {  // NULL, or 3 words per CTA (see ffn_trace)
   constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
   static_assert(!WQ || MODE == 3, "quantised weights only in the single-launch form");
   using R = Ring<WQ>;
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
   griddep_wait();  // offsets, perm_src and (down alone) h come from the preceding kernels
   // The producer takes its first tile id from the counter too (issued here so
   // that the atomic's round trip overlaps the tile-table set-up below).
+  if (trace != nullptr && threadIdx.x == 0) trace[3 * blockIdx.x] = global_timer_ns();
   int first_tile = 0;
   if (threadIdx.x == TMA_WARP * 32) first_tile = atomicAdd(sched, 1);
   int my_chunks = 0;
@@ -364,6 +366,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
         }
         tile = next;
       }
+      if (trace != nullptr) trace[3 * blockIdx.x + 2] = static_cast<uint64_t>(n - 1);  // tiles
       if (!ok) {
         for (int i = max(0, it - RST); i < it; ++i)
           mbar_wait(&fullb[i % RST], (i / RST) & 1, abort_flag, 10000000ull, kSiteFfnFull);
@@ -663,7 +666,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
+  if (threadIdx.x == 0) {
+    if (trace != nullptr) trace[3 * blockIdx.x + 1] = global_timer_ns();
+    tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
+  }
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, R::TMEM_COLS);

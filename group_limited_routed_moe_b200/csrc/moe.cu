@@ -39,6 +39,15 @@ constexpr int64_t kSkinnyMaxT = 256;    // weights-as-M (skinny) GEMMs up to thi
 thread_local char g_err[512] = "";
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 
+// Per-CTA timing record of the expert-FFN launches (moe_set_ffn_trace); NULL
+// when off.  A launch of `ctas` CTAs records only if the buffer holds them all.
+std::atomic<uint64_t*> g_trace{nullptr};
+std::atomic<int64_t> g_trace_cap{0};
+uint64_t* ffn_trace(int ctas) {
+  uint64_t* p = g_trace.load();
+  return (p != nullptr && g_trace_cap.load() >= ctas) ? p : nullptr;
+}
+
 int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -298,7 +307,7 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
                       reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                       reinterpret_cast<uint16_t*>(h), static_cast<uint16_t*>(nullptr),
                       sched_words(offsets, 1), static_cast<int*>(nullptr),
-                      static_cast<const float*>(nullptr), g_timeout_ns.load());
+                      static_cast<const float*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -310,7 +319,7 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
                     T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<1, true> : ffn::ffn_gemm_kernel<1, false>,
                     dim3(sms), dim3(ffn::Cfg<1>::THREADS), ffn::SMEM_BYTES, s, tb1, tb1, tb1, xb,
                     offsets, perm_src, T, hb, static_cast<uint16_t*>(nullptr),
-                    sched_words(offsets, 1), static_cast<int*>(nullptr), g_timeout_ns.load());
+                    sched_words(offsets, 1), static_cast<int*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
 }
 
 int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, int64_t T,
@@ -328,7 +337,7 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                       static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
                       reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
                       static_cast<int*>(nullptr), static_cast<const float*>(nullptr),
-                      g_timeout_ns.load());
+                      g_timeout_ns.load(), ffn_trace(sms));
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -339,7 +348,7 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                     static_cast<const __nv_bfloat16*>(nullptr), offsets,
                     static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
                     reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
-                    static_cast<int*>(nullptr), g_timeout_ns.load());
+                    static_cast<int*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
 }
 
 // n_exp: experts in the pack (128, or the shared experts' count), d_off: start
@@ -361,7 +370,7 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                       reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                       reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
                       sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                      static_cast<const float*>(nullptr), g_timeout_ns.load());
+                      static_cast<const float*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
   // both GEMMs in one launch (see expert_ffn.cuh)
   CUtensorMap tb1, tb2, ta2;
@@ -378,7 +387,7 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                     reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                     reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
                     sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                    g_timeout_ns.load());
+                    g_timeout_ns.load(), ffn_trace(sms));
 }
 
 // Packed block-FP8 layer -> packed bf16/fp16 layer.
@@ -413,7 +422,7 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
                     th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                     reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
                     sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                    static_cast<const void*>(p8 + fp8::kSguOff), g_timeout_ns.load());
+                    static_cast<const void*>(p8 + fp8::kSguOff), g_timeout_ns.load(), ffn_trace(sms));
 }
 
 // Packed NVFP4 layer -> packed bf16/fp16 layer.
@@ -445,7 +454,7 @@ int do_expert_ffn_fp4(const moe_bf16* x, const void* packed4, const int32_t* off
                     th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
                     reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
                     sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                    static_cast<const void*>(p4 + fp4::kMguOff), g_timeout_ns.load());
+                    static_cast<const void*>(p4 + fp4::kMguOff), g_timeout_ns.load(), ffn_trace(sms));
 }
 
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
@@ -542,6 +551,19 @@ int moe_get_device_status(int device) {
                 "multiplier leaves the normal range of its operand type");
   return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out (status 0x%08x, site %u)", v,
               v & 0x7FFFFFFFu);
+}
+
+int moe_set_ffn_trace(uint64_t* buf, int64_t capacity_ctas) {
+  if (buf == nullptr) {
+    g_trace.store(nullptr);
+    g_trace_cap.store(0);
+    return MOE_OK;
+  }
+  REQUIRE(aligned(buf, 8), "trace buffer must be 8-byte aligned");
+  REQUIRE(capacity_ctas > 0, "trace capacity must be positive");
+  g_trace_cap.store(capacity_ctas);
+  g_trace.store(buf);
+  return MOE_OK;
 }
 
 int moe_set_wait_timeout_ns(uint64_t ns) {
@@ -977,6 +999,48 @@ int moe_pack_shared(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16
   pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_up, packed_shared, kH, kI, 1, d_off);
   pack_transpose_kernel<<<gd, 256, 0, s>>>(w_down, packed_shared, kI, kH, 2, d_off);
   return launch_check("pack_transpose_kernel launch (shared)");
+}
+
+// ---- a slice of a layer's experts (expert parallelism) ---------------------------
+size_t moe_packed_experts_bytes(int n_experts) {
+  if (n_experts < 1 || n_experts > kE) return 0;
+  return static_cast<size_t>(n_experts) * (kPackGuPerExpert + kPackDPerExpert) * 2;
+}
+
+int moe_pack_experts(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                     int n_experts, moe_bf16* packed, moe_stream_t stream) {
+  REQUIRE(n_experts >= 1 && n_experts <= kE, "n_experts=%d outside [1, %d]", n_experts, kE);
+  REQUIRE(w_gate && w_up && w_down && packed, "null pointer");
+  REQUIRE(aligned(packed, 128), "packed must be 128-byte aligned");
+  int rc = device_setup(nullptr, nullptr);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t d_off = int64_t(n_experts) * kPackGuPerExpert;
+  const dim3 ggu(kI / 32, kH / 32, n_experts), gd(kH / 32, kI / 32, n_experts);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_gate, packed, kH, kI, 0, d_off);
+  pack_transpose_kernel<<<ggu, 256, 0, s>>>(w_up, packed, kH, kI, 1, d_off);
+  pack_transpose_kernel<<<gd, 256, 0, s>>>(w_down, packed, kI, kH, 2, d_off);
+  return launch_check("pack_transpose_kernel launch (expert slice)");
+}
+
+int moe_expert_ffn_slice(const moe_bf16* x, const moe_bf16* packed, int n_experts,
+                         const int32_t* offsets, const int32_t* perm_src, int64_t T, moe_bf16* h,
+                         moe_bf16* y_perm, moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(n_experts >= 1 && n_experts <= kE, "n_experts=%d outside [1, %d]", n_experts, kE);
+  REQUIRE(x && packed && offsets && perm_src && h && y_perm, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed, 128) && aligned(h, 128),
+          "x, packed and h must be 128-byte aligned");
+  REQUIRE(aligned(y_perm, 16) && aligned(offsets, 16) && aligned(perm_src, 16),
+          "pointers must be 16-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  return do_expert_ffn(x, packed, offsets, perm_src, T, h, y_perm, sms,
+                       reinterpret_cast<cudaStream_t>(stream), n_experts,
+                       int64_t(n_experts) * kPackGuPerExpert);
 }
 
 size_t moe_layer_shared_workspace_bytes(int64_t T, int n_shared, int fp8_routed) {

@@ -18,6 +18,10 @@
 namespace moe {
 
 constexpr int kPermSmallMaxT = 1024;   // single-block path up to this many tokens
+// A slot holding this id is empty: it gets no row (inv_perm = -1) and is not
+// counted.  A token's slots may mix experts and empty slots; the expert-parallel
+// receiver uses it for the slots of a row whose expert lives on another rank.
+constexpr int kEmptySlot = -1;
 constexpr int kPermBlockTokens = 128;  // tokens per block on the multi-block path
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
@@ -63,7 +67,7 @@ __global__ void __launch_bounds__(1024)
   for (int p = tid; p < n; p += blockDim.x) {
     const int e = idx[p];
     if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
-      record_status(kSiteBadIndex);
+      if (e != kEmptySlot) record_status(kSiteBadIndex);
       continue;
     }
     const int t = p >> 3;
@@ -87,7 +91,10 @@ __global__ void __launch_bounds__(1024)
   if (tid < kOffsetsLen - kSchedWord) offsets[kSchedWord + tid] = 0;  // GEMM tile counters
   for (int p = tid; p < n; p += blockDim.x) {
     const int e = idx[p];
-    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
+      inv_perm[p] = -1;  // an empty slot (or a bad id, reported above) has no row
+      continue;
+    }
     const int t = p >> 3;
     const int r = off[e] + pre[e][t >> 5] + __popc(bm[e][t >> 5] & ((1u << (t & 31)) - 1u));
     perm_src[r] = p;
@@ -110,7 +117,7 @@ __global__ void __launch_bounds__(256)
   for (int q = tid; q < nt * kTopK; q += blockDim.x) {
     const int e = idx[t0 * kTopK + q];
     if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
-      record_status(kSiteBadIndex);
+      if (e != kEmptySlot) record_status(kSiteBadIndex);
       continue;
     }
     const int tl = q >> 3;
@@ -221,7 +228,10 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   for (int q = tid; q < nt * kTopK; q += blockDim.x) {
     const int e = idx[t0 * kTopK + q];
-    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
+      inv_perm[t0 * kTopK + q] = -1;  // an empty slot (or a bad id) has no row
+      continue;
+    }
     const int tl = q >> 3, w = tl >> 5;
     int rank = __popc(bm[e][w] & ((1u << (tl & 31)) - 1u));
     for (int v = 0; v < w; ++v) rank += __popc(bm[e][v]);
@@ -257,7 +267,10 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   for (int q = tid; q < nt * kTopK; q += blockDim.x) {
     const int e = idx[t0 * kTopK + q];
-    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) continue;
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(kE)) {
+      inv_perm[t0 * kTopK + q] = -1;  // an empty slot (or a bad id) has no row
+      continue;
+    }
     const int tl = q >> 3, w = tl >> 5;
     int rank = __popc(bm[e][w] & ((1u << (tl & 31)) - 1u));
     for (int v = 0; v < w; ++v) rank += __popc(bm[e][v]);

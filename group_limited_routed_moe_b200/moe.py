@@ -47,6 +47,7 @@ _SIGS = {
     "moe_last_error_string": ([], ctypes.c_char_p),
     "moe_get_device_status": ([_i32], _i32),
     "moe_init_device": ([], _i32),
+    "moe_set_ffn_trace": ([_p, _i64], _i32),
     "moe_set_wait_timeout_ns": ([_u64], _i32),
     "moe_selftest_wait_timeout": ([_p], _i32),
     "moe_packed_weight_bytes": ([], _sz),
@@ -77,6 +78,9 @@ _SIGS = {
     "moe_layer_shared_workspace_bytes": ([_i64, _i32, _i32], _sz),
     "moe_layer_shared": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_layer_shared_nvfp4": ([_p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_packed_experts_bytes": ([_i32], _sz),
+    "moe_pack_experts": ([_p, _p, _p, _i32, _p, _p], _i32),
+    "moe_expert_ffn_slice": ([_p, _p, _i32, _p, _p, _i64, _p, _p, _p], _i32),
     "moe_route_e256": ([_p, _p, _i64, _p, _p, _p], _i32),
     "moe_layer_e256_workspace_bytes": ([_i64, _i32], _sz),
     "moe_layer_e256": ([_p, _p, _p, _p, _p, _p, _i32, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
@@ -479,6 +483,35 @@ def moe_layer_nvfp4(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | 
 
 # ----------------------------------------------------------------- shared experts
 
+def moe_pack_experts(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                     packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Pack a slice of n experts ([n,1536,512], [n,1536,512], [n,512,1536] bf16),
+    renumbered 0..n-1 (see include/moe.h)."""
+    n = w_gate.shape[0]
+    for t, shp in ((w_gate, (n, HIDDEN, INTER)), (w_up, (n, HIDDEN, INTER)),
+                   (w_down, (n, INTER, HIDDEN))):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shp or not t.is_contiguous() \
+                or not t.is_cuda:
+            raise ValueError(f"expected contiguous CUDA bf16 {shp}")
+    nbytes = int(lib.moe_packed_experts_bytes(n))
+    if packed is None:
+        packed = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=w_gate.device)
+    _check("moe_pack_experts", lib.moe_pack_experts(_ptr(w_gate), _ptr(w_up), _ptr(w_down), n,
+                                                    _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_expert_ffn_slice(x: torch.Tensor, packed: torch.Tensor, n_experts: int,
+                         offsets: torch.Tensor, perm_src: torch.Tensor, h: torch.Tensor,
+                         y_perm: torch.Tensor, stream=None) -> torch.Tensor:
+    """moe_expert_ffn over a packed slice of n_experts experts (local ids)."""
+    _check("moe_expert_ffn_slice",
+           lib.moe_expert_ffn_slice(_ptr(x), _ptr(packed), n_experts, _ptr(offsets),
+                                    _ptr(perm_src), x.shape[0], _ptr(h), _ptr(y_perm),
+                                    _stream(stream)))
+    return y_perm
+
+
 def packed_shared_bytes(n_shared: int) -> int:
     return int(lib.moe_packed_shared_bytes(n_shared))
 
@@ -676,6 +709,18 @@ def init_device() -> None:
     """Per-device set-up of the library on the current device (do it before
     capturing library calls into a CUDA graph)."""
     _check("moe_init_device", lib.moe_init_device())
+
+
+def set_ffn_trace(buf: torch.Tensor | None) -> None:
+    """Per-CTA timing record of the expert-FFN launches into buf (int64 [n, 3]:
+    start ns, end ns, tiles), or off with None (see include/moe.h)."""
+    if buf is None:
+        _check("moe_set_ffn_trace", lib.moe_set_ffn_trace(None, 0))
+        return
+    if buf.dtype != torch.int64 or buf.dim() != 2 or buf.shape[1] != 3 or not buf.is_cuda \
+            or not buf.is_contiguous():
+        raise ValueError("expected a contiguous CUDA int64 tensor [n, 3]")
+    _check("moe_set_ffn_trace", lib.moe_set_ffn_trace(_ptr(buf), buf.shape[0]))
 
 
 def set_wait_timeout_ns(ns: int) -> None:

@@ -115,6 +115,21 @@ int moe_init_device(void);
  * Applies to launches issued after the call. */
 int moe_set_wait_timeout_ns(uint64_t ns);
 
+/* Diagnostics with no counterpart in the pages: a per-CTA timing record of
+ * the persistent expert-FFN launches, for measuring how evenly their tiles
+ * spread over the SMs (the tail of a grouped GEMM whose experts hold very
+ * different row counts).  While set, every expert-FFN launch of at most
+ * `capacity_ctas` CTAs writes, for CTA b:
+ *   buf[3b]     the device clock (%globaltimer, ns) when b started work, after
+ *               the preceding kernel's results became visible;
+ *   buf[3b + 1] the device clock when b had finished its last tile;
+ *   buf[3b + 2] the number of tiles b ran.
+ * Each launch overwrites the record of the one before (so the record is that
+ * of the last expert-FFN launch).  buf: device memory of 3 * capacity_ctas
+ * uint64 words, 8-byte aligned, caller-owned; NULL turns the record off (the
+ * default).  A launch with more CTAs than capacity_ctas records nothing. */
+int moe_set_ffn_trace(uint64_t* buf, int64_t capacity_ctas);
+
 /* Launches one block whose bounded wait on a barrier that nothing completes
  * must run out after the current limit: a self-test of the timeout path.  The
  * kernel returns normally and leaves the context usable; afterwards
@@ -170,14 +185,18 @@ size_t moe_permute_workspace_bytes(int64_t T);
  * expert, so that each expert runs on exactly the rows that picked it with no
  * host round trip (issue #1247, "What it does not cover", bullet on bf16
  * experts: the per-expert row loop there needs a host sync per layer).
- *   topk_idx : [T][8] int32 (from moe_route)
+ *   topk_idx : [T][8] int32 (from moe_route); an id of -1 marks an empty
+ *              slot, which gets no row (the expert-parallel receiver's rows
+ *              carry only the slots whose experts it owns)
  *   counts   : [128] int32 (out)  rows per expert
  *   offsets  : [MOE_OFFSETS_LEN] int32 (out): [0..128] exclusive prefix of counts,
- *              offsets[128] = 8T; [132..263] zeroed work counters that the
- *              expert-FFN kernels use and leave at zero (words 129..131 unused)
+ *              offsets[128] = the number of non-empty slots (8T when none is
+ *              empty); [132..263] zeroed work counters that the expert-FFN
+ *              kernels use and leave at zero (words 129..131 unused)
  *   perm_src : [8T] int32 (out)   permuted row r holds item t*8+slot; rows are
  *                                 expert-major, token-ascending inside an expert
  *   inv_perm : [8T] int32 (out)   item t*8+slot sits at row inv_perm[t*8+slot]
+ *                                 (-1 for an empty slot; moe_combine skips it)
  *   workspace: moe_permute_workspace_bytes(T) bytes (may be NULL when 0). */
 int moe_permute(const int32_t* topk_idx, int64_t T, int32_t* counts,
                 int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
@@ -472,6 +491,31 @@ int moe_layer_shared_nvfp4(const moe_bf16* x, const float* logits, const float* 
                            int64_t T, const moe_bf16* residual, moe_bf16* out,
                            int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                            size_t workspace_bytes, moe_stream_t stream);
+
+/* ---- a slice of a layer's experts (expert parallelism) --------------------- */
+
+/* With expert parallelism every rank holds only its own experts.  The pages put
+ * 128 experts in 8 groups of 16 and keep 4 groups per token ("Ling-3.0-tiny on
+ * a Qualcomm board", TensorFold issue #1247, first comment, opening
+ * paragraph), so with one or more whole groups per rank a token's rows go to
+ * at most 4 ranks.  These calls pack and run a contiguous slice of n_experts
+ * experts, renumbered 0 .. n_experts-1 (the rank's local ids).
+ *
+ * Bytes of a packed slice of n_experts experts (0 outside [1, 128]). */
+size_t moe_packed_experts_bytes(int n_experts);
+
+/* moe_pack_weights for a slice: w_gate, w_up [n][1536][512], w_down
+ * [n][512][1536] bf16 -> packed (moe_packed_experts_bytes(n) bytes, 128-byte
+ * aligned): the slice's gate/up blocks, then its W_down blocks in fp16, each
+ * in moe_pack_weights' per-expert layout. */
+int moe_pack_experts(const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                     int n_experts, moe_bf16* packed, moe_stream_t stream);
+
+/* moe_expert_ffn on a packed slice: offsets and perm_src from moe_permute of
+ * local ids (every id < n_experts, or -1 for an empty slot), T the rows of x. */
+int moe_expert_ffn_slice(const moe_bf16* x, const moe_bf16* packed, int n_experts,
+                         const int32_t* offsets, const int32_t* perm_src, int64_t T,
+                         moe_f16* h, moe_f16* y_perm, moe_stream_t stream);
 
 /* ---- second MoE shape: 256 experts, top-6 ------------------------------------- */
 
