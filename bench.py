@@ -733,7 +733,7 @@ def summary_of(line, main_name):
             "ffn_hbm_frac": k["expert_ffn"]["hbm_frac"],
             "ffn_tensor_frac": k["expert_ffn"]["tensor_frac"],
             "ffn_idle_sm_frac": k["expert_ffn"]["tail"]["idle_sm_frac"]}
-    for k in ("stack23_T1", "stack23_T8189"):
+    for k in ("stack23_T1", "stack23_T8189", "stack23_T1_routed", "stack23_T8189_routed"):
         if k in line:
             out[k] = {"us_per_layer": line[k]["us_per_layer"], "tok_s": line[k]["value"]}
     for k in ("decode_T16_e256", "decode_T16_shared1"):
@@ -857,12 +857,27 @@ def stack_packs(dev):
     return packs
 
 
-def stack_line(T, dev, packs, steps, warmup, peaks, barrier):
+def stack_routers(dev):
+    """The stack's 23 router matrices (seed 4, layers 0..22), packed."""
+    import torch
+    from group_limited_routed_moe_b200 import moe
+    out = []
+    for l in range(STACK_LAYERS):
+        bits = synth.router_weight_bits_np(STACK_SEED, l)
+        out.append(moe.moe_pack_router(
+            torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)))
+    return out
+
+
+def stack_line(T, dev, packs, steps, warmup, peaks, barrier, routers=None):
     """The 23-layer stack on T tokens: seeded router logits per layer, a bf16
     residual add between layers, the 23 moe_layer calls captured once as a CUDA
     graph and replayed (no host sync between layers).  Each replay streams every
     layer's touched experts, far more than L2 holds, so there is no flush; the
-    input is restored before each replay, outside the timed events."""
+    input is restored before each replay, outside the timed events.  With
+    `routers`, every layer is moe_layer_routed: its logits are projected from
+    its own input h by its own router matrix (activation-dependent routing),
+    and the seeded logits are not used."""
     import torch
     from group_limited_routed_moe_b200 import moe
     tok = synth.make_tokens(T, STACK_SEED)
@@ -881,8 +896,12 @@ def stack_line(T, dev, packs, steps, warmup, peaks, barrier):
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
             for l in range(STACK_LAYERS):
-                moe.moe_layer(h, lgs[l], bs[l], packs[l], residual=h, out=h, topk_idx_out=idx[l],
-                              workspace=ws, stream=s)
+                if routers is None:
+                    moe.moe_layer(h, lgs[l], bs[l], packs[l], residual=h, out=h,
+                                  topk_idx_out=idx[l], workspace=ws, stream=s)
+                else:
+                    moe.moe_layer_routed(h, routers[l], bs[l], packs[l], residual=h, out=h,
+                                         topk_idx_out=idx[l], workspace=ws, stream=s)
     torch.cuda.synchronize()
     cur = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -910,7 +929,15 @@ def stack_line(T, dev, packs, steps, warmup, peaks, barrier):
     flops = STACK_LAYERS * FLOPS_PER_ROW * 8 * T
     nb = (T + 127) // 128
     n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
+    if routers is not None:
+        nbytes += STACK_LAYERS * 1536 * 128 * 2  # the router matrices
+        flops += STACK_LAYERS * 2 * T * 1536 * 128
+        if T > 64:
+            n_rp += 1  # the tensor-core projection runs as its own launch above 64 tokens
     return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "routing": ("from each layer's own input (moe_layer_routed: router projection, "
+                        "routing and sort in one launch up to 64 tokens)" if routers is not None
+                        else "seeded per-layer logits (moe_layer)"),
             "layers": STACK_LAYERS, "T": T, "us_per_layer": round(ms * 1e3 / STACK_LAYERS, 2),
             "distinct_experts_all_layers": distinct,
             "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4),
@@ -1057,9 +1084,12 @@ def run_ours(args):
         line["gpu_launches"] += line["prefill_T2048_skewed"]["gpu_launches"]
     if not args.no_stack:
         packs = stack_packs(dev)
-        for T_s, key in ((1, "stack23_T1"), (8189, "stack23_T8189")):
+        routers = stack_routers(dev)
+        for T_s, key, rt in ((1, "stack23_T1", None), (8189, "stack23_T8189", None),
+                             (1, "stack23_T1_routed", routers),
+                             (8189, "stack23_T8189_routed", routers)):
             n = max(10, args.steps // 2) if T_s == 1 else max(5, args.steps // 10)
-            line[key] = stack_line(T_s, dev, packs, n, args.warmup, peaks, barrier)
+            line[key] = stack_line(T_s, dev, packs, n, args.warmup, peaks, barrier, routers=rt)
             line["gpu_launches"] += line[key]["gpu_launches"]
         del packs
     if args.e256_prefill:

@@ -25,6 +25,7 @@
 #include "route.cuh"
 #include "route_permute_small.cuh"
 #include "router.cuh"
+#include "router_small.cuh"
 
 using namespace moe;
 
@@ -274,6 +275,34 @@ int do_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, float
   return launch_pdl("router_kernel launch", router::router_kernel, dim3(grid),
                     dim3(router::THREADS), router::SMEM_BYTES, s, tw, tx, T, logits,
                     g_timeout_ns.load());
+}
+
+// Router projection + routing (+ the counting sort when counts != nullptr) in
+// one launch of one 8-CTA cluster, for T <= kFusedRoutePermMaxT.
+int do_router_route_small(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
+                          int64_t T, float* logits, int32_t* idx, float* w, int32_t* counts,
+                          int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
+                          cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rsmall::kCluster);
+  cfg.blockDim = dim3(rsmall::kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = rsmall::kCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, rsmall::router_route_permute_small_kernel,
+      reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<const __nv_bfloat16*>(packed_router),
+      bias, static_cast<int>(T), logits, idx, w, counts, offsets, perm_src, inv_perm);
+  if (e != cudaSuccess) return cuda_fail(e, "router_route_permute_small_kernel launch");
+  return MOE_OK;
 }
 
 // Steps 1 and 2 as moe_layer runs them: one fused block for a few tokens.
@@ -746,14 +775,20 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
   moe_bf16* h = reinterpret_cast<moe_bf16*>(ws + L.h);
   moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
 
-  if (packed_router != nullptr) {
-    float* lg = reinterpret_cast<float*>(ws + L.logits);
-    rc = do_router(x, packed_router, T, lg, sms, s);
-    logits = lg;
+  if (packed_router != nullptr && T <= kFusedRoutePermMaxT) {
+    // router projection, routing and the sort in one launch
+    rc = do_router_route_small(x, packed_router, bias, T, reinterpret_cast<float*>(ws + L.logits),
+                               idx, w, counts, offsets, perm_src, inv_perm, s);
+  } else {
+    if (packed_router != nullptr) {
+      float* lg = reinterpret_cast<float*>(ws + L.logits);
+      rc = do_router(x, packed_router, T, lg, sms, s);
+      logits = lg;
+    }
+    if (!rc)
+      rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
+                            ws + L.perm_ws, s);
   }
-  if (!rc)
-    rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
-                          ws + L.perm_ws, s);
   if (!rc) {
     if (quant && qfmt == 2)
       rc = do_expert_ffn_fp4(x, packed_q, offsets, perm_src, T, h, y,
@@ -818,6 +853,30 @@ int moe_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, floa
   rc = device_setup(nullptr, &sms);
   if (rc) return rc;
   return do_router(x, packed_router, T, logits, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_route_from_x(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
+                     int64_t T, float* logits, int32_t* topk_idx, float* topk_w,
+                     moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(x && packed_router && logits && topk_idx && topk_w, "null pointer");
+  REQUIRE(aligned(x, 128) && aligned(packed_router, 128),
+          "x and packed_router must be 128-byte aligned");
+  REQUIRE(aligned(logits, 16) && (!bias || aligned(bias, 16)) && aligned(topk_idx, 16) &&
+              aligned(topk_w, 16),
+          "pointers must be 16-byte aligned");
+  int sms = 0;
+  rc = device_setup(nullptr, &sms);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T <= kFusedRoutePermMaxT)
+    return do_router_route_small(x, packed_router, bias, T, logits, topk_idx, topk_w, nullptr,
+                                 nullptr, nullptr, nullptr, s);
+  rc = do_router(x, packed_router, T, logits, sms, s);
+  if (rc) return rc;
+  return do_route(logits, bias, T, topk_idx, topk_w, s);
 }
 
 // ---- block-FP8 experts ---------------------------------------------------------

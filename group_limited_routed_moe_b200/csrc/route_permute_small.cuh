@@ -25,12 +25,15 @@ constexpr int kFusedRoutePermMaxT = 64;
 constexpr int kFusedRoutePermThreads = 1024;
 
 // Routes one token with the whole warp.  Lane k < 8 receives the k-th selected
-// expert in sel and its combine weight in w (other lanes: sel = -1).
+// expert in sel and its combine weight in w (other lanes: sel = -1).  The
+// token's logits are read from global memory, or (ROW_SMEM) from shared memory.
+template <bool ROW_SMEM = false>
 __device__ __forceinline__ void route_token_warp(const float* __restrict__ row,
                                                  const float* __restrict__ bias, int lane,
                                                  int& sel, float& w) {
   const unsigned FULL = 0xFFFFFFFFu;
-  const float4 v = __ldg(reinterpret_cast<const float4*>(row) + lane);
+  const float4 v = ROW_SMEM ? reinterpret_cast<const float4*>(row)[lane]
+                            : __ldg(reinterpret_cast<const float4*>(row) + lane);
   const float4 b = bias != nullptr ? __ldg(reinterpret_cast<const float4*>(bias) + lane)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
   const float lg[4] = {v.x, v.y, v.z, v.w};
@@ -121,7 +124,8 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ row,
 
   // weights over lanes 0..7 (slots), in route_kernel's order: r / sum r with
   // r = sigmoid(l) / sigmoid(m), m the largest chosen logit
-  const double l = lane < kTopK ? static_cast<double>(__ldg(row + sel)) : 0.0;
+  const double l =
+      lane < kTopK ? static_cast<double>(ROW_SMEM ? row[sel] : __ldg(row + sel)) : 0.0;
   double m = l;
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) m = fmax(m, __shfl_xor_sync(FULL, m, off, 8));
@@ -131,6 +135,40 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ row,
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) tot += __shfl_xor_sync(FULL, tot, off, 8);
   w = static_cast<float>(r / tot);
+}
+
+// The counting sort of a block's T <= 64 tokens (ids in sidx, bm zeroed, the
+// caller's threads synchronised after writing sidx): counts, offsets (and the
+// zeroed GEMM counters), perm_src and inv_perm, stable in token order.
+__device__ __forceinline__ void sort_small_block(const int* sidx, int T, uint32_t (*bm)[2],
+                                                 int* cnt, int* off, int32_t* __restrict__ counts,
+                                                 int32_t* __restrict__ offsets,
+                                                 int32_t* __restrict__ perm_src,
+                                                 int32_t* __restrict__ inv_perm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = T * kTopK;
+  for (int p = tid; p < n; p += blockDim.x) {
+    const int e = sidx[p], t = p >> 3;
+    atomicOr(&bm[e][t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  if (tid < kE) cnt[tid] = __popc(bm[tid][0]) + __popc(bm[tid][1]);
+  __syncthreads();
+  if (warp == 0) scan_experts_warp0(cnt, off, lane);
+  __syncthreads();
+  if (tid < kE) {
+    counts[tid] = cnt[tid];
+    offsets[tid] = off[tid];
+  }
+  if (tid == 0) offsets[kE] = off[kE];
+  if (tid < kOffsetsLen - kSchedWord) offsets[kSchedWord + tid] = 0;  // GEMM tile counters
+  for (int p = tid; p < n; p += blockDim.x) {
+    const int e = sidx[p], t = p >> 3, wd = t >> 5;
+    const int r = off[e] + (wd ? __popc(bm[e][0]) : 0) +
+                  __popc(bm[e][wd] & ((1u << (t & 31)) - 1u));
+    perm_src[r] = p;
+    inv_perm[p] = r;
+  }
 }
 
 // T <= kFusedRoutePermMaxT tokens, one block of kFusedRoutePermThreads threads.
@@ -160,31 +198,8 @@ __global__ void __launch_bounds__(kFusedRoutePermThreads, 1)
     }
   }
   __syncthreads();
-
   // counting sort of the T*8 items by expert, stable in token order
-  const int n = T * kTopK;
-  for (int p = tid; p < n; p += blockDim.x) {
-    const int e = sidx[p], t = p >> 3;
-    atomicOr(&bm[e][t >> 5], 1u << (t & 31));
-  }
-  __syncthreads();
-  if (tid < kE) cnt[tid] = __popc(bm[tid][0]) + __popc(bm[tid][1]);
-  __syncthreads();
-  if (warp == 0) scan_experts_warp0(cnt, off, lane);
-  __syncthreads();
-  if (tid < kE) {
-    counts[tid] = cnt[tid];
-    offsets[tid] = off[tid];
-  }
-  if (tid == 0) offsets[kE] = off[kE];
-  if (tid < kOffsetsLen - kSchedWord) offsets[kSchedWord + tid] = 0;  // GEMM tile counters
-  for (int p = tid; p < n; p += blockDim.x) {
-    const int e = sidx[p], t = p >> 3, wd = t >> 5;
-    const int r = off[e] + (wd ? __popc(bm[e][0]) : 0) +
-                  __popc(bm[e][wd] & ((1u << (t & 31)) - 1u));
-    perm_src[r] = p;
-    inv_perm[p] = r;
-  }
+  sort_small_block(sidx, T, bm, cnt, off, counts, offsets, perm_src, inv_perm);
 }
 
 }  // namespace moe

@@ -65,6 +65,7 @@ _SIGS = {
     "moe_pack_router": ([_p, _p, _p], _i32),
     "moe_router": ([_p, _p, _i64, _p, _p], _i32),
     "moe_layer_routed": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "moe_route_from_x": ([_p, _p, _p, _i64, _p, _p, _p, _p], _i32),
     "moe_permute_fixed_scratch_max_tokens": ([], _i64),
     "moe_permute_fixed_scratch": ([_p, _i64, _p, _p, _p, _p, _p], _i32),
     "moe_packed_fp8_bytes": ([], _sz),
@@ -304,6 +305,24 @@ def moe_router(x: torch.Tensor, packed_router: torch.Tensor, logits=None, stream
     _check("moe_router", lib.moe_router(_ptr(x), _ptr(packed_router), T, _ptr(logits),
                                         _stream(stream)))
     return logits
+
+
+def moe_route_from_x(x: torch.Tensor, packed_router: torch.Tensor, bias: torch.Tensor | None,
+                     logits=None, topk_idx=None, topk_w=None, stream=None):
+    """Router projection and routing from x [T,1536] bf16: returns (logits [T,128]
+    fp32, topk_idx [T,8] int32, topk_w [T,8] fp32)."""
+    T = x.shape[0]
+    dev = x.device
+    if logits is None:
+        logits = torch.empty((T, N_EXPERTS), dtype=torch.float32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty((T, TOPK), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, TOPK), dtype=torch.float32, device=dev)
+    _check("moe_route_from_x", lib.moe_route_from_x(_ptr(x), _ptr(packed_router), _ptr(bias), T,
+                                                    _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                                                    _stream(stream)))
+    return logits, topk_idx, topk_w
 
 
 def moe_layer_routed(x: torch.Tensor, packed_router: torch.Tensor, bias: torch.Tensor | None,

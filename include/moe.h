@@ -266,6 +266,18 @@ int moe_pack_router(const moe_bf16* w_router, moe_bf16* packed_router, moe_strea
 int moe_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, float* logits,
                moe_stream_t stream);
 
+/* Router projection and routing from x: logits [T][128] fp32 (out), then
+ * moe_route on them (topk_idx, topk_w out).  Up to 64 tokens both run in one
+ * launch: a cluster of 8 CTAs, each computing 16 experts' logits for every
+ * token on the CUDA cores (one warp per dot product, in a fixed order) and
+ * storing them into the first CTA's shared memory, which then routes.  Above
+ * 64 tokens: moe_router (tensor cores), then moe_route.  The two projections
+ * sum in different orders; each is within the fp32 accumulation bound of the
+ * exact product. */
+int moe_route_from_x(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
+                     int64_t T, float* logits, int32_t* topk_idx, float* topk_w,
+                     moe_stream_t stream);
+
 /* ---- the fused layer ---------------------------------------------------- */
 
 /* Workspace bytes moe_layer needs for T tokens. */
@@ -283,9 +295,12 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias,
               moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
               void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* moe_layer with the router projection in front: the logits come from
- * moe_router(x, packed_router) into the workspace (same workspace size as
- * moe_layer), then route -> permute -> expert FFN -> combine as above. */
+/* moe_layer with the router projection in front: the logits are computed
+ * from x into the workspace (same workspace size as moe_layer), then route ->
+ * permute -> expert FFN -> combine as above.  Up to 64 tokens the projection,
+ * routing and the sort are one launch (as in moe_route_from_x), so the layer
+ * is three launches like moe_layer; above, moe_router's tensor-core
+ * projection runs first. */
 int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
                      const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
                      moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,

@@ -1,5 +1,10 @@
-"""GPU parity of the router projection (moe_router, moe_layer_routed) against
-the float64 oracle.
+"""GPU parity of the router projection (moe_router, moe_route_from_x,
+moe_layer_routed) against the float64 oracle.
+
+Two projections are checked: the tensor-core GEMM (moe_router, and the routed
+layer above 64 tokens) and the one-launch router + routing + sort of up to 64
+tokens (moe_route_from_x and the routed layer at decode), whose logits are
+CUDA-core dot products in another summation order.
 
 Logits are fp32 sums of 1536 exact bf16 x bf16 products, so they may differ
 from the float64 value by the accumulation rounding: at most K * 2**-23 *
@@ -68,7 +73,41 @@ def test_router_one_hot_rows_exact():
     assert np.array_equal(logits.double().cpu().numpy(), O.bf16_bits_to_f64(w_bits)[ks])
 
 
-@pytest.mark.parametrize("T", [16, 333, 2048])
+@pytest.mark.parametrize("T", [1, 4, 16, 63, 64, 65, 333])
+def test_route_from_x_parity(T):
+    """Logits within the accumulation bound of the float64 product, and the
+    routing equal, bit for bit, to moe_route on those same logits."""
+    moe = _moe()
+    w_bits, packed = _router(seed=2)
+    tok = synth.make_tokens(T, 70 + T)
+    x, _, bias = tokens_dev(tok)
+    lg, idx, w = moe.moe_route_from_x(x, packed, bias)
+    idx2, w2 = moe.moe_route(lg, bias)
+    torch.cuda.synchronize()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    got = lg.double().cpu().numpy()
+    ref = O.router_logits(tok.x_bits, w_bits)
+    assert np.all(np.abs(got - ref) <= _bound(tok.x_bits, w_bits))
+    assert O.rel_l2(got, ref) <= 1e-5
+    assert torch.equal(idx, idx2)
+    assert torch.equal(w.view(torch.int32), w2.view(torch.int32))
+
+
+def test_route_from_x_one_hot_rows_exact():
+    """The one-launch projection of x = e_k returns row k of W_router bit for
+    bit (one exact product per logit), for every token slot of a 48-token batch."""
+    moe = _moe()
+    w_bits, packed = _router(seed=1)
+    ks = [0, 1, 63, 64, 777, 1535, 8, 1000] * 6
+    x = np.zeros((len(ks), K), np.float32)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    lg, _, _ = moe.moe_route_from_x(to_dev_bf16(synth.f32_to_bf16_bits(x)), packed, None)
+    torch.cuda.synchronize()
+    assert np.array_equal(lg.double().cpu().numpy(), O.bf16_bits_to_f64(w_bits)[ks])
+
+
+@pytest.mark.parametrize("T", [1, 16, 64, 333, 2048])
 def test_layer_routed_equals_router_then_layer(T):
     moe = _moe()
     W = layer0_weights()
@@ -78,7 +117,7 @@ def test_layer_routed_equals_router_then_layer(T):
     idx1 = torch.empty((T, 8), dtype=torch.int32, device=DEV)
     w1 = torch.empty((T, 8), dtype=torch.float32, device=DEV)
     out1 = moe.moe_layer_routed(x, packed, bias, W.packed, topk_idx_out=idx1, topk_w_out=w1)
-    lg = moe.moe_router(x, packed)
+    lg, _, _ = moe.moe_route_from_x(x, packed, bias)  # the same projection as the layer's
     idx2 = torch.empty_like(idx1)
     w2 = torch.empty_like(w1)
     out2 = moe.moe_layer(x, lg, bias, W.packed, topk_idx_out=idx2, topk_w_out=w2)
@@ -89,7 +128,7 @@ def test_layer_routed_equals_router_then_layer(T):
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("T", [16, 2048])
+@pytest.mark.parametrize("T", [1, 16, 64, 2048])
 def test_layer_routed_against_oracle(T):
     """End to end from x: routing on the fp32 router logits against the
     oracle's routing on float64 logits, and the layer output on every token
@@ -108,7 +147,7 @@ def test_layer_routed_against_oracle(T):
     rr = O.route(lg_ref, tok.bias)
     # the logit error actually incurred (its size is checked against the
     # accumulation bound in test_router_logits_parity), with a margin of 4x
-    lg_gpu = moe.moe_router(x, packed).double().cpu().numpy()
+    lg_gpu = moe.moe_route_from_x(x, packed, bias)[0].double().cpu().numpy()
     err = np.abs(lg_gpu - lg_ref)
     assert np.all(err <= _bound(tok.x_bits, w_bits))
     delta = 4 * err.max(axis=1) + 1e-12  # per token, on any logit

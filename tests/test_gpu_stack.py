@@ -119,3 +119,64 @@ def test_stack_T8189_sampled(stack):
     _compare(to_host_bits(h[torch.as_tensor(rows, device=DEV)]), ref, x_bits[rows],
              f"T=8189, {len(rows)} sampled tokens")
     assert torch.all(h[T:] == 0)
+
+
+# ---------------------------------------------------------------- routed from activations
+
+@pytest.fixture(scope="module")
+def routers():
+    from group_limited_routed_moe_b200 import moe
+    return [moe.moe_pack_router(to_dev_bf16(synth.router_weight_bits_np(SEED, l)))
+            for l in range(N_LAYERS)]
+
+
+@pytest.mark.parametrize("T", [1, 64, 333])
+def test_routed_stack_graph_equals_eager(stack, routers, T):
+    """The 23-layer stack routed from its own activations (moe_layer_routed per
+    layer, logits projected from that layer's input) replayed from one CUDA
+    graph equals, bit for bit, the same 23 calls issued one by one, layer by
+    layer (every layer's routing and the final h).  Its first layer routes as a
+    single moe_layer_routed call on x, which tests/test_gpu_router.py checks
+    against the float64 oracle; the later layers' inputs come from the GPU, and
+    an oracle input never does, so those are checked for consistency here."""
+    from group_limited_routed_moe_b200 import moe
+    x_bits = synth.make_tokens(T, SEED + 100).x_bits
+    biases = [torch.from_numpy(synth.layer_logits(T, SEED, l)[1]).to(DEV) for l in range(N_LAYERS)]
+    x0 = to_dev_bf16(x_bits)
+    ws = moe.alloc_layer_workspace(T, DEV)
+
+    def run(h, idx, stream):
+        for l, W in enumerate(stack):
+            moe.moe_layer_routed(h, routers[l], biases[l], W.packed, residual=h, out=h,
+                                 topk_idx_out=idx[l], workspace=ws, stream=stream)
+
+    idx_e = [torch.empty((T, 8), dtype=torch.int32, device=DEV) for _ in range(N_LAYERS)]
+    h_e = x0.clone()
+    run(h_e, idx_e, torch.cuda.current_stream())
+    first_idx = torch.empty((T, 8), dtype=torch.int32, device=DEV)
+    moe.moe_layer_routed(x0, routers[0], biases[0], stack[0].packed, residual=x0,
+                         topk_idx_out=first_idx)
+    torch.cuda.synchronize()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+
+    idx_g = [torch.empty((T, 8), dtype=torch.int32, device=DEV) for _ in range(N_LAYERS)]
+    h_g = x0.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            run(h_g, idx_g, s)
+    h_g.copy_(x0)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    del g
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    for l in range(N_LAYERS):
+        assert torch.equal(idx_g[l], idx_e[l]), l
+    assert torch.equal(h_g.view(torch.int16), h_e.view(torch.int16))
+    assert torch.isfinite(h_g.float()).all()
+    # the stack's first layer routes as the single routed layer on x
+    assert torch.equal(idx_e[0], first_idx)
+    assert any(not torch.equal(idx_e[l], idx_e[l - 1]) for l in range(1, N_LAYERS))
