@@ -248,6 +248,38 @@ __device__ __forceinline__ void umma_f16_ta_k128(uint32_t d_tmem, uint32_t a_tme
       : "memory");
 }
 
+// Eight MMAs over K = 128 as umma_f16_ta_k128, with MMA k accumulating into
+// d[k % 4]: four independent accumulator chains, so that an MMA never waits for
+// the one issued just before it to finish with its accumulator (one chain of
+// dependent M = 128, N = 32 MMAs runs at about a quarter of the rate of four).
+// The first four accumulate only if `accumulate`, the other four always.
+__device__ __forceinline__ void umma_f16_ta_k128_4acc(uint32_t d0, uint32_t d1, uint32_t d2,
+                                                      uint32_t d3, uint32_t a_tmem, uint64_t b0,
+                                                      uint64_t b1, uint32_t idesc,
+                                                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
+      "setp.ne.b32 p, %8, 0;\n\t"
+      "setp.eq.b32 q, %8, %8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %5, %7, p;\n\t"
+      "add.u32 a, %4, 8;\n\tadd.u64 b, %5, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, p;\n\t"
+      "add.u32 a, %4, 16;\n\tadd.u64 b, %5, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [a], b, %7, p;\n\t"
+      "add.u32 a, %4, 24;\n\tadd.u64 b, %5, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%3], [a], b, %7, p;\n\t"
+      "add.u32 a, %4, 32;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %6, %7, q;\n\t"
+      "add.u32 a, %4, 40;\n\tadd.u64 b, %6, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, q;\n\t"
+      "add.u32 a, %4, 48;\n\tadd.u64 b, %6, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [a], b, %7, q;\n\t"
+      "add.u32 a, %4, 56;\n\tadd.u64 b, %6, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%3], [a], b, %7, q;\n\t}" ::"r"(d0),
+      "r"(d1), "r"(d2), "r"(d3), "r"(a_tmem), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(

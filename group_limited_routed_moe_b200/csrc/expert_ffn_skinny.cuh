@@ -32,7 +32,8 @@
 //
 // Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31), 4 token gather (phase 1:
 // cp.async of x rows by perm_src, barrier-tracked; padding rows kept at zero),
-// 5 TMA producer, 6 MMA issuer.  Accumulators: 2 x 32 TMEM columns.  Every
+// 5 TMA producer, 6 MMA issuer.  Accumulators: 2 buffers x 4 chains x 32 TMEM
+// columns (each tile's K steps go round-robin to 4 chains).  Every
 // wait, including the up -> gate hand-off, is a bounded mbarrier wait.
 //
 // Block-FP8 weights (WQ = true, MODE 3 only): the weight stream is 8-bit E4M3
@@ -73,12 +74,29 @@ constexpr int A_BYTES = BMW * BK * 2;  // 16 KB
 constexpr int B_BYTES = BNT * BK * 2;  // 4 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
-constexpr int TMEM_COLS = 2 * BNT;
+// Accumulator chains per tile: the tile's K steps (16 each) go round-robin to
+// NCH accumulators of BNT columns, summed in the epilogue as
+// (chain 0 + chain 1) + (chain 2 + chain 3).  One chain of dependent
+// M = 128, N = 32 MMAs waits for each MMA's accumulator before the next; four
+// independent chains keep four in flight, which is what sets the rate at
+// which one CTA streams a weight tile.
+constexpr int NCH = 4;
+constexpr int ACC_COLS = NCH * BNT;  // one accumulator buffer (all chains)
 constexpr int XSTRIDE = BNT + 1;  // floats per row of the up-value exchange tile
 constexpr int XCHG_BYTES = 64 * XSTRIDE * 4;
-constexpr int THREADS = 224;
-constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;
-constexpr int CONV_WARP0 = 7;  // block-FP8: converter warps 7 .. 7 + NCONV - 1
+// MMA-issuing warps.  One thread's tcgen05.mma instructions follow one
+// another at a few hundred cycles each (measured: about 170 cycles per
+// M = 128, N = 32 MMA from one thread; two warps issuing at once halve that per
+// MMA, four quarter it), and a weight tile's stages go through the MMAs one
+// after another, so a single issuing thread set how fast one CTA streams a
+// tile.  Issuer i issues the MMAs of the accumulator chains c with
+// c % NISS == i, for every stage; each commits to the stage's empty barrier
+// and to the tile's accumulator-full barrier, which count NISS arrivals.
+constexpr int NISS = 2;
+constexpr int THREADS = 32 * (6 + NISS);
+constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;  // issuers: warps 6 .. 6 + NISS - 1
+constexpr int CONV_WARP0 = 6 + NISS;  // quantised weights: converter warps from here
+static_assert(NCH % NISS == 0, "each accumulator chain belongs to one issuer");
 constexpr int kConvGroups = 2;  // block-FP8: converter warps per tensor-memory lane quarter
 
 // Ring geometry (WQ: 0 bf16, 1 block-FP8, 2 NVFP4 weights).  bf16 weights:
@@ -100,8 +118,8 @@ struct Ring {
   static constexpr int BYTES = RSTAGES * RSTAGE_BYTES;
   static constexpr int NA = WQ ? 4 : 0;
   static constexpr int A_COLS = KS / 2;  // 32-bit columns of one operand slot
-  static constexpr int A_COL0 = 2 * BNT;
-  static constexpr int TMEM_COLS = WQ ? 512 : 2 * BNT;
+  static constexpr int A_COL0 = 2 * ACC_COLS;             // after two accumulator buffers
+  static constexpr int TMEM_COLS = WQ ? 512 : 2 * ACC_COLS;
   static constexpr int NCONV = WQ ? 4 * kConvGroups : 0;
   static constexpr int THREADS = skinny::THREADS + 32 * NCONV;
 };
@@ -140,7 +158,7 @@ struct Tail {
   uint64_t apair[2];  // block-FP8: the operand slots of a pair of stages written
   uint64_t xfull;   // up half written to the exchange tile (64 lane arrivals)
   uint64_t xempty;  // gate half done reading it (64 lane arrivals)
-  uint64_t drain;
+  uint64_t drain[NISS];
   TileQueue tq;
   uint32_t tmem_base;
   int abort_flag;
@@ -219,19 +237,19 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < RST; ++s) {
       mbar_init(&fullb[s], HAS1 ? 1 + 32 : 1);  // TMA arrive (+ 32 gather lanes)
-      mbar_init(&emptyb[s], 1);                  // MMA commit
+      mbar_init(&emptyb[s], NISS);               // one MMA commit per issuer
     }
     // every converter warp arrives once per stage, two stages per pair
     for (int p = 0; p < 2; ++p) mbar_init(&S->apair[p], 2 * R::NCONV);
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&S->tfull[a], 1);
+      mbar_init(&S->tfull[a], NISS);
       mbar_init(&S->tempty[a], 4);
     }
     mbar_init(&S->xfull, 64);
     mbar_init(&S->xempty, 64);
-    mbar_init(&S->drain, 1);
+    for (int i = 0; i < NISS; ++i) mbar_init(&S->drain[i], 1);
     // gather warp, MMA thread, epilogue warps, converter warps
-    tileq_init(&S->tq, (HAS1 ? 1 : 0) + 1 + 4 + R::NCONV);
+    tileq_init(&S->tq, (HAS1 ? 1 : 0) + NISS + 4 + R::NCONV);
     S->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -372,8 +390,9 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
           mbar_wait(&fullb[i % RST], (i / RST) & 1, abort_flag, 10000000ull, kSiteFfnFull);
       }
     }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp >= MMA_WARP && warp < MMA_WARP + NISS) {
+    // ------------------------------------------------ MMA issuers
+    const int iss = warp - MMA_WARP;  // this thread issues chains iss, iss + NISS, ...
     if (lane == 0) {
       int it = 0, tc = 0;
       bool ok = true;
@@ -393,7 +412,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + a * BNT;
+        const uint32_t d = tmem_base + a * ACC_COLS;  // chain c at d + c * BNT
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % RST;
           const uint32_t ph = (it / RST) & 1;
@@ -414,8 +433,12 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
               tc_fence_after();
             }
             const int a = it % NA;
-            umma_f16_ta_k128(d, tmem_base + R::A_COL0 + R::A_COLS * a, bdesc,
-                             bdesc + (B_BYTES >> 4), idesc, kb != 0 ? 1u : 0u);
+            const uint32_t at = tmem_base + R::A_COL0 + R::A_COLS * a;
+#pragma unroll
+            for (int k = iss; k < 8; k += NISS) {  // K step k of the stage into chain k % 4
+              const uint64_t b = (k < 4 ? bdesc : bdesc + (B_BYTES >> 4)) + 2 * (k & 3);
+              umma_f16_ta(d + (k & 3) * BNT, at + 8 * k, b, idesc, (kb != 0 || k >= 4) ? 1u : 0u);
+            }
             // frees the ring stage and, for the converters, operand slot a
             umma_commit(&emptyb[s]);
           } else {
@@ -425,16 +448,17 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             }
             tc_fence_after();
             const uint64_t adesc = smem_desc_k128(smem_u32(sA(s)));
+            static_assert(BK / 16 == NCH, "one K step of a stage per accumulator chain");
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)
-              umma_f16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            for (int k = iss; k < BK / 16; k += NISS)
+              umma_f16(d + k * BNT, adesc + 2 * k, bdesc + 2 * k, idesc, kb != 0 ? 1u : 0u);
             umma_commit(&emptyb[s]);
           }
         }
         if (ok) umma_commit(&S->tfull[a]);
       }
-      umma_commit(&S->drain);
-      mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
+      umma_commit(&S->drain[iss]);
+      mbar_wait(&S->drain[iss], 0, abort_flag, 10000000ull, kSiteFfnDrain);
     }
   } else if (HAS1 && warp == GATHER_WARP) {
     // ------------------------------------------------ token gather (phase 1)
@@ -610,7 +634,17 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
       tc_fence_after();
       uint32_t v[32];
-      tmem_ld_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * BNT, v);
+      {  // (chain 0 + chain 1) + (chain 2 + chain 3)
+        const uint32_t acc = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * ACC_COLS;
+        uint32_t u[32], w2[32];
+        tmem_ld_2x32(acc, acc + BNT, v, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+        tmem_ld_2x32(acc + 2 * BNT, acc + 3 * BNT, u, w2);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          v[i] = __float_as_uint(__uint_as_float(v[i]) + (__uint_as_float(u[i]) + __uint_as_float(w2[i])));
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->tempty[a]);  // accumulator copied out: MMA may reuse it

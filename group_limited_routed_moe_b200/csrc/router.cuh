@@ -11,8 +11,8 @@
 // stores one token's 32 consecutive logits per instruction (128 contiguous
 // bytes).  T = 8189 gives 128 tiles, one per SM; T <= 64 is one tile, whose
 // token rows past T are zero-filled by the TMA.  Persistent CTAs walk the tiles
-// round-robin (all tiles cost the same).  Warp roles: 0-3 epilogue, 4 TMA, 5
-// MMA; 8 stages of (16 KB of W_router + 8 KB of x); 2 x 64 TMEM columns.
+// round-robin (all tiles cost the same).  Warp roles: 0-3 epilogue, 4 TMA, 5-6
+// MMA; 8 stages of (16 KB of W_router + 8 KB of x); 2 x 4 x 64 TMEM columns.
 // Every wait is a bounded mbarrier wait.
 #pragma once
 #include "common.cuh"
@@ -29,9 +29,19 @@ constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 8 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
-constexpr int TMEM_COLS = 2 * BN;
-constexpr int THREADS = 192;
-constexpr int TMA_WARP = 4, MMA_WARP = 5;
+// The 4 K steps of a stage go to 4 accumulator chains (summed in the
+// epilogue as (c0 + c1) + (c2 + c3)), so consecutive MMAs do not wait on each
+// other's accumulator: 2 buffers x 4 chains x 64 columns.
+constexpr int NCH = 4;
+constexpr int ACC_COLS = NCH * BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+// Two MMA-issuing warps: issuer i issues the stage's K steps of chains i and
+// i + 2 (one thread's tcgen05.mma instructions follow one another at a few
+// hundred cycles each, and a tile's 96 MMAs would otherwise run one by one).
+constexpr int NISS = 2;
+static_assert(NCH % NISS == 0, "each chain belongs to one issuer");
+constexpr int THREADS = 32 * (5 + NISS);
+constexpr int TMA_WARP = 4, MMA_WARP = 5;  // issuers: warps 5 .. 5 + NISS - 1
 constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kFmtBF16);
 
 struct Tail {
@@ -39,7 +49,7 @@ struct Tail {
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t drain;
+  uint64_t drain[NISS];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -76,13 +86,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&S->full[s], 1);
-      mbar_init(&S->empty[s], 1);
+      mbar_init(&S->empty[s], NISS);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&S->tfull[a], 1);
+      mbar_init(&S->tfull[a], NISS);
       mbar_init(&S->tempty[a], 4);
     }
-    mbar_init(&S->drain, 1);
+    for (int i = 0; i < NISS; ++i) mbar_init(&S->drain[i], 1);
     S->abort_flag = 0;
     fence_barrier_init();
   }
@@ -121,7 +131,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, abort_flag, 10000000ull, kSiteFfnFull);
       }
     }
-  } else if (warp == MMA_WARP) {
+  } else if (warp >= MMA_WARP && warp < MMA_WARP + NISS) {
+    const int iss = warp - MMA_WARP;
     if (lane == 0) {
       int it = 0, tc = 0;
       bool ok = true;
@@ -133,7 +144,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + a * BN;
+        const uint32_t d = tmem_base + a * ACC_COLS;  // chain k at d + k * BN
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -144,15 +155,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint64_t adesc = smem_desc_k128(smem_u32(sA(s)));
           const uint64_t bdesc = smem_desc_k128(smem_u32(sB(s)));
+          static_assert(BK / 16 == NCH, "one K step of a stage per chain");
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_f16(d, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+          for (int k = iss; k < BK / 16; k += NISS)
+            umma_f16(d + k * BN, adesc + 2 * k, bdesc + 2 * k, IDESC, kb != 0 ? 1u : 0u);
           umma_commit(&S->empty[s]);
         }
         if (ok) umma_commit(&S->tfull[a]);
       }
-      umma_commit(&S->drain);
-      mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
+      umma_commit(&S->drain[iss]);
+      mbar_wait(&S->drain[iss], 0, abort_flag, 10000000ull, kSiteFfnDrain);
     }
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue: lane = expert 32w + lane
@@ -166,8 +178,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       float* dst = logits + t0 * kE + warp * 32 + lane;
 #pragma unroll 1
       for (int h = 0; h < BN / 32; ++h) {
-        uint32_t v[32];
-        tmem_ld_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * BN + h * 32, v);
+        uint32_t v[32], u[32], w2[32];
+        const uint32_t acc =
+            tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * ACC_COLS + h * 32;
+        tmem_ld_2x32(acc, acc + BN, v, u);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = __float_as_uint(__uint_as_float(v[t]) + __uint_as_float(u[t]));
+        tmem_ld_2x32(acc + 2 * BN, acc + 3 * BN, u, w2);
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          v[t] = __float_as_uint(__uint_as_float(v[t]) + (__uint_as_float(u[t]) + __uint_as_float(w2[t])));
 #pragma unroll
         for (int t = 0; t < 32; ++t)
           if (t0 + h * 32 + t < T) dst[(h * 32 + t) * kE] = __uint_as_float(v[t]);
