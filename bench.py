@@ -20,7 +20,7 @@ the dominant kernel's roofline come from a second pass of K steps over the
 same batch through the five step calls, with events between them.  The
 decode batch is also timed as a replayed CUDA graph of the moe_layer call.
 The end-to-end figure (`e2e`) goes through the public host-buffer API
-(moe.HostPipeline over moe_layer_from_host): every step copies its own x and
+(moe.HostPipeline over the C ABI's moe_layer_host): every step copies its own x and
 router logits in and its output out, with two steps in flight on two streams
 so that copies and layers overlap.
 Multi-GPU (torchrun): every rank runs its own independent batch (data-parallel
@@ -1050,8 +1050,9 @@ def run_ours(args):
         "e2e": {"value": round(job_tokens_per_s(wl.T, world, e2e_ms), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "in_flight": 3,
-                "note": ("moe.HostPipeline: each step copies its inputs in and its output "
-                         "out; 3 steps in flight on 3 streams, their copies overlapping the "
+                "note": ("moe.HostPipeline over the C ABI's moe_layer_host: each step copies "
+                         "its inputs in and its output out (one cudaMemcpyAsync per buffer); "
+                         "3 steps in flight on 3 streams, their copies overlapping the "
                          "other step's layer, the layers one after another; no L2 flush "
                          "(each step streams the touched experts' weights, more than L2 holds)")},
         "gpu_launches": run.launches_per_step * args.steps,

@@ -278,7 +278,7 @@ int do_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, float
 }
 
 // Router projection + routing (+ the counting sort when counts != nullptr) in
-// one launch of one 8-CTA cluster, for T <= kFusedRoutePermMaxT.
+// one launch of one 8-CTA cluster, for T <= rsmall::kMaxT.
 int do_router_route_small(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
                           int64_t T, float* logits, int32_t* idx, float* w, int32_t* counts,
                           int32_t* offsets, int32_t* perm_src, int32_t* inv_perm,
@@ -286,7 +286,7 @@ int do_router_route_small(const moe_bf16* x, const moe_bf16* packed_router, cons
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rsmall::kCluster);
   cfg.blockDim = dim3(rsmall::kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = static_cast<size_t>(T) * kE * sizeof(float);
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -775,7 +775,7 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
   moe_bf16* h = reinterpret_cast<moe_bf16*>(ws + L.h);
   moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
 
-  if (packed_router != nullptr && T <= kFusedRoutePermMaxT) {
+  if (packed_router != nullptr && T <= rsmall::kMaxT) {
     // router projection, routing and the sort in one launch
     rc = do_router_route_small(x, packed_router, bias, T, reinterpret_cast<float*>(ws + L.logits),
                                idx, w, counts, offsets, perm_src, inv_perm, s);
@@ -828,6 +828,79 @@ int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const flo
                     out, topk_idx_out, topk_w_out, workspace, workspace_bytes, stream);
 }
 
+// ---- the layer from host buffers --------------------------------------------------
+namespace {
+struct HostWs {
+  size_t x, logits, out, layer, total;
+};
+HostWs host_ws(int64_t T, int fmt) {
+  HostWs H{};
+  size_t o = 0;
+  auto take = [&](size_t bytes, size_t align) {
+    o = align_up(o, align);
+    const size_t at = o;
+    o += bytes;
+    return at;
+  };
+  H.x = take(static_cast<size_t>(T) * kH * 2, 1024);
+  H.logits = take(static_cast<size_t>(T) * kE * 4, 1024);
+  H.out = take(static_cast<size_t>(T) * kH * 2, 1024);
+  H.layer = take(layer_ws(T, fmt != 0).total, 1024);
+  H.total = align_up(o, 1024);
+  return H;
+}
+}  // namespace
+
+size_t moe_layer_host_workspace_bytes(int64_t T, int weight_format) {
+  if (T < 0 || T > kMaxTokens || weight_format < 0 || weight_format > 2) return 0;
+  return host_ws(T, weight_format).total;
+}
+
+int moe_layer_host(const moe_bf16* x_host, const float* logits_host, const float* bias,
+                   const void* packed, int weight_format, int64_t T, moe_bf16* out_host,
+                   void* workspace, size_t workspace_bytes, void* wait_event, void* done_event,
+                   moe_stream_t stream) {
+  int rc = check_T(T);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE(weight_format >= 0 && weight_format <= 2, "weight_format=%d outside [0, 2]",
+          weight_format);
+  REQUIRE(x_host && logits_host && packed && out_host && workspace, "null pointer");
+  REQUIRE(aligned(workspace, 1024), "workspace must be 1024-byte aligned");
+  const HostWs H = host_ws(T, weight_format);
+  if (workspace_bytes < H.total)
+    return fail(MOE_ERR_WORKSPACE, "moe_layer_host workspace needs %zu bytes, got %zu", H.total,
+                workspace_bytes);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  auto* x = reinterpret_cast<moe_bf16*>(ws + H.x);
+  auto* lg = reinterpret_cast<float*>(ws + H.logits);
+  auto* out = reinterpret_cast<moe_bf16*>(ws + H.out);
+  // one copy per buffer; host memory should be page-locked for the copies to
+  // overlap other work
+  MOE_CUDA(cudaMemcpyAsync(x, x_host, static_cast<size_t>(T) * kH * 2, cudaMemcpyHostToDevice, s),
+           "cudaMemcpyAsync (x)");
+  MOE_CUDA(cudaMemcpyAsync(lg, logits_host, static_cast<size_t>(T) * kE * 4,
+                           cudaMemcpyHostToDevice, s),
+           "cudaMemcpyAsync (logits)");
+  if (wait_event != nullptr)
+    MOE_CUDA(cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(wait_event), 0), "cudaStreamWaitEvent");
+  const size_t lbytes = H.total - H.layer;
+  if (weight_format == 0)
+    rc = layer_impl("moe_layer_host", x, lg, nullptr, bias, static_cast<const moe_bf16*>(packed), T,
+                    nullptr, out, nullptr, nullptr, ws + H.layer, lbytes, stream);
+  else
+    rc = layer_impl("moe_layer_host", x, lg, nullptr, bias, nullptr, T, nullptr, out, nullptr,
+                    nullptr, ws + H.layer, lbytes, stream, packed, nullptr, 0, weight_format);
+  if (rc) return rc;
+  if (done_event != nullptr)
+    MOE_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(done_event), s), "cudaEventRecord");
+  MOE_CUDA(cudaMemcpyAsync(out_host, out, static_cast<size_t>(T) * kH * 2, cudaMemcpyDeviceToHost,
+                           s),
+           "cudaMemcpyAsync (out)");
+  return MOE_OK;
+}
+
 size_t moe_router_packed_bytes(void) { return static_cast<size_t>(kE) * kH * 2; }
 
 int moe_pack_router(const moe_bf16* w_router, moe_bf16* packed_router, moe_stream_t stream) {
@@ -871,7 +944,7 @@ int moe_route_from_x(const moe_bf16* x, const moe_bf16* packed_router, const flo
   rc = device_setup(nullptr, &sms);
   if (rc) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (T <= kFusedRoutePermMaxT)
+  if (T <= rsmall::kMaxT)
     return do_router_route_small(x, packed_router, bias, T, logits, topk_idx, topk_w, nullptr,
                                  nullptr, nullptr, nullptr, s);
   rc = do_router(x, packed_router, T, logits, sms, s);

@@ -1,6 +1,7 @@
 // router_small.cuh -- the router projection, routing and the counting sort in
-// one launch for small batches (T <= 64), so that a decode layer routed from
-// its own activations costs no launch more than one given its logits.
+// one launch for the smallest batches (T <= kRouterFusedMaxT), so that a
+// decode layer routed from its own activations costs no launch more than one
+// given its logits.
 //
 //   logits[t][e] = sum_k x[t][k] W_router[k][e]   (bf16 in, fp32 accumulate)
 // then steps 1 and 2 exactly as route_permute_small_kernel runs them.
@@ -34,7 +35,11 @@ constexpr int kCluster = 8;
 constexpr int kExpertsPerCta = kE / kCluster;  // 16
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxT = kFusedRoutePermMaxT;  // 64
+// Above this many tokens the CUDA-core dot products cost more than the
+// tensor-core router's launch (measured: the one-launch kernel takes 12.3 us
+// at T = 1, 22.6 us at T = 16 and 57 us at T = 64, against 13.4 + 12.3 us for
+// the router and routing kernels at any of them).
+constexpr int kMaxT = 8;
 constexpr int kChunks = kH * 2 / 16;        // 16-byte chunks per row: 192
 constexpr int kChunksPerLane = kChunks / 32;  // 6
 
@@ -66,7 +71,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int e0 = crank * kExpertsPerCta;
 
-  __shared__ __align__(16) float slog[kMaxT * kE];  // the leader's copy of all logits
+  // the leader's copy of all logits, T x 128 floats (dynamic: a few KB, so
+  // that the cluster's CTAs fit beside a resident expert-FFN CTA)
+  extern __shared__ __align__(16) float slog[];
   __shared__ int sidx[kMaxT * kTopK];
   __shared__ uint32_t bm[kE][2];
   __shared__ int cnt[kE];

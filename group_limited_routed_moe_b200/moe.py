@@ -62,6 +62,8 @@ _SIGS = {
     "moe_layer_workspace_bytes": ([_i64], _sz),
     "moe_layer": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
     "moe_router_packed_bytes": ([], _sz),
+    "moe_layer_host_workspace_bytes": ([_i64, _i32], _sz),
+    "moe_layer_host": ([_p, _p, _p, _p, _i32, _i64, _p, _p, _sz, _p, _p, _p], _i32),
     "moe_pack_router": ([_p, _p, _p], _i32),
     "moe_router": ([_p, _p, _i64, _p, _p], _i32),
     "moe_layer_routed": ([_p, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
@@ -631,26 +633,57 @@ def moe_layer_e256(x: torch.Tensor, logits: torch.Tensor, bias: torch.Tensor | N
     return out
 
 
-def moe_layer_from_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: torch.Tensor | None,
-                        packed_w: torch.Tensor, x_dev: torch.Tensor, logits_dev: torch.Tensor,
-                        out_dev: torch.Tensor, out_host: torch.Tensor,
-                        workspace: torch.Tensor, stream=None) -> torch.Tensor:
-    """End-to-end call from pinned host buffers: H2D copy of x and the router
-    logits, the layer, D2H copy of the output, all on one stream."""
-    s = stream if stream is not None else torch.cuda.current_stream()
-    with torch.cuda.stream(s):
-        x_dev.copy_(x_host, non_blocking=True)
-        logits_dev.copy_(logits_host, non_blocking=True)
-        moe_layer(x_dev, logits_dev, bias, packed_w, out=out_dev, workspace=workspace, stream=s)
-        out_host.copy_(out_dev, non_blocking=True)
+WEIGHT_FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2}
+
+
+def alloc_layer_host_workspace(T: int, device, weight_format: int = 0) -> torch.Tensor:
+    n = int(lib.moe_layer_host_workspace_bytes(T, weight_format))
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 1024
+    return raw[off:off + n]
+
+
+def _event(ev):
+    return None if ev is None else ctypes.c_void_p(ev.cuda_event)
+
+
+def moe_layer_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: torch.Tensor | None,
+                   packed: torch.Tensor, out_host: torch.Tensor, workspace: torch.Tensor,
+                   weight_format: int = 0, wait_event=None, done_event=None, stream=None):
+    """The layer from host buffers through the C ABI (moe_layer_host): x and
+    the router logits copied in, the layer, the output copied out, all on
+    `stream`.  wait_event / done_event: recorded torch.cuda.Event objects, or
+    None (see include/moe.h)."""
+    for t, shp, dt in ((x_host, (None, HIDDEN), torch.bfloat16), (logits_host, (None, N_EXPERTS),
+                       torch.float32), (out_host, (None, HIDDEN), torch.bfloat16)):
+        if t.is_cuda or t.dtype != dt or t.dim() != 2 or t.shape[1] != shp[1] \
+                or not t.is_contiguous():
+            raise ValueError("host buffers: contiguous CPU tensors of the layer's shapes")
+    T = x_host.shape[0]
+    _check("moe_layer_host",
+           lib.moe_layer_host(_ptr(x_host), _ptr(logits_host), _ptr(bias), _ptr(packed),
+                              weight_format, T, _ptr(out_host), _ptr(workspace),
+                              workspace.numel(), _event(wait_event), _event(done_event),
+                              _stream(stream)))
     return out_host
+
+
+def moe_layer_from_host(x_host: torch.Tensor, logits_host: torch.Tensor, bias: torch.Tensor | None,
+                        packed_w: torch.Tensor, out_host: torch.Tensor,
+                        workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """End-to-end call from pinned host buffers (bf16 experts): moe_layer_host
+    with a workspace from alloc_layer_host_workspace."""
+    return moe_layer_host(x_host, logits_host, bias, packed_w, out_host, workspace, 0,
+                          stream=stream)
 
 
 class HostPipeline:
     """Layer calls from pinned host buffers with `depth` calls in flight.
 
-    Each slot owns device buffers (x, logits, out, workspace) and a stream; call
-    k uses slot k % depth.  Its host-to-device copies may overlap the previous
+    Each slot owns a device workspace and a stream; call k uses slot k % depth
+    and goes through the C ABI's moe_layer_host (copies in, layer, copy out)
+    unless shared experts are given (their layer call has no host-buffer
+    form: then the copies are torch copies around moe_layer_shared).  Its host-to-device copies may overlap the previous
     call's layer, and its device-to-host copy the next call's layer, but the
     layers themselves run one after another (each waits for the previous
     call's layer), so two calls never share the weights they stream through
@@ -669,14 +702,19 @@ class HostPipeline:
         self.T, self.depth, self.k, self.shared = T, depth, 0, shared
         self.fp8, self.nvfp4 = fp8 or nvfp4, nvfp4
         self.last_layer = None
+        self.fmt = 2 if nvfp4 else 1 if fp8 else 0
         self.slots = []
         for _ in range(depth):
+            st = torch.cuda.Stream(device)
+            done = torch.cuda.Event()
+            done.record(st)  # creates the event before the library records it
             self.slots.append({
-                "stream": torch.cuda.Stream(device),
+                "stream": st, "done": done,
                 "x": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
                 "logits": torch.empty((T, N_EXPERTS), dtype=torch.float32, device=device),
                 "out": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=device),
-                "ws": self._workspace(T, device),
+                "ws": (self._workspace(T, device) if shared is not None else
+                       alloc_layer_host_workspace(T, device, self.fmt)),
             })
 
     def _workspace(self, T, device):
@@ -691,6 +729,11 @@ class HostPipeline:
         slot = self.slots[self.k % self.depth]
         self.k += 1
         st = slot["stream"]
+        if self.shared is None:
+            moe_layer_host(x_host, logits_host, bias, packed_w, out_host, slot["ws"], self.fmt,
+                           wait_event=self.last_layer, done_event=slot["done"], stream=st)
+            self.last_layer = slot["done"]
+            return out_host
         with torch.cuda.stream(st):
             slot["x"].copy_(x_host, non_blocking=True)
             slot["logits"].copy_(logits_host, non_blocking=True)

@@ -267,11 +267,11 @@ int moe_router(const moe_bf16* x, const moe_bf16* packed_router, int64_t T, floa
                moe_stream_t stream);
 
 /* Router projection and routing from x: logits [T][128] fp32 (out), then
- * moe_route on them (topk_idx, topk_w out).  Up to 64 tokens both run in one
+ * moe_route on them (topk_idx, topk_w out).  Up to 8 tokens both run in one
  * launch: a cluster of 8 CTAs, each computing 16 experts' logits for every
  * token on the CUDA cores (one warp per dot product, in a fixed order) and
  * storing them into the first CTA's shared memory, which then routes.  Above
- * 64 tokens: moe_router (tensor cores), then moe_route.  The two projections
+ * 8 tokens: moe_router (tensor cores), then moe_route.  The two projections
  * sum in different orders; each is within the fp32 accumulation bound of the
  * exact product. */
 int moe_route_from_x(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
@@ -297,7 +297,7 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias,
 
 /* moe_layer with the router projection in front: the logits are computed
  * from x into the workspace (same workspace size as moe_layer), then route ->
- * permute -> expert FFN -> combine as above.  Up to 64 tokens the projection,
+ * permute -> expert FFN -> combine as above.  Up to 8 tokens the projection,
  * routing and the sort are one launch (as in moe_route_from_x), so the layer
  * is three launches like moe_layer; above, moe_router's tensor-core
  * projection runs first. */
@@ -305,6 +305,37 @@ int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const flo
                      const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
                      moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
                      void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---- the layer from host buffers ---------------------------------------- */
+
+/* Workspace bytes of moe_layer_host (weight_format 0 bf16, 1 block FP8, 2
+ * NVFP4); 0 for an invalid argument. */
+size_t moe_layer_host_workspace_bytes(int64_t T, int weight_format);
+
+/* One layer from HOST buffers, the call a serving loop makes per batch: the
+ * token rows and their router logits are copied host -> device into the
+ * workspace, the layer runs on those copies (moe_layer, moe_layer_fp8 or
+ * moe_layer_nvfp4 by weight_format), and its output is copied device -> host,
+ * all asynchronously on `stream`, one cudaMemcpyAsync per buffer.
+ *   x_host      : [T][1536] bf16, host memory (page-locked for the copies to
+ *                 overlap other work)
+ *   logits_host : [T][128] fp32, host memory
+ *   bias        : [128] fp32 device memory, or NULL
+ *   packed      : the device-resident packed layer of that format
+ *   out_host    : [T][1536] bf16, host memory; complete once the stream has
+ *                 reached the end of the call (synchronise before reading)
+ *   workspace   : moe_layer_host_workspace_bytes(T, weight_format) bytes of
+ *                 device memory, 1024-byte aligned
+ *   wait_event  : NULL, or a cudaEvent_t the layer waits for after the input
+ *                 copies (so that calls on several streams can overlap one
+ *                 call's copies with another's layer while the layers
+ *                 themselves run one after another)
+ *   done_event  : NULL, or a cudaEvent_t recorded when the layer has finished
+ *                 (before the output copy) */
+int moe_layer_host(const moe_bf16* x_host, const float* logits_host, const float* bias,
+                   const void* packed, int weight_format, int64_t T, moe_bf16* out_host,
+                   void* workspace, size_t workspace_bytes, void* wait_event, void* done_event,
+                   moe_stream_t stream);
 
 /* ---- block-FP8 experts ---------------------------------------------------- */
 

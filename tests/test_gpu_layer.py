@@ -119,19 +119,41 @@ def test_layer_residual():
     assert np.all(np.abs(got - exact) <= ulp + 0.02 * np.sqrt(np.mean(upd ** 2)))
 
 
-def test_layer_from_host_e2e():
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4"])
+def test_layer_from_host_e2e(fmt):
+    """moe_layer_host (C ABI, host buffers in and out) against the oracle, and
+    bit for bit against the device-buffer layer call of the same format."""
     moe = _moe()
     W = layer0_weights()
-    tok = synth.make_tokens(16, 0)
+    T = 16
+    tok = synth.make_tokens(T, 0)
     x_h = torch.from_numpy(tok.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     lg_h = torch.from_numpy(tok.logits).pin_memory()
-    x_d = torch.empty((16, 1536), dtype=torch.bfloat16, device=DEV)
-    lg_d = torch.empty((16, 128), dtype=torch.float32, device=DEV)
-    out_d = torch.empty_like(x_d)
-    out_h = torch.empty((16, 1536), dtype=torch.bfloat16).pin_memory()
-    ws = moe.alloc_layer_workspace(16, DEV)
+    out_h = torch.full((T, 1536), float("nan"), dtype=torch.bfloat16).pin_memory()
     bias = torch.from_numpy(tok.bias).to(DEV)
-    moe.moe_layer_from_host(x_h, lg_h, bias, W.packed, x_d, lg_d, out_d, out_h, ws)
+    f = moe.WEIGHT_FORMATS[fmt]
+    if fmt == "bf16":
+        packed, layer = W.packed, moe.moe_layer
+    else:
+        qs = []
+        for which in (synth.W_GATE, synth.W_UP, synth.W_DOWN):
+            if fmt == "fp8":
+                q, sc = synth.fp8_weights_torch(0, 0, which, DEV, "pow2")
+                qs += [q, sc]
+            else:
+                qs += list(synth.nvfp4_weights_torch(0, 0, which, DEV, "pow2"))
+        packed = (moe.moe_pack_weights_fp8 if fmt == "fp8" else moe.moe_pack_weights_nvfp4)(*qs)
+        layer = moe.moe_layer_fp8 if fmt == "fp8" else moe.moe_layer_nvfp4
+        del qs
+    ws = moe.alloc_layer_host_workspace(T, DEV, f)
+    moe.moe_layer_host(x_h, lg_h, bias, packed, out_h, ws, f)
+    x_d, lg_d, _ = tokens_dev(tok)
+    direct = layer(x_d, lg_d, bias, packed)
+    torch.cuda.synchronize()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    assert torch.equal(out_h.view(torch.int16), direct.cpu().view(torch.int16))
+    if fmt != "bf16":
+        return  # the quantised layers' oracle parity is tested in their own files
     torch.cuda.synchronize()
     ref, _ = oracle_layer(tok, W)
     got = O.bf16_bits_to_f64(out_h.view(torch.int16).numpy().view(np.uint16))

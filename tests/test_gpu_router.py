@@ -2,7 +2,7 @@
 moe_layer_routed) against the float64 oracle.
 
 Two projections are checked: the tensor-core GEMM (moe_router, and the routed
-layer above 64 tokens) and the one-launch router + routing + sort of up to 64
+layer above 8 tokens) and the one-launch router + routing + sort of up to 8
 tokens (moe_route_from_x and the routed layer at decode), whose logits are
 CUDA-core dot products in another summation order.
 
@@ -73,7 +73,7 @@ def test_router_one_hot_rows_exact():
     assert np.array_equal(logits.double().cpu().numpy(), O.bf16_bits_to_f64(w_bits)[ks])
 
 
-@pytest.mark.parametrize("T", [1, 4, 16, 63, 64, 65, 333])
+@pytest.mark.parametrize("T", [1, 4, 7, 8, 9, 16, 64, 65, 333])
 def test_route_from_x_parity(T):
     """Logits within the accumulation bound of the float64 product, and the
     routing equal, bit for bit, to moe_route on those same logits."""
@@ -95,10 +95,10 @@ def test_route_from_x_parity(T):
 
 def test_route_from_x_one_hot_rows_exact():
     """The one-launch projection of x = e_k returns row k of W_router bit for
-    bit (one exact product per logit), for every token slot of a 48-token batch."""
+    bit (one exact product per logit), for every token slot of an 8-token batch."""
     moe = _moe()
     w_bits, packed = _router(seed=1)
-    ks = [0, 1, 63, 64, 777, 1535, 8, 1000] * 6
+    ks = [0, 1, 63, 64, 777, 1535, 8, 1000]
     x = np.zeros((len(ks), K), np.float32)
     for i, k in enumerate(ks):
         x[i, k] = 1.0
@@ -107,7 +107,7 @@ def test_route_from_x_one_hot_rows_exact():
     assert np.array_equal(lg.double().cpu().numpy(), O.bf16_bits_to_f64(w_bits)[ks])
 
 
-@pytest.mark.parametrize("T", [1, 16, 64, 333, 2048])
+@pytest.mark.parametrize("T", [1, 8, 16, 64, 333, 2048])
 def test_layer_routed_equals_router_then_layer(T):
     moe = _moe()
     W = layer0_weights()
@@ -128,7 +128,7 @@ def test_layer_routed_equals_router_then_layer(T):
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("T", [1, 16, 64, 2048])
+@pytest.mark.parametrize("T", [1, 8, 16, 2048])
 def test_layer_routed_against_oracle(T):
     """End to end from x: routing on the fp32 router logits against the
     oracle's routing on float64 logits, and the layer output on every token
