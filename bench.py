@@ -936,7 +936,7 @@ def stack_line(T, dev, packs, steps, warmup, peaks, barrier, routers=None):
             n_rp += 1  # the tensor-core projection runs as its own launch above 64 tokens
     return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "routing": ("from each layer's own input (moe_layer_routed: router projection, "
-                        "routing and sort in one launch up to 64 tokens)" if routers is not None
+                        "routing and sort in one launch up to 8 tokens)" if routers is not None
                         else "seeded per-layer logits (moe_layer)"),
             "layers": STACK_LAYERS, "T": T, "us_per_layer": round(ms * 1e3 / STACK_LAYERS, 2),
             "distinct_experts_all_layers": distinct,
