@@ -1046,7 +1046,8 @@ def run_ours(args):
         "roofline": roofline_for(wl, run, per, peaks, peak_kind),
         "router": router,
         "layer": dict(layer_fractions(wl, run, steps_ms, per, peaks),
-                      layer_us_after_write_only_flush=round(dirty_ms * 1e3, 2)),
+                      layer_us_after_write_only_flush=round(dirty_ms * 1e3, 2),
+                      ffn_tail=ffn_trace_run(run)),
         "e2e": {"value": round(job_tokens_per_s(wl.T, world, e2e_ms), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "in_flight": 3,
