@@ -110,6 +110,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits, on the way out of a kernel, for this thread's own asynchronous work
+// (a TMA copy it issued, or its MMAs through a commit) to land before the CTA
+// frees its shared or tensor memory.  Bounded (10 ms), and not cut short by
+// the CTA's abort flag, which is usually what sent the thread here.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, unsigned site) {
+  int no_abort = 0;
+  mbar_wait(bar, parity, &no_abort, 10000000ull, site);
+}
+
 // ---------------------------------------------------------------- cp.async
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {

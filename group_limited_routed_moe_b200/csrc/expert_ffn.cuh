@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
       if (!ok) {
         // let the copies already issued land before the block can exit
         for (int i = max(0, it - STAGES); i < it; ++i)
-          mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, abort_flag, 10000000ull, kSiteFfnFull);
+          mbar_wait_drain(&S->full[i % STAGES], (i / STAGES) & 1, kSiteFfnFull);
       }
     }
   } else if (warp == C::MMA_WARP) {
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
       }
       // every MMA this thread issued must be complete before TMEM is freed
       umma_commit(&S->drain);
-      mbar_wait(&S->drain, 0, abort_flag, 10000000ull, kSiteFfnDrain);
+      mbar_wait_drain(&S->drain, 0, kSiteFfnDrain);
     }
   } else if (C::HAS1 && warp >= C::GATHER_WARP0 && warp < C::GATHER_WARP0 + 8) {
     // ------------------------------------------------ A gather producers (gate/up tiles)

@@ -32,9 +32,10 @@
 //
 // Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31), 4 token gather (phase 1:
 // cp.async of x rows by perm_src, barrier-tracked; padding rows kept at zero),
-// 5 TMA producer, 6 MMA issuer.  Accumulators: 2 buffers x 4 chains x 32 TMEM
-// columns (each tile's K steps go round-robin to 4 chains).  Every
-// wait, including the up -> gate hand-off, is a bounded mbarrier wait.
+// 5 TMA producer, 6-7 MMA issuers.  Accumulators: 2 buffers x 2 chains x 32
+// TMEM columns (each tile's K steps go round-robin to the 2 chains, one per
+// issuer).  Every wait, including the up -> gate hand-off, is a bounded
+// mbarrier wait.
 //
 // Block-FP8 weights (WQ = true, MODE 3 only): the weight stream is 8-bit E4M3
 // codes, half the bytes.  A stage covers K = 128 (one scale block): the TMA
@@ -75,12 +76,11 @@ constexpr int B_BYTES = BNT * BK * 2;  // 4 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
 // Accumulator chains per tile: the tile's K steps (16 each) go round-robin to
-// NCH accumulators of BNT columns, summed in the epilogue as
-// (chain 0 + chain 1) + (chain 2 + chain 3).  One chain of dependent
-// M = 128, N = 32 MMAs waits for each MMA's accumulator before the next; four
-// independent chains keep four in flight, which is what sets the rate at
-// which one CTA streams a weight tile.
-constexpr int NCH = 4;
+// NCH accumulators of BNT columns, one per MMA-issuing warp, summed in the
+// epilogue as chain 0 + chain 1.  One thread's issue rate, not the
+// accumulator dependency, sets the pace (four chains, two per issuer,
+// measured no faster), and the epilogue reads half as many columns.
+constexpr int NCH = 2;
 constexpr int ACC_COLS = NCH * BNT;  // one accumulator buffer (all chains)
 constexpr int XSTRIDE = BNT + 1;  // floats per row of the up-value exchange tile
 constexpr int XCHG_BYTES = 64 * XSTRIDE * 4;
@@ -96,7 +96,7 @@ constexpr int NISS = 2;
 constexpr int THREADS = 32 * (6 + NISS);
 constexpr int GATHER_WARP = 4, TMA_WARP = 5, MMA_WARP = 6;  // issuers: warps 6 .. 6 + NISS - 1
 constexpr int CONV_WARP0 = 6 + NISS;  // quantised weights: converter warps from here
-static_assert(NCH % NISS == 0, "each accumulator chain belongs to one issuer");
+static_assert(NCH == NISS, "each issuer owns one accumulator chain");
 constexpr int kConvGroups = 2;  // block-FP8: converter warps per tensor-memory lane quarter
 
 // Ring geometry (WQ: 0 bf16, 1 block-FP8, 2 NVFP4 weights).  bf16 weights:
@@ -385,9 +385,9 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
         tile = next;
       }
       if (trace != nullptr) trace[3 * blockIdx.x + 2] = static_cast<uint64_t>(n - 1);  // tiles
-      if (!ok) {
+      if (!ok) {  // the loads already issued land before the CTA exits (bounded)
         for (int i = max(0, it - RST); i < it; ++i)
-          mbar_wait(&fullb[i % RST], (i / RST) & 1, abort_flag, 10000000ull, kSiteFfnFull);
+          mbar_wait_drain(&fullb[i % RST], (i / RST) & 1, kSiteFfnFull);
       }
     }
   } else if (warp >= MMA_WARP && warp < MMA_WARP + NISS) {
@@ -435,9 +435,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             const int a = it % NA;
             const uint32_t at = tmem_base + R::A_COL0 + R::A_COLS * a;
 #pragma unroll
-            for (int k = iss; k < 8; k += NISS) {  // K step k of the stage into chain k % 4
+            for (int k = iss; k < 8; k += NISS) {  // K step k of the stage into chain k % NCH
               const uint64_t b = (k < 4 ? bdesc : bdesc + (B_BYTES >> 4)) + 2 * (k & 3);
-              umma_f16_ta(d + (k & 3) * BNT, at + 8 * k, b, idesc, (kb != 0 || k >= 4) ? 1u : 0u);
+              umma_f16_ta(d + (k % NCH) * BNT, at + 8 * k, b, idesc,
+                          (kb != 0 || k >= NCH) ? 1u : 0u);
             }
             // frees the ring stage and, for the converters, operand slot a
             umma_commit(&emptyb[s]);
@@ -448,17 +449,17 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             }
             tc_fence_after();
             const uint64_t adesc = smem_desc_k128(smem_u32(sA(s)));
-            static_assert(BK / 16 == NCH, "one K step of a stage per accumulator chain");
 #pragma unroll
-            for (int k = iss; k < BK / 16; k += NISS)
-              umma_f16(d + k * BNT, adesc + 2 * k, bdesc + 2 * k, idesc, kb != 0 ? 1u : 0u);
+            for (int k = iss; k < BK / 16; k += NISS)  // K step k of the stage into chain k % NCH
+              umma_f16(d + (k % NCH) * BNT, adesc + 2 * k, bdesc + 2 * k, idesc,
+                       (kb != 0 || k >= NCH) ? 1u : 0u);
             umma_commit(&emptyb[s]);
           }
         }
         if (ok) umma_commit(&S->tfull[a]);
       }
       umma_commit(&S->drain[iss]);
-      mbar_wait(&S->drain[iss], 0, abort_flag, 10000000ull, kSiteFfnDrain);
+      mbar_wait_drain(&S->drain[iss], 0, kSiteFfnDrain);
     }
   } else if (HAS1 && warp == GATHER_WARP) {
     // ------------------------------------------------ token gather (phase 1)
@@ -634,16 +635,13 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
       tc_fence_after();
       uint32_t v[32];
-      {  // (chain 0 + chain 1) + (chain 2 + chain 3)
+      {  // chain 0 + chain 1
+        static_assert(NCH == 2, "the epilogue sums two chains");
         const uint32_t acc = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * ACC_COLS;
-        uint32_t u[32], w2[32];
+        uint32_t u[32];
         tmem_ld_2x32(acc, acc + BNT, v, u);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
-        tmem_ld_2x32(acc + 2 * BNT, acc + 3 * BNT, u, w2);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          v[i] = __float_as_uint(__uint_as_float(v[i]) + (__uint_as_float(u[i]) + __uint_as_float(w2[i])));
       }
       tc_fence_before();
       __syncwarp();

@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok) {
         for (int i = max(0, it - STAGES); i < it; ++i)
-          mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, abort_flag, 10000000ull, kSiteFfnFull);
+          mbar_wait_drain(&S->full[i % STAGES], (i / STAGES) & 1, kSiteFfnFull);
       }
     }
   } else if (warp >= MMA_WARP && warp < MMA_WARP + NISS) {
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ok) umma_commit(&S->tfull[a]);
       }
       umma_commit(&S->drain[iss]);
-      mbar_wait(&S->drain[iss], 0, abort_flag, 10000000ull, kSiteFfnDrain);
+      mbar_wait_drain(&S->drain[iss], 0, kSiteFfnDrain);
     }
   } else if (warp < 4) {
     // ------------------------------------------------ epilogue: lane = expert 32w + lane
