@@ -49,6 +49,34 @@ __device__ __forceinline__ unsigned long long route_key(double z) {
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
+// Order bits of an fp32 value: unsigned order equals the value order (for
+// non-NaN values; +0 and -0 differ, which the caller removes).
+__device__ __forceinline__ uint32_t ord32(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return (b >> 31) ? ~b : (b | 0x80000000u);
+}
+
+// route_key(z) for z = l + b (fp32 logit and bias), with the same order over
+// all keys, computed without float64 in the middle tier.  The exact sum is
+// the fp32 pair (s, e) of Knuth's two-sum: s = fl(l + b), e = (l + b) - s,
+// exact unless l + b overflows.  Rounding is monotone, so s1 < s2 implies
+// z1 < z2, and for s1 == s2 the order is e's: (s, e) ordered
+// lexicographically is z's order.  The middle tier's key is therefore s's
+// order bits over e's, after -0 is made +0 (z = -0 and z = +0 are one score).
+// The tiers use the float64 form, as does a NaN.  Middle keys lie between
+// ord32(-700) << 32 and ord32(10) << 32 | 0xFFFFFFFF, inside the middle tier's
+// range of route_key, so they sort against the tier keys as route_key's do.
+__device__ __forceinline__ unsigned long long route_key_lb(float l, float b) {
+  const float s = __fadd_rn(l, b);
+  const float bb = __fsub_rn(s, l);
+  const float e = __fadd_rn(__fsub_rn(l, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+  const bool top = s > 10.f || (s == 10.f && e > 0.f);     // z > 10
+  const bool low = s < -700.f || (s == -700.f && e < 0.f);  // z < -700
+  if (top || low || s != s) return route_key(static_cast<double>(l) + static_cast<double>(b));
+  return (static_cast<unsigned long long>(ord32(__fadd_rn(s, 0.f))) << 32) |
+         ord32(__fadd_rn(e, 0.f));
+}
+
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int64_t T,
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
@@ -84,21 +112,25 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   // keys, and the group's two best scores (found on the keys, evaluated in float64)
   unsigned long long key[16];
   unsigned long long k1 = 0ull, k2 = 0ull;
-  double z1 = 0.0, z2 = 0.0;
+  float l1 = 0.f, b1 = 0.f, l2 = 0.f, b2 = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const double z = static_cast<double>(lg[i]) + static_cast<double>(bs[i]);
-    key[i] = route_key(z);
+    key[i] = route_key_lb(lg[i], bs[i]);
     if (key[i] > k1) {
       k2 = k1;
-      z2 = z1;
+      l2 = l1;
+      b2 = b1;
       k1 = key[i];
-      z1 = z;
+      l1 = lg[i];
+      b1 = bs[i];
     } else if (key[i] > k2) {
       k2 = key[i];
-      z2 = z;
+      l2 = lg[i];
+      b2 = bs[i];
     }
   }
+  const double z1 = static_cast<double>(l1) + static_cast<double>(b1);
+  const double z2 = static_cast<double>(l2) + static_cast<double>(b2);
   const double gscore = sigmoid_f64(z1) + sigmoid_f64(z2);
 
   // rank of this group among the token's 8 (ties: lower index ranks first)

@@ -42,21 +42,25 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ row,
   // keys, and this lane's two best scores
   unsigned long long key[4];
   unsigned long long k1 = 0ull, k2 = 0ull;
-  double z1 = 0.0, z2 = 0.0;
+  float l1 = 0.f, b1 = 0.f, l2 = 0.f, b2 = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const double z = static_cast<double>(lg[i]) + static_cast<double>(bs[i]);
-    key[i] = route_key(z);
+    key[i] = route_key_lb(lg[i], bs[i]);
     if (key[i] > k1) {
       k2 = k1;
-      z2 = z1;
+      l2 = l1;
+      b2 = b1;
       k1 = key[i];
-      z1 = z;
+      l1 = lg[i];
+      b1 = bs[i];
     } else if (key[i] > k2) {
       k2 = key[i];
-      z2 = z;
+      l2 = lg[i];
+      b2 = bs[i];
     }
   }
+  double z1 = static_cast<double>(l1) + static_cast<double>(b1);
+  double z2 = static_cast<double>(l2) + static_cast<double>(b2);
   // the group's two best scores: merge the top-2 lists of its 4 lanes
 #pragma unroll
   for (int off = 1; off <= 2; off <<= 1) {
