@@ -56,25 +56,38 @@ __device__ __forceinline__ uint32_t ord32(float x) {
   return (b >> 31) ? ~b : (b | 0x80000000u);
 }
 
-// route_key(z) for z = l + b (fp32 logit and bias), with the same order over
-// all keys, computed without float64 in the middle tier.  The exact sum is
-// the fp32 pair (s, e) of Knuth's two-sum: s = fl(l + b), e = (l + b) - s,
-// exact unless l + b overflows.  Rounding is monotone, so s1 < s2 implies
-// z1 < z2, and for s1 == s2 the order is e's: (s, e) ordered
-// lexicographically is z's order.  The middle tier's key is therefore s's
-// order bits over e's, after -0 is made +0 (z = -0 and z = +0 are one score).
-// The tiers use the float64 form, as does a NaN.  Middle keys lie between
-// ord32(-700) << 32 and ord32(10) << 32 | 0xFFFFFFFF, inside the middle tier's
-// range of route_key, so they sort against the tier keys as route_key's do.
+// The middle tier's key of a float64 z in [-700, 10] as two fp32 words: the
+// pair (s, r) = (fl32(z), z - fl32(z)) represents z exactly (r is an fp32
+// value: see route_key_lb), and s ordered first, then r, is z's order.  -0 is
+// made +0 first (z = -0 and z = +0 are one score).  These keys lie between
+// ord32(-700) << 32 and ord32(10) << 32 | 0xFFFFFFFF, inside route_key's
+// middle range, so they sort against its tier keys as its own middle keys do.
+__device__ __forceinline__ unsigned long long middle_key(float s, float r) {
+  return (static_cast<unsigned long long>(ord32(__fadd_rn(s, 0.f))) << 32) |
+         ord32(__fadd_rn(r, 0.f));
+}
+
+// route_key for z = l + b, the float64 sum of an fp32 logit and bias, giving
+// every z the same order as route_key(z) without float64 arithmetic in the
+// usual case.  Knuth's two-sum gives s = fl32(l + b) and e = (l + b) - s, both
+// fp32 and exact.  When the exponents of s and e are less than 30 apart, l + b
+// has at most 53 significant bits, so the float64 sum is s + e exactly and
+// (s, e) is middle_key's pair.  Otherwise (a bias or logit more than 2^29
+// times smaller than the other) the float64 sum rounds, and the key is taken
+// from that sum: its pair (fl32(z), z - fl32(z)) is still exact, because z -
+// fl32(z) is then the smaller operand cut to the float64 grid, at most 24
+// significant bits.  The tiers (z > 10, z < -700) and a NaN take route_key.
 __device__ __forceinline__ unsigned long long route_key_lb(float l, float b) {
   const float s = __fadd_rn(l, b);
   const float bb = __fsub_rn(s, l);
   const float e = __fadd_rn(__fsub_rn(l, __fsub_rn(s, bb)), __fsub_rn(b, bb));
-  const bool top = s > 10.f || (s == 10.f && e > 0.f);     // z > 10
-  const bool low = s < -700.f || (s == -700.f && e < 0.f);  // z < -700
-  if (top || low || s != s) return route_key(static_cast<double>(l) + static_cast<double>(b));
-  return (static_cast<unsigned long long>(ord32(__fadd_rn(s, 0.f))) << 32) |
-         ord32(__fadd_rn(e, 0.f));
+  const int gap = static_cast<int>((__float_as_uint(s) >> 23) & 0xFFu) -
+                  static_cast<int>((__float_as_uint(e) >> 23) & 0xFFu);
+  if ((e == 0.f || gap < 30) && s > -700.f && s < 10.f) return middle_key(s, e);
+  const double z = static_cast<double>(l) + static_cast<double>(b);
+  if (!(z >= -700.0 && z <= 10.0)) return route_key(z);  // tiers and NaN
+  const float s64 = static_cast<float>(z);
+  return middle_key(s64, static_cast<float>(z - static_cast<double>(s64)));
 }
 
 __global__ void __launch_bounds__(kRouteWarps * 32)

@@ -85,6 +85,68 @@ def test_route_extreme_logits():
     _route_check(lg, b, exact_ties=True)
 
 
+def _key_boundary_rows():
+    """Logits and a bias that put scores on the edges of the routing keys: the
+    float64 sum z = logit + bias rounding away a tiny bias (a float64 tie the
+    exact sum would split), z = -0 against z = +0, z on either side of 10 and of
+    -700 (the saturation tiers) by less than an fp32 ulp of the logit, and a
+    bias 2^-40 times the logit that float64 still holds.  Other logits are -3
+    (or -800 where the row tests the low tier)."""
+    f = np.float32
+    lg = np.full((6, 128), -3.0, f)
+    b = np.zeros(128, f)
+    b[5] = f(1e-30)                 # row 0: z = 2 + 1e-30 rounds to 2 = z of expert 6
+    lg[0, [5, 6]] = 2.0
+    b[8] = f(-0.0)                  # row 1: z = -0 (expert 8) and +0 (expert 9) are one score
+    lg[1, 8], lg[1, 9] = f(-0.0), f(0.0)
+    b[16], b[18] = f(-2.0 ** -20), f(2.0 ** -20)   # row 2: z just below / above 10, and 10
+    lg[2, [16, 18, 19]] = 10.0
+    lg[2, 17] = np.nextafter(f(10.0), f(0.0))      # equal to expert 16's z
+    b[32], b[33] = f(1e-5), f(-1e-5)               # row 3: around -700 (33 drops to the low tier)
+    lg[3, :] = -800.0
+    lg[3, [32, 33, 34]] = -700.0
+    lg[3, 35] = np.nextafter(f(-700.0), f(0.0))
+    b[48] = f(2.0 ** -40)           # row 4: 0.5 + 2^-40 is exact in float64, above 0.5
+    lg[4, [48, 49]] = 0.5
+    lg[5, [5, 6, 8, 9, 48, 49]] = [2.0, 2.0, -0.0, 0.0, 0.5, 0.5]  # the same pairs together
+    return lg, b
+
+
+def test_route_key_boundaries():
+    """The routing keys order scores exactly as the oracle's float64 sums do
+    on the edges above, through moe_route and through the one-launch routing
+    and sort of a small layer (whose ids must match too)."""
+    moe = _moe()
+    lg, b = _key_boundary_rows()
+    gi, _, rr = _route_check(lg, b, exact_ties=True)
+    assert list(gi[0, :2]) == [5, 6] and list(gi[1, :2]) == [8, 9]
+    assert list(gi[2, :4]) == [18, 19, 16, 17] and list(gi[3, :4]) == [35, 32, 34, 33]
+    assert list(gi[4, :2]) == [48, 49]
+    W = layer0_weights()
+    tok = synth.make_tokens(lg.shape[0], 5)
+    x, _, _ = tokens_dev(tok)
+    idx = torch.empty((lg.shape[0], 8), dtype=torch.int32, device=DEV)
+    w = torch.empty((lg.shape[0], 8), dtype=torch.float32, device=DEV)
+    moe.moe_layer(x, torch.from_numpy(lg).to(DEV), torch.from_numpy(b).to(DEV), W.packed,
+                  topk_idx_out=idx, topk_w_out=w)
+    torch.cuda.synchronize()
+    assert moe.get_device_status(0) == moe.MOE_OK, moe.last_error()
+    assert np.array_equal(idx.cpu().numpy(), rr.topk_idx)
+    assert np.abs(w.cpu().numpy() - rr.topk_w).max() <= W_TOL
+
+
+def test_route_key_fp32_overflow():
+    """logit + bias above the fp32 range: the float64 sum decides (top tier)."""
+    f = np.float32
+    lg = np.full((2, 128), -3.0, f)
+    b = np.zeros(128, f)
+    b[70] = f(3e38)
+    lg[0, 70] = f(3e38)
+    lg[1, [70, 71]] = [f(-3e38), f(3e38)]   # z = 0 for expert 70, 3e38 for 71
+    gi, _, _ = _route_check(lg, b, exact_ties=True)
+    assert gi[0, 0] == 70 and gi[1, 0] == 71
+
+
 @pytest.mark.parametrize("T", [1, 4, 16, 1000, 1024, 1025, 2048, 8189])
 def test_permute_parity(T):
     moe = _moe()
