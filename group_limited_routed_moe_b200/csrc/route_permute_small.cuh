@@ -12,7 +12,7 @@
 // weights summed over slots in the same order), so the ids and weights equal
 // route_kernel's.  Only the work split differs: a whole warp per token, lane l
 // owning experts 4l..4l+3 (group l/4), so that each of the 8 selection rounds
-// is a 4-key scan and a 5-level shuffle reduction.  The sort is permute.cuh's
+// is a 4-key scan and three warp reductions (redux.sync).  The sort is permute.cuh's
 // bitmap counting sort with T <= 64 (two 32-token words per expert).
 #pragma once
 #include "common.cuh"
@@ -110,16 +110,14 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ row,
         bi = i;
       }
     }
-    int be = 4 * lane + bi;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const unsigned long long ok = __shfl_xor_sync(FULL, bk, off);
-      const int oe = __shfl_xor_sync(FULL, be, off);
-      if (ok > bk || (ok == bk && oe < be)) {
-        bk = ok;
-        be = oe;
-      }
-    }
+    // the warp's largest key, lowest expert id among equal keys: three
+    // warp reductions (high word, low word among the lanes holding the
+    // largest high word, expert id among the lanes holding the largest key)
+    const uint32_t hi = static_cast<uint32_t>(bk >> 32), lo = static_cast<uint32_t>(bk);
+    const uint32_t mh = __reduce_max_sync(FULL, hi);
+    const uint32_t ml = __reduce_max_sync(FULL, hi == mh ? lo : 0u);
+    const int be = static_cast<int>(__reduce_min_sync(
+        FULL, (hi == mh && lo == ml) ? static_cast<uint32_t>(4 * lane + bi) : 0xFFFFFFFFu));
     if (lane == k) sel = be;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
