@@ -230,9 +230,15 @@ int do_route(const float* logits, const float* bias, int64_t T, int32_t* idx, fl
                     dim3(kRouteWarps * 32), 0, s, logits, bias, T, idx, w);
 }
 
+// Tokens per block of the multi-block counting sort at T.
+int perm_block_tokens(int64_t T) {
+  return T <= kPermSmallBlocksMaxT ? kPermBlockTokensSmall : kPermBlockTokens;
+}
+
 size_t permute_ws_bytes(int64_t T) {
   if (T <= kPermSmallMaxT) return 0;
-  const int64_t nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  const int bt = perm_block_tokens(T);
+  const int64_t nb = (T + bt - 1) / bt;
   return align_up(static_cast<size_t>(nb) * kE * sizeof(int32_t), 256);
 }
 
@@ -242,16 +248,29 @@ int do_permute(const int32_t* idx, int64_t T, int32_t* counts, int32_t* offsets,
     return launch_pdl("permute_small_kernel launch", permute_small_kernel, dim3(1), dim3(1024), 0,
                       s, idx, static_cast<int>(T), counts, offsets, perm_src, inv_perm);
   }
-  const int64_t nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
   int32_t* hist = static_cast<int32_t*>(ws);
-  int rc = launch_pdl("permute_count_kernel launch", permute_count_kernel,
+  if (perm_block_tokens(T) == kPermBlockTokensSmall) {  // count, then the fused scan + scatter
+    constexpr int bt = kPermBlockTokensSmall;
+    const int64_t nb = (T + bt - 1) / bt;
+    static_assert((kPermSmallBlocksMaxT + bt - 1) / bt <= kPermFusedMaxBlocks,
+                  "64-token blocks only where the fused scan + scatter covers the batch");
+    int rc = launch_pdl("permute_count_kernel launch", permute_count_kernel<bt>,
+                        dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T, hist);
+    if (rc) return rc;
+    return launch_pdl("permute_scan_scatter_kernel launch", permute_scan_scatter_kernel<bt>,
+                      dim3(static_cast<unsigned>(nb)), dim3(kPermScanThreads), 0, s, idx, T,
+                      static_cast<const int32_t*>(hist), static_cast<int>(nb), counts, offsets,
+                      perm_src, inv_perm);
+  }
+  const int64_t nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  int rc = launch_pdl("permute_count_kernel launch", permute_count_kernel<kPermBlockTokens>,
                       dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T, hist);
   if (rc) return rc;
   if (nb <= kPermFusedMaxBlocks) {
-    return launch_pdl("permute_scan_scatter_kernel launch", permute_scan_scatter_kernel,
-                      dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, idx, T,
-                      static_cast<const int32_t*>(hist), static_cast<int>(nb), counts, offsets,
-                      perm_src, inv_perm);
+    return launch_pdl("permute_scan_scatter_kernel launch",
+                      permute_scan_scatter_kernel<kPermBlockTokens>, dim3(static_cast<unsigned>(nb)),
+                      dim3(kPermScanThreads), 0, s, idx, T, static_cast<const int32_t*>(hist),
+                      static_cast<int>(nb), counts, offsets, perm_src, inv_perm);
   }
   rc = launch_pdl("permute_scan_kernel launch", permute_scan_kernel, dim3(1), dim3(1024), 0, s,
                   hist, static_cast<int>(nb), counts, offsets);

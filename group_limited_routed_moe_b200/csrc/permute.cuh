@@ -22,7 +22,13 @@ constexpr int kPermSmallMaxT = 1024;   // single-block path up to this many toke
 // counted.  A token's slots may mix experts and empty slots; the expert-parallel
 // receiver uses it for the slots of a row whose expert lives on another rank.
 constexpr int kEmptySlot = -1;
-constexpr int kPermBlockTokens = 128;  // tokens per block on the multi-block path
+// Tokens per block on the multi-block path: 64 while the fused scan + scatter
+// covers the batch (up to kPermSmallBlocksMaxT tokens: twice the blocks in
+// flight as with 128, for latency-bound kernels), 128 above (fewer histogram
+// rows for the separate scan).
+constexpr int kPermBlockTokens = 128;
+constexpr int kPermBlockTokensSmall = 64;
+constexpr int64_t kPermSmallBlocksMaxT = 16384;
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
@@ -104,15 +110,16 @@ __global__ void __launch_bounds__(1024)
 
 // ---- multi-block path -----------------------------------------------------
 // (a) per-block expert histogram hist[b][e]
+template <int BT>
 __global__ void __launch_bounds__(256)
     permute_count_kernel(const int32_t* __restrict__ idx, int64_t T, int32_t* __restrict__ hist) {
   griddep_launch_dependents();
   griddep_wait();
-  __shared__ uint32_t bm[kE][kPermBlockTokens / 32];
+  __shared__ uint32_t bm[kE][BT / 32];
   const int tid = threadIdx.x;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPermBlockTokens;
-  const int nt = static_cast<int>((T - t0) < kPermBlockTokens ? (T - t0) : kPermBlockTokens);
-  for (int i = tid; i < kE * (kPermBlockTokens / 32); i += blockDim.x) (&bm[0][0])[i] = 0u;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BT;
+  const int nt = static_cast<int>((T - t0) < BT ? (T - t0) : BT);
+  for (int i = tid; i < kE * (BT / 32); i += blockDim.x) (&bm[0][0])[i] = 0u;
   __syncthreads();
   for (int q = tid; q < nt * kTopK; q += blockDim.x) {
     const int e = idx[t0 * kTopK + q];
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(256)
   if (tid < kE) {
     int c = 0;
 #pragma unroll
-    for (int w = 0; w < kPermBlockTokens / 32; ++w) c += __popc(bm[tid][w]);
+    for (int w = 0; w < BT / 32; ++w) c += __popc(bm[tid][w]);
     hist[static_cast<int64_t>(blockIdx.x) * kE + tid] = c;
   }
 }
@@ -172,32 +179,36 @@ __global__ void __launch_bounds__(1024)
 
 // (b') fused scan + scatter for up to kPermFusedMaxBlocks blocks: every block
 //      re-derives the expert offsets and its own bases from the histogram
-//      (nb x 128 reads per block), so no separate scan launch is needed.
+//      (nb x 128 reads per block, split over kPermScanParts threads per
+//      expert), so no separate scan launch is needed.
 constexpr int kPermFusedMaxBlocks = 256;
+constexpr int kPermScanParts = 4;
+constexpr int kPermScanThreads = kPermScanParts * kE;  // 512
 
-__global__ void __launch_bounds__(256)
+template <int BT>
+__global__ void __launch_bounds__(kPermScanThreads)
     permute_scan_scatter_kernel(const int32_t* __restrict__ idx, int64_t T,
                                 const int32_t* __restrict__ hist, int nb,
                                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                 int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm) {
   griddep_launch_dependents();
   griddep_wait();
-  constexpr int W = kPermBlockTokens / 32;
+  constexpr int W = BT / 32;
   __shared__ uint32_t bm[kE][W];
-  __shared__ int part[2][kE];
-  __shared__ int before_s[2][kE];
+  __shared__ int part[kPermScanParts][kE];
+  __shared__ int before_s[kPermScanParts][kE];
   __shared__ int cnt[kE];
   __shared__ int off[kE + 1];
   __shared__ int base[kE];
   const int tid = threadIdx.x, lane = tid & 31;
   const int b = blockIdx.x;
-  const int64_t t0 = static_cast<int64_t>(b) * kPermBlockTokens;
-  const int nt = static_cast<int>((T - t0) < kPermBlockTokens ? (T - t0) : kPermBlockTokens);
+  const int64_t t0 = static_cast<int64_t>(b) * BT;
+  const int nt = static_cast<int>((T - t0) < BT ? (T - t0) : BT);
   for (int i = tid; i < kE * W; i += blockDim.x) (&bm[0][0])[i] = 0u;
-  {  // column sums: thread (h, e) sums blocks h, h+2, h+4, ...
+  {  // column sums: thread (h, e) sums blocks h, h + kPermScanParts, ...
     const int e = tid & (kE - 1), h = tid >> 7;
     int tot = 0, bef = 0;
-    for (int bb = h; bb < nb; bb += 2) {
+    for (int bb = h; bb < nb; bb += kPermScanParts) {
       const int v = hist[static_cast<int64_t>(bb) * kE + e];
       tot += v;
       if (bb < b) bef += v;
@@ -206,11 +217,21 @@ __global__ void __launch_bounds__(256)
     before_s[h][e] = bef;
   }
   __syncthreads();
-  if (tid < kE) cnt[tid] = part[0][tid] + part[1][tid];
+  if (tid < kE) {
+    int c = 0;
+#pragma unroll
+    for (int h = 0; h < kPermScanParts; ++h) c += part[h][tid];
+    cnt[tid] = c;
+  }
   __syncthreads();
   if (tid < 32) scan_experts_warp0(cnt, off, lane);
   __syncthreads();
-  if (tid < kE) base[tid] = off[tid] + before_s[0][tid] + before_s[1][tid];
+  if (tid < kE) {
+    int bef = 0;
+#pragma unroll
+    for (int h = 0; h < kPermScanParts; ++h) bef += before_s[h][tid];
+    base[tid] = off[tid] + bef;
+  }
   if (b == 0) {
     if (tid < kE) {
       counts[tid] = cnt[tid];

@@ -85,8 +85,9 @@ def test_fixed_scratch_permute_matches_moe_permute(T, hot):
 
 @pytest.mark.gpu
 def test_fixed_scratch_permute_large_then_small():
-    """T = 65536 (512 blocks) fills every histogram row; T = 2000 (16 blocks,
-    the multi-block path) then runs on the same stream with rows 16..511 stale."""
+    """T = 65536 (512 blocks of 128 tokens) fills every histogram row; T = 2000
+    (32 blocks of 64 tokens, the multi-block path) then runs on the same stream
+    with rows 32..511 stale."""
     stream = torch.cuda.current_stream()
     for T, seed, hot in ((65536, 5, 0), (2000, 6, 16), (65536, 7, 8), (1100, 8, 0)):
         idx = _routing(T, seed, hot).cuda()
