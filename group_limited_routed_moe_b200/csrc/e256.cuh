@@ -24,21 +24,17 @@ constexpr int kPerLane = kE2 / 32;        // 8 experts per lane, 4 lanes per gro
 constexpr int kBlockTokens = 128;         // tokens per block of the counting sort
 constexpr int kRouteWarps2 = 8;           // tokens (warps) per route block
 
-// One warp per token.  Lane l owns experts 8l .. 8l+7 (group l / 4).
-__global__ void __launch_bounds__(kRouteWarps2 * 32)
-    route_e256_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                      int64_t T, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+// Routes one token with the whole warp.  Lane l owns experts 8l .. 8l+7
+// (group l / 4); lane k < 6 receives the k-th chosen expert in sel and its
+// combine weight in w (other lanes: sel = -1, w = 0).
+__device__ __forceinline__ void route_token_e256(const float* __restrict__ row,
+                                                 const float* __restrict__ bias, int lane,
+                                                 int& sel, float& w) {
   const unsigned FULL = 0xFFFFFFFFu;
-  griddep_launch_dependents();
-  griddep_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps2 + (threadIdx.x >> 5);
-  if (t >= T) return;  // whole warp
   const int grp = lane >> 2;
-
   float lg[kPerLane], bs[kPerLane];
   {
-    const float4* src = reinterpret_cast<const float4*>(logits + t * kE2 + kPerLane * lane);
+    const float4* src = reinterpret_cast<const float4*>(row + kPerLane * lane);
     const float4* bsrc = reinterpret_cast<const float4*>(bias + kPerLane * lane);
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -90,7 +86,7 @@ __global__ void __launch_bounds__(kRouteWarps2 * 32)
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) key[i] = 0ull;
   }
-  int sel = -1;  // lane k ends up holding the k-th chosen expert
+  sel = -1;  // lane k ends up holding the k-th chosen expert
 #pragma unroll 1
   for (int k = 0; k < kTopK2; ++k) {
     unsigned long long bk = key[0];
@@ -98,13 +94,13 @@ __global__ void __launch_bounds__(kRouteWarps2 * 32)
 #pragma unroll
     for (int i = 1; i < kPerLane; ++i)
       if (key[i] > bk) { bk = key[i]; bi = i; }  // strict: lower index on ties
-    int be = kPerLane * lane + bi;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const unsigned long long ok = __shfl_xor_sync(FULL, bk, off);
-      const int oe = __shfl_xor_sync(FULL, be, off);
-      if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
-    }
+    // the warp's largest key, lowest expert id among equal keys (three warp
+    // reductions, as in route_token_warp)
+    const uint32_t hi = static_cast<uint32_t>(bk >> 32), lo = static_cast<uint32_t>(bk);
+    const uint32_t mh = __reduce_max_sync(FULL, hi);
+    const uint32_t ml = __reduce_max_sync(FULL, hi == mh ? lo : 0u);
+    const int be = static_cast<int>(__reduce_min_sync(
+        FULL, (hi == mh && lo == ml) ? static_cast<uint32_t>(kPerLane * lane + bi) : 0xFFFFFFFFu));
     if (lane == k) sel = be;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i)
@@ -112,7 +108,7 @@ __global__ void __launch_bounds__(kRouteWarps2 * 32)
   }
   // combine weights over the 6 chosen, as route.cuh
   const bool mine = lane < kTopK2;
-  const double l = mine ? static_cast<double>(__ldg(logits + t * kE2 + sel)) : -INFINITY;
+  const double l = mine ? static_cast<double>(__ldg(row + sel)) : -INFINITY;
   double m = l;
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) m = fmax(m, __shfl_xor_sync(FULL, m, off));
@@ -122,9 +118,114 @@ __global__ void __launch_bounds__(kRouteWarps2 * 32)
   double tot = r;
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) tot += __shfl_xor_sync(FULL, tot, off);
-  if (mine) {
+  w = mine ? static_cast<float>(r / tot) : 0.f;
+}
+
+// One warp per token.
+__global__ void __launch_bounds__(kRouteWarps2 * 32)
+    route_e256_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                      int64_t T, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps2 + (threadIdx.x >> 5);
+  if (t >= T) return;  // whole warp
+  int sel;
+  float w;
+  route_token_e256(logits + t * kE2, bias, lane, sel, w);
+  if (lane < kTopK2) {
     topk_idx[t * kTopK2 + lane] = sel;
-    topk_w[t * kTopK2 + lane] = static_cast<float>(r / tot);
+    topk_w[t * kTopK2 + lane] = w;
+  }
+}
+
+// Writes the two halves' 264-word offsets arrays from the 257 expert offsets
+// (absolute rows; work counters zeroed).  Thread e < 256 of the block.
+__device__ __forceinline__ void write_halves(int e, const int* off, int32_t* __restrict__ off_lo,
+                                             int32_t* __restrict__ off_hi) {
+  const int half = e >> 7, j = e & 127;
+  int32_t* dst = half ? off_hi : off_lo;
+  dst[j] = off[e];
+  if (j == 127) dst[128] = off[e + 1];
+  for (int i = 129 + j; i < kOffsetsLen; i += 128) dst[i] = 0;
+}
+
+// Small batches (T <= kSmallMaxT): routing and the counting sort in one block,
+// as route_permute_small_kernel does for 128 experts.  Each warp routes a token
+// at a time; the block keeps every token's 6 expert ids in shared memory,
+// builds a 64-token bitmap per expert, counts, scans and scatters.  Outputs as
+// route_e256_kernel followed by the three counting-sort kernels.
+constexpr int kSmallMaxT = 64;
+constexpr int kSmallThreads = 512;
+__global__ void __launch_bounds__(kSmallThreads, 1)
+    route_sort_small_e256_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                 int T, int32_t* __restrict__ topk_idx,
+                                 float* __restrict__ topk_w, int32_t* __restrict__ counts,
+                                 int32_t* __restrict__ offsets, int32_t* __restrict__ off_lo,
+                                 int32_t* __restrict__ off_hi, int32_t* __restrict__ perm_src,
+                                 int32_t* __restrict__ inv_perm) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ int sidx[kSmallMaxT * kTopK2];
+  __shared__ uint32_t bm[kE2][2];  // bm[e][t / 32] bit t % 32: token t chose expert e
+  __shared__ int wsum[kE2 / 32];
+  __shared__ int off[kE2 + 1];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kE2 * 2; i += blockDim.x) (&bm[0][0])[i] = 0u;
+  for (int t = warp; t < T; t += kSmallThreads / 32) {
+    int sel;
+    float w;
+    route_token_e256(logits + static_cast<int64_t>(t) * kE2, bias, lane, sel, w);
+    if (lane < kTopK2) {
+      topk_idx[t * kTopK2 + lane] = sel;
+      topk_w[t * kTopK2 + lane] = w;
+      sidx[t * kTopK2 + lane] = sel;
+    }
+  }
+  __syncthreads();
+  for (int p = tid; p < T * kTopK2; p += blockDim.x) {
+    const int e = sidx[p], t = p / kTopK2;
+    atomicOr(&bm[e][t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  // counts and their exclusive scan over the 256 experts (threads 0..255)
+  int c = 0, incl = 0;
+  if (tid < kE2) {
+    c = __popc(bm[tid][0]) + __popc(bm[tid][1]);
+    incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+  }
+  __syncthreads();
+  if (tid < kE2) {
+    int base = 0;
+    for (int j = 0; j < warp; ++j) base += wsum[j];
+    off[tid] = base + incl - c;
+    if (tid == kE2 - 1) off[kE2] = base + incl;
+    counts[tid] = c;
+  }
+  __syncthreads();
+  if (tid < kE2) {
+    offsets[tid] = off[tid];
+    if (tid == kE2 - 1) offsets[kE2] = off[kE2];
+    write_halves(tid, off, off_lo, off_hi);
+  }
+  // rows: the 8-slot numbering t*8 + slot (slots 6 and 7 unused)
+  for (int p = tid; p < T * kTopK; p += blockDim.x) {
+    const int t = p >> 3, slot = p & 7;
+    if (slot >= kTopK2) {
+      inv_perm[p] = -1;
+      continue;
+    }
+    const int e = sidx[t * kTopK2 + slot], wd = t >> 5;
+    const int r = off[e] + (wd ? __popc(bm[e][0]) : 0) +
+                  __popc(bm[e][wd] & ((1u << (t & 31)) - 1u));
+    perm_src[r] = p;
+    inv_perm[p] = r;
   }
 }
 
@@ -184,7 +285,6 @@ __global__ void __launch_bounds__(256)
     run += v;
   }
   // halves: absolute rows, then zeroed work counters
-  __syncthreads();
   const int half = e >> 7, j = e & 127;
   int32_t* dst = half ? off_hi : off_lo;
   dst[j] = start;

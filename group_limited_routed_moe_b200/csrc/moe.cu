@@ -1334,18 +1334,25 @@ int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
   moe_bf16* y = reinterpret_cast<moe_bf16*>(ws + L.y);
   const int nb = static_cast<int>((T + e256::kBlockTokens - 1) / e256::kBlockTokens);
 
-  rc = do_route_e256(logits, bias, T, idx, w, s);
-  if (!rc)
-    rc = launch_pdl("count_e256_kernel launch", e256::count_e256_kernel, dim3(nb), dim3(256), 0,
-                    s, static_cast<const int32_t*>(idx), T, hist);
-  if (!rc)
-    rc = launch_pdl("scan_e256_kernel launch", e256::scan_e256_kernel, dim3(1), dim3(256), 0, s,
-                    hist, nb, reinterpret_cast<int32_t*>(ws + L.counts),
-                    reinterpret_cast<int32_t*>(ws + L.offsets), off_lo, off_hi);
-  if (!rc)
-    rc = launch_pdl("scatter_e256_kernel launch", e256::scatter_e256_kernel, dim3(nb), dim3(256),
-                    0, s, static_cast<const int32_t*>(idx), T, static_cast<const int32_t*>(hist),
-                    perm_src, inv_perm);
+  if (T <= e256::kSmallMaxT) {  // routing and the counting sort in one block
+    rc = launch_pdl("route_sort_small_e256_kernel launch", e256::route_sort_small_e256_kernel,
+                    dim3(1), dim3(e256::kSmallThreads), 0, s, logits, bias, static_cast<int>(T), idx,
+                    w, reinterpret_cast<int32_t*>(ws + L.counts),
+                    reinterpret_cast<int32_t*>(ws + L.offsets), off_lo, off_hi, perm_src, inv_perm);
+  } else {
+    rc = do_route_e256(logits, bias, T, idx, w, s);
+    if (!rc)
+      rc = launch_pdl("count_e256_kernel launch", e256::count_e256_kernel, dim3(nb), dim3(256), 0,
+                      s, static_cast<const int32_t*>(idx), T, hist);
+    if (!rc)
+      rc = launch_pdl("scan_e256_kernel launch", e256::scan_e256_kernel, dim3(1), dim3(256), 0, s,
+                      hist, nb, reinterpret_cast<int32_t*>(ws + L.counts),
+                      reinterpret_cast<int32_t*>(ws + L.offsets), off_lo, off_hi);
+    if (!rc)
+      rc = launch_pdl("scatter_e256_kernel launch", e256::scatter_e256_kernel, dim3(nb), dim3(256),
+                      0, s, static_cast<const int32_t*>(idx), T, static_cast<const int32_t*>(hist),
+                      perm_src, inv_perm);
+  }
   // experts 0..127 and 128..255: the 128-expert kernels on each half's pack
   if (!rc) rc = do_expert_ffn(x, packed_lo, off_lo, perm_src, T, h, y, sms, s);
   if (!rc) rc = do_expert_ffn(x, packed_hi, off_hi, perm_src, T, h, y, sms, s);

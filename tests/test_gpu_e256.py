@@ -100,6 +100,45 @@ def test_route_e256_ties():
     assert np.abs(w.cpu().numpy() - rr.topk_w).max() <= W_TOL
 
 
+@pytest.mark.parametrize("T", [1, 7, 16, 33, 64, 65])
+def test_layer_e256_small_routing_equals_route_kernel(T):
+    """Up to 64 tokens the layer routes and sorts in one block
+    (route_sort_small_e256_kernel); its ids and weights must be the routing
+    kernel's bit for bit (65 takes the multi-block path)."""
+    moe = _moe()
+    W = weights()
+    tok = synth.make_tokens_e256(T, 40 + T)
+    x, lg, bias = _dev(tok)
+    idx = torch.empty((T, 6), dtype=torch.int32, device=DEV)
+    wts = torch.empty((T, 6), dtype=torch.float32, device=DEV)
+    moe.moe_layer_e256(x, lg, bias, W.packed[0], W.packed[1], None, 0, topk_idx_out=idx,
+                       topk_w_out=wts)
+    idx2, w2 = moe.moe_route_e256(lg, bias)
+    torch.cuda.synchronize()
+    _status_ok()
+    assert torch.equal(idx, idx2)
+    assert torch.equal(wts.view(torch.int32), w2.view(torch.int32))
+
+
+def test_layer_e256_small_routing_ties():
+    """The tie rows of test_route_e256_ties through the one-block routing."""
+    moe = _moe()
+    W = weights()
+    lg = np.zeros((3, 256), np.float32)
+    lg[1, ::32] = 60.0
+    lg[2, 200:206] = 40.0
+    x = to_dev_bf16(synth.make_tokens_e256(3, 5).x_bits)
+    idx = torch.empty((3, 6), dtype=torch.int32, device=DEV)
+    wts = torch.empty((3, 6), dtype=torch.float32, device=DEV)
+    moe.moe_layer_e256(x, torch.from_numpy(lg).to(DEV), None, W.packed[0], W.packed[1], None, 0,
+                       topk_idx_out=idx, topk_w_out=wts)
+    torch.cuda.synchronize()
+    _status_ok()
+    rr = O.route_e256(lg, None)
+    assert np.array_equal(idx.cpu().numpy(), rr.topk_idx)
+    assert np.abs(wts.cpu().numpy() - rr.topk_w).max() <= W_TOL
+
+
 @pytest.mark.parametrize("T,n_shared", [(1, 2), (16, 2), (64, 0), (300, 2), (2048, 2)])
 def test_layer_e256_against_oracle(T, n_shared):
     moe = _moe()
