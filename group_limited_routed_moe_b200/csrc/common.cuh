@@ -474,14 +474,17 @@ __device__ __forceinline__ int tileq_peek(TileQueue* q, int n) {
 
 // End of a launch: the last CTA to finish zeroes the two counter words (and
 // the n_extra words at `extra`, if any).
-__device__ __forceinline__ void tileq_retire(int* sched, int* extra = nullptr, int n_extra = 0) {
+// Returns true in the CTA that retired last (the one that reset the words).
+__device__ __forceinline__ bool tileq_retire(int* sched, int* extra = nullptr, int n_extra = 0) {
   __threadfence();
   const int fin = atomicAdd(sched + 1, 1);
   if (fin == static_cast<int>(gridDim.x) - 1) {
     atomicExch(sched, 0);
     atomicExch(sched + 1, 0);
     for (int i = 0; i < n_extra; ++i) atomicExch(extra + i, 0);
+    return true;
   }
+  return false;
 }
 
 constexpr int kDoneWord = kSchedWord + 4;  // offsets[136 .. 263]: per-expert done counters

@@ -150,6 +150,26 @@ constexpr uint32_t kIdesc2 = idesc_f32acc(BMW, BNT, kFmtF16);
 // storing warp): a down tile of expert e waits for kDoneStep * 8 * chunks(e).
 constexpr int kDoneStep = 2;
 
+// Weight packs of one launch ("segments"): up to kMaxSeg packs of up to 128
+// experts each, every one with its own offsets array (the down tiles' done
+// counters live in it), row sources and h / y_perm rows.  The 256-expert shape
+// runs its two halves and its shared experts as three segments of one launch;
+// every other call is one segment.  Tile ids run over all segments' gate/up
+// tiles, then all segments' down tiles.
+constexpr int kMaxSeg = 3;
+struct SegMaps {
+  CUtensorMap w1[kMaxSeg];  // gate/up weights (phase 1)
+  CUtensorMap w2[kMaxSeg];  // down weights (phase 2)
+  CUtensorMap h[kMaxSeg];   // h rows (phase 2)
+};
+struct SegPtrs {
+  int n;                             // segments in the launch, 1 .. kMaxSeg
+  const int32_t* offsets[kMaxSeg];   // offsets array (129 offsets, then the work counters)
+  const int32_t* perm_src[kMaxSeg];  // row sources (8t + slot)
+  uint16_t* h_out[kMaxSeg];
+  uint16_t* y_out[kMaxSeg];
+};
+
 struct Tail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
@@ -163,24 +183,30 @@ struct Tail {
   uint32_t tmem_base;
   int abort_flag;
   int wsum[4];
-  int cstart[kE + 1];  // exclusive prefix of the experts' 32-token chunk counts
-  int cnt[kE];
-  int off[kE];
+  int segbase[kMaxSeg + 1];       // exclusive prefix of the segments' chunk counts
+  int cstart[kMaxSeg][kE + 1];    // per segment: exclusive prefix of the experts' 32-token chunks
+  int cnt[kMaxSeg][kE];
+  int off[kMaxSeg][kE];
 };
 constexpr int TAIL_BYTES = (static_cast<int>(sizeof(Tail)) + 127) / 128 * 128;
 constexpr int SMEM_BYTES = TILE_BYTES + TAIL_BYTES + XCHG_BYTES + 1024;
 
-// Tile u of a phase whose experts have FBLK weight blocks per chunk.
-__device__ __forceinline__ void decode_tile(const Tail* S, int u, int FBLK, int& e, int& f,
-                                            int& c) {
+// Tile u of a phase whose experts have FBLK weight blocks per chunk, over all
+// segments: segment g, expert e, weight block f, chunk c.
+__device__ __forceinline__ void decode_tile(const Tail* S, int nseg, int u, int FBLK, int& g,
+                                            int& e, int& f, int& c) {
+  g = 0;
+  while (g + 1 < nseg && S->segbase[g + 1] * FBLK <= u) ++g;
+  u -= S->segbase[g] * FBLK;
+  const int* cs = S->cstart[g];
   int lo = 0, hi = kE - 1;  // largest e with cstart[e] * FBLK <= u
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (S->cstart[mid] * FBLK <= u) lo = mid; else hi = mid - 1;
+    if (cs[mid] * FBLK <= u) lo = mid; else hi = mid - 1;
   }
   e = lo;
-  const int rem = u - S->cstart[e] * FBLK;
-  const int nch = (S->cnt[e] + BNT - 1) / BNT;
+  const int rem = u - cs[e] * FBLK;
+  const int nch = (S->cnt[g][e] + BNT - 1) / BNT;
   f = rem / nch;
   c = rem - f * nch;
 }
@@ -188,30 +214,28 @@ __device__ __forceinline__ void decode_tile(const Tail* S, int u, int FBLK, int&
 // Phase and coordinates of tile id `tile` of a launch in mode MODE (1: gate/up,
 // 2: down, 3: both, gate/up tile ids first).
 struct TileInfo {
-  int phase, e, f, c;
+  int phase, g, e, f, c;
 };
 template <int MODE>
-__device__ __forceinline__ TileInfo tile_info(const Tail* S, int tile, int total1) {
+__device__ __forceinline__ TileInfo tile_info(const Tail* S, int nseg, int tile, int total1) {
   TileInfo t;
   t.phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
   const int u = (MODE == 3 && t.phase == 2) ? tile - total1 : tile;
-  decode_tile(S, u, fblk(t.phase), t.e, t.f, t.c);
+  decode_tile(S, nseg, u, fblk(t.phase), t.g, t.e, t.f, t.c);
   return t;
 }
 
 template <int MODE, int WQ = 0>
 __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
-    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w1,  // gate/up weights (phase 1)
-                       const __grid_constant__ CUtensorMap tmap_w2,  // down weights (phase 2)
-                       const __grid_constant__ CUtensorMap tmap_h,   // h rows (phase 2)
-                       const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
-                       const int32_t* __restrict__ perm_src, int64_t T,
-                       uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
-                       int* __restrict__ sched, int* __restrict__ done,
+    skinny_gemm_kernel(const __grid_constant__ SegMaps maps, const __grid_constant__ SegPtrs seg,
+                       const __nv_bfloat16* __restrict__ x, int64_t T, int* __restrict__ sched,
                        const void* __restrict__ wscale,  // FP8 scales (SGU, SD) or FP4 MGU, MD
                        uint64_t timeout_ns,
                        uint64_t* __restrict__ trace) {  // NULL, or 3 words per CTA (see ffn_trace)
   constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
+  const int nseg = seg.n;
+  // segment g's per-expert done counters (single-launch form only)
+  auto done_of = [&](int g) { return const_cast<int*>(seg.offsets[g]) + kDoneWord; };
   static_assert(!WQ || MODE == 3, "quantised weights only in the single-launch form");
   using R = Ring<WQ>;
   constexpr int RST = R::RSTAGES;
@@ -255,10 +279,12 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     fence_proxy_async_smem();
   }
   if (warp == TMA_WARP && lane == 0) {
-    if (HAS1) tma_prefetch_desc(&tmap_w1);
-    if (HAS2) {
-      tma_prefetch_desc(&tmap_w2);
-      tma_prefetch_desc(&tmap_h);
+    for (int g = 0; g < nseg; ++g) {
+      if (HAS1) tma_prefetch_desc(&maps.w1[g]);
+      if (HAS2) {
+        tma_prefetch_desc(&maps.w2[g]);
+        tma_prefetch_desc(&maps.h[g]);
+      }
     }
   }
 
@@ -268,40 +294,50 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
   if (trace != nullptr && threadIdx.x == 0) trace[3 * blockIdx.x] = global_timer_ns();
   int first_tile = 0;
   if (threadIdx.x == TMA_WARP * 32) first_tile = atomicAdd(sched, 1);
-  int my_chunks = 0;
-  if (threadIdx.x < kE) {
-    const int e = threadIdx.x;
-    const int o0 = offsets[e], o1 = offsets[e + 1];
-    int c = o1 - o0;
-    if (o0 < 0 || c < 0 || static_cast<int64_t>(o1) > nrows) {
-      record_status(kSiteBadIndex);
-      c = 0;
-    }
-    S->cnt[e] = c;
-    S->off[e] = o0;
-    my_chunks = (c + BNT - 1) / BNT;
-  }
-  int incl = my_chunks;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
   if (warp == MMA_WARP) tmem_alloc(&S->tmem_base, R::TMEM_COLS);
-  __syncthreads();
-  if (threadIdx.x < kE) {
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += S->wsum[w];
-    S->cstart[threadIdx.x] = base + incl - my_chunks;
-    if (threadIdx.x == kE - 1) S->cstart[kE] = base + incl;
+  // per segment: the experts' row counts and first rows, and the prefix of
+  // their 32-token chunks
+  for (int g = 0; g < nseg; ++g) {
+    int my_chunks = 0;
+    if (threadIdx.x < kE) {
+      const int e = threadIdx.x;
+      const int32_t* offsets = seg.offsets[g];
+      const int o0 = offsets[e], o1 = offsets[e + 1];
+      int c = o1 - o0;
+      if (o0 < 0 || c < 0 || static_cast<int64_t>(o1) > nrows) {
+        record_status(kSiteBadIndex);
+        c = 0;
+      }
+      S->cnt[g][e] = c;
+      S->off[g][e] = o0;
+      my_chunks = (c + BNT - 1) / BNT;
+    }
+    int incl = my_chunks;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
+    __syncthreads();
+    if (threadIdx.x < kE) {
+      int base = 0;
+      for (int w = 0; w < warp; ++w) base += S->wsum[w];
+      S->cstart[g][threadIdx.x] = base + incl - my_chunks;
+      if (threadIdx.x == kE - 1) S->cstart[g][kE] = base + incl;
+    }
+    __syncthreads();  // wsum is reused by the next segment
+  }
+  if (threadIdx.x == 0) {
+    S->segbase[0] = 0;
+    for (int g = 0; g < nseg; ++g) S->segbase[g + 1] = S->segbase[g] + S->cstart[g][kE];
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem_base = S->tmem_base;
-  const int nchunks = S->cstart[kE];
+  const int nchunks = S->segbase[nseg];
   const int total1 = HAS1 ? nchunks * fblk(1) : 0;
   const int total_tiles = total1 + (HAS2 ? nchunks * fblk(2) : 0);
 
@@ -319,12 +355,12 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
         }
         if (pub < 0) break;
         const int next = atomicAdd(sched, 1);
-        const TileInfo ti = tile_info<MODE>(S, tile, total1);
-        const int e = ti.e, f = ti.f, c = ti.c;
+        const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
+        const int g = ti.g, e = ti.e, f = ti.f, c = ti.c;
         if (MODE == 3 && ti.phase == 2) {
           // every gate/up tile of expert e has stored its h values
-          const int need = kDoneStep * fblk(1) * ((S->cnt[e] + BNT - 1) / BNT);
-          if (!wait_count(done + e, need, abort_flag, timeout_ns, kSiteFfnDone)) {
+          const int need = kDoneStep * fblk(1) * ((S->cnt[g][e] + BNT - 1) / BNT);
+          if (!wait_count(done_of(g) + e, need, abort_flag, timeout_ns, kSiteFfnDone)) {
             ok = false;
             break;
           }
@@ -337,7 +373,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
         } else {
           wrow0 = e * kH + f * BMW;
         }
-        const int hrow = S->off[e] + c * BNT;
+        const int hrow = S->off[g][e] + c * BNT;
+        const CUtensorMap* tmap_w1 = &maps.w1[g];
+        const CUtensorMap* tmap_w2 = &maps.w2[g];
+        const CUtensorMap* tmap_h = &maps.h[g];
         const int KB = kblocks(ti.phase, KS);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % RST;
@@ -348,7 +387,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
           }
           if (WQ) {  // codes: two 64-row boxes (128 or 64 bytes); in phase 2 two 64-wide h tiles
             const int r1 = ti.phase == 1 ? wrow1 : wrow0 + 64;
-            const CUtensorMap* tw = ti.phase == 1 ? &tmap_w1 : &tmap_w2;
+            const CUtensorMap* tw = ti.phase == 1 ? tmap_w1 : tmap_w2;
             const void* scl;
             uint32_t scl_bytes;
             int kx;  // x coordinate of the code boxes, in bytes
@@ -369,17 +408,17 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             tma_load_2d(smem_u32(sA(s)), tw, kx, wrow0, &fullb[s]);
             tma_load_2d(smem_u32(sA(s)) + R::RA_BYTES / 2, tw, kx, r1, &fullb[s]);
             if (ti.phase == 2) {
-              tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * KS, hrow, &fullb[s]);
-              tma_load_2d(smem_u32(sB(s)) + B_BYTES, &tmap_h, kb * KS + BK, hrow, &fullb[s]);
+              tma_load_2d(smem_u32(sB(s)), tmap_h, kb * KS, hrow, &fullb[s]);
+              tma_load_2d(smem_u32(sB(s)) + B_BYTES, tmap_h, kb * KS + BK, hrow, &fullb[s]);
             }
           } else if (ti.phase == 1) {
             mbar_arrive_expect_tx(&fullb[s], A_BYTES);
-            tma_load_2d(smem_u32(sA(s)), &tmap_w1, kb * BK, wrow0, &fullb[s]);
-            tma_load_2d(smem_u32(sA(s)) + A_BYTES / 2, &tmap_w1, kb * BK, wrow1, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)), tmap_w1, kb * BK, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)) + A_BYTES / 2, tmap_w1, kb * BK, wrow1, &fullb[s]);
           } else {
             mbar_arrive_expect_tx(&fullb[s], A_BYTES + B_BYTES);
-            tma_load_2d(smem_u32(sA(s)), &tmap_w2, kb * BK, wrow0, &fullb[s]);
-            tma_load_2d(smem_u32(sB(s)), &tmap_h, kb * BK, hrow, &fullb[s]);
+            tma_load_2d(smem_u32(sA(s)), tmap_w2, kb * BK, wrow0, &fullb[s]);
+            tma_load_2d(smem_u32(sB(s)), tmap_h, kb * BK, hrow, &fullb[s]);
           }
         }
         tile = next;
@@ -470,7 +509,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     while (ok) {
       const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
       if (ti.phase == 2) {
         // down tile: the TMA brings the h rows; only keep the stage barriers' count
         for (int kb = 0; kb < kblocks(2, KS); ++kb, ++it) {
@@ -486,8 +525,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       }
       const int row_in_e = ti.c * BNT + lane;
       const char* src = nullptr;
-      if (row_in_e < S->cnt[ti.e]) {
-        const int p = perm_src[S->off[ti.e] + row_in_e];
+      if (row_in_e < S->cnt[ti.g][ti.e]) {
+        const int p = seg.perm_src[ti.g][S->off[ti.g][ti.e] + row_in_e];
         if (p >= 0 && static_cast<int64_t>(p) < nrows)
           src = reinterpret_cast<const char*>(x + static_cast<int64_t>(p >> 3) * kH);
       }
@@ -543,7 +582,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     while (ok) {
       const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
       for (int kb = 0; kb < kblocks(ti.phase, KS); ++kb, ++it) {
         const int s = it % RST;
         const uint32_t ph = (it / RST) & 1;
@@ -628,8 +667,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     for (int tc = 0;; ++tc) {
       const int tile = tileq_pop(&S->tq, tc, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      const TileInfo ti = tile_info<MODE>(S, tile, total1);
-      const int e = ti.e, f = ti.f, c = ti.c;
+      const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
+      const int g = ti.g, e = ti.e, f = ti.f, c = ti.c;
       const int a = tc & 1;
       const uint32_t use = tc >> 1;
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
@@ -646,8 +685,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->tempty[a]);  // accumulator copied out: MMA may reuse it
-      const int ntok = min(BNT, S->cnt[e] - c * BNT);
-      const int64_t row0 = static_cast<int64_t>(S->off[e]) + c * BNT;
+      const int ntok = min(BNT, S->cnt[g][e] - c * BNT);
+      const int64_t row0 = static_cast<int64_t>(S->off[g][e]) + c * BNT;
+      uint16_t* const h_out = seg.h_out[g];
+      uint16_t* const y_out = seg.y_out[g];
       if (ti.phase == 1) {
         const uint32_t xph = static_cast<uint32_t>(n1++) & 1;
         if (warp >= 2) {  // up half: hand the values to the gate half
@@ -678,7 +719,7 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
             asm volatile("fence.proxy.async.global;" ::: "memory");
             __threadfence();
             __syncwarp();
-            if (lane == 0) atomicAdd(done + e, 1);
+            if (lane == 0) atomicAdd(done_of(g) + e, 1);
           }
         }
       } else {
@@ -700,7 +741,10 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     if (trace != nullptr) trace[3 * blockIdx.x + 1] = global_timer_ns();
-    tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
+    const bool last = tileq_retire(sched, MODE == 3 ? done_of(0) : nullptr, MODE == 3 ? kE : 0);
+    if (MODE == 3 && last)  // the other segments' done counters too
+      for (int g = 1; g < nseg; ++g)
+        for (int i = 0; i < kE; ++i) atomicExch(done_of(g) + i, 0);
   }
   if (warp == MMA_WARP) {
     tc_fence_after();

@@ -344,18 +344,30 @@ int* sched_words(const int32_t* offsets, int phase) {
   return const_cast<int*>(offsets) + kSchedWord + 2 * (phase - 1);
 }
 
+// One weight pack's pointers for the skinny kernel (a launch of one segment).
+skinny::SegPtrs one_segment(const int32_t* offsets, const int32_t* perm_src, moe_bf16* h,
+                            moe_bf16* y) {
+  skinny::SegPtrs p{};
+  p.n = 1;
+  p.offsets[0] = offsets;
+  p.perm_src[0] = perm_src;
+  p.h_out[0] = reinterpret_cast<uint16_t*>(h);
+  p.y_out[0] = reinterpret_cast<uint16_t*>(y);
+  return p;
+}
+
 int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                const int32_t* perm_src, int64_t T, moe_bf16* h, int sms, cudaStream_t s) {
   if (T <= kSkinnyMaxT) {
-    CUtensorMap tw;
-    int rc = make_tmap(&tw, packed, kH, uint64_t(kE) * 2 * kI, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    skinny::SegMaps maps{};
+    int rc = make_tmap(&maps.w1[0], packed, kH, uint64_t(kE) * 2 * kI, 64,
+                       CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc) return rc;
     return launch_pdl("skinny_gemm_kernel<1> launch", skinny::skinny_gemm_kernel<1>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw, tw, tw,
-                      reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-                      reinterpret_cast<uint16_t*>(h), static_cast<uint16_t*>(nullptr),
-                      sched_words(offsets, 1), static_cast<int*>(nullptr),
-                      static_cast<const float*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps,
+                      one_segment(offsets, perm_src, h, nullptr),
+                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
   CUtensorMap tb1;
   int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -375,17 +387,16 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
   CUtensorMap tb2, ta2;
   const uint64_t rows = static_cast<uint64_t>(T) * kTopK;
   if (T <= kSkinnyMaxT) {
-    int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, skinny::BMW,
+    skinny::SegMaps maps{};
+    int rc = make_tmap(&maps.w2[0], packed + kPackGuElems, kI, uint64_t(kE) * kH, skinny::BMW,
                        CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-    if (!rc) rc = make_tmap(&ta2, h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (!rc) rc = make_tmap(&maps.h[0], h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
     return launch_pdl("skinny_gemm_kernel<2> launch", skinny::skinny_gemm_kernel<2>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tb2, tb2, ta2,
-                      static_cast<const __nv_bfloat16*>(nullptr), offsets,
-                      static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
-                      reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
-                      static_cast<int*>(nullptr), static_cast<const float*>(nullptr),
-                      g_timeout_ns.load(), ffn_trace(sms));
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps,
+                      one_segment(offsets, nullptr, nullptr, y),
+                      static_cast<const __nv_bfloat16*>(nullptr), T, sched_words(offsets, 2),
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
   int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -399,26 +410,37 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                     static_cast<int*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
 }
 
+// Tensor maps of segment g of a skinny launch: a bf16 pack of n_exp experts
+// (its down region from element d_off) and its h buffer of h_rows rows (a
+// chunk's box past the last row reads zeros, never past the buffer).
+int skinny_maps(skinny::SegMaps* maps, int g, const moe_bf16* packed, int n_exp, int64_t d_off,
+                const moe_bf16* h, int64_t h_rows) {
+  int rc = make_tmap(&maps->w1[g], packed, kH, uint64_t(n_exp) * 2 * kI, 64,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  if (!rc) rc = make_tmap(&maps->w2[g], packed + d_off, kI, uint64_t(n_exp) * kH, skinny::BMW,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (!rc) rc = make_tmap(&maps->h[g], h, kI, static_cast<uint64_t>(h_rows), skinny::BNT,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  return rc;
+}
+
 // n_exp: experts in the pack (128, or the shared experts' count), d_off: start
 // of its down region in elements; only experts with rows in `offsets` are read.
+// h_rows: rows of the h buffer (default 8T).
 int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                   const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, int sms,
-                  cudaStream_t s, int n_exp = kE, int64_t d_off = kPackGuElems) {
+                  cudaStream_t s, int n_exp = kE, int64_t d_off = kPackGuElems,
+                  int64_t h_rows = -1) {
+  if (h_rows < 0) h_rows = T * kTopK;
   if (T <= kSkinnyMaxT) {  // both GEMMs in one launch (see expert_ffn_skinny.cuh)
-    CUtensorMap tw1, tw2, th;
-    int rc = make_tmap(&tw1, packed, kH, uint64_t(n_exp) * 2 * kI, 64,
-                       CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-    if (!rc) rc = make_tmap(&tw2, packed + d_off, kI, uint64_t(n_exp) * kH, skinny::BMW,
-                            CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-    if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
-                            CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    skinny::SegMaps maps{};
+    int rc = skinny_maps(&maps, 0, packed, n_exp, d_off, h, h_rows);
     if (rc) return rc;
     return launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, tw1, tw2, th,
-                      reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-                      reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
-                      sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                      static_cast<const float*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps,
+                      one_segment(offsets, perm_src, h, y),
+                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
   // both GEMMs in one launch (see expert_ffn.cuh)
   CUtensorMap tb1, tb2, ta2;
@@ -426,7 +448,7 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   if (!rc) rc = make_tmap(&tb2, packed + d_off, kI, uint64_t(n_exp) * kH, ffn::BN,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-  if (!rc) rc = make_tmap(&ta2, h, kI, static_cast<uint64_t>(T) * kTopK, ffn::BM,
+  if (!rc) rc = make_tmap(&ta2, h, kI, static_cast<uint64_t>(h_rows), ffn::BM,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
   return launch_pdl("ffn_gemm_kernel<3> launch",
@@ -459,17 +481,16 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
     return do_expert_ffn(x, dq, offsets, perm_src, T, h, y, sms, s);
   }
   const uint8_t* p8 = static_cast<const uint8_t*>(packed8);
-  CUtensorMap tw1, tw2, th;
-  int rc = make_tmap_u8(&tw1, p8, kH, uint64_t(kE) * 2 * kI);
-  if (!rc) rc = make_tmap_u8(&tw2, p8 + fp8::kGuBytes, kI, uint64_t(kE) * kH);
-  if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
+  skinny::SegMaps maps{};
+  int rc = make_tmap_u8(&maps.w1[0], p8, kH, uint64_t(kE) * 2 * kI);
+  if (!rc) rc = make_tmap_u8(&maps.w2[0], p8 + fp8::kGuBytes, kI, uint64_t(kE) * kH);
+  if (!rc) rc = make_tmap(&maps.h[0], h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
   return launch_pdl("skinny_gemm_kernel<3, fp8> launch", skinny::skinny_gemm_kernel<3, 1>,
-                    dim3(sms), dim3(skinny::Ring<1>::THREADS), skinny::SMEM_BYTES, s, tw1, tw2,
-                    th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-                    reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
-                    sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
+                    dim3(sms), dim3(skinny::Ring<1>::THREADS), skinny::SMEM_BYTES, s, maps,
+                    one_segment(offsets, perm_src, h, y),
+                    reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
                     static_cast<const void*>(p8 + fp8::kSguOff), g_timeout_ns.load(), ffn_trace(sms));
 }
 
@@ -491,17 +512,17 @@ int do_expert_ffn_fp4(const moe_bf16* x, const void* packed4, const int32_t* off
     return do_expert_ffn(x, dq, offsets, perm_src, T, h, y, sms, s);
   }
   const uint8_t* p4 = static_cast<const uint8_t*>(packed4);
-  CUtensorMap tw1, tw2, th;
-  int rc = make_tmap_u8(&tw1, p4, fp4::kGuRowBytes, uint64_t(kE) * 2 * kI, 64);
-  if (!rc) rc = make_tmap_u8(&tw2, p4 + fp4::kGuBytes, fp4::kDRowBytes, uint64_t(kE) * kH, 64);
-  if (!rc) rc = make_tmap(&th, h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
+  skinny::SegMaps maps{};
+  int rc = make_tmap_u8(&maps.w1[0], p4, fp4::kGuRowBytes, uint64_t(kE) * 2 * kI, 64);
+  if (!rc)
+    rc = make_tmap_u8(&maps.w2[0], p4 + fp4::kGuBytes, fp4::kDRowBytes, uint64_t(kE) * kH, 64);
+  if (!rc) rc = make_tmap(&maps.h[0], h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
   return launch_pdl("skinny_gemm_kernel<3, nvfp4> launch", skinny::skinny_gemm_kernel<3, 2>,
-                    dim3(sms), dim3(skinny::Ring<2>::THREADS), skinny::SMEM_BYTES, s, tw1, tw2,
-                    th, reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-                    reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
-                    sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
+                    dim3(sms), dim3(skinny::Ring<2>::THREADS), skinny::SMEM_BYTES, s, maps,
+                    one_segment(offsets, perm_src, h, y),
+                    reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
                     static_cast<const void*>(p4 + fp4::kMguOff), g_timeout_ns.load(), ffn_trace(sms));
 }
 
@@ -518,16 +539,20 @@ int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
 // The shared experts' FFN: their row set (every token, once per shared
 // expert), then the grouped FFN on the shared pack.
 constexpr int kMaxShared = kTopK;  // n_shared * T rows fit the routed buffers' bounds
+int do_shared_rows(int n_shared, int64_t T, int32_t* offsets, int32_t* perm_src, cudaStream_t s) {
+  const int64_t n = std::max<int64_t>(kOffsetsLen, n_shared * T);
+  return launch_pdl("shared_rows_kernel launch", shared_rows_kernel,
+                    dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, T, n_shared,
+                    offsets, perm_src);
+}
+
 int do_shared_ffn(const moe_bf16* x, const moe_bf16* packed_shared, int n_shared, int64_t T,
                   int32_t* offsets, int32_t* perm_src, moe_bf16* h, moe_bf16* y, int sms,
                   cudaStream_t s) {
-  const int64_t n = std::max<int64_t>(kOffsetsLen, n_shared * T);
-  int rc = launch_pdl("shared_rows_kernel launch", shared_rows_kernel,
-                      dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, T, n_shared,
-                      offsets, perm_src);
+  int rc = do_shared_rows(n_shared, T, offsets, perm_src, s);
   if (rc) return rc;
   return do_expert_ffn(x, packed_shared, offsets, perm_src, T, h, y, sms, s, n_shared,
-                       int64_t(n_shared) * kPackGuPerExpert);
+                       int64_t(n_shared) * kPackGuPerExpert, int64_t(n_shared) * T);
 }
 
 // workspace carve-up of moe_layer
@@ -1353,14 +1378,43 @@ int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
                       0, s, static_cast<const int32_t*>(idx), T, static_cast<const int32_t*>(hist),
                       perm_src, inv_perm);
   }
-  // experts 0..127 and 128..255: the 128-expert kernels on each half's pack
-  if (!rc) rc = do_expert_ffn(x, packed_lo, off_lo, perm_src, T, h, y, sms, s);
-  if (!rc) rc = do_expert_ffn(x, packed_hi, off_hi, perm_src, T, h, y, sms, s);
   moe_bf16* y_sh = reinterpret_cast<moe_bf16*>(ws + L.sh_y);
-  if (!rc && n_shared > 0)
-    rc = do_shared_ffn(x, packed_shared, n_shared, T, reinterpret_cast<int32_t*>(ws + L.sh_offsets),
-                       reinterpret_cast<int32_t*>(ws + L.sh_perm),
-                       reinterpret_cast<moe_bf16*>(ws + L.sh_h), y_sh, sms, s);
+  int32_t* sh_offsets = reinterpret_cast<int32_t*>(ws + L.sh_offsets);
+  int32_t* sh_perm = reinterpret_cast<int32_t*>(ws + L.sh_perm);
+  moe_bf16* sh_h = reinterpret_cast<moe_bf16*>(ws + L.sh_h);
+  if (T <= kSkinnyMaxT) {
+    // one skinny launch over experts 0..127, 128..255 and the shared experts
+    // (three segments: each pack, its offsets, its rows)
+    if (!rc && n_shared > 0) rc = do_shared_rows(n_shared, T, sh_offsets, sh_perm, s);
+    skinny::SegMaps maps{};
+    skinny::SegPtrs p{};
+    const moe_bf16* packs[3] = {packed_lo, packed_hi, packed_shared};
+    const int32_t* offs[3] = {off_lo, off_hi, sh_offsets};
+    const int32_t* perms[3] = {perm_src, perm_src, sh_perm};
+    moe_bf16* hs[3] = {h, h, sh_h};
+    moe_bf16* ys[3] = {y, y, y_sh};
+    p.n = n_shared > 0 ? 3 : 2;
+    for (int g = 0; g < p.n && !rc; ++g) {
+      const int n_exp = g < 2 ? kE : n_shared;
+      rc = skinny_maps(&maps, g, packs[g], n_exp, g < 2 ? kPackGuElems : int64_t(n_shared) * kPackGuPerExpert,
+                       hs[g], g < 2 ? T * kTopK : int64_t(n_shared) * T);
+      p.offsets[g] = offs[g];
+      p.perm_src[g] = perms[g];
+      p.h_out[g] = reinterpret_cast<uint16_t*>(hs[g]);
+      p.y_out[g] = reinterpret_cast<uint16_t*>(ys[g]);
+    }
+    if (!rc)
+      rc = launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps, p,
+                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(off_lo, 1),
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+  } else {
+    // experts 0..127 and 128..255: the 128-expert kernels on each half's pack
+    if (!rc) rc = do_expert_ffn(x, packed_lo, off_lo, perm_src, T, h, y, sms, s);
+    if (!rc) rc = do_expert_ffn(x, packed_hi, off_hi, perm_src, T, h, y, sms, s);
+    if (!rc && n_shared > 0)
+      rc = do_shared_ffn(x, packed_shared, n_shared, T, sh_offsets, sh_perm, sh_h, y_sh, sms, s);
+  }
   if (!rc)
     rc = launch_pdl("combine_kernel launch", combine_kernel<e256::kTopK2>,
                     dim3(static_cast<unsigned>(T)), dim3(kCombineThreads), 0, s,
