@@ -833,21 +833,47 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
       rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
                             ws + L.perm_ws, s);
   }
-  if (!rc) {
-    if (quant && qfmt == 2)
-      rc = do_expert_ffn_fp4(x, packed_q, offsets, perm_src, T, h, y,
-                             reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
-    else if (quant)
-      rc = do_expert_ffn_fp8(x, packed_q, offsets, perm_src, T, h, y,
-                             reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
-    else
-      rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
-  }
   moe_bf16* y_sh = reinterpret_cast<moe_bf16*>(ws + L.sh_y);
-  if (!rc && n_shared > 0)
-    rc = do_shared_ffn(x, packed_shared, n_shared, T, reinterpret_cast<int32_t*>(ws + L.sh_offsets),
-                       reinterpret_cast<int32_t*>(ws + L.sh_perm),
-                       reinterpret_cast<moe_bf16*>(ws + L.sh_h), y_sh, sms, s);
+  int32_t* sh_offsets = reinterpret_cast<int32_t*>(ws + L.sh_offsets);
+  int32_t* sh_perm = reinterpret_cast<int32_t*>(ws + L.sh_perm);
+  moe_bf16* sh_h = reinterpret_cast<moe_bf16*>(ws + L.sh_h);
+  if (!rc && !quant && n_shared > 0 && T <= kSkinnyMaxT) {
+    // the routed experts and the shared experts as two segments of one launch
+    rc = do_shared_rows(n_shared, T, sh_offsets, sh_perm, s);
+    skinny::SegMaps maps{};
+    skinny::SegPtrs p{};
+    p.n = 2;
+    if (!rc) rc = skinny_maps(&maps, 0, packed_w, kE, kPackGuElems, h, T * kTopK);
+    if (!rc)
+      rc = skinny_maps(&maps, 1, packed_shared, n_shared, int64_t(n_shared) * kPackGuPerExpert,
+                       sh_h, int64_t(n_shared) * T);
+    p.offsets[0] = offsets;
+    p.perm_src[0] = perm_src;
+    p.h_out[0] = reinterpret_cast<uint16_t*>(h);
+    p.y_out[0] = reinterpret_cast<uint16_t*>(y);
+    p.offsets[1] = sh_offsets;
+    p.perm_src[1] = sh_perm;
+    p.h_out[1] = reinterpret_cast<uint16_t*>(sh_h);
+    p.y_out[1] = reinterpret_cast<uint16_t*>(y_sh);
+    if (!rc)
+      rc = launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps, p,
+                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+  } else {
+    if (!rc) {
+      if (quant && qfmt == 2)
+        rc = do_expert_ffn_fp4(x, packed_q, offsets, perm_src, T, h, y,
+                               reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
+      else if (quant)
+        rc = do_expert_ffn_fp8(x, packed_q, offsets, perm_src, T, h, y,
+                               reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
+      else
+        rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
+    }
+    if (!rc && n_shared > 0)
+      rc = do_shared_ffn(x, packed_shared, n_shared, T, sh_offsets, sh_perm, sh_h, y_sh, sms, s);
+  }
   if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s, y_sh, n_shared);
   return rc;
 }
