@@ -489,6 +489,29 @@ __device__ __forceinline__ bool tileq_retire(int* sched, int* extra = nullptr, i
 
 constexpr int kDoneWord = kSchedWord + 4;  // offsets[136 .. 263]: per-expert done counters
 
+// Weight packs of one expert-FFN launch ("segments"): up to kMaxSeg packs of
+// up to 128 experts each, every one with its own offsets array (the down
+// tiles' done counters live in it), row sources and h / y_perm rows.  The
+// 256-expert shape runs its two halves and its shared experts as three
+// segments of one launch, the shared experts of the 128-expert shape run as a
+// second segment beside the routed pack; every other call is one segment.
+// Tile ids run over all segments' gate/up tiles, then all segments' down
+// tiles.
+constexpr int kMaxSeg = 3;
+struct SegMaps {
+  CUtensorMap w1[kMaxSeg];  // gate/up weights (phase 1)
+  CUtensorMap w2[kMaxSeg];  // down weights (phase 2)
+  CUtensorMap h[kMaxSeg];   // h rows (phase 2)
+};
+struct SegPtrs {
+  int n;                             // segments in the launch, 1 .. kMaxSeg
+  const int32_t* offsets[kMaxSeg];   // offsets array (129 offsets, then the work counters)
+  const int32_t* perm_src[kMaxSeg];  // row sources (8t + slot)
+  uint16_t* h_out[kMaxSeg];
+  uint16_t* y_out[kMaxSeg];
+};
+
+
 // Waits until *counter >= need (acquire), bounded in time; then orders the
 // async proxy (TMA) after it.
 __device__ __forceinline__ bool wait_count(const int* counter, int need, volatile int* abort_flag,

@@ -104,38 +104,43 @@ struct SmemTail {
   uint32_t tmem_base;
   int abort_flag;
   int wsum[4];
-  int mstart[kE + 1];  // exclusive prefix of the experts' 128-row m-tile counts
-  int cnt[kE];
-  int off[kE];
+  int segbase[kMaxSeg + 1];     // exclusive prefix of the segments' m-tile counts
+  int mstart[kMaxSeg][kE + 1];  // per segment: exclusive prefix of the experts' 128-row m-tiles
+  int cnt[kMaxSeg][kE];
+  int off[kMaxSeg][kE];
 };
 constexpr int TAIL_BYTES = (static_cast<int>(sizeof(SmemTail)) + 127) / 128 * 128;
 constexpr int SMEM_BYTES = TILE_BYTES + TAIL_BYTES + 4 * EPI_WARP_BYTES + 1024;
 
-// Tile u of a phase with NT n-tiles per expert: expert e, m-tile m, n-tile j
-// (expert-major, then j, then m).
-__device__ __forceinline__ void decode_tile(const SmemTail* S, int u, int NT, int& e, int& m,
-                                            int& j) {
+// Tile u of a phase with NT n-tiles per expert, over all segments: segment g,
+// expert e, m-tile m, n-tile j (segment-major, then expert, then j, then m).
+__device__ __forceinline__ void decode_tile(const SmemTail* S, int nseg, int u, int NT, int& g,
+                                            int& e, int& m, int& j) {
+  g = 0;
+  while (g + 1 < nseg && S->segbase[g + 1] * NT <= u) ++g;
+  u -= S->segbase[g] * NT;
+  const int* ms = S->mstart[g];
   int lo = 0, hi = kE - 1;  // largest e with mstart[e] * NT <= u
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (S->mstart[mid] * NT <= u) lo = mid; else hi = mid - 1;
+    if (ms[mid] * NT <= u) lo = mid; else hi = mid - 1;
   }
   e = lo;
-  const int rem = u - S->mstart[e] * NT;
-  const int mt = (S->cnt[e] + BM - 1) / BM;
+  const int rem = u - ms[e] * NT;
+  const int mt = (S->cnt[g][e] + BM - 1) / BM;
   j = rem / mt;
   m = rem - j * mt;
 }
 
 struct TileInfo {
-  int phase, e, m, j;
+  int phase, g, e, m, j;
 };
 template <int MODE>
-__device__ __forceinline__ TileInfo tile_info(const SmemTail* S, int tile, int total1) {
+__device__ __forceinline__ TileInfo tile_info(const SmemTail* S, int nseg, int tile, int total1) {
   TileInfo t;
   t.phase = MODE == 3 ? (tile < total1 ? 1 : 2) : MODE;
   const int u = (MODE == 3 && t.phase == 2) ? tile - total1 : tile;
-  decode_tile(S, u, nt_of(t.phase), t.e, t.m, t.j);
+  decode_tile(S, nseg, u, nt_of(t.phase), t.g, t.e, t.m, t.j);
   return t;
 }
 
@@ -167,15 +172,14 @@ __device__ __forceinline__ void store_block_32x32(const uint32_t (&pk)[16], uint
 
 template <int MODE, bool ZERO_PAD>
 __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
-    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b1,  // packed W_gate/W_up (phase 1)
-                    const __grid_constant__ CUtensorMap tmap_b2,  // packed W_down (phase 2)
-                    const __grid_constant__ CUtensorMap tmap_a2,  // h rows (phase 2)
-                    const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ offsets,
-                    const int32_t* __restrict__ perm_src, int64_t T,
-                    uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_out,
-                    int* __restrict__ sched, int* __restrict__ done, uint64_t timeout_ns,
+    ffn_gemm_kernel(const __grid_constant__ SegMaps maps,  // w1: packed W_gate/W_up, w2: W_down, h
+                    const __grid_constant__ SegPtrs seg, const __nv_bfloat16* __restrict__ x,
+                    int64_t T, int* __restrict__ sched, uint64_t timeout_ns,
                     uint64_t* __restrict__ trace) {
   using C = Cfg<MODE>;
+  const int nseg = seg.n;
+  // segment g's per-expert done counters (single-launch form only)
+  auto done_of = [&](int g) { return const_cast<int*>(seg.offsets[g]) + kDoneWord; };
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -206,10 +210,12 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
     fence_proxy_async_smem();
   }
   if (warp == C::TMA_WARP && lane == 0) {
-    if (C::HAS1) tma_prefetch_desc(&tmap_b1);
-    if (C::HAS2) {
-      tma_prefetch_desc(&tmap_b2);
-      tma_prefetch_desc(&tmap_a2);
+    for (int g = 0; g < nseg; ++g) {
+      if (C::HAS1) tma_prefetch_desc(&maps.w1[g]);
+      if (C::HAS2) {
+        tma_prefetch_desc(&maps.w2[g]);
+        tma_prefetch_desc(&maps.h[g]);
+      }
     }
   }
 
@@ -220,27 +226,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
   if (trace != nullptr && threadIdx.x == 0) trace[3 * blockIdx.x] = global_timer_ns();
   int first_tile = 0;
   if (threadIdx.x == C::TMA_WARP * 32) first_tile = atomicAdd(sched, 1);
-  int my_mt = 0;
-  if (threadIdx.x < kE) {
-    const int e = threadIdx.x;
-    const int o0 = offsets[e], o1 = offsets[e + 1];
-    int c = o1 - o0;
-    if (o0 < 0 || c < 0 || static_cast<int64_t>(o1) > nrows) {
-      record_status(kSiteBadIndex);
-      c = 0;
-    }
-    S->cnt[e] = c;
-    S->off[e] = o0;
-    my_mt = (c + BM - 1) / BM;
-  }
-  int incl = my_mt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
-
   if (C::HAS1) {
     // Start the A ring at zero: rows past an expert's count are never loaded,
     // and with whatever the previous kernel left in shared memory there the
@@ -250,19 +235,49 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
     fence_proxy_async_smem();
   }
   if (warp == C::MMA_WARP) tmem_alloc(&S->tmem_base, TMEM_COLS);
-  __syncthreads();
-  if (threadIdx.x < kE) {
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += S->wsum[w];
-    S->mstart[threadIdx.x] = base + incl - my_mt;
-    if (threadIdx.x == kE - 1) S->mstart[kE] = base + incl;
+  // per segment: the experts' row counts and first rows, and the prefix of
+  // their 128-row m-tiles
+  for (int g = 0; g < nseg; ++g) {
+    int my_mt = 0;
+    if (threadIdx.x < kE) {
+      const int e = threadIdx.x;
+      const int32_t* offsets = seg.offsets[g];
+      const int o0 = offsets[e], o1 = offsets[e + 1];
+      int c = o1 - o0;
+      if (o0 < 0 || c < 0 || static_cast<int64_t>(o1) > nrows) {
+        record_status(kSiteBadIndex);
+        c = 0;
+      }
+      S->cnt[g][e] = c;
+      S->off[g][e] = o0;
+      my_mt = (c + BM - 1) / BM;
+    }
+    int incl = my_mt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (threadIdx.x < kE && lane == 31) S->wsum[warp] = incl;
+    __syncthreads();
+    if (threadIdx.x < kE) {
+      int base = 0;
+      for (int w = 0; w < warp; ++w) base += S->wsum[w];
+      S->mstart[g][threadIdx.x] = base + incl - my_mt;
+      if (threadIdx.x == kE - 1) S->mstart[g][kE] = base + incl;
+    }
+    __syncthreads();  // wsum is reused by the next segment
+  }
+  if (threadIdx.x == 0) {
+    S->segbase[0] = 0;
+    for (int g = 0; g < nseg; ++g) S->segbase[g + 1] = S->segbase[g] + S->mstart[g][kE];
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem_base = S->tmem_base;
-  const int mtiles = S->mstart[kE];
+  const int mtiles = S->segbase[nseg];
   const int total1 = C::HAS1 ? mtiles * nt_of(1) : 0;
   const int total_tiles = total1 + (C::HAS2 ? mtiles * nt_of(2) : 0);
 
@@ -280,17 +295,17 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
         }
         if (pub < 0) break;
         const int next = atomicAdd(sched, 1);  // used after the loads
-        const TileInfo ti = tile_info<MODE>(S, tile, total1);
+        const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
         if (MODE == 3 && ti.phase == 2) {
           // every gate/up tile of expert e has stored its h rows
-          const int need = kDoneStep * nt_of(1) * ((S->cnt[ti.e] + BM - 1) / BM);
-          if (!wait_count(done + ti.e, need, abort_flag, timeout_ns, kSiteFfnDone)) {
+          const int need = kDoneStep * nt_of(1) * ((S->cnt[ti.g][ti.e] + BM - 1) / BM);
+          if (!wait_count(done_of(ti.g) + ti.e, need, abort_flag, timeout_ns, kSiteFfnDone)) {
             ok = false;
             break;
           }
         }
         const int brow = ti.e * brows_of(ti.phase) + ti.j * BN;
-        const int arow = S->off[ti.e] + ti.m * BM;
+        const int arow = S->off[ti.g][ti.e] + ti.m * BM;
         for (int kb = 0; kb < kb_of(ti.phase); ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -300,11 +315,11 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
           }
           if (ti.phase == 2) {
             mbar_arrive_expect_tx(&S->full[s], A_BYTES + B_BYTES);
-            tma_load_2d(smem_u32(sA + s * A_BYTES), &tmap_a2, kb * BK, arow, &S->full[s]);
-            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b2, kb * BK, brow, &S->full[s]);
+            tma_load_2d(smem_u32(sA + s * A_BYTES), &maps.h[ti.g], kb * BK, arow, &S->full[s]);
+            tma_load_2d(smem_u32(sB + s * B_BYTES), &maps.w2[ti.g], kb * BK, brow, &S->full[s]);
           } else {
             mbar_arrive_expect_tx(&S->full[s], B_BYTES);
-            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmap_b1, kb * BK, brow, &S->full[s]);
+            tma_load_2d(smem_u32(sB + s * B_BYTES), &maps.w1[ti.g], kb * BK, brow, &S->full[s]);
           }
         }
         tile = next;
@@ -379,7 +394,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int row_in_e = tj.m * BM + rsub + 32 * i;
-        pv[i] = row_in_e < S->cnt[tj.e] ? perm_src[S->off[tj.e] + row_in_e] : -1;
+        pv[i] = row_in_e < S->cnt[tj.g][tj.e] ? seg.perm_src[tj.g][S->off[tj.g][tj.e] + row_in_e] : -1;
       }
     };
     int it = 0, n = 0;
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
     while (ok) {
       const int tile = tileq_pop(&S->tq, n++, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      const TileInfo ti = tile_info<MODE>(S, tile, total1);
+      const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
       if (ti.phase == 2) {
         for (int kb = 0; kb < kb_of(2); ++kb, ++it) {
           const int s = it % STAGES;
@@ -421,7 +436,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
         if (kb >= kb_of(1) - STAGES && pf_tile < 0) {  // the next tile, once it is published
           const int nx = tileq_peek(&S->tq, n);
           if (nx >= 0) {
-            const TileInfo tn = tile_info<MODE>(S, nx, total1);
+            const TileInfo tn = tile_info<MODE>(S, nseg, nx, total1);
             if (tn.phase == 1) {
               load_rows(tn, pf_p);
               pf_tile = nx;
@@ -454,17 +469,19 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
     for (int tc = 0;; ++tc) {
       const int tile = tileq_pop(&S->tq, tc, lane == 0, abort_flag, timeout_ns);
       if (tile < 0) break;
-      const TileInfo ti = tile_info<MODE>(S, tile, total1);
-      const int e = ti.e, m = ti.m, j = ti.j;
+      const TileInfo ti = tile_info<MODE>(S, nseg, tile, total1);
+      const int g = ti.g, e = ti.e, m = ti.m, j = ti.j;
       const int a = tc & 1;
       const uint32_t use = tc >> 1;
       if (!mbar_wait(&S->tfull[a], use & 1, abort_flag, timeout_ns, kSiteFfnTmemFull)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a * BN;
-      const int nvalid = min(32, max(0, S->cnt[e] - (m * BM + warp * 32)));
+      const int nvalid = min(32, max(0, S->cnt[g][e] - (m * BM + warp * 32)));
       const uint32_t stage = smem_u32(sEpi + warp * EPI_WARP_BYTES);
       bool bad = false;  // range check of this thread's row; rows >= nvalid hold garbage
-      const int64_t row0 = static_cast<int64_t>(S->off[e]) + m * BM + warp * 32;
+      const int64_t row0 = static_cast<int64_t>(S->off[g][e]) + m * BM + warp * 32;
+      uint16_t* const h_out = seg.h_out[g];
+      uint16_t* const y_out = seg.y_out[g];
       // A warp whose 32 rows are all padding has nothing to read or store (at
       // T=2048 with skewed routing that was a fifth of the gate/up time).
       if (nvalid == 0) {
@@ -508,7 +525,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __threadfence();
         __syncwarp();
-        if (lane == 0) atomicAdd(done + e, 1);
+        if (lane == 0) atomicAdd(done_of(g) + e, 1);
       }
     }
     if (range_bad) record_status(kSiteFp16Range);
@@ -518,7 +535,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     if (trace != nullptr) trace[3 * blockIdx.x + 1] = global_timer_ns();
-    tileq_retire(sched, MODE == 3 ? done : nullptr, MODE == 3 ? kE : 0);
+    const bool last = tileq_retire(sched, MODE == 3 ? done_of(0) : nullptr, MODE == 3 ? kE : 0);
+    if (MODE == 3 && last)  // the other segments' done counters too
+      for (int g = 1; g < nseg; ++g)
+        for (int i = 0; i < kE; ++i) atomicExch(done_of(g) + i, 0);
   }
   if (warp == C::MMA_WARP) {
     tc_fence_after();

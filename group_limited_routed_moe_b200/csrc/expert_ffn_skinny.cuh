@@ -150,26 +150,6 @@ constexpr uint32_t kIdesc2 = idesc_f32acc(BMW, BNT, kFmtF16);
 // storing warp): a down tile of expert e waits for kDoneStep * 8 * chunks(e).
 constexpr int kDoneStep = 2;
 
-// Weight packs of one launch ("segments"): up to kMaxSeg packs of up to 128
-// experts each, every one with its own offsets array (the down tiles' done
-// counters live in it), row sources and h / y_perm rows.  The 256-expert shape
-// runs its two halves and its shared experts as three segments of one launch;
-// every other call is one segment.  Tile ids run over all segments' gate/up
-// tiles, then all segments' down tiles.
-constexpr int kMaxSeg = 3;
-struct SegMaps {
-  CUtensorMap w1[kMaxSeg];  // gate/up weights (phase 1)
-  CUtensorMap w2[kMaxSeg];  // down weights (phase 2)
-  CUtensorMap h[kMaxSeg];   // h rows (phase 2)
-};
-struct SegPtrs {
-  int n;                             // segments in the launch, 1 .. kMaxSeg
-  const int32_t* offsets[kMaxSeg];   // offsets array (129 offsets, then the work counters)
-  const int32_t* perm_src[kMaxSeg];  // row sources (8t + slot)
-  uint16_t* h_out[kMaxSeg];
-  uint16_t* y_out[kMaxSeg];
-};
-
 struct Tail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];

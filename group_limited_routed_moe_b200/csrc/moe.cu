@@ -345,9 +345,9 @@ int* sched_words(const int32_t* offsets, int phase) {
 }
 
 // One weight pack's pointers for the skinny kernel (a launch of one segment).
-skinny::SegPtrs one_segment(const int32_t* offsets, const int32_t* perm_src, moe_bf16* h,
+SegPtrs one_segment(const int32_t* offsets, const int32_t* perm_src, moe_bf16* h,
                             moe_bf16* y) {
-  skinny::SegPtrs p{};
+  SegPtrs p{};
   p.n = 1;
   p.offsets[0] = offsets;
   p.perm_src[0] = perm_src;
@@ -359,7 +359,7 @@ skinny::SegPtrs one_segment(const int32_t* offsets, const int32_t* perm_src, moe
 int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                const int32_t* perm_src, int64_t T, moe_bf16* h, int sms, cudaStream_t s) {
   if (T <= kSkinnyMaxT) {
-    skinny::SegMaps maps{};
+    SegMaps maps{};
     int rc = make_tmap(&maps.w1[0], packed, kH, uint64_t(kE) * 2 * kI, 64,
                        CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc) return rc;
@@ -369,25 +369,23 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
                       reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
                       static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
-  CUtensorMap tb1;
-  int rc = make_tmap(&tb1, packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
+  SegMaps maps{};
+  int rc = make_tmap(&maps.w1[0], packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   if (rc) return rc;
-  const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-  auto* hb = reinterpret_cast<uint16_t*>(h);
   return launch_pdl("ffn_gemm_kernel<1> launch",
                     T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<1, true> : ffn::ffn_gemm_kernel<1, false>,
-                    dim3(sms), dim3(ffn::Cfg<1>::THREADS), ffn::SMEM_BYTES, s, tb1, tb1, tb1, xb,
-                    offsets, perm_src, T, hb, static_cast<uint16_t*>(nullptr),
-                    sched_words(offsets, 1), static_cast<int*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+                    dim3(sms), dim3(ffn::Cfg<1>::THREADS), ffn::SMEM_BYTES, s, maps,
+                    one_segment(offsets, perm_src, h, nullptr),
+                    reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
+                    g_timeout_ns.load(), ffn_trace(sms));
 }
 
 int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, int64_t T,
             moe_bf16* y, int sms, cudaStream_t s) {
-  CUtensorMap tb2, ta2;
   const uint64_t rows = static_cast<uint64_t>(T) * kTopK;
   if (T <= kSkinnyMaxT) {
-    skinny::SegMaps maps{};
+    SegMaps maps{};
     int rc = make_tmap(&maps.w2[0], packed + kPackGuElems, kI, uint64_t(kE) * kH, skinny::BMW,
                        CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (!rc) rc = make_tmap(&maps.h[0], h, kI, rows, skinny::BNT, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -398,22 +396,22 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                       static_cast<const __nv_bfloat16*>(nullptr), T, sched_words(offsets, 2),
                       static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
   }
-  int rc = make_tmap(&tb2, packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
+  SegMaps maps{};
+  int rc = make_tmap(&maps.w2[0], packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-  if (!rc) rc = make_tmap(&ta2, h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (!rc) rc = make_tmap(&maps.h[0], h, kI, rows, ffn::BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (rc) return rc;
   return launch_pdl("ffn_gemm_kernel<2> launch", ffn::ffn_gemm_kernel<2, false>, dim3(sms),
-                    dim3(ffn::Cfg<2>::THREADS), ffn::SMEM_BYTES, s, tb2, tb2, ta2,
-                    static_cast<const __nv_bfloat16*>(nullptr), offsets,
-                    static_cast<const int32_t*>(nullptr), T, static_cast<uint16_t*>(nullptr),
-                    reinterpret_cast<uint16_t*>(y), sched_words(offsets, 2),
-                    static_cast<int*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+                    dim3(ffn::Cfg<2>::THREADS), ffn::SMEM_BYTES, s, maps,
+                    one_segment(offsets, nullptr, nullptr, y),
+                    static_cast<const __nv_bfloat16*>(nullptr), T, sched_words(offsets, 2),
+                    g_timeout_ns.load(), ffn_trace(sms));
 }
 
 // Tensor maps of segment g of a skinny launch: a bf16 pack of n_exp experts
 // (its down region from element d_off) and its h buffer of h_rows rows (a
 // chunk's box past the last row reads zeros, never past the buffer).
-int skinny_maps(skinny::SegMaps* maps, int g, const moe_bf16* packed, int n_exp, int64_t d_off,
+int skinny_maps(SegMaps* maps, int g, const moe_bf16* packed, int n_exp, int64_t d_off,
                 const moe_bf16* h, int64_t h_rows) {
   int rc = make_tmap(&maps->w1[g], packed, kH, uint64_t(n_exp) * 2 * kI, 64,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
@@ -424,6 +422,42 @@ int skinny_maps(skinny::SegMaps* maps, int g, const moe_bf16* packed, int n_exp,
   return rc;
 }
 
+// Tensor maps of segment g of a wide launch: as skinny_maps, with the wide
+// kernel's boxes (256 weight rows, 128 h rows).
+int wide_maps(SegMaps* maps, int g, const moe_bf16* packed, int n_exp, int64_t d_off,
+              const moe_bf16* h, int64_t h_rows) {
+  int rc = make_tmap(&maps->w1[g], packed, kH, uint64_t(n_exp) * 2 * kI, ffn::BN,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  if (!rc) rc = make_tmap(&maps->w2[g], packed + d_off, kI, uint64_t(n_exp) * kH, ffn::BN,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (!rc) rc = make_tmap(&maps->h[g], h, kI, static_cast<uint64_t>(h_rows), ffn::BM,
+                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  return rc;
+}
+
+// The maps of segment g for the kernel that runs T tokens.
+int ffn_maps(SegMaps* maps, int g, const moe_bf16* packed, int n_exp, int64_t d_off,
+             const moe_bf16* h, int64_t h_rows, int64_t T) {
+  return T <= kSkinnyMaxT ? skinny_maps(maps, g, packed, n_exp, d_off, h, h_rows)
+                          : wide_maps(maps, g, packed, n_exp, d_off, h, h_rows);
+}
+
+// The single-launch expert FFN over the segments p (maps from ffn_maps); the
+// tile counters are segment 0's.
+int do_ffn_segments(const SegMaps& maps, const SegPtrs& p, const moe_bf16* x, int64_t T, int sms,
+                    cudaStream_t s) {
+  const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  if (T <= kSkinnyMaxT)
+    return launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
+                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps, p, xb, T,
+                      sched_words(p.offsets[0], 1), static_cast<const void*>(nullptr),
+                      g_timeout_ns.load(), ffn_trace(sms));
+  return launch_pdl("ffn_gemm_kernel<3> launch",
+                    T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<3, true> : ffn::ffn_gemm_kernel<3, false>,
+                    dim3(sms), dim3(ffn::Cfg<3>::THREADS), ffn::SMEM_BYTES, s, maps, p, xb, T,
+                    sched_words(p.offsets[0], 1), g_timeout_ns.load(), ffn_trace(sms));
+}
+
 // n_exp: experts in the pack (128, or the shared experts' count), d_off: start
 // of its down region in elements; only experts with rows in `offsets` are read.
 // h_rows: rows of the h buffer (default 8T).
@@ -432,32 +466,11 @@ int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offs
                   cudaStream_t s, int n_exp = kE, int64_t d_off = kPackGuElems,
                   int64_t h_rows = -1) {
   if (h_rows < 0) h_rows = T * kTopK;
-  if (T <= kSkinnyMaxT) {  // both GEMMs in one launch (see expert_ffn_skinny.cuh)
-    skinny::SegMaps maps{};
-    int rc = skinny_maps(&maps, 0, packed, n_exp, d_off, h, h_rows);
-    if (rc) return rc;
-    return launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps,
-                      one_segment(offsets, perm_src, h, y),
-                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
-                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
-  }
-  // both GEMMs in one launch (see expert_ffn.cuh)
-  CUtensorMap tb1, tb2, ta2;
-  int rc = make_tmap(&tb1, packed, kH, uint64_t(n_exp) * 2 * kI, ffn::BN,
-                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-  if (!rc) rc = make_tmap(&tb2, packed + d_off, kI, uint64_t(n_exp) * kH, ffn::BN,
-                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-  if (!rc) rc = make_tmap(&ta2, h, kI, static_cast<uint64_t>(h_rows), ffn::BM,
-                          CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  // both GEMMs in one launch (see expert_ffn_skinny.cuh, expert_ffn.cuh)
+  SegMaps maps{};
+  int rc = ffn_maps(&maps, 0, packed, n_exp, d_off, h, h_rows, T);
   if (rc) return rc;
-  return launch_pdl("ffn_gemm_kernel<3> launch",
-                    T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<3, true> : ffn::ffn_gemm_kernel<3, false>,
-                    dim3(sms), dim3(ffn::Cfg<3>::THREADS), ffn::SMEM_BYTES, s, tb1, tb2, ta2,
-                    reinterpret_cast<const __nv_bfloat16*>(x), offsets, perm_src, T,
-                    reinterpret_cast<uint16_t*>(h), reinterpret_cast<uint16_t*>(y),
-                    sched_words(offsets, 1), const_cast<int*>(offsets) + kDoneWord,
-                    g_timeout_ns.load(), ffn_trace(sms));
+  return do_ffn_segments(maps, one_segment(offsets, perm_src, h, y), x, T, sms, s);
 }
 
 // Packed block-FP8 layer -> packed bf16/fp16 layer.
@@ -481,7 +494,7 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
     return do_expert_ffn(x, dq, offsets, perm_src, T, h, y, sms, s);
   }
   const uint8_t* p8 = static_cast<const uint8_t*>(packed8);
-  skinny::SegMaps maps{};
+  SegMaps maps{};
   int rc = make_tmap_u8(&maps.w1[0], p8, kH, uint64_t(kE) * 2 * kI);
   if (!rc) rc = make_tmap_u8(&maps.w2[0], p8 + fp8::kGuBytes, kI, uint64_t(kE) * kH);
   if (!rc) rc = make_tmap(&maps.h[0], h, kI, static_cast<uint64_t>(T) * kTopK, skinny::BNT,
@@ -512,7 +525,7 @@ int do_expert_ffn_fp4(const moe_bf16* x, const void* packed4, const int32_t* off
     return do_expert_ffn(x, dq, offsets, perm_src, T, h, y, sms, s);
   }
   const uint8_t* p4 = static_cast<const uint8_t*>(packed4);
-  skinny::SegMaps maps{};
+  SegMaps maps{};
   int rc = make_tmap_u8(&maps.w1[0], p4, fp4::kGuRowBytes, uint64_t(kE) * 2 * kI, 64);
   if (!rc)
     rc = make_tmap_u8(&maps.w2[0], p4 + fp4::kGuBytes, fp4::kDRowBytes, uint64_t(kE) * kH, 64);
@@ -837,16 +850,16 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
   int32_t* sh_offsets = reinterpret_cast<int32_t*>(ws + L.sh_offsets);
   int32_t* sh_perm = reinterpret_cast<int32_t*>(ws + L.sh_perm);
   moe_bf16* sh_h = reinterpret_cast<moe_bf16*>(ws + L.sh_h);
-  if (!rc && !quant && n_shared > 0 && T <= kSkinnyMaxT) {
+  if (!rc && !quant && n_shared > 0) {
     // the routed experts and the shared experts as two segments of one launch
     rc = do_shared_rows(n_shared, T, sh_offsets, sh_perm, s);
-    skinny::SegMaps maps{};
-    skinny::SegPtrs p{};
+    SegMaps maps{};
+    SegPtrs p{};
     p.n = 2;
-    if (!rc) rc = skinny_maps(&maps, 0, packed_w, kE, kPackGuElems, h, T * kTopK);
+    if (!rc) rc = ffn_maps(&maps, 0, packed_w, kE, kPackGuElems, h, T * kTopK, T);
     if (!rc)
-      rc = skinny_maps(&maps, 1, packed_shared, n_shared, int64_t(n_shared) * kPackGuPerExpert,
-                       sh_h, int64_t(n_shared) * T);
+      rc = ffn_maps(&maps, 1, packed_shared, n_shared, int64_t(n_shared) * kPackGuPerExpert,
+                    sh_h, int64_t(n_shared) * T, T);
     p.offsets[0] = offsets;
     p.perm_src[0] = perm_src;
     p.h_out[0] = reinterpret_cast<uint16_t*>(h);
@@ -855,11 +868,7 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
     p.perm_src[1] = sh_perm;
     p.h_out[1] = reinterpret_cast<uint16_t*>(sh_h);
     p.y_out[1] = reinterpret_cast<uint16_t*>(y_sh);
-    if (!rc)
-      rc = launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps, p,
-                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
-                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+    if (!rc) rc = do_ffn_segments(maps, p, x, T, sms, s);
   } else {
     if (!rc) {
       if (quant && qfmt == 2)
@@ -1408,12 +1417,12 @@ int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
   int32_t* sh_offsets = reinterpret_cast<int32_t*>(ws + L.sh_offsets);
   int32_t* sh_perm = reinterpret_cast<int32_t*>(ws + L.sh_perm);
   moe_bf16* sh_h = reinterpret_cast<moe_bf16*>(ws + L.sh_h);
-  if (T <= kSkinnyMaxT) {
-    // one skinny launch over experts 0..127, 128..255 and the shared experts
-    // (three segments: each pack, its offsets, its rows)
+  {
+    // one launch over experts 0..127, 128..255 and the shared experts (three
+    // segments: each pack, its offsets, its rows)
     if (!rc && n_shared > 0) rc = do_shared_rows(n_shared, T, sh_offsets, sh_perm, s);
-    skinny::SegMaps maps{};
-    skinny::SegPtrs p{};
+    SegMaps maps{};
+    SegPtrs p{};
     const moe_bf16* packs[3] = {packed_lo, packed_hi, packed_shared};
     const int32_t* offs[3] = {off_lo, off_hi, sh_offsets};
     const int32_t* perms[3] = {perm_src, perm_src, sh_perm};
@@ -1421,25 +1430,16 @@ int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
     moe_bf16* ys[3] = {y, y, y_sh};
     p.n = n_shared > 0 ? 3 : 2;
     for (int g = 0; g < p.n && !rc; ++g) {
-      const int n_exp = g < 2 ? kE : n_shared;
-      rc = skinny_maps(&maps, g, packs[g], n_exp, g < 2 ? kPackGuElems : int64_t(n_shared) * kPackGuPerExpert,
-                       hs[g], g < 2 ? T * kTopK : int64_t(n_shared) * T);
+      const bool routed = g < 2;
+      rc = ffn_maps(&maps, g, packs[g], routed ? kE : n_shared,
+                    routed ? kPackGuElems : int64_t(n_shared) * kPackGuPerExpert, hs[g],
+                    routed ? T * kTopK : int64_t(n_shared) * T, T);
       p.offsets[g] = offs[g];
       p.perm_src[g] = perms[g];
       p.h_out[g] = reinterpret_cast<uint16_t*>(hs[g]);
       p.y_out[g] = reinterpret_cast<uint16_t*>(ys[g]);
     }
-    if (!rc)
-      rc = launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
-                      dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps, p,
-                      reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(off_lo, 1),
-                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
-  } else {
-    // experts 0..127 and 128..255: the 128-expert kernels on each half's pack
-    if (!rc) rc = do_expert_ffn(x, packed_lo, off_lo, perm_src, T, h, y, sms, s);
-    if (!rc) rc = do_expert_ffn(x, packed_hi, off_hi, perm_src, T, h, y, sms, s);
-    if (!rc && n_shared > 0)
-      rc = do_shared_ffn(x, packed_shared, n_shared, T, sh_offsets, sh_perm, sh_h, y_sh, sms, s);
+    if (!rc) rc = do_ffn_segments(maps, p, x, T, sms, s);
   }
   if (!rc)
     rc = launch_pdl("combine_kernel launch", combine_kernel<e256::kTopK2>,
