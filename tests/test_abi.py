@@ -20,7 +20,13 @@ def test_sizes():
     assert moe.packed_weight_bytes() == 128 * 3 * 1536 * 512 * 2
     assert moe.lib.moe_max_tokens() == 1 << 22
     assert moe.lib.moe_permute_workspace_bytes(1024) == 0
-    assert moe.lib.moe_permute_workspace_bytes(1025) == 9 * 128 * 4 + (256 - (9 * 128 * 4) % 256) % 256
+    # one histogram row of 128 experts per block: blocks of 64 tokens up to
+    # 16384 tokens, of 128 above; rounded up to 256 bytes
+    def ws(blocks):
+        return blocks * 128 * 4 + (256 - (blocks * 128 * 4) % 256) % 256
+    assert moe.lib.moe_permute_workspace_bytes(1025) == ws(17)
+    assert moe.lib.moe_permute_workspace_bytes(16384) == ws(256)
+    assert moe.lib.moe_permute_workspace_bytes(16385) == ws(129)
     assert moe.lib.moe_permute_workspace_bytes(-1) == 0
     prev = 0
     for T in (1, 4, 16, 2048, 8192):
