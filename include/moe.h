@@ -518,9 +518,11 @@ size_t moe_layer_shared_workspace_bytes(int64_t T, int n_shared, int fp8_routed)
 /* moe_layer (packed_w, bf16 routed experts) or moe_layer_fp8 (packed_fp8):
  * exactly one of the two is non-NULL; plus n_shared (0..8) shared experts
  * from packed_shared.  The shared experts' rows (every token once per shared
- * expert) go through the same grouped expert-FFN kernels as the routed ones,
- * in a second launch; the combine adds their outputs.  With n_shared = 0 the
- * result is bit for bit that of moe_layer / moe_layer_fp8. */
+ * expert) go through the same grouped expert-FFN kernels as the routed ones:
+ * with bf16 routed experts as a second weight pack of the routed experts'
+ * launch, with block-FP8 or NVFP4 routed experts in a second launch; the
+ * combine adds their outputs.  With n_shared = 0 the result is bit for bit
+ * that of moe_layer / moe_layer_fp8. */
 int moe_layer_shared(const moe_bf16* x, const float* logits, const float* bias,
                      const moe_bf16* packed_w, const void* packed_fp8,
                      const moe_bf16* packed_shared, int n_shared, int64_t T,
@@ -584,9 +586,10 @@ size_t moe_layer_e256_workspace_bytes(int64_t T, int n_shared);
 /* The whole layer on the second shape: routing, a stable counting sort over
  * the 256 experts, the grouped expert FFN of experts 0..127 (packed_lo) and
  * 128..255 (packed_hi) -- each packed by moe_pack_weights from that half's
- * [128][...] weights -- in two launches of the 128-expert kernels, the
- * n_shared (0..8) shared experts of packed_shared (moe_pack_shared), and the
- * combine:
+ * [128][...] weights -- and of the n_shared (0..8) shared experts of
+ * packed_shared (moe_pack_shared), all three packs in one launch of the
+ * 128-expert kernels, and the combine (up to 64 tokens the routing and the
+ * sort are one launch):
  *   out[t] = bf16( residual[t] + sum_{slot < 6} w[t,slot] FFN_{e_slot}(x[t]) + sum_s FFN_s(x[t]) ).
  * topk_idx_out / topk_w_out: optional [T][6]. */
 int moe_layer_e256(const moe_bf16* x, const float* logits, const float* bias,
