@@ -52,10 +52,6 @@
 //   next warp  MMA issuer: tcgen05.mma 128x256x16, accumulator in TMEM,
 //              double-buffered (2 x 256 columns) so the epilogue of tile i
 //              overlaps the MMAs of tile i+1.
-// One launch can run up to kMaxSeg weight packs ("segments", see common.cuh):
-// each has its own tensor maps, offsets array, row sources and h / y_perm
-// rows, and tile ids run over every segment's gate/up tiles, then every
-// segment's down tiles.
 // Shared-memory ring: 4 stages of (A 128x64 + B 256x64) 16-bit elements.
 // The epilogue transposes each warp's 32 x 32 fp16 block through a padded
 // shared tile so that global stores are whole 64-byte row segments.
