@@ -148,13 +148,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "memory");
   return v;
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // ---------------------------------------------------------------- TMA
 
@@ -227,68 +220,6 @@ __device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Eight MMAs over K = 128 with A in tensor memory (columns a_tmem + 8k) and B
-// as two 64-wide SW128 tiles (descriptors b0 for k < 4, b1 for k >= 4, each
-// advanced by 32 bytes per k); the first accumulates into D only if
-// `accumulate`, the other seven always.
-__device__ __forceinline__ void umma_f16_ta_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
-                                                 uint64_t b1, uint32_t idesc,
-                                                 uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "setp.eq.b32 q, %5, %5;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
-      "add.u32 a, %1, 8;\n\tadd.u64 b, %2, 2;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
-      "add.u32 a, %1, 16;\n\tadd.u64 b, %2, 4;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
-      "add.u32 a, %1, 24;\n\tadd.u64 b, %2, 6;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
-      "add.u32 a, %1, 32;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %3, %4, q;\n\t"
-      "add.u32 a, %1, 40;\n\tadd.u64 b, %3, 2;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
-      "add.u32 a, %1, 48;\n\tadd.u64 b, %3, 4;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t"
-      "add.u32 a, %1, 56;\n\tadd.u64 b, %3, 6;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, q;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Eight MMAs over K = 128 as umma_f16_ta_k128, with MMA k accumulating into
-// d[k % 4]: four independent accumulator chains, so that an MMA never waits for
-// the one issued just before it to finish with its accumulator (one chain of
-// dependent M = 128, N = 32 MMAs runs at about a quarter of the rate of four).
-// The first four accumulate only if `accumulate`, the other four always.
-__device__ __forceinline__ void umma_f16_ta_k128_4acc(uint32_t d0, uint32_t d1, uint32_t d2,
-                                                      uint32_t d3, uint32_t a_tmem, uint64_t b0,
-                                                      uint64_t b1, uint32_t idesc,
-                                                      uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
-      "setp.ne.b32 p, %8, 0;\n\t"
-      "setp.eq.b32 q, %8, %8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %5, %7, p;\n\t"
-      "add.u32 a, %4, 8;\n\tadd.u64 b, %5, 2;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, p;\n\t"
-      "add.u32 a, %4, 16;\n\tadd.u64 b, %5, 4;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [a], b, %7, p;\n\t"
-      "add.u32 a, %4, 24;\n\tadd.u64 b, %5, 6;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%3], [a], b, %7, p;\n\t"
-      "add.u32 a, %4, 32;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %6, %7, q;\n\t"
-      "add.u32 a, %4, 40;\n\tadd.u64 b, %6, 2;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, q;\n\t"
-      "add.u32 a, %4, 48;\n\tadd.u64 b, %6, 4;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [a], b, %7, q;\n\t"
-      "add.u32 a, %4, 56;\n\tadd.u64 b, %6, 6;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%3], [a], b, %7, q;\n\t}" ::"r"(d0),
-      "r"(d1), "r"(d2), "r"(d3), "r"(a_tmem), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -341,22 +272,6 @@ __device__ __forceinline__ void tmem_ld_2x32(uint32_t taddr0, uint32_t taddr1, u
       : "memory");
 }
 
-// One load of 32 consecutive fp32 columns of the calling warp's 32 TMEM lanes.
-__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&a)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
-        "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]),
-        "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]),
-        "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]),
-        "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
-      : "r"(taddr)
-      : "memory");
-}
-
 // Stores 32 consecutive 32-bit columns of the calling warp's 32 TMEM lanes
 // (one lane per thread), asynchronously: tmem_wait_st() waits for them.
 __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* a) {
@@ -373,11 +288,6 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* a) {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// Barrier among `nthreads` threads (multiple of 32) of the block, id 1..15.
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ void st_global_b16(void* p, uint16_t v) {
