@@ -100,7 +100,11 @@ def load_peaks():
 # (weights-as-M) kernel of smaller ones with its bf16, FP8 and NVFP4 forms.
 WIDE_SOURCES = ("common.cuh", "expert_ffn.cuh")
 SKINNY_SOURCES = ("common.cuh", "expert_ffn.cuh", "expert_ffn_skinny.cuh", "fp8.cuh", "fp4.cuh",
-                  "pack.cuh")
+                  "pack.cuh", "combine.cuh")
+# Up to this many tokens the expert-FFN launch of a layer also runs its combine
+# (kFusedCombineMaxT in csrc/combine.cuh), except beside a separate
+# shared-expert launch (quantised routed experts with shared experts).
+FUSED_COMBINE_MAX_T = 1
 
 
 def kernel_sources(workload: str):
@@ -231,10 +235,12 @@ class LayerRun:
         # moe_layer launches: route + permute (one fused kernel up to 64 tokens;
         # route and one permute kernel up to 1024; route, count and fused scan/scatter
         # up to 256 blocks of 128 tokens; route, count, scan, scatter beyond), the
-        # expert FFN (gate/up and down in one launch), combine
+        # expert FFN (gate/up and down in one launch), combine (inside the FFN
+        # launch up to FUSED_COMBINE_MAX_T tokens)
         nb = (T + 127) // 128
         n_rp = 1 if T <= 64 else 2 if T <= 1024 else (3 if nb <= 256 else 4)
-        self.launches_per_step = n_rp + 2  # + the expert FFN (one launch) + combine
+        fused = T <= FUSED_COMBINE_MAX_T and not (quant and shared is not None)
+        self.launches_per_step = n_rp + 1 + (0 if fused else 1)
         fws = moe.lib.moe_expert_ffn_fp8_workspace_bytes(T) if quant else 0
         self.ffn_ws = torch.empty(fws, dtype=torch.uint8, device=dev) if fws else None
         if fws:
@@ -247,7 +253,9 @@ class LayerRun:
             raw = torch.empty(n + 1024, dtype=torch.uint8, device=dev)
             off = (-raw.data_ptr()) % 1024
             self.lws = raw[off:off + n]
-            self.launches_per_step += 2  # the shared row set and the shared experts' FFN
+            # the shared row set; with quantised routed experts also the shared
+            # experts' own FFN launch (bf16: a second segment of the routed launch)
+            self.launches_per_step += 2 if quant else 1
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         self.read_buf = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
         self.write_only_flush = False
@@ -946,7 +954,8 @@ def stack_line(T, dev, packs, steps, warmup, peaks, barrier, routers=None):
                      "the combine), no host sync between layers; no L2 flush (each step streams "
                      f"{nbytes / 1e9:.2f} GB of expert weights)"),
             "status_ok": status == moe.MOE_OK,
-            "gpu_launches": (n_rp + 2) * STACK_LAYERS * steps, "clocks": clk.summary()}
+            "gpu_launches": (n_rp + (1 if T <= FUSED_COMBINE_MAX_T else 2)) * STACK_LAYERS * steps,
+            "clocks": clk.summary()}
 
 
 def fp8_layer(dev):
@@ -1087,8 +1096,10 @@ def run_ours(args):
     if not args.no_stack:
         packs = stack_packs(dev)
         routers = stack_routers(dev)
-        for T_s, key, rt in ((1, "stack23_T1", None), (8189, "stack23_T8189", None),
-                             (1, "stack23_T1_routed", routers),
+        # both decode stacks first: right after a prefill stack the SM clock was
+        # seen settling below its maximum for a while
+        for T_s, key, rt in ((1, "stack23_T1", None), (1, "stack23_T1_routed", routers),
+                             (8189, "stack23_T8189", None),
                              (8189, "stack23_T8189_routed", routers)):
             n = max(10, args.steps // 2) if T_s == 1 else max(5, args.steps // 10)
             line[key] = stack_line(T_s, dev, packs, n, args.warmup, peaks, barrier, routers=rt)

@@ -17,21 +17,36 @@ namespace moe {
 
 constexpr int kCombineThreads = kH / 8;  // 192
 
-// NS: slots a token uses (8, or 6 in the 256-expert shape); topk_w has NS
-// entries per token, inv_perm always kTopK (slots NS .. 7 unused).
-template <int NS>
-__global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const uint16_t* __restrict__ y_perm, const float* __restrict__ topk_w,
-                   const int32_t* __restrict__ inv_perm, int64_t T,
-                   const __nv_bfloat16* residual, __nv_bfloat16* out,
-                   const uint16_t* __restrict__ y_shared, int n_shared) {
-  griddep_launch_dependents();
-  griddep_wait();
-  const int64_t t = blockIdx.x;
-  if (t >= T) return;
-  const int col = threadIdx.x * 8;
-  const int64_t nrows = T * kTopK;
+// The combine run at the end of a single-launch expert FFN by the CTA that
+// retires last, in place of a combine launch: up to kFusedCombineMaxT tokens.
+// One token's 192 output vectors are one pass of one CTA, and the layer is
+// about 1 us faster than with the combine launch; two tokens (two passes)
+// measured slower than the launch.  y_perm is segment 0's y rows, the shared
+// rows (n_shared > 0) segment 1's.  out == nullptr: no combine in the launch.
+constexpr int kFusedCombineMaxT = 1;
+struct FusedCombine {
+  const float* topk_w;
+  const int32_t* inv_perm;
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* out;
+  int n_shared;
+};
 
+// out[t][col .. col + 7] for token t (one thread, one 16-byte vector), the
+// arithmetic of the whole file comment.  NS: slots a token uses (8, or 6 in the
+// 256-expert shape); topk_w has NS entries per token, inv_perm always kTopK
+// (slots NS .. 7 unused).  L2_ONLY: y_perm was written by the calling kernel
+// itself (and so were the shared rows), so both are read around the
+// non-coherent cache.
+template <int NS, bool L2_ONLY = false>
+__device__ __forceinline__ void combine_token_vec(const uint16_t* __restrict__ y_perm,
+                                                  const float* __restrict__ topk_w,
+                                                  const int32_t* __restrict__ inv_perm, int64_t T,
+                                                  int64_t t, int col, const __nv_bfloat16* residual,
+                                                  __nv_bfloat16* out,
+                                                  const uint16_t* __restrict__ y_shared,
+                                                  int n_shared) {
+  const int64_t nrows = T * kTopK;
   uint4 v[NS];
   float w[NS];
 #pragma unroll
@@ -39,7 +54,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     const int64_t r = __ldg(inv_perm + t * kTopK + s);
     w[s] = __ldg(topk_w + t * NS + s);
     if (r >= 0 && r < nrows) {
-      v[s] = __ldg(reinterpret_cast<const uint4*>(y_perm + r * kH + col));
+      const uint4* src = reinterpret_cast<const uint4*>(y_perm + r * kH + col);
+      v[s] = L2_ONLY ? __ldcg(src) : __ldg(src);
     } else {
       v[s] = make_uint4(0u, 0u, 0u, 0u);
       w[s] = 0.f;
@@ -58,7 +74,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     }
   }
   for (int s = 0; s < n_shared; ++s) {
-    const uint4 sv = __ldg(reinterpret_cast<const uint4*>(y_shared + (s * T + t) * kH + col));
+    const uint4* src = reinterpret_cast<const uint4*>(y_shared + (s * T + t) * kH + col);
+    const uint4 sv = L2_ONLY ? __ldcg(src) : __ldg(src);
     const uint32_t q[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -81,6 +98,20 @@ __global__ void __launch_bounds__(kCombineThreads)
   o.z = pack_bf16x2(acc[4], acc[5]);
   o.w = pack_bf16x2(acc[6], acc[7]);
   *reinterpret_cast<uint4*>(out + t * kH + col) = o;
+}
+
+template <int NS>
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const uint16_t* __restrict__ y_perm, const float* __restrict__ topk_w,
+                   const int32_t* __restrict__ inv_perm, int64_t T,
+                   const __nv_bfloat16* residual, __nv_bfloat16* out,
+                   const uint16_t* __restrict__ y_shared, int n_shared) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t t = blockIdx.x;
+  if (t >= T) return;
+  combine_token_vec<NS>(y_perm, topk_w, inv_perm, T, t, threadIdx.x * 8, residual, out,
+                        y_shared, n_shared);
 }
 
 }  // namespace moe

@@ -29,6 +29,9 @@
 // wait ends however many CTAs of the grid are resident.  SMs that finish their last
 // gate/up tile go straight on to down tiles of experts that are ready instead
 // of idling until the slowest gate/up tile ends and a second launch ramps up.
+// For a single token the layer's combine also runs in this launch: the CTA
+// whose retirement completes the grid's count has every y row behind it and
+// writes the layer's output, one kernel boundary fewer on the decode path.
 //
 // Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31), 4 token gather (phase 1:
 // cp.async of x rows by perm_src, barrier-tracked; padding rows kept at zero),
@@ -59,6 +62,7 @@
 // copy; a converter thread turns 64 codes of its row into 32 columns of
 // bf16 (gate/up) or fp16 (down) pairs with the integer route of fp4.cuh.
 #pragma once
+#include "combine.cuh"
 #include "common.cuh"
 #include "expert_ffn.cuh"
 #include "fp4.cuh"
@@ -162,6 +166,7 @@ struct Tail {
   TileQueue tq;
   uint32_t tmem_base;
   int abort_flag;
+  int last_cta;  // this CTA retired last (it runs the fused combine)
   int wsum[4];
   int segbase[kMaxSeg + 1];       // exclusive prefix of the segments' chunk counts
   int cstart[kMaxSeg][kE + 1];    // per segment: exclusive prefix of the experts' 32-token chunks
@@ -211,7 +216,8 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
                        const __nv_bfloat16* __restrict__ x, int64_t T, int* __restrict__ sched,
                        const void* __restrict__ wscale,  // FP8 scales (SGU, SD) or FP4 MGU, MD
                        uint64_t timeout_ns,
-                       uint64_t* __restrict__ trace) {  // NULL, or 3 words per CTA (see ffn_trace)
+                       uint64_t* __restrict__ trace,  // NULL, or 3 words per CTA (see ffn_trace)
+                       const __grid_constant__ FusedCombine cmb) {
   constexpr bool HAS1 = MODE != 2, HAS2 = MODE != 1;
   const int nseg = seg.n;
   // segment g's per-expert done counters (single-launch form only)
@@ -717,6 +723,11 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     if (range_bad) record_status(kSiteFp16Range);
   }
 
+  // Fused combine: every storing thread fences its y stores before the CTA
+  // counts itself retired, the last CTA fences after seeing the final count,
+  // so it reads every CTA's y rows.
+  const bool fuse = MODE == 3 && cmb.out != nullptr;
+  if (fuse && warp < 4) __threadfence();
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -725,10 +736,25 @@ __global__ void __launch_bounds__(Ring<WQ>::THREADS, 1)
     if (MODE == 3 && last)  // the other segments' done counters too
       for (int g = 1; g < nseg; ++g)
         for (int i = 0; i < kE; ++i) atomicExch(done_of(g) + i, 0);
+    if (fuse && last) __threadfence();
+    S->last_cta = last;
   }
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, R::TMEM_COLS);
+  }
+  if (fuse) {
+    __syncthreads();
+    if (S->last_cta) {
+      const uint16_t* y_shared = cmb.n_shared > 0 ? seg.y_out[1] : nullptr;
+      const int64_t nvec = T * kCombineThreads;
+      for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+        const int64_t t = v / kCombineThreads;
+        const int col = static_cast<int>(v - t * kCombineThreads) * 8;
+        combine_token_vec<kTopK, true>(seg.y_out[0], cmb.topk_w, cmb.inv_perm, T, t, col,
+                                       cmb.residual, cmb.out, y_shared, cmb.n_shared);
+      }
+    }
   }
 }
 

@@ -367,7 +367,8 @@ int do_gate_up(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets
                       dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps,
                       one_segment(offsets, perm_src, h, nullptr),
                       reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
-                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms),
+                      FusedCombine{});
   }
   SegMaps maps{};
   int rc = make_tmap(&maps.w1[0], packed, kH, uint64_t(kE) * 2 * kI, ffn::BN,
@@ -394,7 +395,8 @@ int do_down(const moe_bf16* h, const moe_bf16* packed, const int32_t* offsets, i
                       dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps,
                       one_segment(offsets, nullptr, nullptr, y),
                       static_cast<const __nv_bfloat16*>(nullptr), T, sched_words(offsets, 2),
-                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms));
+                      static_cast<const void*>(nullptr), g_timeout_ns.load(), ffn_trace(sms),
+                      FusedCombine{});
   }
   SegMaps maps{};
   int rc = make_tmap(&maps.w2[0], packed + kPackGuElems, kI, uint64_t(kE) * kH, ffn::BN,
@@ -443,15 +445,16 @@ int ffn_maps(SegMaps* maps, int g, const moe_bf16* packed, int n_exp, int64_t d_
 }
 
 // The single-launch expert FFN over the segments p (maps from ffn_maps); the
-// tile counters are segment 0's.
+// tile counters are segment 0's.  cmb.out != nullptr (T <= kFusedCombineMaxT
+// only): the launch also runs the layer's combine.
 int do_ffn_segments(const SegMaps& maps, const SegPtrs& p, const moe_bf16* x, int64_t T, int sms,
-                    cudaStream_t s) {
+                    cudaStream_t s, const FusedCombine& cmb = FusedCombine{}) {
   const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   if (T <= kSkinnyMaxT)
     return launch_pdl("skinny_gemm_kernel<3> launch", skinny::skinny_gemm_kernel<3>, dim3(sms),
                       dim3(skinny::THREADS), skinny::SMEM_BYTES, s, maps, p, xb, T,
                       sched_words(p.offsets[0], 1), static_cast<const void*>(nullptr),
-                      g_timeout_ns.load(), ffn_trace(sms));
+                      g_timeout_ns.load(), ffn_trace(sms), cmb);
   return launch_pdl("ffn_gemm_kernel<3> launch",
                     T <= kZeroPadMaxT ? ffn::ffn_gemm_kernel<3, true> : ffn::ffn_gemm_kernel<3, false>,
                     dim3(sms), dim3(ffn::Cfg<3>::THREADS), ffn::SMEM_BYTES, s, maps, p, xb, T,
@@ -464,13 +467,13 @@ int do_ffn_segments(const SegMaps& maps, const SegPtrs& p, const moe_bf16* x, in
 int do_expert_ffn(const moe_bf16* x, const moe_bf16* packed, const int32_t* offsets,
                   const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, int sms,
                   cudaStream_t s, int n_exp = kE, int64_t d_off = kPackGuElems,
-                  int64_t h_rows = -1) {
+                  int64_t h_rows = -1, const FusedCombine& cmb = FusedCombine{}) {
   if (h_rows < 0) h_rows = T * kTopK;
   // both GEMMs in one launch (see expert_ffn_skinny.cuh, expert_ffn.cuh)
   SegMaps maps{};
   int rc = ffn_maps(&maps, 0, packed, n_exp, d_off, h, h_rows, T);
   if (rc) return rc;
-  return do_ffn_segments(maps, one_segment(offsets, perm_src, h, y), x, T, sms, s);
+  return do_ffn_segments(maps, one_segment(offsets, perm_src, h, y), x, T, sms, s, cmb);
 }
 
 // Packed block-FP8 layer -> packed bf16/fp16 layer.
@@ -487,7 +490,7 @@ int do_dequant_fp8(const void* packed8, moe_bf16* packed, int sms, cudaStream_t 
 // `dq` (moe_packed_weight_bytes) and run by the bf16 kernel.
 int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* offsets,
                       const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, moe_bf16* dq,
-                      int sms, cudaStream_t s) {
+                      int sms, cudaStream_t s, const FusedCombine& cmb = FusedCombine{}) {
   if (T > kSkinnyMaxT) {
     int rc = do_dequant_fp8(packed8, dq, sms, s);
     if (rc) return rc;
@@ -504,7 +507,8 @@ int do_expert_ffn_fp8(const moe_bf16* x, const void* packed8, const int32_t* off
                     dim3(sms), dim3(skinny::Ring<1>::THREADS), skinny::SMEM_BYTES, s, maps,
                     one_segment(offsets, perm_src, h, y),
                     reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
-                    static_cast<const void*>(p8 + fp8::kSguOff), g_timeout_ns.load(), ffn_trace(sms));
+                    static_cast<const void*>(p8 + fp8::kSguOff), g_timeout_ns.load(), ffn_trace(sms),
+                    cmb);
 }
 
 // Packed NVFP4 layer -> packed bf16/fp16 layer.
@@ -518,7 +522,7 @@ int do_dequant_fp4(const void* packed4, moe_bf16* packed, int sms, cudaStream_t 
 // per-16 block multipliers in the skinny kernel up to kSkinnyMaxT tokens.
 int do_expert_ffn_fp4(const moe_bf16* x, const void* packed4, const int32_t* offsets,
                       const int32_t* perm_src, int64_t T, moe_bf16* h, moe_bf16* y, moe_bf16* dq,
-                      int sms, cudaStream_t s) {
+                      int sms, cudaStream_t s, const FusedCombine& cmb = FusedCombine{}) {
   if (T > kSkinnyMaxT) {
     int rc = do_dequant_fp4(packed4, dq, sms, s);
     if (rc) return rc;
@@ -536,7 +540,8 @@ int do_expert_ffn_fp4(const moe_bf16* x, const void* packed4, const int32_t* off
                     dim3(sms), dim3(skinny::Ring<2>::THREADS), skinny::SMEM_BYTES, s, maps,
                     one_segment(offsets, perm_src, h, y),
                     reinterpret_cast<const __nv_bfloat16*>(x), T, sched_words(offsets, 1),
-                    static_cast<const void*>(p4 + fp4::kMguOff), g_timeout_ns.load(), ffn_trace(sms));
+                    static_cast<const void*>(p4 + fp4::kMguOff), g_timeout_ns.load(), ffn_trace(sms),
+                    cmb);
 }
 
 int do_combine(const moe_bf16* y, const float* w, const int32_t* inv, int64_t T,
@@ -846,6 +851,13 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
       rc = do_route_permute(logits, bias, T, idx, w, counts, offsets, perm_src, inv_perm,
                             ws + L.perm_ws, s);
   }
+  // A single token: the FFN launch runs the combine too (not with a
+  // separate shared-expert launch, which the combine must follow).
+  const bool fused = T <= kFusedCombineMaxT && !(quant && n_shared > 0);
+  FusedCombine cmb{};
+  if (fused)
+    cmb = FusedCombine{w, inv_perm, reinterpret_cast<const __nv_bfloat16*>(residual),
+                       reinterpret_cast<__nv_bfloat16*>(out), n_shared};
   moe_bf16* y_sh = reinterpret_cast<moe_bf16*>(ws + L.sh_y);
   int32_t* sh_offsets = reinterpret_cast<int32_t*>(ws + L.sh_offsets);
   int32_t* sh_perm = reinterpret_cast<int32_t*>(ws + L.sh_perm);
@@ -868,22 +880,23 @@ int layer_impl(const char* fn, const moe_bf16* x, const float* logits,
     p.perm_src[1] = sh_perm;
     p.h_out[1] = reinterpret_cast<uint16_t*>(sh_h);
     p.y_out[1] = reinterpret_cast<uint16_t*>(y_sh);
-    if (!rc) rc = do_ffn_segments(maps, p, x, T, sms, s);
+    if (!rc) rc = do_ffn_segments(maps, p, x, T, sms, s, cmb);
   } else {
     if (!rc) {
       if (quant && qfmt == 2)
         rc = do_expert_ffn_fp4(x, packed_q, offsets, perm_src, T, h, y,
-                               reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
+                               reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s, cmb);
       else if (quant)
         rc = do_expert_ffn_fp8(x, packed_q, offsets, perm_src, T, h, y,
-                               reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s);
+                               reinterpret_cast<moe_bf16*>(ws + L.dq), sms, s, cmb);
       else
-        rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s);
+        rc = do_expert_ffn(x, packed_w, offsets, perm_src, T, h, y, sms, s, kE, kPackGuElems, -1,
+                           cmb);
     }
     if (!rc && n_shared > 0)
       rc = do_shared_ffn(x, packed_shared, n_shared, T, sh_offsets, sh_perm, sh_h, y_sh, sms, s);
   }
-  if (!rc) rc = do_combine(y, w, inv_perm, T, residual, out, s, y_sh, n_shared);
+  if (!rc && !fused) rc = do_combine(y, w, inv_perm, T, residual, out, s, y_sh, n_shared);
   return rc;
 }
 }  // namespace

@@ -284,7 +284,11 @@ int moe_route_from_x(const moe_bf16* x, const moe_bf16* packed_router, const flo
 size_t moe_layer_workspace_bytes(int64_t T);
 
 /* The whole layer: route -> permute -> expert FFN -> combine, back to back on
- * `stream` with no host synchronisation.  Arguments as in the steps above;
+ * `stream` with no host synchronisation.  For a single token the combine
+ * runs at the end of the expert-FFN launch (by its CTA that retires last, with
+ * the arithmetic of moe_combine, bit for bit), one launch fewer; this holds for
+ * every layer call below except quantised routed experts with shared experts.
+ * Arguments as in the steps above;
  *   residual   : NULL, or [T][1536] bf16 added before the final rounding
  *                (a stack layer computes h <- bf16(h + moe(h)) with
  *                residual = x = out allowed)
@@ -299,8 +303,8 @@ int moe_layer(const moe_bf16* x, const float* logits, const float* bias,
  * from x into the workspace (same workspace size as moe_layer), then route ->
  * permute -> expert FFN -> combine as above.  Up to 8 tokens the projection,
  * routing and the sort are one launch (as in moe_route_from_x), so the layer
- * is three launches like moe_layer; above, moe_router's tensor-core
- * projection runs first. */
+ * is as many launches as moe_layer (two for one token, three up to 8);
+ * above, moe_router's tensor-core projection runs first. */
 int moe_layer_routed(const moe_bf16* x, const moe_bf16* packed_router, const float* bias,
                      const moe_bf16* packed_w, int64_t T, const moe_bf16* residual,
                      moe_bf16* out, int32_t* topk_idx_out, float* topk_w_out,
