@@ -286,8 +286,10 @@ size_t moe_layer_workspace_bytes(int64_t T);
 /* The whole layer: route -> permute -> expert FFN -> combine, back to back on
  * `stream` with no host synchronisation.  For a single token the combine
  * runs at the end of the expert-FFN launch (by its CTA that retires last, with
- * the arithmetic of moe_combine, bit for bit), one launch fewer; this holds for
- * every layer call below except quantised routed experts with shared experts.
+ * the arithmetic of moe_combine, bit for bit), one launch fewer.  The same
+ * holds for moe_layer_routed, moe_layer_fp8, moe_layer_nvfp4, moe_layer_host
+ * and moe_layer_shared with bf16 routed experts; moe_layer_e256 and the
+ * quantised layers with shared experts keep the combine launch.
  * Arguments as in the steps above;
  *   residual   : NULL, or [T][1536] bf16 added before the final rounding
  *                (a stack layer computes h <- bf16(h + moe(h)) with
