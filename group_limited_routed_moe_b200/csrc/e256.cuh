@@ -14,6 +14,7 @@
 // perm_src >> 3 and the combine's inv_perm stride stay as they are.
 #pragma once
 #include "common.cuh"
+#include "permute.cuh"
 #include "route.cuh"
 
 namespace moe {
@@ -261,8 +262,8 @@ __global__ void __launch_bounds__(256)
   griddep_launch_dependents();
   griddep_wait();
   const int e = threadIdx.x, lane = e & 31, w = e >> 5;
-  int c = 0;
-  for (int b = 0; b < nb; ++b) c += hist[static_cast<int64_t>(b) * kE2 + e];
+  int c = 0, unused = 0;
+  hist_column_sum(hist, kE2, e, 0, nb, 1, 0, c, unused);
   int incl = c;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -277,13 +278,7 @@ __global__ void __launch_bounds__(256)
   counts[e] = c;
   offsets[e] = start;
   if (e == kE2 - 1) offsets[kE2] = start + c;
-  int run = start;
-  for (int b = 0; b < nb; ++b) {
-    const int64_t i = static_cast<int64_t>(b) * kE2 + e;
-    const int v = hist[i];
-    hist[i] = run;
-    run += v;
-  }
+  hist_column_exclusive(hist, kE2, e, 0, nb, start);
   // halves: absolute rows, then zeroed work counters
   const int half = e >> 7, j = e & 127;
   int32_t* dst = half ? off_hi : off_lo;

@@ -39,6 +39,60 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
+// Walks down one expert's column of a per-block histogram hist[b][e] (row
+// length ld) with kHistBatch loads in flight per thread.  The column's words
+// are independent, so a plain loop would pay an L2 round trip per block; in
+// the fused scan + scatter a thread walks 32 blocks at T=8189, in the
+// separate scan up to 4096.  Integer sums, so the order changes nothing.
+constexpr int kHistBatch = 8;
+
+// tot += hist[b][e] and, for b < lim, bef += hist[b][e], over b = b0, b0 +
+// step, ... < b1.
+__device__ __forceinline__ void hist_column_sum(const int32_t* __restrict__ hist, int ld, int e,
+                                                int b0, int b1, int step, int lim, int& tot,
+                                                int& bef) {
+  int b = b0;
+  for (; b + (kHistBatch - 1) * step < b1; b += kHistBatch * step) {
+    int v[kHistBatch];
+#pragma unroll
+    for (int u = 0; u < kHistBatch; ++u) v[u] = hist[static_cast<int64_t>(b + u * step) * ld + e];
+#pragma unroll
+    for (int u = 0; u < kHistBatch; ++u) {
+      tot += v[u];
+      if (b + u * step < lim) bef += v[u];
+    }
+  }
+  for (; b < b1; b += step) {
+    const int v = hist[static_cast<int64_t>(b) * ld + e];
+    tot += v;
+    if (b < lim) bef += v;
+  }
+}
+
+// hist[b][e] <- run, then run += its old value, for b = b0 .. b1 - 1 in order
+// (the column's exclusive prefix sum from run); returns the final run.
+__device__ __forceinline__ int hist_column_exclusive(int32_t* __restrict__ hist, int ld, int e,
+                                                     int b0, int b1, int run) {
+  int b = b0;
+  for (; b + kHistBatch <= b1; b += kHistBatch) {
+    int v[kHistBatch];
+#pragma unroll
+    for (int u = 0; u < kHistBatch; ++u) v[u] = hist[static_cast<int64_t>(b + u) * ld + e];
+#pragma unroll
+    for (int u = 0; u < kHistBatch; ++u) {
+      hist[static_cast<int64_t>(b + u) * ld + e] = run;
+      run += v[u];
+    }
+  }
+  for (; b < b1; ++b) {
+    const int64_t i = static_cast<int64_t>(b) * ld + e;
+    const int v = hist[i];
+    hist[i] = run;
+    run += v;
+  }
+  return run;
+}
+
 // Exclusive scan of cnt[0..127] into off[0..128], run by warp 0 only.
 __device__ __forceinline__ void scan_experts_warp0(const int* cnt, int* off, int lane) {
   const int c0 = cnt[4 * lane], c1 = cnt[4 * lane + 1], c2 = cnt[4 * lane + 2],
@@ -153,19 +207,14 @@ __global__ void __launch_bounds__(1024)
   const int tid = threadIdx.x, e = tid % kE, part = tid / kE, lane = tid & 31;
   const int per = (nb + kParts - 1) / kParts;
   const int b0 = min(nb, part * per), b1 = min(nb, b0 + per);
-  int s = 0;
-  for (int b = b0; b < b1; ++b) s += hist[static_cast<int64_t>(b) * kE + e];
+  int s = 0, unused = 0;
+  hist_column_sum(hist, kE, e, b0, b1, 1, 0, s, unused);
   part_sum[part][e] = s;
   __syncthreads();
   int run = 0;
   for (int p = 0; p < part; ++p) run += part_sum[p][e];
   if (part == kParts - 1) cnt[e] = run + s;
-  for (int b = b0; b < b1; ++b) {
-    const int64_t i = static_cast<int64_t>(b) * kE + e;
-    const int h = hist[i];
-    hist[i] = run;
-    run += h;
-  }
+  hist_column_exclusive(hist, kE, e, b0, b1, run);
   __syncthreads();
   if (tid < 32) scan_experts_warp0(cnt, off, lane);
   __syncthreads();
@@ -208,11 +257,7 @@ __global__ void __launch_bounds__(kPermScanThreads)
   {  // column sums: thread (h, e) sums blocks h, h + kPermScanParts, ...
     const int e = tid & (kE - 1), h = tid >> 7;
     int tot = 0, bef = 0;
-    for (int bb = h; bb < nb; bb += kPermScanParts) {
-      const int v = hist[static_cast<int64_t>(bb) * kE + e];
-      tot += v;
-      if (bb < b) bef += v;
-    }
+    hist_column_sum(hist, kE, e, h, nb, kPermScanParts, b, tot, bef);
     part[h][e] = tot;
     before_s[h][e] = bef;
   }
