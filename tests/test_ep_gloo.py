@@ -13,7 +13,9 @@ grouped expert FFN and the source's combine), passed explicitly as
     of every token that routed to one of its experts, with the right local
     ids, and the layer output reassembled from the returned rows equals the
     oracle's layer on the rank's own tokens (same float64 arithmetic in
-    another summation order: relative 1e-12).
+    another summation order: relative 1e-12);
+  - edge cases: an empty batch, one rank holding every expert, and a rank
+    without tokens that still serves the rows routed to its experts.
 """
 import os
 
@@ -186,3 +188,38 @@ def test_gloo_two_ranks_exchange():
         assert exc is None, f"rank {rank}: {exc}"
         assert ok_rows, f"rank {rank} received the wrong rows"
         assert err <= 1e-12, f"rank {rank}: rel-L2 {err}"
+
+
+def test_plan_empty_batch_and_one_rank():
+    """No tokens: every count is zero and every index array empty.  One rank
+    (W = 1) owns all 128 experts: every token is one row whose local ids are
+    its expert ids, and the returned rows come back in item order."""
+    for W in (2, 8):
+        p = ep.plan_dispatch(torch.zeros((0, 8), dtype=torch.int32), W)
+        assert p.send_counts.tolist() == [0] * W and p.ret_counts.tolist() == [0] * W
+        assert p.send_tok.numel() == 0 and p.send_local.shape == (0, 8)
+        assert p.ret_index.numel() == 0
+    tok, rr = _tokens(0)
+    p = ep.plan_dispatch(torch.from_numpy(rr.topk_idx), 1)
+    assert p.send_counts.tolist() == [T_PER_RANK] and p.ret_counts.tolist() == [T_PER_RANK * 8]
+    assert p.send_tok.tolist() == list(range(T_PER_RANK))
+    np.testing.assert_array_equal(p.send_local.numpy(), rr.topk_idx)
+    np.testing.assert_array_equal(p.ret_index.numpy(), np.arange(T_PER_RANK * 8))
+
+
+def test_in_process_with_a_rank_without_tokens():
+    """Two ranks, the second with an empty batch: it still serves the rows
+    routed to its experts, and the first rank's layer equals the oracle's."""
+    experts = _OracleExperts()
+    tok, rr = _tokens(0)
+    layers = [ep.ExpertParallelMoE(r, 2, compute=_oracle_compute(r, 2, experts),
+                                   combine=_oracle_combine) for r in range(2)]
+    xs = [torch.from_numpy(tok.x_bits.view(np.int16)).view(torch.bfloat16),
+          torch.zeros((0, ep.HIDDEN), dtype=torch.bfloat16)]
+    idxs = [torch.from_numpy(rr.topk_idx), torch.zeros((0, 8), dtype=torch.int32)]
+    ws = [rr.topk_w, np.zeros((0, 8), np.float32)]
+    outs = ep.forward_in_process(layers, xs, idxs, ws)
+    assert O.rel_l2(outs[0].numpy(), _expected_layer(tok, rr)) <= 1e-12
+    assert tuple(outs[1].shape) == (0, ep.HIDDEN)
+    # rank 1 served exactly the rows of rank 0's tokens with an expert in 64..127
+    assert sum(layers[1].recv_counts) == int(((rr.topk_idx // 64) == 1).any(axis=1).sum())
