@@ -40,10 +40,11 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 }
 
 // Walks down one expert's column of a per-block histogram hist[b][e] (row
-// length ld) with kHistBatch loads in flight per thread.  The column's words
-// are independent, so a plain loop would pay an L2 round trip per block; in
-// the fused scan + scatter a thread walks 32 blocks at T=8189, in the
-// separate scan up to 4096.  Integer sums, so the order changes nothing.
+// length ld), issuing kHistBatch independent loads before summing them, so
+// the walk does not rely on the compiler to overlap its L2 round trips.  A
+// thread walks 32 blocks in the fused scan + scatter at T=8189 (the same time
+// as a plain loop there) and up to 4096 in the separate scan of the largest
+// batches.  Integer sums, so the order changes nothing.
 constexpr int kHistBatch = 8;
 
 // tot += hist[b][e] and, for b < lim, bef += hist[b][e], over b = b0, b0 +
